@@ -1,0 +1,324 @@
+/*
+ * pdn_oracle.c -- fp64 CPU oracle for the gated delta-rule forward recurrence.
+ *
+ * TEST INFRASTRUCTURE ONLY. This file is the plain, slow, token-by-token
+ * definition that the CUDA library is checked against. Only tests/,
+ * __graft_entry__.smoke() and bench.py's CPU-baseline leg may load it. It
+ * shares no code, header, table or helper with the CUDA library; the two only
+ * consume the same seeded inputs.
+ *
+ * Sources (web explainer pages; "ja"/"de"/"fr" name the page language):
+ *   [PDN]  "Preconditioned DeltaNet: Curvature-aware Sequence Modeling for
+ *          Linear Recurrences" (gist.science/{ja,de,fr}/paper/2604.21100)
+ *   [GDN2] "Gated DeltaNet-2" (gist.science/ja/paper/2605.22791)
+ *   [FG2]  "FG2-GDN: Enhancing Long-Context Gated Delta Networks with Doubly
+ *          Fine-Grained Control" (gist.science/ja/paper/2604.19021)
+ *
+ * State convention: S is d_v x d_k (row j = value channel, column i = key
+ * channel) and the read-out is o_t = S_t q_t. The pages on GDN-2 and FG2 print
+ * the transposed (d_k x d_v) state; their formulas are transposed here.
+ *
+ * Every variant is written as one generic token step
+ *     S <- S Diag(alpha_t)                       (decay, applied first)
+ *     S <- S + (u_t - S r_t) w_t^T               (delta step: read key r,
+ *                                                 write key w, target u)
+ *     o_t = q_scale * S q_t
+ * with (r, w, u) per variant:
+ *   DN/GDN/KDA      r = k,          w = beta k,          u = v
+ *   PDN/PGDN/PKDA   r = k,          w = beta (B_t . k),  u = v
+ *   FG2-GDN         r = sqrt(b).k,  w = sqrt(b).k,       u = sqrt(b).v
+ *   GDN-2           r = e . k,      w = k,               u = g . v
+ * (". " is the elementwise product.)
+ *
+ * Parity status of each function is stated in its comment.
+ */
+#include <math.h>
+#include <pthread.h>
+#include <stdlib.h>
+#include <string.h>
+#include <unistd.h>
+
+enum { OR_DN = 0, OR_GDN = 1, OR_KDA = 2, OR_PDN = 3, OR_PGDN = 4, OR_PKDA = 5,
+       OR_FG2 = 6, OR_GDN2 = 7 };
+enum { OR_DECAY_NONE = 0, OR_DECAY_SCALAR = 1, OR_DECAY_CHANNEL = 2 };
+
+/* ------------------------------------------------------------------------ */
+/* Diagonal preconditioner coefficients B_t for one (batch, head) sequence.
+ *
+ * [PDN] ja §2.2 "diagonal preconditioner implementation", de §2
+ * "Praktische Umsetzung", fr §2.B-C:
+ *   A_t = A_{t-1} + k_t . k_t             (diagonal of the key Gram matrix,
+ *                                          accumulated with no decay)
+ *   P_t = Diag(A_t)^{-1}                   (raw form, replaced by B_t)
+ *   stabilised: log space, centred, squashed by r/(1+|r|), then an inverse
+ *   exponential that keeps B_t inside [1/x, x].
+ * Readings where the pages are silent (listed in the design doc):
+ *   - centring mu_t = mean over the d_k channels of log(A_{t,i} + eps);
+ *   - eps is added inside the log (A_0 = 0 would give log 0);
+ *   - "inverse exponential" read as B = x^(-s), decreasing in A like A^{-1};
+ *   - A_t includes the current token.
+ * Pinned by: x = 1 gives B = 1; equal channels give B = 1; d_k = 2 gives
+ * B_0 B_1 = 1; B inside [1/x, x]; B decreasing in A (tests/test_oracle_pins.py).
+ * Parity against the original paper's exact constants: unpinned (mu, eps and
+ * the base are not printed on the pages). */
+static void precond_step(int dk, const double *kt, double *A, double x,
+                         double eps, double *Bt) {
+  double mu = 0.0;
+  for (int i = 0; i < dk; ++i) {
+    A[i] += kt[i] * kt[i];
+    Bt[i] = log(A[i] + eps); /* temporarily holds log(A + eps) */
+    mu += Bt[i];
+  }
+  mu /= (double)dk;
+  const double lnx = log(x);
+  for (int i = 0; i < dk; ++i) {
+    const double r = Bt[i] - mu;
+    const double s = r / (1.0 + fabs(r));
+    Bt[i] = exp(-s * lnx);
+  }
+}
+
+int oracle_precond(int T, int dk, const double *k, const double *A0, double x,
+                   double eps, double *Bcoef, double *AT) {
+  if (T < 0 || dk <= 0 || !k || !Bcoef) return 1;
+  double *A = (double *)calloc((size_t)dk, sizeof(double));
+  if (!A) return 2;
+  if (A0) memcpy(A, A0, sizeof(double) * (size_t)dk);
+  for (int t = 0; t < T; ++t)
+    precond_step(dk, k + (size_t)t * dk, A, x, eps, Bcoef + (size_t)t * dk);
+  if (AT) memcpy(AT, A, sizeof(double) * (size_t)dk);
+  free(A);
+  return 0;
+}
+
+/* ------------------------------------------------------------------------ */
+/* One generic token step on a d_v x d_k state (row-major, S[j*dk + i]).
+ * alpha: per key channel decay multipliers (NULL = no decay).
+ * Pinned by: beta = 0 closed form (decay only); S_t r_t = u_t whenever
+ * w.r = 1; brute-force product expansion for T <= 3; the recursive
+ * least-squares identity with a dense preconditioned write key. */
+static void token_step(int dk, int dv, double *S, const double *alpha,
+                       const double *r, const double *w, const double *u,
+                       const double *q, double q_scale, double *o) {
+  for (int j = 0; j < dv; ++j) {
+    double *Sj = S + (size_t)j * dk;
+    if (alpha)
+      for (int i = 0; i < dk; ++i) Sj[i] *= alpha[i];
+    double y = 0.0;
+    for (int i = 0; i < dk; ++i) y += Sj[i] * r[i];
+    const double delta = u[j] - y;
+    for (int i = 0; i < dk; ++i) Sj[i] += delta * w[i];
+    if (o) {
+      double z = 0.0;
+      for (int i = 0; i < dk; ++i) z += Sj[i] * q[i];
+      o[j] = q_scale * z;
+    }
+  }
+}
+
+/* ------------------------------------------------------------------------ */
+typedef struct {
+  int variant, decay, B, T, H, dk, dv;
+  const double *q, *k, *v, *log_alpha, *beta, *erase, *write_gate, *S0, *A0;
+  double q_scale, x, eps;
+  double *o, *ST, *AT;
+  /* generic mode */
+  const double *r, *w, *u;
+  int generic;
+  int next_unit; /* shared work counter, protected by mu */
+  pthread_mutex_t mu;
+  int error;
+} job_t;
+
+static int uses_precond(int variant) {
+  return variant == OR_PDN || variant == OR_PGDN || variant == OR_PKDA;
+}
+
+/* Forms r, w, u for one token (variant table in the file header).
+ * [GDN2] ja §1 "Gated Delta Rule-2": erase gate on the key side
+ *   (e_t = b_t . k_t), write gate on the value side (z_t = w_t . v_t).
+ * [FG2] ja §2.1: per-channel beta vector applied as sqrt(beta) to both
+ *   k and v (requires d_k = d_v).
+ * [PDN] ja §2.2 "read key / write key": read key k_t, write key B_t . k_t
+ *   (apply-to-key), scaled by the gain beta_t as in DeltaNet. */
+static void form_vectors(const job_t *J, size_t tok, size_t tokh, const double *Bt,
+                         double *r, double *w, double *u) {
+  const int dk = J->dk, dv = J->dv;
+  const double *kt = J->k + tok * dk;
+  const double *vt = J->v + tok * dv;
+  switch (J->variant) {
+  case OR_DN: case OR_GDN: case OR_KDA: {
+    const double b = J->beta[tokh];
+    for (int i = 0; i < dk; ++i) { r[i] = kt[i]; w[i] = b * kt[i]; }
+    for (int j = 0; j < dv; ++j) u[j] = vt[j];
+  } break;
+  case OR_PDN: case OR_PGDN: case OR_PKDA: {
+    const double b = J->beta[tokh];
+    for (int i = 0; i < dk; ++i) { r[i] = kt[i]; w[i] = b * Bt[i] * kt[i]; }
+    for (int j = 0; j < dv; ++j) u[j] = vt[j];
+  } break;
+  case OR_FG2: {
+    const double *bt = J->beta + tok * dk;
+    for (int i = 0; i < dk; ++i) {
+      const double sb = sqrt(bt[i]);
+      r[i] = sb * kt[i];
+      w[i] = sb * kt[i];
+    }
+    for (int j = 0; j < dv; ++j) u[j] = sqrt(bt[j]) * vt[j];
+  } break;
+  case OR_GDN2: {
+    const double *et = J->erase + tok * dk;
+    const double *gt = J->write_gate + tok * dv;
+    for (int i = 0; i < dk; ++i) { r[i] = et[i] * kt[i]; w[i] = kt[i]; }
+    for (int j = 0; j < dv; ++j) u[j] = gt[j] * vt[j];
+  } break;
+  }
+}
+
+static int run_unit(job_t *J, int unit) {
+  const int b = unit / J->H, h = unit % J->H;
+  const int dk = J->dk, dv = J->dv, T = J->T, H = J->H;
+  double *S = (double *)malloc(sizeof(double) * (size_t)dk * dv);
+  double *A = (double *)calloc((size_t)dk, sizeof(double));
+  double *Bt = (double *)malloc(sizeof(double) * (size_t)dk);
+  double *alpha = (double *)malloc(sizeof(double) * (size_t)dk);
+  double *r = (double *)malloc(sizeof(double) * (size_t)dk);
+  double *w = (double *)malloc(sizeof(double) * (size_t)dk);
+  double *u = (double *)malloc(sizeof(double) * (size_t)dv);
+  if (!S || !A || !Bt || !alpha || !r || !w || !u) {
+    free(S); free(A); free(Bt); free(alpha); free(r); free(w); free(u);
+    return 2;
+  }
+  const size_t sidx = ((size_t)b * H + h) * (size_t)dk * dv;
+  if (J->S0) memcpy(S, J->S0 + sidx, sizeof(double) * (size_t)dk * dv);
+  else memset(S, 0, sizeof(double) * (size_t)dk * dv);
+  if (J->A0) memcpy(A, J->A0 + ((size_t)b * H + h) * dk, sizeof(double) * (size_t)dk);
+
+  for (int t = 0; t < T; ++t) {
+    const size_t tokh = ((size_t)b * T + t) * H + h; /* [B,T,H] index */
+    const double *al = NULL;
+    const int decay = J->generic ? (J->log_alpha ? OR_DECAY_CHANNEL : OR_DECAY_NONE)
+                                 : J->decay;
+    if (decay == OR_DECAY_SCALAR) {
+      const double a = exp(J->log_alpha[tokh]);
+      for (int i = 0; i < dk; ++i) alpha[i] = a;
+      al = alpha;
+    } else if (decay == OR_DECAY_CHANNEL) {
+      const double *la = J->log_alpha + tokh * dk;
+      for (int i = 0; i < dk; ++i) alpha[i] = exp(la[i]);
+      al = alpha;
+    }
+    const double *rr, *ww, *uu;
+    if (J->generic) {
+      rr = J->r + tokh * dk;
+      ww = J->w + tokh * dk;
+      uu = J->u + tokh * dv;
+    } else {
+      if (uses_precond(J->variant))
+        precond_step(dk, J->k + tokh * dk, A, J->x, J->eps, Bt);
+      form_vectors(J, tokh, tokh, Bt, r, w, u);
+      rr = r; ww = w; uu = u;
+    }
+    token_step(dk, dv, S, al, rr, ww, uu, J->q + tokh * dk, J->q_scale,
+               J->o ? J->o + tokh * dv : NULL);
+  }
+  if (J->ST) memcpy(J->ST + sidx, S, sizeof(double) * (size_t)dk * dv);
+  if (J->AT) memcpy(J->AT + ((size_t)b * H + h) * dk, A, sizeof(double) * (size_t)dk);
+  free(S); free(A); free(Bt); free(alpha); free(r); free(w); free(u);
+  return 0;
+}
+
+static void *worker(void *arg) {
+  job_t *J = (job_t *)arg;
+  for (;;) {
+    pthread_mutex_lock(&J->mu);
+    const int unit = J->next_unit++;
+    pthread_mutex_unlock(&J->mu);
+    if (unit >= J->B * J->H) break;
+    const int rc = run_unit(J, unit);
+    if (rc) {
+      pthread_mutex_lock(&J->mu);
+      J->error = rc;
+      pthread_mutex_unlock(&J->mu);
+    }
+  }
+  return NULL;
+}
+
+static int run_job(job_t *J, int nthreads) {
+  if (nthreads <= 0) {
+    long n = sysconf(_SC_NPROCESSORS_ONLN);
+    nthreads = n > 0 ? (int)n : 1;
+  }
+  const int units = J->B * J->H;
+  if (nthreads > units) nthreads = units;
+  if (nthreads < 1) nthreads = 1;
+  J->next_unit = 0;
+  J->error = 0;
+  pthread_mutex_init(&J->mu, NULL);
+  pthread_t *th = (pthread_t *)malloc(sizeof(pthread_t) * (size_t)nthreads);
+  if (!th) return 2;
+  int started = 0;
+  for (int i = 0; i < nthreads; ++i)
+    if (pthread_create(&th[i], NULL, worker, J) == 0) ++started;
+  if (started == 0) worker(J);
+  for (int i = 0; i < started; ++i) pthread_join(th[i], NULL);
+  free(th);
+  pthread_mutex_destroy(&J->mu);
+  return J->error;
+}
+
+/* Variant forward: o [B,T,H,dv], ST [B,H,dv,dk], AT [B,H,dk] (any may be NULL).
+ * Inputs use the [B,T,H,d] layout; log_alpha is [B,T,H] (scalar decay) or
+ * [B,T,H,dk] (channel decay); beta is [B,T,H] or [B,T,H,dk] (FG2);
+ * erase [B,T,H,dk] and write_gate [B,T,H,dv] for GDN-2 only.
+ * Returns 0 on success, 1 on bad arguments, 2 on allocation failure. */
+int oracle_forward(int variant, int decay, int B, int T, int H, int dk, int dv,
+                   const double *q, const double *k, const double *v,
+                   const double *log_alpha, const double *beta,
+                   const double *erase, const double *write_gate,
+                   const double *S0, const double *A0, double q_scale, double x,
+                   double eps, double *o, double *ST, double *AT, int nthreads) {
+  if (B < 0 || T < 0 || H < 0 || dk <= 0 || dv <= 0) return 1;
+  if (variant < OR_DN || variant > OR_GDN2) return 1;
+  if (decay < OR_DECAY_NONE || decay > OR_DECAY_CHANNEL) return 1;
+  if (!q || !k || !v) return 1;
+  if (decay != OR_DECAY_NONE && !log_alpha) return 1;
+  if (variant == OR_GDN2) {
+    if (!erase || !write_gate) return 1;
+  } else if (!beta) {
+    return 1;
+  }
+  if (variant == OR_FG2 && dk != dv) return 1;
+  job_t J;
+  memset(&J, 0, sizeof(J));
+  J.variant = variant; J.decay = decay;
+  J.B = B; J.T = T; J.H = H; J.dk = dk; J.dv = dv;
+  J.q = q; J.k = k; J.v = v; J.log_alpha = log_alpha; J.beta = beta;
+  J.erase = erase; J.write_gate = write_gate; J.S0 = S0; J.A0 = A0;
+  J.q_scale = q_scale; J.x = x; J.eps = eps;
+  J.o = o; J.ST = ST; J.AT = AT;
+  J.generic = 0;
+  return run_job(&J, nthreads);
+}
+
+/* Generic form: caller supplies the read key r [B,T,H,dk], write key
+ * w [B,T,H,dk], target u [B,T,H,dv] and an optional channel log-decay
+ * [B,T,H,dk] directly. Used by the pins that need an arbitrary (e.g. dense,
+ * non-diagonal) write key, such as the least-squares equivalence
+ * ([PDN] ja §2.1, Theorem 3.1). */
+int oracle_generic(int B, int T, int H, int dk, int dv, const double *q,
+                   const double *r, const double *w, const double *u,
+                   const double *log_alpha, const double *S0, double q_scale,
+                   double *o, double *ST, int nthreads) {
+  if (B < 0 || T < 0 || H < 0 || dk <= 0 || dv <= 0) return 1;
+  if (!q || !r || !w || !u) return 1;
+  job_t J;
+  memset(&J, 0, sizeof(J));
+  J.B = B; J.T = T; J.H = H; J.dk = dk; J.dv = dv;
+  J.q = q; J.k = r; J.v = u; J.r = r; J.w = w; J.u = u;
+  J.log_alpha = log_alpha; J.S0 = S0; J.q_scale = q_scale;
+  J.o = o; J.ST = ST;
+  J.generic = 1;
+  return run_job(&J, nthreads);
+}
