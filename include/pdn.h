@@ -1,0 +1,151 @@
+/*
+ * pdn.h -- C ABI of the B200 (sm_100a) gated delta-rule forward library.
+ *
+ * The operation is the forward pass of the gated delta-rule linear
+ * recurrence in its generic form (state S is d_v x d_k, o_t = S_t q_t):
+ *
+ *   S_t = S_{t-1} Diag(alpha_t) (I - r_t w_t^T) + u_t w_t^T,   o_t = q_scale S_t q_t
+ *
+ * with read key r, write key w and target u chosen per variant:
+ *   DN / GDN / KDA      r = k,          w = beta k,          u = v
+ *       (DeltaNet; scalar decay = Gated DeltaNet; channel decay = Kimi Delta
+ *        Attention -- "Gated DeltaNet-2", ja §1, reductions paragraph)
+ *   PDN / PGDN / PKDA   r = k,          w = beta (B_t . k),  u = v
+ *       (apply-to-key diagonal preconditioner: A_t = A_{t-1} + k_t . k_t,
+ *        B_t = x^(-s), s = c/(1+|c|), c = log(A_t + eps) - mean_i log(A_ti + eps)
+ *        -- "Preconditioned DeltaNet", ja §2.2, fr §2.B-C, "Eq. 9")
+ *   FG2_GDN             r = sqrt(b).k,  w = sqrt(b).k,       u = sqrt(b).v
+ *       (per-channel gain vector b, needs d_k == d_v -- "FG2-GDN", ja §2.1)
+ *   GDN2                r = e.k,        w = k,               u = g.v
+ *       (decoupled key-side erase gate e and value-side write gate g --
+ *        "Gated DeltaNet-2", ja §1 "Gated Delta Rule-2"; the page prints the
+ *        transposed d_k x d_v state)
+ * The chunked forward evaluates the same result through the chunkwise WY/UT
+ * form the pages describe ("Gated DeltaNet-2", ja §3; "Preconditioned
+ * DeltaNet", ja §2.3). The decode step advances one token with the state
+ * carried between calls (constant-memory decoding, "Gated DeltaNet-2", ja,
+ * problem statement).
+ *
+ * Conventions (all entry points):
+ *   - Every tensor pointer is a DEVICE pointer, contiguous, 16-byte aligned,
+ *     owned by the caller; the library allocates no device memory per call.
+ *   - Layouts are row-major: q, k [B,T,H,d_k]; v, o [B,T,H,d_v];
+ *     S0, ST [B,H,d_v,d_k] fp32; A0, AT [B,H,d_k] fp32.
+ *   - Work is enqueued on the caller's CUDA stream (`stream`, a cudaStream_t;
+ *     NULL = legacy default stream) and runs asynchronously. Argument errors
+ *     are returned synchronously before anything is enqueued; launch errors
+ *     are returned as PDN_ERR_CUDA. Errors detected on the device (a bounded
+ *     wait that ran out) are recorded in a per-device error word read by
+ *     pdn_get_device_error(). No device code traps.
+ */
+#ifndef PDN_H
+#define PDN_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  PDN_OK = 0,
+  PDN_ERR_INVALID_ARG = 1, /* bad shape, pointer, alignment or variant/gate mix */
+  PDN_ERR_UNSUPPORTED = 2, /* valid problem that this build has no kernel for */
+  PDN_ERR_CUDA = 3,        /* a CUDA runtime call or kernel launch failed */
+  PDN_ERR_TIMEOUT = 4,     /* a bounded device wait ran out (device error word) */
+  PDN_ERR_WORKSPACE = 5    /* workspace pointer NULL or smaller than required */
+} pdn_status_t;
+
+/* Variant: the gain / preconditioner axes of the pages' decay-gain-
+ * preconditioner-solve taxonomy ("Preconditioned DeltaNet", de §2 "DGPS"). */
+typedef enum {
+  PDN_VAR_DN = 0,      /* decay must be NONE    */
+  PDN_VAR_GDN = 1,     /* decay must be SCALAR  */
+  PDN_VAR_KDA = 2,     /* decay must be CHANNEL */
+  PDN_VAR_PDN = 3,     /* decay must be NONE    */
+  PDN_VAR_PGDN = 4,    /* decay must be SCALAR  */
+  PDN_VAR_PKDA = 5,    /* decay must be CHANNEL */
+  PDN_VAR_FG2_GDN = 6, /* any decay; needs d_k == d_v */
+  PDN_VAR_GDN2 = 7     /* any decay */
+} pdn_variant_t;
+
+/* Decay axis: none (alpha = 1), scalar alpha per (token, head), or a
+ * per-key-channel alpha vector (KDA, "Gated DeltaNet-2" ja §1: D_t). */
+typedef enum { PDN_DECAY_NONE = 0, PDN_DECAY_SCALAR = 1, PDN_DECAY_CHANNEL = 2 } pdn_decay_t;
+
+/* Element type of q, k, v, o and of the per-channel gate tensors. The state
+ * and the preconditioner accumulator are always fp32. */
+typedef enum { PDN_F32 = 0, PDN_BF16 = 1 } pdn_dtype_t;
+
+/* Kernel selection for pdn_chunk_fwd: AUTO picks the tensor-core (tcgen05)
+ * kernel where one exists for the problem, else the CUDA-core kernel. */
+typedef enum { PDN_IMPL_AUTO = 0, PDN_IMPL_SIMT = 1, PDN_IMPL_TC = 2 } pdn_impl_t;
+
+typedef struct {
+  int B, T, H;          /* batch, tokens per sequence, heads; B,H >= 1, T >= 0 */
+  int d_k, d_v;         /* head dims: multiples of 16, 16..128                 */
+  int chunk;            /* chunk length: 16, 32 or 64 (0 = 64)                */
+  pdn_variant_t variant;
+  pdn_decay_t decay;
+  pdn_dtype_t dtype;
+  pdn_impl_t impl;
+  float q_scale;        /* read-out scale (the pages use 1)                   */
+  float precond_x;      /* preconditioner bound x, B_t in [1/x, x]; 1 <= x <= 2 */
+  float precond_eps;    /* > 0, added inside the log                          */
+} pdn_problem_t;
+
+typedef struct {
+  const void *q, *k, *v;  /* dtype; [B,T,H,d_k], [B,T,H,d_k], [B,T,H,d_v]        */
+  const void *log_alpha;  /* log decay: NULL (NONE) | fp32 [B,T,H] (SCALAR)      */
+                          /*            | dtype [B,T,H,d_k] (CHANNEL); values <= 0 */
+  const void *beta;       /* gain: fp32 [B,T,H]; FG2_GDN: dtype [B,T,H,d_k] in [0,1]; */
+                          /*       GDN2: must be NULL                              */
+  const void *erase;      /* GDN2 only: dtype [B,T,H,d_k] erase gate, else NULL   */
+  const void *write;      /* GDN2 only: dtype [B,T,H,d_v] write gate, else NULL   */
+  const float *S0;        /* initial state [B,H,d_v,d_k]; NULL = zeros            */
+  float *ST;              /* final state [B,H,d_v,d_k]; NULL = not returned       */
+  const float *A0;        /* preconditioner accumulator [B,H,d_k] (PDN/PGDN/PKDA  */
+  float *AT;              /* only, else both NULL); NULL A0 = zeros               */
+  void *o;                /* output [B,T,H,d_v], dtype                            */
+} pdn_tensors_t;
+
+/* Bytes of caller-provided workspace pdn_chunk_fwd needs for problem p
+ * (0 if none; (size_t)-1 if p is invalid). */
+size_t pdn_chunk_fwd_workspace(const pdn_problem_t *p);
+
+/* Which kernel pdn_chunk_fwd runs for problem p: PDN_IMPL_SIMT (CUDA cores)
+ * or PDN_IMPL_TC (tcgen05 tensor cores); -1 if p is invalid or no kernel of
+ * this build supports it. Host-only, touches no device. */
+int pdn_chunk_fwd_impl(const pdn_problem_t *p);
+
+/* Chunked forward over T tokens (prefill / training forward).
+ * Writes o, and ST / AT when non-NULL. S0 may alias ST and A0 may alias AT
+ * (in-place continuation). `workspace` must be 256-byte aligned and hold at
+ * least pdn_chunk_fwd_workspace(p) bytes (may be NULL when that is 0).
+ * Returns PDN_OK once the work is enqueued. */
+pdn_status_t pdn_chunk_fwd(const pdn_problem_t *p, const pdn_tensors_t *t,
+                           void *workspace, size_t ws_bytes, void *stream);
+
+/* One decode step: p->T must be 1. The state and, for preconditioned
+ * variants, the accumulator are updated IN PLACE: pass S0 == ST (non-NULL)
+ * and A0 == AT (non-NULL for PDN/PGDN/PKDA, NULL otherwise). */
+pdn_status_t pdn_decode_step(const pdn_problem_t *p, const pdn_tensors_t *t, void *stream);
+
+/* Synchronises `stream`, returns the first device-side error recorded on the
+ * current device since the last call (PDN_OK if none) and clears it. */
+pdn_status_t pdn_get_device_error(void *stream);
+
+/* Self-test of the bounded-wait mechanism every device wait uses: launches
+ * one block that waits on an mbarrier nothing arrives on, giving up after
+ * `spin_limit` polls. The kernel records PDN_ERR_TIMEOUT in the device error
+ * word and returns; the host reads it with pdn_get_device_error(). */
+pdn_status_t pdn_selftest_bounded_wait(long long spin_limit, void *stream);
+
+/* Human-readable name of a status code (static storage). */
+const char *pdn_status_string(pdn_status_t s);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PDN_H */

@@ -1,0 +1,200 @@
+// api.cu -- the C ABI declared in include/pdn.h: argument validation, kernel
+// selection and the per-device error word. No device memory is allocated.
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+#include <mutex>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace pdn {
+namespace {
+
+// First device-side error recorded by any kernel of this library (0 = none).
+// One instance per device that loads the library.
+__device__ int g_device_error;
+
+constexpr int kMaxDevices = 64;
+int *g_err_ptr[kMaxDevices];
+std::mutex g_err_mu;
+
+int *device_error_word() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lock(g_err_mu);
+  if (!g_err_ptr[dev]) {
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_device_error) != cudaSuccess) return nullptr;
+    g_err_ptr[dev] = static_cast<int *>(p);
+  }
+  return g_err_ptr[dev];
+}
+
+bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
+
+bool head_dim_ok(int d) { return d >= 16 && d <= 128 && d % 16 == 0; }
+
+pdn_decay_t required_decay(pdn_variant_t v, bool *fixed) {
+  *fixed = true;
+  switch (v) {
+    case PDN_VAR_DN: case PDN_VAR_PDN: return PDN_DECAY_NONE;
+    case PDN_VAR_GDN: case PDN_VAR_PGDN: return PDN_DECAY_SCALAR;
+    case PDN_VAR_KDA: case PDN_VAR_PKDA: return PDN_DECAY_CHANNEL;
+    default: *fixed = false; return PDN_DECAY_NONE;
+  }
+}
+
+// Shape / scalar checks shared by every entry point.
+pdn_status_t check_problem(const pdn_problem_t *p) {
+  if (!p) return PDN_ERR_INVALID_ARG;
+  if (p->B < 1 || p->H < 1 || p->T < 0) return PDN_ERR_INVALID_ARG;
+  if (!head_dim_ok(p->d_k) || !head_dim_ok(p->d_v)) return PDN_ERR_INVALID_ARG;
+  const int chunk = p->chunk == 0 ? 64 : p->chunk;
+  if (chunk != 16 && chunk != 32 && chunk != 64) return PDN_ERR_INVALID_ARG;
+  if ((int)p->variant < PDN_VAR_DN || (int)p->variant > PDN_VAR_GDN2) return PDN_ERR_INVALID_ARG;
+  if ((int)p->decay < PDN_DECAY_NONE || (int)p->decay > PDN_DECAY_CHANNEL) return PDN_ERR_INVALID_ARG;
+  if (p->dtype != PDN_F32 && p->dtype != PDN_BF16) return PDN_ERR_INVALID_ARG;
+  if ((int)p->impl < PDN_IMPL_AUTO || (int)p->impl > PDN_IMPL_TC) return PDN_ERR_INVALID_ARG;
+  bool fixed;
+  const pdn_decay_t need = required_decay(p->variant, &fixed);
+  if (fixed && p->decay != need) return PDN_ERR_INVALID_ARG;
+  if (p->variant == PDN_VAR_FG2_GDN && p->d_k != p->d_v) return PDN_ERR_INVALID_ARG;
+  if (!isfinite(p->q_scale)) return PDN_ERR_INVALID_ARG;
+  if (is_precond(p->variant)) {
+    if (!(p->precond_x >= 1.0f && p->precond_x <= 2.0f)) return PDN_ERR_INVALID_ARG;
+    if (!(p->precond_eps > 0.0f) || !isfinite(p->precond_eps)) return PDN_ERR_INVALID_ARG;
+  }
+  // flattened grids and 64-bit element offsets
+  const long long units = (long long)p->B * p->H * ((p->d_v + 31) / 32);
+  if (units > 0x7fffffffLL) return PDN_ERR_INVALID_ARG;
+  return PDN_OK;
+}
+
+pdn_status_t check_tensors(const pdn_problem_t *p, const pdn_tensors_t *t) {
+  if (!t) return PDN_ERR_INVALID_ARG;
+  if (!t->q || !t->k || !t->v || !t->o) return PDN_ERR_INVALID_ARG;
+  const void *all[] = {t->q, t->k, t->v, t->o, t->log_alpha, t->beta, t->erase,
+                       t->write, t->S0, t->ST, t->A0, t->AT};
+  for (const void *ptr : all)
+    if (ptr && !aligned16(ptr)) return PDN_ERR_INVALID_ARG;
+  if ((p->decay == PDN_DECAY_NONE) != (t->log_alpha == nullptr)) return PDN_ERR_INVALID_ARG;
+  if (p->variant == PDN_VAR_GDN2) {
+    if (t->beta || !t->erase || !t->write) return PDN_ERR_INVALID_ARG;
+  } else {
+    if (!t->beta || t->erase || t->write) return PDN_ERR_INVALID_ARG;
+  }
+  if (!is_precond(p->variant) && (t->A0 || t->AT)) return PDN_ERR_INVALID_ARG;
+  return PDN_OK;
+}
+
+KParams make_params(const pdn_problem_t *p, const pdn_tensors_t *t, int *err) {
+  KParams P;
+  memset(&P, 0, sizeof(P));
+  P.B = p->B; P.T = p->T; P.H = p->H; P.dk = p->d_k; P.dv = p->d_v;
+  P.chunk = p->chunk == 0 ? 64 : p->chunk;
+  P.variant = p->variant; P.decay = p->decay; P.dtype = p->dtype;
+  P.q_scale = p->q_scale;
+  P.x = is_precond(p->variant) ? p->precond_x : 1.0f;
+  P.lnx = logf(P.x);
+  P.eps = is_precond(p->variant) ? p->precond_eps : 1.0f;
+  P.q = t->q; P.k = t->k; P.v = t->v; P.log_alpha = t->log_alpha; P.beta = t->beta;
+  P.erase = t->erase; P.write = t->write;
+  P.S0 = t->S0; P.ST = t->ST; P.A0 = t->A0; P.AT = t->AT; P.o = t->o;
+  P.err = err;
+  return P;
+}
+
+bool use_tc(const pdn_problem_t *p, const KParams &P) {
+  if (p->impl == PDN_IMPL_SIMT) return false;
+  return tc_supported(P) != 0;
+}
+
+}  // namespace
+}  // namespace pdn
+
+using namespace pdn;
+
+extern "C" size_t pdn_chunk_fwd_workspace(const pdn_problem_t *p) {
+  if (check_problem(p) != PDN_OK) return (size_t)-1;
+  pdn_tensors_t dummy;
+  memset(&dummy, 0, sizeof(dummy));
+  const KParams P = make_params(p, &dummy, nullptr);
+  return use_tc(p, P) ? tc_workspace_bytes(P) : 0;
+}
+
+extern "C" int pdn_chunk_fwd_impl(const pdn_problem_t *p) {
+  if (check_problem(p) != PDN_OK) return -1;
+  pdn_tensors_t dummy;
+  memset(&dummy, 0, sizeof(dummy));
+  const KParams P = make_params(p, &dummy, nullptr);
+  if (use_tc(p, P)) return PDN_IMPL_TC;
+  if (p->impl == PDN_IMPL_TC || !simt_supported(P)) return -1;
+  return PDN_IMPL_SIMT;
+}
+
+extern "C" pdn_status_t pdn_chunk_fwd(const pdn_problem_t *p, const pdn_tensors_t *t,
+                                      void *workspace, size_t ws_bytes, void *stream) {
+  pdn_status_t st = check_problem(p);
+  if (st != PDN_OK) return st;
+  if ((st = check_tensors(p, t)) != PDN_OK) return st;
+  KParams P = make_params(p, t, nullptr);
+  const bool tc = use_tc(p, P);
+  if (p->impl == PDN_IMPL_TC && !tc) return PDN_ERR_UNSUPPORTED;
+  if (!tc && !simt_supported(P)) return PDN_ERR_UNSUPPORTED;
+  const size_t need = tc ? tc_workspace_bytes(P) : 0;
+  if (need > 0) {
+    if (!workspace || ws_bytes < need || ((uintptr_t)workspace & 255u)) return PDN_ERR_WORKSPACE;
+  }
+  P.err = device_error_word();
+  if (!P.err) return PDN_ERR_CUDA;
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const cudaError_t e = tc ? launch_chunk_tc(P, workspace, s) : launch_chunk_simt(P, s);
+  return e == cudaSuccess ? PDN_OK : PDN_ERR_CUDA;
+}
+
+extern "C" pdn_status_t pdn_decode_step(const pdn_problem_t *p, const pdn_tensors_t *t,
+                                        void *stream) {
+  pdn_status_t st = check_problem(p);
+  if (st != PDN_OK) return st;
+  if ((st = check_tensors(p, t)) != PDN_OK) return st;
+  if (p->T != 1) return PDN_ERR_INVALID_ARG;
+  if (!t->ST || t->S0 != t->ST) return PDN_ERR_INVALID_ARG;
+  if (is_precond(p->variant) && (!t->AT || t->A0 != t->AT)) return PDN_ERR_INVALID_ARG;
+  KParams P = make_params(p, t, device_error_word());
+  if (!P.err) return PDN_ERR_CUDA;
+  return launch_decode(P, static_cast<cudaStream_t>(stream)) == cudaSuccess ? PDN_OK
+                                                                             : PDN_ERR_CUDA;
+}
+
+extern "C" pdn_status_t pdn_get_device_error(void *stream) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return PDN_ERR_CUDA;
+  int *w = device_error_word();
+  if (!w) return PDN_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpy(&v, w, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return PDN_ERR_CUDA;
+  const int zero = 0;
+  if (cudaMemcpy(w, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess) return PDN_ERR_CUDA;
+  return static_cast<pdn_status_t>(v);
+}
+
+extern "C" pdn_status_t pdn_selftest_bounded_wait(long long spin_limit, void *stream) {
+  if (spin_limit < 0) return PDN_ERR_INVALID_ARG;
+  int *w = device_error_word();
+  if (!w) return PDN_ERR_CUDA;
+  return launch_selftest_wait(spin_limit, w, static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? PDN_OK : PDN_ERR_CUDA;
+}
+
+extern "C" const char *pdn_status_string(pdn_status_t s) {
+  switch (s) {
+    case PDN_OK: return "PDN_OK";
+    case PDN_ERR_INVALID_ARG: return "PDN_ERR_INVALID_ARG";
+    case PDN_ERR_UNSUPPORTED: return "PDN_ERR_UNSUPPORTED";
+    case PDN_ERR_CUDA: return "PDN_ERR_CUDA";
+    case PDN_ERR_TIMEOUT: return "PDN_ERR_TIMEOUT";
+    case PDN_ERR_WORKSPACE: return "PDN_ERR_WORKSPACE";
+  }
+  return "PDN_ERR_UNKNOWN";
+}

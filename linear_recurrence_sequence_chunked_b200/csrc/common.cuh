@@ -1,0 +1,73 @@
+// common.cuh -- device helpers shared by the kernels of the gated delta-rule
+// library (parameter block, element loads, variant rules, preconditioner).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/pdn.h"
+
+namespace pdn {
+
+// Everything a kernel needs, passed by value.
+struct KParams {
+  int B, T, H, dk, dv, chunk;
+  int variant, decay, dtype;
+  float q_scale, x, lnx, eps;
+  const void *q, *k, *v, *log_alpha, *beta, *erase, *write;
+  const float *S0;
+  float *ST;
+  const float *A0;
+  float *AT;
+  void *o;
+  int *err;  // per-device error word (first error wins)
+};
+
+__host__ __device__ inline bool is_precond(int variant) {
+  return variant == PDN_VAR_PDN || variant == PDN_VAR_PGDN || variant == PDN_VAR_PKDA;
+}
+
+// Element load as fp32 from a tensor of the problem dtype.
+template <typename T>
+__device__ __forceinline__ float ldf(const void *p, size_t i);
+template <>
+__device__ __forceinline__ float ldf<float>(const void *p, size_t i) {
+  return __ldg(reinterpret_cast<const float *>(p) + i);
+}
+template <>
+__device__ __forceinline__ float ldf<__nv_bfloat16>(const void *p, size_t i) {
+  return __bfloat162float(reinterpret_cast<const __nv_bfloat16 *>(p)[i]);
+}
+
+template <typename T>
+__device__ __forceinline__ void stf(void *p, size_t i, float x);
+template <>
+__device__ __forceinline__ void stf<float>(void *p, size_t i, float x) {
+  reinterpret_cast<float *>(p)[i] = x;
+}
+template <>
+__device__ __forceinline__ void stf<__nv_bfloat16>(void *p, size_t i, float x) {
+  reinterpret_cast<__nv_bfloat16 *>(p)[i] = __float2bfloat16_rn(x);
+}
+
+// Flat index of token (b, t, h) in a [B,T,H] tensor.
+__device__ __forceinline__ size_t tok_index(const KParams &P, int b, int t, int h) {
+  return ((size_t)b * P.T + t) * P.H + h;
+}
+
+// Stabilised diagonal preconditioner coefficient ("Preconditioned DeltaNet",
+// ja §2.2 / fr §2.C): c = log(A + eps) - mean_i log(A_i + eps) is squashed to
+// s = c / (1 + |c|) in (-1, 1) and mapped to B = x^(-s) in [1/x, x].
+// `logA` is log(A + eps) for this channel, `mu` the per-token channel mean.
+__device__ __forceinline__ float precond_coef(float logA, float mu, float lnx) {
+  const float c = logA - mu;
+  const float s = c / (1.0f + fabsf(c));
+  return expf(-s * lnx);
+}
+
+__device__ __forceinline__ void record_error(int *err, int code) {
+  if (err) atomicCAS(err, 0, code);
+}
+
+}  // namespace pdn

@@ -1,0 +1,203 @@
+"""ctypes binding of ``libpdn.so`` (the C ABI in ``include/pdn.h``).
+
+The functions named like the C entry points (``pdn_chunk_fwd``,
+``pdn_decode_step``, ...) only marshal arguments: every step of the
+computation runs in the library's CUDA kernels. ``chunk_fwd`` and
+``decode_step`` are conveniences that take torch tensors, allocate the outputs
+with torch and call those entry points on torch's current stream.
+
+There is no CPU fallback: importing the binding without a built library
+raises, and so does calling it on a machine without a CUDA device.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libpdn.so")
+
+PDN_OK, PDN_ERR_INVALID_ARG, PDN_ERR_UNSUPPORTED, PDN_ERR_CUDA, PDN_ERR_TIMEOUT, \
+    PDN_ERR_WORKSPACE = range(6)
+VARIANTS = {"DN": 0, "GDN": 1, "KDA": 2, "PDN": 3, "PGDN": 4, "PKDA": 5, "FG2_GDN": 6, "GDN2": 7}
+DECAYS = {"none": 0, "scalar": 1, "channel": 2}
+DTYPES = {torch.float32: 0, torch.bfloat16: 1}
+IMPLS = {"auto": 0, "simt": 1, "tc": 2}
+PRECOND_VARIANTS = ("PDN", "PGDN", "PKDA")
+
+
+class PdnProblem(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int), ("T", ctypes.c_int), ("H", ctypes.c_int),
+                ("d_k", ctypes.c_int), ("d_v", ctypes.c_int), ("chunk", ctypes.c_int),
+                ("variant", ctypes.c_int), ("decay", ctypes.c_int), ("dtype", ctypes.c_int),
+                ("impl", ctypes.c_int), ("q_scale", ctypes.c_float),
+                ("precond_x", ctypes.c_float), ("precond_eps", ctypes.c_float)]
+
+
+class PdnTensors(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in
+                ("q", "k", "v", "log_alpha", "beta", "erase", "write", "S0", "ST", "A0", "AT", "o")]
+
+
+class PdnError(RuntimeError):
+    def __init__(self, code, where):
+        self.code = code
+        super().__init__("%s returned %s" % (where, status_string(code)))
+
+
+_lib = None
+
+
+def load() -> ctypes.CDLL:
+    """Load libpdn.so (built in-tree by ``build.py``); raises if it is missing."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(_LIB_PATH):
+            raise ImportError("libpdn.so is not built (run python -m "
+                              "linear_recurrence_sequence_chunked_b200.build)")
+        lib = ctypes.CDLL(_LIB_PATH)
+        P, T, vp = ctypes.POINTER(PdnProblem), ctypes.POINTER(PdnTensors), ctypes.c_void_p
+        lib.pdn_chunk_fwd_workspace.restype = ctypes.c_size_t
+        lib.pdn_chunk_fwd_workspace.argtypes = [P]
+        lib.pdn_chunk_fwd_impl.restype = ctypes.c_int
+        lib.pdn_chunk_fwd_impl.argtypes = [P]
+        lib.pdn_chunk_fwd.restype = ctypes.c_int
+        lib.pdn_chunk_fwd.argtypes = [P, T, vp, ctypes.c_size_t, vp]
+        lib.pdn_decode_step.restype = ctypes.c_int
+        lib.pdn_decode_step.argtypes = [P, T, vp]
+        lib.pdn_get_device_error.restype = ctypes.c_int
+        lib.pdn_get_device_error.argtypes = [vp]
+        lib.pdn_selftest_bounded_wait.restype = ctypes.c_int
+        lib.pdn_selftest_bounded_wait.argtypes = [ctypes.c_longlong, vp]
+        lib.pdn_status_string.restype = ctypes.c_char_p
+        lib.pdn_status_string.argtypes = [ctypes.c_int]
+        _lib = lib
+    return _lib
+
+
+# ------------------------------------------------------------------ C-ABI names
+def pdn_chunk_fwd_workspace(problem: PdnProblem) -> int:
+    return load().pdn_chunk_fwd_workspace(ctypes.byref(problem))
+
+
+def pdn_chunk_fwd_impl(problem: PdnProblem) -> int:
+    return load().pdn_chunk_fwd_impl(ctypes.byref(problem))
+
+
+def pdn_chunk_fwd(problem: PdnProblem, tensors: PdnTensors, workspace: int, ws_bytes: int,
+                  stream: int) -> int:
+    return load().pdn_chunk_fwd(ctypes.byref(problem), ctypes.byref(tensors), workspace,
+                                ws_bytes, stream)
+
+
+def pdn_decode_step(problem: PdnProblem, tensors: PdnTensors, stream: int) -> int:
+    return load().pdn_decode_step(ctypes.byref(problem), ctypes.byref(tensors), stream)
+
+
+def pdn_get_device_error(stream: int) -> int:
+    return load().pdn_get_device_error(stream)
+
+
+def pdn_selftest_bounded_wait(spin_limit: int, stream: int) -> int:
+    return load().pdn_selftest_bounded_wait(spin_limit, stream)
+
+
+def pdn_status_string(code: int) -> str:
+    return load().pdn_status_string(code).decode()
+
+
+status_string = pdn_status_string
+
+
+# ------------------------------------------------------------------ torch helpers
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("all tensors must live on a CUDA device")
+    if not t.is_contiguous():
+        raise ValueError("all tensors must be contiguous")
+    return t.data_ptr()
+
+
+def make_problem(variant: str, B: int, T: int, H: int, d_k: int, d_v: int, dtype,
+                 decay: Optional[str] = None, chunk: int = 64, impl: str = "auto",
+                 q_scale: float = 1.0, precond_x: float = 1.5,
+                 precond_eps: float = 1e-6) -> PdnProblem:
+    if decay is None:
+        decay = {"DN": "none", "PDN": "none", "GDN": "scalar", "PGDN": "scalar"}.get(variant, "channel")
+    return PdnProblem(B, T, H, d_k, d_v, chunk, VARIANTS[variant], DECAYS[decay], DTYPES[dtype],
+                      IMPLS[impl], q_scale, precond_x, precond_eps)
+
+
+def make_tensors(q, k, v, o, log_alpha=None, beta=None, erase=None, write=None, S0=None,
+                 ST=None, A0=None, AT=None) -> PdnTensors:
+    return PdnTensors(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(erase),
+                      _ptr(write), _ptr(S0), _ptr(ST), _ptr(A0), _ptr(AT), _ptr(o))
+
+
+def _decay_of(log_alpha):
+    if log_alpha is None:
+        return "none"
+    return "scalar" if log_alpha.dim() == 3 else "channel"
+
+
+def _check(code, where):
+    if code != PDN_OK:
+        raise PdnError(code, where)
+
+
+def chunk_fwd(variant: str, q, k, v, log_alpha=None, beta=None, erase=None, write=None,
+              S0=None, A0=None, chunk: int = 64, impl: str = "auto", q_scale: float = 1.0,
+              precond_x: float = 1.5, precond_eps: float = 1e-6, want_state: bool = True,
+              out=None, workspace=None):
+    """Chunked forward on torch tensors (all on one CUDA device, contiguous).
+
+    Returns (o, S_T, A_T); S_T/A_T are None when not requested / not used.
+    """
+    B, T, H, d_k = k.shape
+    d_v = v.shape[3]
+    dev = k.device
+    p = make_problem(variant, B, T, H, d_k, d_v, k.dtype, _decay_of(log_alpha), chunk, impl,
+                     q_scale, precond_x, precond_eps)
+    o = out if out is not None else torch.empty(B, T, H, d_v, dtype=k.dtype, device=dev)
+    ST = torch.empty(B, H, d_v, d_k, dtype=torch.float32, device=dev) if want_state else None
+    AT = (torch.empty(B, H, d_k, dtype=torch.float32, device=dev)
+          if (want_state and variant in PRECOND_VARIANTS) else None)
+    t = make_tensors(q, k, v, o, log_alpha, beta, erase, write, S0, ST, A0, AT)
+    need = pdn_chunk_fwd_workspace(p)
+    if need == ctypes.c_size_t(-1).value:
+        raise PdnError(PDN_ERR_INVALID_ARG, "pdn_chunk_fwd_workspace")
+    ws_ptr, ws_bytes = None, 0
+    if need > 0:
+        if workspace is None or workspace.numel() * workspace.element_size() < need:
+            workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+        ws_ptr, ws_bytes = workspace.data_ptr(), workspace.numel() * workspace.element_size()
+    stream = torch.cuda.current_stream(dev).cuda_stream
+    _check(pdn_chunk_fwd(p, t, ws_ptr, ws_bytes, stream), "pdn_chunk_fwd")
+    return o, ST, AT
+
+
+def decode_step(variant: str, q, k, v, S, A=None, log_alpha=None, beta=None, erase=None,
+                write=None, q_scale: float = 1.0, precond_x: float = 1.5,
+                precond_eps: float = 1e-6, out=None):
+    """One decode token per sequence: q, k [B,1,H,d_k], v [B,1,H,d_v]; updates
+    the fp32 state S [B,H,d_v,d_k] (and accumulator A [B,H,d_k]) in place and
+    returns o [B,1,H,d_v]."""
+    B, T, H, d_k = k.shape
+    d_v = v.shape[3]
+    p = make_problem(variant, B, T, H, d_k, d_v, k.dtype, _decay_of(log_alpha), 64, "auto",
+                     q_scale, precond_x, precond_eps)
+    o = out if out is not None else torch.empty(B, T, H, d_v, dtype=k.dtype, device=k.device)
+    t = make_tensors(q, k, v, o, log_alpha, beta, erase, write, S, S, A, A)
+    stream = torch.cuda.current_stream(k.device).cuda_stream
+    _check(pdn_decode_step(p, t, stream), "pdn_decode_step")
+    return o
+
+
+def device_error(stream: Optional[int] = None) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream().cuda_stream
+    return pdn_get_device_error(stream)

@@ -1,0 +1,163 @@
+"""Host-side checks of the C ABI (no GPU needed, no compute calls):
+the library loads, exports every function include/pdn.h declares, its structs
+have the layout the binding assumes, and invalid arguments are rejected
+before anything touches a device."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+from linear_recurrence_sequence_chunked_b200 import build as pdn_build
+from linear_recurrence_sequence_chunked_b200 import pdn
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "pdn.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    pdn_build.build()
+    return pdn.load()
+
+
+def declared_functions():
+    names = []
+    for h in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if not h.endswith(".h"):
+            continue
+        text = open(os.path.join(ROOT, "include", h)).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        names += re.findall(r"^\s*[A-Za-z_][\w\s\*]*?\b(pdn_\w+)\s*\(", text, flags=re.M)
+    return sorted(set(names))
+
+
+def test_header_declares_entry_points():
+    names = declared_functions()
+    for n in ("pdn_chunk_fwd", "pdn_chunk_fwd_workspace", "pdn_decode_step",
+              "pdn_get_device_error", "pdn_status_string", "pdn_selftest_bounded_wait"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for n in declared_functions():
+        assert hasattr(lib, n), "libpdn.so does not export %s" % n
+    out = subprocess.run(["nm", "-D", "--defined-only", pdn._LIB_PATH], capture_output=True,
+                         text=True).stdout
+    for n in declared_functions():
+        assert re.search(r"\bT %s$" % n, out, flags=re.M), n
+
+
+def test_struct_layout_matches_header(tmp_path):
+    """Compile a probe against include/pdn.h with the host compiler and
+    compare sizeof/offsetof with the ctypes mirrors."""
+    src = tmp_path / "layout.c"
+    fields_p = [f[0] for f in pdn.PdnProblem._fields_]
+    fields_t = [f[0] for f in pdn.PdnTensors._fields_]
+    lines = ['#include <stdio.h>', '#include <stddef.h>', '#include "pdn.h"', 'int main(void){',
+             'printf("%zu %zu\\n", sizeof(pdn_problem_t), sizeof(pdn_tensors_t));']
+    for f in fields_p:
+        lines.append('printf("p %s %%zu\\n", offsetof(pdn_problem_t, %s));' % (f, f))
+    for f in fields_t:
+        lines.append('printf("t %s %%zu\\n", offsetof(pdn_tensors_t, %s));' % (f, f))
+    lines.append("return 0;}")
+    src.write_text("\n".join(lines))
+    exe = tmp_path / "layout"
+    subprocess.check_call(["gcc", "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe)])
+    out = subprocess.check_output([str(exe)], text=True).split("\n")
+    sp, stt = map(int, out[0].split())
+    assert sp == ctypes.sizeof(pdn.PdnProblem)
+    assert stt == ctypes.sizeof(pdn.PdnTensors)
+    for line in out[1:]:
+        if not line:
+            continue
+        kind, name, off = line.split()
+        cls = pdn.PdnProblem if kind == "p" else pdn.PdnTensors
+        assert getattr(cls, name).offset == int(off), name
+
+
+def test_status_strings(lib):
+    assert pdn.pdn_status_string(0) == "PDN_OK"
+    assert pdn.pdn_status_string(4) == "PDN_ERR_TIMEOUT"
+    assert pdn.pdn_status_string(99) == "PDN_ERR_UNKNOWN"
+
+
+FAKE = 0x7f0000000000  # a 16-byte aligned address that is never dereferenced
+
+
+def _tensors(**over):
+    d = dict(q=FAKE, k=FAKE + 0x1000, v=FAKE + 0x2000, log_alpha=FAKE + 0x3000,
+             beta=FAKE + 0x4000, erase=None, write=None, S0=None, ST=None, A0=None, AT=None,
+             o=FAKE + 0x5000)
+    d.update(over)
+    return pdn.PdnTensors(**d)
+
+
+def _problem(**over):
+    p = dict(B=2, T=100, H=4, d_k=64, d_v=64, chunk=64, variant=pdn.VARIANTS["PGDN"],
+             decay=pdn.DECAYS["scalar"], dtype=1, impl=0, q_scale=1.0, precond_x=1.5,
+             precond_eps=1e-6)
+    p.update(over)
+    return pdn.PdnProblem(**p)
+
+
+INVALID_PROBLEMS = [
+    dict(B=0), dict(H=0), dict(T=-1), dict(d_k=0), dict(d_k=24), dict(d_v=256), dict(chunk=48),
+    dict(variant=9), dict(decay=3), dict(dtype=5), dict(impl=7),
+    dict(decay=pdn.DECAYS["channel"]),              # PGDN needs scalar decay
+    dict(precond_x=2.5), dict(precond_x=0.5), dict(precond_eps=0.0),
+    dict(q_scale=float("nan")),
+]
+
+
+@pytest.mark.parametrize("over", INVALID_PROBLEMS)
+def test_invalid_problem_rejected(lib, over):
+    p = _problem(**over)
+    assert pdn.pdn_chunk_fwd(p, _tensors(), None, 0, None) == pdn.PDN_ERR_INVALID_ARG
+    assert pdn.pdn_chunk_fwd_workspace(p) == ctypes.c_size_t(-1).value
+
+
+INVALID_TENSORS = [
+    dict(q=None), dict(o=None), dict(k=FAKE + 8),           # missing / misaligned
+    dict(log_alpha=None),                                    # PGDN needs a decay
+    dict(beta=None),                                         # needs beta
+    dict(erase=FAKE + 0x6000),                               # GDN2-only gate
+    dict(S0=FAKE + 0x7004),                                  # misaligned state
+]
+
+
+@pytest.mark.parametrize("over", INVALID_TENSORS)
+def test_invalid_tensors_rejected(lib, over):
+    assert pdn.pdn_chunk_fwd(_problem(), _tensors(**over), None, 0, None) == pdn.PDN_ERR_INVALID_ARG
+
+
+def test_variant_specific_rules(lib):
+    # FG2 needs d_k == d_v
+    p = _problem(variant=pdn.VARIANTS["FG2_GDN"], d_v=32)
+    assert pdn.pdn_chunk_fwd(p, _tensors(), None, 0, None) == pdn.PDN_ERR_INVALID_ARG
+    # GDN2 takes erase/write and no beta
+    p = _problem(variant=pdn.VARIANTS["GDN2"], decay=pdn.DECAYS["channel"])
+    assert pdn.pdn_chunk_fwd(p, _tensors(), None, 0, None) == pdn.PDN_ERR_INVALID_ARG
+    # a non-preconditioned variant must not get an accumulator
+    p = _problem(variant=pdn.VARIANTS["GDN"])
+    assert pdn.pdn_chunk_fwd(p, _tensors(A0=FAKE + 0x8000), None, 0, None) == pdn.PDN_ERR_INVALID_ARG
+
+
+def test_decode_rules(lib):
+    p = _problem(T=1)
+    # state must be updated in place
+    assert pdn.pdn_decode_step(p, _tensors(S0=FAKE + 0x9000, ST=FAKE + 0xa000,
+                                           A0=FAKE + 0xb000, AT=FAKE + 0xb000),
+                               None) == pdn.PDN_ERR_INVALID_ARG
+    # preconditioned decode needs the accumulator, in place
+    assert pdn.pdn_decode_step(p, _tensors(S0=FAKE + 0x9000, ST=FAKE + 0x9000),
+                               None) == pdn.PDN_ERR_INVALID_ARG
+    # T must be 1
+    p = _problem(T=2)
+    assert pdn.pdn_decode_step(p, _tensors(S0=FAKE + 0x9000, ST=FAKE + 0x9000, A0=FAKE + 0xb000,
+                                           AT=FAKE + 0xb000), None) == pdn.PDN_ERR_INVALID_ARG
+
+
+def test_selftest_rejects_negative_limit(lib):
+    assert pdn.pdn_selftest_bounded_wait(-1, None) == pdn.PDN_ERR_INVALID_ARG
