@@ -82,7 +82,8 @@ typedef enum { PDN_F32 = 0, PDN_BF16 = 1 } pdn_dtype_t;
 typedef enum { PDN_IMPL_AUTO = 0, PDN_IMPL_SIMT = 1, PDN_IMPL_TC = 2 } pdn_impl_t;
 
 typedef struct {
-  int B, T, H;          /* batch, tokens per sequence, heads; B,H >= 1, T >= 0 */
+  int B, T, H;          /* batch, tokens per sequence, heads; B,H >= 1, T >= 0
+                           (T == 0: per-token tensors may be NULL; ST = S0) */
   int d_k, d_v;         /* head dims: multiples of 16, 16..128                 */
   int chunk;            /* chunk length: 16, 32 or 64 (0 = 64)                */
   pdn_variant_t variant;

@@ -74,16 +74,22 @@ pdn_status_t check_problem(const pdn_problem_t *p) {
 
 pdn_status_t check_tensors(const pdn_problem_t *p, const pdn_tensors_t *t) {
   if (!t) return PDN_ERR_INVALID_ARG;
-  if (!t->q || !t->k || !t->v || !t->o) return PDN_ERR_INVALID_ARG;
   const void *all[] = {t->q, t->k, t->v, t->o, t->log_alpha, t->beta, t->erase,
                        t->write, t->S0, t->ST, t->A0, t->AT};
   for (const void *ptr : all)
     if (ptr && !aligned16(ptr)) return PDN_ERR_INVALID_ARG;
-  if ((p->decay == PDN_DECAY_NONE) != (t->log_alpha == nullptr)) return PDN_ERR_INVALID_ARG;
-  if (p->variant == PDN_VAR_GDN2) {
-    if (t->beta || !t->erase || !t->write) return PDN_ERR_INVALID_ARG;
+  // With T == 0 the per-token tensors are empty and may be NULL; nothing
+  // reads them.
+  if (p->T == 0) {
+    if (p->variant == PDN_VAR_GDN2 && t->beta) return PDN_ERR_INVALID_ARG;
   } else {
-    if (!t->beta || t->erase || t->write) return PDN_ERR_INVALID_ARG;
+    if (!t->q || !t->k || !t->v || !t->o) return PDN_ERR_INVALID_ARG;
+    if ((p->decay == PDN_DECAY_NONE) != (t->log_alpha == nullptr)) return PDN_ERR_INVALID_ARG;
+    if (p->variant == PDN_VAR_GDN2) {
+      if (t->beta || !t->erase || !t->write) return PDN_ERR_INVALID_ARG;
+    } else {
+      if (!t->beta || t->erase || t->write) return PDN_ERR_INVALID_ARG;
+    }
   }
   if (!is_precond(p->variant) && (t->A0 || t->AT)) return PDN_ERR_INVALID_ARG;
   return PDN_OK;

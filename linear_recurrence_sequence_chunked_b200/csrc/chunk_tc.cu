@@ -1,16 +1,694 @@
-// chunk_tc.cu -- tensor-core (tcgen05) chunked forward. Not yet available in
-// this build: every problem is routed to the CUDA-core kernel.
+// chunk_tc.cu -- chunked forward of the gated delta rule on the sm_100a tensor
+// cores (tcgen05.mma, bf16 operands, fp32 accumulators in tensor memory).
+//
+// One CTA owns one (batch, head) chain, d_k = d_v = 128, and walks its chunks
+// of C = 64 tokens in order. The fp32 master state S (d_v x d_k) lives in
+// tensor memory for the whole sequence; a bf16 copy in shared memory is the
+// MMA operand. Per chunk (the chunkwise WY/UT form: "Gated DeltaNet-2", ja §3,
+// decay absorbed into the erase/write matrices, lower-triangular (I+T)^{-1}
+// solve for the erase-side auxiliary Y and the write-side auxiliary U;
+// "Preconditioned DeltaNet", ja §2.3, prefix-sum preconditioner in the chunk
+// form; "FG2-GDN", ja §2.3, same diagonal-plus-low-rank chunk algorithm):
+//
+//   prep (CUDA cores): G = in-chunk cumulative log decay, preconditioner
+//     A_t = A_{t-1} + k.k, B_t = x^{-s}, write key w per variant, then
+//     Rh = e^G.r, Qh = q_scale e^G.q, Wh = e^{-G}.w, Wb = e^{G_C-G}.w  (bf16)
+//   MMA1  [Rh;Qh] Wh^T                -> M (strict lower) and P (lower)
+//   solve T = (I + M)^{-1}            (blocked 16x16 substitution, fp32)
+//   MMA2  Y^T  = Rh^T T^T
+//   MMA3  U^T  = U^T T^T
+//   MMA5  D^T  = U^T - S Y^T          (negated-A accumulate, in place)
+//   MMA6  O^T  = S Qh^T
+//   MMA7  O^T += D^T P^T
+//   MMA8  S   += D^T Wb               (S pre-scaled by Diag(e^{G_C}))
+//
+// Every MMA is M = 128 (d_v or d_k rows on the 128 TMEM lanes), N = 64 or
+// 128, K = 16 per instruction, operands in the no-swizzle canonical layout:
+// "TL" tiles of 8-row x 16-byte core matrices, row-groups major. A TL tile
+// with rows = tokens serves both as a K-major operand (K = channels) and as
+// an MN-major operand (K = tokens), so no operand is transposed in memory.
+//
+// The exponent factorisation needs the in-chunk cumulative log decay of each
+// channel to stay above about -80 (fp32 range of e^{-G}).
 #include "common.cuh"
 #include "internal.h"
+#include "ptx.cuh"
 
 namespace pdn {
+namespace {
 
-int tc_supported(const KParams &) { return 0; }
+constexpr int kThreads = 256;
+constexpr int kC = 64;    // chunk length
+constexpr int kD = 128;   // d_k = d_v
+
+// ---- shared memory map (bytes) -------------------------------------------
+constexpr uint32_t OFF_RQ = 0;          // TL 128 x 128: rows 0-63 Rh, 64-127 Qh
+constexpr uint32_t OFF_WH = 32768;      // TL  64 x 128
+constexpr uint32_t OFF_WB = 49152;      // TL  64 x 128
+constexpr uint32_t OFF_U = 65536;       // TL  64 x 128 (v staged here)
+constexpr uint32_t OFF_SB = 81920;      // TL 128 x 128 (bf16 copy of S, rows = d_v)
+constexpr uint32_t KS_LD = 272;         // staged row stride (bytes), padded
+constexpr uint32_t OFF_KS = 114688;     // raw k, row-major [64][128] bf16
+constexpr uint32_t OFF_QS = OFF_KS + 64 * KS_LD;
+constexpr uint32_t OFF_RA = OFF_QS + 64 * KS_LD;  // region A (phase-dependent)
+constexpr int LB_LD = 132;              // floats per row of the fp32 prep buffers
+constexpr uint32_t OFF_LBUF = OFF_RA;                    // prep: log2(A + eps)
+constexpr uint32_t OFF_GBUF = OFF_RA + 64 * LB_LD * 4;   // prep: cumulative log decay
+constexpr uint32_t OFF_TM = OFF_RA;                      // TL 64 x 64: T
+constexpr uint32_t OFF_PM = OFF_RA + 8192;               // TL 64 x 64: P
+constexpr uint32_t OFF_MS = OFF_RA + 16384;              // fp32 [64][65]: M
+constexpr uint32_t OFF_TS = OFF_MS + 64 * 65 * 4;        // fp32 [64][65]: T
+constexpr uint32_t OFF_YT = OFF_RA + 16384;              // TL 128 x 64: Y^T (rows d_k)
+constexpr uint32_t OFF_DT = OFF_RA + 32768;              // TL 128 x 64: D^T (rows d_v)
+constexpr uint32_t RA_BYTES = 2 * 64 * LB_LD * 4;
+constexpr uint32_t OFF_SMALL = OFF_RA + RA_BYTES;
+constexpr uint32_t OFF_ACAR = OFF_SMALL;          // float[128] accumulator carry
+constexpr uint32_t OFF_GC = OFF_SMALL + 512;      // float[128] G at chunk end
+constexpr uint32_t OFF_EGC = OFF_SMALL + 1024;    // float[128] e^{G_C}
+constexpr uint32_t OFF_MU = OFF_SMALL + 1536;     // float[64] mean log2(A + eps)
+constexpr uint32_t OFF_BETA = OFF_SMALL + 1792;   // float[64] scalar gain
+constexpr uint32_t OFF_GS = OFF_SMALL + 2048;     // float[64] scalar cumulative decay
+constexpr uint32_t OFF_LAS = OFF_SMALL + 2304;    // float[64] scalar log decay
+constexpr uint32_t OFF_BAR = OFF_SMALL + 2560;    // uint64 mbarrier
+constexpr uint32_t OFF_TBASE = OFF_SMALL + 2568;  // uint32 TMEM base
+constexpr uint32_t SMEM_BYTES = OFF_SMALL + 2576;
+static_assert(OFF_TS + 64 * 65 * 4 <= OFF_RA + RA_BYTES, "region A overflow");
+static_assert(OFF_DT + 16384 <= OFF_RA + RA_BYTES, "region A overflow");
+static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+
+// ---- TMEM columns ---------------------------------------------------------
+constexpr uint32_t TM_D1 = 0;    // [Rh;Qh] Wh^T    (128 x 64)
+constexpr uint32_t TM_YT = 64;   // Y^T             (128 x 64)
+constexpr uint32_t TM_UD = 128;  // U^T, then D^T   (128 x 64)
+constexpr uint32_t TM_OT = 192;  // O^T             (128 x 64)
+constexpr uint32_t TM_S = 256;   // S               (128 x 128)
+constexpr uint32_t TM_COLS = 512;
+
+constexpr long long kSpinLimit = 1LL << 22;
+
+// TL tile offsets (bytes) of the 16-byte row segment (row, 8-column group).
+__device__ __forceinline__ uint32_t tl128(int row, int c8) {
+  return (uint32_t)(((row >> 3) * 16 + c8) * 128 + (row & 7) * 16);
+}
+__device__ __forceinline__ uint32_t tl64(int row, int c8) {
+  return (uint32_t)(((row >> 3) * 8 + c8) * 128 + (row & 7) * 16);
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<uint32_t *>(&v);
+}
+__device__ __forceinline__ uint4 pack8(const float (&v)[8]) {
+  return make_uint4(pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]), pack_bf16(v[4], v[5]),
+                    pack_bf16(v[6], v[7]));
+}
+__device__ __forceinline__ void unpack8(uint4 u, float (&v)[8]) {
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    __nv_bfloat162 b = *reinterpret_cast<const __nv_bfloat162 *>(&w[i]);
+    v[2 * i] = __low2float(b);
+    v[2 * i + 1] = __high2float(b);
+  }
+}
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, bool valid) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
+               "r"(valid ? 16 : 0)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.wait_all;" ::: "memory");
+}
+
+// Stage raw k, q (row-major, padded rows) and v (TL tile) of one chunk.
+__device__ __forceinline__ void stage_chunk(const KParams &P, uint32_t sbase, int b, int h,
+                                            int c0, int Cn, int tid) {
+  const __nv_bfloat16 *k = reinterpret_cast<const __nv_bfloat16 *>(P.k);
+  const __nv_bfloat16 *q = reinterpret_cast<const __nv_bfloat16 *>(P.q);
+  const __nv_bfloat16 *v = reinterpret_cast<const __nv_bfloat16 *>(P.v);
+#pragma unroll
+  for (int m = 0; m < 4; ++m) {
+    const int u = tid + kThreads * m;  // 1024 units of (token, 8 channels)
+    const int t = u >> 4, c8 = u & 15;
+    const bool ok = t < Cn;
+    const size_t e = ok ? (tok_index(P, b, c0 + t, h) * kD + c8 * 8) : 0;
+    cp_async16(sbase + OFF_KS + t * KS_LD + c8 * 16, k + e, ok);
+    cp_async16(sbase + OFF_QS + t * KS_LD + c8 * 16, q + e, ok);
+    cp_async16(sbase + OFF_U + tl128(t, c8), v + e, ok);
+  }
+  cp_async_commit();
+}
+
+__device__ __forceinline__ void mma_sync_point() {
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+}
+
+template <int kVariant, int kDecay>
+__global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const KParams P) {
+  extern __shared__ __align__(1024) uint8_t smem[];
+  const uint32_t sb = smem_u32(smem);
+  float *Acar = reinterpret_cast<float *>(smem + OFF_ACAR);
+  float *GC = reinterpret_cast<float *>(smem + OFF_GC);
+  float *EGC = reinterpret_cast<float *>(smem + OFF_EGC);
+  float *MU = reinterpret_cast<float *>(smem + OFF_MU);
+  float *BETA = reinterpret_cast<float *>(smem + OFF_BETA);
+  float *GS = reinterpret_cast<float *>(smem + OFF_GS);
+  float *LAS = reinterpret_cast<float *>(smem + OFF_LAS);
+  uint64_t *bar = reinterpret_cast<uint64_t *>(smem + OFF_BAR);
+  uint32_t *tbase_p = reinterpret_cast<uint32_t *>(smem + OFF_TBASE);
+  float *LBUF = reinterpret_cast<float *>(smem + OFF_LBUF);
+  float *GBUF = reinterpret_cast<float *>(smem + OFF_GBUF);
+  float *MS = reinterpret_cast<float *>(smem + OFF_MS);
+  float *TS = reinterpret_cast<float *>(smem + OFF_TS);
+
+  constexpr bool kPre = kVariant == PDN_VAR_PDN || kVariant == PDN_VAR_PGDN ||
+                        kVariant == PDN_VAR_PKDA;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int bh = blockIdx.x;
+  const int b = bh / P.H, h = bh % P.H;
+  const int nchunks = (P.T + kC - 1) / kC;
+  const float log2x = P.lnx * 1.4426950408889634f;
+  const uint32_t lane_q = (uint32_t)(32 * (warp & 3)) << 16;  // this warp's TMEM lane quarter
+  const int half = warp >> 2;
+
+  // ---- set-up: TMEM, barrier, accumulator, first chunk in flight ----
+  if (warp == 0) {
+    tmem_alloc(tbase_p, TM_COLS);
+    tmem_relinquish();
+  }
+  if (tid == 0) {
+    mbar_init(bar, 1);
+    fence_mbarrier_init();
+  }
+  if (tid < kD) Acar[tid] = (kPre && P.A0) ? P.A0[(size_t)bh * kD + tid] : 0.f;
+  stage_chunk(P, sb, b, h, 0, min(kC, P.T), tid);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tm = *tbase_p;
+  uint32_t phase = 0;
+  bool aborted = false;
+
+  auto wait_mma = [&]() -> bool {
+    const bool ok = mbar_wait_bounded(bar, phase, kSpinLimit);
+    phase ^= 1u;
+    tc_fence_after();
+    const bool any_fail = __syncthreads_or(!ok);
+    if (any_fail && tid == 0) record_error(P.err, PDN_ERR_TIMEOUT);
+    return !any_fail;
+  };
+
+  for (int n = 0; n < nchunks && !aborted; ++n) {
+    const int c0 = n * kC;
+    const int Cn = min(kC, P.T - c0);
+    cp_async_wait_all();
+    __syncthreads();
+
+    // ---- prep P0: per-token scalars ----
+    if (tid < kC) {
+      const bool ok = tid < Cn;
+      const size_t e = ok ? tok_index(P, b, c0 + tid, h) : 0;
+      float be = 0.f, la = 0.f;
+      if (kVariant != PDN_VAR_FG2_GDN && kVariant != PDN_VAR_GDN2)
+        be = ok ? __ldg(reinterpret_cast<const float *>(P.beta) + e) : 0.f;
+      if (kDecay == PDN_DECAY_SCALAR)
+        la = ok ? __ldg(reinterpret_cast<const float *>(P.log_alpha) + e) : 0.f;
+      BETA[tid] = be;
+      LAS[tid] = la;
+    }
+    __syncthreads();
+
+    // ---- prep P1: per-channel scans over the chunk ----
+    if (tid < kD) {
+      const int i = tid;
+      float a = Acar[i], g = 0.f;
+      const __nv_bfloat16 *la_c = reinterpret_cast<const __nv_bfloat16 *>(P.log_alpha);
+#pragma unroll 8
+      for (int t = 0; t < kC; ++t) {
+        if (kDecay == PDN_DECAY_CHANNEL) {
+          const float la = t < Cn ? __bfloat162float(la_c[tok_index(P, b, c0 + t, h) * kD + i])
+                                  : 0.f;
+          g += la;
+          GBUF[t * LB_LD + i] = g;
+        } else if (kDecay == PDN_DECAY_SCALAR) {
+          g += LAS[t];
+          if (i == 0) GS[t] = g;
+        }
+        if (kPre) {
+          const float kk = __bfloat162float(
+              *reinterpret_cast<const __nv_bfloat16 *>(smem + OFF_KS + t * KS_LD + i * 2));
+          a = fmaf(kk, kk, a);
+          LBUF[t * LB_LD + i] = __log2f(a + P.eps);
+        }
+      }
+      Acar[i] = a;
+      GC[i] = g;
+      EGC[i] = __expf(g);
+    }
+    __syncthreads();
+
+    // ---- prep P2: per-token channel mean of log2(A + eps) ----
+    if (kPre) {
+      const int t = tid >> 2, qd = tid & 3;
+      float s = 0.f;
+#pragma unroll 8
+      for (int k2 = 0; k2 < 32; ++k2) s += LBUF[t * LB_LD + qd * 32 + ((k2 + lane) & 31)];
+      s += __shfl_xor_sync(0xffffffffu, s, 1);
+      s += __shfl_xor_sync(0xffffffffu, s, 2);
+      if (qd == 0) MU[t] = s * (1.f / kD);
+      __syncthreads();
+    }
+
+    // ---- prep P3: operand tiles (token, 8-channel) units ----
+    {
+      const int t = 8 * warp + (lane & 7);
+      const bool ok = t < Cn;
+      const size_t etok = ok ? tok_index(P, b, c0 + t, h) * kD : 0;
+      float eg_s = 1.f, emg_s = 1.f, ewb_s = 1.f;
+      if (kDecay == PDN_DECAY_SCALAR) {
+        const float g = GS[t];
+        eg_s = __expf(g);
+        emg_s = __expf(-g);
+        ewb_s = __expf(GC[0] - g);
+      }
+      const float be = BETA[t];
+      const float mu = kPre ? MU[t] : 0.f;
+#pragma unroll
+      for (int m = 0; m < 4; ++m) {
+        const int c8 = 4 * m + (lane >> 3);
+        const int i0 = 8 * c8;
+        float kf[8], qf[8], r[8], w[8];
+        unpack8(*reinterpret_cast<const uint4 *>(smem + OFF_KS + t * KS_LD + c8 * 16), kf);
+        unpack8(*reinterpret_cast<const uint4 *>(smem + OFF_QS + t * KS_LD + c8 * 16), qf);
+        if (kPre) {
+          const float4 l0 = *reinterpret_cast<const float4 *>(LBUF + t * LB_LD + i0);
+          const float4 l1 = *reinterpret_cast<const float4 *>(LBUF + t * LB_LD + i0 + 4);
+          const float L[8] = {l0.x, l0.y, l0.z, l0.w, l1.x, l1.y, l1.z, l1.w};
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            const float cc = (L[c] - mu) * 0.6931471805599453f;
+            const float s = __fdividef(cc, 1.f + fabsf(cc));
+            r[c] = kf[c];
+            w[c] = be * exp2f(-s * log2x) * kf[c];
+          }
+        } else if (kVariant == PDN_VAR_FG2_GDN) {
+          float gb[8];
+          if (ok)
+            unpack8(__ldg(reinterpret_cast<const uint4 *>(
+                        reinterpret_cast<const __nv_bfloat16 *>(P.beta) + etok + i0)), gb);
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            r[c] = ok ? sqrtf(gb[c]) * kf[c] : 0.f;
+            w[c] = r[c];
+          }
+        } else if (kVariant == PDN_VAR_GDN2) {
+          float ge[8];
+          if (ok)
+            unpack8(__ldg(reinterpret_cast<const uint4 *>(
+                        reinterpret_cast<const __nv_bfloat16 *>(P.erase) + etok + i0)), ge);
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            r[c] = ok ? ge[c] * kf[c] : 0.f;
+            w[c] = kf[c];
+          }
+        } else {
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            r[c] = kf[c];
+            w[c] = be * kf[c];
+          }
+        }
+        float rh[8], qh[8], wh[8], wb[8];
+        if (kDecay == PDN_DECAY_CHANNEL) {
+          const float4 g0 = *reinterpret_cast<const float4 *>(GBUF + t * LB_LD + i0);
+          const float4 g1 = *reinterpret_cast<const float4 *>(GBUF + t * LB_LD + i0 + 4);
+          const float G[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            const float eg = __expf(G[c]);
+            rh[c] = r[c] * eg;
+            qh[c] = P.q_scale * qf[c] * eg;
+            wh[c] = w[c] * __expf(-G[c]);
+            wb[c] = w[c] * __expf(GC[i0 + c] - G[c]);
+          }
+        } else {
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            rh[c] = r[c] * eg_s;
+            qh[c] = P.q_scale * qf[c] * eg_s;
+            wh[c] = w[c] * emg_s;
+            wb[c] = w[c] * ewb_s;
+          }
+        }
+        *reinterpret_cast<uint4 *>(smem + OFF_RQ + tl128(t, c8)) = pack8(rh);
+        *reinterpret_cast<uint4 *>(smem + OFF_RQ + tl128(64 + t, c8)) = pack8(qh);
+        *reinterpret_cast<uint4 *>(smem + OFF_WH + tl128(t, c8)) = pack8(wh);
+        *reinterpret_cast<uint4 *>(smem + OFF_WB + tl128(t, c8)) = pack8(wb);
+        if (kVariant == PDN_VAR_FG2_GDN || kVariant == PDN_VAR_GDN2) {
+          // u = sqrt(beta) . v (FG2) or write-gate . v (GDN-2), in the staged tile
+          float uf[8], gt[8];
+          uint4 *up = reinterpret_cast<uint4 *>(smem + OFF_U + tl128(t, c8));
+          unpack8(*up, uf);
+          if (ok) {
+            const void *gp = kVariant == PDN_VAR_FG2_GDN ? P.beta : P.write;
+            unpack8(__ldg(reinterpret_cast<const uint4 *>(
+                        reinterpret_cast<const __nv_bfloat16 *>(gp) + etok + i0)), gt);
+          }
+#pragma unroll
+          for (int c = 0; c < 8; ++c)
+            uf[c] = ok ? uf[c] * (kVariant == PDN_VAR_FG2_GDN ? sqrtf(gt[c]) : gt[c]) : 0.f;
+          *up = pack8(uf);
+        }
+      }
+    }
+    __syncthreads();
+
+    // ---- state epilogue of the previous chunk (or the initial state) ----
+    // S (TMEM, fp32) -> bf16 operand copy; TMEM S <- S Diag(e^{G_C}) for this chunk.
+    {
+      const int j = 32 * (warp & 3) + lane;
+      if (n > 0) {
+        // O of the previous chunk
+        const int pc0 = c0 - kC;
+#pragma unroll
+        for (int cc = 0; cc < 2; ++cc) {
+          float v[16];
+          tmem_ld16(tm + lane_q + TM_OT + 32 * half + 16 * cc, v);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const int t = 32 * half + 16 * cc + e;
+            reinterpret_cast<__nv_bfloat16 *>(P.o)[tok_index(P, b, pc0 + t, h) * kD + j] =
+                __float2bfloat16_rn(v[e]);
+          }
+        }
+      }
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc) {
+        const int col = 64 * half + 16 * cc;
+        float v[16];
+        if (n == 0) {
+          if (P.S0) {
+            const float4 *src = reinterpret_cast<const float4 *>(
+                P.S0 + ((size_t)bh * kD + j) * kD + col);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float4 x = __ldg(src + e);
+              v[4 * e] = x.x; v[4 * e + 1] = x.y; v[4 * e + 2] = x.z; v[4 * e + 3] = x.w;
+            }
+          } else {
+#pragma unroll
+            for (int e = 0; e < 16; ++e) v[e] = 0.f;
+          }
+        } else {
+          tmem_ld16(tm + lane_q + TM_S + col, v);
+          tmem_wait_ld();
+        }
+        float lo[8], hi[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) { lo[e] = v[e]; hi[e] = v[8 + e]; }
+        *reinterpret_cast<uint4 *>(smem + OFF_SB + tl128(j, col / 8)) = pack8(lo);
+        *reinterpret_cast<uint4 *>(smem + OFF_SB + tl128(j, col / 8 + 1)) = pack8(hi);
+#pragma unroll
+        for (int e = 0; e < 16; ++e) v[e] *= EGC[col + e];
+        tmem_st16(tm + lane_q + TM_S + col, v);
+      }
+      tmem_wait_st();
+    }
+    mma_sync_point();
+
+    // ---- MMA1: D1 = [Rh;Qh] Wh^T ----
+    if (tid == 0) {
+      const uint32_t id = make_idesc_bf16(128, 64, false, false);
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk)
+        mma_bf16_ss(tm + TM_D1, make_sdesc(sb + OFF_RQ + 256 * kk, 128, 2048),
+                    make_sdesc(sb + OFF_WH + 256 * kk, 128, 2048), id, kk > 0);
+      mma_commit(bar);
+    }
+    if (!wait_mma()) { aborted = true; break; }
+
+    // ---- solve: M, P from TMEM; T = (I + M)^{-1} by 16x16 blocks ----
+    {
+      const int row = 32 * (warp & 3) + lane;
+#pragma unroll
+      for (int cc = 0; cc < 2; ++cc) {
+        float v[16];
+        tmem_ld16(tm + lane_q + TM_D1 + 32 * half + 16 * cc, v);
+        tmem_wait_ld();
+        const int s0 = 32 * half + 16 * cc;
+        if (row < kC) {
+#pragma unroll
+          for (int e = 0; e < 16; ++e) MS[row * 65 + s0 + e] = (s0 + e < row) ? v[e] : 0.f;
+        } else {
+          const int t = row - kC;
+          float lo[8], hi[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            lo[e] = (s0 + e <= t) ? v[e] : 0.f;
+            hi[e] = (s0 + 8 + e <= t) ? v[8 + e] : 0.f;
+          }
+          *reinterpret_cast<uint4 *>(smem + OFF_PM + tl64(t, s0 / 8)) = pack8(lo);
+          *reinterpret_cast<uint4 *>(smem + OFF_PM + tl64(t, s0 / 8 + 1)) = pack8(hi);
+        }
+      }
+    }
+    tc_fence_before();
+    __syncthreads();
+    // diagonal blocks: forward substitution, one column per thread
+    if (tid < 64) {
+      const int base = 16 * (tid >> 4), c = tid & 15;
+      float x[16];
+#pragma unroll
+      for (int r = 0; r < 16; ++r) {
+        float acc = (r == c) ? 1.f : 0.f;
+#pragma unroll
+        for (int s = 0; s < r; ++s) acc = fmaf(-MS[(base + r) * 65 + base + s], x[s], acc);
+        x[r] = acc;
+      }
+#pragma unroll
+      for (int r = 0; r < 16; ++r) TS[(base + r) * 65 + base + c] = x[r];
+    }
+    __syncthreads();
+    // off-diagonal blocks by distance d: T_ij = -T_ii sum_{k=j}^{i-1} M_ik T_kj
+#pragma unroll
+    for (int d = 1; d < 4; ++d) {
+      const int r = (tid >> 4) & 15, c = tid & 15;
+      const int npairs = 4 - d;
+      // X_ij = sum_{s=16j}^{16i-1} M[16i+r][s] T[s][16j+c], parked in the T_ij slot
+      float xs[3];
+#pragma unroll
+      for (int p = 0; p < 3; ++p) {
+        xs[p] = 0.f;
+        if (p < npairs) {
+          const int i = p + d, j = p;
+          float acc = 0.f;
+          for (int s = 16 * j; s < 16 * i; ++s)
+            acc = fmaf(MS[(16 * i + r) * 65 + s], TS[s * 65 + 16 * j + c], acc);
+          xs[p] = acc;
+        }
+      }
+      __syncthreads();
+#pragma unroll
+      for (int p = 0; p < 3; ++p)
+        if (p < npairs) TS[(16 * (p + d) + r) * 65 + 16 * p + c] = xs[p];
+      __syncthreads();
+#pragma unroll
+      for (int p = 0; p < 3; ++p) {
+        if (p < npairs) {
+          const int i = p + d, j = p;
+          float acc = 0.f;
+#pragma unroll
+          for (int s = 0; s < 16; ++s)
+            acc = fmaf(TS[(16 * i + r) * 65 + 16 * i + s], TS[(16 * i + s) * 65 + 16 * j + c], acc);
+          xs[p] = -acc;
+        }
+      }
+      __syncthreads();
+#pragma unroll
+      for (int p = 0; p < 3; ++p)
+        if (p < npairs) TS[(16 * (p + d) + r) * 65 + 16 * p + c] = xs[p];
+      __syncthreads();
+    }
+    // T (lower triangle incl. diagonal) -> bf16 TL tile
+#pragma unroll
+    for (int m = 0; m < 2; ++m) {
+      const int t = 8 * warp + (lane & 7), s8 = 4 * m + (lane >> 3);
+      float v[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) v[e] = (8 * s8 + e <= t) ? TS[t * 65 + 8 * s8 + e] : 0.f;
+      *reinterpret_cast<uint4 *>(smem + OFF_TM + tl64(t, s8)) = pack8(v);
+    }
+    mma_sync_point();
+
+    // ---- MMA2: Y^T = Rh^T T^T ; MMA3: U^T = U^T T^T ----
+    if (tid == 0) {
+      const uint32_t id = make_idesc_bf16(128, 64, true, false);
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk) {
+        const uint64_t bd = make_sdesc(sb + OFF_TM + 256 * kk, 128, 1024);
+        mma_bf16_ss(tm + TM_YT, make_sdesc(sb + OFF_RQ + 4096 * kk, 2048, 128), bd, id, kk > 0);
+        mma_bf16_ss(tm + TM_UD, make_sdesc(sb + OFF_U + 4096 * kk, 2048, 128), bd, id, kk > 0);
+      }
+      mma_commit(bar);
+    }
+    if (!wait_mma()) { aborted = true; break; }
+
+    // next chunk's raw inputs fly while this chunk finishes
+    if (n + 1 < nchunks) stage_chunk(P, sb, b, h, c0 + kC, min(kC, P.T - c0 - kC), tid);
+
+    // ---- Y^T -> bf16 operand (rows d_k, columns tokens) ----
+    {
+      const int i = 32 * (warp & 3) + lane;
+#pragma unroll
+      for (int cc = 0; cc < 2; ++cc) {
+        float v[16];
+        tmem_ld16(tm + lane_q + TM_YT + 32 * half + 16 * cc, v);
+        tmem_wait_ld();
+        float lo[8], hi[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) { lo[e] = v[e]; hi[e] = v[8 + e]; }
+        const int t8 = 4 * half + 2 * cc;
+        *reinterpret_cast<uint4 *>(smem + OFF_YT + tl64(i, t8)) = pack8(lo);
+        *reinterpret_cast<uint4 *>(smem + OFF_YT + tl64(i, t8 + 1)) = pack8(hi);
+      }
+    }
+    mma_sync_point();
+
+    // ---- MMA5: D^T = U^T - S Y^T ; MMA6: O^T = S Qh^T ----
+    if (tid == 0) {
+      const uint32_t id5 = make_idesc_bf16(128, 64, false, true, true);
+      const uint32_t id6 = make_idesc_bf16(128, 64, false, false);
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) {
+        const uint64_t ad = make_sdesc(sb + OFF_SB + 256 * kk, 128, 2048);
+        mma_bf16_ss(tm + TM_UD, ad, make_sdesc(sb + OFF_YT + 2048 * kk, 1024, 128), id5, 1);
+        mma_bf16_ss(tm + TM_OT, ad, make_sdesc(sb + OFF_RQ + 16384 + 256 * kk, 128, 2048), id6,
+                    kk > 0);
+      }
+      mma_commit(bar);
+    }
+    if (!wait_mma()) { aborted = true; break; }
+
+    // ---- D^T -> bf16 operand (rows d_v, columns tokens) ----
+    {
+      const int j = 32 * (warp & 3) + lane;
+#pragma unroll
+      for (int cc = 0; cc < 2; ++cc) {
+        float v[16];
+        tmem_ld16(tm + lane_q + TM_UD + 32 * half + 16 * cc, v);
+        tmem_wait_ld();
+        float lo[8], hi[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) { lo[e] = v[e]; hi[e] = v[8 + e]; }
+        const int t8 = 4 * half + 2 * cc;
+        *reinterpret_cast<uint4 *>(smem + OFF_DT + tl64(j, t8)) = pack8(lo);
+        *reinterpret_cast<uint4 *>(smem + OFF_DT + tl64(j, t8 + 1)) = pack8(hi);
+      }
+    }
+    mma_sync_point();
+
+    // ---- MMA7: O^T += D^T P^T ; MMA8: S += D^T Wb ----
+    if (tid == 0) {
+      const uint32_t id7 = make_idesc_bf16(128, 64, false, false);
+      const uint32_t id8 = make_idesc_bf16(128, 128, false, true);
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk) {
+        const uint64_t ad = make_sdesc(sb + OFF_DT + 256 * kk, 128, 1024);
+        mma_bf16_ss(tm + TM_OT, ad, make_sdesc(sb + OFF_PM + 256 * kk, 128, 1024), id7, 1);
+        mma_bf16_ss(tm + TM_S, ad, make_sdesc(sb + OFF_WB + 4096 * kk, 2048, 128), id8, 1);
+      }
+      mma_commit(bar);
+    }
+    if (!wait_mma()) { aborted = true; break; }
+  }
+
+  // ---- final: O of the last chunk, S_T, A_T ----
+  if (!aborted && nchunks > 0) {
+    const int j = 32 * (warp & 3) + lane;
+    const int pc0 = (nchunks - 1) * kC;
+    const int Cn = P.T - pc0;
+#pragma unroll
+    for (int cc = 0; cc < 2; ++cc) {
+      float v[16];
+      tmem_ld16(tm + lane_q + TM_OT + 32 * half + 16 * cc, v);
+      tmem_wait_ld();
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        const int t = 32 * half + 16 * cc + e;
+        if (t < Cn)
+          reinterpret_cast<__nv_bfloat16 *>(P.o)[tok_index(P, b, pc0 + t, h) * kD + j] =
+              __float2bfloat16_rn(v[e]);
+      }
+    }
+    if (P.ST) {
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc) {
+        const int col = 64 * half + 16 * cc;
+        float v[16];
+        tmem_ld16(tm + lane_q + TM_S + col, v);
+        tmem_wait_ld();
+        float4 *dst = reinterpret_cast<float4 *>(P.ST + ((size_t)bh * kD + j) * kD + col);
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          dst[e] = make_float4(v[4 * e], v[4 * e + 1], v[4 * e + 2], v[4 * e + 3]);
+      }
+    }
+    if (kPre && P.AT && tid < kD) P.AT[(size_t)bh * kD + tid] = Acar[tid];
+  }
+  cp_async_wait_all();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 0) tmem_dealloc(tm, TM_COLS);
+}
+
+template <int V, int Dc>
+cudaError_t launch_one(const KParams &P, cudaStream_t stream) {
+  auto kern = chunk_tc_kernel<V, Dc>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)SMEM_BYTES);
+  if (e != cudaSuccess) return e;
+  kern<<<(unsigned)(P.B * P.H), kThreads, SMEM_BYTES, stream>>>(P);
+  return cudaGetLastError();
+}
+
+template <int V>
+cudaError_t launch_decay(const KParams &P, cudaStream_t stream) {
+  switch (P.decay) {
+    case PDN_DECAY_NONE: return launch_one<V, PDN_DECAY_NONE>(P, stream);
+    case PDN_DECAY_SCALAR: return launch_one<V, PDN_DECAY_SCALAR>(P, stream);
+    default: return launch_one<V, PDN_DECAY_CHANNEL>(P, stream);
+  }
+}
+
+}  // namespace
+
+int tc_supported(const KParams &P) {
+  return P.dtype == PDN_BF16 && P.dk == kD && P.dv == kD && P.chunk == kC && P.T > 0 &&
+         (long long)P.B * P.H <= 0x7fffffffLL;
+}
 
 size_t tc_workspace_bytes(const KParams &) { return 0; }
 
-cudaError_t launch_chunk_tc(const KParams &, void *, cudaStream_t) {
-  return cudaErrorNotSupported;
+cudaError_t launch_chunk_tc(const KParams &P, void *, cudaStream_t stream) {
+  switch (P.variant) {
+    case PDN_VAR_DN: return launch_decay<PDN_VAR_DN>(P, stream);
+    case PDN_VAR_GDN: return launch_decay<PDN_VAR_GDN>(P, stream);
+    case PDN_VAR_KDA: return launch_decay<PDN_VAR_KDA>(P, stream);
+    case PDN_VAR_PDN: return launch_decay<PDN_VAR_PDN>(P, stream);
+    case PDN_VAR_PGDN: return launch_decay<PDN_VAR_PGDN>(P, stream);
+    case PDN_VAR_PKDA: return launch_decay<PDN_VAR_PKDA>(P, stream);
+    case PDN_VAR_FG2_GDN: return launch_decay<PDN_VAR_FG2_GDN>(P, stream);
+    default: return launch_decay<PDN_VAR_GDN2>(P, stream);
+  }
 }
 
 }  // namespace pdn

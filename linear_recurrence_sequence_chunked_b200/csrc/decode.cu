@@ -21,7 +21,7 @@ namespace {
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
 constexpr int kMaxD = 128;
-constexpr int kRB = 8;  // rows in flight per warp
+constexpr int kRows = kMaxD / kWarps;  // state rows per warp (all in flight at once)
 
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
@@ -53,6 +53,20 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const KParams P) {
   const int dk = P.dk, dv = P.dv;
   const size_t tokh = tok_index(P, b, 0, h);
   const bool precond = is_precond(P.variant);
+
+  // Issue every state-row load first: they do not depend on the token, so
+  // the per-token prologue below runs while they are in flight.
+  const int warp = tid >> 5, lane = tid & 31;
+  const int c = lane * 4;
+  const bool act = c < dk;
+  float *S = P.ST + (size_t)bh * dv * dk;
+  float4 s[kRows];
+#pragma unroll
+  for (int m = 0; m < kRows; ++m) {
+    const int j = warp + m * kWarps;
+    s[m] = (act && j < dv) ? __ldcs(reinterpret_cast<const float4 *>(S + (size_t)j * dk + c))
+                           : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
 
   // per-token vectors
   float kv = 0.f, qv = 0.f, logA = 0.f;
@@ -103,10 +117,7 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const KParams P) {
   }
   const float wq = block_sum(chan ? w * qv : 0.f, s_red);  // ends with __syncthreads
 
-  // stream the state rows
-  const int warp = tid >> 5, lane = tid & 31;
-  const int c = lane * 4;
-  const bool act = c < dk;
+  // update the state rows
   float4 rr = make_float4(0.f, 0.f, 0.f, 0.f), ww = rr, qq = rr, aa = rr;
   if (act) {
     rr = make_float4(s_r[c], s_r[c + 1], s_r[c + 2], s_r[c + 3]);
@@ -114,31 +125,21 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const KParams P) {
     qq = make_float4(s_q[c], s_q[c + 1], s_q[c + 2], s_q[c + 3]);
     aa = make_float4(s_al[c], s_al[c + 1], s_al[c + 2], s_al[c + 3]);
   }
-  float *S = P.ST + (size_t)bh * dv * dk;
-  for (int jb = warp; jb < dv; jb += kWarps * kRB) {
-    float4 s[kRB];
 #pragma unroll
-    for (int m = 0; m < kRB; ++m) {
-      const int j = jb + m * kWarps;
-      s[m] = (act && j < dv) ? __ldcs(reinterpret_cast<const float4 *>(S + (size_t)j * dk + c))
-                             : make_float4(0.f, 0.f, 0.f, 0.f);
-    }
-#pragma unroll
-    for (int m = 0; m < kRB; ++m) {
-      const int j = jb + m * kWarps;
-      float4 x = s[m];
-      x.x *= aa.x; x.y *= aa.y; x.z *= aa.z; x.w *= aa.w;
-      const float y = warp_sum(x.x * rr.x + x.y * rr.y + x.z * rr.z + x.w * rr.w);
-      const float z = warp_sum(x.x * qq.x + x.y * qq.y + x.z * qq.z + x.w * qq.w);
-      if (j < dv) {
-        const float delta = s_u[j] - y;
-        x.x = fmaf(delta, ww.x, x.x);
-        x.y = fmaf(delta, ww.y, x.y);
-        x.z = fmaf(delta, ww.z, x.z);
-        x.w = fmaf(delta, ww.w, x.w);
-        if (act) __stcs(reinterpret_cast<float4 *>(S + (size_t)j * dk + c), x);
-        if (lane == 0) stf<Tin>(P.o, tokh * dv + j, P.q_scale * fmaf(delta, wq, z));
-      }
+  for (int m = 0; m < kRows; ++m) {
+    const int j = warp + m * kWarps;
+    float4 x = s[m];
+    x.x *= aa.x; x.y *= aa.y; x.z *= aa.z; x.w *= aa.w;
+    const float y = warp_sum(x.x * rr.x + x.y * rr.y + x.z * rr.z + x.w * rr.w);
+    const float z = warp_sum(x.x * qq.x + x.y * qq.y + x.z * qq.z + x.w * qq.w);
+    if (j < dv) {
+      const float delta = s_u[j] - y;
+      x.x = fmaf(delta, ww.x, x.x);
+      x.y = fmaf(delta, ww.y, x.y);
+      x.z = fmaf(delta, ww.z, x.z);
+      x.w = fmaf(delta, ww.w, x.w);
+      if (act) __stcs(reinterpret_cast<float4 *>(S + (size_t)j * dk + c), x);
+      if (lane == 0) stf<Tin>(P.o, tokh * dv + j, P.q_scale * fmaf(delta, wq, z));
     }
   }
 }

@@ -119,7 +119,7 @@ def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
         raise ValueError("all tensors must live on a CUDA device")
     if not t.is_contiguous():
         raise ValueError("all tensors must be contiguous")
-    return t.data_ptr()
+    return t.data_ptr() or None
 
 
 def make_problem(variant: str, B: int, T: int, H: int, d_k: int, d_v: int, dtype,

@@ -1,0 +1,115 @@
+"""GPU parity of the tensor-core (tcgen05) chunk kernel against the fp64
+oracle: every variant and decay at d = 128, ragged lengths, carried state,
+and the full-size workloads on sampled (batch, head) chains."""
+import numpy as np
+import pytest
+import torch
+
+from linear_recurrence_sequence_chunked_b200 import pdn
+from linear_recurrence_sequence_chunked_b200.workloads import WORKLOADS, Workload, make_inputs, slice_chain
+
+from parity_util import assert_parity, nmax_err, run_gpu, run_oracle
+
+pytestmark = pytest.mark.gpu
+
+VARIANTS = ["DN", "GDN", "KDA", "PDN", "PGDN", "PKDA", "FG2_GDN", "GDN2"]
+DECAY = {"DN": "none", "PDN": "none", "GDN": "scalar", "PGDN": "scalar",
+         "KDA": "channel", "PKDA": "channel", "FG2_GDN": "channel", "GDN2": "channel"}
+
+
+def tc_work(variant, decay=None, B=2, T=200, H=2, seed=0, **kw):
+    return Workload("tc-%s" % variant, variant, B, T, H, 128, 128, "bf16",
+                    decay or DECAY[variant], seed=seed, **kw)
+
+
+def test_tc_kernel_is_selected():
+    p = pdn.make_problem("PGDN", 4, 4096, 16, 128, 128, torch.bfloat16)
+    assert pdn.pdn_chunk_fwd_impl(p) == pdn.IMPLS["tc"]
+    p = pdn.make_problem("PGDN", 1, 64, 2, 64, 64, torch.bfloat16)
+    assert pdn.pdn_chunk_fwd_impl(p) == pdn.IMPLS["simt"]
+
+
+@pytest.mark.parametrize("variant", VARIANTS)
+def test_tc_variants(variant):
+    w = tc_work(variant, q_scale=0.9)
+    x = make_inputs(w)
+    g = torch.Generator().manual_seed(2)
+    S0 = 0.3 * torch.randn(w.B, w.H, 128, 128, generator=g)
+    A0 = torch.rand(w.B, w.H, 128, generator=g) * 3 if variant in ("PDN", "PGDN", "PKDA") else None
+    o, ST, AT = run_gpu(w, x, S0, A0, impl="tc")
+    assert_parity(w, o, ST, AT, *run_oracle(w, x, S0, A0))
+
+
+@pytest.mark.parametrize("decay", ["none", "scalar", "channel"])
+@pytest.mark.parametrize("variant", ["FG2_GDN", "GDN2"])
+def test_tc_free_decay(variant, decay):
+    w = tc_work(variant, decay=decay, T=130)
+    x = make_inputs(w)
+    o, ST, AT = run_gpu(w, x, impl="tc")
+    assert_parity(w, o, ST, AT, *run_oracle(w, x))
+
+
+@pytest.mark.parametrize("T", [1, 63, 64, 65, 128, 1000])
+def test_tc_lengths(T):
+    w = tc_work("PKDA", T=T, B=1, H=3)
+    x = make_inputs(w)
+    o, ST, AT = run_gpu(w, x, impl="tc")
+    assert_parity(w, o, ST, AT, *run_oracle(w, x))
+
+
+def test_tc_matches_simt():
+    """Both kernels on the same bf16 inputs agree to the bf16 tolerance."""
+    w = tc_work("PGDN", B=2, H=4, T=333)
+    x = make_inputs(w)
+    a = run_gpu(w, x, impl="tc")
+    b = run_gpu(w, x, impl="simt")
+    assert nmax_err(a[0].float().cpu().numpy(), b[0].float().cpu().numpy()) < 2e-2
+    assert nmax_err(a[1].cpu().numpy(), b[1].cpu().numpy()) < 2e-2
+
+
+def test_tc_continuation():
+    w = tc_work("PGDN", T=512, B=2, H=2)
+    x = make_inputs(w)
+    o, ST, AT = run_gpu(w, x, impl="tc")
+    x1 = {n: (t[:, :192] if t is not None else None) for n, t in x.items()}
+    x2 = {n: (t[:, 192:] if t is not None else None) for n, t in x.items()}
+    _, S1, A1 = run_gpu(w.replace(T=192), x1, impl="tc")
+    o2, S2, _ = run_gpu(w.replace(T=320), x2, S1.cpu(), A1.cpu(), impl="tc")
+    assert nmax_err(o2.float().cpu().numpy(), o[:, 192:].float().cpu().numpy()) < 1e-2
+    assert nmax_err(S2.cpu().numpy(), ST.cpu().numpy()) < 1e-2
+
+
+def test_tc_deterministic():
+    w = tc_work("PKDA", B=2, H=4, T=300)
+    x = make_inputs(w)
+    a = run_gpu(w, x, impl="tc")
+    b = run_gpu(w, x, impl="tc")
+    assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1]) and torch.equal(a[2], b[2])
+
+
+FULL = ["pgdn_bf16_4k", "pkda_bf16_8k", "fg2_bf16_32k", "gdn2_bf16_32k"]
+SAMPLES = [(0, 0), (1, 7), (-1, -1)]
+
+
+@pytest.mark.parametrize("name", FULL)
+def test_full_workload_sampled_chains(name):
+    """The full-size workloads in the launch configuration bench.py times
+    (auto kernel selection), every output and the final state of three
+    sampled (batch, head) chains checked against the oracle."""
+    w = WORKLOADS[name]
+    x = make_inputs(w, device="cuda", generator_device="cuda")
+    o, ST, AT = pdn.chunk_fwd(w.variant, x["q"], x["k"], x["v"], log_alpha=x["log_alpha"],
+                              beta=x["beta"], erase=x["erase"], write=x["write"],
+                              precond_x=w.precond_x, precond_eps=w.precond_eps)
+    torch.cuda.synchronize()
+    assert pdn.device_error() == pdn.PDN_OK
+    for b, h in SAMPLES:
+        b %= w.B
+        h %= w.H
+        xs = slice_chain(x, b, h)
+        ro, rS, rA = run_oracle(w.replace(B=1, H=1), xs)
+        eo = nmax_err(o[b:b + 1, :, h:h + 1].float().cpu().numpy(), ro)
+        es = nmax_err(ST[b:b + 1, h:h + 1].cpu().numpy(), rS)
+        assert eo <= 2e-2 and es <= 2e-2, (name, b, h, eo, es)
+        if AT is not None:
+            assert nmax_err(AT[b:b + 1, h:h + 1].cpu().numpy(), rA) <= 1e-5
