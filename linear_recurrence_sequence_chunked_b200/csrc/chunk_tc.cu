@@ -34,6 +34,11 @@
 #include "internal.h"
 #include "ptx.cuh"
 
+// Phase boundary hook for out-of-tree timing harnesses; empty in the library.
+#ifndef PDN_PHASE_MARK
+#define PDN_PHASE_MARK(k)
+#endif
+
 namespace pdn {
 namespace {
 
@@ -46,7 +51,9 @@ constexpr uint32_t OFF_RQ = 0;          // TL 128 x 128: rows 0-63 Rh, 64-127 Qh
 constexpr uint32_t OFF_WH = 32768;      // TL  64 x 128
 constexpr uint32_t OFF_WB = 49152;      // TL  64 x 128
 constexpr uint32_t OFF_U = 65536;       // TL  64 x 128 (v staged here)
-constexpr uint32_t OFF_SB = 81920;      // TL 128 x 128 (bf16 copy of S, rows = d_v)
+constexpr uint32_t OFF_SB = 81920;      // TL 128 x 128 bf16 copy of S (rows = d_v); between
+                                        // the S-products and the next state epilogue it
+                                        // stages the next chunk's channel log-decay
 constexpr uint32_t KS_LD = 272;         // staged row stride (bytes), padded
 constexpr uint32_t OFF_KS = 114688;     // raw k, row-major [64][128] bf16
 constexpr uint32_t OFF_QS = OFF_KS + 64 * KS_LD;
@@ -54,10 +61,12 @@ constexpr uint32_t OFF_RA = OFF_QS + 64 * KS_LD;  // region A (phase-dependent)
 constexpr int LB_LD = 132;              // floats per row of the fp32 prep buffers
 constexpr uint32_t OFF_LBUF = OFF_RA;                    // prep: log2(A + eps)
 constexpr uint32_t OFF_GBUF = OFF_RA + 64 * LB_LD * 4;   // prep: cumulative log decay
+constexpr int MS_LD = 65, TS_LD = 66, YS_LD = 34;        // fp32 solve scratch strides
 constexpr uint32_t OFF_TM = OFF_RA;                      // TL 64 x 64: T
 constexpr uint32_t OFF_PM = OFF_RA + 8192;               // TL 64 x 64: P
 constexpr uint32_t OFF_MS = OFF_RA + 16384;              // fp32 [64][65]: M
-constexpr uint32_t OFF_TS = OFF_MS + 64 * 65 * 4;        // fp32 [64][65]: T
+constexpr uint32_t OFF_TS = OFF_MS + 64 * MS_LD * 4;     // fp32 [64][66]: T
+constexpr uint32_t OFF_YS = OFF_TS + 64 * TS_LD * 4;     // fp32 [32][34]: merge scratch
 constexpr uint32_t OFF_YT = OFF_RA + 16384;              // TL 128 x 64: Y^T (rows d_k)
 constexpr uint32_t OFF_DT = OFF_RA + 32768;              // TL 128 x 64: D^T (rows d_v)
 constexpr uint32_t RA_BYTES = 2 * 64 * LB_LD * 4;
@@ -65,14 +74,16 @@ constexpr uint32_t OFF_SMALL = OFF_RA + RA_BYTES;
 constexpr uint32_t OFF_ACAR = OFF_SMALL;          // float[128] accumulator carry
 constexpr uint32_t OFF_GC = OFF_SMALL + 512;      // float[128] G at chunk end
 constexpr uint32_t OFF_EGC = OFF_SMALL + 1024;    // float[128] e^{G_C}
-constexpr uint32_t OFF_MU = OFF_SMALL + 1536;     // float[64] mean log2(A + eps)
-constexpr uint32_t OFF_BETA = OFF_SMALL + 1792;   // float[64] scalar gain
-constexpr uint32_t OFF_GS = OFF_SMALL + 2048;     // float[64] scalar cumulative decay
-constexpr uint32_t OFF_LAS = OFF_SMALL + 2304;    // float[64] scalar log decay
-constexpr uint32_t OFF_BAR = OFF_SMALL + 2560;    // uint64 mbarrier
-constexpr uint32_t OFF_TBASE = OFF_SMALL + 2568;  // uint32 TMEM base
-constexpr uint32_t SMEM_BYTES = OFF_SMALL + 2576;
-static_assert(OFF_TS + 64 * 65 * 4 <= OFF_RA + RA_BYTES, "region A overflow");
+constexpr uint32_t OFF_PARTK = OFF_SMALL + 1536;  // float[128] first-half key energy
+constexpr uint32_t OFF_PARTG = OFF_SMALL + 2048;  // float[128] first-half log decay
+constexpr uint32_t OFF_MU = OFF_SMALL + 2560;     // float[64] mean log2(A + eps)
+constexpr uint32_t OFF_BETA = OFF_SMALL + 2816;   // float[64] scalar gain (staged)
+constexpr uint32_t OFF_GS = OFF_SMALL + 3072;     // float[64] scalar cumulative decay
+constexpr uint32_t OFF_LAS = OFF_SMALL + 3328;    // float[64] scalar log decay (staged)
+constexpr uint32_t OFF_BAR = OFF_SMALL + 3584;    // uint64 mbarrier
+constexpr uint32_t OFF_TBASE = OFF_SMALL + 3592;  // uint32 TMEM base
+constexpr uint32_t SMEM_BYTES = OFF_SMALL + 3600;
+static_assert(OFF_YS + 32 * YS_LD * 4 <= OFF_RA + RA_BYTES, "region A overflow");
 static_assert(OFF_DT + 16384 <= OFF_RA + RA_BYTES, "region A overflow");
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 
@@ -85,6 +96,9 @@ constexpr uint32_t TM_S = 256;   // S               (128 x 128)
 constexpr uint32_t TM_COLS = 512;
 
 constexpr long long kSpinLimit = 1LL << 22;
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+constexpr float kMinG = -80.f;  // floor of the in-chunk cumulative log decay (fp32 range)
 
 // TL tile offsets (bytes) of the 16-byte row segment (row, 8-column group).
 __device__ __forceinline__ uint32_t tl128(int row, int c8) {
@@ -111,34 +125,52 @@ __device__ __forceinline__ void unpack8(uint4 u, float (&v)[8]) {
     v[2 * i + 1] = __high2float(b);
   }
 }
-
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, bool valid) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
-               "r"(valid ? 16 : 0)
-               : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() {
-  asm volatile("cp.async.commit_group;" ::: "memory");
-}
-__device__ __forceinline__ void cp_async_wait_all() {
-  asm volatile("cp.async.wait_all;" ::: "memory");
+__device__ __forceinline__ void ld8f(const float *p, float (&v)[8]) {
+  const float4 a = *reinterpret_cast<const float4 *>(p);
+  const float4 b = *reinterpret_cast<const float4 *>(p + 4);
+  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+  v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
 }
 
-// Stage raw k, q (row-major, padded rows) and v (TL tile) of one chunk.
-__device__ __forceinline__ void stage_chunk(const KParams &P, uint32_t sbase, int b, int h,
-                                            int c0, int Cn, int tid) {
+// ---- staging of the next chunk's raw inputs (cp.async, zero-filled tail) ----
+template <int kVariant, int kDecay>
+__device__ __forceinline__ void stage_kq(const KParams &P, uint32_t sb, int b, int h, int c0,
+                                         int Cn, int tid) {
   const __nv_bfloat16 *k = reinterpret_cast<const __nv_bfloat16 *>(P.k);
   const __nv_bfloat16 *q = reinterpret_cast<const __nv_bfloat16 *>(P.q);
-  const __nv_bfloat16 *v = reinterpret_cast<const __nv_bfloat16 *>(P.v);
+  const size_t tstride = (size_t)P.H * kD;
+  const size_t base = tok_index(P, b, c0, h) * kD + (tid & 15) * 8;
 #pragma unroll
   for (int m = 0; m < 4; ++m) {
-    const int u = tid + kThreads * m;  // 1024 units of (token, 8 channels)
-    const int t = u >> 4, c8 = u & 15;
+    const int t = (tid >> 4) + 16 * m, c8 = tid & 15;
     const bool ok = t < Cn;
-    const size_t e = ok ? (tok_index(P, b, c0 + t, h) * kD + c8 * 8) : 0;
-    cp_async16(sbase + OFF_KS + t * KS_LD + c8 * 16, k + e, ok);
-    cp_async16(sbase + OFF_QS + t * KS_LD + c8 * 16, q + e, ok);
-    cp_async16(sbase + OFF_U + tl128(t, c8), v + e, ok);
+    const size_t e = ok ? base + t * tstride : 0;
+    cp_async16(sb + OFF_KS + t * KS_LD + c8 * 16, k + e, ok);
+    cp_async16(sb + OFF_QS + t * KS_LD + c8 * 16, q + e, ok);
+  }
+  if (tid < kC) {
+    const bool ok = tid < Cn;
+    const size_t e = ok ? tok_index(P, b, c0 + tid, h) : 0;
+    if (kVariant != PDN_VAR_FG2_GDN && kVariant != PDN_VAR_GDN2)
+      cp_async4(sb + OFF_BETA + 4 * tid, reinterpret_cast<const float *>(P.beta) + e, ok);
+    if (kDecay == PDN_DECAY_SCALAR)
+      cp_async4(sb + OFF_LAS + 4 * tid, reinterpret_cast<const float *>(P.log_alpha) + e, ok);
+  }
+  cp_async_commit();
+}
+
+// v into its TL operand tile (or the channel log-decay, row-major, into SB).
+__device__ __forceinline__ void stage_rows(const KParams &P, const void *src_t, uint32_t dst,
+                                           bool tl, int b, int h, int c0, int Cn, int tid) {
+  const __nv_bfloat16 *src = reinterpret_cast<const __nv_bfloat16 *>(src_t);
+  const size_t tstride = (size_t)P.H * kD;
+  const size_t base = tok_index(P, b, c0, h) * kD + (tid & 15) * 8;
+#pragma unroll
+  for (int m = 0; m < 4; ++m) {
+    const int t = (tid >> 4) + 16 * m, c8 = tid & 15;
+    const bool ok = t < Cn;
+    const size_t e = ok ? base + t * tstride : 0;
+    cp_async16(dst + (tl ? tl128(t, c8) : (uint32_t)(t * 256 + c8 * 16)), src + e, ok);
   }
   cp_async_commit();
 }
@@ -157,6 +189,8 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const KParams P) 
   float *Acar = reinterpret_cast<float *>(smem + OFF_ACAR);
   float *GC = reinterpret_cast<float *>(smem + OFF_GC);
   float *EGC = reinterpret_cast<float *>(smem + OFF_EGC);
+  float *PARTK = reinterpret_cast<float *>(smem + OFF_PARTK);
+  float *PARTG = reinterpret_cast<float *>(smem + OFF_PARTG);
   float *MU = reinterpret_cast<float *>(smem + OFF_MU);
   float *BETA = reinterpret_cast<float *>(smem + OFF_BETA);
   float *GS = reinterpret_cast<float *>(smem + OFF_GS);
@@ -167,16 +201,19 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const KParams P) 
   float *GBUF = reinterpret_cast<float *>(smem + OFF_GBUF);
   float *MS = reinterpret_cast<float *>(smem + OFF_MS);
   float *TS = reinterpret_cast<float *>(smem + OFF_TS);
+  float *YS = reinterpret_cast<float *>(smem + OFF_YS);
 
   constexpr bool kPre = kVariant == PDN_VAR_PDN || kVariant == PDN_VAR_PGDN ||
                         kVariant == PDN_VAR_PKDA;
+  constexpr bool kScalarBeta = kVariant != PDN_VAR_FG2_GDN && kVariant != PDN_VAR_GDN2;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int bh = blockIdx.x;
   const int b = bh / P.H, h = bh % P.H;
   const int nchunks = (P.T + kC - 1) / kC;
-  const float log2x = P.lnx * 1.4426950408889634f;
+  const float log2x = P.lnx * kLog2e;
   const uint32_t lane_q = (uint32_t)(32 * (warp & 3)) << 16;  // this warp's TMEM lane quarter
   const int half = warp >> 2;
+  const size_t tstride = (size_t)P.H * kD;  // elements between consecutive tokens
 
   // ---- set-up: TMEM, barrier, accumulator, first chunk in flight ----
   if (warp == 0) {
@@ -188,7 +225,12 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const KParams P) 
     fence_mbarrier_init();
   }
   if (tid < kD) Acar[tid] = (kPre && P.A0) ? P.A0[(size_t)bh * kD + tid] : 0.f;
-  stage_chunk(P, sb, b, h, 0, min(kC, P.T), tid);
+  {
+    const int Cn0 = min(kC, P.T);
+    stage_kq<kVariant, kDecay>(P, sb, b, h, 0, Cn0, tid);
+    stage_rows(P, P.v, sb + OFF_U, true, b, h, 0, Cn0, tid);
+    if (kDecay == PDN_DECAY_CHANNEL) stage_rows(P, P.log_alpha, sb + OFF_SB, false, b, h, 0, Cn0, tid);
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -208,78 +250,91 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const KParams P) 
   for (int n = 0; n < nchunks && !aborted; ++n) {
     const int c0 = n * kC;
     const int Cn = min(kC, P.T - c0);
+    const int Cn_next = min(kC, P.T - c0 - kC);  // <= 0 past the last chunk
+    PDN_PHASE_MARK(0);
     cp_async_wait_all();
     __syncthreads();
+    PDN_PHASE_MARK(1);
 
-    // ---- prep P0: per-token scalars ----
-    if (tid < kC) {
-      const bool ok = tid < Cn;
-      const size_t e = ok ? tok_index(P, b, c0 + tid, h) : 0;
-      float be = 0.f, la = 0.f;
-      if (kVariant != PDN_VAR_FG2_GDN && kVariant != PDN_VAR_GDN2)
-        be = ok ? __ldg(reinterpret_cast<const float *>(P.beta) + e) : 0.f;
-      if (kDecay == PDN_DECAY_SCALAR)
-        la = ok ? __ldg(reinterpret_cast<const float *>(P.log_alpha) + e) : 0.f;
-      BETA[tid] = be;
-      LAS[tid] = la;
-    }
-    __syncthreads();
-
-    // ---- prep P1: per-channel scans over the chunk ----
-    if (tid < kD) {
-      const int i = tid;
-      float a = Acar[i], g = 0.f;
-      const __nv_bfloat16 *la_c = reinterpret_cast<const __nv_bfloat16 *>(P.log_alpha);
-#pragma unroll 8
-      for (int t = 0; t < kC; ++t) {
-        if (kDecay == PDN_DECAY_CHANNEL) {
-          const float la = t < Cn ? __bfloat162float(la_c[tok_index(P, b, c0 + t, h) * kD + i])
-                                  : 0.f;
-          g += la;
-          GBUF[t * LB_LD + i] = g;
-        } else if (kDecay == PDN_DECAY_SCALAR) {
-          g += LAS[t];
-          if (i == 0) GS[t] = g;
-        }
+    // ---- prep P1: per-channel scans; thread = (channel, half of the chunk) ----
+    {
+      const int i = tid & 127, hf = tid >> 7, t0 = 32 * hf;
+      float kk[32], la[32];
+      float ks = 0.f, gs = 0.f;
+#pragma unroll
+      for (int e = 0; e < 32; ++e) {
+        kk[e] = 0.f;
+        la[e] = 0.f;
         if (kPre) {
-          const float kk = __bfloat162float(
-              *reinterpret_cast<const __nv_bfloat16 *>(smem + OFF_KS + t * KS_LD + i * 2));
-          a = fmaf(kk, kk, a);
-          LBUF[t * LB_LD + i] = __log2f(a + P.eps);
+          kk[e] = __bfloat162float(
+              *reinterpret_cast<const __nv_bfloat16 *>(smem + OFF_KS + (t0 + e) * KS_LD + i * 2));
+          ks = fmaf(kk[e], kk[e], ks);
         }
+        if (kDecay == PDN_DECAY_CHANNEL)
+          la[e] = __bfloat162float(
+              *reinterpret_cast<const __nv_bfloat16 *>(smem + OFF_SB + (t0 + e) * 256 + i * 2));
+        else if (kDecay == PDN_DECAY_SCALAR)
+          la[e] = LAS[t0 + e];
+        gs += la[e];
       }
-      Acar[i] = a;
-      GC[i] = g;
-      EGC[i] = __expf(g);
+      if (hf == 0) {
+        PARTK[i] = ks;
+        PARTG[i] = gs;
+      }
+      __syncthreads();
+      float a = Acar[i] + (hf ? PARTK[i] : 0.f);
+      float g = hf ? PARTG[i] : 0.f;
+#pragma unroll
+      for (int e = 0; e < 32; ++e) {
+        const int t = t0 + e;
+        if (kPre) {
+          a = fmaf(kk[e], kk[e], a);
+          LBUF[t * LB_LD + i] = lg2_approx(a + P.eps);
+        }
+        g += la[e];
+        if (kDecay == PDN_DECAY_CHANNEL) GBUF[t * LB_LD + i] = g;
+        else if (kDecay == PDN_DECAY_SCALAR && i == 0) GS[t] = g;
+      }
+      if (hf) {
+        Acar[i] = a;
+        GC[i] = g;
+        EGC[i] = ex2_approx(fmaxf(g, kMinG) * kLog2e);
+      }
     }
     __syncthreads();
+    PDN_PHASE_MARK(2);
+    PDN_PHASE_MARK(3);
 
     // ---- prep P2: per-token channel mean of log2(A + eps) ----
     if (kPre) {
       const int t = tid >> 2, qd = tid & 3;
       float s = 0.f;
-#pragma unroll 8
-      for (int k2 = 0; k2 < 32; ++k2) s += LBUF[t * LB_LD + qd * 32 + ((k2 + lane) & 31)];
+#pragma unroll
+      for (int k4 = 0; k4 < 8; ++k4) {
+        const float4 x = *reinterpret_cast<const float4 *>(LBUF + t * LB_LD + qd * 32 + 4 * k4);
+        s += (x.x + x.y) + (x.z + x.w);
+      }
       s += __shfl_xor_sync(0xffffffffu, s, 1);
       s += __shfl_xor_sync(0xffffffffu, s, 2);
       if (qd == 0) MU[t] = s * (1.f / kD);
       __syncthreads();
     }
+    PDN_PHASE_MARK(4);
 
-    // ---- prep P3: operand tiles (token, 8-channel) units ----
+    // ---- prep P3: operand tiles, (token, 8-channel) units ----
     {
       const int t = 8 * warp + (lane & 7);
       const bool ok = t < Cn;
       const size_t etok = ok ? tok_index(P, b, c0 + t, h) * kD : 0;
       float eg_s = 1.f, emg_s = 1.f, ewb_s = 1.f;
       if (kDecay == PDN_DECAY_SCALAR) {
-        const float g = GS[t];
-        eg_s = __expf(g);
-        emg_s = __expf(-g);
-        ewb_s = __expf(GC[0] - g);
+        eg_s = ex2_approx(fmaxf(GS[t], kMinG) * kLog2e);
+        emg_s = rcp_approx(eg_s);
+        ewb_s = EGC[0] * emg_s;
       }
-      const float be = BETA[t];
+      const float be = kScalarBeta ? BETA[t] : 0.f;
       const float mu = kPre ? MU[t] : 0.f;
+      const float qs = P.q_scale;
 #pragma unroll
       for (int m = 0; m < 4; ++m) {
         const int c8 = 4 * m + (lane >> 3);
@@ -288,34 +343,37 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const KParams P) 
         unpack8(*reinterpret_cast<const uint4 *>(smem + OFF_KS + t * KS_LD + c8 * 16), kf);
         unpack8(*reinterpret_cast<const uint4 *>(smem + OFF_QS + t * KS_LD + c8 * 16), qf);
         if (kPre) {
-          const float4 l0 = *reinterpret_cast<const float4 *>(LBUF + t * LB_LD + i0);
-          const float4 l1 = *reinterpret_cast<const float4 *>(LBUF + t * LB_LD + i0 + 4);
-          const float L[8] = {l0.x, l0.y, l0.z, l0.w, l1.x, l1.y, l1.z, l1.w};
+          float L[8];
+          ld8f(LBUF + t * LB_LD + i0, L);
 #pragma unroll
           for (int c = 0; c < 8; ++c) {
-            const float cc = (L[c] - mu) * 0.6931471805599453f;
-            const float s = __fdividef(cc, 1.f + fabsf(cc));
+            const float cc = (L[c] - mu) * kLn2;
+            const float s = cc * rcp_approx(1.f + fabsf(cc));
             r[c] = kf[c];
-            w[c] = be * exp2f(-s * log2x) * kf[c];
+            w[c] = be * ex2_approx(-s * log2x) * kf[c];
           }
         } else if (kVariant == PDN_VAR_FG2_GDN) {
           float gb[8];
+#pragma unroll
+          for (int c = 0; c < 8; ++c) gb[c] = 0.f;
           if (ok)
             unpack8(__ldg(reinterpret_cast<const uint4 *>(
                         reinterpret_cast<const __nv_bfloat16 *>(P.beta) + etok + i0)), gb);
 #pragma unroll
           for (int c = 0; c < 8; ++c) {
-            r[c] = ok ? sqrtf(gb[c]) * kf[c] : 0.f;
+            r[c] = sqrtf(gb[c]) * kf[c];
             w[c] = r[c];
           }
         } else if (kVariant == PDN_VAR_GDN2) {
           float ge[8];
+#pragma unroll
+          for (int c = 0; c < 8; ++c) ge[c] = 0.f;
           if (ok)
             unpack8(__ldg(reinterpret_cast<const uint4 *>(
                         reinterpret_cast<const __nv_bfloat16 *>(P.erase) + etok + i0)), ge);
 #pragma unroll
           for (int c = 0; c < 8; ++c) {
-            r[c] = ok ? ge[c] * kf[c] : 0.f;
+            r[c] = ge[c] * kf[c];
             w[c] = kf[c];
           }
         } else {
@@ -327,22 +385,23 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const KParams P) 
         }
         float rh[8], qh[8], wh[8], wb[8];
         if (kDecay == PDN_DECAY_CHANNEL) {
-          const float4 g0 = *reinterpret_cast<const float4 *>(GBUF + t * LB_LD + i0);
-          const float4 g1 = *reinterpret_cast<const float4 *>(GBUF + t * LB_LD + i0 + 4);
-          const float G[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+          float G[8], E[8];
+          ld8f(GBUF + t * LB_LD + i0, G);
+          ld8f(EGC + i0, E);
 #pragma unroll
           for (int c = 0; c < 8; ++c) {
-            const float eg = __expf(G[c]);
+            const float eg = ex2_approx(fmaxf(G[c], kMinG) * kLog2e);
+            const float emg = rcp_approx(eg);
             rh[c] = r[c] * eg;
-            qh[c] = P.q_scale * qf[c] * eg;
-            wh[c] = w[c] * __expf(-G[c]);
-            wb[c] = w[c] * __expf(GC[i0 + c] - G[c]);
+            qh[c] = qs * qf[c] * eg;
+            wh[c] = w[c] * emg;
+            wb[c] = w[c] * (E[c] * emg);
           }
         } else {
 #pragma unroll
           for (int c = 0; c < 8; ++c) {
             rh[c] = r[c] * eg_s;
-            qh[c] = P.q_scale * qf[c] * eg_s;
+            qh[c] = (qs * eg_s) * qf[c];
             wh[c] = w[c] * emg_s;
             wb[c] = w[c] * ewb_s;
           }
@@ -354,6 +413,8 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const KParams P) 
         if (kVariant == PDN_VAR_FG2_GDN || kVariant == PDN_VAR_GDN2) {
           // u = sqrt(beta) . v (FG2) or write-gate . v (GDN-2), in the staged tile
           float uf[8], gt[8];
+#pragma unroll
+          for (int c = 0; c < 8; ++c) gt[c] = 0.f;
           uint4 *up = reinterpret_cast<uint4 *>(smem + OFF_U + tl128(t, c8));
           unpack8(*up, uf);
           if (ok) {
@@ -363,30 +424,40 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const KParams P) 
           }
 #pragma unroll
           for (int c = 0; c < 8; ++c)
-            uf[c] = ok ? uf[c] * (kVariant == PDN_VAR_FG2_GDN ? sqrtf(gt[c]) : gt[c]) : 0.f;
+            uf[c] *= (kVariant == PDN_VAR_FG2_GDN ? sqrtf(gt[c]) : gt[c]);
           *up = pack8(uf);
         }
       }
     }
     __syncthreads();
+    PDN_PHASE_MARK(5);
+
+    // k, q and the scalar gates of the next chunk fly during the rest of this one
+    if (Cn_next > 0) stage_kq<kVariant, kDecay>(P, sb, b, h, c0 + kC, Cn_next, tid);
 
     // ---- state epilogue of the previous chunk (or the initial state) ----
-    // S (TMEM, fp32) -> bf16 operand copy; TMEM S <- S Diag(e^{G_C}) for this chunk.
+    // O of the previous chunk -> HBM; S (TMEM, fp32) -> bf16 operand copy;
+    // TMEM S <- S Diag(e^{G_C}) for this chunk.
     {
       const int j = 32 * (warp & 3) + lane;
       if (n > 0) {
-        // O of the previous chunk
-        const int pc0 = c0 - kC;
+        __nv_bfloat16 *orow = reinterpret_cast<__nv_bfloat16 *>(P.o) +
+                              tok_index(P, b, c0 - kC, h) * kD + (j & ~1);
+        const bool odd = lane & 1;
 #pragma unroll
         for (int cc = 0; cc < 2; ++cc) {
           float v[16];
           tmem_ld16(tm + lane_q + TM_OT + 32 * half + 16 * cc, v);
           tmem_wait_ld();
+          // lane pairs (j, j^1) exchange values so each stores two adjacent columns
 #pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const int t = 32 * half + 16 * cc + e;
-            reinterpret_cast<__nv_bfloat16 *>(P.o)[tok_index(P, b, pc0 + t, h) * kD + j] =
-                __float2bfloat16_rn(v[e]);
+          for (int e2 = 0; e2 < 8; ++e2) {
+            const float send = odd ? v[2 * e2] : v[2 * e2 + 1];
+            const float recv = __shfl_xor_sync(0xffffffffu, send, 1);
+            const int t = 32 * half + 16 * cc + 2 * e2 + (odd ? 1 : 0);
+            const float lo = odd ? recv : v[2 * e2];
+            const float hi = odd ? v[2 * e2 + 1] : recv;
+            *reinterpret_cast<uint32_t *>(orow + t * tstride) = pack_bf16(lo, hi);
           }
         }
       }
@@ -416,13 +487,19 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const KParams P) 
         for (int e = 0; e < 8; ++e) { lo[e] = v[e]; hi[e] = v[8 + e]; }
         *reinterpret_cast<uint4 *>(smem + OFF_SB + tl128(j, col / 8)) = pack8(lo);
         *reinterpret_cast<uint4 *>(smem + OFF_SB + tl128(j, col / 8 + 1)) = pack8(hi);
+        float E[8];
+        ld8f(EGC + col, E);
 #pragma unroll
-        for (int e = 0; e < 16; ++e) v[e] *= EGC[col + e];
+        for (int e = 0; e < 8; ++e) v[e] *= E[e];
+        ld8f(EGC + col + 8, E);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) v[8 + e] *= E[e];
         tmem_st16(tm + lane_q + TM_S + col, v);
       }
       tmem_wait_st();
     }
     mma_sync_point();
+    PDN_PHASE_MARK(6);
 
     // ---- MMA1: D1 = [Rh;Qh] Wh^T ----
     if (tid == 0) {
@@ -434,8 +511,9 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const KParams P) 
       mma_commit(bar);
     }
     if (!wait_mma()) { aborted = true; break; }
+    PDN_PHASE_MARK(7);
 
-    // ---- solve: M, P from TMEM; T = (I + M)^{-1} by 16x16 blocks ----
+    // ---- solve: M, P from TMEM; T = (I + M)^{-1} ----
     {
       const int row = 32 * (warp & 3) + lane;
 #pragma unroll
@@ -446,7 +524,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const KParams P) 
         const int s0 = 32 * half + 16 * cc;
         if (row < kC) {
 #pragma unroll
-          for (int e = 0; e < 16; ++e) MS[row * 65 + s0 + e] = (s0 + e < row) ? v[e] : 0.f;
+          for (int e = 0; e < 16; ++e) MS[row * MS_LD + s0 + e] = (s0 + e < row) ? v[e] : 0.f;
         } else {
           const int t = row - kC;
           float lo[8], hi[8];
@@ -462,71 +540,113 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const KParams P) 
     }
     tc_fence_before();
     __syncthreads();
-    // diagonal blocks: forward substitution, one column per thread
+    PDN_PHASE_MARK(8);
+    // L0: the four 16x16 diagonal blocks by forward substitution (one column
+    // per thread); the other threads zero the upper off-diagonal blocks that
+    // the merges below read.
     if (tid < 64) {
       const int base = 16 * (tid >> 4), c = tid & 15;
       float x[16];
 #pragma unroll
       for (int r = 0; r < 16; ++r) {
-        float acc = (r == c) ? 1.f : 0.f;
+        float acc0 = (r == c) ? 1.f : 0.f, acc1 = 0.f;
 #pragma unroll
-        for (int s = 0; s < r; ++s) acc = fmaf(-MS[(base + r) * 65 + base + s], x[s], acc);
-        x[r] = acc;
+        for (int s = 0; s < r; s += 2) {
+          acc0 = fmaf(-MS[(base + r) * MS_LD + base + s], x[s], acc0);
+          if (s + 1 < r) acc1 = fmaf(-MS[(base + r) * MS_LD + base + s + 1], x[s + 1], acc1);
+        }
+        x[r] = acc0 + acc1;
       }
 #pragma unroll
-      for (int r = 0; r < 16; ++r) TS[(base + r) * 65 + base + c] = x[r];
+      for (int r = 0; r < 16; ++r) TS[(base + r) * TS_LD + base + c] = x[r];
+    } else {
+      // rows 0-15 x cols 16-31 and rows 32-47 x cols 48-63 (512 entries, 192 threads)
+      for (int e = tid - 64; e < 512; e += kThreads - 64) {
+        const int blk = e >> 8, r = (e >> 4) & 15, c = e & 15;
+        TS[(32 * blk + r) * TS_LD + 32 * blk + 16 + c] = 0.f;
+      }
     }
     __syncthreads();
-    // off-diagonal blocks by distance d: T_ij = -T_ii sum_{k=j}^{i-1} M_ik T_kj
+    PDN_PHASE_MARK(9);
+    // L1: merge 16 -> 32 within rows/cols [32p, 32p+32): lower-left block
+    //   X = -T_D (M_CA T_A), 2x2 outputs per thread (128 threads).
+    if (tid < 128) {
+      const int p = tid >> 6, rb = (tid >> 3) & 7, cb = tid & 7;
+      const int o = 32 * p, r0 = 2 * rb, c0b = 2 * cb;
+      float a00 = 0.f, a01 = 0.f, a10 = 0.f, a11 = 0.f;
 #pragma unroll
-    for (int d = 1; d < 4; ++d) {
-      const int r = (tid >> 4) & 15, c = tid & 15;
-      const int npairs = 4 - d;
-      // X_ij = sum_{s=16j}^{16i-1} M[16i+r][s] T[s][16j+c], parked in the T_ij slot
-      float xs[3];
-#pragma unroll
-      for (int p = 0; p < 3; ++p) {
-        xs[p] = 0.f;
-        if (p < npairs) {
-          const int i = p + d, j = p;
-          float acc = 0.f;
-          for (int s = 16 * j; s < 16 * i; ++s)
-            acc = fmaf(MS[(16 * i + r) * 65 + s], TS[s * 65 + 16 * j + c], acc);
-          xs[p] = acc;
-        }
+      for (int s = 0; s < 16; ++s) {
+        const float m0 = MS[(o + 16 + r0) * MS_LD + o + s];
+        const float m1 = MS[(o + 16 + r0 + 1) * MS_LD + o + s];
+        const float2 tv = *reinterpret_cast<const float2 *>(TS + (o + s) * TS_LD + o + c0b);
+        a00 = fmaf(m0, tv.x, a00); a01 = fmaf(m0, tv.y, a01);
+        a10 = fmaf(m1, tv.x, a10); a11 = fmaf(m1, tv.y, a11);
       }
-      __syncthreads();
-#pragma unroll
-      for (int p = 0; p < 3; ++p)
-        if (p < npairs) TS[(16 * (p + d) + r) * 65 + 16 * p + c] = xs[p];
-      __syncthreads();
-#pragma unroll
-      for (int p = 0; p < 3; ++p) {
-        if (p < npairs) {
-          const int i = p + d, j = p;
-          float acc = 0.f;
-#pragma unroll
-          for (int s = 0; s < 16; ++s)
-            acc = fmaf(TS[(16 * i + r) * 65 + 16 * i + s], TS[(16 * i + s) * 65 + 16 * j + c], acc);
-          xs[p] = -acc;
-        }
-      }
-      __syncthreads();
-#pragma unroll
-      for (int p = 0; p < 3; ++p)
-        if (p < npairs) TS[(16 * (p + d) + r) * 65 + 16 * p + c] = xs[p];
-      __syncthreads();
+      float *y = YS + p * 16 * YS_LD;
+      *reinterpret_cast<float2 *>(y + r0 * YS_LD + c0b) = make_float2(a00, a01);
+      *reinterpret_cast<float2 *>(y + (r0 + 1) * YS_LD + c0b) = make_float2(a10, a11);
     }
+    __syncthreads();
+    if (tid < 128) {
+      const int p = tid >> 6, rb = (tid >> 3) & 7, cb = tid & 7;
+      const int o = 32 * p, r0 = 2 * rb, c0b = 2 * cb;
+      const float *y = YS + p * 16 * YS_LD;
+      float a00 = 0.f, a01 = 0.f, a10 = 0.f, a11 = 0.f;
+#pragma unroll
+      for (int s = 0; s < 16; ++s) {
+        const float t0v = TS[(o + 16 + r0) * TS_LD + o + 16 + s];
+        const float t1v = TS[(o + 16 + r0 + 1) * TS_LD + o + 16 + s];
+        const float2 yv = *reinterpret_cast<const float2 *>(y + s * YS_LD + c0b);
+        a00 = fmaf(t0v, yv.x, a00); a01 = fmaf(t0v, yv.y, a01);
+        a10 = fmaf(t1v, yv.x, a10); a11 = fmaf(t1v, yv.y, a11);
+      }
+      *reinterpret_cast<float2 *>(TS + (o + 16 + r0) * TS_LD + o + c0b) = make_float2(-a00, -a01);
+      *reinterpret_cast<float2 *>(TS + (o + 16 + r0 + 1) * TS_LD + o + c0b) =
+          make_float2(-a10, -a11);
+    }
+    __syncthreads();
+    // L2: merge 32 -> 64: X = -T_D (M[32:64, 0:32] T_A), 2x2 outputs per thread.
+    {
+      const int r0 = 2 * (tid >> 4), c0b = 2 * (tid & 15);
+      float a00 = 0.f, a01 = 0.f, a10 = 0.f, a11 = 0.f;
+#pragma unroll 8
+      for (int s = 0; s < 32; ++s) {
+        const float m0 = MS[(32 + r0) * MS_LD + s];
+        const float m1 = MS[(32 + r0 + 1) * MS_LD + s];
+        const float2 tv = *reinterpret_cast<const float2 *>(TS + s * TS_LD + c0b);
+        a00 = fmaf(m0, tv.x, a00); a01 = fmaf(m0, tv.y, a01);
+        a10 = fmaf(m1, tv.x, a10); a11 = fmaf(m1, tv.y, a11);
+      }
+      *reinterpret_cast<float2 *>(YS + r0 * YS_LD + c0b) = make_float2(a00, a01);
+      *reinterpret_cast<float2 *>(YS + (r0 + 1) * YS_LD + c0b) = make_float2(a10, a11);
+    }
+    __syncthreads();
+    {
+      const int r0 = 2 * (tid >> 4), c0b = 2 * (tid & 15);
+      float a00 = 0.f, a01 = 0.f, a10 = 0.f, a11 = 0.f;
+#pragma unroll 8
+      for (int s = 0; s < 32; ++s) {
+        const float t0v = TS[(32 + r0) * TS_LD + 32 + s];
+        const float t1v = TS[(32 + r0 + 1) * TS_LD + 32 + s];
+        const float2 yv = *reinterpret_cast<const float2 *>(YS + s * YS_LD + c0b);
+        a00 = fmaf(t0v, yv.x, a00); a01 = fmaf(t0v, yv.y, a01);
+        a10 = fmaf(t1v, yv.x, a10); a11 = fmaf(t1v, yv.y, a11);
+      }
+      *reinterpret_cast<float2 *>(TS + (32 + r0) * TS_LD + c0b) = make_float2(-a00, -a01);
+      *reinterpret_cast<float2 *>(TS + (32 + r0 + 1) * TS_LD + c0b) = make_float2(-a10, -a11);
+    }
+    __syncthreads();
     // T (lower triangle incl. diagonal) -> bf16 TL tile
 #pragma unroll
     for (int m = 0; m < 2; ++m) {
       const int t = 8 * warp + (lane & 7), s8 = 4 * m + (lane >> 3);
       float v[8];
 #pragma unroll
-      for (int e = 0; e < 8; ++e) v[e] = (8 * s8 + e <= t) ? TS[t * 65 + 8 * s8 + e] : 0.f;
+      for (int e = 0; e < 8; ++e) v[e] = (8 * s8 + e <= t) ? TS[t * TS_LD + 8 * s8 + e] : 0.f;
       *reinterpret_cast<uint4 *>(smem + OFF_TM + tl64(t, s8)) = pack8(v);
     }
     mma_sync_point();
+    PDN_PHASE_MARK(10);
 
     // ---- MMA2: Y^T = Rh^T T^T ; MMA3: U^T = U^T T^T ----
     if (tid == 0) {
@@ -540,9 +660,10 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const KParams P) 
       mma_commit(bar);
     }
     if (!wait_mma()) { aborted = true; break; }
+    PDN_PHASE_MARK(11);
 
-    // next chunk's raw inputs fly while this chunk finishes
-    if (n + 1 < nchunks) stage_chunk(P, sb, b, h, c0 + kC, min(kC, P.T - c0 - kC), tid);
+    // the next chunk's v flies while this chunk finishes
+    if (Cn_next > 0) stage_rows(P, P.v, sb + OFF_U, true, b, h, c0 + kC, Cn_next, tid);
 
     // ---- Y^T -> bf16 operand (rows d_k, columns tokens) ----
     {
@@ -561,6 +682,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const KParams P) 
       }
     }
     mma_sync_point();
+    PDN_PHASE_MARK(12);
 
     // ---- MMA5: D^T = U^T - S Y^T ; MMA6: O^T = S Qh^T ----
     if (tid == 0) {
@@ -576,6 +698,11 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const KParams P) 
       mma_commit(bar);
     }
     if (!wait_mma()) { aborted = true; break; }
+    PDN_PHASE_MARK(13);
+
+    // SB is free until the next state epilogue: stage the next chunk's channel decay there
+    if (kDecay == PDN_DECAY_CHANNEL && Cn_next > 0)
+      stage_rows(P, P.log_alpha, sb + OFF_SB, false, b, h, c0 + kC, Cn_next, tid);
 
     // ---- D^T -> bf16 operand (rows d_v, columns tokens) ----
     {
@@ -594,6 +721,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const KParams P) 
       }
     }
     mma_sync_point();
+    PDN_PHASE_MARK(14);
 
     // ---- MMA7: O^T += D^T P^T ; MMA8: S += D^T Wb ----
     if (tid == 0) {
@@ -608,6 +736,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const KParams P) 
       mma_commit(bar);
     }
     if (!wait_mma()) { aborted = true; break; }
+    PDN_PHASE_MARK(15);
   }
 
   // ---- final: O of the last chunk, S_T, A_T ----
@@ -615,6 +744,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const KParams P) 
     const int j = 32 * (warp & 3) + lane;
     const int pc0 = (nchunks - 1) * kC;
     const int Cn = P.T - pc0;
+    __nv_bfloat16 *ocol = reinterpret_cast<__nv_bfloat16 *>(P.o) + tok_index(P, b, pc0, h) * kD + j;
 #pragma unroll
     for (int cc = 0; cc < 2; ++cc) {
       float v[16];
@@ -623,9 +753,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const KParams P) 
 #pragma unroll
       for (int e = 0; e < 16; ++e) {
         const int t = 32 * half + 16 * cc + e;
-        if (t < Cn)
-          reinterpret_cast<__nv_bfloat16 *>(P.o)[tok_index(P, b, pc0 + t, h) * kD + j] =
-              __float2bfloat16_rn(v[e]);
+        if (t < Cn) ocol[t * tstride] = __float2bfloat16_rn(v[e]);
       }
     }
     if (P.ST) {
