@@ -61,11 +61,11 @@ constexpr uint32_t OFF_RA = OFF_QS + 64 * KS_LD;  // region A (phase-dependent)
 constexpr int LB_LD = 132;              // floats per row of the fp32 prep buffers
 constexpr uint32_t OFF_LBUF = OFF_RA;                    // prep: log2(A + eps)
 constexpr uint32_t OFF_GBUF = OFF_RA + 64 * LB_LD * 4;   // prep: cumulative log decay
-constexpr int MS_LD = 65, TS_LD = 66, YS_LD = 34;        // fp32 solve scratch strides
+constexpr int MS_LD = 68, TS_LD = 68, YS_LD = 34;        // fp32 solve scratch strides
 constexpr uint32_t OFF_TM = OFF_RA;                      // TL 64 x 64: T
 constexpr uint32_t OFF_PM = OFF_RA + 8192;               // TL 64 x 64: P
-constexpr uint32_t OFF_MS = OFF_RA + 16384;              // fp32 [64][65]: M
-constexpr uint32_t OFF_TS = OFF_MS + 64 * MS_LD * 4;     // fp32 [64][66]: T
+constexpr uint32_t OFF_MS = OFF_RA + 16384;              // fp32 [64][68]: M
+constexpr uint32_t OFF_TS = OFF_MS + 64 * MS_LD * 4;     // fp32 [64][68]: T
 constexpr uint32_t OFF_YS = OFF_TS + 64 * TS_LD * 4;     // fp32 [32][34]: merge scratch
 constexpr uint32_t OFF_YT = OFF_RA + 16384;              // TL 128 x 64: Y^T (rows d_k)
 constexpr uint32_t OFF_DT = OFF_RA + 32768;              // TL 128 x 64: D^T (rows d_v)
@@ -80,9 +80,10 @@ constexpr uint32_t OFF_MU = OFF_SMALL + 2560;     // float[64] mean log2(A + eps
 constexpr uint32_t OFF_BETA = OFF_SMALL + 2816;   // float[64] scalar gain (staged)
 constexpr uint32_t OFF_GS = OFF_SMALL + 3072;     // float[64] scalar cumulative decay
 constexpr uint32_t OFF_LAS = OFF_SMALL + 3328;    // float[64] scalar log decay (staged)
-constexpr uint32_t OFF_BAR = OFF_SMALL + 3584;    // uint64 mbarrier
-constexpr uint32_t OFF_TBASE = OFF_SMALL + 3592;  // uint32 TMEM base
-constexpr uint32_t SMEM_BYTES = OFF_SMALL + 3600;
+constexpr uint32_t OFF_BAR = OFF_SMALL + 3584;    // uint64[kNumBars] mbarriers
+constexpr int kNumBars = 6;                       // one per MMA group, see below
+constexpr uint32_t OFF_TBASE = OFF_BAR + 8 * kNumBars;  // uint32 TMEM base
+constexpr uint32_t SMEM_BYTES = OFF_TBASE + 16;
 static_assert(OFF_YS + 32 * YS_LD * 4 <= OFF_RA + RA_BYTES, "region A overflow");
 static_assert(OFF_DT + 16384 <= OFF_RA + RA_BYTES, "region A overflow");
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
@@ -91,8 +92,9 @@ static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 constexpr uint32_t TM_D1 = 0;    // [Rh;Qh] Wh^T    (128 x 64)
 constexpr uint32_t TM_YT = 64;   // Y^T             (128 x 64)
 constexpr uint32_t TM_UD = 128;  // U^T, then D^T   (128 x 64)
-constexpr uint32_t TM_OT = 192;  // O^T             (128 x 64)
+constexpr uint32_t TM_OT = 192;  // O^T, even chunks (128 x 64)
 constexpr uint32_t TM_S = 256;   // S               (128 x 128)
+constexpr uint32_t TM_OT1 = 384; // O^T, odd chunks  (128 x 64)
 constexpr uint32_t TM_COLS = 512;
 
 constexpr long long kSpinLimit = 1LL << 22;
@@ -175,6 +177,66 @@ __device__ __forceinline__ void stage_rows(const KParams &P, const void *src_t, 
   cp_async_commit();
 }
 
+__device__ __forceinline__ uint32_t ot_col(int n) { return (n & 1) ? TM_OT1 : TM_OT; }
+
+// Writes the 64 x 128 output tile of chunk starting at token pc0 (rows of
+// O^T in TMEM lanes, tokens in columns) to HBM. Warp-collective; the warp
+// covers its TMEM lane quarter (32 value channels) and all 64 tokens.
+__device__ __forceinline__ void store_o_tile(const KParams &P, uint32_t taddr, int b, int h,
+                                             int pc0, int Cn, int lane, int quarter) {
+  const size_t tstride = (size_t)P.H * kD;
+  const int j = 32 * quarter + lane;
+  __nv_bfloat16 *orow = reinterpret_cast<__nv_bfloat16 *>(P.o) + tok_index(P, b, pc0, h) * kD + (j & ~1);
+  const bool odd = lane & 1;
+#pragma unroll
+  for (int hc = 0; hc < 2; ++hc) {
+    float ov[2][16];
+    tmem_ld16(taddr + 32 * hc, ov[0]);
+    tmem_ld16(taddr + 32 * hc + 16, ov[1]);
+    tmem_wait_ld();
+#pragma unroll
+    for (int cc = 0; cc < 2; ++cc) {
+      const float *v = ov[cc];
+      // lane pairs (j, j^1) exchange values so each stores two adjacent columns
+#pragma unroll
+      for (int e2 = 0; e2 < 8; ++e2) {
+        const float send = odd ? v[2 * e2] : v[2 * e2 + 1];
+        const float recv = __shfl_xor_sync(0xffffffffu, send, 1);
+        const int t = 32 * hc + 16 * cc + 2 * e2 + (odd ? 1 : 0);
+        const float lo = odd ? recv : v[2 * e2];
+        const float hi = odd ? v[2 * e2 + 1] : recv;
+        if (t < Cn) *reinterpret_cast<uint32_t *>(orow + t * tstride) = pack_bf16(lo, hi);
+      }
+    }
+  }
+}
+
+// Same for the 32 tokens [t0, t0 + 32) of the tile (taddr points at column t0).
+__device__ __forceinline__ void store_o_half(const KParams &P, uint32_t taddr, int b, int h,
+                                             int pc0, int Cn, int t0, int lane, int quarter) {
+  const size_t tstride = (size_t)P.H * kD;
+  const int j = 32 * quarter + lane;
+  __nv_bfloat16 *orow = reinterpret_cast<__nv_bfloat16 *>(P.o) + tok_index(P, b, pc0, h) * kD + (j & ~1);
+  const bool odd = lane & 1;
+  float ov[2][16];
+  tmem_ld16(taddr, ov[0]);
+  tmem_ld16(taddr + 16, ov[1]);
+  tmem_wait_ld();
+#pragma unroll
+  for (int cc = 0; cc < 2; ++cc) {
+    const float *v = ov[cc];
+#pragma unroll
+    for (int e2 = 0; e2 < 8; ++e2) {
+      const float send = odd ? v[2 * e2] : v[2 * e2 + 1];
+      const float recv = __shfl_xor_sync(0xffffffffu, send, 1);
+      const int t = t0 + 16 * cc + 2 * e2 + (odd ? 1 : 0);
+      const float lo = odd ? recv : v[2 * e2];
+      const float hi = odd ? v[2 * e2 + 1] : recv;
+      if (t < Cn) *reinterpret_cast<uint32_t *>(orow + t * tstride) = pack_bf16(lo, hi);
+    }
+  }
+}
+
 __device__ __forceinline__ void mma_sync_point() {
   fence_proxy_async_smem();
   tc_fence_before();
@@ -213,7 +275,6 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const KParams P) 
   const float log2x = P.lnx * kLog2e;
   const uint32_t lane_q = (uint32_t)(32 * (warp & 3)) << 16;  // this warp's TMEM lane quarter
   const int half = warp >> 2;
-  const size_t tstride = (size_t)P.H * kD;  // elements between consecutive tokens
 
   // ---- set-up: TMEM, barrier, accumulator, first chunk in flight ----
   if (warp == 0) {
@@ -221,7 +282,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const KParams P) 
     tmem_relinquish();
   }
   if (tid == 0) {
-    mbar_init(bar, 1);
+    for (int i = 0; i < kNumBars; ++i) mbar_init(bar + i, 1);
     fence_mbarrier_init();
   }
   if (tid < kD) Acar[tid] = (kPre && P.A0) ? P.A0[(size_t)bh * kD + tid] : 0.f;
@@ -235,14 +296,23 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const KParams P) 
   __syncthreads();
   tc_fence_after();
   const uint32_t tm = *tbase_p;
-  uint32_t phase = 0;
   bool aborted = false;
+  // MMA groups, each committed to its own mbarrier once per chunk (so the
+  // wait parity is the chunk index mod 2):
+  uint64_t *bar_m1 = bar + 0;  // MMA1  [Rh;Qh] Wh^T
+  uint64_t *bar_m6 = bar + 1;  // MMA6  O^T = S Qh^T
+  uint64_t *bar_m2 = bar + 2;  // MMA2  Y^T
+  uint64_t *bar_m3 = bar + 3;  // MMA3  U^T
+  uint64_t *bar_m5 = bar + 4;  // MMA5  D^T -= S Y^T
+  uint64_t *bar_m7 = bar + 5;  // MMA7/8
 
-  auto wait_mma = [&]() -> bool {
-    const bool ok = mbar_wait_bounded(bar, phase, kSpinLimit);
-    phase ^= 1u;
-    tc_fence_after();
+  // Only warp 0 polls; the other warps park at the block barrier, leaving
+  // the issue slots and the shared-memory pipe to warps with work.
+  auto wait_mma = [&](uint64_t *b_, int n_) -> bool {
+    bool ok = true;
+    if (warp == 0) ok = mbar_wait_bounded(b_, (uint32_t)(n_ & 1), kSpinLimit);
     const bool any_fail = __syncthreads_or(!ok);
+    tc_fence_after();
     if (any_fail && tid == 0) record_error(P.err, PDN_ERR_TIMEOUT);
     return !any_fail;
   };
@@ -282,6 +352,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const KParams P) 
         PARTG[i] = gs;
       }
       __syncthreads();
+      PDN_PHASE_MARK(16);
       float a = Acar[i] + (hf ? PARTK[i] : 0.f);
       float g = hf ? PARTG[i] : 0.f;
 #pragma unroll
@@ -435,53 +506,54 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const KParams P) 
     // k, q and the scalar gates of the next chunk fly during the rest of this one
     if (Cn_next > 0) stage_kq<kVariant, kDecay>(P, sb, b, h, c0 + kC, Cn_next, tid);
 
+    // ---- MMA1: D1 = [Rh;Qh] Wh^T  (runs under the state epilogue) ----
+    mma_sync_point();
+    if (tid == 0) {
+      const uint32_t id = make_idesc_bf16(128, 64, false, false);
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk)
+        mma_bf16_ss(tm + TM_D1, make_sdesc(sb + OFF_RQ + 256 * kk, 128, 2048),
+                    make_sdesc(sb + OFF_WH + 256 * kk, 128, 2048), id, kk > 0);
+      mma_commit(bar_m1);
+    }
+
     // ---- state epilogue of the previous chunk (or the initial state) ----
     // O of the previous chunk -> HBM; S (TMEM, fp32) -> bf16 operand copy;
     // TMEM S <- S Diag(e^{G_C}) for this chunk.
     {
       const int j = 32 * (warp & 3) + lane;
-      if (n > 0) {
-        __nv_bfloat16 *orow = reinterpret_cast<__nv_bfloat16 *>(P.o) +
-                              tok_index(P, b, c0 - kC, h) * kD + (j & ~1);
-        const bool odd = lane & 1;
+      if (n > 0) store_o_half(P, tm + lane_q + ot_col(n - 1) + 32 * half, b, h, c0 - kC, kC,
+                              32 * half, lane, warp & 3);
 #pragma unroll
-        for (int cc = 0; cc < 2; ++cc) {
-          float v[16];
-          tmem_ld16(tm + lane_q + TM_OT + 32 * half + 16 * cc, v);
-          tmem_wait_ld();
-          // lane pairs (j, j^1) exchange values so each stores two adjacent columns
-#pragma unroll
-          for (int e2 = 0; e2 < 8; ++e2) {
-            const float send = odd ? v[2 * e2] : v[2 * e2 + 1];
-            const float recv = __shfl_xor_sync(0xffffffffu, send, 1);
-            const int t = 32 * half + 16 * cc + 2 * e2 + (odd ? 1 : 0);
-            const float lo = odd ? recv : v[2 * e2];
-            const float hi = odd ? v[2 * e2 + 1] : recv;
-            *reinterpret_cast<uint32_t *>(orow + t * tstride) = pack_bf16(lo, hi);
-          }
-        }
-      }
-#pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
-        const int col = 64 * half + 16 * cc;
-        float v[16];
+      for (int cp = 0; cp < 2; ++cp) {
+        float sv[2][16];
         if (n == 0) {
-          if (P.S0) {
-            const float4 *src = reinterpret_cast<const float4 *>(
-                P.S0 + ((size_t)bh * kD + j) * kD + col);
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const float4 x = __ldg(src + e);
-              v[4 * e] = x.x; v[4 * e + 1] = x.y; v[4 * e + 2] = x.z; v[4 * e + 3] = x.w;
+          for (int u = 0; u < 2; ++u) {
+            const int col = 64 * half + 32 * cp + 16 * u;
+            if (P.S0) {
+              const float4 *src = reinterpret_cast<const float4 *>(
+                  P.S0 + ((size_t)bh * kD + j) * kD + col);
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const float4 x = __ldg(src + e);
+                sv[u][4 * e] = x.x; sv[u][4 * e + 1] = x.y;
+                sv[u][4 * e + 2] = x.z; sv[u][4 * e + 3] = x.w;
+              }
+            } else {
+#pragma unroll
+              for (int e = 0; e < 16; ++e) sv[u][e] = 0.f;
             }
-          } else {
-#pragma unroll
-            for (int e = 0; e < 16; ++e) v[e] = 0.f;
           }
         } else {
-          tmem_ld16(tm + lane_q + TM_S + col, v);
+          tmem_ld16(tm + lane_q + TM_S + 64 * half + 32 * cp, sv[0]);
+          tmem_ld16(tm + lane_q + TM_S + 64 * half + 32 * cp + 16, sv[1]);
           tmem_wait_ld();
         }
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+        const int col = 64 * half + 32 * cp + 16 * u;
+        float *v = sv[u];
         float lo[8], hi[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) { lo[e] = v[e]; hi[e] = v[8 + e]; }
@@ -494,23 +566,24 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const KParams P) 
         ld8f(EGC + col + 8, E);
 #pragma unroll
         for (int e = 0; e < 8; ++e) v[8 + e] *= E[e];
-        tmem_st16(tm + lane_q + TM_S + col, v);
+        tmem_st16(tm + lane_q + TM_S + col, *reinterpret_cast<float(*)[16]>(v));
+        }
       }
       tmem_wait_st();
     }
     mma_sync_point();
     PDN_PHASE_MARK(6);
 
-    // ---- MMA1: D1 = [Rh;Qh] Wh^T ----
+    // ---- MMA6: O^T = S Qh^T  (runs under the solve) ----
     if (tid == 0) {
-      const uint32_t id = make_idesc_bf16(128, 64, false, false);
+      const uint32_t id6 = make_idesc_bf16(128, 64, false, false);
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk)
-        mma_bf16_ss(tm + TM_D1, make_sdesc(sb + OFF_RQ + 256 * kk, 128, 2048),
-                    make_sdesc(sb + OFF_WH + 256 * kk, 128, 2048), id, kk > 0);
-      mma_commit(bar);
+        mma_bf16_ss(tm + ot_col(n), make_sdesc(sb + OFF_SB + 256 * kk, 128, 2048),
+                    make_sdesc(sb + OFF_RQ + 16384 + 256 * kk, 128, 2048), id6, kk > 0);
+      mma_commit(bar_m6);
     }
-    if (!wait_mma()) { aborted = true; break; }
+    if (!wait_mma(bar_m1, n)) { aborted = true; break; }
     PDN_PHASE_MARK(7);
 
     // ---- solve: M, P from TMEM; T = (I + M)^{-1} ----
@@ -524,7 +597,14 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const KParams P) 
         const int s0 = 32 * half + 16 * cc;
         if (row < kC) {
 #pragma unroll
-          for (int e = 0; e < 16; ++e) MS[row * MS_LD + s0 + e] = (s0 + e < row) ? v[e] : 0.f;
+          for (int e4 = 0; e4 < 4; ++e4) {
+            float4 x;
+            x.x = (s0 + 4 * e4 + 0 < row) ? v[4 * e4 + 0] : 0.f;
+            x.y = (s0 + 4 * e4 + 1 < row) ? v[4 * e4 + 1] : 0.f;
+            x.z = (s0 + 4 * e4 + 2 < row) ? v[4 * e4 + 2] : 0.f;
+            x.w = (s0 + 4 * e4 + 3 < row) ? v[4 * e4 + 3] : 0.f;
+            *reinterpret_cast<float4 *>(MS + row * MS_LD + s0 + 4 * e4) = x;
+          }
         } else {
           const int t = row - kC;
           float lo[8], hi[8];
@@ -575,12 +655,16 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const KParams P) 
       const int o = 32 * p, r0 = 2 * rb, c0b = 2 * cb;
       float a00 = 0.f, a01 = 0.f, a10 = 0.f, a11 = 0.f;
 #pragma unroll
-      for (int s = 0; s < 16; ++s) {
-        const float m0 = MS[(o + 16 + r0) * MS_LD + o + s];
-        const float m1 = MS[(o + 16 + r0 + 1) * MS_LD + o + s];
-        const float2 tv = *reinterpret_cast<const float2 *>(TS + (o + s) * TS_LD + o + c0b);
-        a00 = fmaf(m0, tv.x, a00); a01 = fmaf(m0, tv.y, a01);
-        a10 = fmaf(m1, tv.x, a10); a11 = fmaf(m1, tv.y, a11);
+      for (int s4 = 0; s4 < 16; s4 += 4) {
+        const float4 m0 = *reinterpret_cast<const float4 *>(MS + (o + 16 + r0) * MS_LD + o + s4);
+        const float4 m1 = *reinterpret_cast<const float4 *>(MS + (o + 16 + r0 + 1) * MS_LD + o + s4);
+        const float mv0[4] = {m0.x, m0.y, m0.z, m0.w}, mv1[4] = {m1.x, m1.y, m1.z, m1.w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const float2 tv = *reinterpret_cast<const float2 *>(TS + (o + s4 + k) * TS_LD + o + c0b);
+          a00 = fmaf(mv0[k], tv.x, a00); a01 = fmaf(mv0[k], tv.y, a01);
+          a10 = fmaf(mv1[k], tv.x, a10); a11 = fmaf(mv1[k], tv.y, a11);
+        }
       }
       float *y = YS + p * 16 * YS_LD;
       *reinterpret_cast<float2 *>(y + r0 * YS_LD + c0b) = make_float2(a00, a01);
@@ -593,12 +677,16 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const KParams P) 
       const float *y = YS + p * 16 * YS_LD;
       float a00 = 0.f, a01 = 0.f, a10 = 0.f, a11 = 0.f;
 #pragma unroll
-      for (int s = 0; s < 16; ++s) {
-        const float t0v = TS[(o + 16 + r0) * TS_LD + o + 16 + s];
-        const float t1v = TS[(o + 16 + r0 + 1) * TS_LD + o + 16 + s];
-        const float2 yv = *reinterpret_cast<const float2 *>(y + s * YS_LD + c0b);
-        a00 = fmaf(t0v, yv.x, a00); a01 = fmaf(t0v, yv.y, a01);
-        a10 = fmaf(t1v, yv.x, a10); a11 = fmaf(t1v, yv.y, a11);
+      for (int s4 = 0; s4 < 16; s4 += 4) {
+        const float4 t0 = *reinterpret_cast<const float4 *>(TS + (o + 16 + r0) * TS_LD + o + 16 + s4);
+        const float4 t1 = *reinterpret_cast<const float4 *>(TS + (o + 16 + r0 + 1) * TS_LD + o + 16 + s4);
+        const float tv0[4] = {t0.x, t0.y, t0.z, t0.w}, tv1[4] = {t1.x, t1.y, t1.z, t1.w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const float2 yv = *reinterpret_cast<const float2 *>(y + (s4 + k) * YS_LD + c0b);
+          a00 = fmaf(tv0[k], yv.x, a00); a01 = fmaf(tv0[k], yv.y, a01);
+          a10 = fmaf(tv1[k], yv.x, a10); a11 = fmaf(tv1[k], yv.y, a11);
+        }
       }
       *reinterpret_cast<float2 *>(TS + (o + 16 + r0) * TS_LD + o + c0b) = make_float2(-a00, -a01);
       *reinterpret_cast<float2 *>(TS + (o + 16 + r0 + 1) * TS_LD + o + c0b) =
@@ -609,13 +697,17 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const KParams P) 
     {
       const int r0 = 2 * (tid >> 4), c0b = 2 * (tid & 15);
       float a00 = 0.f, a01 = 0.f, a10 = 0.f, a11 = 0.f;
-#pragma unroll 8
-      for (int s = 0; s < 32; ++s) {
-        const float m0 = MS[(32 + r0) * MS_LD + s];
-        const float m1 = MS[(32 + r0 + 1) * MS_LD + s];
-        const float2 tv = *reinterpret_cast<const float2 *>(TS + s * TS_LD + c0b);
-        a00 = fmaf(m0, tv.x, a00); a01 = fmaf(m0, tv.y, a01);
-        a10 = fmaf(m1, tv.x, a10); a11 = fmaf(m1, tv.y, a11);
+#pragma unroll 4
+      for (int s4 = 0; s4 < 32; s4 += 4) {
+        const float4 m0 = *reinterpret_cast<const float4 *>(MS + (32 + r0) * MS_LD + s4);
+        const float4 m1 = *reinterpret_cast<const float4 *>(MS + (32 + r0 + 1) * MS_LD + s4);
+        const float mv0[4] = {m0.x, m0.y, m0.z, m0.w}, mv1[4] = {m1.x, m1.y, m1.z, m1.w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const float2 tv = *reinterpret_cast<const float2 *>(TS + (s4 + k) * TS_LD + c0b);
+          a00 = fmaf(mv0[k], tv.x, a00); a01 = fmaf(mv0[k], tv.y, a01);
+          a10 = fmaf(mv1[k], tv.x, a10); a11 = fmaf(mv1[k], tv.y, a11);
+        }
       }
       *reinterpret_cast<float2 *>(YS + r0 * YS_LD + c0b) = make_float2(a00, a01);
       *reinterpret_cast<float2 *>(YS + (r0 + 1) * YS_LD + c0b) = make_float2(a10, a11);
@@ -624,13 +716,17 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const KParams P) 
     {
       const int r0 = 2 * (tid >> 4), c0b = 2 * (tid & 15);
       float a00 = 0.f, a01 = 0.f, a10 = 0.f, a11 = 0.f;
-#pragma unroll 8
-      for (int s = 0; s < 32; ++s) {
-        const float t0v = TS[(32 + r0) * TS_LD + 32 + s];
-        const float t1v = TS[(32 + r0 + 1) * TS_LD + 32 + s];
-        const float2 yv = *reinterpret_cast<const float2 *>(YS + s * YS_LD + c0b);
-        a00 = fmaf(t0v, yv.x, a00); a01 = fmaf(t0v, yv.y, a01);
-        a10 = fmaf(t1v, yv.x, a10); a11 = fmaf(t1v, yv.y, a11);
+#pragma unroll 4
+      for (int s4 = 0; s4 < 32; s4 += 4) {
+        const float4 t0 = *reinterpret_cast<const float4 *>(TS + (32 + r0) * TS_LD + 32 + s4);
+        const float4 t1 = *reinterpret_cast<const float4 *>(TS + (32 + r0 + 1) * TS_LD + 32 + s4);
+        const float tv0[4] = {t0.x, t0.y, t0.z, t0.w}, tv1[4] = {t1.x, t1.y, t1.z, t1.w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const float2 yv = *reinterpret_cast<const float2 *>(YS + (s4 + k) * YS_LD + c0b);
+          a00 = fmaf(tv0[k], yv.x, a00); a01 = fmaf(tv0[k], yv.y, a01);
+          a10 = fmaf(tv1[k], yv.x, a10); a11 = fmaf(tv1[k], yv.y, a11);
+        }
       }
       *reinterpret_cast<float2 *>(TS + (32 + r0) * TS_LD + c0b) = make_float2(-a00, -a01);
       *reinterpret_cast<float2 *>(TS + (32 + r0 + 1) * TS_LD + c0b) = make_float2(-a10, -a11);
@@ -641,8 +737,9 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const KParams P) 
     for (int m = 0; m < 2; ++m) {
       const int t = 8 * warp + (lane & 7), s8 = 4 * m + (lane >> 3);
       float v[8];
+      ld8f(TS + t * TS_LD + 8 * s8, v);
 #pragma unroll
-      for (int e = 0; e < 8; ++e) v[e] = (8 * s8 + e <= t) ? TS[t * TS_LD + 8 * s8 + e] : 0.f;
+      for (int e = 0; e < 8; ++e) v[e] = (8 * s8 + e <= t) ? v[e] : 0.f;
       *reinterpret_cast<uint4 *>(smem + OFF_TM + tl64(t, s8)) = pack8(v);
     }
     mma_sync_point();
@@ -655,15 +752,17 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const KParams P) 
       for (int kk = 0; kk < 4; ++kk) {
         const uint64_t bd = make_sdesc(sb + OFF_TM + 256 * kk, 128, 1024);
         mma_bf16_ss(tm + TM_YT, make_sdesc(sb + OFF_RQ + 4096 * kk, 2048, 128), bd, id, kk > 0);
+      }
+      mma_commit(bar_m2);
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk) {
+        const uint64_t bd = make_sdesc(sb + OFF_TM + 256 * kk, 128, 1024);
         mma_bf16_ss(tm + TM_UD, make_sdesc(sb + OFF_U + 4096 * kk, 2048, 128), bd, id, kk > 0);
       }
-      mma_commit(bar);
+      mma_commit(bar_m3);
     }
-    if (!wait_mma()) { aborted = true; break; }
+    if (!wait_mma(bar_m2, n)) { aborted = true; break; }
     PDN_PHASE_MARK(11);
-
-    // the next chunk's v flies while this chunk finishes
-    if (Cn_next > 0) stage_rows(P, P.v, sb + OFF_U, true, b, h, c0 + kC, Cn_next, tid);
 
     // ---- Y^T -> bf16 operand (rows d_k, columns tokens) ----
     {
@@ -684,20 +783,20 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const KParams P) 
     mma_sync_point();
     PDN_PHASE_MARK(12);
 
-    // ---- MMA5: D^T = U^T - S Y^T ; MMA6: O^T = S Qh^T ----
+    // ---- MMA5: D^T = U^T - S Y^T (accumulates onto MMA3's U^T, issued after it) ----
     if (tid == 0) {
       const uint32_t id5 = make_idesc_bf16(128, 64, false, true, true);
-      const uint32_t id6 = make_idesc_bf16(128, 64, false, false);
 #pragma unroll
-      for (int kk = 0; kk < 8; ++kk) {
-        const uint64_t ad = make_sdesc(sb + OFF_SB + 256 * kk, 128, 2048);
-        mma_bf16_ss(tm + TM_UD, ad, make_sdesc(sb + OFF_YT + 2048 * kk, 1024, 128), id5, 1);
-        mma_bf16_ss(tm + TM_OT, ad, make_sdesc(sb + OFF_RQ + 16384 + 256 * kk, 128, 2048), id6,
-                    kk > 0);
-      }
-      mma_commit(bar);
+      for (int kk = 0; kk < 8; ++kk)
+        mma_bf16_ss(tm + TM_UD, make_sdesc(sb + OFF_SB + 256 * kk, 128, 2048),
+                    make_sdesc(sb + OFF_YT + 2048 * kk, 1024, 128), id5, 1);
+      mma_commit(bar_m5);
     }
-    if (!wait_mma()) { aborted = true; break; }
+    // the next chunk's v flies while MMA5 runs (MMA3 has finished reading U)
+    if (!wait_mma(bar_m3, n)) { aborted = true; break; }
+    if (Cn_next > 0) stage_rows(P, P.v, sb + OFF_U, true, b, h, c0 + kC, Cn_next, tid);
+    if (!wait_mma(bar_m6, n)) { aborted = true; break; }
+    if (!wait_mma(bar_m5, n)) { aborted = true; break; }
     PDN_PHASE_MARK(13);
 
     // SB is free until the next state epilogue: stage the next chunk's channel decay there
@@ -730,12 +829,12 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const KParams P) 
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk) {
         const uint64_t ad = make_sdesc(sb + OFF_DT + 256 * kk, 128, 1024);
-        mma_bf16_ss(tm + TM_OT, ad, make_sdesc(sb + OFF_PM + 256 * kk, 128, 1024), id7, 1);
+        mma_bf16_ss(tm + ot_col(n), ad, make_sdesc(sb + OFF_PM + 256 * kk, 128, 1024), id7, 1);
         mma_bf16_ss(tm + TM_S, ad, make_sdesc(sb + OFF_WB + 4096 * kk, 2048, 128), id8, 1);
       }
-      mma_commit(bar);
+      mma_commit(bar_m7);
     }
-    if (!wait_mma()) { aborted = true; break; }
+    if (!wait_mma(bar_m7, n)) { aborted = true; break; }
     PDN_PHASE_MARK(15);
   }
 
@@ -743,19 +842,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const KParams P) 
   if (!aborted && nchunks > 0) {
     const int j = 32 * (warp & 3) + lane;
     const int pc0 = (nchunks - 1) * kC;
-    const int Cn = P.T - pc0;
-    __nv_bfloat16 *ocol = reinterpret_cast<__nv_bfloat16 *>(P.o) + tok_index(P, b, pc0, h) * kD + j;
-#pragma unroll
-    for (int cc = 0; cc < 2; ++cc) {
-      float v[16];
-      tmem_ld16(tm + lane_q + TM_OT + 32 * half + 16 * cc, v);
-      tmem_wait_ld();
-#pragma unroll
-      for (int e = 0; e < 16; ++e) {
-        const int t = 32 * half + 16 * cc + e;
-        if (t < Cn) ocol[t * tstride] = __float2bfloat16_rn(v[e]);
-      }
-    }
+    if (warp < 4) store_o_tile(P, tm + lane_q + ot_col(nchunks - 1), b, h, pc0, P.T - pc0, lane, warp);
     if (P.ST) {
 #pragma unroll
       for (int cc = 0; cc < 4; ++cc) {

@@ -10,7 +10,9 @@
 // rows: lane l holds key channels 4l..4l+3 as one float4, two warp
 // reductions give y_j and z_j, and the updated row is written back in place.
 // The kernel is bound by HBM: 8 d_k d_v bytes of state traffic per
-// (token, head) against about 7 d_k d_v flops.
+// (token, head) against about 7 d_k d_v flops. For d_k = d_v = 128 a
+// persistent variant streams the state through shared memory with bulk
+// copies (see decode_tma_kernel).
 #include "common.cuh"
 #include "internal.h"
 #include "ptx.cuh"
@@ -144,6 +146,259 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const KParams P) {
   }
 }
 
+// ---------------------------------------------------------------------------
+// d_k = d_v = 128: persistent, warp-specialised variant. One CTA per SM walks
+// the (batch, head) items. A producer warp streams each item's 64 KiB state
+// into a ring of shared-memory buffers with 1-D bulk copies (TMA) and streams
+// the updated buffer back with bulk stores; eight consumer warps do the
+// per-token prologue and the row updates in shared memory. Full/empty
+// mbarriers hand buffers between the two; every wait is bounded.
+constexpr int kTmaBufs = 3;
+constexpr int kD128 = 128;
+constexpr int kConsumers = kThreads;      // 8 consumer warps
+constexpr int kTmaThreads = kThreads + 32;  // + 1 producer warp
+constexpr uint32_t kStateBytes = kD128 * kD128 * 4;
+constexpr uint32_t kPart = 16384;  // bytes per bulk copy
+constexpr long long kDecSpin = 1LL << 22;
+
+struct DecSmem {
+  float buf[kTmaBufs][kD128 * kD128];
+  float r[kD128], w[kD128], q[kD128], al[kD128], u[kD128];
+  float red[kWarps];
+  uint64_t full[kTmaBufs];
+  uint64_t empty[kTmaBufs];
+  int vote[kWarps];
+  int abort_flag;
+};
+
+// Barrier among the consumer warps only (id 1); the producer never joins it.
+__device__ __forceinline__ void consumer_sync() {
+  asm volatile("bar.sync 1, %0;" ::"r"(kConsumers) : "memory");
+}
+
+__device__ __forceinline__ float consumer_sum(float v, float *red) {
+  v = warp_sum(v);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  consumer_sync();
+  if (lane == 0) red[warp] = v;
+  consumer_sync();
+  float s = 0.f;
+#pragma unroll
+  for (int w = 0; w < kWarps; ++w) s += red[w];
+  return s;
+}
+
+__device__ __forceinline__ void issue_state_load(DecSmem &sm, int s, const float *S) {
+  mbar_arrive_expect_tx(&sm.full[s], kStateBytes);
+#pragma unroll
+  for (int p = 0; p < (int)(kStateBytes / kPart); ++p)
+    bulk_g2s(reinterpret_cast<uint8_t *>(sm.buf[s]) + p * kPart,
+             reinterpret_cast<const uint8_t *>(S) + p * kPart, kPart, &sm.full[s]);
+}
+
+__device__ __forceinline__ void issue_state_store(DecSmem &sm, int s, float *S) {
+#pragma unroll
+  for (int p = 0; p < (int)(kStateBytes / kPart); ++p)
+    bulk_s2g(reinterpret_cast<uint8_t *>(S) + p * kPart,
+             reinterpret_cast<const uint8_t *>(sm.buf[s]) + p * kPart, kPart);
+  bulk_commit();
+}
+
+template <typename Tin>
+__global__ void __launch_bounds__(kTmaThreads, 1) decode_tma_kernel(const KParams P, int items) {
+  extern __shared__ __align__(128) uint8_t smem_raw[];
+  DecSmem &sm = *reinterpret_cast<DecSmem *>(smem_raw);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int G = gridDim.x;
+  const int nloc = blockIdx.x < items ? (items - blockIdx.x + G - 1) / G : 0;
+  const bool precond = is_precond(P.variant);
+  auto state_of = [&](int k) { return P.ST + (size_t)(blockIdx.x + k * G) * (kD128 * kD128); };
+
+  if (tid == 0) {
+    for (int s = 0; s < kTmaBufs; ++s) {
+      mbar_init(&sm.full[s], 1);
+      mbar_init(&sm.empty[s], kWarps);
+    }
+    sm.abort_flag = 0;
+    fence_mbarrier_init();
+  }
+  __syncthreads();
+
+  if (warp == kWarps) {
+    // ---------------- producer warp
+    if (lane == 0) {
+      int loaded = 0;  // loads issued
+      for (int k = 0; k < nloc; ++k) {
+        const int s = k % kTmaBufs;
+        if (k >= kTmaBufs) {
+          // the consumers are done with item k - kTmaBufs in buffer s
+          if (!mbar_wait_bounded(&sm.empty[s], (uint32_t)(((k / kTmaBufs) - 1) & 1), kDecSpin) ||
+              *reinterpret_cast<volatile int *>(&sm.abort_flag)) {
+            atomicExch(&sm.abort_flag, 1);
+            break;
+          }
+          issue_state_store(sm, s, state_of(k - kTmaBufs));
+          bulk_wait_read0();
+        }
+        issue_state_load(sm, s, state_of(k));
+        loaded = k + 1;
+      }
+      // write back the last items, then wait for all stores
+      for (int k = (loaded > kTmaBufs ? loaded - kTmaBufs : 0); k < loaded; ++k) {
+        const int s = k % kTmaBufs;
+        if (!mbar_wait_bounded(&sm.empty[s], (uint32_t)((k / kTmaBufs) & 1), kDecSpin)) {
+          atomicExch(&sm.abort_flag, 1);
+          // drain the load into this buffer before giving up on it
+          mbar_wait_bounded(&sm.full[s], (uint32_t)((k / kTmaBufs) & 1), kDecSpin);
+          continue;
+        }
+        issue_state_store(sm, s, state_of(k));
+      }
+      bulk_wait0();
+      if (sm.abort_flag) record_error(P.err, PDN_ERR_TIMEOUT);
+    }
+    return;
+  }
+
+  // ---------------- consumer warps
+  // Token data of one item, loaded one item ahead (thread = key/value channel).
+  struct Tok {
+    float k, q, v, a, beta, la, ge, gw;
+  };
+  const bool chan = tid < kD128;
+  auto load_tok = [&](int kk) {
+    Tok t{0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 1.f, 1.f};
+    const int item = blockIdx.x + kk * G;
+    const size_t tokh = tok_index(P, item / P.H, 0, item % P.H);
+    if (chan) {
+      const size_t e = tokh * kD128 + tid;
+      t.k = ldf<Tin>(P.k, e);
+      t.q = ldf<Tin>(P.q, e);
+      t.v = ldf<Tin>(P.v, e);
+      if (precond) t.a = P.AT[(size_t)item * kD128 + tid];
+      if (P.variant == PDN_VAR_FG2_GDN) t.beta = ldf<Tin>(P.beta, e);
+      else if (P.variant != PDN_VAR_GDN2) t.beta = ldf<float>(P.beta, tokh);
+      if (P.decay == PDN_DECAY_SCALAR) t.la = ldf<float>(P.log_alpha, tokh);
+      else if (P.decay == PDN_DECAY_CHANNEL) t.la = ldf<Tin>(P.log_alpha, e);
+      if (P.variant == PDN_VAR_GDN2) {
+        t.ge = ldf<Tin>(P.erase, e);
+        t.gw = ldf<Tin>(P.write, e);
+      }
+    }
+    return t;
+  };
+  Tok cur = nloc > 0 ? load_tok(0) : Tok{};
+  for (int k = 0; k < nloc; ++k) {
+    const int s = k % kTmaBufs;
+    const int item = blockIdx.x + k * G;
+    const int b = item / P.H, h = item % P.H;
+    const size_t tokh = tok_index(P, b, 0, h);
+    const Tok nxt = (k + 1 < nloc) ? load_tok(k + 1) : cur;
+
+    // per-token vectors (overlap the bulk loads in flight)
+    const float kv = cur.k, qv = cur.q;
+    float logA = 0.f;
+    if (chan && precond) {
+      const float a = cur.a + kv * kv;
+      P.AT[(size_t)item * kD128 + tid] = a;
+      logA = logf(a + P.eps);
+    }
+    float mu = 0.f;
+    if (precond) mu = consumer_sum(chan ? logA : 0.f, sm.red) / (float)kD128;
+    float w = 0.f;
+    if (chan) {
+      float r, u = cur.v;
+      switch (P.variant) {
+        case PDN_VAR_PDN: case PDN_VAR_PGDN: case PDN_VAR_PKDA:
+          r = kv;
+          w = cur.beta * precond_coef(logA, mu, P.lnx) * kv;
+          break;
+        case PDN_VAR_FG2_GDN: {
+          const float sb = sqrtf(cur.beta);
+          r = sb * kv;
+          w = r;
+          u *= sb;
+        } break;
+        case PDN_VAR_GDN2:
+          r = cur.ge * kv;
+          w = kv;
+          u *= cur.gw;
+          break;
+        default:
+          r = kv;
+          w = cur.beta * kv;
+      }
+      sm.r[tid] = r;
+      sm.w[tid] = w;
+      sm.q[tid] = qv;
+      sm.al[tid] = P.decay == PDN_DECAY_NONE ? 1.f : expf(cur.la);
+      sm.u[tid] = u;
+    }
+    const float wq = consumer_sum(chan ? w * qv : 0.f, sm.red);  // ends with consumer_sync
+
+    // Wait for the state. The decision to stop must be the same in every
+    // consumer warp (they meet at named barriers): each warp votes once,
+    // after a consumer barrier all warps read all votes.
+    const bool ok = mbar_wait_bounded(&sm.full[s], (uint32_t)((k / kTmaBufs) & 1), kDecSpin);
+    int vote = __all_sync(0xffffffffu, ok) ? 1 : 0;
+    if (lane == 0) {
+      if (*reinterpret_cast<volatile int *>(&sm.abort_flag)) vote = 0;
+      sm.vote[warp] = vote;
+    }
+    consumer_sync();
+    bool all_ok = true;
+#pragma unroll
+    for (int i = 0; i < kWarps; ++i) all_ok = all_ok && sm.vote[i];
+    if (!all_ok) {
+      if (tid == 0) atomicExch(&sm.abort_flag, 1);
+      break;
+    }
+
+    const int c = lane * 4;
+    const float4 rr = make_float4(sm.r[c], sm.r[c + 1], sm.r[c + 2], sm.r[c + 3]);
+    const float4 ww = make_float4(sm.w[c], sm.w[c + 1], sm.w[c + 2], sm.w[c + 3]);
+    const float4 qq = make_float4(sm.q[c], sm.q[c + 1], sm.q[c + 2], sm.q[c + 3]);
+    const float4 aa = make_float4(sm.al[c], sm.al[c + 1], sm.al[c + 2], sm.al[c + 3]);
+    float *S = sm.buf[s];
+#pragma unroll 4
+    for (int m = 0; m < kD128 / kWarps; ++m) {
+      const int j = warp + m * kWarps;
+      float4 x = *reinterpret_cast<const float4 *>(S + j * kD128 + c);
+      x.x *= aa.x; x.y *= aa.y; x.z *= aa.z; x.w *= aa.w;
+      const float y = warp_sum(x.x * rr.x + x.y * rr.y + x.z * rr.z + x.w * rr.w);
+      const float z = warp_sum(x.x * qq.x + x.y * qq.y + x.z * qq.z + x.w * qq.w);
+      const float delta = sm.u[j] - y;
+      x.x = fmaf(delta, ww.x, x.x);
+      x.y = fmaf(delta, ww.y, x.y);
+      x.z = fmaf(delta, ww.z, x.z);
+      x.w = fmaf(delta, ww.w, x.w);
+      *reinterpret_cast<float4 *>(S + j * kD128 + c) = x;
+      if (lane == 0) stf<Tin>(P.o, tokh * kD128 + j, P.q_scale * fmaf(delta, wq, z));
+    }
+    // hand the buffer back: generic writes -> async proxy, then one arrive per warp
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&sm.empty[s]);
+    // r/w/q/al/u are rewritten by the next prologue: all warps must be past the rows
+    consumer_sync();
+    cur = nxt;
+  }
+}
+
+int g_num_sms[64];
+
+int num_sms() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (!g_num_sms[dev]) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+      n = 148;
+    g_num_sms[dev] = n;
+  }
+  return g_num_sms[dev];
+}
+
 __global__ void selftest_wait_kernel(long long limit, int *err) {
   __shared__ __align__(8) uint64_t bar;
   if (threadIdx.x == 0) {
@@ -160,6 +415,24 @@ __global__ void selftest_wait_kernel(long long limit, int *err) {
 cudaError_t launch_decode(const KParams &P, cudaStream_t stream) {
   const long long grid = (long long)P.B * P.H;
   if (grid <= 0) return cudaSuccess;
+  if (P.dk == kD128 && P.dv == kD128) {
+    const int items = (int)grid;
+    const int ctas = items < num_sms() ? items : num_sms();
+    const size_t smem = sizeof(DecSmem);
+    cudaError_t e;
+    if (P.dtype == PDN_F32) {
+      e = cudaFuncSetAttribute(decode_tma_kernel<float>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      if (e != cudaSuccess) return e;
+      decode_tma_kernel<float><<<ctas, kTmaThreads, smem, stream>>>(P, items);
+    } else {
+      e = cudaFuncSetAttribute(decode_tma_kernel<__nv_bfloat16>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      if (e != cudaSuccess) return e;
+      decode_tma_kernel<__nv_bfloat16><<<ctas, kTmaThreads, smem, stream>>>(P, items);
+    }
+    return cudaGetLastError();
+  }
   if (P.dtype == PDN_F32)
     decode_kernel<float><<<(unsigned)grid, kThreads, 0, stream>>>(P);
   else

@@ -91,3 +91,24 @@ def test_decode_workload_shape_sampled():
     assert nmax_err(o.float().cpu().numpy(), ro) <= 2e-2
     assert nmax_err(S.cpu().numpy(), rS) <= 2e-2
     assert nmax_err(A.cpu().numpy(), rA) <= 1e-6
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("variant", VARIANTS)
+def test_decode_d128_many_heads(variant, dtype):
+    """d = 128 with more (batch, head) items than SMs, so the persistent
+    streaming kernel cycles each CTA through its ring of state buffers."""
+    w = Workload("dec128", variant, 40, 3, 8, 128, 128, dtype, DECAY[variant], q_scale=1.1)
+    x = make_inputs(w)
+    g = torch.Generator().manual_seed(4)
+    S0 = 0.2 * torch.randn(w.B, w.H, 128, 128, generator=g)
+    A0 = torch.rand(w.B, w.H, 128, generator=g) if variant in ("PDN", "PGDN", "PKDA") else None
+    S = S0.cuda()
+    A = A0.cuda() if A0 is not None else None
+    o = decode_all(w, x, S, A, w.T)
+    ro, rS, rA = run_oracle(w, x, S0, A0)
+    tol = TOL[dtype]
+    assert nmax_err(o.float().cpu().numpy(), ro) <= tol
+    assert nmax_err(S.cpu().numpy(), rS) <= tol
+    if A is not None:
+        assert nmax_err(A.cpu().numpy(), rA) <= 1e-6
