@@ -101,6 +101,30 @@ DECODE_SOURCES = ["linear_recurrence_sequence_chunked_b200/csrc/decode.cu",
                   "linear_recurrence_sequence_chunked_b200/csrc/common.cuh"]
 
 
+# ------------------------------------------------------------------ multi-rank host logic
+def rank_seed(seed, rank):
+    """Each rank draws its own independent batch (weak scaling: per-GPU work
+    is fixed, nothing is exchanged on the data path)."""
+    return seed + 1000 * rank
+
+
+def max_over_ranks(x, world, device=None):
+    """The slowest rank's device time; one all-reduce of a scalar (any
+    torch.distributed backend), outside the data path."""
+    if world == 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def throughput(units_per_rank, world, ms_max):
+    """Whole-job units per second: every rank's units over the max time."""
+    return world * units_per_rank / (ms_max / 1e3)
+
+
 # ------------------------------------------------------------------ clocks
 class ClockSampler:
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
@@ -218,17 +242,13 @@ def run_ours(args):
             dist.barrier()
         torch.cuda.synchronize()
 
-    def max_over_ranks(x):
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+    def mor(x):
+        return max_over_ranks(x, world, dev)
 
     w = WORKLOADS[args.workload]
     peaks, peaks_kind = load_peaks()
     # each rank: its own independent batch (different seed)
-    wr = w.replace(seed=w.seed + 1000 * rank)
+    wr = w.replace(seed=rank_seed(w.seed, rank))
     x = make_inputs(wr, device=dev, generator_device=dev)
     g = {n: x[n] for n in ("log_alpha", "beta", "erase", "write")}
     impl = args.kernel
@@ -270,9 +290,9 @@ def run_ours(args):
         barrier()
     clocks = clk.summary()
     ms_local = sum(a.elapsed_time(b) for a, b in ev)
-    ms = max_over_ranks(ms_local)
+    ms = mor(ms_local)
     tokens = world * w.B * w.T * args.steps
-    value = tokens / (ms / 1e3)
+    value = throughput(w.B * w.T * args.steps, world, ms)
     ms_launch = ms_local / args.steps
     flops = chunk_flops_per_token_head(w.chunk, w.dk, w.dv) * w.B * w.T * w.H
     ach_tflops = flops / (ms_launch / 1e3) / 1e12
@@ -329,7 +349,7 @@ def run_ours(args):
             e2e_step()
         e1.record(stream)
         barrier()
-        ems = max_over_ranks(e0.elapsed_time(e1))
+        ems = mor(e0.elapsed_time(e1))
         result["e2e"] = {"value": tokens / (ems / 1e3), "unit": "tokens/s",
                          "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                          "ms_per_step": ems / args.steps}
@@ -339,7 +359,7 @@ def run_ours(args):
     # ---------------- decode workload
     if not args.no_decode:
         result["decode"] = bench_decode(args, dev, stream, peaks, peaks_kind, world, rank,
-                                        max_over_ranks, barrier)
+                                        mor, barrier)
         result["gpu_launches"] += result["decode"]["gpu_launches"]
 
     # ---------------- CPU baseline (rank 0, N=1 only)
@@ -354,7 +374,7 @@ def run_ours(args):
         print(json.dumps(result), flush=True)
 
 
-def bench_decode(args, dev, stream, peaks, peaks_kind, world, rank, max_over_ranks, barrier):
+def bench_decode(args, dev, stream, peaks, peaks_kind, world, rank, mor, barrier):
     import torch
 
     from linear_recurrence_sequence_chunked_b200 import pdn
@@ -362,7 +382,7 @@ def bench_decode(args, dev, stream, peaks, peaks_kind, world, rank, max_over_ran
 
     w = WORKLOADS["pgdn_decode_256"]
     steps = args.decode_steps
-    wr = w.replace(seed=w.seed + 1000 * rank)
+    wr = w.replace(seed=rank_seed(w.seed, rank))
     x = make_inputs(wr, device=dev, generator_device=dev, T=steps)
     # step-major copies so that each step's token slice is contiguous
     xs = {n: (t.transpose(0, 1).contiguous() if t is not None else None) for n, t in x.items()}
@@ -399,11 +419,11 @@ def bench_decode(args, dev, stream, peaks, peaks_kind, world, rank, max_over_ran
     if pdn.device_error() != pdn.PDN_OK:
         raise SystemExit("device error in decode")
     ms_local = e0.elapsed_time(e1)
-    ms = max_over_ranks(ms_local)
+    ms = mor(ms_local)
     per_step = ms_local / steps
     byts = decode_bytes_per_token_head(w) * w.B * w.H
     gbs = byts / (per_step / 1e3) / 1e9
-    return {"workload": w.name, "value": world * w.B * steps / (ms / 1e3), "unit": "tokens/s",
+    return {"workload": w.name, "value": throughput(w.B * steps, world, ms), "unit": "tokens/s",
             "steps": steps, "ms_per_step": ms / steps, "gpu_launches": steps,
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"],
                          "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"],
@@ -421,7 +441,7 @@ def run_reference(args):
     if rank != 0:
         return
     w = WORKLOADS[args.workload]
-    secs = max(2.0, min(20.0, 150.0 / max(1, args.steps + args.warmup)))
+    secs = max(0.5, min(20.0, 150.0 / max(1, args.steps + args.warmup), args.cpu_seconds))
     rates = []
     desc = cores = None
     for i in range(args.warmup + args.steps):
