@@ -299,7 +299,13 @@ def run_ours(args):
     peak = peaks["bf16_tflops"]
     if pdn.device_error() != pdn.PDN_OK:
         raise SystemExit("device error during the timed region")
-    tc = pdn.pdn_chunk_fwd_impl(prob) == pdn.IMPLS["tc"]
+    impl_id = pdn.pdn_chunk_fwd_impl(prob)
+    tc = impl_id in (pdn.IMPLS["tc"], pdn.IMPLS["tc_fused"])
+    kernel_name = {1: "simt", 2: "tcgen05 split (K0 prefix, K1 intra, K2 state)",
+                   3: "tcgen05 fused"}.get(impl_id, "?")
+    launches_per_step = 1
+    if impl_id == pdn.IMPLS["tc"]:
+        launches_per_step = 4 if w.variant in pdn.PRECOND_VARIANTS else 2
 
     result = {
         "metric": "fwd tokens/s per layer (H16,d128,T4K) + % roofline; decode tokens/s",
@@ -309,7 +315,7 @@ def run_ours(args):
         "data": "synthetic",
         "config": {"workload": w.name, "variant": w.variant, "B": w.B, "T": w.T, "H": w.H,
                    "d_k": w.dk, "d_v": w.dv, "chunk": w.chunk, "inputs": w.dtype,
-                   "state": "f32", "kernel": "tcgen05" if tc else "simt",
+                   "state": "f32", "kernel": kernel_name,
                    "per_gpu_batch": w.B, "global_batch": w.B * world,
                    "l2": "flushed between timed steps (256 MiB write)",
                    "parallelism": "dp%d" % world},
@@ -318,7 +324,7 @@ def run_ours(args):
                      "flops_per_launch": flops,
                      "traffic": traffic_for("chunk_fwd:" + w.name, CHUNK_SOURCES)},
         "clocks": clocks,
-        "gpu_launches": args.steps,
+        "gpu_launches": args.steps * launches_per_step,
     }
 
     # ---------------- e2e: pinned host buffers, copies inside the timed region
@@ -353,7 +359,7 @@ def run_ours(args):
         result["e2e"] = {"value": tokens / (ems / 1e3), "unit": "tokens/s",
                          "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                          "ms_per_step": ems / args.steps}
-        result["gpu_launches"] += args.steps
+        result["gpu_launches"] += args.steps * launches_per_step
         del hx, ho, dx
 
     # ---------------- decode workload
@@ -474,7 +480,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="pgdn_bf16_4k")
-    ap.add_argument("--kernel", choices=["auto", "simt", "tc"], default="auto")
+    ap.add_argument("--kernel", choices=["auto", "simt", "tc", "tc_fused"], default="auto")
     ap.add_argument("--decode-steps", type=int, default=1024)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-decode", action="store_true")

@@ -77,9 +77,14 @@ typedef enum { PDN_DECAY_NONE = 0, PDN_DECAY_SCALAR = 1, PDN_DECAY_CHANNEL = 2 }
  * and the preconditioner accumulator are always fp32. */
 typedef enum { PDN_F32 = 0, PDN_BF16 = 1 } pdn_dtype_t;
 
-/* Kernel selection for pdn_chunk_fwd: AUTO picks the tensor-core (tcgen05)
- * kernel where one exists for the problem, else the CUDA-core kernel. */
-typedef enum { PDN_IMPL_AUTO = 0, PDN_IMPL_SIMT = 1, PDN_IMPL_TC = 2 } pdn_impl_t;
+/* Kernel selection for pdn_chunk_fwd. TC is the tensor-core (tcgen05) path
+ * that runs the intra-chunk work of all chunks at once and then the
+ * sequential state pass (needs a workspace); TC_FUSED is the single-kernel
+ * tensor-core path (no workspace); SIMT is the CUDA-core kernel (any
+ * supported shape, fp32 arithmetic). AUTO picks TC, else TC_FUSED, else SIMT.
+ * The tensor-core paths take bf16 inputs with d_k = d_v = 128, chunk 64. */
+typedef enum { PDN_IMPL_AUTO = 0, PDN_IMPL_SIMT = 1, PDN_IMPL_TC = 2,
+               PDN_IMPL_TC_FUSED = 3 } pdn_impl_t;
 
 typedef struct {
   int B, T, H;          /* batch, tokens per sequence, heads; B,H >= 1, T >= 0
@@ -114,9 +119,9 @@ typedef struct {
  * (0 if none; (size_t)-1 if p is invalid). */
 size_t pdn_chunk_fwd_workspace(const pdn_problem_t *p);
 
-/* Which kernel pdn_chunk_fwd runs for problem p: PDN_IMPL_SIMT (CUDA cores)
- * or PDN_IMPL_TC (tcgen05 tensor cores); -1 if p is invalid or no kernel of
- * this build supports it. Host-only, touches no device. */
+/* Which path pdn_chunk_fwd runs for problem p: PDN_IMPL_SIMT, PDN_IMPL_TC or
+ * PDN_IMPL_TC_FUSED; -1 if p is invalid or no kernel of this build supports
+ * it. Host-only, touches no device. */
 int pdn_chunk_fwd_impl(const pdn_problem_t *p);
 
 /* Chunked forward over T tokens (prefill / training forward).

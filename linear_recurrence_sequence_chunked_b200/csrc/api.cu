@@ -56,7 +56,7 @@ pdn_status_t check_problem(const pdn_problem_t *p) {
   if ((int)p->variant < PDN_VAR_DN || (int)p->variant > PDN_VAR_GDN2) return PDN_ERR_INVALID_ARG;
   if ((int)p->decay < PDN_DECAY_NONE || (int)p->decay > PDN_DECAY_CHANNEL) return PDN_ERR_INVALID_ARG;
   if (p->dtype != PDN_F32 && p->dtype != PDN_BF16) return PDN_ERR_INVALID_ARG;
-  if ((int)p->impl < PDN_IMPL_AUTO || (int)p->impl > PDN_IMPL_TC) return PDN_ERR_INVALID_ARG;
+  if ((int)p->impl < PDN_IMPL_AUTO || (int)p->impl > PDN_IMPL_TC_FUSED) return PDN_ERR_INVALID_ARG;
   bool fixed;
   const pdn_decay_t need = required_decay(p->variant, &fixed);
   if (fixed && p->decay != need) return PDN_ERR_INVALID_ARG;
@@ -112,9 +112,21 @@ KParams make_params(const pdn_problem_t *p, const pdn_tensors_t *t, int *err) {
   return P;
 }
 
-bool use_tc(const pdn_problem_t *p, const KParams &P) {
-  if (p->impl == PDN_IMPL_SIMT) return false;
-  return tc_supported(P) != 0;
+// The path pdn_chunk_fwd takes, or -1 when the requested one cannot run.
+int select_impl(const pdn_problem_t *p, const KParams &P) {
+  switch (p->impl) {
+    case PDN_IMPL_SIMT: return simt_supported(P) ? PDN_IMPL_SIMT : -1;
+    case PDN_IMPL_TC: return split_supported(P) ? PDN_IMPL_TC : -1;
+    case PDN_IMPL_TC_FUSED: return tc_supported(P) ? PDN_IMPL_TC_FUSED : -1;
+    default:
+      if (split_supported(P)) return PDN_IMPL_TC;
+      if (tc_supported(P)) return PDN_IMPL_TC_FUSED;
+      return simt_supported(P) ? PDN_IMPL_SIMT : -1;
+  }
+}
+
+size_t workspace_for(int impl, const KParams &P) {
+  return impl == PDN_IMPL_TC ? split_workspace_bytes(P) : 0;
 }
 
 }  // namespace
@@ -127,7 +139,8 @@ extern "C" size_t pdn_chunk_fwd_workspace(const pdn_problem_t *p) {
   pdn_tensors_t dummy;
   memset(&dummy, 0, sizeof(dummy));
   const KParams P = make_params(p, &dummy, nullptr);
-  return use_tc(p, P) ? tc_workspace_bytes(P) : 0;
+  const int impl = select_impl(p, P);
+  return impl < 0 ? 0 : workspace_for(impl, P);
 }
 
 extern "C" int pdn_chunk_fwd_impl(const pdn_problem_t *p) {
@@ -135,9 +148,7 @@ extern "C" int pdn_chunk_fwd_impl(const pdn_problem_t *p) {
   pdn_tensors_t dummy;
   memset(&dummy, 0, sizeof(dummy));
   const KParams P = make_params(p, &dummy, nullptr);
-  if (use_tc(p, P)) return PDN_IMPL_TC;
-  if (p->impl == PDN_IMPL_TC || !simt_supported(P)) return -1;
-  return PDN_IMPL_SIMT;
+  return select_impl(p, P);
 }
 
 extern "C" pdn_status_t pdn_chunk_fwd(const pdn_problem_t *p, const pdn_tensors_t *t,
@@ -146,17 +157,19 @@ extern "C" pdn_status_t pdn_chunk_fwd(const pdn_problem_t *p, const pdn_tensors_
   if (st != PDN_OK) return st;
   if ((st = check_tensors(p, t)) != PDN_OK) return st;
   KParams P = make_params(p, t, nullptr);
-  const bool tc = use_tc(p, P);
-  if (p->impl == PDN_IMPL_TC && !tc) return PDN_ERR_UNSUPPORTED;
-  if (!tc && !simt_supported(P)) return PDN_ERR_UNSUPPORTED;
-  const size_t need = tc ? tc_workspace_bytes(P) : 0;
+  const int impl = select_impl(p, P);
+  if (impl < 0) return PDN_ERR_UNSUPPORTED;
+  const size_t need = workspace_for(impl, P);
   if (need > 0) {
     if (!workspace || ws_bytes < need || ((uintptr_t)workspace & 255u)) return PDN_ERR_WORKSPACE;
   }
   P.err = device_error_word();
   if (!P.err) return PDN_ERR_CUDA;
   const cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const cudaError_t e = tc ? launch_chunk_tc(P, workspace, s) : launch_chunk_simt(P, s);
+  cudaError_t e;
+  if (impl == PDN_IMPL_TC) e = launch_chunk_split(P, workspace, s);
+  else if (impl == PDN_IMPL_TC_FUSED) e = launch_chunk_tc(P, workspace, s);
+  else e = launch_chunk_simt(P, s);
   return e == cudaSuccess ? PDN_OK : PDN_ERR_CUDA;
 }
 

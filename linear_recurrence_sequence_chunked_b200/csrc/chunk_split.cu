@@ -1,0 +1,863 @@
+// chunk_split.cu -- chunked forward in three kernels: the intra-chunk work,
+// which does not depend on the state, runs for every chunk at once; only the
+// state pass stays sequential per (batch, head).
+//
+//   K0  key-energy prefix: A at the start of every chunk (preconditioned
+//       variants; "Preconditioned DeltaNet", fr §2.B: A_t = A_{t-1} + k.k)
+//   K1  one CTA per (batch, head, chunk): gates and preconditioner, M and P
+//       (MMA), T = (I + M)^{-1}, Y^T = Rh^T T^T (MMA); writes bf16 operand
+//       tiles of the chunk to the workspace in the shared-memory image the
+//       state kernel's MMAs consume
+//   K2  one CTA per (batch, head): per chunk, bulk-loads those tiles one chunk
+//       ahead, U^T = U^T T^T, D^T = U^T - S Y^T, O^T = S Qh^T + D^T P^T,
+//       S <- S Diag(e^{G_C}) + D^T Wb; fp32 state in tensor memory
+//
+// Same chunk algebra as the single-kernel path ("Gated DeltaNet-2", ja §3:
+// decay absorbed into the erase/write matrices, (I+T)^{-1} solve for the
+// auxiliaries Y and U); the split trades extra HBM traffic (about 80 KiB of
+// operand tiles per chunk and head, written once and read once) for running
+// the intra-chunk work with thousands of CTAs instead of one per chain.
+#include "common.cuh"
+#include "internal.h"
+#include "ptx.cuh"
+#include "tiles.cuh"
+
+namespace pdn {
+namespace {
+
+constexpr int kC = 64;
+constexpr int kD = 128;
+
+// ---- workspace: one block per (batch, head, chunk) -------------------------
+constexpr uint32_t WS_Q = 0;        // TL 64 x 128: Qh (rows tokens)
+constexpr uint32_t WS_Y = 16384;    // TL 128 x 64: Y^T (rows d_k, columns tokens)
+constexpr uint32_t WS_U = 32768;    // TL 64 x 128: u (rows tokens)
+constexpr uint32_t WS_WB = 49152;   // TL 64 x 128: Wb (rows tokens)
+constexpr uint32_t WS_T = 65536;    // TL 64 x 64: T = (I + M)^{-1}
+constexpr uint32_t WS_P = 73728;    // TL 64 x 64: P
+constexpr uint32_t WS_E = 81920;    // float[128]: e^{G_C}
+constexpr uint32_t WS_SET = 82432;  // bytes the state kernel loads per chunk
+constexpr uint32_t WS_A = 82432;    // float[128]: accumulator A at the chunk start
+constexpr size_t WS_CH = 82944;     // bytes per block (256-aligned)
+
+__device__ __forceinline__ uint8_t *ws_block(void *ws, int bh, int N, int c) {
+  return reinterpret_cast<uint8_t *>(ws) + ((size_t)bh * N + c) * WS_CH;
+}
+
+constexpr long long kSpin = 1LL << 22;
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+constexpr float kMinG = -80.f;
+
+// ===========================================================================
+// K0: per-chunk key energy, then the exclusive prefix over chunks
+// ===========================================================================
+__global__ void __launch_bounds__(kD) k0_chunk_energy(const KParams P, void *ws, int N) {
+  const int bh = blockIdx.y, i = threadIdx.x;
+  const int b = bh / P.H, h = bh % P.H;
+  const __nv_bfloat16 *k = reinterpret_cast<const __nv_bfloat16 *>(P.k);
+  const size_t tstride = (size_t)P.H * kD;
+  for (int cc = 0; cc < 8; ++cc) {
+    const int c = blockIdx.x * 8 + cc;
+    if (c >= N) break;
+    const int c0 = c * kC, Cn = min(kC, P.T - c0);
+    const __nv_bfloat16 *kp = k + tok_index(P, b, c0, h) * kD + i;
+    float s = 0.f;
+#pragma unroll 8
+    for (int t = 0; t < Cn; ++t) {
+      const float kv = __bfloat162float(kp[t * tstride]);
+      s = fmaf(kv, kv, s);
+    }
+    reinterpret_cast<float *>(ws_block(ws, bh, N, c) + WS_A)[i] = s;
+  }
+}
+
+__global__ void __launch_bounds__(kD) k0_prefix(const KParams P, void *ws, int N) {
+  const int bh = blockIdx.x, i = threadIdx.x;
+  float a = P.A0 ? P.A0[(size_t)bh * kD + i] : 0.f;
+  for (int c0 = 0; c0 < N; c0 += 8) {
+    float s[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e)
+      s[e] = (c0 + e < N) ? reinterpret_cast<float *>(ws_block(ws, bh, N, c0 + e) + WS_A)[i] : 0.f;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      if (c0 + e < N) reinterpret_cast<float *>(ws_block(ws, bh, N, c0 + e) + WS_A)[i] = a;
+      a += s[e];
+    }
+  }
+  if (P.AT) P.AT[(size_t)bh * kD + i] = a;
+}
+
+// ===========================================================================
+// K1: intra-chunk work, one CTA per (batch, head, chunk)
+// ===========================================================================
+constexpr int kK1Threads = 256;
+constexpr int LB_LD = 132;                        // floats per row of the prep buffers
+constexpr int MS_LD = 68, TS_LD = 68, YS_LD = 34; // fp32 solve scratch strides
+constexpr uint32_t K1_RQ = 0;                     // TL 128 x 128: Rh rows 0-63, Qh rows 64-127
+constexpr uint32_t K1_WH = 32768;                 // TL 64 x 128
+constexpr uint32_t K1_RA = 49152;                 // region A
+constexpr uint32_t K1_LBUF = K1_RA;               // prep: log2(A + eps)
+constexpr uint32_t K1_GBUF_PRE = K1_RA + 64 * LB_LD * 4;  // prep: cumulative log decay
+constexpr uint32_t K1_TM = K1_RA;                 // TL 64 x 64
+constexpr uint32_t K1_PM = K1_RA + 8192;          // TL 64 x 64
+constexpr uint32_t K1_MS = K1_RA + 16384;         // fp32 [64][68]
+constexpr uint32_t K1_TS = K1_MS + 64 * MS_LD * 4;// fp32 [64][68]
+constexpr uint32_t K1_YS = K1_TS + 64 * TS_LD * 4;// fp32 [32][34]
+constexpr uint32_t K1_YT = K1_RA + 16384;         // TL 128 x 64 (after the solve)
+constexpr uint32_t K1_SOLVE_END = K1_YS + 32 * YS_LD * 4;
+
+// Region A holds the prep buffers the variant needs, then the solve scratch.
+template <int kVariant, int kDecay>
+struct K1Layout {
+  static constexpr bool kPre =
+      kVariant == PDN_VAR_PDN || kVariant == PDN_VAR_PGDN || kVariant == PDN_VAR_PKDA;
+  static constexpr uint32_t kGbuf = kPre ? K1_GBUF_PRE : K1_RA;
+  static constexpr uint32_t kPrepEnd =
+      K1_RA + (kPre ? 64 * LB_LD * 4 : 0) + (kDecay == PDN_DECAY_CHANNEL ? 64 * LB_LD * 4 : 0);
+  static constexpr uint32_t kSmall = (kPrepEnd > K1_SOLVE_END ? kPrepEnd : K1_SOLVE_END);
+  static constexpr uint32_t kAcar = kSmall, kGC = kSmall + 512, kEGC = kSmall + 1024;
+  static constexpr uint32_t kPartK = kSmall + 1536, kPartG = kSmall + 2048;
+  static constexpr uint32_t kMu = kSmall + 2560, kBeta = kSmall + 2816, kGS = kSmall + 3072;
+  static constexpr uint32_t kLas = kSmall + 3328, kBar = kSmall + 3584;
+  static constexpr uint32_t kTbase = kSmall + 3600;
+  static constexpr uint32_t kBytes = kSmall + 3616;
+};
+
+__device__ __forceinline__ void sync_for_mma() {
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+}
+
+template <int kVariant, int kDecay>
+__global__ void __launch_bounds__(kK1Threads) k1_intra(const KParams P, void *ws, int N) {
+  using L = K1Layout<kVariant, kDecay>;
+  constexpr bool kPre = L::kPre;
+  constexpr bool kScalarBeta = kVariant != PDN_VAR_FG2_GDN && kVariant != PDN_VAR_GDN2;
+  extern __shared__ __align__(1024) uint8_t smem[];
+  const uint32_t sb = smem_u32(smem);
+  float *Acar = reinterpret_cast<float *>(smem + L::kAcar);
+  float *GC = reinterpret_cast<float *>(smem + L::kGC);
+  float *EGC = reinterpret_cast<float *>(smem + L::kEGC);
+  float *PARTK = reinterpret_cast<float *>(smem + L::kPartK);
+  float *PARTG = reinterpret_cast<float *>(smem + L::kPartG);
+  float *MU = reinterpret_cast<float *>(smem + L::kMu);
+  float *BETA = reinterpret_cast<float *>(smem + L::kBeta);
+  float *GS = reinterpret_cast<float *>(smem + L::kGS);
+  float *LAS = reinterpret_cast<float *>(smem + L::kLas);
+  uint64_t *bar = reinterpret_cast<uint64_t *>(smem + L::kBar);
+  uint32_t *tbase_p = reinterpret_cast<uint32_t *>(smem + L::kTbase);
+  float *LBUF = reinterpret_cast<float *>(smem + K1_LBUF);
+  float *GBUF = reinterpret_cast<float *>(smem + L::kGbuf);
+  float *MS = reinterpret_cast<float *>(smem + K1_MS);
+  float *TS = reinterpret_cast<float *>(smem + K1_TS);
+  float *YS = reinterpret_cast<float *>(smem + K1_YS);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int c = blockIdx.x, bh = blockIdx.y;
+  const int b = bh / P.H, h = bh % P.H;
+  const int c0 = c * kC, Cn = min(kC, P.T - c0);
+  const size_t tstride = (size_t)P.H * kD;
+  const size_t tok0 = tok_index(P, b, c0, h) * kD;  // element offset of token c0
+  uint8_t *blk = ws_block(ws, bh, N, c);
+  const float log2x = P.lnx * kLog2e;
+  const uint32_t lane_q = (uint32_t)(32 * (warp & 3)) << 16;
+  const int half = warp >> 2;
+
+  if (warp == 0) {
+    tmem_alloc(tbase_p, 128);
+    tmem_relinquish();
+  }
+  if (tid == 0) {
+    mbar_init(bar + 0, 1);
+    mbar_init(bar + 1, 1);
+    fence_mbarrier_init();
+  }
+  // ---- P0: per-token scalars, accumulator at the chunk start ----
+  if (tid < kC) {
+    const bool ok = tid < Cn;
+    const size_t e = ok ? tok_index(P, b, c0 + tid, h) : 0;
+    BETA[tid] = (kScalarBeta && ok) ? __ldg(reinterpret_cast<const float *>(P.beta) + e) : 0.f;
+    LAS[tid] = (kDecay == PDN_DECAY_SCALAR && ok)
+                   ? __ldg(reinterpret_cast<const float *>(P.log_alpha) + e) : 0.f;
+  }
+  if (tid < kD) Acar[tid] = kPre ? reinterpret_cast<const float *>(blk + WS_A)[tid] : 0.f;
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tm = *tbase_p;
+
+  // ---- P1: per-channel scans; thread = (channel, half of the chunk) ----
+  {
+    const int i = tid & 127, hf = tid >> 7, t0 = 32 * hf;
+    const __nv_bfloat16 *kp = reinterpret_cast<const __nv_bfloat16 *>(P.k) + tok0 + i;
+    const __nv_bfloat16 *lp = reinterpret_cast<const __nv_bfloat16 *>(P.log_alpha) + tok0 + i;
+    float kk[32], la[32];
+    float ks = 0.f, gs = 0.f;
+#pragma unroll
+    for (int e = 0; e < 32; ++e) {
+      const int t = t0 + e;
+      kk[e] = 0.f;
+      la[e] = 0.f;
+      if (kPre && t < Cn) kk[e] = __bfloat162float(kp[t * tstride]);
+      if (kDecay == PDN_DECAY_CHANNEL) la[e] = t < Cn ? __bfloat162float(lp[t * tstride]) : 0.f;
+      else if (kDecay == PDN_DECAY_SCALAR) la[e] = LAS[t];
+    }
+#pragma unroll
+    for (int e = 0; e < 32; ++e) {
+      ks = fmaf(kk[e], kk[e], ks);
+      gs += la[e];
+    }
+    if (hf == 0) {
+      PARTK[i] = ks;
+      PARTG[i] = gs;
+    }
+    __syncthreads();
+    float a = Acar[i] + (hf ? PARTK[i] : 0.f);
+    float g = hf ? PARTG[i] : 0.f;
+#pragma unroll
+    for (int e = 0; e < 32; ++e) {
+      const int t = t0 + e;
+      if (kPre) {
+        a = fmaf(kk[e], kk[e], a);
+        LBUF[t * LB_LD + i] = lg2_approx(a + P.eps);
+      }
+      g += la[e];
+      if (kDecay == PDN_DECAY_CHANNEL) GBUF[t * LB_LD + i] = g;
+      else if (kDecay == PDN_DECAY_SCALAR && i == 0) GS[t] = g;
+    }
+    if (hf) {
+      GC[i] = g;
+      const float e = ex2_approx(fmaxf(g, kMinG) * kLog2e);
+      EGC[i] = e;
+      reinterpret_cast<float *>(blk + WS_E)[i] = e;
+    }
+  }
+  __syncthreads();
+
+  // ---- P2: per-token channel mean of log2(A + eps) ----
+  if (kPre) {
+    const int t = tid >> 2, qd = tid & 3;
+    float s = 0.f;
+#pragma unroll
+    for (int k4 = 0; k4 < 8; ++k4) {
+      const float4 x = *reinterpret_cast<const float4 *>(LBUF + t * LB_LD + qd * 32 + 4 * k4);
+      s += (x.x + x.y) + (x.z + x.w);
+    }
+    s += __shfl_xor_sync(0xffffffffu, s, 1);
+    s += __shfl_xor_sync(0xffffffffu, s, 2);
+    if (qd == 0) MU[t] = s * (1.f / kD);
+    __syncthreads();
+  }
+
+  // ---- P3: operand tiles, (token, 8-channel) units ----
+  {
+    const int t = 8 * warp + (lane & 7);
+    const bool ok = t < Cn;
+    const size_t etok = tok0 + (size_t)t * tstride;
+    float eg_s = 1.f, emg_s = 1.f, ewb_s = 1.f;
+    if (kDecay == PDN_DECAY_SCALAR) {
+      eg_s = ex2_approx(fmaxf(GS[t], kMinG) * kLog2e);
+      emg_s = rcp_approx(eg_s);
+      ewb_s = EGC[0] * emg_s;
+    }
+    const float be = kScalarBeta ? BETA[t] : 0.f;
+    const float mu = kPre ? MU[t] : 0.f;
+    const float qs = P.q_scale;
+    const __nv_bfloat16 *kb = reinterpret_cast<const __nv_bfloat16 *>(P.k);
+    const __nv_bfloat16 *qb = reinterpret_cast<const __nv_bfloat16 *>(P.q);
+    const __nv_bfloat16 *vb = reinterpret_cast<const __nv_bfloat16 *>(P.v);
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+      const int c8 = 4 * m + (lane >> 3);
+      const int i0 = 8 * c8;
+      float kf[8], qf[8], vf[8], r[8], w[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) { kf[e] = 0.f; qf[e] = 0.f; vf[e] = 0.f; }
+      if (ok) {
+        unpack8(__ldg(reinterpret_cast<const uint4 *>(kb + etok + i0)), kf);
+        unpack8(__ldg(reinterpret_cast<const uint4 *>(qb + etok + i0)), qf);
+        unpack8(__ldg(reinterpret_cast<const uint4 *>(vb + etok + i0)), vf);
+      }
+      if (kPre) {
+        float Lv[8];
+        ld8f(LBUF + t * LB_LD + i0, Lv);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const float cc = (Lv[e] - mu) * kLn2;
+          const float s = cc * rcp_approx(1.f + fabsf(cc));
+          r[e] = kf[e];
+          w[e] = be * ex2_approx(-s * log2x) * kf[e];
+        }
+      } else if (kVariant == PDN_VAR_FG2_GDN) {
+        float gb[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) gb[e] = 0.f;
+        if (ok)
+          unpack8(__ldg(reinterpret_cast<const uint4 *>(
+                      reinterpret_cast<const __nv_bfloat16 *>(P.beta) + etok + i0)), gb);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const float sq = sqrtf(gb[e]);
+          r[e] = sq * kf[e];
+          w[e] = r[e];
+          vf[e] *= sq;
+        }
+      } else if (kVariant == PDN_VAR_GDN2) {
+        float ge[8], gw[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) { ge[e] = 0.f; gw[e] = 0.f; }
+        if (ok) {
+          unpack8(__ldg(reinterpret_cast<const uint4 *>(
+                      reinterpret_cast<const __nv_bfloat16 *>(P.erase) + etok + i0)), ge);
+          unpack8(__ldg(reinterpret_cast<const uint4 *>(
+                      reinterpret_cast<const __nv_bfloat16 *>(P.write) + etok + i0)), gw);
+        }
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          r[e] = ge[e] * kf[e];
+          w[e] = kf[e];
+          vf[e] *= gw[e];
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          r[e] = kf[e];
+          w[e] = be * kf[e];
+        }
+      }
+      float rh[8], qh[8], wh[8], wb[8];
+      if (kDecay == PDN_DECAY_CHANNEL) {
+        float G[8], E[8];
+        ld8f(GBUF + t * LB_LD + i0, G);
+        ld8f(EGC + i0, E);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const float eg = ex2_approx(fmaxf(G[e], kMinG) * kLog2e);
+          const float emg = rcp_approx(eg);
+          rh[e] = r[e] * eg;
+          qh[e] = qs * qf[e] * eg;
+          wh[e] = w[e] * emg;
+          wb[e] = w[e] * (E[e] * emg);
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          rh[e] = r[e] * eg_s;
+          qh[e] = (qs * eg_s) * qf[e];
+          wh[e] = w[e] * emg_s;
+          wb[e] = w[e] * ewb_s;
+        }
+      }
+      *reinterpret_cast<uint4 *>(smem + K1_RQ + tl128(t, c8)) = pack8(rh);
+      *reinterpret_cast<uint4 *>(smem + K1_RQ + tl128(64 + t, c8)) = pack8(qh);
+      *reinterpret_cast<uint4 *>(smem + K1_WH + tl128(t, c8)) = pack8(wh);
+      *reinterpret_cast<uint4 *>(blk + WS_WB + tl128(t, c8)) = pack8(wb);
+      *reinterpret_cast<uint4 *>(blk + WS_U + tl128(t, c8)) = pack8(vf);
+    }
+  }
+
+  // ---- MMA1: D1 = [Rh;Qh] Wh^T ----
+  sync_for_mma();
+  if (tid == 0) {
+    const uint32_t id = make_idesc_bf16(128, 64, false, false);
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk)
+      mma_bf16_ss(tm + 0, make_sdesc(sb + K1_RQ + 256 * kk, 128, 2048),
+                  make_sdesc(sb + K1_WH + 256 * kk, 128, 2048), id, kk > 0);
+    mma_commit(bar + 0);
+  }
+  bool ok_all = true;
+  {
+    bool ok = true;
+    if (warp == 0) ok = mbar_wait_bounded(bar + 0, 0, kSpin);
+    ok_all = !__syncthreads_or(!ok);
+    tc_fence_after();
+  }
+
+  if (ok_all) {
+    // ---- solve: M, P from TMEM; T = (I + M)^{-1} ----
+    {
+      const int row = 32 * (warp & 3) + lane;
+#pragma unroll
+      for (int cc = 0; cc < 2; ++cc) {
+        float v[16];
+        tmem_ld16(tm + lane_q + 32 * half + 16 * cc, v);
+        tmem_wait_ld();
+        const int s0 = 32 * half + 16 * cc;
+        if (row < kC) {
+#pragma unroll
+          for (int e4 = 0; e4 < 4; ++e4) {
+            float4 x;
+            x.x = (s0 + 4 * e4 + 0 < row) ? v[4 * e4 + 0] : 0.f;
+            x.y = (s0 + 4 * e4 + 1 < row) ? v[4 * e4 + 1] : 0.f;
+            x.z = (s0 + 4 * e4 + 2 < row) ? v[4 * e4 + 2] : 0.f;
+            x.w = (s0 + 4 * e4 + 3 < row) ? v[4 * e4 + 3] : 0.f;
+            *reinterpret_cast<float4 *>(MS + row * MS_LD + s0 + 4 * e4) = x;
+          }
+        } else {
+          const int t = row - kC;
+          float lo[8], hi[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            lo[e] = (s0 + e <= t) ? v[e] : 0.f;
+            hi[e] = (s0 + 8 + e <= t) ? v[8 + e] : 0.f;
+          }
+          *reinterpret_cast<uint4 *>(smem + K1_PM + tl64(t, s0 / 8)) = pack8(lo);
+          *reinterpret_cast<uint4 *>(smem + K1_PM + tl64(t, s0 / 8 + 1)) = pack8(hi);
+        }
+      }
+    }
+    tc_fence_before();
+    __syncthreads();
+    // L0: 16x16 diagonal blocks; the other threads zero the upper blocks the merges read
+    if (tid < 64) {
+      const int base = 16 * (tid >> 4), cc = tid & 15;
+      float x[16];
+#pragma unroll
+      for (int r = 0; r < 16; ++r) {
+        float acc0 = (r == cc) ? 1.f : 0.f, acc1 = 0.f;
+#pragma unroll
+        for (int s = 0; s < r; s += 2) {
+          acc0 = fmaf(-MS[(base + r) * MS_LD + base + s], x[s], acc0);
+          if (s + 1 < r) acc1 = fmaf(-MS[(base + r) * MS_LD + base + s + 1], x[s + 1], acc1);
+        }
+        x[r] = acc0 + acc1;
+      }
+#pragma unroll
+      for (int r = 0; r < 16; ++r) TS[(base + r) * TS_LD + base + cc] = x[r];
+    } else {
+      for (int e = tid - 64; e < 512; e += kK1Threads - 64) {
+        const int blk2 = e >> 8, r = (e >> 4) & 15, cc = e & 15;
+        TS[(32 * blk2 + r) * TS_LD + 32 * blk2 + 16 + cc] = 0.f;
+      }
+    }
+    __syncthreads();
+    // L1: merge 16 -> 32 within [32p, 32p + 32): X = -T_D (M_CA T_A)
+    if (tid < 128) {
+      const int p = tid >> 6, rb = (tid >> 3) & 7, cb = tid & 7;
+      const int o = 32 * p, r0 = 2 * rb, c0b = 2 * cb;
+      float a00 = 0.f, a01 = 0.f, a10 = 0.f, a11 = 0.f;
+#pragma unroll
+      for (int s4 = 0; s4 < 16; s4 += 4) {
+        const float4 m0 = *reinterpret_cast<const float4 *>(MS + (o + 16 + r0) * MS_LD + o + s4);
+        const float4 m1 = *reinterpret_cast<const float4 *>(MS + (o + 16 + r0 + 1) * MS_LD + o + s4);
+        const float mv0[4] = {m0.x, m0.y, m0.z, m0.w}, mv1[4] = {m1.x, m1.y, m1.z, m1.w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const float2 tv = *reinterpret_cast<const float2 *>(TS + (o + s4 + k) * TS_LD + o + c0b);
+          a00 = fmaf(mv0[k], tv.x, a00); a01 = fmaf(mv0[k], tv.y, a01);
+          a10 = fmaf(mv1[k], tv.x, a10); a11 = fmaf(mv1[k], tv.y, a11);
+        }
+      }
+      float *y = YS + p * 16 * YS_LD;
+      *reinterpret_cast<float2 *>(y + r0 * YS_LD + c0b) = make_float2(a00, a01);
+      *reinterpret_cast<float2 *>(y + (r0 + 1) * YS_LD + c0b) = make_float2(a10, a11);
+    }
+    __syncthreads();
+    if (tid < 128) {
+      const int p = tid >> 6, rb = (tid >> 3) & 7, cb = tid & 7;
+      const int o = 32 * p, r0 = 2 * rb, c0b = 2 * cb;
+      const float *y = YS + p * 16 * YS_LD;
+      float a00 = 0.f, a01 = 0.f, a10 = 0.f, a11 = 0.f;
+#pragma unroll
+      for (int s4 = 0; s4 < 16; s4 += 4) {
+        const float4 t0 = *reinterpret_cast<const float4 *>(TS + (o + 16 + r0) * TS_LD + o + 16 + s4);
+        const float4 t1 = *reinterpret_cast<const float4 *>(TS + (o + 16 + r0 + 1) * TS_LD + o + 16 + s4);
+        const float tv0[4] = {t0.x, t0.y, t0.z, t0.w}, tv1[4] = {t1.x, t1.y, t1.z, t1.w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const float2 yv = *reinterpret_cast<const float2 *>(y + (s4 + k) * YS_LD + c0b);
+          a00 = fmaf(tv0[k], yv.x, a00); a01 = fmaf(tv0[k], yv.y, a01);
+          a10 = fmaf(tv1[k], yv.x, a10); a11 = fmaf(tv1[k], yv.y, a11);
+        }
+      }
+      *reinterpret_cast<float2 *>(TS + (o + 16 + r0) * TS_LD + o + c0b) = make_float2(-a00, -a01);
+      *reinterpret_cast<float2 *>(TS + (o + 16 + r0 + 1) * TS_LD + o + c0b) = make_float2(-a10, -a11);
+    }
+    __syncthreads();
+    // L2: merge 32 -> 64: X = -T_D (M[32:64, 0:32] T_A)
+    {
+      const int r0 = 2 * (tid >> 4), c0b = 2 * (tid & 15);
+      float a00 = 0.f, a01 = 0.f, a10 = 0.f, a11 = 0.f;
+#pragma unroll 4
+      for (int s4 = 0; s4 < 32; s4 += 4) {
+        const float4 m0 = *reinterpret_cast<const float4 *>(MS + (32 + r0) * MS_LD + s4);
+        const float4 m1 = *reinterpret_cast<const float4 *>(MS + (32 + r0 + 1) * MS_LD + s4);
+        const float mv0[4] = {m0.x, m0.y, m0.z, m0.w}, mv1[4] = {m1.x, m1.y, m1.z, m1.w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const float2 tv = *reinterpret_cast<const float2 *>(TS + (s4 + k) * TS_LD + c0b);
+          a00 = fmaf(mv0[k], tv.x, a00); a01 = fmaf(mv0[k], tv.y, a01);
+          a10 = fmaf(mv1[k], tv.x, a10); a11 = fmaf(mv1[k], tv.y, a11);
+        }
+      }
+      *reinterpret_cast<float2 *>(YS + r0 * YS_LD + c0b) = make_float2(a00, a01);
+      *reinterpret_cast<float2 *>(YS + (r0 + 1) * YS_LD + c0b) = make_float2(a10, a11);
+    }
+    __syncthreads();
+    {
+      const int r0 = 2 * (tid >> 4), c0b = 2 * (tid & 15);
+      float a00 = 0.f, a01 = 0.f, a10 = 0.f, a11 = 0.f;
+#pragma unroll 4
+      for (int s4 = 0; s4 < 32; s4 += 4) {
+        const float4 t0 = *reinterpret_cast<const float4 *>(TS + (32 + r0) * TS_LD + 32 + s4);
+        const float4 t1 = *reinterpret_cast<const float4 *>(TS + (32 + r0 + 1) * TS_LD + 32 + s4);
+        const float tv0[4] = {t0.x, t0.y, t0.z, t0.w}, tv1[4] = {t1.x, t1.y, t1.z, t1.w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const float2 yv = *reinterpret_cast<const float2 *>(YS + (s4 + k) * YS_LD + c0b);
+          a00 = fmaf(tv0[k], yv.x, a00); a01 = fmaf(tv0[k], yv.y, a01);
+          a10 = fmaf(tv1[k], yv.x, a10); a11 = fmaf(tv1[k], yv.y, a11);
+        }
+      }
+      *reinterpret_cast<float2 *>(TS + (32 + r0) * TS_LD + c0b) = make_float2(-a00, -a01);
+      *reinterpret_cast<float2 *>(TS + (32 + r0 + 1) * TS_LD + c0b) = make_float2(-a10, -a11);
+    }
+    __syncthreads();
+#pragma unroll
+    for (int m = 0; m < 2; ++m) {
+      const int t = 8 * warp + (lane & 7), s8 = 4 * m + (lane >> 3);
+      float v[8];
+      ld8f(TS + t * TS_LD + 8 * s8, v);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) v[e] = (8 * s8 + e <= t) ? v[e] : 0.f;
+      *reinterpret_cast<uint4 *>(smem + K1_TM + tl64(t, s8)) = pack8(v);
+    }
+
+    // ---- MMA2: Y^T = Rh^T T^T ----
+    sync_for_mma();
+    if (tid == 0) {
+      const uint32_t id = make_idesc_bf16(128, 64, true, false);
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk)
+        mma_bf16_ss(tm + 64, make_sdesc(sb + K1_RQ + 4096 * kk, 2048, 128),
+                    make_sdesc(sb + K1_TM + 256 * kk, 128, 1024), id, kk > 0);
+      mma_commit(bar + 1);
+    }
+    {
+      bool ok = true;
+      if (warp == 0) ok = mbar_wait_bounded(bar + 1, 0, kSpin);
+      ok_all = !__syncthreads_or(!ok);
+      tc_fence_after();
+    }
+    if (ok_all) {
+      // Y^T -> bf16 tile (rows d_k, columns tokens)
+      const int i = 32 * (warp & 3) + lane;
+#pragma unroll
+      for (int cc = 0; cc < 2; ++cc) {
+        float v[16];
+        tmem_ld16(tm + lane_q + 64 + 32 * half + 16 * cc, v);
+        tmem_wait_ld();
+        float lo[8], hi[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) { lo[e] = v[e]; hi[e] = v[8 + e]; }
+        const int t8 = 4 * half + 2 * cc;
+        *reinterpret_cast<uint4 *>(smem + K1_YT + tl64(i, t8)) = pack8(lo);
+        *reinterpret_cast<uint4 *>(smem + K1_YT + tl64(i, t8 + 1)) = pack8(hi);
+      }
+      // ---- the tiles that live in shared memory go out with bulk stores ----
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncthreads();
+      if (tid == 0) {
+        bulk_s2g(blk + WS_Q, smem + K1_RQ + 16384, 16384);
+        bulk_s2g(blk + WS_Y, smem + K1_YT, 16384);
+        bulk_s2g(blk + WS_T, smem + K1_TM, 8192);
+        bulk_s2g(blk + WS_P, smem + K1_PM, 8192);
+        bulk_commit();
+        bulk_wait0();
+      }
+    }
+  }
+  if (!ok_all && tid == 0) record_error(P.err, PDN_ERR_TIMEOUT);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 0) tmem_dealloc(tm, 128);
+}
+
+// ===========================================================================
+// K2: state pass, one CTA per (batch, head)
+// ===========================================================================
+constexpr int kK2Threads = 512;  // 16 warps: TMEM lane quarter x column group
+constexpr uint32_t K2_SET0 = 0;
+constexpr uint32_t K2_SET1 = WS_SET;
+constexpr uint32_t K2_SB = 2 * WS_SET;             // TL 128 x 128 bf16 copy of S
+constexpr uint32_t K2_DT = K2_SB + 32768;          // TL 128 x 64: D^T
+constexpr uint32_t K2_BAR = K2_DT + 16384;         // full[2], m5, m6, m7
+constexpr uint32_t K2_TBASE = K2_BAR + 5 * 8;
+constexpr uint32_t K2_BYTES = K2_TBASE + 16;
+static_assert(K2_BYTES <= 232448, "state kernel shared memory budget");
+
+constexpr uint32_t TM_UD = 0, TM_OT0 = 64, TM_OT1 = 128, TM_S = 256;
+
+__device__ __forceinline__ void issue_set_load(uint8_t *dst, const uint8_t *src, uint64_t *bar) {
+  mbar_arrive_expect_tx(bar, WS_SET);
+#pragma unroll
+  for (int p = 0; p < 5; ++p) bulk_g2s(dst + p * 16384, src + p * 16384, 16384, bar);
+  bulk_g2s(dst + 81920, src + 81920, WS_SET - 81920, bar);
+}
+
+// 16 output tokens [16 cg, 16 cg + 16) of O^T (TMEM lanes = value channels)
+// for one warp (its lane quarter), two adjacent channels per 32-bit store.
+__device__ __forceinline__ void k2_store_o(const KParams &P, uint32_t taddr, int b, int h,
+                                           int pc0, int Cn, int lane, int quarter, int cg) {
+  const size_t tstride = (size_t)P.H * kD;
+  const int j = 32 * quarter + lane;
+  __nv_bfloat16 *orow =
+      reinterpret_cast<__nv_bfloat16 *>(P.o) + tok_index(P, b, pc0, h) * kD + (j & ~1);
+  const bool odd = lane & 1;
+  float v[16];
+  tmem_ld16(taddr + 16 * cg, v);
+  tmem_wait_ld();
+#pragma unroll
+  for (int e2 = 0; e2 < 8; ++e2) {
+    const float send = odd ? v[2 * e2] : v[2 * e2 + 1];
+    const float recv = __shfl_xor_sync(0xffffffffu, send, 1);
+    const int t = 16 * cg + 2 * e2 + (odd ? 1 : 0);
+    const float lo = odd ? recv : v[2 * e2];
+    const float hi = odd ? v[2 * e2 + 1] : recv;
+    if (t < Cn) *reinterpret_cast<uint32_t *>(orow + t * tstride) = pack_bf16(lo, hi);
+  }
+}
+
+__global__ void __launch_bounds__(kK2Threads, 1) k2_state(const KParams P, void *ws, int N) {
+  extern __shared__ __align__(1024) uint8_t smem[];
+  const uint32_t sb = smem_u32(smem);
+  uint64_t *full = reinterpret_cast<uint64_t *>(smem + K2_BAR);
+  uint64_t *bar5 = full + 2, *bar6 = full + 3, *bar7 = full + 4;
+  uint32_t *tbase_p = reinterpret_cast<uint32_t *>(smem + K2_TBASE);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int quarter = warp & 3, cg = warp >> 2;  // TMEM lanes 32*quarter.., column group 0..3
+  const uint32_t lane_q = (uint32_t)(32 * quarter) << 16;
+  const int bh = blockIdx.x, b = bh / P.H, h = bh % P.H;
+  const int j = 32 * quarter + lane;  // value channel owned in the epilogues
+
+  if (warp == 0) {
+    tmem_alloc(tbase_p, 512);
+    tmem_relinquish();
+  }
+  if (tid == 0) {
+    for (int i = 0; i < 5; ++i) mbar_init(full + i, 1);
+    fence_mbarrier_init();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tm = *tbase_p;
+  if (tid == 0 && N > 0) issue_set_load(smem + K2_SET0, ws_block(ws, bh, N, 0), full + 0);
+
+  auto wait_all = [&](uint64_t *bb, uint32_t parity) -> bool {
+    bool ok = true;
+    if (warp == 0) ok = mbar_wait_bounded(bb, parity, kSpin);
+    const bool fail = __syncthreads_or(!ok);
+    tc_fence_after();
+    return !fail;
+  };
+
+  bool aborted = false;
+  for (int n = 0; n < N; ++n) {
+    const int s = n & 1;
+    const uint32_t set = s ? K2_SET1 : K2_SET0;
+    const uint32_t ot = s ? TM_OT1 : TM_OT0;
+    // the other set was last read by the previous chunk's MMAs (complete): refill it
+    if (tid == 0 && n + 1 < N)
+      issue_set_load(smem + (s ? K2_SET0 : K2_SET1), ws_block(ws, bh, N, n + 1), full + (s ^ 1));
+    if (!wait_all(full + s, (uint32_t)((n >> 1) & 1))) { aborted = true; break; }
+
+    // ---- state epilogue: S -> bf16 operand; TMEM S <- S Diag(e^{G_C}) ----
+    {
+      const float *egc = reinterpret_cast<const float *>(smem + set + WS_E);
+      float sv[2][16];
+      const int col0 = 32 * cg;
+      if (n == 0) {
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          if (P.S0) {
+            const float4 *src =
+                reinterpret_cast<const float4 *>(P.S0 + ((size_t)bh * kD + j) * kD + col0 + 16 * u);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float4 x = __ldg(src + e);
+              sv[u][4 * e] = x.x; sv[u][4 * e + 1] = x.y; sv[u][4 * e + 2] = x.z; sv[u][4 * e + 3] = x.w;
+            }
+          } else {
+#pragma unroll
+            for (int e = 0; e < 16; ++e) sv[u][e] = 0.f;
+          }
+        }
+      } else {
+        tmem_ld16(tm + lane_q + TM_S + col0, sv[0]);
+        tmem_ld16(tm + lane_q + TM_S + col0 + 16, sv[1]);
+        tmem_wait_ld();
+      }
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const int col = col0 + 16 * u;
+        float lo[8], hi[8], E[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) { lo[e] = sv[u][e]; hi[e] = sv[u][8 + e]; }
+        *reinterpret_cast<uint4 *>(smem + K2_SB + tl128(j, col / 8)) = pack8(lo);
+        *reinterpret_cast<uint4 *>(smem + K2_SB + tl128(j, col / 8 + 1)) = pack8(hi);
+        ld8f(egc + col, E);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) sv[u][e] *= E[e];
+        ld8f(egc + col + 8, E);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) sv[u][8 + e] *= E[e];
+        tmem_st16(tm + lane_q + TM_S + col, sv[u]);
+      }
+      tmem_wait_st();
+    }
+    sync_for_mma();
+
+    // ---- MMA3: U^T = U^T T^T ; MMA5: D^T = U^T - S Y^T ; MMA6: O^T = S Qh^T ----
+    if (tid == 0) {
+      const uint32_t id3 = make_idesc_bf16(128, 64, true, false);
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk)
+        mma_bf16_ss(tm + TM_UD, make_sdesc(sb + set + WS_U + 4096 * kk, 2048, 128),
+                    make_sdesc(sb + set + WS_T + 256 * kk, 128, 1024), id3, kk > 0);
+      const uint32_t id5 = make_idesc_bf16(128, 64, false, true, true);
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk)
+        mma_bf16_ss(tm + TM_UD, make_sdesc(sb + K2_SB + 256 * kk, 128, 2048),
+                    make_sdesc(sb + set + WS_Y + 2048 * kk, 1024, 128), id5, 1);
+      mma_commit(bar5);
+      const uint32_t id6 = make_idesc_bf16(128, 64, false, false);
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk)
+        mma_bf16_ss(tm + ot, make_sdesc(sb + K2_SB + 256 * kk, 128, 2048),
+                    make_sdesc(sb + set + WS_Q + 256 * kk, 128, 2048), id6, kk > 0);
+      mma_commit(bar6);
+    }
+    // the previous chunk's output leaves while the MMAs run
+    if (n > 0)
+      k2_store_o(P, tm + lane_q + (s ? TM_OT0 : TM_OT1), b, h, (n - 1) * kC, kC, lane, quarter, cg);
+    tc_fence_before();
+    if (!wait_all(bar5, (uint32_t)(n & 1))) { aborted = true; break; }
+
+    // ---- D^T -> bf16 operand (rows d_v, columns tokens) ----
+    {
+      float v[16];
+      tmem_ld16(tm + lane_q + TM_UD + 16 * cg, v);
+      tmem_wait_ld();
+      float lo[8], hi[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) { lo[e] = v[e]; hi[e] = v[8 + e]; }
+      *reinterpret_cast<uint4 *>(smem + K2_DT + tl64(j, 2 * cg)) = pack8(lo);
+      *reinterpret_cast<uint4 *>(smem + K2_DT + tl64(j, 2 * cg + 1)) = pack8(hi);
+    }
+    sync_for_mma();
+
+    // ---- MMA7: O^T += D^T P^T ; MMA8: S += D^T Wb ----
+    if (tid == 0) {
+      const uint32_t id7 = make_idesc_bf16(128, 64, false, false);
+      const uint32_t id8 = make_idesc_bf16(128, 128, false, true);
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk) {
+        const uint64_t ad = make_sdesc(sb + K2_DT + 256 * kk, 128, 1024);
+        mma_bf16_ss(tm + ot, ad, make_sdesc(sb + set + WS_P + 256 * kk, 128, 1024), id7, 1);
+        mma_bf16_ss(tm + TM_S, ad, make_sdesc(sb + set + WS_WB + 4096 * kk, 2048, 128), id8, 1);
+      }
+      mma_commit(bar7);
+    }
+    if (!wait_all(bar6, (uint32_t)(n & 1))) { aborted = true; break; }
+    if (!wait_all(bar7, (uint32_t)(n & 1))) { aborted = true; break; }
+  }
+
+  if (!aborted && N > 0) {
+    const int pc0 = (N - 1) * kC;
+    k2_store_o(P, tm + lane_q + (((N - 1) & 1) ? TM_OT1 : TM_OT0), b, h, pc0, P.T - pc0, lane,
+               quarter, cg);
+    if (P.ST) {
+      float v[2][16];
+      const int col0 = 32 * cg;
+      tmem_ld16(tm + lane_q + TM_S + col0, v[0]);
+      tmem_ld16(tm + lane_q + TM_S + col0 + 16, v[1]);
+      tmem_wait_ld();
+      float4 *dst = reinterpret_cast<float4 *>(P.ST + ((size_t)bh * kD + j) * kD + col0);
+#pragma unroll
+      for (int u = 0; u < 2; ++u)
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          dst[4 * u + e] = make_float4(v[u][4 * e], v[u][4 * e + 1], v[u][4 * e + 2], v[u][4 * e + 3]);
+    }
+  }
+  if (aborted) {
+    if (tid == 0) record_error(P.err, PDN_ERR_TIMEOUT);
+    // drain the operand loads still in flight before shared memory goes away
+    if (tid == 0)
+      for (int s = 0; s < 2; ++s) mbar_wait_bounded(full + s, 0, kSpin), mbar_wait_bounded(full + s, 1, kSpin);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 0) tmem_dealloc(tm, 512);
+}
+
+template <int V, int Dc>
+cudaError_t launch_k1(const KParams &P, void *ws, int N, cudaStream_t stream) {
+  using L = K1Layout<V, Dc>;
+  auto kern = k1_intra<V, Dc>;
+  cudaError_t e =
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L::kBytes);
+  if (e != cudaSuccess) return e;
+  kern<<<dim3((unsigned)N, (unsigned)(P.B * P.H)), kK1Threads, L::kBytes, stream>>>(P, ws, N);
+  return cudaGetLastError();
+}
+
+template <int V>
+cudaError_t launch_k1_decay(const KParams &P, void *ws, int N, cudaStream_t stream) {
+  switch (P.decay) {
+    case PDN_DECAY_NONE: return launch_k1<V, PDN_DECAY_NONE>(P, ws, N, stream);
+    case PDN_DECAY_SCALAR: return launch_k1<V, PDN_DECAY_SCALAR>(P, ws, N, stream);
+    default: return launch_k1<V, PDN_DECAY_CHANNEL>(P, ws, N, stream);
+  }
+}
+
+}  // namespace
+
+int split_supported(const KParams &P) {
+  const long long N = (P.T + kC - 1) / kC;
+  return P.dtype == PDN_BF16 && P.dk == kD && P.dv == kD && P.chunk == kC && P.T > 0 &&
+         (long long)P.B * P.H <= 65535 && N <= 65535;
+}
+
+size_t split_workspace_bytes(const KParams &P) {
+  const size_t N = (size_t)((P.T + kC - 1) / kC);
+  return (size_t)P.B * P.H * N * WS_CH;
+}
+
+cudaError_t launch_chunk_split(const KParams &P, void *ws, cudaStream_t stream) {
+  const int N = (P.T + kC - 1) / kC;
+  const int BH = P.B * P.H;
+  cudaError_t e;
+  if (is_precond(P.variant)) {
+    k0_chunk_energy<<<dim3((unsigned)((N + 7) / 8), (unsigned)BH), kD, 0, stream>>>(P, ws, N);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    k0_prefix<<<BH, kD, 0, stream>>>(P, ws, N);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  switch (P.variant) {
+    case PDN_VAR_DN: e = launch_k1_decay<PDN_VAR_DN>(P, ws, N, stream); break;
+    case PDN_VAR_GDN: e = launch_k1_decay<PDN_VAR_GDN>(P, ws, N, stream); break;
+    case PDN_VAR_KDA: e = launch_k1_decay<PDN_VAR_KDA>(P, ws, N, stream); break;
+    case PDN_VAR_PDN: e = launch_k1_decay<PDN_VAR_PDN>(P, ws, N, stream); break;
+    case PDN_VAR_PGDN: e = launch_k1_decay<PDN_VAR_PGDN>(P, ws, N, stream); break;
+    case PDN_VAR_PKDA: e = launch_k1_decay<PDN_VAR_PKDA>(P, ws, N, stream); break;
+    case PDN_VAR_FG2_GDN: e = launch_k1_decay<PDN_VAR_FG2_GDN>(P, ws, N, stream); break;
+    default: e = launch_k1_decay<PDN_VAR_GDN2>(P, ws, N, stream); break;
+  }
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(k2_state, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)K2_BYTES);
+  if (e != cudaSuccess) return e;
+  k2_state<<<BH, kK2Threads, K2_BYTES, stream>>>(P, ws, N);
+  return cudaGetLastError();
+}
+
+}  // namespace pdn

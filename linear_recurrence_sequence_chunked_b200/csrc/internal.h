@@ -16,6 +16,12 @@ int tc_supported(const KParams &P);
 size_t tc_workspace_bytes(const KParams &P);
 cudaError_t launch_chunk_tc(const KParams &P, void *workspace, cudaStream_t stream);
 
+// Tensor-core three-kernel path: intra-chunk work for all chunks at once,
+// then the sequential state pass; needs a workspace.
+int split_supported(const KParams &P);
+size_t split_workspace_bytes(const KParams &P);
+cudaError_t launch_chunk_split(const KParams &P, void *workspace, cudaStream_t stream);
+
 // One decode step (state streamed through once).
 cudaError_t launch_decode(const KParams &P, cudaStream_t stream);
 

@@ -24,7 +24,7 @@ PDN_OK, PDN_ERR_INVALID_ARG, PDN_ERR_UNSUPPORTED, PDN_ERR_CUDA, PDN_ERR_TIMEOUT,
 VARIANTS = {"DN": 0, "GDN": 1, "KDA": 2, "PDN": 3, "PGDN": 4, "PKDA": 5, "FG2_GDN": 6, "GDN2": 7}
 DECAYS = {"none": 0, "scalar": 1, "channel": 2}
 DTYPES = {torch.float32: 0, torch.bfloat16: 1}
-IMPLS = {"auto": 0, "simt": 1, "tc": 2}
+IMPLS = {"auto": 0, "simt": 1, "tc": 2, "tc_fused": 3}
 PRECOND_VARIANTS = ("PDN", "PGDN", "PKDA")
 
 

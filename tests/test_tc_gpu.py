@@ -22,68 +22,82 @@ def tc_work(variant, decay=None, B=2, T=200, H=2, seed=0, **kw):
                     decay or DECAY[variant], seed=seed, **kw)
 
 
+TC_IMPLS = ["tc", "tc_fused"]
+
+
 def test_tc_kernel_is_selected():
     p = pdn.make_problem("PGDN", 4, 4096, 16, 128, 128, torch.bfloat16)
     assert pdn.pdn_chunk_fwd_impl(p) == pdn.IMPLS["tc"]
+    assert pdn.pdn_chunk_fwd_workspace(p) > 0
+    p = pdn.make_problem("PGDN", 4, 4096, 16, 128, 128, torch.bfloat16, impl="tc_fused")
+    assert pdn.pdn_chunk_fwd_impl(p) == pdn.IMPLS["tc_fused"]
+    assert pdn.pdn_chunk_fwd_workspace(p) == 0
     p = pdn.make_problem("PGDN", 1, 64, 2, 64, 64, torch.bfloat16)
     assert pdn.pdn_chunk_fwd_impl(p) == pdn.IMPLS["simt"]
 
 
+@pytest.mark.parametrize("impl", TC_IMPLS)
 @pytest.mark.parametrize("variant", VARIANTS)
-def test_tc_variants(variant):
+def test_tc_variants(variant, impl):
     w = tc_work(variant, q_scale=0.9)
     x = make_inputs(w)
     g = torch.Generator().manual_seed(2)
     S0 = 0.3 * torch.randn(w.B, w.H, 128, 128, generator=g)
     A0 = torch.rand(w.B, w.H, 128, generator=g) * 3 if variant in ("PDN", "PGDN", "PKDA") else None
-    o, ST, AT = run_gpu(w, x, S0, A0, impl="tc")
+    o, ST, AT = run_gpu(w, x, S0, A0, impl=impl)
     assert_parity(w, o, ST, AT, *run_oracle(w, x, S0, A0))
 
 
+@pytest.mark.parametrize("impl", TC_IMPLS)
 @pytest.mark.parametrize("decay", ["none", "scalar", "channel"])
 @pytest.mark.parametrize("variant", ["FG2_GDN", "GDN2"])
-def test_tc_free_decay(variant, decay):
+def test_tc_free_decay(variant, decay, impl):
     w = tc_work(variant, decay=decay, T=130)
     x = make_inputs(w)
-    o, ST, AT = run_gpu(w, x, impl="tc")
+    o, ST, AT = run_gpu(w, x, impl=impl)
     assert_parity(w, o, ST, AT, *run_oracle(w, x))
 
 
+@pytest.mark.parametrize("impl", TC_IMPLS)
 @pytest.mark.parametrize("T", [1, 63, 64, 65, 128, 1000])
-def test_tc_lengths(T):
+def test_tc_lengths(T, impl):
     w = tc_work("PKDA", T=T, B=1, H=3)
     x = make_inputs(w)
-    o, ST, AT = run_gpu(w, x, impl="tc")
+    o, ST, AT = run_gpu(w, x, impl=impl)
     assert_parity(w, o, ST, AT, *run_oracle(w, x))
 
 
 def test_tc_matches_simt():
-    """Both kernels on the same bf16 inputs agree to the bf16 tolerance."""
+    """The three paths on the same bf16 inputs agree to the bf16 tolerance."""
     w = tc_work("PGDN", B=2, H=4, T=333)
     x = make_inputs(w)
-    a = run_gpu(w, x, impl="tc")
     b = run_gpu(w, x, impl="simt")
-    assert nmax_err(a[0].float().cpu().numpy(), b[0].float().cpu().numpy()) < 2e-2
-    assert nmax_err(a[1].cpu().numpy(), b[1].cpu().numpy()) < 2e-2
+    for impl in TC_IMPLS:
+        a = run_gpu(w, x, impl=impl)
+        assert nmax_err(a[0].float().cpu().numpy(), b[0].float().cpu().numpy()) < 2e-2
+        assert nmax_err(a[1].cpu().numpy(), b[1].cpu().numpy()) < 2e-2
+        assert nmax_err(a[2].cpu().numpy(), b[2].cpu().numpy()) < 1e-5
 
 
-def test_tc_continuation():
+@pytest.mark.parametrize("impl", TC_IMPLS)
+def test_tc_continuation(impl):
     w = tc_work("PGDN", T=512, B=2, H=2)
     x = make_inputs(w)
-    o, ST, AT = run_gpu(w, x, impl="tc")
+    o, ST, AT = run_gpu(w, x, impl=impl)
     x1 = {n: (t[:, :192] if t is not None else None) for n, t in x.items()}
     x2 = {n: (t[:, 192:] if t is not None else None) for n, t in x.items()}
-    _, S1, A1 = run_gpu(w.replace(T=192), x1, impl="tc")
-    o2, S2, _ = run_gpu(w.replace(T=320), x2, S1.cpu(), A1.cpu(), impl="tc")
+    _, S1, A1 = run_gpu(w.replace(T=192), x1, impl=impl)
+    o2, S2, _ = run_gpu(w.replace(T=320), x2, S1.cpu(), A1.cpu(), impl=impl)
     assert nmax_err(o2.float().cpu().numpy(), o[:, 192:].float().cpu().numpy()) < 1e-2
     assert nmax_err(S2.cpu().numpy(), ST.cpu().numpy()) < 1e-2
 
 
-def test_tc_deterministic():
+@pytest.mark.parametrize("impl", TC_IMPLS)
+def test_tc_deterministic(impl):
     w = tc_work("PKDA", B=2, H=4, T=300)
     x = make_inputs(w)
-    a = run_gpu(w, x, impl="tc")
-    b = run_gpu(w, x, impl="tc")
+    a = run_gpu(w, x, impl=impl)
+    b = run_gpu(w, x, impl=impl)
     assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1]) and torch.equal(a[2], b[2])
 
 
