@@ -132,6 +132,29 @@ int pdn_chunk_fwd_impl(const pdn_problem_t *p);
 pdn_status_t pdn_chunk_fwd(const pdn_problem_t *p, const pdn_tensors_t *t,
                            void *workspace, size_t ws_bytes, void *stream);
 
+/* Allocation-free chunked forward. The paper has no counterpart: this entry
+ * point exists for callers that cannot allocate device memory for a
+ * workspace (code under a framework allocator that owns all device memory,
+ * latency-critical loops that cannot afford cudaMalloc's synchronisation,
+ * plugins handed only their input and output buffers). It runs the same
+ * tensor-core path as pdn_chunk_fwd with PDN_IMPL_TC (p->impl is ignored),
+ * using as its workspace a 64 MiB device array built into the library, so it
+ * calls no cudaMalloc/cudaFree and no allocating library routine; the caller
+ * still passes all inputs and outputs in `t`.
+ *   - Limit: problems whose workspace fits 64 MiB, i.e. B * H * ceil(T/64)
+ *     <= 809; larger problems return PDN_ERR_WORKSPACE before any launch.
+ *     Problems the tensor-core path does not take return PDN_ERR_UNSUPPORTED.
+ *   - The array is held by every GPU that loads the library until the
+ *     process exits. The first call on a device looks up its device address
+ *     (and may load the library's device code): make that first call before
+ *     any stream capture.
+ *   - All calls on a device share the one array and it keeps the last call's
+ *     contents; calls that overlap on the GPU (different streams or host
+ *     threads) race and must be serialised by the caller. Nothing needs
+ *     clearing between calls: every scratch byte a call reads it writes
+ *     first. */
+pdn_status_t pdn_chunk_fwd_noalloc(const pdn_problem_t *p, const pdn_tensors_t *t, void *stream);
+
 /* One decode step: p->T must be 1. The state and, for preconditioned
  * variants, the accumulator are updated IN PLACE: pass S0 == ST (non-NULL)
  * and A0 == AT (non-NULL for PDN/PGDN/PKDA, NULL otherwise). */

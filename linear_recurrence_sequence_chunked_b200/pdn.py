@@ -65,6 +65,8 @@ def load() -> ctypes.CDLL:
         lib.pdn_chunk_fwd_impl.argtypes = [P]
         lib.pdn_chunk_fwd.restype = ctypes.c_int
         lib.pdn_chunk_fwd.argtypes = [P, T, vp, ctypes.c_size_t, vp]
+        lib.pdn_chunk_fwd_noalloc.restype = ctypes.c_int
+        lib.pdn_chunk_fwd_noalloc.argtypes = [P, T, vp]
         lib.pdn_decode_step.restype = ctypes.c_int
         lib.pdn_decode_step.argtypes = [P, T, vp]
         lib.pdn_get_device_error.restype = ctypes.c_int
@@ -90,6 +92,12 @@ def pdn_chunk_fwd(problem: PdnProblem, tensors: PdnTensors, workspace: int, ws_b
                   stream: int) -> int:
     return load().pdn_chunk_fwd(ctypes.byref(problem), ctypes.byref(tensors), workspace,
                                 ws_bytes, stream)
+
+
+def pdn_chunk_fwd_noalloc(problem: PdnProblem, tensors: PdnTensors, stream: int) -> int:
+    """Allocation-free chunked forward (see include/pdn.h): scratch comes
+    from a fixed array inside the library instead of a caller workspace."""
+    return load().pdn_chunk_fwd_noalloc(ctypes.byref(problem), ctypes.byref(tensors), stream)
 
 
 def pdn_decode_step(problem: PdnProblem, tensors: PdnTensors, stream: int) -> int:
