@@ -22,6 +22,14 @@
 #include "ptx.cuh"
 #include "tiles.cuh"
 
+// Phase boundary hooks for out-of-tree timing harnesses; empty in the library.
+#ifndef PDN_K1_MARK
+#define PDN_K1_MARK(k)
+#endif
+#ifndef PDN_K2_MARK
+#define PDN_K2_MARK(k)
+#endif
+
 namespace pdn {
 namespace {
 
@@ -98,8 +106,12 @@ constexpr int MS_LD = 68, TS_LD = 68, YS_LD = 34; // fp32 solve scratch strides
 constexpr uint32_t K1_RQ = 0;                     // TL 128 x 128: Rh rows 0-63, Qh rows 64-127
 constexpr uint32_t K1_WH = 32768;                 // TL 64 x 128
 constexpr uint32_t K1_RA = 49152;                 // region A
-constexpr uint32_t K1_LBUF = K1_RA;               // prep: log2(A + eps)
-constexpr uint32_t K1_GBUF_PRE = K1_RA + 64 * LB_LD * 4;  // prep: cumulative log decay
+constexpr uint32_t KS_LD = 272;                   // staged row stride (bytes), padded
+constexpr uint32_t K1_KS = K1_RA;                 // prep: raw k, row-major [64][128] bf16
+constexpr uint32_t K1_QS = K1_RA + 64 * KS_LD;    // prep: raw q
+constexpr uint32_t K1_BC = K1_QS + 64 * KS_LD;    // prep: preconditioner coefficient B, bf16
+constexpr uint32_t K1_GBUF = K1_BC + 64 * KS_LD;  // prep: cumulative log decay, fp32 [64][132]
+constexpr uint32_t K1_LAS_STAGE = K1_GBUF + 64 * LB_LD * 4;  // prep: raw channel log decay
 constexpr uint32_t K1_TM = K1_RA;                 // TL 64 x 64
 constexpr uint32_t K1_PM = K1_RA + 8192;          // TL 64 x 64
 constexpr uint32_t K1_MS = K1_RA + 16384;         // fp32 [64][68]
@@ -108,21 +120,23 @@ constexpr uint32_t K1_YS = K1_TS + 64 * TS_LD * 4;// fp32 [32][34]
 constexpr uint32_t K1_YT = K1_RA + 16384;         // TL 128 x 64 (after the solve)
 constexpr uint32_t K1_SOLVE_END = K1_YS + 32 * YS_LD * 4;
 
-// Region A holds the prep buffers the variant needs, then the solve scratch.
+// Region A holds the prep buffers the variant needs (staged k and q, the
+// bf16 preconditioner coefficients, the fp32 cumulative log decay and the
+// staged channel log decay), then the solve scratch.
 template <int kVariant, int kDecay>
 struct K1Layout {
   static constexpr bool kPre =
       kVariant == PDN_VAR_PDN || kVariant == PDN_VAR_PGDN || kVariant == PDN_VAR_PKDA;
-  static constexpr uint32_t kGbuf = kPre ? K1_GBUF_PRE : K1_RA;
   static constexpr uint32_t kPrepEnd =
-      K1_RA + (kPre ? 64 * LB_LD * 4 : 0) + (kDecay == PDN_DECAY_CHANNEL ? 64 * LB_LD * 4 : 0);
+      kDecay == PDN_DECAY_CHANNEL ? K1_LAS_STAGE + 64 * 256 : K1_GBUF;
   static constexpr uint32_t kSmall = (kPrepEnd > K1_SOLVE_END ? kPrepEnd : K1_SOLVE_END);
   static constexpr uint32_t kAcar = kSmall, kGC = kSmall + 512, kEGC = kSmall + 1024;
   static constexpr uint32_t kPartK = kSmall + 1536, kPartG = kSmall + 2048;
-  static constexpr uint32_t kMu = kSmall + 2560, kBeta = kSmall + 2816, kGS = kSmall + 3072;
-  static constexpr uint32_t kLas = kSmall + 3328, kBar = kSmall + 3584;
-  static constexpr uint32_t kTbase = kSmall + 3600;
-  static constexpr uint32_t kBytes = kSmall + 3616;
+  static constexpr uint32_t kMup = kSmall + 2560;  // float[4][64] per-warp partial means
+  static constexpr uint32_t kMu = kSmall + 3584, kBeta = kSmall + 3840, kGS = kSmall + 4096;
+  static constexpr uint32_t kLas = kSmall + 4352, kBar = kSmall + 4608;
+  static constexpr uint32_t kTbase = kSmall + 4624;
+  static constexpr uint32_t kBytes = kSmall + 4640;
 };
 
 __device__ __forceinline__ void sync_for_mma() {
@@ -144,14 +158,14 @@ __global__ void __launch_bounds__(kK1Threads) k1_intra(const KParams P, void *ws
   float *EGC = reinterpret_cast<float *>(smem + L::kEGC);
   float *PARTK = reinterpret_cast<float *>(smem + L::kPartK);
   float *PARTG = reinterpret_cast<float *>(smem + L::kPartG);
+  float *MUP = reinterpret_cast<float *>(smem + L::kMup);
   float *MU = reinterpret_cast<float *>(smem + L::kMu);
   float *BETA = reinterpret_cast<float *>(smem + L::kBeta);
   float *GS = reinterpret_cast<float *>(smem + L::kGS);
   float *LAS = reinterpret_cast<float *>(smem + L::kLas);
   uint64_t *bar = reinterpret_cast<uint64_t *>(smem + L::kBar);
   uint32_t *tbase_p = reinterpret_cast<uint32_t *>(smem + L::kTbase);
-  float *LBUF = reinterpret_cast<float *>(smem + K1_LBUF);
-  float *GBUF = reinterpret_cast<float *>(smem + L::kGbuf);
+  float *GBUF = reinterpret_cast<float *>(smem + K1_GBUF);
   float *MS = reinterpret_cast<float *>(smem + K1_MS);
   float *TS = reinterpret_cast<float *>(smem + K1_TS);
   float *YS = reinterpret_cast<float *>(smem + K1_YS);
@@ -166,6 +180,7 @@ __global__ void __launch_bounds__(kK1Threads) k1_intra(const KParams P, void *ws
   const float log2x = P.lnx * kLog2e;
   const uint32_t lane_q = (uint32_t)(32 * (warp & 3)) << 16;
   const int half = warp >> 2;
+  PDN_K1_MARK(0);
 
   if (warp == 0) {
     tmem_alloc(tbase_p, 128);
@@ -176,7 +191,23 @@ __global__ void __launch_bounds__(kK1Threads) k1_intra(const KParams P, void *ws
     mbar_init(bar + 1, 1);
     fence_mbarrier_init();
   }
-  // ---- P0: per-token scalars, accumulator at the chunk start ----
+  // ---- P0: stage k, q (and the channel log decay) with cp.async; per-token
+  // scalars and the accumulator at the chunk start ----
+  {
+    const int c8 = tid & 15;
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+      const int t = (tid >> 4) + 16 * m;
+      const bool ok = t < Cn;
+      const size_t e = ok ? tok0 + (size_t)t * tstride + c8 * 8 : 0;
+      cp_async16(sb + K1_KS + t * KS_LD + c8 * 16, reinterpret_cast<const __nv_bfloat16 *>(P.k) + e, ok);
+      cp_async16(sb + K1_QS + t * KS_LD + c8 * 16, reinterpret_cast<const __nv_bfloat16 *>(P.q) + e, ok);
+      if (kDecay == PDN_DECAY_CHANNEL)
+        cp_async16(sb + K1_LAS_STAGE + t * 256 + c8 * 16,
+                   reinterpret_cast<const __nv_bfloat16 *>(P.log_alpha) + e, ok);
+    }
+    cp_async_commit();
+  }
   if (tid < kC) {
     const bool ok = tid < Cn;
     const size_t e = ok ? tok_index(P, b, c0 + tid, h) : 0;
@@ -185,29 +216,34 @@ __global__ void __launch_bounds__(kK1Threads) k1_intra(const KParams P, void *ws
                    ? __ldg(reinterpret_cast<const float *>(P.log_alpha) + e) : 0.f;
   }
   if (tid < kD) Acar[tid] = kPre ? reinterpret_cast<const float *>(blk + WS_A)[tid] : 0.f;
+  cp_async_wait_all();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tm = *tbase_p;
+  PDN_K1_MARK(1);
 
   // ---- P1: per-channel scans; thread = (channel, half of the chunk) ----
+  // Prefix sums of k.k (accumulator) and of the log decay over the chunk's
+  // tokens, then (preconditioned variants) the per-token channel mean of
+  // log2(A + eps) by a warp transpose-reduce, and B = x^(-s) per element.
   {
     const int i = tid & 127, hf = tid >> 7, t0 = 32 * hf;
-    const __nv_bfloat16 *kp = reinterpret_cast<const __nv_bfloat16 *>(P.k) + tok0 + i;
-    const __nv_bfloat16 *lp = reinterpret_cast<const __nv_bfloat16 *>(P.log_alpha) + tok0 + i;
     float kk[32], la[32];
     float ks = 0.f, gs = 0.f;
 #pragma unroll
     for (int e = 0; e < 32; ++e) {
       const int t = t0 + e;
-      kk[e] = 0.f;
-      la[e] = 0.f;
-      if (kPre && t < Cn) kk[e] = __bfloat162float(kp[t * tstride]);
-      if (kDecay == PDN_DECAY_CHANNEL) la[e] = t < Cn ? __bfloat162float(lp[t * tstride]) : 0.f;
-      else if (kDecay == PDN_DECAY_SCALAR) la[e] = LAS[t];
-    }
-#pragma unroll
-    for (int e = 0; e < 32; ++e) {
+      kk[e] = kPre ? __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(
+                         smem + K1_KS + t * KS_LD + i * 2))
+                   : 0.f;
+      if (kDecay == PDN_DECAY_CHANNEL)
+        la[e] = __bfloat162float(
+            *reinterpret_cast<const __nv_bfloat16 *>(smem + K1_LAS_STAGE + t * 256 + i * 2));
+      else if (kDecay == PDN_DECAY_SCALAR)
+        la[e] = LAS[t];
+      else
+        la[e] = 0.f;
       ks = fmaf(kk[e], kk[e], ks);
       gs += la[e];
     }
@@ -221,37 +257,51 @@ __global__ void __launch_bounds__(kK1Threads) k1_intra(const KParams P, void *ws
 #pragma unroll
     for (int e = 0; e < 32; ++e) {
       const int t = t0 + e;
-      if (kPre) {
-        a = fmaf(kk[e], kk[e], a);
-        LBUF[t * LB_LD + i] = lg2_approx(a + P.eps);
-      }
+      a = fmaf(kk[e], kk[e], a);
+      kk[e] = kPre ? lg2_approx(a + P.eps) : 0.f;  // kk now holds log2(A_t + eps)
       g += la[e];
       if (kDecay == PDN_DECAY_CHANNEL) GBUF[t * LB_LD + i] = g;
       else if (kDecay == PDN_DECAY_SCALAR && i == 0) GS[t] = g;
     }
     if (hf) {
       GC[i] = g;
-      const float e = ex2_approx(fmaxf(g, kMinG) * kLog2e);
-      EGC[i] = e;
-      reinterpret_cast<float *>(blk + WS_E)[i] = e;
+      const float eg = ex2_approx(fmaxf(g, kMinG) * kLog2e);
+      EGC[i] = eg;
+      reinterpret_cast<float *>(blk + WS_E)[i] = eg;
+    }
+    if (kPre) {
+      // transpose-reduce: after 5 butterfly steps lane l holds the sum over
+      // the warp's 32 channels of token t0 + l
+      float v[32];
+#pragma unroll
+      for (int e = 0; e < 32; ++e) v[e] = kk[e];
+#pragma unroll
+      for (int off = 16, len = 16; off >= 1; off >>= 1, len >>= 1) {
+        const bool upper = (lane & off) != 0;
+#pragma unroll
+        for (int e = 0; e < len; ++e) {
+          const float send = upper ? v[e] : v[e + len];
+          const float keep = upper ? v[e + len] : v[e];
+          v[e] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+        }
+      }
+      MUP[(warp & 3) * 64 + t0 + lane] = v[0];
+      __syncthreads();
+      if (tid < kC) MU[tid] = (MUP[tid] + MUP[64 + tid] + MUP[128 + tid] + MUP[192 + tid]) * (1.f / kD);
+      __syncthreads();
+      const float log2x_ = log2x;
+#pragma unroll
+      for (int e = 0; e < 32; ++e) {
+        const float cc = (kk[e] - MU[t0 + e]) * kLn2;
+        const float sq = cc * rcp_approx(1.f + fabsf(cc));
+        *reinterpret_cast<__nv_bfloat16 *>(smem + K1_BC + (t0 + e) * KS_LD + i * 2) =
+            __float2bfloat16_rn(ex2_approx(-sq * log2x_));
+      }
     }
   }
   __syncthreads();
-
-  // ---- P2: per-token channel mean of log2(A + eps) ----
-  if (kPre) {
-    const int t = tid >> 2, qd = tid & 3;
-    float s = 0.f;
-#pragma unroll
-    for (int k4 = 0; k4 < 8; ++k4) {
-      const float4 x = *reinterpret_cast<const float4 *>(LBUF + t * LB_LD + qd * 32 + 4 * k4);
-      s += (x.x + x.y) + (x.z + x.w);
-    }
-    s += __shfl_xor_sync(0xffffffffu, s, 1);
-    s += __shfl_xor_sync(0xffffffffu, s, 2);
-    if (qd == 0) MU[t] = s * (1.f / kD);
-    __syncthreads();
-  }
+  PDN_K1_MARK(2);
+  PDN_K1_MARK(3);
 
   // ---- P3: operand tiles, (token, 8-channel) units ----
   {
@@ -265,10 +315,7 @@ __global__ void __launch_bounds__(kK1Threads) k1_intra(const KParams P, void *ws
       ewb_s = EGC[0] * emg_s;
     }
     const float be = kScalarBeta ? BETA[t] : 0.f;
-    const float mu = kPre ? MU[t] : 0.f;
     const float qs = P.q_scale;
-    const __nv_bfloat16 *kb = reinterpret_cast<const __nv_bfloat16 *>(P.k);
-    const __nv_bfloat16 *qb = reinterpret_cast<const __nv_bfloat16 *>(P.q);
     const __nv_bfloat16 *vb = reinterpret_cast<const __nv_bfloat16 *>(P.v);
 #pragma unroll
     for (int m = 0; m < 4; ++m) {
@@ -276,21 +323,17 @@ __global__ void __launch_bounds__(kK1Threads) k1_intra(const KParams P, void *ws
       const int i0 = 8 * c8;
       float kf[8], qf[8], vf[8], r[8], w[8];
 #pragma unroll
-      for (int e = 0; e < 8; ++e) { kf[e] = 0.f; qf[e] = 0.f; vf[e] = 0.f; }
-      if (ok) {
-        unpack8(__ldg(reinterpret_cast<const uint4 *>(kb + etok + i0)), kf);
-        unpack8(__ldg(reinterpret_cast<const uint4 *>(qb + etok + i0)), qf);
-        unpack8(__ldg(reinterpret_cast<const uint4 *>(vb + etok + i0)), vf);
-      }
+      for (int e = 0; e < 8; ++e) vf[e] = 0.f;
+      unpack8(*reinterpret_cast<const uint4 *>(smem + K1_KS + t * KS_LD + c8 * 16), kf);
+      unpack8(*reinterpret_cast<const uint4 *>(smem + K1_QS + t * KS_LD + c8 * 16), qf);
+      if (ok) unpack8(__ldg(reinterpret_cast<const uint4 *>(vb + etok + i0)), vf);
       if (kPre) {
-        float Lv[8];
-        ld8f(LBUF + t * LB_LD + i0, Lv);
+        float Bv[8];
+        unpack8(*reinterpret_cast<const uint4 *>(smem + K1_BC + t * KS_LD + c8 * 16), Bv);
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
-          const float cc = (Lv[e] - mu) * kLn2;
-          const float s = cc * rcp_approx(1.f + fabsf(cc));
           r[e] = kf[e];
-          w[e] = be * ex2_approx(-s * log2x) * kf[e];
+          w[e] = be * Bv[e] * kf[e];
         }
       } else if (kVariant == PDN_VAR_FG2_GDN) {
         float gb[8];
@@ -362,6 +405,7 @@ __global__ void __launch_bounds__(kK1Threads) k1_intra(const KParams P, void *ws
 
   // ---- MMA1: D1 = [Rh;Qh] Wh^T ----
   sync_for_mma();
+  PDN_K1_MARK(4);
   if (tid == 0) {
     const uint32_t id = make_idesc_bf16(128, 64, false, false);
 #pragma unroll
@@ -377,6 +421,7 @@ __global__ void __launch_bounds__(kK1Threads) k1_intra(const KParams P, void *ws
     ok_all = !__syncthreads_or(!ok);
     tc_fence_after();
   }
+  PDN_K1_MARK(5);
 
   if (ok_all) {
     // ---- solve: M, P from TMEM; T = (I + M)^{-1} ----
@@ -413,6 +458,7 @@ __global__ void __launch_bounds__(kK1Threads) k1_intra(const KParams P, void *ws
     }
     tc_fence_before();
     __syncthreads();
+    PDN_K1_MARK(6);
     // L0: 16x16 diagonal blocks; the other threads zero the upper blocks the merges read
     if (tid < 64) {
       const int base = 16 * (tid >> 4), cc = tid & 15;
@@ -436,6 +482,7 @@ __global__ void __launch_bounds__(kK1Threads) k1_intra(const KParams P, void *ws
       }
     }
     __syncthreads();
+    PDN_K1_MARK(7);
     // L1: merge 16 -> 32 within [32p, 32p + 32): X = -T_D (M_CA T_A)
     if (tid < 128) {
       const int p = tid >> 6, rb = (tid >> 3) & 7, cb = tid & 7;
@@ -530,6 +577,7 @@ __global__ void __launch_bounds__(kK1Threads) k1_intra(const KParams P, void *ws
 
     // ---- MMA2: Y^T = Rh^T T^T ----
     sync_for_mma();
+    PDN_K1_MARK(8);
     if (tid == 0) {
       const uint32_t id = make_idesc_bf16(128, 64, true, false);
 #pragma unroll
@@ -544,6 +592,7 @@ __global__ void __launch_bounds__(kK1Threads) k1_intra(const KParams P, void *ws
       ok_all = !__syncthreads_or(!ok);
       tc_fence_after();
     }
+    PDN_K1_MARK(9);
     if (ok_all) {
       // Y^T -> bf16 tile (rows d_k, columns tokens)
       const int i = 32 * (warp & 3) + lane;
@@ -573,6 +622,7 @@ __global__ void __launch_bounds__(kK1Threads) k1_intra(const KParams P, void *ws
       }
     }
   }
+  PDN_K1_MARK(10);
   if (!ok_all && tid == 0) record_error(P.err, PDN_ERR_TIMEOUT);
   tc_fence_before();
   __syncthreads();
@@ -583,13 +633,20 @@ __global__ void __launch_bounds__(kK1Threads) k1_intra(const KParams P, void *ws
 // ===========================================================================
 // K2: state pass, one CTA per (batch, head)
 // ===========================================================================
-constexpr int kK2Threads = 512;  // 16 warps: TMEM lane quarter x column group
+// 16 compute warps run the state chain (TMEM lane quarter x column group);
+// 4 helper warps (one per lane quarter) write each chunk's output from TMEM
+// and prefetch operand sets, off the chain's critical path. They meet only at
+// mbarriers: full[s] (operand set s landed), bar5 (D^T ready), bar7 (chunk's
+// MMAs done), ofree[x] (output buffer x written out).
+constexpr int kK2Compute = 512;
+constexpr int kK2Threads = kK2Compute + 128;
 constexpr uint32_t K2_SET0 = 0;
 constexpr uint32_t K2_SET1 = WS_SET;
 constexpr uint32_t K2_SB = 2 * WS_SET;             // TL 128 x 128 bf16 copy of S
 constexpr uint32_t K2_DT = K2_SB + 32768;          // TL 128 x 64: D^T
-constexpr uint32_t K2_BAR = K2_DT + 16384;         // full[2], m5, m6, m7
-constexpr uint32_t K2_TBASE = K2_BAR + 5 * 8;
+constexpr uint32_t K2_BAR = K2_DT + 16384;         // full[2], bar5, bar7, ofree[2]
+constexpr uint32_t K2_ABORT = K2_BAR + 6 * 8;
+constexpr uint32_t K2_TBASE = K2_ABORT + 8;
 constexpr uint32_t K2_BYTES = K2_TBASE + 16;
 static_assert(K2_BYTES <= 232448, "state kernel shared memory budget");
 
@@ -602,26 +659,51 @@ __device__ __forceinline__ void issue_set_load(uint8_t *dst, const uint8_t *src,
   bulk_g2s(dst + 81920, src + 81920, WS_SET - 81920, bar);
 }
 
-// 16 output tokens [16 cg, 16 cg + 16) of O^T (TMEM lanes = value channels)
-// for one warp (its lane quarter), two adjacent channels per 32-bit store.
+// Barrier among the compute warps only (id 1).
+__device__ __forceinline__ void compute_sync() {
+  asm volatile("bar.sync 1, %0;" ::"n"(kK2Compute) : "memory");
+}
+// OR of a predicate over the compute warps; the same result in every thread.
+__device__ __forceinline__ bool compute_or(bool v) {
+  uint32_t r;
+  asm volatile(
+      "{ .reg .pred p, q; setp.ne.u32 q, %1, 0; bar.red.or.pred p, 1, %2, q; "
+      "selp.u32 %0, 1, 0, p; }"
+      : "=r"(r)
+      : "r"((uint32_t)v), "n"(kK2Compute)
+      : "memory");
+  return r != 0;
+}
+__device__ __forceinline__ void compute_sync_for_mma() {
+  fence_proxy_async_smem();
+  tc_fence_before();
+  compute_sync();
+  tc_fence_after();
+}
+
+// 64 output tokens of O^T (TMEM lanes = value channels) for one warp's lane
+// quarter, two adjacent channels per 32-bit store.
 __device__ __forceinline__ void k2_store_o(const KParams &P, uint32_t taddr, int b, int h,
-                                           int pc0, int Cn, int lane, int quarter, int cg) {
+                                           int pc0, int Cn, int lane, int quarter) {
   const size_t tstride = (size_t)P.H * kD;
   const int j = 32 * quarter + lane;
   __nv_bfloat16 *orow =
       reinterpret_cast<__nv_bfloat16 *>(P.o) + tok_index(P, b, pc0, h) * kD + (j & ~1);
   const bool odd = lane & 1;
-  float v[16];
-  tmem_ld16(taddr + 16 * cg, v);
-  tmem_wait_ld();
 #pragma unroll
-  for (int e2 = 0; e2 < 8; ++e2) {
-    const float send = odd ? v[2 * e2] : v[2 * e2 + 1];
-    const float recv = __shfl_xor_sync(0xffffffffu, send, 1);
-    const int t = 16 * cg + 2 * e2 + (odd ? 1 : 0);
-    const float lo = odd ? recv : v[2 * e2];
-    const float hi = odd ? v[2 * e2 + 1] : recv;
-    if (t < Cn) *reinterpret_cast<uint32_t *>(orow + t * tstride) = pack_bf16(lo, hi);
+  for (int cg = 0; cg < 4; ++cg) {
+    float v[16];
+    tmem_ld16(taddr + 16 * cg, v);
+    tmem_wait_ld();
+#pragma unroll
+    for (int e2 = 0; e2 < 8; ++e2) {
+      const float send = odd ? v[2 * e2] : v[2 * e2 + 1];
+      const float recv = __shfl_xor_sync(0xffffffffu, send, 1);
+      const int t = 16 * cg + 2 * e2 + (odd ? 1 : 0);
+      const float lo = odd ? recv : v[2 * e2];
+      const float hi = odd ? v[2 * e2 + 1] : recv;
+      if (t < Cn) *reinterpret_cast<uint32_t *>(orow + t * tstride) = pack_bf16(lo, hi);
+    }
   }
 }
 
@@ -629,152 +711,199 @@ __global__ void __launch_bounds__(kK2Threads, 1) k2_state(const KParams P, void 
   extern __shared__ __align__(1024) uint8_t smem[];
   const uint32_t sb = smem_u32(smem);
   uint64_t *full = reinterpret_cast<uint64_t *>(smem + K2_BAR);
-  uint64_t *bar5 = full + 2, *bar6 = full + 3, *bar7 = full + 4;
+  uint64_t *bar5 = full + 2, *bar7 = full + 3, *ofree = full + 4;
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + K2_ABORT);
   uint32_t *tbase_p = reinterpret_cast<uint32_t *>(smem + K2_TBASE);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int quarter = warp & 3, cg = warp >> 2;  // TMEM lanes 32*quarter.., column group 0..3
+  const int quarter = warp & 3;
   const uint32_t lane_q = (uint32_t)(32 * quarter) << 16;
   const int bh = blockIdx.x, b = bh / P.H, h = bh % P.H;
-  const int j = 32 * quarter + lane;  // value channel owned in the epilogues
 
   if (warp == 0) {
     tmem_alloc(tbase_p, 512);
     tmem_relinquish();
   }
   if (tid == 0) {
-    for (int i = 0; i < 5; ++i) mbar_init(full + i, 1);
+    for (int i = 0; i < 4; ++i) mbar_init(full + i, 1);
+    mbar_init(ofree + 0, 4);
+    mbar_init(ofree + 1, 4);
+    *abort_flag = 0;
     fence_mbarrier_init();
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tm = *tbase_p;
-  if (tid == 0 && N > 0) issue_set_load(smem + K2_SET0, ws_block(ws, bh, N, 0), full + 0);
 
-  auto wait_all = [&](uint64_t *bb, uint32_t parity) -> bool {
-    bool ok = true;
-    if (warp == 0) ok = mbar_wait_bounded(bb, parity, kSpin);
-    const bool fail = __syncthreads_or(!ok);
-    tc_fence_after();
-    return !fail;
-  };
+  if (tid >= kK2Compute) {
+    // ======================= helper warps =======================
+    const bool loader = tid == kK2Compute;
+    if (loader && N > 0) issue_set_load(smem + K2_SET0, ws_block(ws, bh, N, 0), full + 0);
+    if (loader && N > 1) issue_set_load(smem + K2_SET1, ws_block(ws, bh, N, 1), full + 1);
+    for (int n = 0; n < N; ++n) {
+      const int s = n & 1;
+      bool ok = true;
+      if (lane == 0) ok = mbar_wait_bounded(bar7, (uint32_t)(n & 1), kSpin) && !*abort_flag;
+      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+      tc_fence_after();
+      if (!ok) {
+        if (lane == 0) *abort_flag = 1;
+        break;
+      }
+      // chunk n's MMAs are done with operand set s: refill it two chunks ahead
+      if (loader && n + 2 < N) issue_set_load(smem + (s ? K2_SET1 : K2_SET0), ws_block(ws, bh, N, n + 2), full + s);
+      const int pc0 = n * kC;
+      k2_store_o(P, tm + lane_q + (s ? TM_OT1 : TM_OT0), b, h, pc0, min(kC, P.T - pc0), lane, quarter);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(ofree + s);
+    }
+  } else {
+    // ======================= compute warps =======================
+    const int cg = warp >> 2;          // column group 0..3
+    const int j = 32 * quarter + lane; // value channel owned in the epilogues
+    for (int n = 0; n < N; ++n) {
+      const int s = n & 1;
+      const uint32_t set = s ? K2_SET1 : K2_SET0;
+      const uint32_t ot = s ? TM_OT1 : TM_OT0;
+      PDN_K2_MARK(0);
+      {
+        bool ok = true;
+        if (warp == 0) ok = mbar_wait_bounded(full + s, (uint32_t)((n >> 1) & 1), kSpin);
+        if (compute_or(!ok || *abort_flag)) {
+          if (tid == 0) *abort_flag = 1;
+          break;
+        }
+      }
+      PDN_K2_MARK(1);
 
-  bool aborted = false;
-  for (int n = 0; n < N; ++n) {
-    const int s = n & 1;
-    const uint32_t set = s ? K2_SET1 : K2_SET0;
-    const uint32_t ot = s ? TM_OT1 : TM_OT0;
-    // the other set was last read by the previous chunk's MMAs (complete): refill it
-    if (tid == 0 && n + 1 < N)
-      issue_set_load(smem + (s ? K2_SET0 : K2_SET1), ws_block(ws, bh, N, n + 1), full + (s ^ 1));
-    if (!wait_all(full + s, (uint32_t)((n >> 1) & 1))) { aborted = true; break; }
-
-    // ---- state epilogue: S -> bf16 operand; TMEM S <- S Diag(e^{G_C}) ----
-    {
-      const float *egc = reinterpret_cast<const float *>(smem + set + WS_E);
-      float sv[2][16];
-      const int col0 = 32 * cg;
-      if (n == 0) {
+      // ---- state epilogue: S -> bf16 operand; TMEM S <- S Diag(e^{G_C}) ----
+      {
+        const float *egc = reinterpret_cast<const float *>(smem + set + WS_E);
+        float sv[2][16];
+        const int col0 = 32 * cg;
+        if (n == 0) {
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            if (P.S0) {
+              const float4 *src = reinterpret_cast<const float4 *>(
+                  P.S0 + ((size_t)bh * kD + j) * kD + col0 + 16 * u);
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const float4 x = __ldg(src + e);
+                sv[u][4 * e] = x.x; sv[u][4 * e + 1] = x.y;
+                sv[u][4 * e + 2] = x.z; sv[u][4 * e + 3] = x.w;
+              }
+            } else {
+#pragma unroll
+              for (int e = 0; e < 16; ++e) sv[u][e] = 0.f;
+            }
+          }
+        } else {
+          tmem_ld16(tm + lane_q + TM_S + col0, sv[0]);
+          tmem_ld16(tm + lane_q + TM_S + col0 + 16, sv[1]);
+          tmem_wait_ld();
+        }
 #pragma unroll
         for (int u = 0; u < 2; ++u) {
-          if (P.S0) {
-            const float4 *src =
-                reinterpret_cast<const float4 *>(P.S0 + ((size_t)bh * kD + j) * kD + col0 + 16 * u);
+          const int col = col0 + 16 * u;
+          float lo[8], hi[8], E[8];
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const float4 x = __ldg(src + e);
-              sv[u][4 * e] = x.x; sv[u][4 * e + 1] = x.y; sv[u][4 * e + 2] = x.z; sv[u][4 * e + 3] = x.w;
-            }
-          } else {
+          for (int e = 0; e < 8; ++e) { lo[e] = sv[u][e]; hi[e] = sv[u][8 + e]; }
+          *reinterpret_cast<uint4 *>(smem + K2_SB + tl128(j, col / 8)) = pack8(lo);
+          *reinterpret_cast<uint4 *>(smem + K2_SB + tl128(j, col / 8 + 1)) = pack8(hi);
+          ld8f(egc + col, E);
 #pragma unroll
-            for (int e = 0; e < 16; ++e) sv[u][e] = 0.f;
-          }
+          for (int e = 0; e < 8; ++e) sv[u][e] *= E[e];
+          ld8f(egc + col + 8, E);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) sv[u][8 + e] *= E[e];
+          tmem_st16(tm + lane_q + TM_S + col, sv[u]);
         }
-      } else {
-        tmem_ld16(tm + lane_q + TM_S + col0, sv[0]);
-        tmem_ld16(tm + lane_q + TM_S + col0 + 16, sv[1]);
+        tmem_wait_st();
+      }
+      compute_sync_for_mma();
+      PDN_K2_MARK(2);
+
+      // ---- MMA3: U^T = U^T T^T ; MMA5: D^T = U^T - S Y^T ; MMA6: O^T = S Qh^T ----
+      if (tid == 0) {
+        const uint32_t id3 = make_idesc_bf16(128, 64, true, false);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          mma_bf16_ss(tm + TM_UD, make_sdesc(sb + set + WS_U + 4096 * kk, 2048, 128),
+                      make_sdesc(sb + set + WS_T + 256 * kk, 128, 1024), id3, kk > 0);
+        const uint32_t id5 = make_idesc_bf16(128, 64, false, true, true);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_bf16_ss(tm + TM_UD, make_sdesc(sb + K2_SB + 256 * kk, 128, 2048),
+                      make_sdesc(sb + set + WS_Y + 2048 * kk, 1024, 128), id5, 1);
+        mma_commit(bar5);
+        // the helpers must have written out the output buffer chunk n-2 left here
+        bool ok = true;
+        if (n >= 2) ok = mbar_wait_bounded(ofree + s, (uint32_t)(((n - 2) >> 1) & 1), kSpin);
+        if (ok) {
+          const uint32_t id6 = make_idesc_bf16(128, 64, false, false);
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            mma_bf16_ss(tm + ot, make_sdesc(sb + K2_SB + 256 * kk, 128, 2048),
+                        make_sdesc(sb + set + WS_Q + 256 * kk, 128, 2048), id6, kk > 0);
+        } else {
+          *abort_flag = 1;
+        }
+      }
+      PDN_K2_MARK(3);
+      {
+        bool ok = true;
+        if (warp == 0) ok = mbar_wait_bounded(bar5, (uint32_t)(n & 1), kSpin);
+        const bool stop = compute_or(!ok || *abort_flag);
+        tc_fence_after();
+        if (stop) {
+          if (tid == 0) *abort_flag = 1;
+          break;
+        }
+      }
+      PDN_K2_MARK(4);
+
+      // ---- D^T -> bf16 operand (rows d_v, columns tokens) ----
+      {
+        float v[16];
+        tmem_ld16(tm + lane_q + TM_UD + 16 * cg, v);
         tmem_wait_ld();
+        float lo[8], hi[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) { lo[e] = v[e]; hi[e] = v[8 + e]; }
+        *reinterpret_cast<uint4 *>(smem + K2_DT + tl64(j, 2 * cg)) = pack8(lo);
+        *reinterpret_cast<uint4 *>(smem + K2_DT + tl64(j, 2 * cg + 1)) = pack8(hi);
       }
+      compute_sync_for_mma();
+      PDN_K2_MARK(5);
+
+      // ---- MMA7: O^T += D^T P^T ; MMA8: S += D^T Wb ----
+      if (tid == 0) {
+        const uint32_t id7 = make_idesc_bf16(128, 64, false, false);
+        const uint32_t id8 = make_idesc_bf16(128, 128, false, true);
 #pragma unroll
-      for (int u = 0; u < 2; ++u) {
-        const int col = col0 + 16 * u;
-        float lo[8], hi[8], E[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) { lo[e] = sv[u][e]; hi[e] = sv[u][8 + e]; }
-        *reinterpret_cast<uint4 *>(smem + K2_SB + tl128(j, col / 8)) = pack8(lo);
-        *reinterpret_cast<uint4 *>(smem + K2_SB + tl128(j, col / 8 + 1)) = pack8(hi);
-        ld8f(egc + col, E);
-#pragma unroll
-        for (int e = 0; e < 8; ++e) sv[u][e] *= E[e];
-        ld8f(egc + col + 8, E);
-#pragma unroll
-        for (int e = 0; e < 8; ++e) sv[u][8 + e] *= E[e];
-        tmem_st16(tm + lane_q + TM_S + col, sv[u]);
+        for (int kk = 0; kk < 4; ++kk) {
+          const uint64_t ad = make_sdesc(sb + K2_DT + 256 * kk, 128, 1024);
+          mma_bf16_ss(tm + ot, ad, make_sdesc(sb + set + WS_P + 256 * kk, 128, 1024), id7, 1);
+          mma_bf16_ss(tm + TM_S, ad, make_sdesc(sb + set + WS_WB + 4096 * kk, 2048, 128), id8, 1);
+        }
+        mma_commit(bar7);
       }
-      tmem_wait_st();
-    }
-    sync_for_mma();
-
-    // ---- MMA3: U^T = U^T T^T ; MMA5: D^T = U^T - S Y^T ; MMA6: O^T = S Qh^T ----
-    if (tid == 0) {
-      const uint32_t id3 = make_idesc_bf16(128, 64, true, false);
-#pragma unroll
-      for (int kk = 0; kk < 4; ++kk)
-        mma_bf16_ss(tm + TM_UD, make_sdesc(sb + set + WS_U + 4096 * kk, 2048, 128),
-                    make_sdesc(sb + set + WS_T + 256 * kk, 128, 1024), id3, kk > 0);
-      const uint32_t id5 = make_idesc_bf16(128, 64, false, true, true);
-#pragma unroll
-      for (int kk = 0; kk < 8; ++kk)
-        mma_bf16_ss(tm + TM_UD, make_sdesc(sb + K2_SB + 256 * kk, 128, 2048),
-                    make_sdesc(sb + set + WS_Y + 2048 * kk, 1024, 128), id5, 1);
-      mma_commit(bar5);
-      const uint32_t id6 = make_idesc_bf16(128, 64, false, false);
-#pragma unroll
-      for (int kk = 0; kk < 8; ++kk)
-        mma_bf16_ss(tm + ot, make_sdesc(sb + K2_SB + 256 * kk, 128, 2048),
-                    make_sdesc(sb + set + WS_Q + 256 * kk, 128, 2048), id6, kk > 0);
-      mma_commit(bar6);
-    }
-    // the previous chunk's output leaves while the MMAs run
-    if (n > 0)
-      k2_store_o(P, tm + lane_q + (s ? TM_OT0 : TM_OT1), b, h, (n - 1) * kC, kC, lane, quarter, cg);
-    tc_fence_before();
-    if (!wait_all(bar5, (uint32_t)(n & 1))) { aborted = true; break; }
-
-    // ---- D^T -> bf16 operand (rows d_v, columns tokens) ----
-    {
-      float v[16];
-      tmem_ld16(tm + lane_q + TM_UD + 16 * cg, v);
-      tmem_wait_ld();
-      float lo[8], hi[8];
-#pragma unroll
-      for (int e = 0; e < 8; ++e) { lo[e] = v[e]; hi[e] = v[8 + e]; }
-      *reinterpret_cast<uint4 *>(smem + K2_DT + tl64(j, 2 * cg)) = pack8(lo);
-      *reinterpret_cast<uint4 *>(smem + K2_DT + tl64(j, 2 * cg + 1)) = pack8(hi);
-    }
-    sync_for_mma();
-
-    // ---- MMA7: O^T += D^T P^T ; MMA8: S += D^T Wb ----
-    if (tid == 0) {
-      const uint32_t id7 = make_idesc_bf16(128, 64, false, false);
-      const uint32_t id8 = make_idesc_bf16(128, 128, false, true);
-#pragma unroll
-      for (int kk = 0; kk < 4; ++kk) {
-        const uint64_t ad = make_sdesc(sb + K2_DT + 256 * kk, 128, 1024);
-        mma_bf16_ss(tm + ot, ad, make_sdesc(sb + set + WS_P + 256 * kk, 128, 1024), id7, 1);
-        mma_bf16_ss(tm + TM_S, ad, make_sdesc(sb + set + WS_WB + 4096 * kk, 2048, 128), id8, 1);
+      PDN_K2_MARK(6);
+      {
+        bool ok = true;
+        if (warp == 0) ok = mbar_wait_bounded(bar7, (uint32_t)(n & 1), kSpin);
+        const bool stop = compute_or(!ok || *abort_flag);
+        tc_fence_after();
+        if (stop) {
+          if (tid == 0) *abort_flag = 1;
+          break;
+        }
       }
-      mma_commit(bar7);
+      PDN_K2_MARK(7);
     }
-    if (!wait_all(bar6, (uint32_t)(n & 1))) { aborted = true; break; }
-    if (!wait_all(bar7, (uint32_t)(n & 1))) { aborted = true; break; }
-  }
-
-  if (!aborted && N > 0) {
-    const int pc0 = (N - 1) * kC;
-    k2_store_o(P, tm + lane_q + (((N - 1) & 1) ? TM_OT1 : TM_OT0), b, h, pc0, P.T - pc0, lane,
-               quarter, cg);
-    if (P.ST) {
+    if (!*abort_flag && N > 0 && P.ST) {
       float v[2][16];
       const int col0 = 32 * cg;
       tmem_ld16(tm + lane_q + TM_S + col0, v[0]);
@@ -788,15 +917,21 @@ __global__ void __launch_bounds__(kK2Threads, 1) k2_state(const KParams P, void 
           dst[4 * u + e] = make_float4(v[u][4 * e], v[u][4 * e + 1], v[u][4 * e + 2], v[u][4 * e + 3]);
     }
   }
-  if (aborted) {
-    if (tid == 0) record_error(P.err, PDN_ERR_TIMEOUT);
-    // drain the operand loads still in flight before shared memory goes away
-    if (tid == 0)
-      for (int s = 0; s < 2; ++s) mbar_wait_bounded(full + s, 0, kSpin), mbar_wait_bounded(full + s, 1, kSpin);
-  }
+
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  if (*abort_flag) {
+    if (tid == 0) {
+      record_error(P.err, PDN_ERR_TIMEOUT);
+      // drain operand loads still in flight before shared memory goes away
+      for (int s2 = 0; s2 < 2; ++s2) {
+        mbar_wait_bounded(full + s2, 0, kSpin);
+        mbar_wait_bounded(full + s2, 1, kSpin);
+      }
+    }
+    __syncthreads();
+  }
   if (warp == 0) tmem_dealloc(tm, 512);
 }
 
