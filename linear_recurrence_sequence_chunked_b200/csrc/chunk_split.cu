@@ -60,23 +60,39 @@ constexpr float kMinG = -80.f;
 // ===========================================================================
 // K0: per-chunk key energy, then the exclusive prefix over chunks
 // ===========================================================================
-__global__ void __launch_bounds__(kD) k0_chunk_energy(const KParams P, void *ws, int N) {
-  const int bh = blockIdx.y, i = threadIdx.x;
+// One CTA per (batch, head, chunk): thread (8-channel group, token lane)
+// loads 16-byte rows and squares them; the 16 token lanes are summed in
+// shared memory.
+__global__ void __launch_bounds__(256) k0_chunk_energy(const KParams P, void *ws, int N) {
+  __shared__ float part[16][kD + 4];
+  const int c = blockIdx.x, bh = blockIdx.y, tid = threadIdx.x;
   const int b = bh / P.H, h = bh % P.H;
-  const __nv_bfloat16 *k = reinterpret_cast<const __nv_bfloat16 *>(P.k);
+  const int c8 = tid & 15, tl = tid >> 4;
+  const int c0 = c * kC, Cn = min(kC, P.T - c0);
   const size_t tstride = (size_t)P.H * kD;
-  for (int cc = 0; cc < 8; ++cc) {
-    const int c = blockIdx.x * 8 + cc;
-    if (c >= N) break;
-    const int c0 = c * kC, Cn = min(kC, P.T - c0);
-    const __nv_bfloat16 *kp = k + tok_index(P, b, c0, h) * kD + i;
-    float s = 0.f;
-#pragma unroll 8
-    for (int t = 0; t < Cn; ++t) {
-      const float kv = __bfloat162float(kp[t * tstride]);
-      s = fmaf(kv, kv, s);
+  const __nv_bfloat16 *kp =
+      reinterpret_cast<const __nv_bfloat16 *>(P.k) + tok_index(P, b, c0, h) * kD + c8 * 8;
+  float acc[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+#pragma unroll
+  for (int m = 0; m < 4; ++m) {
+    const int t = tl + 16 * m;
+    if (t < Cn) {
+      float kf[8];
+      unpack8(__ldg(reinterpret_cast<const uint4 *>(kp + t * tstride)), kf);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[e] = fmaf(kf[e], kf[e], acc[e]);
     }
-    reinterpret_cast<float *>(ws_block(ws, bh, N, c) + WS_A)[i] = s;
+  }
+#pragma unroll
+  for (int e = 0; e < 8; ++e) part[tl][c8 * 8 + e] = acc[e];
+  __syncthreads();
+  if (tid < kD) {
+    float s = 0.f;
+#pragma unroll
+    for (int r = 0; r < 16; ++r) s += part[r][tid];
+    reinterpret_cast<float *>(ws_block(ws, bh, N, c) + WS_A)[tid] = s;
   }
 }
 
@@ -139,6 +155,20 @@ struct K1Layout {
   static constexpr uint32_t kBytes = kSmall + 4640;
 };
 
+// 2^z for |z| < 1 on the FMA pipe: with y = z ln2 / 2, e^y by its Taylor
+// series to degree 6 (remainder below 1.3e-7 for |y| < 0.35), squared.
+__device__ __forceinline__ float exp2_small(float z) {
+  const float y = z * 0.34657359027997264f;
+  float p = 1.3888888888888889e-3f;   // 1/720
+  p = fmaf(p, y, 8.3333333333333333e-3f);  // 1/120
+  p = fmaf(p, y, 4.1666666666666667e-2f);  // 1/24
+  p = fmaf(p, y, 1.6666666666666667e-1f);  // 1/6
+  p = fmaf(p, y, 0.5f);
+  p = fmaf(p, y, 1.0f);
+  p = fmaf(p, y, 1.0f);
+  return p * p;
+}
+
 __device__ __forceinline__ void sync_for_mma() {
   fence_proxy_async_smem();
   tc_fence_before();
@@ -147,7 +177,7 @@ __device__ __forceinline__ void sync_for_mma() {
 }
 
 template <int kVariant, int kDecay>
-__global__ void __launch_bounds__(kK1Threads) k1_intra(const KParams P, void *ws, int N) {
+__global__ void __launch_bounds__(kK1Threads, 2) k1_intra(const KParams P, void *ws, int N) {
   using L = K1Layout<kVariant, kDecay>;
   constexpr bool kPre = L::kPre;
   constexpr bool kScalarBeta = kVariant != PDN_VAR_FG2_GDN && kVariant != PDN_VAR_GDN2;
@@ -171,16 +201,11 @@ __global__ void __launch_bounds__(kK1Threads) k1_intra(const KParams P, void *ws
   float *YS = reinterpret_cast<float *>(smem + K1_YS);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int c = blockIdx.x, bh = blockIdx.y;
-  const int b = bh / P.H, h = bh % P.H;
-  const int c0 = c * kC, Cn = min(kC, P.T - c0);
   const size_t tstride = (size_t)P.H * kD;
-  const size_t tok0 = tok_index(P, b, c0, h) * kD;  // element offset of token c0
-  uint8_t *blk = ws_block(ws, bh, N, c);
   const float log2x = P.lnx * kLog2e;
   const uint32_t lane_q = (uint32_t)(32 * (warp & 3)) << 16;
   const int half = warp >> 2;
-  PDN_K1_MARK(0);
+  const int total = N * P.B * P.H;  // chunk blocks; block index = bh * N + c
 
   if (warp == 0) {
     tmem_alloc(tbase_p, 128);
@@ -191,36 +216,93 @@ __global__ void __launch_bounds__(kK1Threads) k1_intra(const KParams P, void *ws
     mbar_init(bar + 1, 1);
     fence_mbarrier_init();
   }
-  // ---- P0: stage k, q (and the channel log decay) with cp.async; per-token
-  // scalars and the accumulator at the chunk start ----
-  {
-    const int c8 = tid & 15;
-#pragma unroll
-    for (int m = 0; m < 4; ++m) {
-      const int t = (tid >> 4) + 16 * m;
-      const bool ok = t < Cn;
-      const size_t e = ok ? tok0 + (size_t)t * tstride + c8 * 8 : 0;
-      cp_async16(sb + K1_KS + t * KS_LD + c8 * 16, reinterpret_cast<const __nv_bfloat16 *>(P.k) + e, ok);
-      cp_async16(sb + K1_QS + t * KS_LD + c8 * 16, reinterpret_cast<const __nv_bfloat16 *>(P.q) + e, ok);
-      if (kDecay == PDN_DECAY_CHANNEL)
-        cp_async16(sb + K1_LAS_STAGE + t * 256 + c8 * 16,
-                   reinterpret_cast<const __nv_bfloat16 *>(P.log_alpha) + e, ok);
-    }
-    cp_async_commit();
-  }
-  if (tid < kC) {
-    const bool ok = tid < Cn;
-    const size_t e = ok ? tok_index(P, b, c0 + tid, h) : 0;
-    BETA[tid] = (kScalarBeta && ok) ? __ldg(reinterpret_cast<const float *>(P.beta) + e) : 0.f;
-    LAS[tid] = (kDecay == PDN_DECAY_SCALAR && ok)
-                   ? __ldg(reinterpret_cast<const float *>(P.log_alpha) + e) : 0.f;
-  }
-  if (tid < kD) Acar[tid] = kPre ? reinterpret_cast<const float *>(blk + WS_A)[tid] : 0.f;
-  cp_async_wait_all();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tm = *tbase_p;
+
+  // Per-token and per-channel scalars of a chunk block, loaded one block
+  // ahead into registers. k and q are staged by cp.async at the start of the
+  // block; v one block ahead through shared memory (see stage_v).
+  struct Raw {
+    float beta, las, acar;
+  };
+  auto load_raw = [&](int it) {
+    Raw r;
+    const int c_ = it % N, bh_ = it / N;
+    const int b_ = bh_ / P.H, h_ = bh_ % P.H;
+    const int c0_ = c_ * kC, Cn_ = min(kC, P.T - c0_);
+    r.beta = 0.f;
+    r.las = 0.f;
+    if (tid < kC && tid < Cn_) {
+      const size_t e = tok_index(P, b_, c0_ + tid, h_);
+      if (kScalarBeta) r.beta = __ldg(reinterpret_cast<const float *>(P.beta) + e);
+      if (kDecay == PDN_DECAY_SCALAR) r.las = __ldg(reinterpret_cast<const float *>(P.log_alpha) + e);
+    }
+    r.acar = (kPre && tid < kD) ? reinterpret_cast<const float *>(ws_block(ws, bh_, N, c_) + WS_A)[tid] : 0.f;
+    return r;
+  };
+  // v of a chunk block into the Wh tile's space, rows of 256 bytes with the
+  // 16-byte groups XOR-swizzled by (token & 7); issued while the previous
+  // block is in its solve (the Wh tile is dead once MMA1 has completed).
+  auto stage_v = [&](int it) {
+    const int c_ = it % N, bh_ = it / N;
+    const int b_ = bh_ / P.H, h_ = bh_ % P.H;
+    const int c0_ = c_ * kC, Cn_ = min(kC, P.T - c0_);
+    const size_t tok0_ = tok_index(P, b_, c0_, h_) * kD;
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+      const int t = (tid >> 4) + 16 * m, c8 = tid & 15;
+      const bool ok = t < Cn_;
+      const size_t e = ok ? tok0_ + (size_t)t * tstride + c8 * 8 : 0;
+      cp_async16(sb + K1_WH + t * 256 + ((c8 ^ (t & 7)) << 4),
+                 reinterpret_cast<const __nv_bfloat16 *>(P.v) + e, ok);
+    }
+    cp_async_commit();
+  };
+  Raw pf = load_raw(blockIdx.x < total ? blockIdx.x : 0);
+  if (blockIdx.x < total) stage_v(blockIdx.x);
+
+  int iter = 0;
+  for (int it = blockIdx.x; it < total; it += gridDim.x, ++iter) {
+  const int c = it % N, bh = it / N;
+  const int b = bh / P.H, h = bh % P.H;
+  const int c0 = c * kC, Cn = min(kC, P.T - c0);
+  const size_t tok0 = tok_index(P, b, c0, h) * kD;  // element offset of token c0
+  uint8_t *blk = ws_block(ws, bh, N, c);
+  const uint32_t par = (uint32_t)(iter & 1);  // mbarrier parity of this block's MMAs
+  PDN_K1_MARK(0);
+
+  // ---- P0: k, q (and the channel log decay) by cp.async; the prefetched
+  // scalars into shared memory; then start loading the next block's ----
+  uint4 vcur[4];
+  {
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+      const int t = (tid >> 4) + 16 * m, c8 = tid & 15;
+      {
+        const bool ok = t < Cn;
+        const size_t e = ok ? tok0 + (size_t)t * tstride + c8 * 8 : 0;
+        cp_async16(sb + K1_KS + t * KS_LD + c8 * 16, reinterpret_cast<const __nv_bfloat16 *>(P.k) + e, ok);
+        cp_async16(sb + K1_QS + t * KS_LD + c8 * 16, reinterpret_cast<const __nv_bfloat16 *>(P.q) + e, ok);
+      }
+      if (kDecay == PDN_DECAY_CHANNEL) {
+        const bool ok = t < Cn;
+        const size_t e = ok ? tok0 + (size_t)t * tstride + c8 * 8 : 0;
+        cp_async16(sb + K1_LAS_STAGE + t * 256 + c8 * 16,
+                   reinterpret_cast<const __nv_bfloat16 *>(P.log_alpha) + e, ok);
+      }
+    }
+    cp_async_commit();
+    if (tid < kC) {
+      BETA[tid] = pf.beta;
+      LAS[tid] = pf.las;
+    }
+    if (tid < kD) Acar[tid] = pf.acar;
+  }
+  if (it + (int)gridDim.x < total) pf = load_raw(it + gridDim.x);
+  cp_async_wait_all();
+  __syncthreads();
   PDN_K1_MARK(1);
 
   // ---- P1: per-channel scans; thread = (channel, half of the chunk) ----
@@ -295,9 +377,16 @@ __global__ void __launch_bounds__(kK1Threads) k1_intra(const KParams P, void *ws
         const float cc = (kk[e] - MU[t0 + e]) * kLn2;
         const float sq = cc * rcp_approx(1.f + fabsf(cc));
         *reinterpret_cast<__nv_bfloat16 *>(smem + K1_BC + (t0 + e) * KS_LD + i * 2) =
-            __float2bfloat16_rn(ex2_approx(-sq * log2x_));
+            __float2bfloat16_rn(exp2_small(-sq * log2x_));
       }
     }
+  }
+  // this block's v into registers (operand mapping) before P3 overwrites the
+  // staging space with the Wh tile
+#pragma unroll
+  for (int m = 0; m < 4; ++m) {
+    const int t = 8 * warp + (lane & 7), c8 = 4 * m + (lane >> 3);
+    vcur[m] = *reinterpret_cast<const uint4 *>(smem + K1_WH + t * 256 + ((c8 ^ (t & 7)) << 4));
   }
   __syncthreads();
   PDN_K1_MARK(2);
@@ -316,17 +405,14 @@ __global__ void __launch_bounds__(kK1Threads) k1_intra(const KParams P, void *ws
     }
     const float be = kScalarBeta ? BETA[t] : 0.f;
     const float qs = P.q_scale;
-    const __nv_bfloat16 *vb = reinterpret_cast<const __nv_bfloat16 *>(P.v);
 #pragma unroll
     for (int m = 0; m < 4; ++m) {
       const int c8 = 4 * m + (lane >> 3);
       const int i0 = 8 * c8;
       float kf[8], qf[8], vf[8], r[8], w[8];
-#pragma unroll
-      for (int e = 0; e < 8; ++e) vf[e] = 0.f;
       unpack8(*reinterpret_cast<const uint4 *>(smem + K1_KS + t * KS_LD + c8 * 16), kf);
       unpack8(*reinterpret_cast<const uint4 *>(smem + K1_QS + t * KS_LD + c8 * 16), qf);
-      if (ok) unpack8(__ldg(reinterpret_cast<const uint4 *>(vb + etok + i0)), vf);
+      unpack8(vcur[m], vf);
       if (kPre) {
         float Bv[8];
         unpack8(*reinterpret_cast<const uint4 *>(smem + K1_BC + t * KS_LD + c8 * 16), Bv);
@@ -417,13 +503,14 @@ __global__ void __launch_bounds__(kK1Threads) k1_intra(const KParams P, void *ws
   bool ok_all = true;
   {
     bool ok = true;
-    if (warp == 0) ok = mbar_wait_bounded(bar + 0, 0, kSpin);
+    if (warp == 0) ok = mbar_wait_bounded(bar + 0, par, kSpin);
     ok_all = !__syncthreads_or(!ok);
     tc_fence_after();
   }
   PDN_K1_MARK(5);
 
   if (ok_all) {
+    if (it + (int)gridDim.x < total) stage_v(it + gridDim.x);
     // ---- solve: M, P from TMEM; T = (I + M)^{-1} ----
     {
       const int row = 32 * (warp & 3) + lane;
@@ -588,7 +675,7 @@ __global__ void __launch_bounds__(kK1Threads) k1_intra(const KParams P, void *ws
     }
     {
       bool ok = true;
-      if (warp == 0) ok = mbar_wait_bounded(bar + 1, 0, kSpin);
+      if (warp == 0) ok = mbar_wait_bounded(bar + 1, par, kSpin);
       ok_all = !__syncthreads_or(!ok);
       tc_fence_after();
     }
@@ -623,7 +710,15 @@ __global__ void __launch_bounds__(kK1Threads) k1_intra(const KParams P, void *ws
     }
   }
   PDN_K1_MARK(10);
-  if (!ok_all && tid == 0) record_error(P.err, PDN_ERR_TIMEOUT);
+  if (!ok_all) {
+    if (tid == 0) record_error(P.err, PDN_ERR_TIMEOUT);
+    break;
+  }
+  // the next block rewrites the shared-memory tiles the bulk stores read
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  }  // chunk blocks
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -942,7 +1037,21 @@ cudaError_t launch_k1(const KParams &P, void *ws, int N, cudaStream_t stream) {
   cudaError_t e =
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L::kBytes);
   if (e != cudaSuccess) return e;
-  kern<<<dim3((unsigned)N, (unsigned)(P.B * P.H)), kK1Threads, L::kBytes, stream>>>(P, ws, N);
+  // the largest shared-memory carveout, so that two CTAs fit on an SM
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+  if (e != cudaSuccess) return e;
+  int dev = 0, sms = 148, per_sm = 1;
+  if (cudaGetDevice(&dev) == cudaSuccess)
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kK1Threads, L::kBytes) != cudaSuccess ||
+      per_sm < 1)
+    per_sm = 1;
+  const long long total = (long long)N * P.B * P.H;
+  // At least two CTAs per SM: the blocks are independent, so a CTA that does
+  // not fit yet simply starts when one finishes, at no loss.
+  if (per_sm < 2) per_sm = 2;
+  const long long grid = total < (long long)sms * per_sm ? total : (long long)sms * per_sm;
+  kern<<<(unsigned)grid, kK1Threads, L::kBytes, stream>>>(P, ws, N);
   return cudaGetLastError();
 }
 
@@ -973,7 +1082,7 @@ cudaError_t launch_chunk_split(const KParams &P, void *ws, cudaStream_t stream) 
   const int BH = P.B * P.H;
   cudaError_t e;
   if (is_precond(P.variant)) {
-    k0_chunk_energy<<<dim3((unsigned)((N + 7) / 8), (unsigned)BH), kD, 0, stream>>>(P, ws, N);
+    k0_chunk_energy<<<dim3((unsigned)N, (unsigned)BH), 256, 0, stream>>>(P, ws, N);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     k0_prefix<<<BH, kD, 0, stream>>>(P, ws, N);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
