@@ -29,6 +29,12 @@
 #ifndef PDN_K2_MARK
 #define PDN_K2_MARK(k)
 #endif
+#ifndef PDN_K2_IMARK
+#define PDN_K2_IMARK(k)
+#endif
+#ifndef PDN_K2_HMARK
+#define PDN_K2_HMARK(k)
+#endif
 
 namespace pdn {
 namespace {
@@ -728,24 +734,40 @@ __global__ void __launch_bounds__(kK1Threads, 2) k1_intra(const KParams P, void 
 // ===========================================================================
 // K2: state pass, one CTA per (batch, head)
 // ===========================================================================
-// 16 compute warps run the state chain (TMEM lane quarter x column group);
-// 4 helper warps (one per lane quarter) write each chunk's output from TMEM
-// and prefetch operand sets, off the chain's critical path. They meet only at
-// mbarriers: full[s] (operand set s landed), bar5 (D^T ready), bar7 (chunk's
-// MMAs done), ofree[x] (output buffer x written out).
+// Warp roles. 16 compute warps (TMEM lane quarter x column group) run the
+// epilogues of the state chain and write each chunk's output; the S warp
+// issues the MMAs of the state chain (MMA3, MMA5, MMA8); the O warp issues
+// the output MMAs (MMA6, MMA7); the load warp prefetches operand sets two
+// chunks ahead. They meet only at mbarriers:
+//   full[s]  operand set s landed (bulk copy)
+//   sepi     state epilogue of the chunk done (one arrival per compute warp)
+//   depi     D^T epilogue of the chunk done (one arrival per compute warp)
+//   bar5     MMA3 (U~^T) and MMA5 (D^T) done      (S warp)
+//   bar7     MMA8 (state update) done             (S warp)
+//   bar6     MMA6 (O^T = S Qh^T) done              (O warp)
+//   baro     MMA7 (O^T += D^T P^T) done: the chunk's output and, since the O
+//            warp waits on bar7 first, every MMA of the chunk
+// The O warp issues MMA6 only after MMA5 and MMA7 only after MMA8 have
+// completed, so the tensor pipe never holds output work ahead of the state
+// chain's. The compute warps write chunk n - 1's output while MMA5 of chunk
+// n runs. The A operands that the epilogues produce (S and D^T in bf16) stay
+// in TMEM; only the B operands are read from shared memory. An operand set is
+// refilled in two parts: Qh, Y^T, U^T and T once MMA6 is done with them,
+// Wb, P and e^{G_C} once the chunk's last MMA is.
 constexpr int kK2Compute = 512;
-constexpr int kK2Threads = kK2Compute + 128;
+constexpr int kK2SWarp = kK2Compute / 32, kK2OWarp = kK2SWarp + 1, kK2LoadWarp = kK2SWarp + 2;
+constexpr int kK2Threads = kK2Compute + 96;
 constexpr uint32_t K2_SET0 = 0;
 constexpr uint32_t K2_SET1 = WS_SET;
-constexpr uint32_t K2_SB = 2 * WS_SET;             // TL 128 x 128 bf16 copy of S
-constexpr uint32_t K2_DT = K2_SB + 32768;          // TL 128 x 64: D^T
-constexpr uint32_t K2_BAR = K2_DT + 16384;         // full[2], bar5, bar7, ofree[2]
-constexpr uint32_t K2_ABORT = K2_BAR + 6 * 8;
+constexpr uint32_t K2_BAR = 2 * WS_SET;            // the eight mbarriers above
+constexpr uint32_t K2_ABORT = K2_BAR + 8 * 8;
 constexpr uint32_t K2_TBASE = K2_ABORT + 8;
 constexpr uint32_t K2_BYTES = K2_TBASE + 16;
 static_assert(K2_BYTES <= 232448, "state kernel shared memory budget");
 
-constexpr uint32_t TM_UD = 0, TM_OT0 = 64, TM_OT1 = 128, TM_S = 256;
+// TMEM columns: U~^T then D^T (fp32), the two O^T buffers, S in bf16 pairs
+// (the A operand of MMA5/MMA6), S (fp32), D^T in bf16 pairs (A of MMA7/MMA8).
+constexpr uint32_t TM_UD = 0, TM_OT0 = 64, TM_OT1 = 128, TM_SB = 192, TM_S = 256, TM_DB = 384;
 
 __device__ __forceinline__ void issue_set_load(uint8_t *dst, const uint8_t *src, uint64_t *bar) {
   mbar_arrive_expect_tx(bar, WS_SET);
@@ -753,60 +775,159 @@ __device__ __forceinline__ void issue_set_load(uint8_t *dst, const uint8_t *src,
   for (int p = 0; p < 5; ++p) bulk_g2s(dst + p * 16384, src + p * 16384, 16384, bar);
   bulk_g2s(dst + 81920, src + 81920, WS_SET - 81920, bar);
 }
+// The part of a set MMA3, MMA5 and MMA6 read (Qh, Y^T, U^T, T); the barrier
+// expects the whole set, so its phase completes only with the other part.
+__device__ __forceinline__ void issue_set_load_early(uint8_t *dst, const uint8_t *src, uint64_t *bar) {
+  mbar_arrive_expect_tx(bar, WS_SET);
+#pragma unroll
+  for (int p = 0; p < 3; ++p) bulk_g2s(dst + p * 16384, src + p * 16384, 16384, bar);
+  bulk_g2s(dst + WS_T, src + WS_T, WS_P - WS_T, bar);
+}
+// The rest (Wb, P, e^{G_C}).
+__device__ __forceinline__ void issue_set_load_late(uint8_t *dst, const uint8_t *src, uint64_t *bar) {
+  bulk_g2s(dst + WS_WB, src + WS_WB, WS_T - WS_WB, bar);
+  bulk_g2s(dst + WS_P, src + WS_P, WS_SET - WS_P, bar);
+}
+static_assert(WS_Y == WS_Q + 16384 && WS_U == WS_Y + 16384 && WS_WB == WS_U + 16384 &&
+                  WS_T == WS_WB + 16384 && WS_P > WS_T && WS_E > WS_P && WS_SET > WS_E,
+              "operand set layout the split refill assumes");
 
-// Barrier among the compute warps only (id 1).
-__device__ __forceinline__ void compute_sync() {
-  asm volatile("bar.sync 1, %0;" ::"n"(kK2Compute) : "memory");
-}
-// OR of a predicate over the compute warps; the same result in every thread.
-__device__ __forceinline__ bool compute_or(bool v) {
-  uint32_t r;
-  asm volatile(
-      "{ .reg .pred p, q; setp.ne.u32 q, %1, 0; bar.red.or.pred p, 1, %2, q; "
-      "selp.u32 %0, 1, 0, p; }"
-      : "=r"(r)
-      : "r"((uint32_t)v), "n"(kK2Compute)
-      : "memory");
-  return r != 0;
-}
-__device__ __forceinline__ void compute_sync_for_mma() {
-  fence_proxy_async_smem();
-  tc_fence_before();
-  compute_sync();
+// One lane of the warp waits (bounded) on `bar`; the outcome is the warp's.
+// A wait that runs out, or an abort raised elsewhere, sets the abort flag.
+__device__ __forceinline__ bool k2_warp_wait(uint64_t *bar, uint32_t parity,
+                                             volatile int *abort_flag, int lane) {
+  bool ok = true;
+  if (lane == 0) ok = mbar_wait_bounded(bar, parity, kSpin) && !*abort_flag;
+  ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
   tc_fence_after();
+  if (!ok && lane == 0) *abort_flag = 1;
+  return ok;
+}
+// Publishes this warp's TMEM accesses to the issuing warps.
+__device__ __forceinline__ void k2_warp_arrive(uint64_t *bar, int lane) {
+  tc_fence_before();
+  __syncwarp();
+  if (lane == 0) mbar_arrive(bar);
+}
+// Single-thread bounded wait for the issuing warps.
+__device__ __forceinline__ bool k2_wait(uint64_t *bar, uint32_t parity, volatile int *abort_flag) {
+  const bool ok = mbar_wait_bounded(bar, parity, kSpin) && !*abort_flag;
+  tc_fence_after();
+  return ok;
 }
 
-// 64 output tokens of O^T (TMEM lanes = value channels) for one warp's lane
-// quarter, two adjacent channels per 32-bit store.
+// 16 output tokens (columns 16 cg .. 16 cg + 15 of O^T in TMEM, lanes = value
+// channels) of one lane quarter; two adjacent channels per 32-bit store.
 __device__ __forceinline__ void k2_store_o(const KParams &P, uint32_t taddr, int b, int h,
-                                           int pc0, int Cn, int lane, int quarter) {
+                                           int pc0, int Cn, int lane, int quarter, int cg) {
   const size_t tstride = (size_t)P.H * kD;
   const int j = 32 * quarter + lane;
   __nv_bfloat16 *orow =
       reinterpret_cast<__nv_bfloat16 *>(P.o) + tok_index(P, b, pc0, h) * kD + (j & ~1);
   const bool odd = lane & 1;
+  float v[16];
+  tmem_ld16(taddr + 16 * cg, v);
+  tmem_wait_ld();
 #pragma unroll
-  for (int cg = 0; cg < 4; ++cg) {
-    float v[16];
-    tmem_ld16(taddr + 16 * cg, v);
-    tmem_wait_ld();
+  for (int e2 = 0; e2 < 8; ++e2) {
+    const float send = odd ? v[2 * e2] : v[2 * e2 + 1];
+    const float recv = __shfl_xor_sync(0xffffffffu, send, 1);
+    const int t = 16 * cg + 2 * e2 + (odd ? 1 : 0);
+    const float lo = odd ? recv : v[2 * e2];
+    const float hi = odd ? v[2 * e2 + 1] : recv;
+    if (t < Cn) *reinterpret_cast<uint32_t *>(orow + t * tstride) = pack_bf16(lo, hi);
+  }
+}
+
+// MMA3: U~^T = U^T T^T of the chunk whose operand set is at shared address `set`.
+__device__ __forceinline__ void k2_mma3(uint32_t tm, uint32_t set) {
+  const uint32_t id3 = make_idesc_bf16(128, 64, true, false);
 #pragma unroll
-    for (int e2 = 0; e2 < 8; ++e2) {
-      const float send = odd ? v[2 * e2] : v[2 * e2 + 1];
-      const float recv = __shfl_xor_sync(0xffffffffu, send, 1);
-      const int t = 16 * cg + 2 * e2 + (odd ? 1 : 0);
-      const float lo = odd ? recv : v[2 * e2];
-      const float hi = odd ? v[2 * e2 + 1] : recv;
-      if (t < Cn) *reinterpret_cast<uint32_t *>(orow + t * tstride) = pack_bf16(lo, hi);
+  for (int kk = 0; kk < 4; ++kk)
+    mma_bf16_ss(tm + TM_UD, make_sdesc(set + WS_U + 4096 * kk, 2048, 128),
+                make_sdesc(set + WS_T + 256 * kk, 128, 1024), id3, kk > 0);
+}
+
+struct K2Bars {
+  uint64_t *full, *bar5, *bar6, *bar7, *baro, *sepi, *depi;
+};
+
+// The S warp's program (one lane): MMA3, MMA5, MMA8. False if a wait ran out.
+__device__ __forceinline__ bool k2_issue_s(uint32_t tm, uint32_t sb, const K2Bars &B,
+                                           volatile int *abort_flag, int N) {
+  const uint32_t id5 = make_idesc_bf16(128, 64, false, true, true);
+  const uint32_t id8 = make_idesc_bf16(128, 128, false, true);
+  for (int n = 0; n < N; ++n) {
+    const int s = n & 1;
+    const uint32_t set = sb + (s ? K2_SET1 : K2_SET0);
+    if (n == 0) {
+      if (!k2_wait(B.full + 0, 0, abort_flag)) return false;
+      k2_mma3(tm, set);
+    }
+    // MMA5: D^T = U~^T - S Y^T, once the state epilogue has written S (bf16)
+    if (!k2_wait(B.sepi, (uint32_t)(n & 1), abort_flag)) return false;
+    PDN_K2_IMARK(0);
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk)
+      mma_bf16_ts(tm + TM_UD, tm + TM_SB + 8 * kk, make_sdesc(set + WS_Y + 2048 * kk, 1024, 128),
+                  id5, 1);
+    mma_commit(B.bar5);
+    PDN_K2_IMARK(1);
+    // MMA8: S += D^T Wb, once D^T is in shared memory
+    if (!k2_wait(B.depi, (uint32_t)(n & 1), abort_flag)) return false;
+    PDN_K2_IMARK(2);
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk)
+      mma_bf16_ts(tm + TM_S, tm + TM_DB + 8 * kk, make_sdesc(set + WS_WB + 4096 * kk, 2048, 128),
+                  id8, 1);
+    mma_commit(B.bar7);
+    PDN_K2_IMARK(3);
+    // MMA3 of chunk n + 1 (the D^T epilogue has read this chunk's U~^T)
+    if (n + 1 < N) {
+      if (!k2_wait(B.full + (s ^ 1), (uint32_t)(((n + 1) >> 1) & 1), abort_flag)) return false;
+      k2_mma3(tm, sb + (s ? K2_SET0 : K2_SET1));
     }
   }
+  return true;
+}
+
+// The O warp's program (one lane): MMA6, MMA7. False if a wait ran out.
+__device__ __forceinline__ bool k2_issue_o(uint32_t tm, uint32_t sb, const K2Bars &B,
+                                           volatile int *abort_flag, int N) {
+  const uint32_t id6 = make_idesc_bf16(128, 64, false, false);
+  const uint32_t id7 = make_idesc_bf16(128, 64, false, false);
+  for (int n = 0; n < N; ++n) {
+    const int s = n & 1;
+    const uint32_t set = sb + (s ? K2_SET1 : K2_SET0);
+    const uint32_t ot = s ? TM_OT1 : TM_OT0;
+    // MMA6: O^T = S Qh^T after MMA5 (which also means the compute warps have
+    // written out chunk n - 2's output from this buffer)
+    if (!k2_wait(B.bar5, (uint32_t)(n & 1), abort_flag)) return false;
+    PDN_K2_IMARK(4);
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk)
+      mma_bf16_ts(tm + ot, tm + TM_SB + 8 * kk, make_sdesc(set + WS_Q + 256 * kk, 128, 2048), id6,
+                  kk > 0);
+    mma_commit(B.bar6);
+    PDN_K2_IMARK(5);
+    // MMA7: O^T += D^T P^T after MMA8
+    if (!k2_wait(B.bar7, (uint32_t)(n & 1), abort_flag)) return false;
+    PDN_K2_IMARK(6);
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk)
+      mma_bf16_ts(tm + ot, tm + TM_DB + 8 * kk, make_sdesc(set + WS_P + 256 * kk, 128, 1024), id7,
+                  1);
+    mma_commit(B.baro);
+    PDN_K2_IMARK(7);
+  }
+  return true;
 }
 
 __global__ void __launch_bounds__(kK2Threads, 1) k2_state(const KParams P, void *ws, int N) {
   extern __shared__ __align__(1024) uint8_t smem[];
   const uint32_t sb = smem_u32(smem);
-  uint64_t *full = reinterpret_cast<uint64_t *>(smem + K2_BAR);
-  uint64_t *bar5 = full + 2, *bar7 = full + 3, *ofree = full + 4;
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + K2_BAR);
+  const K2Bars B{bars, bars + 2, bars + 3, bars + 4, bars + 5, bars + 6, bars + 7};
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + K2_ABORT);
   uint32_t *tbase_p = reinterpret_cast<uint32_t *>(smem + K2_TBASE);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -819,9 +940,9 @@ __global__ void __launch_bounds__(kK2Threads, 1) k2_state(const KParams P, void 
     tmem_relinquish();
   }
   if (tid == 0) {
-    for (int i = 0; i < 4; ++i) mbar_init(full + i, 1);
-    mbar_init(ofree + 0, 4);
-    mbar_init(ofree + 1, 4);
+    for (int i = 0; i < 6; ++i) mbar_init(bars + i, 1);
+    mbar_init(B.sepi, kK2Compute / 32);
+    mbar_init(B.depi, kK2Compute / 32);
     *abort_flag = 0;
     fence_mbarrier_init();
   }
@@ -830,46 +951,57 @@ __global__ void __launch_bounds__(kK2Threads, 1) k2_state(const KParams P, void 
   tc_fence_after();
   const uint32_t tm = *tbase_p;
 
-  if (tid >= kK2Compute) {
-    // ======================= helper warps =======================
-    const bool loader = tid == kK2Compute;
-    if (loader && N > 0) issue_set_load(smem + K2_SET0, ws_block(ws, bh, N, 0), full + 0);
-    if (loader && N > 1) issue_set_load(smem + K2_SET1, ws_block(ws, bh, N, 1), full + 1);
-    for (int n = 0; n < N; ++n) {
-      const int s = n & 1;
-      bool ok = true;
-      if (lane == 0) ok = mbar_wait_bounded(bar7, (uint32_t)(n & 1), kSpin) && !*abort_flag;
-      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-      tc_fence_after();
-      if (!ok) {
-        if (lane == 0) *abort_flag = 1;
-        break;
+  if (warp == kK2SWarp) {
+    // ======================= S warp =======================
+    if (lane == 0 && !k2_issue_s(tm, sb, B, abort_flag, N)) *abort_flag = 1;
+    __syncwarp();
+  } else if (warp == kK2OWarp) {
+    // ======================= O warp =======================
+    if (lane == 0 && !k2_issue_o(tm, sb, B, abort_flag, N)) *abort_flag = 1;
+    __syncwarp();
+  } else if (warp == kK2LoadWarp) {
+    // ======================= load warp =======================
+    if (lane == 0) {
+      if (N > 0) issue_set_load(smem + K2_SET0, ws_block(ws, bh, N, 0), B.full + 0);
+      if (N > 1) issue_set_load(smem + K2_SET1, ws_block(ws, bh, N, 1), B.full + 1);
+      // chunk n's set takes chunk n + 2: the first part once MMA6 of chunk n
+      // is done, the rest once every MMA of chunk n is
+      for (int n = 0; n + 2 < N; ++n) {
+        uint8_t *dst = smem + ((n & 1) ? K2_SET1 : K2_SET0);
+        const uint8_t *src = ws_block(ws, bh, N, n + 2);
+        if (!k2_wait(B.bar6, (uint32_t)(n & 1), abort_flag)) {
+          *abort_flag = 1;
+          break;
+        }
+        issue_set_load_early(dst, src, B.full + (n & 1));
+        PDN_K2_HMARK(0);
+        if (!k2_wait(B.baro, (uint32_t)(n & 1), abort_flag)) {
+          // the barrier still expects the late part: bring it in regardless so
+          // that no copy is left in flight, then stop
+          issue_set_load_late(dst, src, B.full + (n & 1));
+          *abort_flag = 1;
+          break;
+        }
+        issue_set_load_late(dst, src, B.full + (n & 1));
+        PDN_K2_HMARK(1);
       }
-      // chunk n's MMAs are done with operand set s: refill it two chunks ahead
-      if (loader && n + 2 < N) issue_set_load(smem + (s ? K2_SET1 : K2_SET0), ws_block(ws, bh, N, n + 2), full + s);
-      const int pc0 = n * kC;
-      k2_store_o(P, tm + lane_q + (s ? TM_OT1 : TM_OT0), b, h, pc0, min(kC, P.T - pc0), lane, quarter);
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(ofree + s);
     }
+    __syncwarp();
   } else {
     // ======================= compute warps =======================
     const int cg = warp >> 2;          // column group 0..3
     const int j = 32 * quarter + lane; // value channel owned in the epilogues
+    bool ok = true;
     for (int n = 0; n < N; ++n) {
       const int s = n & 1;
       const uint32_t set = s ? K2_SET1 : K2_SET0;
-      const uint32_t ot = s ? TM_OT1 : TM_OT0;
       PDN_K2_MARK(0);
-      {
-        bool ok = true;
-        if (warp == 0) ok = mbar_wait_bounded(full + s, (uint32_t)((n >> 1) & 1), kSpin);
-        if (compute_or(!ok || *abort_flag)) {
-          if (tid == 0) *abort_flag = 1;
-          break;
-        }
-      }
+      // operand set n (its e^{G_C}) has landed; MMA6 of chunk n - 1 is done
+      // reading the bf16 copy of S. (MMA8 of chunk n - 1, which the state
+      // needs, was awaited at the end of the previous iteration.)
+      if (!(ok = k2_warp_wait(B.full + s, (uint32_t)((n >> 1) & 1), abort_flag, lane))) break;
+      PDN_K2_MARK(8);
+      if (n > 0 && !(ok = k2_warp_wait(B.bar6, (uint32_t)((n - 1) & 1), abort_flag, lane))) break;
       PDN_K2_MARK(1);
 
       // ---- state epilogue: S -> bf16 operand; TMEM S <- S Diag(e^{G_C}) ----
@@ -899,14 +1031,18 @@ __global__ void __launch_bounds__(kK2Threads, 1) k2_state(const KParams P, void 
           tmem_ld16(tm + lane_q + TM_S + col0 + 16, sv[1]);
           tmem_wait_ld();
         }
+        {
+          uint32_t pk[16];
+#pragma unroll
+          for (int u = 0; u < 2; ++u)
+#pragma unroll
+            for (int e = 0; e < 8; ++e) pk[8 * u + e] = pack_bf16(sv[u][2 * e], sv[u][2 * e + 1]);
+          tmem_st16u(tm + lane_q + TM_SB + 16 * cg, pk);
+        }
 #pragma unroll
         for (int u = 0; u < 2; ++u) {
           const int col = col0 + 16 * u;
-          float lo[8], hi[8], E[8];
-#pragma unroll
-          for (int e = 0; e < 8; ++e) { lo[e] = sv[u][e]; hi[e] = sv[u][8 + e]; }
-          *reinterpret_cast<uint4 *>(smem + K2_SB + tl128(j, col / 8)) = pack8(lo);
-          *reinterpret_cast<uint4 *>(smem + K2_SB + tl128(j, col / 8 + 1)) = pack8(hi);
+          float E[8];
           ld8f(egc + col, E);
 #pragma unroll
           for (int e = 0; e < 8; ++e) sv[u][e] *= E[e];
@@ -917,86 +1053,43 @@ __global__ void __launch_bounds__(kK2Threads, 1) k2_state(const KParams P, void 
         }
         tmem_wait_st();
       }
-      compute_sync_for_mma();
+      k2_warp_arrive(B.sepi, lane);
       PDN_K2_MARK(2);
-
-      // ---- MMA3: U^T = U^T T^T ; MMA5: D^T = U^T - S Y^T ; MMA6: O^T = S Qh^T ----
-      if (tid == 0) {
-        const uint32_t id3 = make_idesc_bf16(128, 64, true, false);
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          mma_bf16_ss(tm + TM_UD, make_sdesc(sb + set + WS_U + 4096 * kk, 2048, 128),
-                      make_sdesc(sb + set + WS_T + 256 * kk, 128, 1024), id3, kk > 0);
-        const uint32_t id5 = make_idesc_bf16(128, 64, false, true, true);
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_bf16_ss(tm + TM_UD, make_sdesc(sb + K2_SB + 256 * kk, 128, 2048),
-                      make_sdesc(sb + set + WS_Y + 2048 * kk, 1024, 128), id5, 1);
-        mma_commit(bar5);
-        // the helpers must have written out the output buffer chunk n-2 left here
-        bool ok = true;
-        if (n >= 2) ok = mbar_wait_bounded(ofree + s, (uint32_t)(((n - 2) >> 1) & 1), kSpin);
-        if (ok) {
-          const uint32_t id6 = make_idesc_bf16(128, 64, false, false);
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            mma_bf16_ss(tm + ot, make_sdesc(sb + K2_SB + 256 * kk, 128, 2048),
-                        make_sdesc(sb + set + WS_Q + 256 * kk, 128, 2048), id6, kk > 0);
-        } else {
-          *abort_flag = 1;
-        }
+      // chunk n - 1's output, while MMA5 runs (this also frees its TMEM
+      // buffer for chunk n + 1 and D^T's shared tile for this chunk)
+      if (n > 0) {
+        if (!(ok = k2_warp_wait(B.baro, (uint32_t)((n - 1) & 1), abort_flag, lane))) break;
+        PDN_K2_MARK(9);
+        const int pc0 = (n - 1) * kC;
+        k2_store_o(P, tm + lane_q + (s ? TM_OT0 : TM_OT1), b, h, pc0, min(kC, P.T - pc0), lane,
+                   quarter, cg);
       }
       PDN_K2_MARK(3);
-      {
-        bool ok = true;
-        if (warp == 0) ok = mbar_wait_bounded(bar5, (uint32_t)(n & 1), kSpin);
-        const bool stop = compute_or(!ok || *abort_flag);
-        tc_fence_after();
-        if (stop) {
-          if (tid == 0) *abort_flag = 1;
-          break;
-        }
-      }
+      if (!(ok = k2_warp_wait(B.bar5, (uint32_t)(n & 1), abort_flag, lane))) break;
       PDN_K2_MARK(4);
 
-      // ---- D^T -> bf16 operand (rows d_v, columns tokens) ----
+      // ---- D^T -> bf16 operand in TMEM (lanes d_v, token pairs per column) ----
       {
         float v[16];
         tmem_ld16(tm + lane_q + TM_UD + 16 * cg, v);
         tmem_wait_ld();
-        float lo[8], hi[8];
+        uint32_t pk[8];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) { lo[e] = v[e]; hi[e] = v[8 + e]; }
-        *reinterpret_cast<uint4 *>(smem + K2_DT + tl64(j, 2 * cg)) = pack8(lo);
-        *reinterpret_cast<uint4 *>(smem + K2_DT + tl64(j, 2 * cg + 1)) = pack8(hi);
+        for (int e = 0; e < 8; ++e) pk[e] = pack_bf16(v[2 * e], v[2 * e + 1]);
+        tmem_st8u(tm + lane_q + TM_DB + 8 * cg, pk);
+        tmem_wait_st();
       }
-      compute_sync_for_mma();
+      k2_warp_arrive(B.depi, lane);
       PDN_K2_MARK(5);
-
-      // ---- MMA7: O^T += D^T P^T ; MMA8: S += D^T Wb ----
-      if (tid == 0) {
-        const uint32_t id7 = make_idesc_bf16(128, 64, false, false);
-        const uint32_t id8 = make_idesc_bf16(128, 128, false, true);
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-          const uint64_t ad = make_sdesc(sb + K2_DT + 256 * kk, 128, 1024);
-          mma_bf16_ss(tm + ot, ad, make_sdesc(sb + set + WS_P + 256 * kk, 128, 1024), id7, 1);
-          mma_bf16_ss(tm + TM_S, ad, make_sdesc(sb + set + WS_WB + 4096 * kk, 2048, 128), id8, 1);
-        }
-        mma_commit(bar7);
-      }
       PDN_K2_MARK(6);
-      {
-        bool ok = true;
-        if (warp == 0) ok = mbar_wait_bounded(bar7, (uint32_t)(n & 1), kSpin);
-        const bool stop = compute_or(!ok || *abort_flag);
-        tc_fence_after();
-        if (stop) {
-          if (tid == 0) *abort_flag = 1;
-          break;
-        }
-      }
+      if (!(ok = k2_warp_wait(B.bar7, (uint32_t)(n & 1), abort_flag, lane))) break;
       PDN_K2_MARK(7);
+    }
+    // the last chunk's output
+    if (ok && N > 0 && k2_warp_wait(B.baro, (uint32_t)((N - 1) & 1), abort_flag, lane)) {
+      const int pc0 = (N - 1) * kC;
+      k2_store_o(P, tm + lane_q + (((N - 1) & 1) ? TM_OT1 : TM_OT0), b, h, pc0,
+                 min(kC, P.T - pc0), lane, quarter, cg);
     }
     if (!*abort_flag && N > 0 && P.ST) {
       float v[2][16];
@@ -1021,8 +1114,8 @@ __global__ void __launch_bounds__(kK2Threads, 1) k2_state(const KParams P, void 
       record_error(P.err, PDN_ERR_TIMEOUT);
       // drain operand loads still in flight before shared memory goes away
       for (int s2 = 0; s2 < 2; ++s2) {
-        mbar_wait_bounded(full + s2, 0, kSpin);
-        mbar_wait_bounded(full + s2, 1, kSpin);
+        mbar_wait_bounded(B.full + s2, 0, kSpin);
+        mbar_wait_bounded(B.full + s2, 1, kSpin);
       }
     }
     __syncthreads();
