@@ -54,8 +54,10 @@ constexpr uint32_t WS_SET = 82432;  // bytes the state kernel loads per chunk
 constexpr uint32_t WS_A = 82432;    // float[128]: accumulator A at the chunk start
 constexpr size_t WS_CH = 82944;     // bytes per block (256-aligned)
 
-__device__ __forceinline__ uint8_t *ws_block(void *ws, int bh, int N, int c) {
-  return reinterpret_cast<uint8_t *>(ws) + ((size_t)bh * N + c) * WS_CH;
+// Chunk-major: the blocks of one chunk index, over all (batch, head), are
+// adjacent, so the state pass's concurrent loads stream one contiguous range.
+__device__ __forceinline__ uint8_t *ws_block(void *ws, int bh, int BH, int c) {
+  return reinterpret_cast<uint8_t *>(ws) + ((size_t)c * BH + bh) * WS_CH;
 }
 
 constexpr long long kSpin = 1LL << 22;
@@ -98,7 +100,7 @@ __global__ void __launch_bounds__(256) k0_chunk_energy(const KParams P, void *ws
     float s = 0.f;
 #pragma unroll
     for (int r = 0; r < 16; ++r) s += part[r][tid];
-    reinterpret_cast<float *>(ws_block(ws, bh, N, c) + WS_A)[tid] = s;
+    reinterpret_cast<float *>(ws_block(ws, bh, P.B * P.H, c) + WS_A)[tid] = s;
   }
 }
 
@@ -109,10 +111,10 @@ __global__ void __launch_bounds__(kD) k0_prefix(const KParams P, void *ws, int N
     float s[8];
 #pragma unroll
     for (int e = 0; e < 8; ++e)
-      s[e] = (c0 + e < N) ? reinterpret_cast<float *>(ws_block(ws, bh, N, c0 + e) + WS_A)[i] : 0.f;
+      s[e] = (c0 + e < N) ? reinterpret_cast<float *>(ws_block(ws, bh, P.B * P.H, c0 + e) + WS_A)[i] : 0.f;
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
-      if (c0 + e < N) reinterpret_cast<float *>(ws_block(ws, bh, N, c0 + e) + WS_A)[i] = a;
+      if (c0 + e < N) reinterpret_cast<float *>(ws_block(ws, bh, P.B * P.H, c0 + e) + WS_A)[i] = a;
       a += s[e];
     }
   }
@@ -211,7 +213,8 @@ __global__ void __launch_bounds__(kK1Threads, 2) k1_intra(const KParams P, void 
   const float log2x = P.lnx * kLog2e;
   const uint32_t lane_q = (uint32_t)(32 * (warp & 3)) << 16;
   const int half = warp >> 2;
-  const int total = N * P.B * P.H;  // chunk blocks; block index = bh * N + c
+  const int BH = P.B * P.H;
+  const int total = N * BH;  // chunk blocks, chunk-major: block index = c * BH + bh
 
   if (warp == 0) {
     tmem_alloc(tbase_p, 128);
@@ -235,7 +238,7 @@ __global__ void __launch_bounds__(kK1Threads, 2) k1_intra(const KParams P, void 
   };
   auto load_raw = [&](int it) {
     Raw r;
-    const int c_ = it % N, bh_ = it / N;
+    const int c_ = it / BH, bh_ = it % BH;
     const int b_ = bh_ / P.H, h_ = bh_ % P.H;
     const int c0_ = c_ * kC, Cn_ = min(kC, P.T - c0_);
     r.beta = 0.f;
@@ -245,14 +248,14 @@ __global__ void __launch_bounds__(kK1Threads, 2) k1_intra(const KParams P, void 
       if (kScalarBeta) r.beta = __ldg(reinterpret_cast<const float *>(P.beta) + e);
       if (kDecay == PDN_DECAY_SCALAR) r.las = __ldg(reinterpret_cast<const float *>(P.log_alpha) + e);
     }
-    r.acar = (kPre && tid < kD) ? reinterpret_cast<const float *>(ws_block(ws, bh_, N, c_) + WS_A)[tid] : 0.f;
+    r.acar = (kPre && tid < kD) ? reinterpret_cast<const float *>(ws_block(ws, bh_, P.B * P.H, c_) + WS_A)[tid] : 0.f;
     return r;
   };
   // v of a chunk block into the Wh tile's space, rows of 256 bytes with the
   // 16-byte groups XOR-swizzled by (token & 7); issued while the previous
   // block is in its solve (the Wh tile is dead once MMA1 has completed).
   auto stage_v = [&](int it) {
-    const int c_ = it % N, bh_ = it / N;
+    const int c_ = it / BH, bh_ = it % BH;
     const int b_ = bh_ / P.H, h_ = bh_ % P.H;
     const int c0_ = c_ * kC, Cn_ = min(kC, P.T - c0_);
     const size_t tok0_ = tok_index(P, b_, c0_, h_) * kD;
@@ -271,11 +274,11 @@ __global__ void __launch_bounds__(kK1Threads, 2) k1_intra(const KParams P, void 
 
   int iter = 0;
   for (int it = blockIdx.x; it < total; it += gridDim.x, ++iter) {
-  const int c = it % N, bh = it / N;
+  const int c = it / BH, bh = it % BH;
   const int b = bh / P.H, h = bh % P.H;
   const int c0 = c * kC, Cn = min(kC, P.T - c0);
   const size_t tok0 = tok_index(P, b, c0, h) * kD;  // element offset of token c0
-  uint8_t *blk = ws_block(ws, bh, N, c);
+  uint8_t *blk = ws_block(ws, bh, P.B * P.H, c);
   const uint32_t par = (uint32_t)(iter & 1);  // mbarrier parity of this block's MMAs
   PDN_K1_MARK(0);
 
@@ -737,9 +740,10 @@ __global__ void __launch_bounds__(kK1Threads, 2) k1_intra(const KParams P, void 
 // Warp roles. 16 compute warps (TMEM lane quarter x column group) run the
 // epilogues of the state chain and write each chunk's output; the S warp
 // issues the MMAs of the state chain (MMA3, MMA5, MMA8); the O warp issues
-// the output MMAs (MMA6, MMA7); the load warp prefetches operand sets two
-// chunks ahead. They meet only at mbarriers:
-//   full[s]  operand set s landed (bulk copy)
+// the output MMAs (MMA6, MMA7); the load warp prefetches operands. They meet
+// only at mbarriers:
+//   fmain[x] main operand buffer x landed (bulk copy)
+//   fut[x]   U/T operand buffer x landed
 //   sepi     state epilogue of the chunk done (one arrival per compute warp)
 //   depi     D^T epilogue of the chunk done (one arrival per compute warp)
 //   bar5     MMA3 (U~^T) and MMA5 (D^T) done      (S warp)
@@ -751,16 +755,25 @@ __global__ void __launch_bounds__(kK1Threads, 2) k1_intra(const KParams P, void 
 // completed, so the tensor pipe never holds output work ahead of the state
 // chain's. The compute warps write chunk n - 1's output while MMA5 of chunk
 // n runs. The A operands that the epilogues produce (S and D^T in bf16) stay
-// in TMEM; only the B operands are read from shared memory. An operand set is
-// refilled in two parts: Qh, Y^T, U^T and T once MMA6 is done with them,
-// Wb, P and e^{G_C} once the chunk's last MMA is.
+// in TMEM; only the B operands are read from shared memory.
+//
+// A chunk's operands come in two parts: the main part (Qh, Y^T, Wb, P,
+// e^{G_C}) in a ring of three buffers, refilled for chunk n + 3 once every MMA
+// of chunk n is done; U^T and T, which MMA3 reads a chunk early, in a ring of
+// two, refilled for chunk n + 2 once MMA3 of chunk n is done. Every load thus
+// has about two chunk periods to land.
 constexpr int kK2Compute = 512;
 constexpr int kK2SWarp = kK2Compute / 32, kK2OWarp = kK2SWarp + 1, kK2LoadWarp = kK2SWarp + 2;
 constexpr int kK2Threads = kK2Compute + 96;
-constexpr uint32_t K2_SET0 = 0;
-constexpr uint32_t K2_SET1 = WS_SET;
-constexpr uint32_t K2_BAR = 2 * WS_SET;            // the eight mbarriers above
-constexpr uint32_t K2_ABORT = K2_BAR + 8 * 8;
+// main buffer: Qh, Y^T, Wb, then P and e^{G_C} (adjacent in the workspace too)
+constexpr uint32_t KM_Q = 0, KM_Y = 16384, KM_WB = 32768, KM_P = 49152, KM_E = KM_P + (WS_E - WS_P);
+constexpr uint32_t KM_SIZE = KM_P + (WS_SET - WS_P);
+// U/T buffer
+constexpr uint32_t KU_U = 0, KU_T = 16384, KU_SIZE = 16384 + (WS_P - WS_T);
+constexpr uint32_t K2_MAIN = 0;                    // three main buffers
+constexpr uint32_t K2_UT = 3 * KM_SIZE;            // two U/T buffers
+constexpr uint32_t K2_BAR = K2_UT + 2 * KU_SIZE;   // the eleven mbarriers above
+constexpr uint32_t K2_ABORT = K2_BAR + 12 * 8;
 constexpr uint32_t K2_TBASE = K2_ABORT + 8;
 constexpr uint32_t K2_BYTES = K2_TBASE + 16;
 static_assert(K2_BYTES <= 232448, "state kernel shared memory budget");
@@ -769,28 +782,28 @@ static_assert(K2_BYTES <= 232448, "state kernel shared memory budget");
 // (the A operand of MMA5/MMA6), S (fp32), D^T in bf16 pairs (A of MMA7/MMA8).
 constexpr uint32_t TM_UD = 0, TM_OT0 = 64, TM_OT1 = 128, TM_SB = 192, TM_S = 256, TM_DB = 384;
 
-__device__ __forceinline__ void issue_set_load(uint8_t *dst, const uint8_t *src, uint64_t *bar) {
-  mbar_arrive_expect_tx(bar, WS_SET);
-#pragma unroll
-  for (int p = 0; p < 5; ++p) bulk_g2s(dst + p * 16384, src + p * 16384, 16384, bar);
-  bulk_g2s(dst + 81920, src + 81920, WS_SET - 81920, bar);
+static_assert(WS_Q == 0 && WS_Y == 16384 && WS_U == 32768 && WS_WB == 49152 && WS_T == 65536 &&
+                  WS_P == WS_T + 8192 && WS_E > WS_P && WS_SET > WS_E,
+              "workspace block layout the operand loads assume");
+static_assert(K2_MAIN % 128 == 0 && KM_SIZE % 128 == 0 && K2_UT % 128 == 0 && KU_SIZE % 128 == 0,
+              "operand buffers 128-byte aligned");
+
+// Main part of chunk block `src` into main buffer `dst`.
+__device__ __forceinline__ void load_main(uint8_t *dst, const uint8_t *src, uint64_t *bar) {
+  mbar_arrive_expect_tx(bar, KM_SIZE);
+  bulk_g2s(dst + KM_Q, src + WS_Q, 16384, bar);
+  bulk_g2s(dst + KM_Y, src + WS_Y, 16384, bar);
+  bulk_g2s(dst + KM_WB, src + WS_WB, 16384, bar);
+  bulk_g2s(dst + KM_P, src + WS_P, WS_SET - WS_P, bar);
 }
-// The part of a set MMA3, MMA5 and MMA6 read (Qh, Y^T, U^T, T); the barrier
-// expects the whole set, so its phase completes only with the other part.
-__device__ __forceinline__ void issue_set_load_early(uint8_t *dst, const uint8_t *src, uint64_t *bar) {
-  mbar_arrive_expect_tx(bar, WS_SET);
-#pragma unroll
-  for (int p = 0; p < 3; ++p) bulk_g2s(dst + p * 16384, src + p * 16384, 16384, bar);
-  bulk_g2s(dst + WS_T, src + WS_T, WS_P - WS_T, bar);
+// U^T and T of chunk block `src` into U/T buffer `dst`.
+__device__ __forceinline__ void load_ut(uint8_t *dst, const uint8_t *src, uint64_t *bar) {
+  mbar_arrive_expect_tx(bar, KU_SIZE);
+  bulk_g2s(dst + KU_U, src + WS_U, 16384, bar);
+  bulk_g2s(dst + KU_T, src + WS_T, WS_P - WS_T, bar);
 }
-// The rest (Wb, P, e^{G_C}).
-__device__ __forceinline__ void issue_set_load_late(uint8_t *dst, const uint8_t *src, uint64_t *bar) {
-  bulk_g2s(dst + WS_WB, src + WS_WB, WS_T - WS_WB, bar);
-  bulk_g2s(dst + WS_P, src + WS_P, WS_SET - WS_P, bar);
-}
-static_assert(WS_Y == WS_Q + 16384 && WS_U == WS_Y + 16384 && WS_WB == WS_U + 16384 &&
-                  WS_T == WS_WB + 16384 && WS_P > WS_T && WS_E > WS_P && WS_SET > WS_E,
-              "operand set layout the split refill assumes");
+__device__ __forceinline__ uint32_t main_buf(int n) { return K2_MAIN + (uint32_t)(n % 3) * KM_SIZE; }
+__device__ __forceinline__ uint32_t ut_buf(int n) { return K2_UT + (uint32_t)(n & 1) * KU_SIZE; }
 
 // One lane of the warp waits (bounded) on `bar`; the outcome is the warp's.
 // A wait that runs out, or an abort raised elsewhere, sets the abort flag.
@@ -839,17 +852,17 @@ __device__ __forceinline__ void k2_store_o(const KParams &P, uint32_t taddr, int
   }
 }
 
-// MMA3: U~^T = U^T T^T of the chunk whose operand set is at shared address `set`.
-__device__ __forceinline__ void k2_mma3(uint32_t tm, uint32_t set) {
+// MMA3: U~^T = U^T T^T of the chunk whose U/T buffer is at shared address `ut`.
+__device__ __forceinline__ void k2_mma3(uint32_t tm, uint32_t ut) {
   const uint32_t id3 = make_idesc_bf16(128, 64, true, false);
 #pragma unroll
   for (int kk = 0; kk < 4; ++kk)
-    mma_bf16_ss(tm + TM_UD, make_sdesc(set + WS_U + 4096 * kk, 2048, 128),
-                make_sdesc(set + WS_T + 256 * kk, 128, 1024), id3, kk > 0);
+    mma_bf16_ss(tm + TM_UD, make_sdesc(ut + KU_U + 4096 * kk, 2048, 128),
+                make_sdesc(ut + KU_T + 256 * kk, 128, 1024), id3, kk > 0);
 }
 
 struct K2Bars {
-  uint64_t *full, *bar5, *bar6, *bar7, *baro, *sepi, *depi;
+  uint64_t *fmain, *fut, *bar5, *bar6, *bar7, *baro, *sepi, *depi;
 };
 
 // The S warp's program (one lane): MMA3, MMA5, MMA8. False if a wait ran out.
@@ -858,18 +871,17 @@ __device__ __forceinline__ bool k2_issue_s(uint32_t tm, uint32_t sb, const K2Bar
   const uint32_t id5 = make_idesc_bf16(128, 64, false, true, true);
   const uint32_t id8 = make_idesc_bf16(128, 128, false, true);
   for (int n = 0; n < N; ++n) {
-    const int s = n & 1;
-    const uint32_t set = sb + (s ? K2_SET1 : K2_SET0);
+    const uint32_t mb = sb + main_buf(n);
     if (n == 0) {
-      if (!k2_wait(B.full + 0, 0, abort_flag)) return false;
-      k2_mma3(tm, set);
+      if (!k2_wait(B.fut + 0, 0, abort_flag)) return false;
+      k2_mma3(tm, sb + ut_buf(0));
     }
     // MMA5: D^T = U~^T - S Y^T, once the state epilogue has written S (bf16)
     if (!k2_wait(B.sepi, (uint32_t)(n & 1), abort_flag)) return false;
     PDN_K2_IMARK(0);
 #pragma unroll
     for (int kk = 0; kk < 8; ++kk)
-      mma_bf16_ts(tm + TM_UD, tm + TM_SB + 8 * kk, make_sdesc(set + WS_Y + 2048 * kk, 1024, 128),
+      mma_bf16_ts(tm + TM_UD, tm + TM_SB + 8 * kk, make_sdesc(mb + KM_Y + 2048 * kk, 1024, 128),
                   id5, 1);
     mma_commit(B.bar5);
     PDN_K2_IMARK(1);
@@ -878,14 +890,14 @@ __device__ __forceinline__ bool k2_issue_s(uint32_t tm, uint32_t sb, const K2Bar
     PDN_K2_IMARK(2);
 #pragma unroll
     for (int kk = 0; kk < 4; ++kk)
-      mma_bf16_ts(tm + TM_S, tm + TM_DB + 8 * kk, make_sdesc(set + WS_WB + 4096 * kk, 2048, 128),
+      mma_bf16_ts(tm + TM_S, tm + TM_DB + 8 * kk, make_sdesc(mb + KM_WB + 4096 * kk, 2048, 128),
                   id8, 1);
     mma_commit(B.bar7);
     PDN_K2_IMARK(3);
     // MMA3 of chunk n + 1 (the D^T epilogue has read this chunk's U~^T)
     if (n + 1 < N) {
-      if (!k2_wait(B.full + (s ^ 1), (uint32_t)(((n + 1) >> 1) & 1), abort_flag)) return false;
-      k2_mma3(tm, sb + (s ? K2_SET0 : K2_SET1));
+      if (!k2_wait(B.fut + ((n + 1) & 1), (uint32_t)(((n + 1) >> 1) & 1), abort_flag)) return false;
+      k2_mma3(tm, sb + ut_buf(n + 1));
     }
   }
   return true;
@@ -897,16 +909,15 @@ __device__ __forceinline__ bool k2_issue_o(uint32_t tm, uint32_t sb, const K2Bar
   const uint32_t id6 = make_idesc_bf16(128, 64, false, false);
   const uint32_t id7 = make_idesc_bf16(128, 64, false, false);
   for (int n = 0; n < N; ++n) {
-    const int s = n & 1;
-    const uint32_t set = sb + (s ? K2_SET1 : K2_SET0);
-    const uint32_t ot = s ? TM_OT1 : TM_OT0;
+    const uint32_t mb = sb + main_buf(n);
+    const uint32_t ot = (n & 1) ? TM_OT1 : TM_OT0;
     // MMA6: O^T = S Qh^T after MMA5 (which also means the compute warps have
     // written out chunk n - 2's output from this buffer)
     if (!k2_wait(B.bar5, (uint32_t)(n & 1), abort_flag)) return false;
     PDN_K2_IMARK(4);
 #pragma unroll
     for (int kk = 0; kk < 8; ++kk)
-      mma_bf16_ts(tm + ot, tm + TM_SB + 8 * kk, make_sdesc(set + WS_Q + 256 * kk, 128, 2048), id6,
+      mma_bf16_ts(tm + ot, tm + TM_SB + 8 * kk, make_sdesc(mb + KM_Q + 256 * kk, 128, 2048), id6,
                   kk > 0);
     mma_commit(B.bar6);
     PDN_K2_IMARK(5);
@@ -915,7 +926,7 @@ __device__ __forceinline__ bool k2_issue_o(uint32_t tm, uint32_t sb, const K2Bar
     PDN_K2_IMARK(6);
 #pragma unroll
     for (int kk = 0; kk < 4; ++kk)
-      mma_bf16_ts(tm + ot, tm + TM_DB + 8 * kk, make_sdesc(set + WS_P + 256 * kk, 128, 1024), id7,
+      mma_bf16_ts(tm + ot, tm + TM_DB + 8 * kk, make_sdesc(mb + KM_P + 256 * kk, 128, 1024), id7,
                   1);
     mma_commit(B.baro);
     PDN_K2_IMARK(7);
@@ -927,7 +938,7 @@ __global__ void __launch_bounds__(kK2Threads, 1) k2_state(const KParams P, void 
   extern __shared__ __align__(1024) uint8_t smem[];
   const uint32_t sb = smem_u32(smem);
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + K2_BAR);
-  const K2Bars B{bars, bars + 2, bars + 3, bars + 4, bars + 5, bars + 6, bars + 7};
+  const K2Bars B{bars, bars + 3, bars + 5, bars + 6, bars + 7, bars + 8, bars + 9, bars + 10};
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + K2_ABORT);
   uint32_t *tbase_p = reinterpret_cast<uint32_t *>(smem + K2_TBASE);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -940,7 +951,7 @@ __global__ void __launch_bounds__(kK2Threads, 1) k2_state(const KParams P, void 
     tmem_relinquish();
   }
   if (tid == 0) {
-    for (int i = 0; i < 6; ++i) mbar_init(bars + i, 1);
+    for (int i = 0; i < 9; ++i) mbar_init(bars + i, 1);
     mbar_init(B.sepi, kK2Compute / 32);
     mbar_init(B.depi, kK2Compute / 32);
     *abort_flag = 0;
@@ -962,28 +973,28 @@ __global__ void __launch_bounds__(kK2Threads, 1) k2_state(const KParams P, void 
   } else if (warp == kK2LoadWarp) {
     // ======================= load warp =======================
     if (lane == 0) {
-      if (N > 0) issue_set_load(smem + K2_SET0, ws_block(ws, bh, N, 0), B.full + 0);
-      if (N > 1) issue_set_load(smem + K2_SET1, ws_block(ws, bh, N, 1), B.full + 1);
-      // chunk n's set takes chunk n + 2: the first part once MMA6 of chunk n
-      // is done, the rest once every MMA of chunk n is
+      const int BH = P.B * P.H;
+      for (int m = 0; m < 3 && m < N; ++m)
+        load_main(smem + main_buf(m), ws_block(ws, bh, BH, m), B.fmain + m);
+      for (int m = 0; m < 2 && m < N; ++m)
+        load_ut(smem + ut_buf(m), ws_block(ws, bh, BH, m), B.fut + m);
+      // after MMA3 of chunk n (bar5), its U/T buffer takes chunk n + 2; after
+      // every MMA of chunk n (baro), its main buffer takes chunk n + 3
       for (int n = 0; n + 2 < N; ++n) {
-        uint8_t *dst = smem + ((n & 1) ? K2_SET1 : K2_SET0);
-        const uint8_t *src = ws_block(ws, bh, N, n + 2);
-        if (!k2_wait(B.bar6, (uint32_t)(n & 1), abort_flag)) {
+        if (!k2_wait(B.bar5, (uint32_t)(n & 1), abort_flag)) {
           *abort_flag = 1;
           break;
         }
-        issue_set_load_early(dst, src, B.full + (n & 1));
+        load_ut(smem + ut_buf(n), ws_block(ws, bh, BH, n + 2), B.fut + (n & 1));
         PDN_K2_HMARK(0);
-        if (!k2_wait(B.baro, (uint32_t)(n & 1), abort_flag)) {
-          // the barrier still expects the late part: bring it in regardless so
-          // that no copy is left in flight, then stop
-          issue_set_load_late(dst, src, B.full + (n & 1));
-          *abort_flag = 1;
-          break;
+        if (n + 3 < N) {
+          if (!k2_wait(B.baro, (uint32_t)(n & 1), abort_flag)) {
+            *abort_flag = 1;
+            break;
+          }
+          load_main(smem + main_buf(n), ws_block(ws, bh, BH, n + 3), B.fmain + (n % 3));
+          PDN_K2_HMARK(1);
         }
-        issue_set_load_late(dst, src, B.full + (n & 1));
-        PDN_K2_HMARK(1);
       }
     }
     __syncwarp();
@@ -994,19 +1005,18 @@ __global__ void __launch_bounds__(kK2Threads, 1) k2_state(const KParams P, void 
     bool ok = true;
     for (int n = 0; n < N; ++n) {
       const int s = n & 1;
-      const uint32_t set = s ? K2_SET1 : K2_SET0;
       PDN_K2_MARK(0);
-      // operand set n (its e^{G_C}) has landed; MMA6 of chunk n - 1 is done
-      // reading the bf16 copy of S. (MMA8 of chunk n - 1, which the state
-      // needs, was awaited at the end of the previous iteration.)
-      if (!(ok = k2_warp_wait(B.full + s, (uint32_t)((n >> 1) & 1), abort_flag, lane))) break;
+      // chunk n's main operands (its e^{G_C}) have landed; MMA6 of chunk n - 1
+      // is done reading the bf16 copy of S. (MMA8 of chunk n - 1, which the
+      // state needs, was awaited at the end of the previous iteration.)
+      if (!(ok = k2_warp_wait(B.fmain + (n % 3), (uint32_t)((n / 3) & 1), abort_flag, lane))) break;
       PDN_K2_MARK(8);
       if (n > 0 && !(ok = k2_warp_wait(B.bar6, (uint32_t)((n - 1) & 1), abort_flag, lane))) break;
       PDN_K2_MARK(1);
 
       // ---- state epilogue: S -> bf16 operand; TMEM S <- S Diag(e^{G_C}) ----
       {
-        const float *egc = reinterpret_cast<const float *>(smem + set + WS_E);
+        const float *egc = reinterpret_cast<const float *>(smem + main_buf(n) + KM_E);
         float sv[2][16];
         const int col0 = 32 * cg;
         if (n == 0) {
@@ -1113,9 +1123,9 @@ __global__ void __launch_bounds__(kK2Threads, 1) k2_state(const KParams P, void 
     if (tid == 0) {
       record_error(P.err, PDN_ERR_TIMEOUT);
       // drain operand loads still in flight before shared memory goes away
-      for (int s2 = 0; s2 < 2; ++s2) {
-        mbar_wait_bounded(B.full + s2, 0, kSpin);
-        mbar_wait_bounded(B.full + s2, 1, kSpin);
+      for (int x = 0; x < 5; ++x) {
+        mbar_wait_bounded(bars + x, 0, kSpin);
+        mbar_wait_bounded(bars + x, 1, kSpin);
       }
     }
     __syncthreads();
