@@ -93,8 +93,10 @@ def traffic_for(kernel_key, files):
     return d.get("bytes_per_launch")
 
 
-CHUNK_SOURCES = ["linear_recurrence_sequence_chunked_b200/csrc/chunk_tc.cu",
-                 "linear_recurrence_sequence_chunked_b200/csrc/chunk_simt.cu",
+# Sources of the kernels one pdn_chunk_fwd call launches on the d = 128 bf16
+# workloads (the three-kernel tensor-core path that automatic selection picks).
+CHUNK_SOURCES = ["linear_recurrence_sequence_chunked_b200/csrc/chunk_split.cu",
+                 "linear_recurrence_sequence_chunked_b200/csrc/tiles.cuh",
                  "linear_recurrence_sequence_chunked_b200/csrc/common.cuh",
                  "linear_recurrence_sequence_chunked_b200/csrc/ptx.cuh"]
 DECODE_SOURCES = ["linear_recurrence_sequence_chunked_b200/csrc/decode.cu",
@@ -301,7 +303,7 @@ def run_ours(args):
         raise SystemExit("device error during the timed region")
     impl_id = pdn.pdn_chunk_fwd_impl(prob)
     tc = impl_id in (pdn.IMPLS["tc"], pdn.IMPLS["tc_fused"])
-    kernel_name = {1: "simt", 2: "tcgen05 split (K0 prefix, K1 intra, K2 state)",
+    kernel_name = {1: "simt", 2: "tcgen05 split (K0 key energy + prefix, K1 intra-chunk, K2 state)",
                    3: "tcgen05 fused"}.get(impl_id, "?")
     launches_per_step = 1
     if impl_id == pdn.IMPLS["tc"]:
@@ -321,6 +323,8 @@ def run_ours(args):
                    "parallelism": "dp%d" % world},
         "roofline": {"bound": "tensor", "achieved": ach_tflops, "peak": peak, "unit": "TFLOP/s",
                      "frac": ach_tflops / peak, "peak_kind": peaks_kind + " bf16 burst",
+                     "launch": "one pdn_chunk_fwd call (%d kernels), CUDA events on its stream"
+                               % launches_per_step,
                      "flops_per_launch": flops,
                      "traffic": traffic_for("chunk_fwd:" + w.name, CHUNK_SOURCES)},
         "clocks": clocks,

@@ -269,8 +269,28 @@ __global__ void __launch_bounds__(kK1Threads, 2) k1_intra(const KParams P, void 
     }
     cp_async_commit();
   };
+  // k of a chunk block into the Rh half of the [Rh; Qh] tile's space (same
+  // swizzled rows); issued once MMA2 of the previous block has read Rh.
+  auto stage_k = [&](int it) {
+    const int c_ = it / BH, bh_ = it % BH;
+    const int b_ = bh_ / P.H, h_ = bh_ % P.H;
+    const int c0_ = c_ * kC, Cn_ = min(kC, P.T - c0_);
+    const size_t tok0_ = tok_index(P, b_, c0_, h_) * kD;
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+      const int t = (tid >> 4) + 16 * m, c8 = tid & 15;
+      const bool ok = t < Cn_;
+      const size_t e = ok ? tok0_ + (size_t)t * tstride + c8 * 8 : 0;
+      cp_async16(sb + K1_RQ + t * 256 + ((c8 ^ (t & 7)) << 4),
+                 reinterpret_cast<const __nv_bfloat16 *>(P.k) + e, ok);
+    }
+    cp_async_commit();
+  };
   Raw pf = load_raw(blockIdx.x < total ? blockIdx.x : 0);
-  if (blockIdx.x < total) stage_v(blockIdx.x);
+  if (blockIdx.x < total) {
+    stage_v(blockIdx.x);
+    stage_k(blockIdx.x);
+  }
 
   int iter = 0;
   for (int it = blockIdx.x; it < total; it += gridDim.x, ++iter) {
@@ -282,17 +302,21 @@ __global__ void __launch_bounds__(kK1Threads, 2) k1_intra(const KParams P, void 
   const uint32_t par = (uint32_t)(iter & 1);  // mbarrier parity of this block's MMAs
   PDN_K1_MARK(0);
 
-  // ---- P0: k, q (and the channel log decay) by cp.async; the prefetched
+  // ---- P0: k (staged a block ahead) into its padded rows; q (and the
+  // channel log decay) by cp.async, q awaited only before P3; the prefetched
   // scalars into shared memory; then start loading the next block's ----
   uint4 vcur[4];
+  cp_async_wait_all();  // this block's k and v
+  __syncthreads();
   {
 #pragma unroll
     for (int m = 0; m < 4; ++m) {
       const int t = (tid >> 4) + 16 * m, c8 = tid & 15;
+      *reinterpret_cast<uint4 *>(smem + K1_KS + t * KS_LD + c8 * 16) =
+          *reinterpret_cast<const uint4 *>(smem + K1_RQ + t * 256 + ((c8 ^ (t & 7)) << 4));
       {
         const bool ok = t < Cn;
         const size_t e = ok ? tok0 + (size_t)t * tstride + c8 * 8 : 0;
-        cp_async16(sb + K1_KS + t * KS_LD + c8 * 16, reinterpret_cast<const __nv_bfloat16 *>(P.k) + e, ok);
         cp_async16(sb + K1_QS + t * KS_LD + c8 * 16, reinterpret_cast<const __nv_bfloat16 *>(P.q) + e, ok);
       }
       if (kDecay == PDN_DECAY_CHANNEL) {
@@ -310,7 +334,7 @@ __global__ void __launch_bounds__(kK1Threads, 2) k1_intra(const KParams P, void 
     if (tid < kD) Acar[tid] = pf.acar;
   }
   if (it + (int)gridDim.x < total) pf = load_raw(it + gridDim.x);
-  cp_async_wait_all();
+  if (kDecay == PDN_DECAY_CHANNEL) cp_async_wait_all();  // P1 scans the channel log decay
   __syncthreads();
   PDN_K1_MARK(1);
 
@@ -391,12 +415,13 @@ __global__ void __launch_bounds__(kK1Threads, 2) k1_intra(const KParams P, void 
     }
   }
   // this block's v into registers (operand mapping) before P3 overwrites the
-  // staging space with the Wh tile
+  // staging space with the Wh tile; q has landed
 #pragma unroll
   for (int m = 0; m < 4; ++m) {
     const int t = 8 * warp + (lane & 7), c8 = 4 * m + (lane >> 3);
     vcur[m] = *reinterpret_cast<const uint4 *>(smem + K1_WH + t * 256 + ((c8 ^ (t & 7)) << 4));
   }
+  cp_async_wait_all();
   __syncthreads();
   PDN_K1_MARK(2);
   PDN_K1_MARK(3);
@@ -690,6 +715,8 @@ __global__ void __launch_bounds__(kK1Threads, 2) k1_intra(const KParams P, void 
     }
     PDN_K1_MARK(9);
     if (ok_all) {
+      // Rh is dead: the next block's k goes into its space
+      if (it + (int)gridDim.x < total) stage_k(it + gridDim.x);
       // Y^T -> bf16 tile (rows d_k, columns tokens)
       const int i = 32 * (warp & 3) + lane;
 #pragma unroll
@@ -714,7 +741,7 @@ __global__ void __launch_bounds__(kK1Threads, 2) k1_intra(const KParams P, void 
         bulk_s2g(blk + WS_T, smem + K1_TM, 8192);
         bulk_s2g(blk + WS_P, smem + K1_PM, 8192);
         bulk_commit();
-        bulk_wait0();
+        bulk_wait_read0();  // the tiles may be rewritten; the writes land on their own
       }
     }
   }
@@ -728,6 +755,8 @@ __global__ void __launch_bounds__(kK1Threads, 2) k1_intra(const KParams P, void 
   __syncthreads();
   tc_fence_after();
   }  // chunk blocks
+  if (tid == 0) bulk_wait0();
+  cp_async_wait_all();  // a prefetch issued before an abort
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
