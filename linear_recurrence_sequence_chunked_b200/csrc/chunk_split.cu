@@ -155,12 +155,13 @@ struct K1Layout {
       kDecay == PDN_DECAY_CHANNEL ? K1_LAS_STAGE + 64 * 256 : K1_GBUF;
   static constexpr uint32_t kSmall = (kPrepEnd > K1_SOLVE_END ? kPrepEnd : K1_SOLVE_END);
   static constexpr uint32_t kAcar = kSmall, kGC = kSmall + 512, kEGC = kSmall + 1024;
-  static constexpr uint32_t kPartK = kSmall + 1536, kPartG = kSmall + 2048;
-  static constexpr uint32_t kMup = kSmall + 2560;  // float[4][64] per-warp partial means
-  static constexpr uint32_t kMu = kSmall + 3584, kBeta = kSmall + 3840, kGS = kSmall + 4096;
-  static constexpr uint32_t kLas = kSmall + 4352, kBar = kSmall + 4608;
-  static constexpr uint32_t kTbase = kSmall + 4624;
-  static constexpr uint32_t kBytes = kSmall + 4640;
+  // float[3][128]: sums over token quarters 0..2 of k.k and of the log decay
+  static constexpr uint32_t kPartK = kSmall + 1536, kPartG = kSmall + 3072;
+  static constexpr uint32_t kMup = kSmall + 4608;  // float[2][64] per channel-half partial means
+  static constexpr uint32_t kMu = kSmall + 5120, kBeta = kSmall + 5376, kGS = kSmall + 5632;
+  static constexpr uint32_t kLas = kSmall + 5888, kBar = kSmall + 6144;
+  static constexpr uint32_t kTbase = kSmall + 6160;
+  static constexpr uint32_t kBytes = kSmall + 6176;
 };
 
 // 2^z for |z| < 1 on the FMA pipe: with y = z ln2 / 2, e^y by its Taylor
@@ -338,60 +339,94 @@ __global__ void __launch_bounds__(kK1Threads, 2) k1_intra(const KParams P, void 
   __syncthreads();
   PDN_K1_MARK(1);
 
-  // ---- P1: per-channel scans; thread = (channel, half of the chunk) ----
+  // ---- P1: per-channel scans; thread = (channel pair, quarter of the chunk) ----
   // Prefix sums of k.k (accumulator) and of the log decay over the chunk's
   // tokens, then (preconditioned variants) the per-token channel mean of
   // log2(A + eps) by a warp transpose-reduce, and B = x^(-s) per element.
   {
-    const int i = tid & 127, hf = tid >> 7, t0 = 32 * hf;
-    float kk[32], la[32];
-    float ks = 0.f, gs = 0.f;
+    const int p = tid & 63, q4 = tid >> 6, t0 = 16 * q4;  // channels 2p, 2p + 1; tokens t0 ..
+    const int i0 = 2 * p;
+    float k0[16], k1[16], l0[16], l1[16];
+    float ks0 = 0.f, ks1 = 0.f, gs0 = 0.f, gs1 = 0.f;
 #pragma unroll
-    for (int e = 0; e < 32; ++e) {
+    for (int e = 0; e < 16; ++e) {
       const int t = t0 + e;
-      kk[e] = kPre ? __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(
-                         smem + K1_KS + t * KS_LD + i * 2))
-                   : 0.f;
-      if (kDecay == PDN_DECAY_CHANNEL)
-        la[e] = __bfloat162float(
-            *reinterpret_cast<const __nv_bfloat16 *>(smem + K1_LAS_STAGE + t * 256 + i * 2));
-      else if (kDecay == PDN_DECAY_SCALAR)
-        la[e] = LAS[t];
-      else
-        la[e] = 0.f;
-      ks = fmaf(kk[e], kk[e], ks);
-      gs += la[e];
+      if (kPre) {
+        const float2 kv = __bfloat1622float2(
+            *reinterpret_cast<const __nv_bfloat162 *>(smem + K1_KS + t * KS_LD + i0 * 2));
+        k0[e] = kv.x;
+        k1[e] = kv.y;
+      } else {
+        k0[e] = 0.f;
+        k1[e] = 0.f;
+      }
+      if (kDecay == PDN_DECAY_CHANNEL) {
+        const float2 lv = __bfloat1622float2(
+            *reinterpret_cast<const __nv_bfloat162 *>(smem + K1_LAS_STAGE + t * 256 + i0 * 2));
+        l0[e] = lv.x;
+        l1[e] = lv.y;
+      } else if (kDecay == PDN_DECAY_SCALAR) {
+        l0[e] = LAS[t];
+        l1[e] = l0[e];
+      } else {
+        l0[e] = 0.f;
+        l1[e] = 0.f;
+      }
+      ks0 = fmaf(k0[e], k0[e], ks0);
+      ks1 = fmaf(k1[e], k1[e], ks1);
+      gs0 += l0[e];
+      gs1 += l1[e];
     }
-    if (hf == 0) {
-      PARTK[i] = ks;
-      PARTG[i] = gs;
+    if (q4 < 3) {
+      *reinterpret_cast<float2 *>(PARTK + q4 * kD + i0) = make_float2(ks0, ks1);
+      *reinterpret_cast<float2 *>(PARTG + q4 * kD + i0) = make_float2(gs0, gs1);
     }
     __syncthreads();
-    float a = Acar[i] + (hf ? PARTK[i] : 0.f);
-    float g = hf ? PARTG[i] : 0.f;
+    float a0 = Acar[i0], a1 = Acar[i0 + 1], g0 = 0.f, g1 = 0.f;
 #pragma unroll
-    for (int e = 0; e < 32; ++e) {
-      const int t = t0 + e;
-      a = fmaf(kk[e], kk[e], a);
-      kk[e] = kPre ? lg2_approx(a + P.eps) : 0.f;  // kk now holds log2(A_t + eps)
-      g += la[e];
-      if (kDecay == PDN_DECAY_CHANNEL) GBUF[t * LB_LD + i] = g;
-      else if (kDecay == PDN_DECAY_SCALAR && i == 0) GS[t] = g;
+    for (int r = 0; r < 3; ++r) {
+      if (r < q4) {
+        const float2 pk = *reinterpret_cast<const float2 *>(PARTK + r * kD + i0);
+        const float2 pg = *reinterpret_cast<const float2 *>(PARTG + r * kD + i0);
+        a0 += pk.x;
+        a1 += pk.y;
+        g0 += pg.x;
+        g1 += pg.y;
+      }
     }
-    if (hf) {
-      GC[i] = g;
-      const float eg = ex2_approx(fmaxf(g, kMinG) * kLog2e);
-      EGC[i] = eg;
-      reinterpret_cast<float *>(blk + WS_E)[i] = eg;
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+      const int t = t0 + e;
+      a0 = fmaf(k0[e], k0[e], a0);
+      a1 = fmaf(k1[e], k1[e], a1);
+      if (kPre) {  // k0, k1 now hold log2(A_t + eps)
+        k0[e] = lg2_approx(a0 + P.eps);
+        k1[e] = lg2_approx(a1 + P.eps);
+      }
+      g0 += l0[e];
+      g1 += l1[e];
+      if (kDecay == PDN_DECAY_CHANNEL)
+        *reinterpret_cast<float2 *>(GBUF + t * LB_LD + i0) = make_float2(g0, g1);
+      else if (kDecay == PDN_DECAY_SCALAR && p == 0)
+        GS[t] = g0;
+    }
+    if (q4 == 3) {
+      GC[i0] = g0;
+      GC[i0 + 1] = g1;
+      const float e0 = ex2_approx(fmaxf(g0, kMinG) * kLog2e);
+      const float e1 = ex2_approx(fmaxf(g1, kMinG) * kLog2e);
+      EGC[i0] = e0;
+      EGC[i0 + 1] = e1;
+      *reinterpret_cast<float2 *>(reinterpret_cast<float *>(blk + WS_E) + i0) = make_float2(e0, e1);
     }
     if (kPre) {
-      // transpose-reduce: after 5 butterfly steps lane l holds the sum over
-      // the warp's 32 channels of token t0 + l
-      float v[32];
+      // transpose-reduce over the warp's 64 channels: four butterfly steps
+      // leave lanes l and l ^ 1 with halves of the sum for token t0 + (l >> 1)
+      float v[16];
 #pragma unroll
-      for (int e = 0; e < 32; ++e) v[e] = kk[e];
+      for (int e = 0; e < 16; ++e) v[e] = k0[e] + k1[e];
 #pragma unroll
-      for (int off = 16, len = 16; off >= 1; off >>= 1, len >>= 1) {
+      for (int off = 16, len = 8; off >= 2; off >>= 1, len >>= 1) {
         const bool upper = (lane & off) != 0;
 #pragma unroll
         for (int e = 0; e < len; ++e) {
@@ -400,17 +435,21 @@ __global__ void __launch_bounds__(kK1Threads, 2) k1_intra(const KParams P, void 
           v[e] = keep + __shfl_xor_sync(0xffffffffu, send, off);
         }
       }
-      MUP[(warp & 3) * 64 + t0 + lane] = v[0];
+      v[0] += __shfl_xor_sync(0xffffffffu, v[0], 1);
+      if ((lane & 1) == 0) MUP[(warp & 1) * 64 + t0 + (lane >> 1)] = v[0];
       __syncthreads();
-      if (tid < kC) MU[tid] = (MUP[tid] + MUP[64 + tid] + MUP[128 + tid] + MUP[192 + tid]) * (1.f / kD);
+      if (tid < kC) MU[tid] = (MUP[tid] + MUP[64 + tid]) * (1.f / kD);
       __syncthreads();
       const float log2x_ = log2x;
 #pragma unroll
-      for (int e = 0; e < 32; ++e) {
-        const float cc = (kk[e] - MU[t0 + e]) * kLn2;
-        const float sq = cc * rcp_approx(1.f + fabsf(cc));
-        *reinterpret_cast<__nv_bfloat16 *>(smem + K1_BC + (t0 + e) * KS_LD + i * 2) =
-            __float2bfloat16_rn(exp2_small(-sq * log2x_));
+      for (int e = 0; e < 16; ++e) {
+        const int t = t0 + e;
+        const float mu = MU[t];
+        const float c0 = (k0[e] - mu) * kLn2, c1 = (k1[e] - mu) * kLn2;
+        const float s0 = c0 * rcp_approx(1.f + fabsf(c0));
+        const float s1 = c1 * rcp_approx(1.f + fabsf(c1));
+        *reinterpret_cast<uint32_t *>(smem + K1_BC + t * KS_LD + i0 * 2) =
+            pack_bf16(exp2_small(-s0 * log2x_), exp2_small(-s1 * log2x_));
       }
     }
   }
