@@ -4,12 +4,12 @@
 //
 //   K0  key-energy prefix: A at the start of every chunk (preconditioned
 //       variants; "Preconditioned DeltaNet", fr §2.B: A_t = A_{t-1} + k.k)
-//   K1  one CTA per (batch, head, chunk): gates and preconditioner, M and P
-//       (MMA), T = (I + M)^{-1}, Y^T = Rh^T T^T (MMA); writes bf16 operand
-//       tiles of the chunk to the workspace in the shared-memory image the
-//       state kernel's MMAs consume
-//   K2  one CTA per (batch, head): per chunk, bulk-loads those tiles one chunk
-//       ahead, U^T = U^T T^T, D^T = U^T - S Y^T, O^T = S Qh^T + D^T P^T,
+//   K1  persistent, two CTAs per SM walking the (chunk, batch, head) blocks:
+//       gates and preconditioner, M and P (MMA), T = (I + M)^{-1},
+//       Y^T = Rh^T T^T (MMA); writes bf16 operand tiles of the chunk to the
+//       workspace in the shared-memory image the state kernel's MMAs consume
+//   K2  one CTA per (batch, head): per chunk, bulk-loads those tiles two
+//       chunks ahead, U^T = U^T T^T, D^T = U^T - S Y^T, O^T = S Qh^T + D^T P^T,
 //       S <- S Diag(e^{G_C}) + D^T Wb; fp32 state in tensor memory
 //
 // Same chunk algebra as the single-kernel path ("Gated DeltaNet-2", ja §3:
