@@ -35,6 +35,9 @@
 #ifndef PDN_K2_HMARK
 #define PDN_K2_HMARK(k)
 #endif
+#ifndef PDN_K2_WMARK
+#define PDN_K2_WMARK(k)
+#endif
 
 namespace pdn {
 namespace {
@@ -163,20 +166,6 @@ struct K1Layout {
   static constexpr uint32_t kTbase = kSmall + 6160;
   static constexpr uint32_t kBytes = kSmall + 6176;
 };
-
-// 2^z for |z| < 1 on the FMA pipe: with y = z ln2 / 2, e^y by its Taylor
-// series to degree 6 (remainder below 1.3e-7 for |y| < 0.35), squared.
-__device__ __forceinline__ float exp2_small(float z) {
-  const float y = z * 0.34657359027997264f;
-  float p = 1.3888888888888889e-3f;   // 1/720
-  p = fmaf(p, y, 8.3333333333333333e-3f);  // 1/120
-  p = fmaf(p, y, 4.1666666666666667e-2f);  // 1/24
-  p = fmaf(p, y, 1.6666666666666667e-1f);  // 1/6
-  p = fmaf(p, y, 0.5f);
-  p = fmaf(p, y, 1.0f);
-  p = fmaf(p, y, 1.0f);
-  return p * p;
-}
 
 __device__ __forceinline__ void sync_for_mma() {
   fence_proxy_async_smem();
@@ -449,7 +438,7 @@ __global__ void __launch_bounds__(kK1Threads, 2) k1_intra(const KParams P, void 
         const float s0 = c0 * rcp_approx(1.f + fabsf(c0));
         const float s1 = c1 * rcp_approx(1.f + fabsf(c1));
         *reinterpret_cast<uint32_t *>(smem + K1_BC + t * KS_LD + i0 * 2) =
-            pack_bf16(exp2_small(-s0 * log2x_), exp2_small(-s1 * log2x_));
+            pack_bf16(ex2_approx(-s0 * log2x_), ex2_approx(-s1 * log2x_));
       }
     }
   }
@@ -816,7 +805,6 @@ __global__ void __launch_bounds__(kK1Threads, 2) k1_intra(const KParams P, void 
 //   depi     D^T epilogue of the chunk done (one arrival per compute warp)
 //   bar5     MMA3 (U~^T) and MMA5 (D^T) done      (S warp)
 //   bar7     MMA8 (state update) done             (S warp)
-//   bar6     MMA6 (O^T = S Qh^T) done              (O warp)
 //   baro     MMA7 (O^T += D^T P^T) done: the chunk's output and, since the O
 //            warp waits on bar7 first, every MMA of the chunk
 // The O warp issues MMA6 only after MMA5 and MMA7 only after MMA8 have
@@ -840,15 +828,20 @@ constexpr uint32_t KM_SIZE = KM_P + (WS_SET - WS_P);
 constexpr uint32_t KU_U = 0, KU_T = 16384, KU_SIZE = 16384 + (WS_P - WS_T);
 constexpr uint32_t K2_MAIN = 0;                    // three main buffers
 constexpr uint32_t K2_UT = 3 * KM_SIZE;            // two U/T buffers
-constexpr uint32_t K2_BAR = K2_UT + 2 * KU_SIZE;   // the eleven mbarriers above
+constexpr uint32_t K2_BAR = K2_UT + 2 * KU_SIZE;   // the ten mbarriers above
 constexpr uint32_t K2_ABORT = K2_BAR + 12 * 8;
 constexpr uint32_t K2_TBASE = K2_ABORT + 8;
 constexpr uint32_t K2_BYTES = K2_TBASE + 16;
 static_assert(K2_BYTES <= 232448, "state kernel shared memory budget");
 
 // TMEM columns: U~^T then D^T (fp32), the two O^T buffers, S in bf16 pairs
-// (the A operand of MMA5/MMA6), S (fp32), D^T in bf16 pairs (A of MMA7/MMA8).
-constexpr uint32_t TM_UD = 0, TM_OT0 = 64, TM_OT1 = 128, TM_SB = 192, TM_S = 256, TM_DB = 384;
+// (the A operand of MMA5/MMA6), S (fp32), D^T in bf16 pairs (A of MMA7/MMA8);
+// the bf16 operands have two buffers each, by chunk parity, so that a chunk's
+// epilogues never wait for the previous chunk's output MMAs.
+constexpr uint32_t TM_UD = 0, TM_OT0 = 64, TM_OT1 = 128, TM_SB0 = 192, TM_S = 256, TM_DB0 = 384,
+                   TM_DB1 = 416, TM_SB1 = 448;
+__device__ __forceinline__ uint32_t tm_sb(int n) { return (n & 1) ? TM_SB1 : TM_SB0; }
+__device__ __forceinline__ uint32_t tm_db(int n) { return (n & 1) ? TM_DB1 : TM_DB0; }
 
 static_assert(WS_Q == 0 && WS_Y == 16384 && WS_U == 32768 && WS_WB == 49152 && WS_T == 65536 &&
                   WS_P == WS_T + 8192 && WS_E > WS_P && WS_SET > WS_E,
@@ -930,7 +923,7 @@ __device__ __forceinline__ void k2_mma3(uint32_t tm, uint32_t ut) {
 }
 
 struct K2Bars {
-  uint64_t *fmain, *fut, *bar5, *bar6, *bar7, *baro, *sepi, *depi;
+  uint64_t *fmain, *fut, *bar5, *bar7, *baro, *sepi, *depi;
 };
 
 // The S warp's program (one lane): MMA3, MMA5, MMA8. False if a wait ran out.
@@ -949,7 +942,7 @@ __device__ __forceinline__ bool k2_issue_s(uint32_t tm, uint32_t sb, const K2Bar
     PDN_K2_IMARK(0);
 #pragma unroll
     for (int kk = 0; kk < 8; ++kk)
-      mma_bf16_ts(tm + TM_UD, tm + TM_SB + 8 * kk, make_sdesc(mb + KM_Y + 2048 * kk, 1024, 128),
+      mma_bf16_ts(tm + TM_UD, tm + tm_sb(n) + 8 * kk, make_sdesc(mb + KM_Y + 2048 * kk, 1024, 128),
                   id5, 1);
     mma_commit(B.bar5);
     PDN_K2_IMARK(1);
@@ -958,7 +951,7 @@ __device__ __forceinline__ bool k2_issue_s(uint32_t tm, uint32_t sb, const K2Bar
     PDN_K2_IMARK(2);
 #pragma unroll
     for (int kk = 0; kk < 4; ++kk)
-      mma_bf16_ts(tm + TM_S, tm + TM_DB + 8 * kk, make_sdesc(mb + KM_WB + 4096 * kk, 2048, 128),
+      mma_bf16_ts(tm + TM_S, tm + tm_db(n) + 8 * kk, make_sdesc(mb + KM_WB + 4096 * kk, 2048, 128),
                   id8, 1);
     mma_commit(B.bar7);
     PDN_K2_IMARK(3);
@@ -985,16 +978,15 @@ __device__ __forceinline__ bool k2_issue_o(uint32_t tm, uint32_t sb, const K2Bar
     PDN_K2_IMARK(4);
 #pragma unroll
     for (int kk = 0; kk < 8; ++kk)
-      mma_bf16_ts(tm + ot, tm + TM_SB + 8 * kk, make_sdesc(mb + KM_Q + 256 * kk, 128, 2048), id6,
+      mma_bf16_ts(tm + ot, tm + tm_sb(n) + 8 * kk, make_sdesc(mb + KM_Q + 256 * kk, 128, 2048), id6,
                   kk > 0);
-    mma_commit(B.bar6);
     PDN_K2_IMARK(5);
     // MMA7: O^T += D^T P^T after MMA8
     if (!k2_wait(B.bar7, (uint32_t)(n & 1), abort_flag)) return false;
     PDN_K2_IMARK(6);
 #pragma unroll
     for (int kk = 0; kk < 4; ++kk)
-      mma_bf16_ts(tm + ot, tm + TM_DB + 8 * kk, make_sdesc(mb + KM_P + 256 * kk, 128, 1024), id7,
+      mma_bf16_ts(tm + ot, tm + tm_db(n) + 8 * kk, make_sdesc(mb + KM_P + 256 * kk, 128, 1024), id7,
                   1);
     mma_commit(B.baro);
     PDN_K2_IMARK(7);
@@ -1006,7 +998,7 @@ __global__ void __launch_bounds__(kK2Threads, 1) k2_state(const KParams P, void 
   extern __shared__ __align__(1024) uint8_t smem[];
   const uint32_t sb = smem_u32(smem);
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + K2_BAR);
-  const K2Bars B{bars, bars + 3, bars + 5, bars + 6, bars + 7, bars + 8, bars + 9, bars + 10};
+  const K2Bars B{bars, bars + 3, bars + 5, bars + 6, bars + 7, bars + 8, bars + 9};
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + K2_ABORT);
   uint32_t *tbase_p = reinterpret_cast<uint32_t *>(smem + K2_TBASE);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -1019,7 +1011,7 @@ __global__ void __launch_bounds__(kK2Threads, 1) k2_state(const KParams P, void 
     tmem_relinquish();
   }
   if (tid == 0) {
-    for (int i = 0; i < 9; ++i) mbar_init(bars + i, 1);
+    for (int i = 0; i < 8; ++i) mbar_init(bars + i, 1);
     mbar_init(B.sepi, kK2Compute / 32);
     mbar_init(B.depi, kK2Compute / 32);
     *abort_flag = 0;
@@ -1074,12 +1066,12 @@ __global__ void __launch_bounds__(kK2Threads, 1) k2_state(const KParams P, void 
     for (int n = 0; n < N; ++n) {
       const int s = n & 1;
       PDN_K2_MARK(0);
-      // chunk n's main operands (its e^{G_C}) have landed; MMA6 of chunk n - 1
-      // is done reading the bf16 copy of S. (MMA8 of chunk n - 1, which the
-      // state needs, was awaited at the end of the previous iteration.)
+      // chunk n's main operands (its e^{G_C}) have landed. (MMA8 of chunk
+      // n - 1, which the state needs, was awaited at the end of the previous
+      // iteration; the bf16 S buffer this chunk writes was last read by MMA5
+      // and MMA6 of chunk n - 2, both done before that chunk's output.)
       if (!(ok = k2_warp_wait(B.fmain + (n % 3), (uint32_t)((n / 3) & 1), abort_flag, lane))) break;
       PDN_K2_MARK(8);
-      if (n > 0 && !(ok = k2_warp_wait(B.bar6, (uint32_t)((n - 1) & 1), abort_flag, lane))) break;
       PDN_K2_MARK(1);
 
       // ---- state epilogue: S -> bf16 operand; TMEM S <- S Diag(e^{G_C}) ----
@@ -1115,7 +1107,7 @@ __global__ void __launch_bounds__(kK2Threads, 1) k2_state(const KParams P, void 
           for (int u = 0; u < 2; ++u)
 #pragma unroll
             for (int e = 0; e < 8; ++e) pk[8 * u + e] = pack_bf16(sv[u][2 * e], sv[u][2 * e + 1]);
-          tmem_st16u(tm + lane_q + TM_SB + 16 * cg, pk);
+          tmem_st16u(tm + lane_q + tm_sb(n) + 16 * cg, pk);
         }
 #pragma unroll
         for (int u = 0; u < 2; ++u) {
@@ -1132,16 +1124,8 @@ __global__ void __launch_bounds__(kK2Threads, 1) k2_state(const KParams P, void 
         tmem_wait_st();
       }
       k2_warp_arrive(B.sepi, lane);
+      PDN_K2_WMARK(0);
       PDN_K2_MARK(2);
-      // chunk n - 1's output, while MMA5 runs (this also frees its TMEM
-      // buffer for chunk n + 1 and D^T's shared tile for this chunk)
-      if (n > 0) {
-        if (!(ok = k2_warp_wait(B.baro, (uint32_t)((n - 1) & 1), abort_flag, lane))) break;
-        PDN_K2_MARK(9);
-        const int pc0 = (n - 1) * kC;
-        k2_store_o(P, tm + lane_q + (s ? TM_OT0 : TM_OT1), b, h, pc0, min(kC, P.T - pc0), lane,
-                   quarter, cg);
-      }
       PDN_K2_MARK(3);
       if (!(ok = k2_warp_wait(B.bar5, (uint32_t)(n & 1), abort_flag, lane))) break;
       PDN_K2_MARK(4);
@@ -1154,11 +1138,21 @@ __global__ void __launch_bounds__(kK2Threads, 1) k2_state(const KParams P, void 
         uint32_t pk[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) pk[e] = pack_bf16(v[2 * e], v[2 * e + 1]);
-        tmem_st8u(tm + lane_q + TM_DB + 8 * cg, pk);
+        tmem_st8u(tm + lane_q + tm_db(n) + 8 * cg, pk);
         tmem_wait_st();
       }
       k2_warp_arrive(B.depi, lane);
+      PDN_K2_WMARK(1);
       PDN_K2_MARK(5);
+      // chunk n - 1's output, while MMA8 runs (the O^T buffer it frees takes
+      // chunk n + 1, whose MMA6 comes after this chunk's epilogues)
+      if (n > 0) {
+        if (!(ok = k2_warp_wait(B.baro, (uint32_t)((n - 1) & 1), abort_flag, lane))) break;
+        PDN_K2_MARK(9);
+        const int pc0 = (n - 1) * kC;
+        k2_store_o(P, tm + lane_q + (s ? TM_OT0 : TM_OT1), b, h, pc0, min(kC, P.T - pc0), lane,
+                   quarter, cg);
+      }
       PDN_K2_MARK(6);
       if (!(ok = k2_warp_wait(B.bar7, (uint32_t)(n & 1), abort_flag, lane))) break;
       PDN_K2_MARK(7);
