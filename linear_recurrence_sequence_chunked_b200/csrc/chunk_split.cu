@@ -107,21 +107,43 @@ __global__ void __launch_bounds__(256) k0_chunk_energy(const KParams P, void *ws
   }
 }
 
-__global__ void __launch_bounds__(kD) k0_prefix(const KParams P, void *ws, int N) {
-  const int bh = blockIdx.x, i = threadIdx.x;
-  float a = P.A0 ? P.A0[(size_t)bh * kD + i] : 0.f;
-  for (int c0 = 0; c0 < N; c0 += 8) {
-    float s[8];
+// A at every chunk start: per (batch, head), an exclusive prefix over the
+// chunk sums, seeded with A0. Four groups of 128 threads take a quarter of the
+// chunks each: their totals first, then the prefixes.
+constexpr int kK0Groups = 4;
+__global__ void __launch_bounds__(kD * kK0Groups) k0_prefix(const KParams P, void *ws, int N) {
+  __shared__ float tot[kK0Groups][kD];
+  const int bh = blockIdx.x, i = threadIdx.x & (kD - 1), g = threadIdx.x / kD;
+  const int BH = P.B * P.H;
+  const int L = (N + kK0Groups - 1) / kK0Groups;
+  const int c_begin = min(N, g * L), c_end = min(N, c_begin + L);
+  float t = 0.f;
+  for (int c0 = c_begin; c0 < c_end; c0 += 8) {
+    float v[8];
 #pragma unroll
     for (int e = 0; e < 8; ++e)
-      s[e] = (c0 + e < N) ? reinterpret_cast<float *>(ws_block(ws, bh, P.B * P.H, c0 + e) + WS_A)[i] : 0.f;
+      v[e] = (c0 + e < c_end) ? reinterpret_cast<const float *>(ws_block(ws, bh, BH, c0 + e) + WS_A)[i]
+                              : 0.f;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) t += v[e];
+  }
+  tot[g][i] = t;
+  __syncthreads();
+  float a = P.A0 ? P.A0[(size_t)bh * kD + i] : 0.f;
+  for (int g2 = 0; g2 < g; ++g2) a += tot[g2][i];
+  for (int c0 = c_begin; c0 < c_end; c0 += 8) {
+    float v[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e)
+      v[e] = (c0 + e < c_end) ? reinterpret_cast<const float *>(ws_block(ws, bh, BH, c0 + e) + WS_A)[i]
+                              : 0.f;
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
-      if (c0 + e < N) reinterpret_cast<float *>(ws_block(ws, bh, P.B * P.H, c0 + e) + WS_A)[i] = a;
-      a += s[e];
+      if (c0 + e < c_end) reinterpret_cast<float *>(ws_block(ws, bh, BH, c0 + e) + WS_A)[i] = a;
+      a += v[e];
     }
   }
-  if (P.AT) P.AT[(size_t)bh * kD + i] = a;
+  if (g == kK0Groups - 1 && P.AT) P.AT[(size_t)bh * kD + i] = a;
 }
 
 // ===========================================================================
@@ -297,6 +319,7 @@ __global__ void __launch_bounds__(kK1Threads, 2) k1_intra(const KParams P, void 
   // scalars into shared memory; then start loading the next block's ----
   uint4 vcur[4];
   cp_async_wait_all();  // this block's k and v
+  if (tid == 0) bulk_wait_read0();  // the previous block's bulk stores have read their tiles
   __syncthreads();
   {
 #pragma unroll
@@ -768,8 +791,7 @@ __global__ void __launch_bounds__(kK1Threads, 2) k1_intra(const KParams P, void 
         bulk_s2g(blk + WS_Y, smem + K1_YT, 16384);
         bulk_s2g(blk + WS_T, smem + K1_TM, 8192);
         bulk_s2g(blk + WS_P, smem + K1_PM, 8192);
-        bulk_commit();
-        bulk_wait_read0();  // the tiles may be rewritten; the writes land on their own
+        bulk_commit();  // their reads are awaited before the next block rewrites the tiles
       }
     }
   }
@@ -1249,7 +1271,7 @@ cudaError_t launch_chunk_split(const KParams &P, void *ws, cudaStream_t stream) 
   if (is_precond(P.variant)) {
     k0_chunk_energy<<<dim3((unsigned)N, (unsigned)BH), 256, 0, stream>>>(P, ws, N);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    k0_prefix<<<BH, kD, 0, stream>>>(P, ws, N);
+    k0_prefix<<<BH, kD * kK0Groups, 0, stream>>>(P, ws, N);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   switch (P.variant) {
