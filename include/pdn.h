@@ -155,6 +155,33 @@ pdn_status_t pdn_chunk_fwd(const pdn_problem_t *p, const pdn_tensors_t *t,
  *     first. */
 pdn_status_t pdn_chunk_fwd_noalloc(const pdn_problem_t *p, const pdn_tensors_t *t, void *stream);
 
+/* Chunked forward from host memory, end to end: copies the inputs in, runs
+ * pdn_chunk_fwd and copies the outputs out, with the batch cut into `slices`
+ * contiguous parts so that on the GPU the host-to-device copy of part i + 1,
+ * the forward of part i and the device-to-host copy of part i - 1 overlap
+ * (the batch elements are independent chains, so the result is that of one
+ * pdn_chunk_fwd over the whole batch).
+ *   - `dev`: the device tensors of the whole problem, as pdn_chunk_fwd takes
+ *     them (they are also the staging buffers). `workspace` as for
+ *     pdn_chunk_fwd on the whole problem.
+ *   - `host`: host pointers, same layouts; they must be page-locked
+ *     (cudaHostAlloc / registered) for the copies to run asynchronously. A
+ *     non-NULL host input (q, k, v, gates, S0, A0) is copied in before use, a
+ *     non-NULL host output (o, ST, AT) receives the result; a NULL one leaves
+ *     that tensor on the device (an input already there, an output kept).
+ *     Every non-NULL host pointer needs its device buffer.
+ *   - 1 <= slices <= B. Work is ordered after the work already on `stream`,
+ *     and `stream` waits for all of it; the compute runs on `stream`, the
+ *     copies on two streams of the library's own, created on first use on
+ *     each device together with their events (nothing is created later).
+ *   - Calls on one device from several host threads are serialised inside
+ *     the call while they enqueue.
+ * Returns PDN_OK once everything is enqueued; argument errors are returned
+ * before anything is enqueued. */
+pdn_status_t pdn_chunk_fwd_host(const pdn_problem_t *p, const pdn_tensors_t *host,
+                                const pdn_tensors_t *dev, void *workspace, size_t ws_bytes,
+                                int slices, void *stream);
+
 /* One decode step: p->T must be 1. The state and, for preconditioned
  * variants, the accumulator are updated IN PLACE: pass S0 == ST (non-NULL)
  * and A0 == AT (non-NULL for PDN/PGDN/PKDA, NULL otherwise). */

@@ -67,6 +67,8 @@ def load() -> ctypes.CDLL:
         lib.pdn_chunk_fwd.argtypes = [P, T, vp, ctypes.c_size_t, vp]
         lib.pdn_chunk_fwd_noalloc.restype = ctypes.c_int
         lib.pdn_chunk_fwd_noalloc.argtypes = [P, T, vp]
+        lib.pdn_chunk_fwd_host.restype = ctypes.c_int
+        lib.pdn_chunk_fwd_host.argtypes = [P, T, T, vp, ctypes.c_size_t, ctypes.c_int, vp]
         lib.pdn_decode_step.restype = ctypes.c_int
         lib.pdn_decode_step.argtypes = [P, T, vp]
         lib.pdn_get_device_error.restype = ctypes.c_int
@@ -98,6 +100,15 @@ def pdn_chunk_fwd_noalloc(problem: PdnProblem, tensors: PdnTensors, stream: int)
     """Allocation-free chunked forward (see include/pdn.h): scratch comes
     from a fixed array inside the library instead of a caller workspace."""
     return load().pdn_chunk_fwd_noalloc(ctypes.byref(problem), ctypes.byref(tensors), stream)
+
+
+def pdn_chunk_fwd_host(problem: PdnProblem, host: PdnTensors, dev: PdnTensors, workspace: int,
+                       ws_bytes: int, slices: int, stream: int) -> int:
+    """Chunked forward from (page-locked) host memory with the copies
+    overlapped with the compute over `slices` parts of the batch (see
+    include/pdn.h)."""
+    return load().pdn_chunk_fwd_host(ctypes.byref(problem), ctypes.byref(host), ctypes.byref(dev),
+                                     workspace, ws_bytes, slices, stream)
 
 
 def pdn_decode_step(problem: PdnProblem, tensors: PdnTensors, stream: int) -> int:
@@ -138,6 +149,25 @@ def make_problem(variant: str, B: int, T: int, H: int, d_k: int, d_v: int, dtype
         decay = {"DN": "none", "PDN": "none", "GDN": "scalar", "PGDN": "scalar"}.get(variant, "channel")
     return PdnProblem(B, T, H, d_k, d_v, chunk, VARIANTS[variant], DECAYS[decay], DTYPES[dtype],
                       IMPLS[impl], q_scale, precond_x, precond_eps)
+
+
+def _host_ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    if t is None:
+        return None
+    if t.is_cuda or not t.is_pinned():
+        raise ValueError("host tensors must be page-locked CPU tensors (pin_memory())")
+    if not t.is_contiguous():
+        raise ValueError("all tensors must be contiguous")
+    return t.data_ptr() or None
+
+
+def make_host_tensors(q=None, k=None, v=None, o=None, log_alpha=None, beta=None, erase=None,
+                      write=None, S0=None, ST=None, A0=None, AT=None) -> PdnTensors:
+    """The `host` argument of pdn_chunk_fwd_host: page-locked CPU tensors;
+    None leaves that tensor on the device."""
+    return PdnTensors(_host_ptr(q), _host_ptr(k), _host_ptr(v), _host_ptr(log_alpha),
+                      _host_ptr(beta), _host_ptr(erase), _host_ptr(write), _host_ptr(S0),
+                      _host_ptr(ST), _host_ptr(A0), _host_ptr(AT), _host_ptr(o))
 
 
 def make_tensors(q, k, v, o, log_alpha=None, beta=None, erase=None, write=None, S0=None,

@@ -161,3 +161,24 @@ def test_decode_rules(lib):
 
 def test_selftest_rejects_negative_limit(lib):
     assert pdn.pdn_selftest_bounded_wait(-1, None) == pdn.PDN_ERR_INVALID_ARG
+
+
+def test_host_pipeline_argument_errors(lib):
+    """pdn_chunk_fwd_host rejects bad arguments before it touches a device."""
+    p = _problem()
+    t = _tensors()
+    need = pdn.pdn_chunk_fwd_workspace(p)
+    ws = FAKE + 0x100000
+    # slices outside [1, B]
+    assert pdn.pdn_chunk_fwd_host(p, t, t, ws, need, 0, None) == pdn.PDN_ERR_INVALID_ARG
+    assert pdn.pdn_chunk_fwd_host(p, t, t, ws, need, p.B + 1, None) == pdn.PDN_ERR_INVALID_ARG
+    # a host tensor without its device buffer
+    assert pdn.pdn_chunk_fwd_host(p, _tensors(S0=FAKE + 0x9000), t, ws, need, 1,
+                                  None) == pdn.PDN_ERR_INVALID_ARG
+    assert pdn.pdn_chunk_fwd_host(p, t, _tensors(q=None), ws, need, 1,
+                                  None) == pdn.PDN_ERR_INVALID_ARG
+    # an invalid problem
+    assert pdn.pdn_chunk_fwd_host(_problem(B=0), t, t, ws, need, 1, None) == pdn.PDN_ERR_INVALID_ARG
+    # a workspace smaller than the whole problem needs
+    if need > 0:
+        assert pdn.pdn_chunk_fwd_host(p, t, t, ws, need - 1, 1, None) == pdn.PDN_ERR_WORKSPACE

@@ -1,0 +1,71 @@
+"""pdn_chunk_fwd_host (inputs and outputs in page-locked host memory, copies
+overlapped with the compute over slices of the batch) against pdn_chunk_fwd
+on device buffers: the batch elements are independent chains, so every
+output must be bitwise the same for any number of slices; and against the
+oracle once."""
+import pytest
+import torch
+
+from linear_recurrence_sequence_chunked_b200 import pdn
+from linear_recurrence_sequence_chunked_b200.workloads import Workload, make_inputs
+
+from parity_util import assert_parity, run_gpu, run_oracle
+
+pytestmark = pytest.mark.gpu
+
+DECAY = {"PGDN": "scalar", "PKDA": "channel", "FG2_GDN": "channel", "GDN2": "channel",
+         "DN": "none"}
+GATES = ("log_alpha", "beta", "erase", "write")
+
+
+def host_run(w, x, S0, A0, slices):
+    dev = torch.device("cuda")
+    hx = {n: (t.pin_memory() if t is not None else None) for n, t in x.items()}
+    ho = torch.empty(w.B, w.T, w.H, w.dv, dtype=x["v"].dtype).pin_memory()
+    hS0 = S0.pin_memory() if S0 is not None else None
+    hA0 = A0.pin_memory() if A0 is not None else None
+    hST = torch.empty(w.B, w.H, w.dv, w.dk).pin_memory()
+    precond = w.variant in pdn.PRECOND_VARIANTS
+    hAT = torch.empty(w.B, w.H, w.dk).pin_memory() if precond else None
+    dx = {n: (torch.empty_like(t, device=dev) if t is not None else None) for n, t in hx.items()}
+    do = torch.empty(ho.shape, dtype=ho.dtype, device=dev)
+    dS0 = torch.empty_like(hS0, device=dev) if hS0 is not None else None
+    dA0 = torch.empty_like(hA0, device=dev) if hA0 is not None else None
+    dST = torch.empty(hST.shape, device=dev)
+    dAT = torch.empty(hAT.shape, device=dev) if precond else None
+    prob = pdn.make_problem(w.variant, w.B, w.T, w.H, w.dk, w.dv, x["k"].dtype, w.decay)
+    ws_bytes = pdn.pdn_chunk_fwd_workspace(prob)
+    ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
+    th = pdn.make_host_tensors(hx["q"], hx["k"], hx["v"], ho, *(hx[n] for n in GATES),
+                               S0=hS0, ST=hST, A0=hA0, AT=hAT)
+    td = pdn.make_tensors(dx["q"], dx["k"], dx["v"], do, *(dx[n] for n in GATES),
+                          S0=dS0, ST=dST, A0=dA0, AT=dAT)
+    stream = torch.cuda.current_stream().cuda_stream
+    rc = pdn.pdn_chunk_fwd_host(prob, th, td, ws.data_ptr(), ws.numel(), slices, stream)
+    assert rc == pdn.PDN_OK, pdn.pdn_status_string(rc)
+    torch.cuda.synchronize()
+    assert pdn.device_error() == pdn.PDN_OK
+    return ho, hST, hAT
+
+
+@pytest.mark.parametrize("variant", ["PGDN", "PKDA", "FG2_GDN", "GDN2", "DN"])
+def test_host_path_matches_device_path(variant):
+    w = Workload("host-" + variant, variant, 3, 130, 2, 128, 128, "bf16", DECAY[variant])
+    x = make_inputs(w)
+    g = torch.Generator().manual_seed(7)
+    S0 = 0.2 * torch.randn(w.B, w.H, 128, 128, generator=g)
+    A0 = torch.rand(w.B, w.H, 128, generator=g) if variant in pdn.PRECOND_VARIANTS else None
+    ref = run_gpu(w, x, S0, A0)
+    for slices in (1, 2, 3):
+        o, ST, AT = host_run(w, x, S0, A0, slices)
+        assert torch.equal(o, ref[0].cpu()), (variant, slices)
+        assert torch.equal(ST, ref[1].cpu()), (variant, slices)
+        if AT is not None:
+            assert torch.equal(AT, ref[2].cpu()), (variant, slices)
+
+
+def test_host_path_parity_with_oracle():
+    w = Workload("host-oracle", "PGDN", 2, 200, 2, 128, 128, "bf16", "scalar")
+    x = make_inputs(w)
+    o, ST, AT = host_run(w, x, None, None, 2)
+    assert_parity(w, o, ST, AT, *run_oracle(w, x))
