@@ -843,8 +843,9 @@ __global__ void __launch_bounds__(kK1Threads, 2) k1_intra(const KParams P, void 
 constexpr int kK2Compute = 512;
 constexpr int kK2SWarp = kK2Compute / 32, kK2OWarp = kK2SWarp + 1, kK2LoadWarp = kK2SWarp + 2;
 constexpr int kK2Threads = kK2Compute + 96;
-// main buffer: Qh, Y^T, Wb, then P and e^{G_C} (adjacent in the workspace too)
-constexpr uint32_t KM_Q = 0, KM_Y = 16384, KM_WB = 32768, KM_P = 49152, KM_E = KM_P + (WS_E - WS_P);
+// main buffer: Qh, Y^T, Wb, then P and e^{G_C} (adjacent in the workspace too;
+// the state epilogue takes e^{G_C} from its own copy, below)
+constexpr uint32_t KM_Q = 0, KM_Y = 16384, KM_WB = 32768, KM_P = 49152;
 constexpr uint32_t KM_SIZE = KM_P + (WS_SET - WS_P);
 // U/T buffer
 constexpr uint32_t KU_U = 0, KU_T = 16384, KU_SIZE = 16384 + (WS_P - WS_T);
@@ -853,7 +854,10 @@ constexpr uint32_t K2_UT = 3 * KM_SIZE;            // two U/T buffers
 constexpr uint32_t K2_BAR = K2_UT + 2 * KU_SIZE;   // the ten mbarriers above
 constexpr uint32_t K2_ABORT = K2_BAR + 12 * 8;
 constexpr uint32_t K2_TBASE = K2_ABORT + 8;
-constexpr uint32_t K2_BYTES = K2_TBASE + 16;
+// e^{G_C} of the current and the next chunk, one copy per compute warp (the
+// 32 key channels of its column group), fetched by the warp itself
+constexpr uint32_t K2_EBUF = (K2_TBASE + 16 + 127) / 128 * 128;
+constexpr uint32_t K2_BYTES = K2_EBUF + 16 * 2 * 128;
 static_assert(K2_BYTES <= 232448, "state kernel shared memory budget");
 
 // TMEM columns: U~^T then D^T (fp32), the two O^T buffers, S in bf16 pairs
@@ -959,7 +963,9 @@ __device__ __forceinline__ bool k2_issue_s(uint32_t tm, uint32_t sb, const K2Bar
       if (!k2_wait(B.fut + 0, 0, abort_flag)) return false;
       k2_mma3(tm, sb + ut_buf(0));
     }
-    // MMA5: D^T = U~^T - S Y^T, once the state epilogue has written S (bf16)
+    // MMA5: D^T = U~^T - S Y^T, once chunk n's main operands have landed and
+    // the state epilogue has written S (bf16)
+    if (!k2_wait(B.fmain + (n % 3), (uint32_t)((n / 3) & 1), abort_flag)) return false;
     if (!k2_wait(B.sepi, (uint32_t)(n & 1), abort_flag)) return false;
     PDN_K2_IMARK(0);
 #pragma unroll
@@ -1085,20 +1091,32 @@ __global__ void __launch_bounds__(kK2Threads, 1) k2_state(const KParams P, void 
     const int cg = warp >> 2;          // column group 0..3
     const int j = 32 * quarter + lane; // value channel owned in the epilogues
     bool ok = true;
+    // this warp's 32 values of e^{G_C} for chunk c into its buffer c & 1
+    auto fetch_e = [&](int c) {
+      if (lane < 8)
+        cp_async16(sb + K2_EBUF + (warp * 2 + (c & 1)) * 128 + lane * 16,
+                   reinterpret_cast<const float *>(ws_block(ws, bh, P.B * P.H, c) + WS_E) + 32 * cg +
+                       4 * lane,
+                   true);
+      cp_async_commit();
+    };
+    if (N > 0) fetch_e(0);
     for (int n = 0; n < N; ++n) {
       const int s = n & 1;
       PDN_K2_MARK(0);
-      // chunk n's main operands (its e^{G_C}) have landed. (MMA8 of chunk
-      // n - 1, which the state needs, was awaited at the end of the previous
-      // iteration; the bf16 S buffer this chunk writes was last read by MMA5
-      // and MMA6 of chunk n - 2, both done before that chunk's output.)
-      if (!(ok = k2_warp_wait(B.fmain + (n % 3), (uint32_t)((n / 3) & 1), abort_flag, lane))) break;
+      // this chunk's e^{G_C} has landed (fetched by the warp a chunk ahead).
+      // (MMA8 of chunk n - 1, which the state needs, was awaited at the end of
+      // the previous iteration; the bf16 S buffer this chunk writes was last
+      // read by MMA5 and MMA6 of chunk n - 2, both done before that chunk's
+      // output.)
+      cp_async_wait_all();
+      __syncwarp();
       PDN_K2_MARK(8);
       PDN_K2_MARK(1);
 
       // ---- state epilogue: S -> bf16 operand; TMEM S <- S Diag(e^{G_C}) ----
       {
-        const float *egc = reinterpret_cast<const float *>(smem + main_buf(n) + KM_E);
+        const float *egc = reinterpret_cast<const float *>(smem + K2_EBUF + (warp * 2 + (n & 1)) * 128);
         float sv[2][16];
         const int col0 = 32 * cg;
         if (n == 0) {
@@ -1135,10 +1153,10 @@ __global__ void __launch_bounds__(kK2Threads, 1) k2_state(const KParams P, void 
         for (int u = 0; u < 2; ++u) {
           const int col = col0 + 16 * u;
           float E[8];
-          ld8f(egc + col, E);
+          ld8f(egc + (col - col0), E);
 #pragma unroll
           for (int e = 0; e < 8; ++e) sv[u][e] *= E[e];
-          ld8f(egc + col + 8, E);
+          ld8f(egc + (col - col0) + 8, E);
 #pragma unroll
           for (int e = 0; e < 8; ++e) sv[u][8 + e] *= E[e];
           tmem_st16(tm + lane_q + TM_S + col, sv[u]);
@@ -1166,6 +1184,7 @@ __global__ void __launch_bounds__(kK2Threads, 1) k2_state(const KParams P, void 
       k2_warp_arrive(B.depi, lane);
       PDN_K2_WMARK(1);
       PDN_K2_MARK(5);
+      if (n + 1 < N) fetch_e(n + 1);
       // chunk n - 1's output, while MMA8 runs (the O^T buffer it frees takes
       // chunk n + 1, whose MMA6 comes after this chunk's epilogues)
       if (n > 0) {
