@@ -52,7 +52,7 @@ enum { OR_DECAY_NONE = 0, OR_DECAY_SCALAR = 1, OR_DECAY_CHANNEL = 2 };
  *   P_t = Diag(A_t)^{-1}                   (raw form, replaced by B_t)
  *   stabilised: log space, centred, squashed by r/(1+|r|), then an inverse
  *   exponential that keeps B_t inside [1/x, x].
- * Readings where the pages are silent (listed in the design doc):
+ * Readings where the pages are silent:
  *   - centring mu_t = mean over the d_k channels of log(A_{t,i} + eps);
  *   - eps is added inside the log (A_0 = 0 would give log 0);
  *   - "inverse exponential" read as B = x^(-s), decreasing in A like A^{-1};

@@ -186,7 +186,7 @@ def variant_vectors(variant, d, b, t, h, Bc=None):
 def test_p6_brute_force_product_expansion(variant, T):
     """For T <= 3 the state is the explicit sum of products
     S_T = S_0 prod_s D_s (I - r_s w_s^T) + sum_t u_t w_t^T prod_{s>t} D_s (I - r_s w_s^T),
-    formed with d_k x d_k matrices (the spec update written out)."""
+    formed with d_k x d_k matrices (the generic update written out)."""
     d = rand_inputs(variant, B=1, T=T, H=1, dk=5, dv=5 if variant == "FG2_GDN" else 4, seed=10 + T)
     o, ST, AT = oracle.forward(variant, **d, q_scale=1.3)
     dk = 5
