@@ -829,6 +829,11 @@ __global__ void __launch_bounds__(kK1Threads, 2) k1_intra(const KParams P, void 
 //   bar7     MMA8 (state update) done             (S warp)
 //   baro     MMA7 (O^T += D^T P^T) done: the chunk's output and, since the O
 //            warp waits on bar7 first, every MMA of the chunk
+//   ufree[x] MMA3 of the chunk in U/T buffer x done (the buffer may be refilled)
+//   mfree[x] every MMA of the chunk in main buffer x done (likewise)
+// The load warp waits only on ufree/mfree: a buffer's barrier cannot move on
+// before the load warp has refilled it, so however far the load warp falls
+// behind, the phase it waits for is never overtaken.
 // The O warp issues MMA6 only after MMA5 and MMA7 only after MMA8 have
 // completed, so the tensor pipe never holds output work ahead of the state
 // chain's. The compute warps write chunk n - 1's output while MMA5 of chunk
@@ -851,8 +856,8 @@ constexpr uint32_t KM_SIZE = KM_P + (WS_SET - WS_P);
 constexpr uint32_t KU_U = 0, KU_T = 16384, KU_SIZE = 16384 + (WS_P - WS_T);
 constexpr uint32_t K2_MAIN = 0;                    // three main buffers
 constexpr uint32_t K2_UT = 3 * KM_SIZE;            // two U/T buffers
-constexpr uint32_t K2_BAR = K2_UT + 2 * KU_SIZE;   // the ten mbarriers above
-constexpr uint32_t K2_ABORT = K2_BAR + 12 * 8;
+constexpr uint32_t K2_BAR = K2_UT + 2 * KU_SIZE;   // the fifteen mbarriers above
+constexpr uint32_t K2_ABORT = K2_BAR + 16 * 8;
 constexpr uint32_t K2_TBASE = K2_ABORT + 8;
 // e^{G_C} of the current and the next chunk, one copy per compute warp (the
 // 32 key channels of its column group), fetched by the warp itself
@@ -949,7 +954,7 @@ __device__ __forceinline__ void k2_mma3(uint32_t tm, uint32_t ut) {
 }
 
 struct K2Bars {
-  uint64_t *fmain, *fut, *bar5, *bar7, *baro, *sepi, *depi;
+  uint64_t *fmain, *fut, *bar5, *bar7, *baro, *sepi, *depi, *ufree, *mfree;
 };
 
 // The S warp's program (one lane): MMA3, MMA5, MMA8. False if a wait ran out.
@@ -962,6 +967,7 @@ __device__ __forceinline__ bool k2_issue_s(uint32_t tm, uint32_t sb, const K2Bar
     if (n == 0) {
       if (!k2_wait(B.fut + 0, 0, abort_flag)) return false;
       k2_mma3(tm, sb + ut_buf(0));
+      mma_commit(B.ufree + 0);
     }
     // MMA5: D^T = U~^T - S Y^T, once chunk n's main operands have landed and
     // the state epilogue has written S (bf16)
@@ -987,6 +993,7 @@ __device__ __forceinline__ bool k2_issue_s(uint32_t tm, uint32_t sb, const K2Bar
     if (n + 1 < N) {
       if (!k2_wait(B.fut + ((n + 1) & 1), (uint32_t)(((n + 1) >> 1) & 1), abort_flag)) return false;
       k2_mma3(tm, sb + ut_buf(n + 1));
+      mma_commit(B.ufree + ((n + 1) & 1));
     }
   }
   return true;
@@ -1001,8 +1008,10 @@ __device__ __forceinline__ bool k2_issue_o(uint32_t tm, uint32_t sb, const K2Bar
     const uint32_t mb = sb + main_buf(n);
     const uint32_t ot = (n & 1) ? TM_OT1 : TM_OT0;
     // MMA6: O^T = S Qh^T after MMA5 (which also means the compute warps have
-    // written out chunk n - 2's output from this buffer)
+    // written out chunk n - 2's output from this buffer), on operands this
+    // warp has seen land
     if (!k2_wait(B.bar5, (uint32_t)(n & 1), abort_flag)) return false;
+    if (!k2_wait(B.fmain + (n % 3), (uint32_t)((n / 3) & 1), abort_flag)) return false;
     PDN_K2_IMARK(4);
 #pragma unroll
     for (int kk = 0; kk < 8; ++kk)
@@ -1017,6 +1026,7 @@ __device__ __forceinline__ bool k2_issue_o(uint32_t tm, uint32_t sb, const K2Bar
       mma_bf16_ts(tm + ot, tm + tm_db(n) + 8 * kk, make_sdesc(mb + KM_P + 256 * kk, 128, 1024), id7,
                   1);
     mma_commit(B.baro);
+    mma_commit(B.mfree + (n % 3));
     PDN_K2_IMARK(7);
   }
   return true;
@@ -1026,7 +1036,8 @@ __global__ void __launch_bounds__(kK2Threads, 1) k2_state(const KParams P, void 
   extern __shared__ __align__(1024) uint8_t smem[];
   const uint32_t sb = smem_u32(smem);
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + K2_BAR);
-  const K2Bars B{bars, bars + 3, bars + 5, bars + 6, bars + 7, bars + 8, bars + 9};
+  const K2Bars B{bars,     bars + 3, bars + 5,  bars + 6, bars + 7,
+                 bars + 8, bars + 9, bars + 10, bars + 12};
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + K2_ABORT);
   uint32_t *tbase_p = reinterpret_cast<uint32_t *>(smem + K2_TBASE);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -1040,6 +1051,7 @@ __global__ void __launch_bounds__(kK2Threads, 1) k2_state(const KParams P, void 
   }
   if (tid == 0) {
     for (int i = 0; i < 8; ++i) mbar_init(bars + i, 1);
+    for (int i = 10; i < 15; ++i) mbar_init(bars + i, 1);
     mbar_init(B.sepi, kK2Compute / 32);
     mbar_init(B.depi, kK2Compute / 32);
     *abort_flag = 0;
@@ -1066,17 +1078,17 @@ __global__ void __launch_bounds__(kK2Threads, 1) k2_state(const KParams P, void 
         load_main(smem + main_buf(m), ws_block(ws, bh, BH, m), B.fmain + m);
       for (int m = 0; m < 2 && m < N; ++m)
         load_ut(smem + ut_buf(m), ws_block(ws, bh, BH, m), B.fut + m);
-      // after MMA3 of chunk n (bar5), its U/T buffer takes chunk n + 2; after
-      // every MMA of chunk n (baro), its main buffer takes chunk n + 3
+      // after MMA3 of chunk n, its U/T buffer takes chunk n + 2; after every
+      // MMA of chunk n, its main buffer takes chunk n + 3
       for (int n = 0; n + 2 < N; ++n) {
-        if (!k2_wait(B.bar5, (uint32_t)(n & 1), abort_flag)) {
+        if (!k2_wait(B.ufree + (n & 1), (uint32_t)((n >> 1) & 1), abort_flag)) {
           *abort_flag = 1;
           break;
         }
         load_ut(smem + ut_buf(n), ws_block(ws, bh, BH, n + 2), B.fut + (n & 1));
         PDN_K2_HMARK(0);
         if (n + 3 < N) {
-          if (!k2_wait(B.baro, (uint32_t)(n & 1), abort_flag)) {
+          if (!k2_wait(B.mfree + (n % 3), (uint32_t)((n / 3) & 1), abort_flag)) {
             *abort_flag = 1;
             break;
           }
