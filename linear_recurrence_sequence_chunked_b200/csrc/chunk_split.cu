@@ -921,23 +921,24 @@ __device__ __forceinline__ bool k2_wait(uint64_t *bar, uint32_t parity, volatile
   return ok;
 }
 
-// 16 output tokens (columns 16 cg .. 16 cg + 15 of O^T in TMEM, lanes = value
-// channels) of one lane quarter; two adjacent channels per 32-bit store.
+// 8 output tokens (columns 16 cg + 8 part .. + 7 of O^T in TMEM, lanes =
+// value channels) of one lane quarter; two adjacent channels per 32-bit store.
 __device__ __forceinline__ void k2_store_o(const KParams &P, uint32_t taddr, int b, int h,
-                                           int pc0, int Cn, int lane, int quarter, int cg) {
+                                           int pc0, int Cn, int lane, int quarter, int cg,
+                                           int part) {
   const size_t tstride = (size_t)P.H * kD;
   const int j = 32 * quarter + lane;
   __nv_bfloat16 *orow =
       reinterpret_cast<__nv_bfloat16 *>(P.o) + tok_index(P, b, pc0, h) * kD + (j & ~1);
   const bool odd = lane & 1;
-  float v[16];
-  tmem_ld16(taddr + 16 * cg, v);
+  float v[8];
+  tmem_ld8(taddr + 16 * cg + 8 * part, v);
   tmem_wait_ld();
 #pragma unroll
-  for (int e2 = 0; e2 < 8; ++e2) {
+  for (int e2 = 0; e2 < 4; ++e2) {
     const float send = odd ? v[2 * e2] : v[2 * e2 + 1];
     const float recv = __shfl_xor_sync(0xffffffffu, send, 1);
-    const int t = 16 * cg + 2 * e2 + (odd ? 1 : 0);
+    const int t = 16 * cg + 8 * part + 2 * e2 + (odd ? 1 : 0);
     const float lo = odd ? recv : v[2 * e2];
     const float hi = odd ? v[2 * e2 + 1] : recv;
     if (t < Cn) *reinterpret_cast<uint32_t *>(orow + t * tstride) = pack_bf16(lo, hi);
@@ -1178,6 +1179,16 @@ __global__ void __launch_bounds__(kK2Threads, 1) k2_state(const KParams P, void 
       k2_warp_arrive(B.sepi, lane);
       PDN_K2_WMARK(0);
       PDN_K2_MARK(2);
+      // chunk n - 1's output in two halves, under MMA5 and under MMA8 (the
+      // O^T buffer they free takes chunk n + 1, whose MMA6 comes after this
+      // chunk's epilogues)
+      const uint32_t ot_prev = tm + lane_q + (s ? TM_OT0 : TM_OT1);
+      const int pc_prev = (n - 1) * kC;
+      if (n > 0) {
+        if (!(ok = k2_warp_wait(B.baro, (uint32_t)((n - 1) & 1), abort_flag, lane))) break;
+        PDN_K2_MARK(9);
+        k2_store_o(P, ot_prev, b, h, pc_prev, min(kC, P.T - pc_prev), lane, quarter, cg, 0);
+      }
       PDN_K2_MARK(3);
       if (!(ok = k2_warp_wait(B.bar5, (uint32_t)(n & 1), abort_flag, lane))) break;
       PDN_K2_MARK(4);
@@ -1197,15 +1208,7 @@ __global__ void __launch_bounds__(kK2Threads, 1) k2_state(const KParams P, void 
       PDN_K2_WMARK(1);
       PDN_K2_MARK(5);
       if (n + 1 < N) fetch_e(n + 1);
-      // chunk n - 1's output, while MMA8 runs (the O^T buffer it frees takes
-      // chunk n + 1, whose MMA6 comes after this chunk's epilogues)
-      if (n > 0) {
-        if (!(ok = k2_warp_wait(B.baro, (uint32_t)((n - 1) & 1), abort_flag, lane))) break;
-        PDN_K2_MARK(9);
-        const int pc0 = (n - 1) * kC;
-        k2_store_o(P, tm + lane_q + (s ? TM_OT0 : TM_OT1), b, h, pc0, min(kC, P.T - pc0), lane,
-                   quarter, cg);
-      }
+      if (n > 0) k2_store_o(P, ot_prev, b, h, pc_prev, min(kC, P.T - pc_prev), lane, quarter, cg, 1);
       PDN_K2_MARK(6);
       if (!(ok = k2_warp_wait(B.bar7, (uint32_t)(n & 1), abort_flag, lane))) break;
       PDN_K2_MARK(7);
@@ -1213,8 +1216,9 @@ __global__ void __launch_bounds__(kK2Threads, 1) k2_state(const KParams P, void 
     // the last chunk's output
     if (ok && N > 0 && k2_warp_wait(B.baro, (uint32_t)((N - 1) & 1), abort_flag, lane)) {
       const int pc0 = (N - 1) * kC;
-      k2_store_o(P, tm + lane_q + (((N - 1) & 1) ? TM_OT1 : TM_OT0), b, h, pc0,
-                 min(kC, P.T - pc0), lane, quarter, cg);
+      for (int part = 0; part < 2; ++part)
+        k2_store_o(P, tm + lane_q + (((N - 1) & 1) ? TM_OT1 : TM_OT0), b, h, pc0,
+                   min(kC, P.T - pc0), lane, quarter, cg, part);
     }
     if (!*abort_flag && N > 0 && P.ST) {
       float v[2][16];
