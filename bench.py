@@ -6,9 +6,11 @@ layer workload: B=4 sequences x T=4096 tokens x H=16 heads, d_k = d_v = 128,
 bf16 q/k/v/o, fp32 state, scalar decay, diagonal preconditioner. Inputs are
 resident in HBM before the timed region; L2 is flushed (256 MiB write) between
 timed steps. The JSON line also carries:
-  e2e         the same metric through the public API with pinned HOST
-              buffers (host->device inputs and device->host output per step);
-  roofline    the chunk kernel against the measured bf16 tensor peak;
+  e2e         the same metric end to end through pdn_chunk_fwd_host from
+              pinned HOST buffers (host->device inputs and device->host
+              output per step, overlapped with the compute over batch slices);
+  roofline    one pdn_chunk_fwd call (its kernels timed as one launch by the
+              CUDA events around it) against the measured bf16 tensor peak;
   decode      the recurrent decode workload (256 sequences x 16 heads,
               fp32 state, 1024 steps), tokens/s and HBM roofline;
   cpu_baseline the fp64 oracle on the host cores on a bounded sample.
