@@ -27,8 +27,9 @@
  * problem statement).
  *
  * Conventions (all entry points):
- *   - Every tensor pointer is a DEVICE pointer, contiguous, 16-byte aligned,
- *     owned by the caller; the library allocates no device memory per call.
+ *   - Every tensor pointer is a DEVICE pointer (except the `host` set of
+ *     pdn_chunk_fwd_host), contiguous, 16-byte aligned, owned by the caller;
+ *     the library allocates no device memory per call.
  *   - Layouts are row-major: q, k [B,T,H,d_k]; v, o [B,T,H,d_v];
  *     S0, ST [B,H,d_v,d_k] fp32; A0, AT [B,H,d_k] fp32.
  *   - Work is enqueued on the caller's CUDA stream (`stream`, a cudaStream_t;
