@@ -76,34 +76,52 @@ constexpr float kMinG = -80.f;
 // shared memory.
 __global__ void __launch_bounds__(256) k0_chunk_energy(const KParams P, void *ws, int N) {
   __shared__ float part[16][kD + 4];
-  const int c = blockIdx.x, bh = blockIdx.y, tid = threadIdx.x;
-  const int b = bh / P.H, h = bh % P.H;
-  const int c8 = tid & 15, tl = tid >> 4;
-  const int c0 = c * kC, Cn = min(kC, P.T - c0);
+  const int tid = threadIdx.x, c8 = tid & 15, tl = tid >> 4;
+  const int BH = P.B * P.H, total = N * BH;
   const size_t tstride = (size_t)P.H * kD;
-  const __nv_bfloat16 *kp =
-      reinterpret_cast<const __nv_bfloat16 *>(P.k) + tok_index(P, b, c0, h) * kD + c8 * 8;
-  float acc[8];
+  // The k rows of chunk block `it` (chunk-major, like the workspace): thread
+  // (c8, tl) takes 8 channels of tokens tl, tl + 16, tl + 32, tl + 48.
+  auto load = [&](int it, uint4 (&r)[4]) {
+    const int c = it / BH, bh = it % BH;
+    const int c0 = c * kC, Cn = min(kC, P.T - c0);
+    const __nv_bfloat16 *kp = reinterpret_cast<const __nv_bfloat16 *>(P.k) +
+                              tok_index(P, bh / P.H, c0, bh % P.H) * kD + c8 * 8;
 #pragma unroll
-  for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+    for (int m = 0; m < 4; ++m) {
+      const int t = tl + 16 * m;
+      r[m] = t < Cn ? __ldg(reinterpret_cast<const uint4 *>(kp + t * tstride))
+                    : make_uint4(0u, 0u, 0u, 0u);
+    }
+  };
+  // grid-stride over the blocks, the next block's rows in flight while the
+  // current one is reduced
+  uint4 cur[4];
+  if ((int)blockIdx.x < total) load(blockIdx.x, cur);
+  for (int it = blockIdx.x; it < total; it += gridDim.x) {
+    uint4 nxt[4];
+    if (it + (int)gridDim.x < total) load(it + gridDim.x, nxt);
+    float acc[8];
 #pragma unroll
-  for (int m = 0; m < 4; ++m) {
-    const int t = tl + 16 * m;
-    if (t < Cn) {
+    for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
       float kf[8];
-      unpack8(__ldg(reinterpret_cast<const uint4 *>(kp + t * tstride)), kf);
+      unpack8(cur[m], kf);
 #pragma unroll
       for (int e = 0; e < 8; ++e) acc[e] = fmaf(kf[e], kf[e], acc[e]);
     }
-  }
 #pragma unroll
-  for (int e = 0; e < 8; ++e) part[tl][c8 * 8 + e] = acc[e];
-  __syncthreads();
-  if (tid < kD) {
-    float s = 0.f;
+    for (int e = 0; e < 8; ++e) part[tl][c8 * 8 + e] = acc[e];
+    __syncthreads();
+    if (tid < kD) {
+      float sum = 0.f;
 #pragma unroll
-    for (int r = 0; r < 16; ++r) s += part[r][tid];
-    reinterpret_cast<float *>(ws_block(ws, bh, P.B * P.H, c) + WS_A)[tid] = s;
+      for (int r = 0; r < 16; ++r) sum += part[r][tid];
+      reinterpret_cast<float *>(ws_block(ws, it % BH, BH, it / BH) + WS_A)[tid] = sum;
+    }
+    __syncthreads();  // part is rewritten by the next block
+#pragma unroll
+    for (int m = 0; m < 4; ++m) cur[m] = nxt[m];
   }
 }
 
@@ -1304,7 +1322,15 @@ cudaError_t launch_chunk_split(const KParams &P, void *ws, cudaStream_t stream) 
   const int BH = P.B * P.H;
   cudaError_t e;
   if (is_precond(P.variant)) {
-    k0_chunk_energy<<<dim3((unsigned)N, (unsigned)BH), 256, 0, stream>>>(P, ws, N);
+    int dev = 0, sms = 148, per_sm = 1;
+    if (cudaGetDevice(&dev) == cudaSuccess)
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k0_chunk_energy, 256, 0) !=
+            cudaSuccess || per_sm < 1)
+      per_sm = 1;
+    const long long blocks = (long long)N * BH;
+    const long long grid0 = blocks < (long long)sms * per_sm ? blocks : (long long)sms * per_sm;
+    k0_chunk_energy<<<(unsigned)grid0, 256, 0, stream>>>(P, ws, N);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     k0_prefix<<<BH, kD * kK0Groups, 0, stream>>>(P, ws, N);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
