@@ -182,3 +182,18 @@ def test_host_pipeline_argument_errors(lib):
     # a workspace smaller than the whole problem needs
     if need > 0:
         assert pdn.pdn_chunk_fwd_host(p, t, t, ws, need - 1, 1, None) == pdn.PDN_ERR_WORKSPACE
+
+
+@pytest.mark.parametrize("B,T,H", [(1, 1, 1), (4, 4096, 16), (2, 130, 3), (3, 64, 2)])
+def test_workspace_size_of_the_tensor_core_paths(lib, B, T, H):
+    """The three-kernel path needs one 82,944-byte block per (batch, head,
+    chunk); the fused and CUDA-core paths need none (host-only queries)."""
+    p = _problem(B=B, T=T, H=H, d_k=128, d_v=128)
+    assert pdn.pdn_chunk_fwd_impl(p) == pdn.IMPLS["tc"]
+    assert pdn.pdn_chunk_fwd_workspace(p) == B * H * ((T + 63) // 64) * 82944
+    p = _problem(B=B, T=T, H=H, d_k=128, d_v=128, impl=pdn.IMPLS["tc_fused"])
+    assert pdn.pdn_chunk_fwd_impl(p) == pdn.IMPLS["tc_fused"]
+    assert pdn.pdn_chunk_fwd_workspace(p) == 0
+    p = _problem(B=B, T=T, H=H, d_k=64, d_v=64)
+    assert pdn.pdn_chunk_fwd_impl(p) == pdn.IMPLS["simt"]
+    assert pdn.pdn_chunk_fwd_workspace(p) == 0
