@@ -11,14 +11,19 @@ the kernels use reproduces the token loop. It is a cross-check of the
 algebra, not a second definition: the definition is the token loop in
 pdn_oracle.c.
 
-Per chunk of C tokens with state S0 (d_v x d_k), cumulative in-chunk log
-decay G_t = sum_{s<=t} log alpha_s, Gamma_t = exp(G_t):
-    Rh = Gamma . r,  Wh = w / Gamma,  Qh = Gamma . q,  Wb = Wh . Gamma_C
-    M  = strict_lower(Rh Wh^T),  P = lower(Qh Wh^T)
+Per chunk of C tokens with state S0 (d_v x d_k) and cumulative in-chunk log
+decay G_t = sum_{s<=t} log alpha_s (per key channel):
+    M_ts = sum_i r_ti w_si e^{G_ti - G_si}        (s < t)
+    P_ts = sum_i q_ti w_si e^{G_ti - G_si}        (s <= t)
+    Rh = e^{G} . r,  Qh = e^{G} . q,  Wb = e^{G_C - G} . w
     Y  = (I + M)^{-1} Rh,  U~ = (I + M)^{-1} u
     D  = U~ - Y S0^T
     O  = q_scale (Qh S0^T + P D)
-    S_C = S0 Diag(Gamma_C) + D^T Wb
+    S_C = S0 Diag(e^{G_C}) + D^T Wb
+The decay between two tokens of a chunk is formed from the difference
+G_t - G_s <= 0 itself, never as the product e^{G_t} e^{-G_s}: the pages put no
+floor on the decay (KDA's D_t = Diag(alpha_t), alpha_t in (0,1)^{d_k},
+"Gated DeltaNet-2" ja §1), and for strong decay e^{-G_s} overflows even fp64.
 """
 from __future__ import annotations
 
@@ -42,18 +47,22 @@ def chunk_forward(q, r, w, u, log_alpha=None, S0=None, chunk=64, q_scale=1.0):
                     G = np.zeros((c1 - c0, dk))
                 else:
                     G = np.cumsum(np.asarray(log_alpha[b, c0:c1, h], np.float64), axis=0)
-                Gam = np.exp(G)
-                Rh = Gam * r[b, c0:c1, h]
-                Wh = w[b, c0:c1, h] / Gam
-                Qh = Gam * q[b, c0:c1, h]
-                Wb = Wh * Gam[-1]
-                M = np.tril(Rh @ Wh.T, -1)
-                P = np.tril(Qh @ Wh.T, 0)
+                n = c1 - c0
+                low = np.tril(np.ones((n, n), bool))
+                # E[t, s, i] = e^{G_ti - G_si} for s <= t, 0 above the diagonal
+                diff = G[:, None, :] - G[None, :, :]
+                E = np.exp(np.where(low[:, :, None], diff, -np.inf))
+                rc, wc, qc = r[b, c0:c1, h], w[b, c0:c1, h], q[b, c0:c1, h]
+                M = np.tril(np.einsum("ti,si,tsi->ts", rc, wc, E), -1)
+                P = np.einsum("ti,si,tsi->ts", qc, wc, E)
+                Rh = np.exp(G) * rc
+                Qh = np.exp(G) * qc
+                Wb = np.exp(G[-1][None, :] - G) * wc
                 Tinv = np.linalg.inv(np.eye(c1 - c0) + M)
                 Y = Tinv @ Rh
                 Ut = Tinv @ u[b, c0:c1, h]
                 D = Ut - Y @ S.T
                 o[b, c0:c1, h] = q_scale * (Qh @ S.T + P @ D)
-                S = S * Gam[-1][None, :] + D.T @ Wb
+                S = S * np.exp(G[-1])[None, :] + D.T @ Wb
             ST[b, h] = S
     return o, ST

@@ -329,6 +329,34 @@ def test_p9_chunk_form_equals_token_loop(chunk, T):
     np.testing.assert_allclose(S2, S1, rtol=1e-10, atol=1e-11)
 
 
+@pytest.mark.parametrize("mean_log_alpha", [-1.5, -3.0, -10.0, "hard"])
+@pytest.mark.parametrize("chunk", [16, 64])
+def test_p9_chunk_form_under_strong_decay(mean_log_alpha, chunk):
+    """The chunk form stays equal to the token loop however strong the decay:
+    the pages bound alpha only to (0, 1) (KDA's D_t = Diag(alpha_t),
+    "Gated DeltaNet-2" ja §1), so mean per-token log decays of -1.5, -3 and -10
+    (whole-chunk decays of e^-96 .. e^-640 per channel) and one channel at
+    log alpha = -30 on every token ("hard") must all reproduce the recurrence,
+    down to fp64 rounding."""
+    rng = np.random.default_rng(29)
+    B, T, H, dk, dv = 1, 150, 2, 8, 6
+    q = unit(rng.standard_normal((B, T, H, dk)))
+    r = unit(rng.standard_normal((B, T, H, dk)))
+    w = 0.8 * unit(rng.standard_normal((B, T, H, dk))) * rng.uniform(0.3, 1.2, (B, T, H, dk))
+    u = rng.standard_normal((B, T, H, dv))
+    if mean_log_alpha == "hard":
+        la = -0.1 * np.abs(rng.standard_normal((B, T, H, dk)))
+        la[..., 3] = -30.0
+    else:
+        la = 2.0 * mean_log_alpha * rng.uniform(0.0, 1.0, (B, T, H, dk))
+    S0 = rng.standard_normal((B, H, dv, dk))
+    o1, S1 = oracle.generic(q, r, w, u, log_alpha=la, S0=S0, q_scale=0.9)
+    o2, S2 = chunked.chunk_forward(q, r, w, u, log_alpha=la, S0=S0, chunk=chunk, q_scale=0.9)
+    assert np.isfinite(o2).all() and np.isfinite(S2).all()
+    np.testing.assert_allclose(o2, o1, rtol=1e-10, atol=1e-11)
+    np.testing.assert_allclose(S2, S1, rtol=1e-10, atol=1e-11)
+
+
 # ---------------------------------------------------------------- P10
 @pytest.mark.parametrize("variant", VARIANTS)
 def test_p10_continuation(variant):
