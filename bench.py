@@ -13,6 +13,10 @@ timed steps. The JSON line also carries:
               CUDA events around it) against the measured bf16 tensor peak;
   decode      the recurrent decode workload (256 sequences x 16 heads,
               fp32 state, 1024 steps), tokens/s and HBM roofline;
+  workloads   the other forward workloads (Preconditioned KDA B8 T8192;
+              FG2-GDN and Gated DeltaNet-2 B2 T32768): tokens/s, tensor and
+              HBM fractions, and per-kernel CUDA-event times (also given for
+              the headline layer under roofline.kernel_ms);
   cpu_baseline the fp64 oracle on the host cores on a bounded sample.
 Multi-GPU (torchrun): every rank runs its own independent batch (weak
 scaling, no collective on the data path); the time is the max over ranks.
@@ -304,9 +308,9 @@ def run_ours(args):
     if pdn.device_error() != pdn.PDN_OK:
         raise SystemExit("device error during the timed region")
     impl_id = pdn.pdn_chunk_fwd_impl(prob)
-    tc = impl_id in (pdn.IMPLS["tc"], pdn.IMPLS["tc_fused"])
-    kernel_name = {1: "simt", 2: "tcgen05 split (K0 key energy + prefix, K1 intra-chunk, K2 state)",
-                   3: "tcgen05 fused"}.get(impl_id, "?")
+    tc = impl_id == pdn.IMPLS["tc"]
+    kernel_name = {1: "simt", 2: "tcgen05 split (K0 key energy + prefix, K1 intra-chunk, K2 state)"
+                   }.get(impl_id, "?")
     launches_per_step = 1
     if impl_id == pdn.IMPLS["tc"]:
         launches_per_step = 4 if w.variant in pdn.PRECOND_VARIANTS else 2
@@ -332,6 +336,8 @@ def run_ours(args):
         "clocks": clocks,
         "gpu_launches": args.steps * launches_per_step,
     }
+
+    result["roofline"]["kernel_ms"] = profiled_kernel_ms(pdn, prob, tens, ws, sptr)
 
     # ---------------- e2e: pinned host buffers, copies inside the timed region
     if not args.no_e2e:
@@ -370,6 +376,18 @@ def run_ours(args):
         result["gpu_launches"] += args.steps * launches_per_step * slices
         del hx, ho, dx
 
+    # ---------------- the other forward workloads
+    if not args.no_extra:
+        del ws
+        torch.cuda.empty_cache()
+        result["workloads"] = {}
+        for name in EXTRA_WORKLOADS:
+            r = bench_workload(args, WORKLOADS[name], dev, stream, peaks, peaks_kind, rank, mor,
+                               barrier)
+            result["workloads"][name] = r
+            result["gpu_launches"] += r["gpu_launches"]
+            torch.cuda.empty_cache()
+
     # ---------------- decode workload
     if not args.no_decode:
         result["decode"] = bench_decode(args, dev, stream, peaks, peaks_kind, world, rank,
@@ -386,6 +404,84 @@ def run_ours(args):
         dist.destroy_process_group()
     if rank == 0:
         print(json.dumps(result), flush=True)
+
+
+EXTRA_WORKLOADS = ("pkda_bf16_8k", "fg2_bf16_32k", "gdn2_bf16_32k")
+
+
+def profiled_kernel_ms(pdn, prob, tens, ws, sptr, reps=3):
+    """Mean per-stage milliseconds of pdn_chunk_fwd (CUDA events between its
+    kernels, outside the timed region): key-energy prefix, intra-chunk
+    kernel, state kernel."""
+    acc = None
+    for _ in range(reps):
+        rc, ms = pdn.pdn_chunk_fwd_profiled(prob, tens, ws.data_ptr(), ws.numel(), sptr)
+        if rc != pdn.PDN_OK:
+            raise pdn.PdnError(rc, "pdn_chunk_fwd_profiled")
+        acc = ms if acc is None else [a + b for a, b in zip(acc, ms)]
+    names = ["k0_key_energy", "k1_intra", "k2_state"] if len(acc) == 3 else ["chunk_simt"]
+    return {n: v / reps for n, v in zip(names, acc)}
+
+
+def bench_workload(args, w, dev, stream, peaks, peaks_kind, rank, mor, barrier):
+    """Times `args.steps` forward calls of workload w (inputs resident in HBM
+    and larger than L2, so no flush), after warm-up."""
+    import torch
+
+    from linear_recurrence_sequence_chunked_b200 import pdn
+    from linear_recurrence_sequence_chunked_b200.workloads import make_inputs
+
+    wr = w.replace(seed=rank_seed(w.seed, rank))
+    x = make_inputs(wr, device=dev, generator_device=dev)
+    g = {n: x[n] for n in ("log_alpha", "beta", "erase", "write")}
+    o = torch.empty(w.B, w.T, w.H, w.dv, dtype=x["v"].dtype, device=dev)
+    prob = pdn.make_problem(w.variant, w.B, w.T, w.H, w.dk, w.dv, x["k"].dtype, w.decay, w.chunk,
+                            "auto", w.q_scale, w.precond_x, w.precond_eps)
+    ws_bytes = pdn.pdn_chunk_fwd_workspace(prob)
+    ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
+    ST = torch.empty(w.B, w.H, w.dv, w.dk, dtype=torch.float32, device=dev)
+    AT = torch.empty(w.B, w.H, w.dk, dtype=torch.float32, device=dev) \
+        if w.variant in pdn.PRECOND_VARIANTS else None
+    tens = pdn.make_tensors(x["q"], x["k"], x["v"], o, **g, ST=ST, AT=AT)
+    sptr = stream.cuda_stream
+
+    def step():
+        rc = pdn.pdn_chunk_fwd(prob, tens, ws.data_ptr(), ws.numel(), sptr)
+        if rc != pdn.PDN_OK:
+            raise pdn.PdnError(rc, "pdn_chunk_fwd")
+
+    for _ in range(args.warmup):
+        step()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    barrier()
+    ms_local = e0.elapsed_time(e1)
+    ms = mor(ms_local)
+    if pdn.device_error() != pdn.PDN_OK:
+        raise SystemExit("device error during the %s timed region" % w.name)
+    per = ms_local / args.steps
+    flops = chunk_flops_per_token_head(w.chunk, w.dk, w.dv) * w.B * w.T * w.H
+    nbytes = fwd_bytes_per_token_head(w) * w.B * w.T * w.H + 4 * w.B * w.H * w.dv * w.dk
+    launches = 4 if w.variant in pdn.PRECOND_VARIANTS else 2
+    res = {"variant": w.variant, "B": w.B, "T": w.T, "H": w.H, "d": w.dk, "inputs": w.dtype,
+           "value": w.B * w.T * args.steps / (ms / 1e3), "unit": "tokens/s",
+           "ms_per_step": ms / args.steps,
+           "tensor": {"achieved": flops / (per / 1e3) / 1e12, "peak": peaks["bf16_tflops"],
+                      "unit": "TFLOP/s", "frac": flops / (per / 1e3) / 1e12 / peaks["bf16_tflops"],
+                      "flops_per_launch": flops},
+           "hbm": {"achieved": nbytes / (per / 1e3) / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                   "frac": nbytes / (per / 1e3) / 1e9 / peaks["hbm_gbs"],
+                   "bytes_per_launch": nbytes},
+           "peak_kind": peaks_kind,
+           "kernel_ms": profiled_kernel_ms(pdn, prob, tens, ws, sptr),
+           "l2": "inputs larger than L2 (no flush)",
+           "gpu_launches": args.steps * launches}
+    del x, g, o, ws, ST, AT, tens
+    return res
 
 
 def bench_decode(args, dev, stream, peaks, peaks_kind, world, rank, mor, barrier):
@@ -488,7 +584,9 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="pgdn_bf16_4k")
-    ap.add_argument("--kernel", choices=["auto", "simt", "tc", "tc_fused"], default="auto")
+    ap.add_argument("--kernel", choices=["auto", "simt", "tc"], default="auto")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="skip the Preconditioned KDA 8k and FG2 / GDN-2 32k workloads")
     ap.add_argument("--decode-steps", type=int, default=1024)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-decode", action="store_true")

@@ -38,6 +38,10 @@
  *     are returned as PDN_ERR_CUDA. Errors detected on the device (a bounded
  *     wait that ran out) are recorded in a per-device error word read by
  *     pdn_get_device_error(). No device code traps.
+ *   - Device addresses the library looks up once per device (the error word,
+ *     the no-alloc scratch array) and the copy streams of pdn_chunk_fwd_host
+ *     belong to the device's primary context: the library must not be used
+ *     across a cudaDeviceReset() of that device.
  */
 #ifndef PDN_H
 #define PDN_H
@@ -80,12 +84,10 @@ typedef enum { PDN_F32 = 0, PDN_BF16 = 1 } pdn_dtype_t;
 
 /* Kernel selection for pdn_chunk_fwd. TC is the tensor-core (tcgen05) path
  * that runs the intra-chunk work of all chunks at once and then the
- * sequential state pass (needs a workspace); TC_FUSED is the single-kernel
- * tensor-core path (no workspace); SIMT is the CUDA-core kernel (any
- * supported shape, fp32 arithmetic). AUTO picks TC, else TC_FUSED, else SIMT.
- * The tensor-core paths take bf16 inputs with d_k = d_v = 128, chunk 64. */
-typedef enum { PDN_IMPL_AUTO = 0, PDN_IMPL_SIMT = 1, PDN_IMPL_TC = 2,
-               PDN_IMPL_TC_FUSED = 3 } pdn_impl_t;
+ * sequential state pass (needs a workspace; bf16 inputs, d_k = d_v = 128,
+ * chunk 64); SIMT is the CUDA-core kernel (any supported shape, fp32
+ * arithmetic). AUTO picks TC where it applies, else SIMT. */
+typedef enum { PDN_IMPL_AUTO = 0, PDN_IMPL_SIMT = 1, PDN_IMPL_TC = 2 } pdn_impl_t;
 
 typedef struct {
   int B, T, H;          /* batch, tokens per sequence, heads; B,H >= 1, T >= 0
@@ -120,9 +122,9 @@ typedef struct {
  * (0 if none; (size_t)-1 if p is invalid). */
 size_t pdn_chunk_fwd_workspace(const pdn_problem_t *p);
 
-/* Which path pdn_chunk_fwd runs for problem p: PDN_IMPL_SIMT, PDN_IMPL_TC or
- * PDN_IMPL_TC_FUSED; -1 if p is invalid or no kernel of this build supports
- * it. Host-only, touches no device. */
+/* Which path pdn_chunk_fwd runs for problem p: PDN_IMPL_SIMT or PDN_IMPL_TC;
+ * -1 if p is invalid or no kernel of this build supports it. Host-only,
+ * touches no device. */
 int pdn_chunk_fwd_impl(const pdn_problem_t *p);
 
 /* Chunked forward over T tokens (prefill / training forward).
@@ -132,6 +134,17 @@ int pdn_chunk_fwd_impl(const pdn_problem_t *p);
  * Returns PDN_OK once the work is enqueued. */
 pdn_status_t pdn_chunk_fwd(const pdn_problem_t *p, const pdn_tensors_t *t,
                            void *workspace, size_t ws_bytes, void *stream);
+
+/* Measurement form of pdn_chunk_fwd: runs the same path on the same
+ * arguments, with CUDA events between its kernels, then synchronises
+ * `stream` and writes the elapsed milliseconds of each stage to kernel_ms
+ * (caller array of at least 3 floats) and their count to *n_kernels:
+ * PDN_IMPL_TC gives 3 (key-energy prefix, intra-chunk kernel, state kernel;
+ * the first is ~0 for variants without a preconditioner), PDN_IMPL_SIMT 1.
+ * Blocking; for benchmarks, not for production calls. */
+pdn_status_t pdn_chunk_fwd_profiled(const pdn_problem_t *p, const pdn_tensors_t *t,
+                                    void *workspace, size_t ws_bytes, void *stream,
+                                    float *kernel_ms, int *n_kernels);
 
 /* Allocation-free chunked forward. The paper has no counterpart: this entry
  * point exists for callers that cannot allocate device memory for a
@@ -153,7 +166,10 @@ pdn_status_t pdn_chunk_fwd(const pdn_problem_t *p, const pdn_tensors_t *t,
  *     contents; calls that overlap on the GPU (different streams or host
  *     threads) race and must be serialised by the caller. Nothing needs
  *     clearing between calls: every scratch byte a call reads it writes
- *     first. */
+ *     first.
+ *   - The array's device address is cached per device; like the device error
+ *     word, it does not survive cudaDeviceReset() (or any other teardown of
+ *     the device's primary context): do not use the library across one. */
 pdn_status_t pdn_chunk_fwd_noalloc(const pdn_problem_t *p, const pdn_tensors_t *t, void *stream);
 
 /* Chunked forward from host memory, end to end: copies the inputs in, runs
@@ -194,9 +210,11 @@ pdn_status_t pdn_get_device_error(void *stream);
 
 /* Self-test of the bounded-wait mechanism every device wait uses: launches
  * one block that waits on an mbarrier nothing arrives on, giving up after
- * `spin_limit` polls. The kernel records PDN_ERR_TIMEOUT in the device error
- * word and returns; the host reads it with pdn_get_device_error(). */
-pdn_status_t pdn_selftest_bounded_wait(long long spin_limit, void *stream);
+ * `limit_ns` nanoseconds of device time (0 <= limit_ns <= 1e10). The kernel
+ * records PDN_ERR_TIMEOUT in the device error word and returns; the host
+ * reads it with pdn_get_device_error(). The library's own waits give up after
+ * two seconds. */
+pdn_status_t pdn_selftest_bounded_wait(long long limit_ns, void *stream);
 
 /* Human-readable name of a status code (static storage). */
 const char *pdn_status_string(pdn_status_t s);

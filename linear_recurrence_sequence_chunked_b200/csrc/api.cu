@@ -32,7 +32,7 @@ int *device_error_word() {
   return g_err_ptr[dev];
 }
 
-bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
+bool aligned(const void *p, uintptr_t a) { return ((uintptr_t)p & (a - 1)) == 0; }
 
 bool head_dim_ok(int d) { return d >= 16 && d <= 128 && d % 16 == 0; }
 
@@ -56,7 +56,7 @@ pdn_status_t check_problem(const pdn_problem_t *p) {
   if ((int)p->variant < PDN_VAR_DN || (int)p->variant > PDN_VAR_GDN2) return PDN_ERR_INVALID_ARG;
   if ((int)p->decay < PDN_DECAY_NONE || (int)p->decay > PDN_DECAY_CHANNEL) return PDN_ERR_INVALID_ARG;
   if (p->dtype != PDN_F32 && p->dtype != PDN_BF16) return PDN_ERR_INVALID_ARG;
-  if ((int)p->impl < PDN_IMPL_AUTO || (int)p->impl > PDN_IMPL_TC_FUSED) return PDN_ERR_INVALID_ARG;
+  if ((int)p->impl < PDN_IMPL_AUTO || (int)p->impl > PDN_IMPL_TC) return PDN_ERR_INVALID_ARG;
   bool fixed;
   const pdn_decay_t need = required_decay(p->variant, &fixed);
   if (fixed && p->decay != need) return PDN_ERR_INVALID_ARG;
@@ -74,10 +74,17 @@ pdn_status_t check_problem(const pdn_problem_t *p) {
 
 pdn_status_t check_tensors(const pdn_problem_t *p, const pdn_tensors_t *t) {
   if (!t) return PDN_ERR_INVALID_ARG;
-  const void *all[] = {t->q, t->k, t->v, t->o, t->log_alpha, t->beta, t->erase,
-                       t->write, t->S0, t->ST, t->A0, t->AT};
-  for (const void *ptr : all)
-    if (ptr && !aligned16(ptr)) return PDN_ERR_INVALID_ARG;
+  // 16-byte alignment for every tensor the kernels read or write in 16-byte
+  // vectors; the fp32 per-(token, head) gates (scalar log decay, scalar beta)
+  // are read one element at a time and need only 4
+  const bool scalar_la = p->decay == PDN_DECAY_SCALAR;
+  const bool scalar_beta = p->variant != PDN_VAR_FG2_GDN && p->variant != PDN_VAR_GDN2;
+  const void *v16[] = {t->q, t->k, t->v, t->o, t->erase, t->write, t->S0, t->ST, t->A0, t->AT,
+                       scalar_la ? nullptr : t->log_alpha, scalar_beta ? nullptr : t->beta};
+  for (const void *ptr : v16)
+    if (ptr && !aligned(ptr, 16)) return PDN_ERR_INVALID_ARG;
+  if (scalar_la && t->log_alpha && !aligned(t->log_alpha, 4)) return PDN_ERR_INVALID_ARG;
+  if (scalar_beta && t->beta && !aligned(t->beta, 4)) return PDN_ERR_INVALID_ARG;
   // With T == 0 the per-token tensors are empty and may be NULL; nothing
   // reads them.
   if (p->T == 0) {
@@ -117,10 +124,8 @@ int select_impl(const pdn_problem_t *p, const KParams &P) {
   switch (p->impl) {
     case PDN_IMPL_SIMT: return simt_supported(P) ? PDN_IMPL_SIMT : -1;
     case PDN_IMPL_TC: return split_supported(P) ? PDN_IMPL_TC : -1;
-    case PDN_IMPL_TC_FUSED: return tc_supported(P) ? PDN_IMPL_TC_FUSED : -1;
     default:
       if (split_supported(P)) return PDN_IMPL_TC;
-      if (tc_supported(P)) return PDN_IMPL_TC_FUSED;
       return simt_supported(P) ? PDN_IMPL_SIMT : -1;
   }
 }
@@ -130,6 +135,24 @@ size_t workspace_for(int impl, const KParams &P) {
 }
 
 }  // namespace
+
+// Everything pdn_chunk_fwd checks before it enqueues work (host-only).
+pdn_status_t check_chunk_fwd(const pdn_problem_t *p, const pdn_tensors_t *t,
+                             const void *workspace, size_t ws_bytes, int *impl_out) {
+  pdn_status_t st = check_problem(p);
+  if (st != PDN_OK) return st;
+  if ((st = check_tensors(p, t)) != PDN_OK) return st;
+  const KParams P = make_params(p, t, nullptr);
+  const int impl = select_impl(p, P);
+  if (impl < 0) return PDN_ERR_UNSUPPORTED;
+  const size_t need = workspace_for(impl, P);
+  if (need > 0) {
+    if (!workspace || ws_bytes < need || ((uintptr_t)workspace & 255u)) return PDN_ERR_WORKSPACE;
+  }
+  if (impl_out) *impl_out = impl;
+  return PDN_OK;
+}
+
 }  // namespace pdn
 
 using namespace pdn;
@@ -153,24 +176,50 @@ extern "C" int pdn_chunk_fwd_impl(const pdn_problem_t *p) {
 
 extern "C" pdn_status_t pdn_chunk_fwd(const pdn_problem_t *p, const pdn_tensors_t *t,
                                       void *workspace, size_t ws_bytes, void *stream) {
-  pdn_status_t st = check_problem(p);
+  int impl = -1;
+  const pdn_status_t st = check_chunk_fwd(p, t, workspace, ws_bytes, &impl);
   if (st != PDN_OK) return st;
-  if ((st = check_tensors(p, t)) != PDN_OK) return st;
   KParams P = make_params(p, t, nullptr);
-  const int impl = select_impl(p, P);
-  if (impl < 0) return PDN_ERR_UNSUPPORTED;
-  const size_t need = workspace_for(impl, P);
-  if (need > 0) {
-    if (!workspace || ws_bytes < need || ((uintptr_t)workspace & 255u)) return PDN_ERR_WORKSPACE;
-  }
   P.err = device_error_word();
   if (!P.err) return PDN_ERR_CUDA;
   const cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaError_t e;
   if (impl == PDN_IMPL_TC) e = launch_chunk_split(P, workspace, s);
-  else if (impl == PDN_IMPL_TC_FUSED) e = launch_chunk_tc(P, workspace, s);
   else e = launch_chunk_simt(P, s);
   return e == cudaSuccess ? PDN_OK : PDN_ERR_CUDA;
+}
+
+extern "C" pdn_status_t pdn_chunk_fwd_profiled(const pdn_problem_t *p, const pdn_tensors_t *t,
+                                               void *workspace, size_t ws_bytes, void *stream,
+                                               float *kernel_ms, int *n_kernels) {
+  if (!kernel_ms || !n_kernels) return PDN_ERR_INVALID_ARG;
+  int impl = -1;
+  const pdn_status_t st = check_chunk_fwd(p, t, workspace, ws_bytes, &impl);
+  if (st != PDN_OK) return st;
+  KParams P = make_params(p, t, nullptr);
+  P.err = device_error_word();
+  if (!P.err) return PDN_ERR_CUDA;
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaEvent_t ev[4] = {};
+  cudaError_t e = cudaSuccess;
+  for (int i = 0; i < 4 && e == cudaSuccess; ++i) e = cudaEventCreate(&ev[i]);
+  if (e == cudaSuccess) {
+    if (impl == PDN_IMPL_TC) {
+      e = launch_chunk_split(P, workspace, s, ev);
+    } else {
+      e = cudaEventRecord(ev[0], s);
+      if (e == cudaSuccess) e = launch_chunk_simt(P, s);
+      if (e == cudaSuccess) e = cudaEventRecord(ev[1], s);
+    }
+  }
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  const int n = impl == PDN_IMPL_TC ? 3 : 1;
+  for (int i = 0; i < n && e == cudaSuccess; ++i) e = cudaEventElapsedTime(&kernel_ms[i], ev[i], ev[i + 1]);
+  for (int i = 0; i < 4; ++i)
+    if (ev[i]) cudaEventDestroy(ev[i]);
+  if (e != cudaSuccess) return PDN_ERR_CUDA;
+  *n_kernels = n;
+  return PDN_OK;
 }
 
 extern "C" pdn_status_t pdn_decode_step(const pdn_problem_t *p, const pdn_tensors_t *t,
@@ -198,11 +247,11 @@ extern "C" pdn_status_t pdn_get_device_error(void *stream) {
   return static_cast<pdn_status_t>(v);
 }
 
-extern "C" pdn_status_t pdn_selftest_bounded_wait(long long spin_limit, void *stream) {
-  if (spin_limit < 0) return PDN_ERR_INVALID_ARG;
+extern "C" pdn_status_t pdn_selftest_bounded_wait(long long limit_ns, void *stream) {
+  if (limit_ns < 0 || limit_ns > 10000000000LL) return PDN_ERR_INVALID_ARG;
   int *w = device_error_word();
   if (!w) return PDN_ERR_CUDA;
-  return launch_selftest_wait(spin_limit, w, static_cast<cudaStream_t>(stream)) == cudaSuccess
+  return launch_selftest_wait(limit_ns, w, static_cast<cudaStream_t>(stream)) == cudaSuccess
              ? PDN_OK : PDN_ERR_CUDA;
 }
 

@@ -11,14 +11,16 @@
 // (I + T)^{-1} solve; "Preconditioned DeltaNet", ja §2.3, prefix-sum
 // preconditioner inside the chunk form):
 //   G_t    = sum_{s<=t} log alpha_s                 (per key channel)
-//   Rh     = e^{G} . r,  Wh = e^{-G} . w,  Qh = q_scale e^{G} . q,
-//   Wb     = e^{G_C - G} . w
-//   M      = strict_lower(Rh Wh^T),  P = lower(Qh Wh^T)
+//   M_ts   = sum_i r_ti w_si e^{G_ti - G_si}  (s < t)
+//   P_ts   = q_scale sum_i q_ti w_si e^{G_ti - G_si}  (s <= t)
+//   Rh     = e^{G} . r,  Qh = q_scale e^{G} . q,  Wb = e^{G_C - G} . w
 //   Delta  = (I + M)^{-1} (U - Rh S0^T)             (forward substitution)
 //   O      = Qh S0^T + P Delta
 //   S_C    = S0 Diag(e^{G_C}) + Delta^T Wb
-// The exponent factorisation needs the in-chunk cumulative log decay of each
-// channel to stay above about -87 (fp32 range of e^{-G}).
+// Every decay factor is e^{x} with x <= 0, so no decay strength leaves the
+// fp32 range (the factorised form e^{G_t} e^{-G_s} would overflow once a
+// channel decays by more than e^{-87} inside a chunk). Channel decay costs
+// one exponential per (t, s, i) term of M and P; scalar decay one per (t, s).
 #include "common.cuh"
 #include "internal.h"
 
@@ -35,11 +37,11 @@ constexpr int kLDC = kMaxC + 1;
 
 struct Smem {
   float R[kMaxC][kLD];   // raw k, then Rh
-  float W[kMaxC][kLD];   // log(A + eps), then Wh
+  float W[kMaxC][kLD];   // log(A + eps), then w, then Wb
   float Q[kMaxC][kLD];   // raw q, then Qh
-  float G[kMaxC][kLD];   // cumulative log decay, then Wb
-  float M[kMaxC][kLDC];  // strict lower Rh Wh^T
-  float Pm[kMaxC][kLDC]; // lower Qh Wh^T
+  float G[kMaxC][kLD];   // cumulative log decay
+  float M[kMaxC][kLDC];  // M (strict lower)
+  float Pm[kMaxC][kLDC]; // P (lower)
   float U[kMaxC][kLDU];  // u, then RHS, then Delta
   float S[kDVB][kLD];    // state block (rows j0.., all key channels)
   float A[kMaxD];        // preconditioner accumulator carry
@@ -107,8 +109,10 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_simt_kernel(const KParams P
     for (int i = tid; i < dk; i += kThreads) {
       float g = 0.f, a = sm.A[i];
       for (int t = 0; t < C; ++t) {
-        const float la = P.decay == PDN_DECAY_CHANNEL ? sm.G[t][i]
-                         : P.decay == PDN_DECAY_SCALAR ? sm.la[t] : 0.f;
+        // a log decay below -100 is raised to it: e^{-100} is below the
+        // smallest normal fp32 number, so every factor it enters stays zero
+        const float la = fmaxf(P.decay == PDN_DECAY_CHANNEL ? sm.G[t][i]
+                               : P.decay == PDN_DECAY_SCALAR ? sm.la[t] : 0.f, -100.f);
         g += la;
         sm.G[t][i] = g;
         if (precond) {
@@ -133,7 +137,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_simt_kernel(const KParams P
       __syncthreads();
     }
 
-    // (d) read key r, write key w, decay factors
+    // (d) read key r, write key w, scaled query (undecayed)
     for (int idx = tid; idx < C * dk; idx += kThreads) {
       const int t = idx / dk, i = idx % dk;
       const bool ok = t < Cn;
@@ -156,12 +160,9 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_simt_kernel(const KParams P
         default:
           w = sm.beta[t] * kv;
       }
-      const float g = sm.G[t][i];
-      const float eg = expf(g);
-      sm.R[t][i] = r * eg;
-      sm.W[t][i] = w * expf(-g);
-      sm.Q[t][i] = P.q_scale * sm.Q[t][i] * eg;
-      sm.G[t][i] = w * expf(sm.GC[i] - g);
+      sm.R[t][i] = r;
+      sm.W[t][i] = w;
+      sm.Q[t][i] = P.q_scale * sm.Q[t][i];
     }
     if (P.variant == PDN_VAR_FG2_GDN || P.variant == PDN_VAR_GDN2) {
       for (int idx = tid; idx < C * kDVB; idx += kThreads) {
@@ -176,21 +177,47 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_simt_kernel(const KParams P
     }
     __syncthreads();
 
-    // (e) M = strict_lower(Rh Wh^T), P = lower(Qh Wh^T); RHS = U - Rh S^T
+    // (e) M and P with their in-chunk decay e^{G_t - G_s} <= 1
     {
       const int t = tid >> 2, p = tid & 3;  // 64 rows x 4 lanes, 16 columns each
       if (t < C) {
         float am[16], ap[16];
 #pragma unroll
         for (int m = 0; m < 16; ++m) { am[m] = 0.f; ap[m] = 0.f; }
-        for (int i = 0; i < dk; ++i) {
-          const float rt = sm.R[t][i], qt = sm.Q[t][i];
+        if (P.decay == PDN_DECAY_CHANNEL) {
+          for (int i = 0; i < dk; ++i) {
+            const float rt = sm.R[t][i], qt = sm.Q[t][i], gt = sm.G[t][i];
 #pragma unroll
-          for (int m = 0; m < 16; ++m) {
-            const int s = p + 4 * m;
-            const float ws = s < C ? sm.W[s][i] : 0.f;
-            am[m] = fmaf(rt, ws, am[m]);
-            ap[m] = fmaf(qt, ws, ap[m]);
+            for (int m = 0; m < 16; ++m) {
+              const int s = p + 4 * m;
+              if (s <= t) {
+                const float x = sm.W[s][i] * expf(gt - sm.G[s][i]);
+                am[m] = fmaf(rt, x, am[m]);
+                ap[m] = fmaf(qt, x, ap[m]);
+              }
+            }
+          }
+        } else {
+          for (int i = 0; i < dk; ++i) {
+            const float rt = sm.R[t][i], qt = sm.Q[t][i];
+#pragma unroll
+            for (int m = 0; m < 16; ++m) {
+              const int s = p + 4 * m;
+              const float ws = s < C ? sm.W[s][i] : 0.f;
+              am[m] = fmaf(rt, ws, am[m]);
+              ap[m] = fmaf(qt, ws, ap[m]);
+            }
+          }
+          if (P.decay == PDN_DECAY_SCALAR) {
+#pragma unroll
+            for (int m = 0; m < 16; ++m) {
+              const int s = p + 4 * m;
+              if (s <= t) {
+                const float f = expf(sm.G[t][0] - sm.G[s][0]);
+                am[m] *= f;
+                ap[m] *= f;
+              }
+            }
           }
         }
 #pragma unroll
@@ -203,6 +230,21 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_simt_kernel(const KParams P
         }
       }
     }
+    __syncthreads();
+    // decayed operands of the state terms: Rh = e^{G} r, Qh = e^{G} q,
+    // Wb = e^{G_C - G} w (all factors <= 1)
+    if (P.decay != PDN_DECAY_NONE) {
+      for (int idx = tid; idx < C * dk; idx += kThreads) {
+        const int t = idx / dk, i = idx % dk;
+        const float g = sm.G[t][i];
+        const float eg = expf(g);
+        sm.R[t][i] *= eg;
+        sm.Q[t][i] *= eg;
+        sm.W[t][i] *= expf(sm.GC[i] - g);
+      }
+      __syncthreads();
+    }
+    // RHS = U - Rh S^T
     for (int idx = tid; idx < C * kDVB; idx += kThreads) {
       const int t = idx / kDVB, jj = idx % kDVB;
       float acc = 0.f;
@@ -243,7 +285,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_simt_kernel(const KParams P
     for (int idx = tid; idx < kDVB * dk; idx += kThreads) {
       const int jj = idx / dk, i = idx % dk;
       float acc = sm.S[jj][i] * sm.EGC[i];
-      for (int t = 0; t < C; ++t) acc = fmaf(sm.U[t][jj], sm.G[t][i], acc);
+      for (int t = 0; t < C; ++t) acc = fmaf(sm.U[t][jj], sm.W[t][i], acc);
       sm.S[jj][i] = acc;
     }
     __syncthreads();

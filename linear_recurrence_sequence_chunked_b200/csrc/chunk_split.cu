@@ -22,23 +22,6 @@
 #include "ptx.cuh"
 #include "tiles.cuh"
 
-// Phase boundary hooks for out-of-tree timing harnesses; empty in the library.
-#ifndef PDN_K1_MARK
-#define PDN_K1_MARK(k)
-#endif
-#ifndef PDN_K2_MARK
-#define PDN_K2_MARK(k)
-#endif
-#ifndef PDN_K2_IMARK
-#define PDN_K2_IMARK(k)
-#endif
-#ifndef PDN_K2_HMARK
-#define PDN_K2_HMARK(k)
-#endif
-#ifndef PDN_K2_WMARK
-#define PDN_K2_WMARK(k)
-#endif
-
 namespace pdn {
 namespace {
 
@@ -63,10 +46,8 @@ __device__ __forceinline__ uint8_t *ws_block(void *ws, int bh, int BH, int c) {
   return reinterpret_cast<uint8_t *>(ws) + ((size_t)c * BH + bh) * WS_CH;
 }
 
-constexpr long long kSpin = 1LL << 22;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
-constexpr float kMinG = -80.f;
 
 // ===========================================================================
 // K0: per-chunk key energy, then the exclusive prefix over chunks
@@ -165,46 +146,80 @@ __global__ void __launch_bounds__(kD * kK0Groups) k0_prefix(const KParams P, voi
 }
 
 // ===========================================================================
-// K1: intra-chunk work, one CTA per (batch, head, chunk)
+// K1: intra-chunk work, persistent over the (chunk, batch, head) blocks
 // ===========================================================================
 constexpr int kK1Threads = 256;
-constexpr int LB_LD = 132;                        // floats per row of the prep buffers
+constexpr int LB_LD = 132;                        // floats per row of the fp32 prep buffer
 constexpr int MS_LD = 68, TS_LD = 68, YS_LD = 34; // fp32 solve scratch strides
-constexpr uint32_t K1_RQ = 0;                     // TL 128 x 128: Rh rows 0-63, Qh rows 64-127
-constexpr uint32_t K1_WH = 32768;                 // TL 64 x 128
-constexpr uint32_t K1_RA = 49152;                 // region A
 constexpr uint32_t KS_LD = 272;                   // staged row stride (bytes), padded
-constexpr uint32_t K1_KS = K1_RA;                 // prep: raw k, row-major [64][128] bf16
-constexpr uint32_t K1_QS = K1_RA + 64 * KS_LD;    // prep: raw q
-constexpr uint32_t K1_BC = K1_QS + 64 * KS_LD;    // prep: preconditioner coefficient B, bf16
-constexpr uint32_t K1_GBUF = K1_BC + 64 * KS_LD;  // prep: cumulative log decay, fp32 [64][132]
-constexpr uint32_t K1_LAS_STAGE = K1_GBUF + 64 * LB_LD * 4;  // prep: raw channel log decay
-constexpr uint32_t K1_TM = K1_RA;                 // TL 64 x 64
-constexpr uint32_t K1_PM = K1_RA + 8192;          // TL 64 x 64
-constexpr uint32_t K1_MS = K1_RA + 16384;         // fp32 [64][68]
-constexpr uint32_t K1_TS = K1_MS + 64 * MS_LD * 4;// fp32 [64][68]
-constexpr uint32_t K1_YS = K1_TS + 64 * TS_LD * 4;// fp32 [32][34]
-constexpr uint32_t K1_YT = K1_RA + 16384;         // TL 128 x 64 (after the solve)
-constexpr uint32_t K1_SOLVE_END = K1_YS + 32 * YS_LD * 4;
 
-// Region A holds the prep buffers the variant needs (staged k and q, the
-// bf16 preconditioner coefficients, the fp32 cumulative log decay and the
-// staged channel log decay), then the solve scratch.
+// In-chunk decay without range limits. G_t is the cumulative log decay from
+// the chunk start (inclusive); every product the chunk form needs is
+// e^{G_t - G_s} with s <= t, at most 1, but its two factors e^{G_t} and
+// e^{-G_s} leave the fp32 range once a channel decays by more than e^{-87}
+// inside the chunk. So:
+//   * scalar decay: MMA1 multiplies the undecayed operands and the epilogue
+//     applies e^{G_t - G_s} per element;
+//   * channel decay: the chunk is cut into four 16-token sub-chunks with
+//     boundary values B_a = G_{16a-1} (B_0 = 0). Row t of sub-chunk a is
+//     scaled by rho_t = e^{G_t - B_a} <= 1 and its columns s by
+//     e^{B_a - G_s}, which is <= 1 for s in an earlier sub-chunk and at most
+//     e^{kSubRange} inside sub-chunk a unless that sub-chunk is flagged; a
+//     flagged sub-chunk's diagonal block is summed pairwise instead. MMA1's
+//     B operand holds one column group per sub-chunk a (the columns
+//     s < 16(a+1), scaled for reference B_a), starting at column grp_off(a).
+// The state-side factors e^{G_t}, e^{G_C - G_s} and e^{G_C} are at most 1
+// and are formed directly. A log decay below kMinLogAlpha per token is
+// raised to it: e^{-100} is below the smallest normal fp32 number, so every
+// factor such a token enters is zero in fp32 either way.
+constexpr float kSubRange = 64.f;
+constexpr float kMinLogAlpha = -100.f;
+__host__ __device__ constexpr int grp_off(int a) { return 8 * a * (a + 1); }
+
 template <int kVariant, int kDecay>
 struct K1Layout {
   static constexpr bool kPre =
       kVariant == PDN_VAR_PDN || kVariant == PDN_VAR_PGDN || kVariant == PDN_VAR_PKDA;
-  static constexpr uint32_t kPrepEnd =
-      kDecay == PDN_DECAY_CHANNEL ? K1_LAS_STAGE + 64 * 256 : K1_GBUF;
-  static constexpr uint32_t kSmall = (kPrepEnd > K1_SOLVE_END ? kPrepEnd : K1_SOLVE_END);
-  static constexpr uint32_t kAcar = kSmall, kGC = kSmall + 512, kEGC = kSmall + 1024;
+  static constexpr bool kCh = kDecay == PDN_DECAY_CHANNEL;
+  static constexpr int kN1 = kCh ? 160 : 64;                // columns of MMA1
+  static constexpr uint32_t kRQ = 0;                        // TL 128 x 128: R rows 0-63, Q rows 64-127
+  static constexpr uint32_t kWH = 32768;                    // TL kN1 x 128: MMA1's B operand
+  static constexpr uint32_t kRA = kWH + kN1 * 256;          // region A
+  // region A during the prep: staged k and q, the bf16 preconditioner
+  // coefficients, the fp32 cumulative log decay and the staged channel log
+  // decay (channel decay)
+  static constexpr uint32_t kKS = kRA;
+  static constexpr uint32_t kQS = kKS + 64 * KS_LD;
+  static constexpr uint32_t kBC = kQS + 64 * KS_LD;
+  static constexpr uint32_t kGBUF = kBC + 64 * KS_LD;
+  static constexpr uint32_t kLasStage = kGBUF + 64 * LB_LD * 4;
+  static constexpr uint32_t kPrepEnd = kCh ? kLasStage + 64 * 256 : kGBUF;
+  // region A from the epilogue of MMA1 on: T and P tiles, the fp32 solve
+  // scratch, then the Y^T tile
+  static constexpr uint32_t kTM = kRA;                      // TL 64 x 64
+  static constexpr uint32_t kPM = kRA + 8192;               // TL 64 x 64
+  static constexpr uint32_t kMS = kRA + 16384;              // fp32 [64][68]
+  static constexpr uint32_t kTS = kMS + 64 * MS_LD * 4;     // fp32 [64][68]
+  static constexpr uint32_t kYS = kTS + 64 * TS_LD * 4;     // fp32 [32][34]
+  static constexpr uint32_t kYT = kRA + 16384;              // TL 128 x 64
+  static constexpr uint32_t kSolveEnd = kYS + 32 * YS_LD * 4;
+  static constexpr uint32_t kSmall = (kPrepEnd > kSolveEnd ? kPrepEnd : kSolveEnd);
+  static constexpr uint32_t kAcar = kSmall, kGC = kSmall + 512;
   // float[3][128]: sums over token quarters 0..2 of k.k and of the log decay
   static constexpr uint32_t kPartK = kSmall + 1536, kPartG = kSmall + 3072;
   static constexpr uint32_t kMup = kSmall + 4608;  // float[2][64] per channel-half partial means
   static constexpr uint32_t kMu = kSmall + 5120, kBeta = kSmall + 5376, kGS = kSmall + 5632;
-  static constexpr uint32_t kLas = kSmall + 5888, kBar = kSmall + 6144;
-  static constexpr uint32_t kTbase = kSmall + 6160;
-  static constexpr uint32_t kBytes = kSmall + 6176;
+  static constexpr uint32_t kLas = kSmall + 5888;
+  static constexpr uint32_t kEGS = kSmall + 6144;  // float[64] e^{G_t}, scalar decay
+  // channel decay, float[9][128]: e^{B_1}, e^{B_2}, e^{B_3}, e^{B_2 - B_1},
+  // e^{B_3 - B_1}, e^{B_3 - B_2}, e^{G_C - B_1}, e^{G_C - B_2}, e^{G_C - B_3}
+  static constexpr uint32_t kTab = kSmall + 6400;
+  static constexpr uint32_t kFlags = kTab + (kCh ? 9 * 512 : 0);  // bit a: sub-chunk a flagged
+  static constexpr uint32_t kBar = kFlags + 16;
+  static constexpr uint32_t kTbase = kBar + 16;
+  static constexpr uint32_t kBytes = kTbase + 16;
+  static constexpr uint32_t kTmemCols = kCh ? 256 : 128;
+  static constexpr uint32_t kTmY = kN1;  // TMEM column of Y^T (after MMA1's columns)
 };
 
 __device__ __forceinline__ void sync_for_mma() {
@@ -214,16 +229,52 @@ __device__ __forceinline__ void sync_for_mma() {
   tc_fence_after();
 }
 
+// Exact diagonal-block entries of row t against columns s0 .. s0 + 15 of a
+// flagged sub-chunk: sum_c x_tc w_sc e^{G_tc - G_sc} for s <= t (s < t when
+// `strict`), from the undecayed bf16 rows x (row t) and w (rows s) and the
+// fp32 cumulative log decay.
+__device__ __forceinline__ void diag_exact(const uint8_t *xrow, const uint8_t *wbase,
+                                           const float *gbuf, int t, int s0, bool strict,
+                                           float (&out)[16]) {
+  float acc[16];
+#pragma unroll
+  for (int e = 0; e < 16; ++e) acc[e] = 0.f;
+  const float *gt = gbuf + t * LB_LD;
+  for (int c8 = 0; c8 < 16; ++c8) {
+    float xf[8], gtv[8];
+    unpack8(*reinterpret_cast<const uint4 *>(xrow + 16 * c8), xf);
+    ld8f(gt + 8 * c8, gtv);
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+      const int s = s0 + e;
+      if (s <= t) {
+        float wf[8], gs[8];
+        unpack8(*reinterpret_cast<const uint4 *>(wbase + s * KS_LD + 16 * c8), wf);
+        ld8f(gbuf + s * LB_LD + 8 * c8, gs);
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          acc[e] = fmaf(xf[k] * wf[k], ex2_approx((gtv[k] - gs[k]) * kLog2e), acc[e]);
+      }
+    }
+  }
+#pragma unroll
+  for (int e = 0; e < 16; ++e) {
+    const int s = s0 + e;
+    out[e] = (s < t || (!strict && s == t)) ? acc[e] : 0.f;
+  }
+}
+
 template <int kVariant, int kDecay>
-__global__ void __launch_bounds__(kK1Threads, 2) k1_intra(const KParams P, void *ws, int N) {
+__global__ void __launch_bounds__(kK1Threads, kDecay == PDN_DECAY_CHANNEL ? 1 : 2) k1_intra(const KParams P, void *ws, int N) {
   using L = K1Layout<kVariant, kDecay>;
   constexpr bool kPre = L::kPre;
+  constexpr bool kCh = L::kCh;
+  constexpr bool kSc = kDecay == PDN_DECAY_SCALAR;
   constexpr bool kScalarBeta = kVariant != PDN_VAR_FG2_GDN && kVariant != PDN_VAR_GDN2;
   extern __shared__ __align__(1024) uint8_t smem[];
   const uint32_t sb = smem_u32(smem);
   float *Acar = reinterpret_cast<float *>(smem + L::kAcar);
   float *GC = reinterpret_cast<float *>(smem + L::kGC);
-  float *EGC = reinterpret_cast<float *>(smem + L::kEGC);
   float *PARTK = reinterpret_cast<float *>(smem + L::kPartK);
   float *PARTG = reinterpret_cast<float *>(smem + L::kPartG);
   float *MUP = reinterpret_cast<float *>(smem + L::kMup);
@@ -231,12 +282,15 @@ __global__ void __launch_bounds__(kK1Threads, 2) k1_intra(const KParams P, void 
   float *BETA = reinterpret_cast<float *>(smem + L::kBeta);
   float *GS = reinterpret_cast<float *>(smem + L::kGS);
   float *LAS = reinterpret_cast<float *>(smem + L::kLas);
+  float *EGS = reinterpret_cast<float *>(smem + L::kEGS);
+  float *TAB = reinterpret_cast<float *>(smem + L::kTab);
+  uint32_t *flags = reinterpret_cast<uint32_t *>(smem + L::kFlags);
   uint64_t *bar = reinterpret_cast<uint64_t *>(smem + L::kBar);
   uint32_t *tbase_p = reinterpret_cast<uint32_t *>(smem + L::kTbase);
-  float *GBUF = reinterpret_cast<float *>(smem + K1_GBUF);
-  float *MS = reinterpret_cast<float *>(smem + K1_MS);
-  float *TS = reinterpret_cast<float *>(smem + K1_TS);
-  float *YS = reinterpret_cast<float *>(smem + K1_YS);
+  float *GBUF = reinterpret_cast<float *>(smem + L::kGBUF);
+  float *MS = reinterpret_cast<float *>(smem + L::kMS);
+  float *TS = reinterpret_cast<float *>(smem + L::kTS);
+  float *YS = reinterpret_cast<float *>(smem + L::kYS);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const size_t tstride = (size_t)P.H * kD;
@@ -247,7 +301,7 @@ __global__ void __launch_bounds__(kK1Threads, 2) k1_intra(const KParams P, void 
   const int total = N * BH;  // chunk blocks, chunk-major: block index = c * BH + bh
 
   if (warp == 0) {
-    tmem_alloc(tbase_p, 128);
+    tmem_alloc(tbase_p, L::kTmemCols);
     tmem_relinquish();
   }
   if (tid == 0) {
@@ -276,14 +330,15 @@ __global__ void __launch_bounds__(kK1Threads, 2) k1_intra(const KParams P, void 
     if (tid < kC && tid < Cn_) {
       const size_t e = tok_index(P, b_, c0_ + tid, h_);
       if (kScalarBeta) r.beta = __ldg(reinterpret_cast<const float *>(P.beta) + e);
-      if (kDecay == PDN_DECAY_SCALAR) r.las = __ldg(reinterpret_cast<const float *>(P.log_alpha) + e);
+      if (kSc) r.las = fmaxf(__ldg(reinterpret_cast<const float *>(P.log_alpha) + e), kMinLogAlpha);
     }
     r.acar = (kPre && tid < kD) ? reinterpret_cast<const float *>(ws_block(ws, bh_, P.B * P.H, c_) + WS_A)[tid] : 0.f;
     return r;
   };
-  // v of a chunk block into the Wh tile's space, rows of 256 bytes with the
-  // 16-byte groups XOR-swizzled by (token & 7); issued while the previous
-  // block is in its solve (the Wh tile is dead once MMA1 has completed).
+  // v of a chunk block into the first 16 KiB of the B-operand space, rows of
+  // 256 bytes with the 16-byte groups XOR-swizzled by (token & 7); issued
+  // while the previous block is in its solve (the B operand is dead once
+  // MMA1 has completed).
   auto stage_v = [&](int it) {
     const int c_ = it / BH, bh_ = it % BH;
     const int b_ = bh_ / P.H, h_ = bh_ % P.H;
@@ -294,13 +349,13 @@ __global__ void __launch_bounds__(kK1Threads, 2) k1_intra(const KParams P, void 
       const int t = (tid >> 4) + 16 * m, c8 = tid & 15;
       const bool ok = t < Cn_;
       const size_t e = ok ? tok0_ + (size_t)t * tstride + c8 * 8 : 0;
-      cp_async16(sb + K1_WH + t * 256 + ((c8 ^ (t & 7)) << 4),
+      cp_async16(sb + L::kWH + t * 256 + ((c8 ^ (t & 7)) << 4),
                  reinterpret_cast<const __nv_bfloat16 *>(P.v) + e, ok);
     }
     cp_async_commit();
   };
-  // k of a chunk block into the Rh half of the [Rh; Qh] tile's space (same
-  // swizzled rows); issued once MMA2 of the previous block has read Rh.
+  // k of a chunk block into the R half of the [R; Q] tile's space (same
+  // swizzled rows); issued once MMA2 of the previous block has read R.
   auto stage_k = [&](int it) {
     const int c_ = it / BH, bh_ = it % BH;
     const int b_ = bh_ / P.H, h_ = bh_ % P.H;
@@ -311,7 +366,7 @@ __global__ void __launch_bounds__(kK1Threads, 2) k1_intra(const KParams P, void 
       const int t = (tid >> 4) + 16 * m, c8 = tid & 15;
       const bool ok = t < Cn_;
       const size_t e = ok ? tok0_ + (size_t)t * tstride + c8 * 8 : 0;
-      cp_async16(sb + K1_RQ + t * 256 + ((c8 ^ (t & 7)) << 4),
+      cp_async16(sb + L::kRQ + t * 256 + ((c8 ^ (t & 7)) << 4),
                  reinterpret_cast<const __nv_bfloat16 *>(P.k) + e, ok);
     }
     cp_async_commit();
@@ -330,7 +385,6 @@ __global__ void __launch_bounds__(kK1Threads, 2) k1_intra(const KParams P, void 
   const size_t tok0 = tok_index(P, b, c0, h) * kD;  // element offset of token c0
   uint8_t *blk = ws_block(ws, bh, P.B * P.H, c);
   const uint32_t par = (uint32_t)(iter & 1);  // mbarrier parity of this block's MMAs
-  PDN_K1_MARK(0);
 
   // ---- P0: k (staged a block ahead) into its padded rows; q (and the
   // channel log decay) by cp.async, q awaited only before P3; the prefetched
@@ -343,17 +397,17 @@ __global__ void __launch_bounds__(kK1Threads, 2) k1_intra(const KParams P, void 
 #pragma unroll
     for (int m = 0; m < 4; ++m) {
       const int t = (tid >> 4) + 16 * m, c8 = tid & 15;
-      *reinterpret_cast<uint4 *>(smem + K1_KS + t * KS_LD + c8 * 16) =
-          *reinterpret_cast<const uint4 *>(smem + K1_RQ + t * 256 + ((c8 ^ (t & 7)) << 4));
+      *reinterpret_cast<uint4 *>(smem + L::kKS + t * KS_LD + c8 * 16) =
+          *reinterpret_cast<const uint4 *>(smem + L::kRQ + t * 256 + ((c8 ^ (t & 7)) << 4));
       {
         const bool ok = t < Cn;
         const size_t e = ok ? tok0 + (size_t)t * tstride + c8 * 8 : 0;
-        cp_async16(sb + K1_QS + t * KS_LD + c8 * 16, reinterpret_cast<const __nv_bfloat16 *>(P.q) + e, ok);
+        cp_async16(sb + L::kQS + t * KS_LD + c8 * 16, reinterpret_cast<const __nv_bfloat16 *>(P.q) + e, ok);
       }
-      if (kDecay == PDN_DECAY_CHANNEL) {
+      if (kCh) {
         const bool ok = t < Cn;
         const size_t e = ok ? tok0 + (size_t)t * tstride + c8 * 8 : 0;
-        cp_async16(sb + K1_LAS_STAGE + t * 256 + c8 * 16,
+        cp_async16(sb + L::kLasStage + t * 256 + c8 * 16,
                    reinterpret_cast<const __nv_bfloat16 *>(P.log_alpha) + e, ok);
       }
     }
@@ -363,11 +417,11 @@ __global__ void __launch_bounds__(kK1Threads, 2) k1_intra(const KParams P, void 
       LAS[tid] = pf.las;
     }
     if (tid < kD) Acar[tid] = pf.acar;
+    if (kCh && tid == 0) *flags = 0u;
   }
   if (it + (int)gridDim.x < total) pf = load_raw(it + gridDim.x);
-  if (kDecay == PDN_DECAY_CHANNEL) cp_async_wait_all();  // P1 scans the channel log decay
+  if (kCh) cp_async_wait_all();  // P1 scans the channel log decay
   __syncthreads();
-  PDN_K1_MARK(1);
 
   // ---- P1: per-channel scans; thread = (channel pair, quarter of the chunk) ----
   // Prefix sums of k.k (accumulator) and of the log decay over the chunk's
@@ -383,19 +437,19 @@ __global__ void __launch_bounds__(kK1Threads, 2) k1_intra(const KParams P, void 
       const int t = t0 + e;
       if (kPre) {
         const float2 kv = __bfloat1622float2(
-            *reinterpret_cast<const __nv_bfloat162 *>(smem + K1_KS + t * KS_LD + i0 * 2));
+            *reinterpret_cast<const __nv_bfloat162 *>(smem + L::kKS + t * KS_LD + i0 * 2));
         k0[e] = kv.x;
         k1[e] = kv.y;
       } else {
         k0[e] = 0.f;
         k1[e] = 0.f;
       }
-      if (kDecay == PDN_DECAY_CHANNEL) {
+      if (kCh) {
         const float2 lv = __bfloat1622float2(
-            *reinterpret_cast<const __nv_bfloat162 *>(smem + K1_LAS_STAGE + t * 256 + i0 * 2));
-        l0[e] = lv.x;
-        l1[e] = lv.y;
-      } else if (kDecay == PDN_DECAY_SCALAR) {
+            *reinterpret_cast<const __nv_bfloat162 *>(smem + L::kLasStage + t * 256 + i0 * 2));
+        l0[e] = fmaxf(lv.x, kMinLogAlpha);
+        l1[e] = fmaxf(lv.y, kMinLogAlpha);
+      } else if (kSc) {
         l0[e] = LAS[t];
         l1[e] = l0[e];
       } else {
@@ -435,18 +489,16 @@ __global__ void __launch_bounds__(kK1Threads, 2) k1_intra(const KParams P, void 
       }
       g0 += l0[e];
       g1 += l1[e];
-      if (kDecay == PDN_DECAY_CHANNEL)
+      if (kCh)
         *reinterpret_cast<float2 *>(GBUF + t * LB_LD + i0) = make_float2(g0, g1);
-      else if (kDecay == PDN_DECAY_SCALAR && p == 0)
+      else if (kSc && p == 0)
         GS[t] = g0;
     }
     if (q4 == 3) {
       GC[i0] = g0;
       GC[i0 + 1] = g1;
-      const float e0 = ex2_approx(fmaxf(g0, kMinG) * kLog2e);
-      const float e1 = ex2_approx(fmaxf(g1, kMinG) * kLog2e);
-      EGC[i0] = e0;
-      EGC[i0 + 1] = e1;
+      const float e0 = ex2_approx(g0 * kLog2e);
+      const float e1 = ex2_approx(g1 * kLog2e);
       *reinterpret_cast<float2 *>(reinterpret_cast<float *>(blk + WS_E) + i0) = make_float2(e0, e1);
     }
     if (kPre) {
@@ -478,33 +530,58 @@ __global__ void __launch_bounds__(kK1Threads, 2) k1_intra(const KParams P, void 
         const float c0 = (k0[e] - mu) * kLn2, c1 = (k1[e] - mu) * kLn2;
         const float s0 = c0 * rcp_approx(1.f + fabsf(c0));
         const float s1 = c1 * rcp_approx(1.f + fabsf(c1));
-        *reinterpret_cast<uint32_t *>(smem + K1_BC + t * KS_LD + i0 * 2) =
+        *reinterpret_cast<uint32_t *>(smem + L::kBC + t * KS_LD + i0 * 2) =
             pack_bf16(ex2_approx(-s0 * log2x_), ex2_approx(-s1 * log2x_));
       }
     }
   }
   // this block's v into registers (operand mapping) before P3 overwrites the
-  // staging space with the Wh tile; q has landed
+  // staging space with the B operand; q has landed
 #pragma unroll
   for (int m = 0; m < 4; ++m) {
     const int t = 8 * warp + (lane & 7), c8 = 4 * m + (lane >> 3);
-    vcur[m] = *reinterpret_cast<const uint4 *>(smem + K1_WH + t * 256 + ((c8 ^ (t & 7)) << 4));
+    vcur[m] = *reinterpret_cast<const uint4 *>(smem + L::kWH + t * 256 + ((c8 ^ (t & 7)) << 4));
   }
   cp_async_wait_all();
   __syncthreads();
-  PDN_K1_MARK(2);
-  PDN_K1_MARK(3);
+  if (kCh) {
+    // per-channel factors between the sub-chunk boundaries, and the flags of
+    // sub-chunks whose decay range exceeds kSubRange in some channel
+    if (tid < kD) {
+      const float B1 = GBUF[15 * LB_LD + tid], B2 = GBUF[31 * LB_LD + tid];
+      const float B3 = GBUF[47 * LB_LD + tid], Gc = GBUF[63 * LB_LD + tid];
+      TAB[0 * kD + tid] = ex2_approx(B1 * kLog2e);
+      TAB[1 * kD + tid] = ex2_approx(B2 * kLog2e);
+      TAB[2 * kD + tid] = ex2_approx(B3 * kLog2e);
+      TAB[3 * kD + tid] = ex2_approx((B2 - B1) * kLog2e);
+      TAB[4 * kD + tid] = ex2_approx((B3 - B1) * kLog2e);
+      TAB[5 * kD + tid] = ex2_approx((B3 - B2) * kLog2e);
+      TAB[6 * kD + tid] = ex2_approx((Gc - B1) * kLog2e);
+      TAB[7 * kD + tid] = ex2_approx((Gc - B2) * kLog2e);
+      TAB[8 * kD + tid] = ex2_approx((Gc - B3) * kLog2e);
+      uint32_t m = 0;
+      if (-B1 > kSubRange) m |= 1u;
+      if (B1 - B2 > kSubRange) m |= 2u;
+      if (B2 - B3 > kSubRange) m |= 4u;
+      if (B3 - Gc > kSubRange) m |= 8u;
+      m = __reduce_or_sync(0xffffffffu, m);
+      if (lane == 0 && m) atomicOr(flags, m);
+    }
+    __syncthreads();
+  }
+  const uint32_t badm = kCh ? *flags : 0u;
 
   // ---- P3: operand tiles, (token, 8-channel) units ----
   {
     const int t = 8 * warp + (lane & 7);
     const bool ok = t < Cn;
     const size_t etok = tok0 + (size_t)t * tstride;
-    float eg_s = 1.f, emg_s = 1.f, ewb_s = 1.f;
-    if (kDecay == PDN_DECAY_SCALAR) {
-      eg_s = ex2_approx(fmaxf(GS[t], kMinG) * kLog2e);
-      emg_s = rcp_approx(eg_s);
-      ewb_s = EGC[0] * emg_s;
+    const int a = t >> 4;  // sub-chunk of the token (channel decay)
+    float eg_s = 1.f, ewb_s = 1.f;
+    if (kSc) {
+      eg_s = ex2_approx(GS[t] * kLog2e);
+      ewb_s = ex2_approx((GC[0] - GS[t]) * kLog2e);
+      if ((lane >> 3) == 0) EGS[t] = eg_s;
     }
     const float be = kScalarBeta ? BETA[t] : 0.f;
     const float qs = P.q_scale;
@@ -513,12 +590,14 @@ __global__ void __launch_bounds__(kK1Threads, 2) k1_intra(const KParams P, void 
       const int c8 = 4 * m + (lane >> 3);
       const int i0 = 8 * c8;
       float kf[8], qf[8], vf[8], r[8], w[8];
-      unpack8(*reinterpret_cast<const uint4 *>(smem + K1_KS + t * KS_LD + c8 * 16), kf);
-      unpack8(*reinterpret_cast<const uint4 *>(smem + K1_QS + t * KS_LD + c8 * 16), qf);
+      unpack8(*reinterpret_cast<const uint4 *>(smem + L::kKS + t * KS_LD + c8 * 16), kf);
+      unpack8(*reinterpret_cast<const uint4 *>(smem + L::kQS + t * KS_LD + c8 * 16), qf);
       unpack8(vcur[m], vf);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) qf[e] *= qs;
       if (kPre) {
         float Bv[8];
-        unpack8(*reinterpret_cast<const uint4 *>(smem + K1_BC + t * KS_LD + c8 * 16), Bv);
+        unpack8(*reinterpret_cast<const uint4 *>(smem + L::kBC + t * KS_LD + c8 * 16), Bv);
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
           r[e] = kf[e];
@@ -561,94 +640,184 @@ __global__ void __launch_bounds__(kK1Threads, 2) k1_intra(const KParams P, void 
           w[e] = be * kf[e];
         }
       }
-      float rh[8], qh[8], wh[8], wb[8];
-      if (kDecay == PDN_DECAY_CHANNEL) {
-        float G[8], E[8];
+      float rr[8], qq[8], wh[8], qh[8], wb[8];
+      if (kCh) {
+        float G[8], Bl[8], Bh[8], eBl[8], wbf[8];
         ld8f(GBUF + t * LB_LD + i0, G);
-        ld8f(EGC + i0, E);
+        ld8f(GBUF + (16 * a + 15) * LB_LD + i0, Bh);  // B_{a+1} (G_C for a = 3)
+        if (a > 0) {
+          ld8f(GBUF + (16 * a - 1) * LB_LD + i0, Bl);
+          ld8f(TAB + (a - 1) * kD + i0, eBl);
+        } else {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) { Bl[e] = 0.f; eBl[e] = 1.f; }
+        }
+        if (a < 3) {
+          ld8f(TAB + (6 + a) * kD + i0, wbf);
+        } else {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) wbf[e] = 1.f;
+        }
+        const bool bad_a = (badm >> a) & 1u;
+        float wy[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
-          const float eg = ex2_approx(fmaxf(G[e], kMinG) * kLog2e);
-          const float emg = rcp_approx(eg);
-          rh[e] = r[e] * eg;
-          qh[e] = qs * qf[e] * eg;
-          wh[e] = w[e] * emg;
-          wb[e] = w[e] * (E[e] * emg);
+          const float rho = ex2_approx((G[e] - Bl[e]) * kLog2e);  // e^{G_t - B_a} <= 1
+          const float y = ex2_approx((Bh[e] - G[e]) * kLog2e);    // e^{B_{a+1} - G_t} <= 1
+          rr[e] = r[e] * rho;
+          qq[e] = qf[e] * rho;
+          qh[e] = qf[e] * (rho * eBl[e]);
+          wb[e] = w[e] * (y * wbf[e]);
+          wh[e] = bad_a ? 0.f : w[e] * rcp_approx(rho);  // diagonal group: e^{B_a - G_t}
+          wy[e] = w[e] * y;
+        }
+        *reinterpret_cast<uint4 *>(smem + L::kWH + tl128(grp_off(a) + t, c8)) = pack8(wh);
+        // later column groups: e^{B_a2 - G_t} = y e^{B_a2 - B_{a+1}}
+#pragma unroll
+        for (int a2 = 1; a2 < 4; ++a2) {
+          if (a2 > a) {
+            float lam[8];
+            if (a2 == a + 1) {
+#pragma unroll
+              for (int e = 0; e < 8; ++e) lam[e] = 1.f;
+            } else {
+              ld8f(TAB + (a == 0 ? (a2 == 2 ? 3 : 4) : 5) * kD + i0, lam);
+            }
+            float x[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) x[e] = wy[e] * lam[e];
+            *reinterpret_cast<uint4 *>(smem + L::kWH + tl128(grp_off(a2) + t, c8)) = pack8(x);
+          }
+        }
+        if (badm) {  // undecayed rows for the exact diagonal blocks
+          *reinterpret_cast<uint4 *>(smem + L::kKS + t * KS_LD + c8 * 16) = pack8(r);
+          *reinterpret_cast<uint4 *>(smem + L::kQS + t * KS_LD + c8 * 16) = pack8(qf);
+          *reinterpret_cast<uint4 *>(smem + L::kBC + t * KS_LD + c8 * 16) = pack8(w);
         }
       } else {
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
-          rh[e] = r[e] * eg_s;
-          qh[e] = (qs * eg_s) * qf[e];
-          wh[e] = w[e] * emg_s;
+          rr[e] = r[e];
+          qq[e] = qf[e];
+          wh[e] = w[e];
+          qh[e] = qf[e] * eg_s;
           wb[e] = w[e] * ewb_s;
         }
+        *reinterpret_cast<uint4 *>(smem + L::kWH + tl128(t, c8)) = pack8(wh);
       }
-      *reinterpret_cast<uint4 *>(smem + K1_RQ + tl128(t, c8)) = pack8(rh);
-      *reinterpret_cast<uint4 *>(smem + K1_RQ + tl128(64 + t, c8)) = pack8(qh);
-      *reinterpret_cast<uint4 *>(smem + K1_WH + tl128(t, c8)) = pack8(wh);
+      *reinterpret_cast<uint4 *>(smem + L::kRQ + tl128(t, c8)) = pack8(rr);
+      *reinterpret_cast<uint4 *>(smem + L::kRQ + tl128(64 + t, c8)) = pack8(qq);
+      *reinterpret_cast<uint4 *>(blk + WS_Q + tl128(t, c8)) = pack8(qh);
       *reinterpret_cast<uint4 *>(blk + WS_WB + tl128(t, c8)) = pack8(wb);
       *reinterpret_cast<uint4 *>(blk + WS_U + tl128(t, c8)) = pack8(vf);
     }
   }
 
-  // ---- MMA1: D1 = [Rh;Qh] Wh^T ----
+  // ---- MMA1: D1 = [R;Q] B^T ----
   sync_for_mma();
-  PDN_K1_MARK(4);
   if (tid == 0) {
-    const uint32_t id = make_idesc_bf16(128, 64, false, false);
+    const uint32_t id = make_idesc_bf16(128, L::kN1, false, false);
 #pragma unroll
     for (int kk = 0; kk < 8; ++kk)
-      mma_bf16_ss(tm + 0, make_sdesc(sb + K1_RQ + 256 * kk, 128, 2048),
-                  make_sdesc(sb + K1_WH + 256 * kk, 128, 2048), id, kk > 0);
+      mma_bf16_ss(tm + 0, make_sdesc(sb + L::kRQ + 256 * kk, 128, 2048),
+                  make_sdesc(sb + L::kWH + 256 * kk, 128, 2048), id, kk > 0);
     mma_commit(bar + 0);
   }
   bool ok_all = true;
   {
     bool ok = true;
-    if (warp == 0) ok = mbar_wait_bounded(bar + 0, par, kSpin);
+    if (warp == 0) ok = mbar_wait_timed(bar + 0, par, kWaitNs);
     ok_all = !__syncthreads_or(!ok);
     tc_fence_after();
   }
-  PDN_K1_MARK(5);
 
   if (ok_all) {
     if (it + (int)gridDim.x < total) stage_v(it + gridDim.x);
-    // ---- solve: M, P from TMEM; T = (I + M)^{-1} ----
-    {
-      const int row = 32 * (warp & 3) + lane;
+    // ---- epilogue of MMA1: M = strict lower (rows 0-63), P = lower (rows
+    // 64-127) with their in-chunk decay, first into registers ----
+    const int row = 32 * (warp & 3) + lane;
+    const int tr = row & 63;
+    const bool isP = row >= 64;
+    float mv[2][16];
+    if (kCh) {
+      const int alo = 2 * (warp & 1);  // sub-chunks alo (lanes 0-15), alo + 1 (lanes 16-31)
+      const int a = alo + (lane >> 4);
+      const bool lo = lane < 16;
 #pragma unroll
       for (int cc = 0; cc < 2; ++cc) {
-        float v[16];
-        tmem_ld16(tm + lane_q + 32 * half + 16 * cc, v);
-        tmem_wait_ld();
         const int s0 = 32 * half + 16 * cc;
-        if (row < kC) {
+        float vl[16], vh[16];
 #pragma unroll
-          for (int e4 = 0; e4 < 4; ++e4) {
-            float4 x;
-            x.x = (s0 + 4 * e4 + 0 < row) ? v[4 * e4 + 0] : 0.f;
-            x.y = (s0 + 4 * e4 + 1 < row) ? v[4 * e4 + 1] : 0.f;
-            x.z = (s0 + 4 * e4 + 2 < row) ? v[4 * e4 + 2] : 0.f;
-            x.w = (s0 + 4 * e4 + 3 < row) ? v[4 * e4 + 3] : 0.f;
-            *reinterpret_cast<float4 *>(MS + row * MS_LD + s0 + 4 * e4) = x;
-          }
-        } else {
-          const int t = row - kC;
-          float lo[8], hi[8];
+        for (int e = 0; e < 16; ++e) { vl[e] = 0.f; vh[e] = 0.f; }
+        const bool okl = s0 <= 16 * alo, okh = s0 <= 16 * (alo + 1);
+        if (okl) tmem_ld16(tm + lane_q + grp_off(alo) + s0, vl);
+        if (okh) tmem_ld16(tm + lane_q + grp_off(alo + 1) + s0, vh);
+        tmem_wait_ld();
+        const int sd = 16 * a;  // first column of this row's diagonal block
 #pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            lo[e] = (s0 + e <= t) ? v[e] : 0.f;
-            hi[e] = (s0 + 8 + e <= t) ? v[8 + e] : 0.f;
-          }
-          *reinterpret_cast<uint4 *>(smem + K1_PM + tl64(t, s0 / 8)) = pack8(lo);
-          *reinterpret_cast<uint4 *>(smem + K1_PM + tl64(t, s0 / 8 + 1)) = pack8(hi);
+        for (int e = 0; e < 16; ++e) {
+          const int s = s0 + e;
+          float x = lo ? vl[e] : vh[e];
+          if (s0 > sd || (s0 == sd && (isP ? s > tr : s >= tr))) x = 0.f;
+          mv[cc][e] = x;
         }
+        if (s0 == sd && ((badm >> a) & 1u))
+          diag_exact(smem + (isP ? L::kQS : L::kKS) + tr * KS_LD, smem + L::kBC, GBUF, tr, s0,
+                     !isP, mv[cc]);
+      }
+      // R with the chunk-start reference for MMA2: e^{G_t} r = e^{B_a} (rho_t r)
+#pragma unroll
+      for (int m = 0; m < 4; ++m) {
+        const int t = 8 * warp + (lane & 7), c8 = 4 * m + (lane >> 3), a2 = t >> 4;
+        if (a2 > 0) {
+          float x[8], eb[8];
+          unpack8(*reinterpret_cast<const uint4 *>(smem + L::kRQ + tl128(t, c8)), x);
+          ld8f(TAB + (a2 - 1) * kD + 8 * c8, eb);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) x[e] *= eb[e];
+          *reinterpret_cast<uint4 *>(smem + L::kRQ + tl128(t, c8)) = pack8(x);
+        }
+      }
+      if (badm) __syncthreads();  // the exact sums read region A, which the scratch below reuses
+    } else {
+#pragma unroll
+      for (int cc = 0; cc < 2; ++cc) {
+        const int s0 = 32 * half + 16 * cc;
+        float v[16];
+        tmem_ld16(tm + lane_q + s0, v);
+        tmem_wait_ld();
+        const float gt = kSc ? GS[tr] : 0.f;
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const int s = s0 + e;
+          float x = 0.f;
+          if (isP ? s <= tr : s < tr) {
+            x = v[e];
+            if (kSc) x *= ex2_approx((gt - GS[s]) * kLog2e);  // e^{G_t - G_s} <= 1
+          }
+          mv[cc][e] = x;
+        }
+      }
+    }
+#pragma unroll
+    for (int cc = 0; cc < 2; ++cc) {
+      const int s0 = 32 * half + 16 * cc;
+      if (!isP) {
+#pragma unroll
+        for (int e4 = 0; e4 < 4; ++e4)
+          *reinterpret_cast<float4 *>(MS + tr * MS_LD + s0 + 4 * e4) =
+              make_float4(mv[cc][4 * e4], mv[cc][4 * e4 + 1], mv[cc][4 * e4 + 2], mv[cc][4 * e4 + 3]);
+      } else {
+        float lo8[8], hi8[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) { lo8[e] = mv[cc][e]; hi8[e] = mv[cc][8 + e]; }
+        *reinterpret_cast<uint4 *>(smem + L::kPM + tl64(tr, s0 / 8)) = pack8(lo8);
+        *reinterpret_cast<uint4 *>(smem + L::kPM + tl64(tr, s0 / 8 + 1)) = pack8(hi8);
       }
     }
     tc_fence_before();
     __syncthreads();
-    PDN_K1_MARK(6);
+    // ---- solve: T = (I + M)^{-1} ----
     // L0: 16x16 diagonal blocks; the other threads zero the upper blocks the merges read
     if (tid < 64) {
       const int base = 16 * (tid >> 4), cc = tid & 15;
@@ -672,7 +841,6 @@ __global__ void __launch_bounds__(kK1Threads, 2) k1_intra(const KParams P, void 
       }
     }
     __syncthreads();
-    PDN_K1_MARK(7);
     // L1: merge 16 -> 32 within [32p, 32p + 32): X = -T_D (M_CA T_A)
     if (tid < 128) {
       const int p = tid >> 6, rb = (tid >> 3) & 7, cb = tid & 7;
@@ -755,6 +923,8 @@ __global__ void __launch_bounds__(kK1Threads, 2) k1_intra(const KParams P, void 
       *reinterpret_cast<float2 *>(TS + (32 + r0 + 1) * TS_LD + c0b) = make_float2(-a10, -a11);
     }
     __syncthreads();
+    // T to its bf16 tile. Scalar decay: MMA2 multiplies the undecayed R, so
+    // its tile holds T Diag(e^{G_s}) and T itself goes to the workspace here.
 #pragma unroll
     for (int m = 0; m < 2; ++m) {
       const int t = 8 * warp + (lane & 7), s8 = 4 * m + (lane >> 3);
@@ -762,58 +932,59 @@ __global__ void __launch_bounds__(kK1Threads, 2) k1_intra(const KParams P, void 
       ld8f(TS + t * TS_LD + 8 * s8, v);
 #pragma unroll
       for (int e = 0; e < 8; ++e) v[e] = (8 * s8 + e <= t) ? v[e] : 0.f;
-      *reinterpret_cast<uint4 *>(smem + K1_TM + tl64(t, s8)) = pack8(v);
+      if (kSc) {
+        *reinterpret_cast<uint4 *>(blk + WS_T + tl64(t, s8)) = pack8(v);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) v[e] *= EGS[8 * s8 + e];
+      }
+      *reinterpret_cast<uint4 *>(smem + L::kTM + tl64(t, s8)) = pack8(v);
     }
 
-    // ---- MMA2: Y^T = Rh^T T^T ----
+    // ---- MMA2: Y^T = R^T T^T ----
     sync_for_mma();
-    PDN_K1_MARK(8);
     if (tid == 0) {
       const uint32_t id = make_idesc_bf16(128, 64, true, false);
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk)
-        mma_bf16_ss(tm + 64, make_sdesc(sb + K1_RQ + 4096 * kk, 2048, 128),
-                    make_sdesc(sb + K1_TM + 256 * kk, 128, 1024), id, kk > 0);
+        mma_bf16_ss(tm + L::kTmY, make_sdesc(sb + L::kRQ + 4096 * kk, 2048, 128),
+                    make_sdesc(sb + L::kTM + 256 * kk, 128, 1024), id, kk > 0);
       mma_commit(bar + 1);
     }
     {
       bool ok = true;
-      if (warp == 0) ok = mbar_wait_bounded(bar + 1, par, kSpin);
+      if (warp == 0) ok = mbar_wait_timed(bar + 1, par, kWaitNs);
       ok_all = !__syncthreads_or(!ok);
       tc_fence_after();
     }
-    PDN_K1_MARK(9);
     if (ok_all) {
-      // Rh is dead: the next block's k goes into its space
+      // R is dead: the next block's k goes into its space
       if (it + (int)gridDim.x < total) stage_k(it + gridDim.x);
       // Y^T -> bf16 tile (rows d_k, columns tokens)
       const int i = 32 * (warp & 3) + lane;
 #pragma unroll
       for (int cc = 0; cc < 2; ++cc) {
         float v[16];
-        tmem_ld16(tm + lane_q + 64 + 32 * half + 16 * cc, v);
+        tmem_ld16(tm + lane_q + L::kTmY + 32 * half + 16 * cc, v);
         tmem_wait_ld();
         float lo[8], hi[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) { lo[e] = v[e]; hi[e] = v[8 + e]; }
         const int t8 = 4 * half + 2 * cc;
-        *reinterpret_cast<uint4 *>(smem + K1_YT + tl64(i, t8)) = pack8(lo);
-        *reinterpret_cast<uint4 *>(smem + K1_YT + tl64(i, t8 + 1)) = pack8(hi);
+        *reinterpret_cast<uint4 *>(smem + L::kYT + tl64(i, t8)) = pack8(lo);
+        *reinterpret_cast<uint4 *>(smem + L::kYT + tl64(i, t8 + 1)) = pack8(hi);
       }
       // ---- the tiles that live in shared memory go out with bulk stores ----
       fence_proxy_async_smem();
       tc_fence_before();
       __syncthreads();
       if (tid == 0) {
-        bulk_s2g(blk + WS_Q, smem + K1_RQ + 16384, 16384);
-        bulk_s2g(blk + WS_Y, smem + K1_YT, 16384);
-        bulk_s2g(blk + WS_T, smem + K1_TM, 8192);
-        bulk_s2g(blk + WS_P, smem + K1_PM, 8192);
+        bulk_s2g(blk + WS_Y, smem + L::kYT, 16384);
+        if (!kSc) bulk_s2g(blk + WS_T, smem + L::kTM, 8192);
+        bulk_s2g(blk + WS_P, smem + L::kPM, 8192);
         bulk_commit();  // their reads are awaited before the next block rewrites the tiles
       }
     }
   }
-  PDN_K1_MARK(10);
   if (!ok_all) {
     if (tid == 0) record_error(P.err, PDN_ERR_TIMEOUT);
     break;
@@ -828,7 +999,7 @@ __global__ void __launch_bounds__(kK1Threads, 2) k1_intra(const KParams P, void 
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 0) tmem_dealloc(tm, 128);
+  if (warp == 0) tmem_dealloc(tm, L::kTmemCols);
 }
 
 // ===========================================================================
@@ -920,7 +1091,7 @@ __device__ __forceinline__ uint32_t ut_buf(int n) { return K2_UT + (uint32_t)(n 
 __device__ __forceinline__ bool k2_warp_wait(uint64_t *bar, uint32_t parity,
                                              volatile int *abort_flag, int lane) {
   bool ok = true;
-  if (lane == 0) ok = mbar_wait_bounded(bar, parity, kSpin) && !*abort_flag;
+  if (lane == 0) ok = mbar_wait_timed(bar, parity, kWaitNs) && !*abort_flag;
   ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
   tc_fence_after();
   if (!ok && lane == 0) *abort_flag = 1;
@@ -934,7 +1105,7 @@ __device__ __forceinline__ void k2_warp_arrive(uint64_t *bar, int lane) {
 }
 // Single-thread bounded wait for the issuing warps.
 __device__ __forceinline__ bool k2_wait(uint64_t *bar, uint32_t parity, volatile int *abort_flag) {
-  const bool ok = mbar_wait_bounded(bar, parity, kSpin) && !*abort_flag;
+  const bool ok = mbar_wait_timed(bar, parity, kWaitNs) && !*abort_flag;
   tc_fence_after();
   return ok;
 }
@@ -992,22 +1163,18 @@ __device__ __forceinline__ bool k2_issue_s(uint32_t tm, uint32_t sb, const K2Bar
     // the state epilogue has written S (bf16)
     if (!k2_wait(B.fmain + (n % 3), (uint32_t)((n / 3) & 1), abort_flag)) return false;
     if (!k2_wait(B.sepi, (uint32_t)(n & 1), abort_flag)) return false;
-    PDN_K2_IMARK(0);
 #pragma unroll
     for (int kk = 0; kk < 8; ++kk)
       mma_bf16_ts(tm + TM_UD, tm + tm_sb(n) + 8 * kk, make_sdesc(mb + KM_Y + 2048 * kk, 1024, 128),
                   id5, 1);
     mma_commit(B.bar5);
-    PDN_K2_IMARK(1);
     // MMA8: S += D^T Wb, once D^T is in shared memory
     if (!k2_wait(B.depi, (uint32_t)(n & 1), abort_flag)) return false;
-    PDN_K2_IMARK(2);
 #pragma unroll
     for (int kk = 0; kk < 4; ++kk)
       mma_bf16_ts(tm + TM_S, tm + tm_db(n) + 8 * kk, make_sdesc(mb + KM_WB + 4096 * kk, 2048, 128),
                   id8, 1);
     mma_commit(B.bar7);
-    PDN_K2_IMARK(3);
     // MMA3 of chunk n + 1 (the D^T epilogue has read this chunk's U~^T)
     if (n + 1 < N) {
       if (!k2_wait(B.fut + ((n + 1) & 1), (uint32_t)(((n + 1) >> 1) & 1), abort_flag)) return false;
@@ -1031,22 +1198,18 @@ __device__ __forceinline__ bool k2_issue_o(uint32_t tm, uint32_t sb, const K2Bar
     // warp has seen land
     if (!k2_wait(B.bar5, (uint32_t)(n & 1), abort_flag)) return false;
     if (!k2_wait(B.fmain + (n % 3), (uint32_t)((n / 3) & 1), abort_flag)) return false;
-    PDN_K2_IMARK(4);
 #pragma unroll
     for (int kk = 0; kk < 8; ++kk)
       mma_bf16_ts(tm + ot, tm + tm_sb(n) + 8 * kk, make_sdesc(mb + KM_Q + 256 * kk, 128, 2048), id6,
                   kk > 0);
-    PDN_K2_IMARK(5);
     // MMA7: O^T += D^T P^T after MMA8
     if (!k2_wait(B.bar7, (uint32_t)(n & 1), abort_flag)) return false;
-    PDN_K2_IMARK(6);
 #pragma unroll
     for (int kk = 0; kk < 4; ++kk)
       mma_bf16_ts(tm + ot, tm + tm_db(n) + 8 * kk, make_sdesc(mb + KM_P + 256 * kk, 128, 1024), id7,
                   1);
     mma_commit(B.baro);
     mma_commit(B.mfree + (n % 3));
-    PDN_K2_IMARK(7);
   }
   return true;
 }
@@ -1105,14 +1268,12 @@ __global__ void __launch_bounds__(kK2Threads, 1) k2_state(const KParams P, void 
           break;
         }
         load_ut(smem + ut_buf(n), ws_block(ws, bh, BH, n + 2), B.fut + (n & 1));
-        PDN_K2_HMARK(0);
         if (n + 3 < N) {
           if (!k2_wait(B.mfree + (n % 3), (uint32_t)((n / 3) & 1), abort_flag)) {
             *abort_flag = 1;
             break;
           }
           load_main(smem + main_buf(n), ws_block(ws, bh, BH, n + 3), B.fmain + (n % 3));
-          PDN_K2_HMARK(1);
         }
       }
     }
@@ -1134,7 +1295,6 @@ __global__ void __launch_bounds__(kK2Threads, 1) k2_state(const KParams P, void 
     if (N > 0) fetch_e(0);
     for (int n = 0; n < N; ++n) {
       const int s = n & 1;
-      PDN_K2_MARK(0);
       // this chunk's e^{G_C} has landed (fetched by the warp a chunk ahead).
       // (MMA8 of chunk n - 1, which the state needs, was awaited at the end of
       // the previous iteration; the bf16 S buffer this chunk writes was last
@@ -1142,8 +1302,6 @@ __global__ void __launch_bounds__(kK2Threads, 1) k2_state(const KParams P, void 
       // output.)
       cp_async_wait_all();
       __syncwarp();
-      PDN_K2_MARK(8);
-      PDN_K2_MARK(1);
 
       // ---- state epilogue: S -> bf16 operand; TMEM S <- S Diag(e^{G_C}) ----
       {
@@ -1195,8 +1353,6 @@ __global__ void __launch_bounds__(kK2Threads, 1) k2_state(const KParams P, void 
         tmem_wait_st();
       }
       k2_warp_arrive(B.sepi, lane);
-      PDN_K2_WMARK(0);
-      PDN_K2_MARK(2);
       // chunk n - 1's output in two halves, under MMA5 and under MMA8 (the
       // O^T buffer they free takes chunk n + 1, whose MMA6 comes after this
       // chunk's epilogues)
@@ -1204,12 +1360,9 @@ __global__ void __launch_bounds__(kK2Threads, 1) k2_state(const KParams P, void 
       const int pc_prev = (n - 1) * kC;
       if (n > 0) {
         if (!(ok = k2_warp_wait(B.baro, (uint32_t)((n - 1) & 1), abort_flag, lane))) break;
-        PDN_K2_MARK(9);
         k2_store_o(P, ot_prev, b, h, pc_prev, min(kC, P.T - pc_prev), lane, quarter, cg, 0);
       }
-      PDN_K2_MARK(3);
       if (!(ok = k2_warp_wait(B.bar5, (uint32_t)(n & 1), abort_flag, lane))) break;
-      PDN_K2_MARK(4);
 
       // ---- D^T -> bf16 operand in TMEM (lanes d_v, token pairs per column) ----
       {
@@ -1223,13 +1376,9 @@ __global__ void __launch_bounds__(kK2Threads, 1) k2_state(const KParams P, void 
         tmem_wait_st();
       }
       k2_warp_arrive(B.depi, lane);
-      PDN_K2_WMARK(1);
-      PDN_K2_MARK(5);
       if (n + 1 < N) fetch_e(n + 1);
       if (n > 0) k2_store_o(P, ot_prev, b, h, pc_prev, min(kC, P.T - pc_prev), lane, quarter, cg, 1);
-      PDN_K2_MARK(6);
       if (!(ok = k2_warp_wait(B.bar7, (uint32_t)(n & 1), abort_flag, lane))) break;
-      PDN_K2_MARK(7);
     }
     // the last chunk's output
     if (ok && N > 0 && k2_warp_wait(B.baro, (uint32_t)((N - 1) & 1), abort_flag, lane)) {
@@ -1261,8 +1410,8 @@ __global__ void __launch_bounds__(kK2Threads, 1) k2_state(const KParams P, void 
       record_error(P.err, PDN_ERR_TIMEOUT);
       // drain operand loads still in flight before shared memory goes away
       for (int x = 0; x < 5; ++x) {
-        mbar_wait_bounded(bars + x, 0, kSpin);
-        mbar_wait_bounded(bars + x, 1, kSpin);
+        mbar_wait_timed(bars + x, 0, kDrainNs);
+        mbar_wait_timed(bars + x, 1, kDrainNs);
       }
     }
     __syncthreads();
@@ -1317,10 +1466,12 @@ size_t split_workspace_bytes(const KParams &P) {
   return (size_t)P.B * P.H * N * WS_CH;
 }
 
-cudaError_t launch_chunk_split(const KParams &P, void *ws, cudaStream_t stream) {
+cudaError_t launch_chunk_split(const KParams &P, void *ws, cudaStream_t stream,
+                               cudaEvent_t *ev) {
   const int N = (P.T + kC - 1) / kC;
   const int BH = P.B * P.H;
   cudaError_t e;
+  if (ev && (e = cudaEventRecord(ev[0], stream)) != cudaSuccess) return e;
   if (is_precond(P.variant)) {
     int dev = 0, sms = 148, per_sm = 1;
     if (cudaGetDevice(&dev) == cudaSuccess)
@@ -1335,6 +1486,7 @@ cudaError_t launch_chunk_split(const KParams &P, void *ws, cudaStream_t stream) 
     k0_prefix<<<BH, kD * kK0Groups, 0, stream>>>(P, ws, N);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
+  if (ev && (e = cudaEventRecord(ev[1], stream)) != cudaSuccess) return e;
   switch (P.variant) {
     case PDN_VAR_DN: e = launch_k1_decay<PDN_VAR_DN>(P, ws, N, stream); break;
     case PDN_VAR_GDN: e = launch_k1_decay<PDN_VAR_GDN>(P, ws, N, stream); break;
@@ -1348,8 +1500,10 @@ cudaError_t launch_chunk_split(const KParams &P, void *ws, cudaStream_t stream) 
   if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(k2_state, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)K2_BYTES);
   if (e != cudaSuccess) return e;
+  if (ev && (e = cudaEventRecord(ev[2], stream)) != cudaSuccess) return e;
   k2_state<<<BH, kK2Threads, K2_BYTES, stream>>>(P, ws, N);
-  return cudaGetLastError();
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  return ev ? cudaEventRecord(ev[3], stream) : cudaSuccess;
 }
 
 }  // namespace pdn

@@ -159,7 +159,6 @@ constexpr int kConsumers = kThreads;      // 8 consumer warps
 constexpr int kTmaThreads = kThreads + 32;  // + 1 producer warp
 constexpr uint32_t kStateBytes = kD128 * kD128 * 4;
 constexpr uint32_t kPart = 16384;  // bytes per bulk copy
-constexpr long long kDecSpin = 1LL << 22;
 
 struct DecSmem {
   float buf[kTmaBufs][kD128 * kD128];
@@ -232,7 +231,7 @@ __global__ void __launch_bounds__(kTmaThreads, 1) decode_tma_kernel(const KParam
         const int s = k % kTmaBufs;
         if (k >= kTmaBufs) {
           // the consumers are done with item k - kTmaBufs in buffer s
-          if (!mbar_wait_bounded(&sm.empty[s], (uint32_t)(((k / kTmaBufs) - 1) & 1), kDecSpin) ||
+          if (!mbar_wait_timed(&sm.empty[s], (uint32_t)(((k / kTmaBufs) - 1) & 1), kWaitNs) ||
               *reinterpret_cast<volatile int *>(&sm.abort_flag)) {
             atomicExch(&sm.abort_flag, 1);
             break;
@@ -246,10 +245,10 @@ __global__ void __launch_bounds__(kTmaThreads, 1) decode_tma_kernel(const KParam
       // write back the last items, then wait for all stores
       for (int k = (loaded > kTmaBufs ? loaded - kTmaBufs : 0); k < loaded; ++k) {
         const int s = k % kTmaBufs;
-        if (!mbar_wait_bounded(&sm.empty[s], (uint32_t)((k / kTmaBufs) & 1), kDecSpin)) {
+        if (!mbar_wait_timed(&sm.empty[s], (uint32_t)((k / kTmaBufs) & 1), kWaitNs)) {
           atomicExch(&sm.abort_flag, 1);
           // drain the load into this buffer before giving up on it
-          mbar_wait_bounded(&sm.full[s], (uint32_t)((k / kTmaBufs) & 1), kDecSpin);
+          mbar_wait_timed(&sm.full[s], (uint32_t)((k / kTmaBufs) & 1), kDrainNs);
           continue;
         }
         issue_state_store(sm, s, state_of(k));
@@ -339,7 +338,7 @@ __global__ void __launch_bounds__(kTmaThreads, 1) decode_tma_kernel(const KParam
     // Wait for the state. The decision to stop must be the same in every
     // consumer warp (they meet at named barriers): each warp votes once,
     // after a consumer barrier all warps read all votes.
-    const bool ok = mbar_wait_bounded(&sm.full[s], (uint32_t)((k / kTmaBufs) & 1), kDecSpin);
+    const bool ok = mbar_wait_timed(&sm.full[s], (uint32_t)((k / kTmaBufs) & 1), kWaitNs);
     int vote = __all_sync(0xffffffffu, ok) ? 1 : 0;
     if (lane == 0) {
       if (*reinterpret_cast<volatile int *>(&sm.abort_flag)) vote = 0;
@@ -399,7 +398,7 @@ int num_sms() {
   return g_num_sms[dev];
 }
 
-__global__ void selftest_wait_kernel(long long limit, int *err) {
+__global__ void selftest_wait_kernel(long long limit_ns, int *err) {
   __shared__ __align__(8) uint64_t bar;
   if (threadIdx.x == 0) {
     mbar_init(&bar, 1);
@@ -407,7 +406,7 @@ __global__ void selftest_wait_kernel(long long limit, int *err) {
   }
   __syncthreads();
   // Nothing ever arrives on `bar`: the phase never completes.
-  if (threadIdx.x == 0 && !mbar_wait_bounded(&bar, 0, limit)) record_error(err, PDN_ERR_TIMEOUT);
+  if (threadIdx.x == 0 && !mbar_wait_timed(&bar, 0, (uint64_t)limit_ns)) record_error(err, PDN_ERR_TIMEOUT);
 }
 
 }  // namespace
@@ -440,8 +439,8 @@ cudaError_t launch_decode(const KParams &P, cudaStream_t stream) {
   return cudaGetLastError();
 }
 
-cudaError_t launch_selftest_wait(long long spin_limit, int *err, cudaStream_t stream) {
-  selftest_wait_kernel<<<1, 32, 0, stream>>>(spin_limit, err);
+cudaError_t launch_selftest_wait(long long limit_ns, int *err, cudaStream_t stream) {
+  selftest_wait_kernel<<<1, 32, 0, stream>>>(limit_ns, err);
   return cudaGetLastError();
 }
 

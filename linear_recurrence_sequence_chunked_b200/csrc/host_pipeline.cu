@@ -15,6 +15,7 @@
 #include <mutex>
 
 #include "common.cuh"
+#include "internal.h"
 
 namespace pdn {
 namespace {
@@ -24,7 +25,7 @@ constexpr int kMaxSlices = 64;
 
 struct HostPipe {
   cudaStream_t in = nullptr, out = nullptr;
-  cudaEvent_t start = nullptr, done = nullptr;
+  cudaEvent_t start = nullptr, done = nullptr, done_in = nullptr;
   cudaEvent_t landed[kMaxSlices] = {}, computed[kMaxSlices] = {};
   bool ready = false;
 };
@@ -37,6 +38,7 @@ cudaError_t make_pipe(HostPipe &hp) {
   if ((e = cudaStreamCreateWithFlags(&hp.out, cudaStreamNonBlocking)) != cudaSuccess) return e;
   if ((e = cudaEventCreateWithFlags(&hp.start, cudaEventDisableTiming)) != cudaSuccess) return e;
   if ((e = cudaEventCreateWithFlags(&hp.done, cudaEventDisableTiming)) != cudaSuccess) return e;
+  if ((e = cudaEventCreateWithFlags(&hp.done_in, cudaEventDisableTiming)) != cudaSuccess) return e;
   for (int i = 0; i < kMaxSlices; ++i) {
     if ((e = cudaEventCreateWithFlags(&hp.landed[i], cudaEventDisableTiming)) != cudaSuccess) return e;
     if ((e = cudaEventCreateWithFlags(&hp.computed[i], cudaEventDisableTiming)) != cudaSuccess)
@@ -84,6 +86,28 @@ cudaError_t copy_out(void *dst, const void *src, size_t per, int b0, int n, cuda
                          cudaMemcpyDeviceToHost, s);
 }
 
+
+using namespace pdn;
+
+// The problem and device tensors of slice [b0, b0 + n) of the batch.
+void slice_of(const pdn_problem_t *p, const pdn_tensors_t *dev, const Sizes &z, int b0, int n,
+              pdn_problem_t *pi, pdn_tensors_t *ti) {
+  *pi = *p;
+  pi->B = n;
+  ti->q = offset(dev->q, z.q * b0);
+  ti->k = offset(dev->k, z.k * b0);
+  ti->v = offset(dev->v, z.v * b0);
+  ti->log_alpha = offset(dev->log_alpha, z.la * b0);
+  ti->beta = offset(dev->beta, z.beta * b0);
+  ti->erase = offset(dev->erase, z.erase * b0);
+  ti->write = offset(dev->write, z.write * b0);
+  ti->S0 = static_cast<const float *>(offset(dev->S0, z.S * b0));
+  ti->ST = static_cast<float *>(offset(dev->ST, z.S * b0));
+  ti->A0 = static_cast<const float *>(offset(dev->A0, z.A * b0));
+  ti->AT = static_cast<float *>(offset(dev->AT, z.A * b0));
+  ti->o = offset(dev->o, z.o * b0);
+}
+
 }  // namespace
 }  // namespace pdn
 
@@ -105,8 +129,19 @@ extern "C" pdn_status_t pdn_chunk_fwd_host(const pdn_problem_t *p, const pdn_ten
                       dev->erase, dev->write, dev->S0, dev->ST, dev->A0, dev->AT};
   for (int i = 0; i < 12; ++i)
     if (hs[i] && !ds[i]) return PDN_ERR_INVALID_ARG;
-  // the whole problem must pass pdn_chunk_fwd's checks before anything runs
-  if (pdn_chunk_fwd_impl(p) < 0) return PDN_ERR_UNSUPPORTED;
+  // the whole problem and every slice's forward must pass pdn_chunk_fwd's
+  // checks before anything is enqueued
+  pdn_status_t st = pdn::check_chunk_fwd(p, dev, workspace, ws_bytes, nullptr);
+  if (st != PDN_OK) return st;
+  const Sizes z = sizes_of(p);
+  for (int i = 0; i < slices; ++i) {
+    const int b0 = (int)((long long)p->B * i / slices);
+    const int b1 = (int)((long long)p->B * (i + 1) / slices);
+    pdn_problem_t pi;
+    pdn_tensors_t ti;
+    slice_of(p, dev, z, b0, b1 - b0, &pi, &ti);
+    if ((st = pdn::check_chunk_fwd(&pi, &ti, workspace, ws_bytes, nullptr)) != PDN_OK) return st;
+  }
 
   int devno = 0;
   if (cudaGetDevice(&devno) != cudaSuccess || devno < 0 || devno >= kMaxDevices) return PDN_ERR_CUDA;
@@ -115,13 +150,13 @@ extern "C" pdn_status_t pdn_chunk_fwd_host(const pdn_problem_t *p, const pdn_ten
   if (!hp.ready && make_pipe(hp) != cudaSuccess) return PDN_ERR_CUDA;
 
   const cudaStream_t s0 = static_cast<cudaStream_t>(stream);
-  const Sizes z = sizes_of(p);
   cudaError_t e = cudaEventRecord(hp.start, s0);
   if (e == cudaSuccess) e = cudaStreamWaitEvent(hp.in, hp.start, 0);
   if (e == cudaSuccess) e = cudaStreamWaitEvent(hp.out, hp.start, 0);
   if (e != cudaSuccess) return PDN_ERR_CUDA;
 
-  for (int i = 0; i < slices; ++i) {
+  st = PDN_OK;
+  for (int i = 0; i < slices && st == PDN_OK; ++i) {
     const int b0 = (int)((long long)p->B * i / slices);
     const int b1 = (int)((long long)p->B * (i + 1) / slices);
     const int n = b1 - b0;
@@ -142,34 +177,28 @@ extern "C" pdn_status_t pdn_chunk_fwd_host(const pdn_problem_t *p, const pdn_ten
       e = copy_in(const_cast<float *>(dev->A0), host->A0, z.A, b0, n, hp.in);
     if (e == cudaSuccess) e = cudaEventRecord(hp.landed[i], hp.in);
     if (e == cudaSuccess) e = cudaStreamWaitEvent(s0, hp.landed[i], 0);
-    if (e != cudaSuccess) return PDN_ERR_CUDA;
+    if (e != cudaSuccess) { st = PDN_ERR_CUDA; break; }
     // forward of part i on the caller's stream
-    pdn_problem_t pi = *p;
-    pi.B = n;
+    pdn_problem_t pi;
     pdn_tensors_t ti;
-    ti.q = offset(dev->q, z.q * b0);
-    ti.k = offset(dev->k, z.k * b0);
-    ti.v = offset(dev->v, z.v * b0);
-    ti.log_alpha = offset(dev->log_alpha, z.la * b0);
-    ti.beta = offset(dev->beta, z.beta * b0);
-    ti.erase = offset(dev->erase, z.erase * b0);
-    ti.write = offset(dev->write, z.write * b0);
-    ti.S0 = static_cast<const float *>(offset(dev->S0, z.S * b0));
-    ti.ST = static_cast<float *>(offset(dev->ST, z.S * b0));
-    ti.A0 = static_cast<const float *>(offset(dev->A0, z.A * b0));
-    ti.AT = static_cast<float *>(offset(dev->AT, z.A * b0));
-    ti.o = offset(dev->o, z.o * b0);
-    const pdn_status_t st = pdn_chunk_fwd(&pi, &ti, workspace, ws_bytes, stream);
-    if (st != PDN_OK) return st;
-    if (cudaEventRecord(hp.computed[i], s0) != cudaSuccess) return PDN_ERR_CUDA;
+    slice_of(p, dev, z, b0, n, &pi, &ti);
+    st = pdn_chunk_fwd(&pi, &ti, workspace, ws_bytes, stream);
+    if (st != PDN_OK) break;
+    if (cudaEventRecord(hp.computed[i], s0) != cudaSuccess) { st = PDN_ERR_CUDA; break; }
     // outputs of part i
     e = cudaStreamWaitEvent(hp.out, hp.computed[i], 0);
     if (e == cudaSuccess) e = copy_out(host->o, dev->o, z.o, b0, n, hp.out);
     if (e == cudaSuccess) e = copy_out(host->ST, dev->ST, z.S, b0, n, hp.out);
     if (e == cudaSuccess) e = copy_out(host->AT, dev->AT, z.A, b0, n, hp.out);
-    if (e != cudaSuccess) return PDN_ERR_CUDA;
+    if (e != cudaSuccess) st = PDN_ERR_CUDA;
   }
+  // the caller's stream waits for everything enqueued, also after an error
+  // part-way (nothing may still be copying once the stream has drained)
   e = cudaEventRecord(hp.done, hp.out);
+  const cudaError_t e2 = cudaEventRecord(hp.done_in, hp.in);
   if (e == cudaSuccess) e = cudaStreamWaitEvent(s0, hp.done, 0);
+  if (e == cudaSuccess) e = e2;
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(s0, hp.done_in, 0);
+  if (st != PDN_OK) return st;
   return e == cudaSuccess ? PDN_OK : PDN_ERR_CUDA;
 }

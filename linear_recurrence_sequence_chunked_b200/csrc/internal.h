@@ -11,21 +11,24 @@ namespace pdn {
 int simt_supported(const KParams &P);
 cudaError_t launch_chunk_simt(const KParams &P, cudaStream_t stream);
 
-// Tensor-core (tcgen05) chunk kernel: bf16 operands, fp32 state in TMEM.
-int tc_supported(const KParams &P);
-size_t tc_workspace_bytes(const KParams &P);
-cudaError_t launch_chunk_tc(const KParams &P, void *workspace, cudaStream_t stream);
-
 // Tensor-core three-kernel path: intra-chunk work for all chunks at once,
 // then the sequential state pass; needs a workspace.
 int split_supported(const KParams &P);
 size_t split_workspace_bytes(const KParams &P);
-cudaError_t launch_chunk_split(const KParams &P, void *workspace, cudaStream_t stream);
+// `ev` (optional, four events) is recorded before the key-energy kernels,
+// before the intra-chunk kernel, before the state kernel and after it.
+cudaError_t launch_chunk_split(const KParams &P, void *workspace, cudaStream_t stream,
+                               cudaEvent_t *ev = nullptr);
 
 // One decode step (state streamed through once).
 cudaError_t launch_decode(const KParams &P, cudaStream_t stream);
 
+// Every check pdn_chunk_fwd makes before it enqueues work (host-only);
+// on PDN_OK, *impl_out (if non-NULL) is the path it would run.
+pdn_status_t check_chunk_fwd(const pdn_problem_t *p, const pdn_tensors_t *t,
+                             const void *workspace, size_t ws_bytes, int *impl_out);
+
 // Bounded-wait self test.
-cudaError_t launch_selftest_wait(long long spin_limit, int *err, cudaStream_t stream);
+cudaError_t launch_selftest_wait(long long limit_ns, int *err, cudaStream_t stream);
 
 }  // namespace pdn

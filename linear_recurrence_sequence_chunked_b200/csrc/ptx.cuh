@@ -78,14 +78,32 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Waits for the phase with the given parity to complete, polling at most
-// `limit` times. Returns false if the wait ran out (the caller records
-// PDN_ERR_TIMEOUT and winds down instead of hanging).
-__device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity,
-                                                  long long limit) {
-  for (long long it = 0; it < limit; ++it)
-    if (mbar_try_wait(bar, parity)) return true;
-  return false;
+// Device wall clock in nanoseconds (the %globaltimer special register).
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// Limits of the bounded waits: a wait that is still open after kWaitNs of
+// device time gives up (the kernel records PDN_ERR_TIMEOUT and winds down
+// instead of hanging); every wait of a healthy run ends within microseconds.
+// kDrainNs bounds the waits for copies in flight while a kernel winds down.
+constexpr uint64_t kWaitNs = 2000000000ull;
+constexpr uint64_t kDrainNs = 10000000ull;
+
+// Waits for the phase with the given parity to complete, for at most
+// `limit_ns` nanoseconds of device time. Returns false if the wait ran out.
+__device__ __forceinline__ bool mbar_wait_timed(uint64_t *bar, uint32_t parity,
+                                                uint64_t limit_ns) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (;;) {
+#pragma unroll 1
+    for (int i = 0; i < 32; ++i)
+      if (mbar_try_wait(bar, parity)) return true;
+    if (globaltimer_ns() - t0 >= limit_ns) return false;
+  }
 }
 
 // ---------------------------------------------------------------- bulk copies (TMA, 1-D)

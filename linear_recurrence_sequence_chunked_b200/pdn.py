@@ -24,7 +24,7 @@ PDN_OK, PDN_ERR_INVALID_ARG, PDN_ERR_UNSUPPORTED, PDN_ERR_CUDA, PDN_ERR_TIMEOUT,
 VARIANTS = {"DN": 0, "GDN": 1, "KDA": 2, "PDN": 3, "PGDN": 4, "PKDA": 5, "FG2_GDN": 6, "GDN2": 7}
 DECAYS = {"none": 0, "scalar": 1, "channel": 2}
 DTYPES = {torch.float32: 0, torch.bfloat16: 1}
-IMPLS = {"auto": 0, "simt": 1, "tc": 2, "tc_fused": 3}
+IMPLS = {"auto": 0, "simt": 1, "tc": 2}
 PRECOND_VARIANTS = ("PDN", "PGDN", "PKDA")
 
 
@@ -65,6 +65,10 @@ def load() -> ctypes.CDLL:
         lib.pdn_chunk_fwd_impl.argtypes = [P]
         lib.pdn_chunk_fwd.restype = ctypes.c_int
         lib.pdn_chunk_fwd.argtypes = [P, T, vp, ctypes.c_size_t, vp]
+        lib.pdn_chunk_fwd_profiled.restype = ctypes.c_int
+        lib.pdn_chunk_fwd_profiled.argtypes = [P, T, vp, ctypes.c_size_t, vp,
+                                               ctypes.POINTER(ctypes.c_float),
+                                               ctypes.POINTER(ctypes.c_int)]
         lib.pdn_chunk_fwd_noalloc.restype = ctypes.c_int
         lib.pdn_chunk_fwd_noalloc.argtypes = [P, T, vp]
         lib.pdn_chunk_fwd_host.restype = ctypes.c_int
@@ -94,6 +98,17 @@ def pdn_chunk_fwd(problem: PdnProblem, tensors: PdnTensors, workspace: int, ws_b
                   stream: int) -> int:
     return load().pdn_chunk_fwd(ctypes.byref(problem), ctypes.byref(tensors), workspace,
                                 ws_bytes, stream)
+
+
+def pdn_chunk_fwd_profiled(problem: PdnProblem, tensors: PdnTensors, workspace: int,
+                           ws_bytes: int, stream: int):
+    """pdn_chunk_fwd with CUDA events between its kernels (blocking). Returns
+    (status, [milliseconds per kernel stage])."""
+    ms = (ctypes.c_float * 4)()
+    n = ctypes.c_int(0)
+    rc = load().pdn_chunk_fwd_profiled(ctypes.byref(problem), ctypes.byref(tensors), workspace,
+                                       ws_bytes, stream, ms, ctypes.byref(n))
+    return rc, [float(ms[i]) for i in range(n.value)]
 
 
 def pdn_chunk_fwd_noalloc(problem: PdnProblem, tensors: PdnTensors, stream: int) -> int:

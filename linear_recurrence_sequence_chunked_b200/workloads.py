@@ -33,7 +33,10 @@ class Workload:
     dv: int
     dtype: str              # "f32" | "bf16"
     decay: str              # "none" | "scalar" | "channel"
-    decay_recipe: str = "softplus"   # "softplus": -0.1*softplus(N(0,1)); "sigmoid": log sigmoid(N(2,1))
+    decay_recipe: str = "softplus"   # "softplus": -0.1*softplus(N(0,1)); "sigmoid": log sigmoid(N(2,1));
+                                     # "strong": 2 * decay_mean * sigmoid(N(0,1)) (mean decay_mean)
+    decay_mean: float = 0.0          # mean per-token log decay of the "strong" recipe
+    hard_decay: bool = False         # channel 3 (channel decay) or every 7th token (scalar) at log alpha = -30
     chunk: int = 64
     precond_x: float = 1.5
     precond_eps: float = 1e-6
@@ -105,8 +108,15 @@ def make_inputs(w: Workload, device="cpu", B: Optional[int] = None, T: Optional[
         z = randn(*shape)
         if w.decay_recipe == "sigmoid":
             la = torch.nn.functional.logsigmoid(z + 2.0)
+        elif w.decay_recipe == "strong":
+            la = 2.0 * w.decay_mean * torch.sigmoid(z)
         else:
             la = -0.1 * torch.nn.functional.softplus(z)
+        if w.hard_decay:
+            if w.decay == "scalar":
+                la[:, ::7] = -30.0
+            else:
+                la[..., 3] = -30.0
         log_alpha = la if w.decay == "scalar" else la.to(dt)
     erase = write = None
     if w.variant == "GDN2":

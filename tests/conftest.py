@@ -24,3 +24,24 @@ def pytest_collection_modifyitems(config, items):
     for it in items:
         if "gpu" in it.keywords:
             it.add_marker(skip)
+
+
+def pytest_terminal_summary(terminalreporter, exitstatus, config):
+    """Lists the elementwise relative errors the parity checks recorded (the
+    bars gate the normalised max-abs error; this figure is reported only)."""
+    try:
+        from parity_util import REPORT
+    except Exception:  # pragma: no cover
+        return
+    if not REPORT:
+        return
+    tr = terminalreporter
+    tr.section("parity errors (normalised max-abs | elementwise rel., floor 1e-3 rms)")
+    worst = {}
+    for name, dt, e_o, e_s, r_o, r_s in REPORT:
+        k = (name, dt)
+        prev = worst.get(k)
+        cur = (max(e_o, e_s), max(r_o, r_s))
+        worst[k] = cur if prev is None else (max(prev[0], cur[0]), max(prev[1], cur[1]))
+    for (name, dt), (e, r) in sorted(worst.items()):
+        tr.write_line("%-34s %-5s norm %.3e  elem %.3e" % (name, dt, e, r))

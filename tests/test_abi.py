@@ -187,13 +187,68 @@ def test_host_pipeline_argument_errors(lib):
 @pytest.mark.parametrize("B,T,H", [(1, 1, 1), (4, 4096, 16), (2, 130, 3), (3, 64, 2)])
 def test_workspace_size_of_the_tensor_core_paths(lib, B, T, H):
     """The three-kernel path needs one 82,944-byte block per (batch, head,
-    chunk); the fused and CUDA-core paths need none (host-only queries)."""
+    chunk); the CUDA-core path needs none (host-only queries)."""
     p = _problem(B=B, T=T, H=H, d_k=128, d_v=128)
     assert pdn.pdn_chunk_fwd_impl(p) == pdn.IMPLS["tc"]
     assert pdn.pdn_chunk_fwd_workspace(p) == B * H * ((T + 63) // 64) * 82944
-    p = _problem(B=B, T=T, H=H, d_k=128, d_v=128, impl=pdn.IMPLS["tc_fused"])
-    assert pdn.pdn_chunk_fwd_impl(p) == pdn.IMPLS["tc_fused"]
-    assert pdn.pdn_chunk_fwd_workspace(p) == 0
+    p = _problem(B=B, T=T, H=H, d_k=128, d_v=128, impl=3)  # no third kernel
+    assert pdn.pdn_chunk_fwd_impl(p) == -1
+    assert pdn.pdn_chunk_fwd_workspace(p) == (1 << 64) - 1
     p = _problem(B=B, T=T, H=H, d_k=64, d_v=64)
     assert pdn.pdn_chunk_fwd_impl(p) == pdn.IMPLS["simt"]
     assert pdn.pdn_chunk_fwd_workspace(p) == 0
+
+
+def test_noalloc_size_gate(lib):
+    """Host-only: B*H*ceil(T/64) = 810 chunk blocks exceeds the built-in array
+    (PDN_ERR_WORKSPACE before anything touches a device); 809 passes the size
+    gate and only then needs a device (PDN_ERR_CUDA here, without one)."""
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("the 809-block case would launch on a real device")
+    fake = 0x7f0000000000
+    t = pdn.PdnTensors(q=fake, k=fake, v=fake, log_alpha=fake, beta=fake, o=fake)
+    mk = lambda T: pdn.make_problem("GDN", 1, T, 1, 128, 128, torch.bfloat16, "scalar", 64, "tc")
+    assert pdn.pdn_chunk_fwd_noalloc(mk(810 * 64), t, None) == pdn.PDN_ERR_WORKSPACE
+    assert pdn.pdn_chunk_fwd_noalloc(mk(809 * 64), t, None) == pdn.PDN_ERR_CUDA
+    assert pdn.pdn_chunk_fwd_noalloc(mk(808 * 64 + 1), t, None) == pdn.PDN_ERR_CUDA
+
+
+def test_scalar_gate_alignment(lib):
+    """fp32 per-(token, head) gates are read one element at a time: 4-byte
+    alignment passes the argument checks (the call then needs a device:
+    PDN_ERR_CUDA without one), 2-byte alignment does not. Vector tensors
+    still need 16 bytes."""
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a passing check would launch on a real device")
+    p = _problem()
+    assert pdn.pdn_chunk_fwd(p, _tensors(log_alpha=FAKE + 0x3004, beta=FAKE + 0x4008), None, 0,
+                             None) == pdn.PDN_ERR_CUDA
+    assert pdn.pdn_chunk_fwd(p, _tensors(log_alpha=FAKE + 0x3002), None, 0,
+                             None) == pdn.PDN_ERR_INVALID_ARG
+    assert pdn.pdn_chunk_fwd(p, _tensors(beta=FAKE + 0x4001), None, 0,
+                             None) == pdn.PDN_ERR_INVALID_ARG
+    # a per-channel gate (FG2 beta vector) keeps the 16-byte rule
+    p = _problem(variant=pdn.VARIANTS["FG2_GDN"], decay=pdn.DECAYS["channel"])
+    assert pdn.pdn_chunk_fwd(p, _tensors(beta=FAKE + 0x4004), None, 0,
+                             None) == pdn.PDN_ERR_INVALID_ARG
+
+
+def test_host_pipeline_validates_before_enqueueing(lib):
+    """Every argument error of pdn_chunk_fwd_host comes back before anything
+    is enqueued (without a device, reaching the enqueue stage would give
+    PDN_ERR_CUDA instead)."""
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a passing check would enqueue on a real device")
+    p = _problem(B=3, T=131, H=1)
+    need = pdn.pdn_chunk_fwd_workspace(p)
+    ws = FAKE + 0x100000
+    t = _tensors()
+    assert pdn.pdn_chunk_fwd_host(p, t, _tensors(k=FAKE + 0x1008), ws, need, 2,
+                                  None) == pdn.PDN_ERR_INVALID_ARG
+    assert pdn.pdn_chunk_fwd_host(p, t, _tensors(log_alpha=FAKE + 0x3002), ws, need, 2,
+                                  None) == pdn.PDN_ERR_INVALID_ARG
+    # T * H odd: slice 1's scalar gates are 4-byte aligned, which is accepted
+    assert pdn.pdn_chunk_fwd_host(p, t, t, ws, need, 2, None) == pdn.PDN_ERR_CUDA

@@ -112,3 +112,24 @@ def test_decode_d128_many_heads(variant, dtype):
     assert nmax_err(S.cpu().numpy(), rS) <= tol
     if A is not None:
         assert nmax_err(A.cpu().numpy(), rA) <= 1e-6
+
+
+def test_decode_workload_full_1024_steps_sampled_chains():
+    """The decode workload as configured: 256 sequences x 16 heads, d 128,
+    fp32 state, one bf16 token per sequence per step for all 1024 steps. The
+    outputs of every step and the final state of sampled (batch, head)
+    chains are checked against the oracle over all 1024 tokens, so drift of
+    the fp32 state over the whole run would show."""
+    w = WORKLOADS["pgdn_decode_256"]
+    steps = w.decode_steps
+    x = make_inputs(w.replace(T=steps), device="cuda", generator_device="cuda")
+    S = torch.zeros(w.B, w.H, w.dv, w.dk, device="cuda")
+    A = torch.zeros(w.B, w.H, w.dk, device="cuda")
+    o = decode_all(w, x, S, A, steps)
+    for b, h in [(0, 0), (97, 5), (255, 15), (128, 9)]:
+        xs = {n: (t[b:b + 1, :, h:h + 1].cpu() if t is not None else None) for n, t in x.items()}
+        ro, rS, rA = run_oracle(w.replace(B=1, H=1, T=steps), xs)
+        eo = nmax_err(o[b:b + 1, :, h:h + 1].float().cpu().numpy(), ro)
+        es = nmax_err(S[b:b + 1, h:h + 1].cpu().numpy(), rS)
+        ea = nmax_err(A[b:b + 1, h:h + 1].cpu().numpy(), rA)
+        assert eo <= 2e-2 and es <= 2e-2 and ea <= 1e-5, (b, h, eo, es, ea)

@@ -69,3 +69,17 @@ def test_host_path_parity_with_oracle():
     x = make_inputs(w)
     o, ST, AT = host_run(w, x, None, None, 2)
     assert_parity(w, o, ST, AT, *run_oracle(w, x))
+
+
+@pytest.mark.parametrize("variant", ["PGDN", "GDN2"])
+def test_host_path_odd_token_head_count(variant):
+    """T * H odd (131 x 1): slice 1's fp32 scalar-gate pointers sit 4 bytes
+    off a 16-byte boundary, which the scalar gates allow; every slicing gives
+    the device path's outputs bitwise."""
+    w = Workload("host-odd-" + variant, variant, 3, 131, 1, 128, 128, "bf16", DECAY[variant])
+    x = make_inputs(w)
+    ref = run_gpu(w, x)
+    for slices in (2, 3):
+        o, ST, AT = host_run(w, x, None, None, slices)
+        assert torch.equal(o, ref[0].cpu()), (variant, slices)
+        assert torch.equal(ST, ref[1].cpu()), (variant, slices)

@@ -22,16 +22,13 @@ def tc_work(variant, decay=None, B=2, T=200, H=2, seed=0, **kw):
                     decay or DECAY[variant], seed=seed, **kw)
 
 
-TC_IMPLS = ["tc", "tc_fused"]
+TC_IMPLS = ["tc"]
 
 
 def test_tc_kernel_is_selected():
     p = pdn.make_problem("PGDN", 4, 4096, 16, 128, 128, torch.bfloat16)
     assert pdn.pdn_chunk_fwd_impl(p) == pdn.IMPLS["tc"]
     assert pdn.pdn_chunk_fwd_workspace(p) > 0
-    p = pdn.make_problem("PGDN", 4, 4096, 16, 128, 128, torch.bfloat16, impl="tc_fused")
-    assert pdn.pdn_chunk_fwd_impl(p) == pdn.IMPLS["tc_fused"]
-    assert pdn.pdn_chunk_fwd_workspace(p) == 0
     p = pdn.make_problem("PGDN", 1, 64, 2, 64, 64, torch.bfloat16)
     assert pdn.pdn_chunk_fwd_impl(p) == pdn.IMPLS["simt"]
 
@@ -68,7 +65,7 @@ def test_tc_lengths(T, impl):
 
 
 def test_tc_matches_simt():
-    """The three paths on the same bf16 inputs agree to the bf16 tolerance."""
+    """The two paths on the same bf16 inputs agree to the bf16 tolerance."""
     w = tc_work("PGDN", B=2, H=4, T=333)
     x = make_inputs(w)
     b = run_gpu(w, x, impl="simt")
