@@ -4,17 +4,18 @@
 //
 //   K0  key-energy prefix: A at the start of every chunk (preconditioned
 //       variants; "Preconditioned DeltaNet", fr §2.B: A_t = A_{t-1} + k.k)
-//   K1  persistent, two CTAs per SM walking the (chunk, batch, head) blocks:
-//       gates and preconditioner, M and P (MMA), T = (I + M)^{-1},
-//       Y^T = Rh^T T^T (MMA); writes bf16 operand tiles of the chunk to the
-//       workspace in the shared-memory image the state kernel's MMAs consume
-//   K2  one CTA per (batch, head): per chunk, bulk-loads those tiles two
-//       chunks ahead, U^T = U^T T^T, D^T = U^T - S Y^T, O^T = S Qh^T + D^T P^T,
+//   K1  persistent over the (chunk, batch, head) blocks (two CTAs per SM,
+//       one for channel decay): gates and preconditioner, M and P (MMA),
+//       T = (I + M)^{-1}, Y^T = R^T T^T (MMA); writes the chunk's bf16
+//       operand tiles to the workspace, straight from registers, in the
+//       shared-memory image the state kernel's MMAs consume
+//   K2  one CTA per (batch, head): per chunk, bulk-loads those tiles ahead,
+//       U^T = U^T T^T, D^T = U^T - S Y^T, O^T = S Qh^T + D^T P^T,
 //       S <- S Diag(e^{G_C}) + D^T Wb; fp32 state in tensor memory
 //
-// Same chunk algebra as the single-kernel path ("Gated DeltaNet-2", ja §3:
+// The chunk algebra is the chunkwise WY/UT form ("Gated DeltaNet-2", ja §3:
 // decay absorbed into the erase/write matrices, (I+T)^{-1} solve for the
-// auxiliaries Y and U); the split trades extra HBM traffic (about 80 KiB of
+// auxiliaries Y and U). Splitting it trades extra HBM traffic (about 80 KiB of
 // operand tiles per chunk and head, written once and read once) for running
 // the intra-chunk work with thousands of CTAs instead of one per chain.
 #include "common.cuh"
@@ -193,15 +194,17 @@ struct K1Layout {
   static constexpr uint32_t kBC = kQS + 64 * KS_LD;
   static constexpr uint32_t kGBUF = kBC + 64 * KS_LD;
   static constexpr uint32_t kLasStage = kGBUF + 64 * LB_LD * 4;
-  static constexpr uint32_t kPrepEnd = kCh ? kLasStage + 64 * 256 : kGBUF;
-  // region A from the epilogue of MMA1 on: T and P tiles, the fp32 solve
-  // scratch, then the Y^T tile
+  // channel decay: FG2's gain vector, or GDN-2's erase and write gates,
+  // staged by cp.async with q (read in P3)
+  static constexpr int kGates = !kCh ? 0 : kVariant == PDN_VAR_FG2_GDN ? 1 : kVariant == PDN_VAR_GDN2 ? 2 : 0;
+  static constexpr uint32_t kGateStage = kLasStage + 64 * 256;
+  static constexpr uint32_t kPrepEnd = kCh ? kGateStage + kGates * 16384 : kGBUF;
+  // region A from the epilogue of MMA1 on: MMA2's T tile and the fp32 solve
+  // scratch
   static constexpr uint32_t kTM = kRA;                      // TL 64 x 64
-  static constexpr uint32_t kPM = kRA + 8192;               // TL 64 x 64
   static constexpr uint32_t kMS = kRA + 16384;              // fp32 [64][68]
   static constexpr uint32_t kTS = kMS + 64 * MS_LD * 4;     // fp32 [64][68]
   static constexpr uint32_t kYS = kTS + 64 * TS_LD * 4;     // fp32 [32][34]
-  static constexpr uint32_t kYT = kRA + 16384;              // TL 128 x 64
   static constexpr uint32_t kSolveEnd = kYS + 32 * YS_LD * 4;
   static constexpr uint32_t kSmall = (kPrepEnd > kSolveEnd ? kPrepEnd : kSolveEnd);
   static constexpr uint32_t kAcar = kSmall, kGC = kSmall + 512;
@@ -211,16 +214,24 @@ struct K1Layout {
   static constexpr uint32_t kMu = kSmall + 5120, kBeta = kSmall + 5376, kGS = kSmall + 5632;
   static constexpr uint32_t kLas = kSmall + 5888;
   static constexpr uint32_t kEGS = kSmall + 6144;  // float[64] e^{G_t}, scalar decay
-  // channel decay, float[9][128]: e^{B_1}, e^{B_2}, e^{B_3}, e^{B_2 - B_1},
-  // e^{B_3 - B_1}, e^{B_3 - B_2}, e^{G_C - B_1}, e^{G_C - B_2}, e^{G_C - B_3}
+  // channel decay, float[13][128]: e^{B_1}, e^{B_2}, e^{B_3}, e^{B_2 - B_1},
+  // e^{B_3 - B_1}, e^{B_3 - B_2}, e^{G_C - B_1}, e^{G_C - B_2}, e^{G_C - B_3},
+  // then e^{B_a - B_{a+1}} for a = 0..3 (B_4 = G_C; read only for sub-chunks
+  // that are not flagged, where it is at most e^{kSubRange})
   static constexpr uint32_t kTab = kSmall + 6400;
-  static constexpr uint32_t kFlags = kTab + (kCh ? 9 * 512 : 0);  // bit a: sub-chunk a flagged
+  static constexpr uint32_t kFlags = kTab + (kCh ? 13 * 512 : 0);  // bit a: sub-chunk a flagged
   static constexpr uint32_t kBar = kFlags + 16;
   static constexpr uint32_t kTbase = kBar + 16;
   static constexpr uint32_t kBytes = kTbase + 16;
   static constexpr uint32_t kTmemCols = kCh ? 256 : 128;
   static constexpr uint32_t kTmY = kN1;  // TMEM column of Y^T (after MMA1's columns)
 };
+static_assert(K1Layout<PDN_VAR_GDN2, PDN_DECAY_CHANNEL>::kBytes <= 232448 &&
+                  K1Layout<PDN_VAR_PKDA, PDN_DECAY_CHANNEL>::kBytes <= 232448 &&
+                  K1Layout<PDN_VAR_FG2_GDN, PDN_DECAY_CHANNEL>::kBytes <= 232448,
+              "intra-chunk kernel shared memory budget");
+static_assert(2 * (K1Layout<PDN_VAR_PGDN, PDN_DECAY_SCALAR>::kBytes + 1024) <= 233472,
+              "two intra-chunk CTAs per SM for scalar decay");
 
 __device__ __forceinline__ void sync_for_mma() {
   fence_proxy_async_smem();
@@ -354,8 +365,12 @@ __global__ void __launch_bounds__(kK1Threads, kDecay == PDN_DECAY_CHANNEL ? 1 : 
     }
     cp_async_commit();
   };
-  // k of a chunk block into the R half of the [R; Q] tile's space (same
-  // swizzled rows); issued once MMA2 of the previous block has read R.
+  // k of a chunk block, rows of 256 bytes swizzled like v: channel decay into
+  // rows 64.. of the B operand (dead once MMA1 has completed, and its 40 KiB
+  // leave room after v), issued right after MMA1; otherwise into the R half
+  // of the [R; Q] tile's space, issued once MMA2 of the previous block has
+  // read R.
+  constexpr uint32_t kKStage = kCh ? L::kWH + 16384 : L::kRQ;
   auto stage_k = [&](int it) {
     const int c_ = it / BH, bh_ = it % BH;
     const int b_ = bh_ / P.H, h_ = bh_ % P.H;
@@ -366,7 +381,7 @@ __global__ void __launch_bounds__(kK1Threads, kDecay == PDN_DECAY_CHANNEL ? 1 : 
       const int t = (tid >> 4) + 16 * m, c8 = tid & 15;
       const bool ok = t < Cn_;
       const size_t e = ok ? tok0_ + (size_t)t * tstride + c8 * 8 : 0;
-      cp_async16(sb + L::kRQ + t * 256 + ((c8 ^ (t & 7)) << 4),
+      cp_async16(sb + kKStage + t * 256 + ((c8 ^ (t & 7)) << 4),
                  reinterpret_cast<const __nv_bfloat16 *>(P.k) + e, ok);
     }
     cp_async_commit();
@@ -391,19 +406,13 @@ __global__ void __launch_bounds__(kK1Threads, kDecay == PDN_DECAY_CHANNEL ? 1 : 
   // scalars into shared memory; then start loading the next block's ----
   uint4 vcur[4];
   cp_async_wait_all();  // this block's k and v
-  if (tid == 0) bulk_wait_read0();  // the previous block's bulk stores have read their tiles
   __syncthreads();
   {
 #pragma unroll
     for (int m = 0; m < 4; ++m) {
       const int t = (tid >> 4) + 16 * m, c8 = tid & 15;
       *reinterpret_cast<uint4 *>(smem + L::kKS + t * KS_LD + c8 * 16) =
-          *reinterpret_cast<const uint4 *>(smem + L::kRQ + t * 256 + ((c8 ^ (t & 7)) << 4));
-      {
-        const bool ok = t < Cn;
-        const size_t e = ok ? tok0 + (size_t)t * tstride + c8 * 8 : 0;
-        cp_async16(sb + L::kQS + t * KS_LD + c8 * 16, reinterpret_cast<const __nv_bfloat16 *>(P.q) + e, ok);
-      }
+          *reinterpret_cast<const uint4 *>(smem + kKStage + t * 256 + ((c8 ^ (t & 7)) << 4));
       if (kCh) {
         const bool ok = t < Cn;
         const size_t e = ok ? tok0 + (size_t)t * tstride + c8 * 8 : 0;
@@ -411,7 +420,22 @@ __global__ void __launch_bounds__(kK1Threads, kDecay == PDN_DECAY_CHANNEL ? 1 : 
                    reinterpret_cast<const __nv_bfloat16 *>(P.log_alpha) + e, ok);
       }
     }
-    cp_async_commit();
+    cp_async_commit();  // group: channel log decay (P1)
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+      const int t = (tid >> 4) + 16 * m, c8 = tid & 15;
+      const bool ok = t < Cn;
+      const size_t e = ok ? tok0 + (size_t)t * tstride + c8 * 8 : 0;
+      cp_async16(sb + L::kQS + t * KS_LD + c8 * 16, reinterpret_cast<const __nv_bfloat16 *>(P.q) + e, ok);
+      // gates, rows of 256 bytes with the 16-byte groups swizzled by (token & 7)
+      const uint32_t gs = sb + L::kGateStage + t * 256 + ((c8 ^ (t & 7)) << 4);
+      if (L::kGates >= 1)
+        cp_async16(gs, reinterpret_cast<const __nv_bfloat16 *>(
+                           kVariant == PDN_VAR_FG2_GDN ? P.beta : P.erase) + e, ok);
+      if (L::kGates == 2)
+        cp_async16(gs + 16384, reinterpret_cast<const __nv_bfloat16 *>(P.write) + e, ok);
+    }
+    cp_async_commit();  // group: q and the gates (P3)
     if (tid < kC) {
       BETA[tid] = pf.beta;
       LAS[tid] = pf.las;
@@ -420,7 +444,7 @@ __global__ void __launch_bounds__(kK1Threads, kDecay == PDN_DECAY_CHANNEL ? 1 : 
     if (kCh && tid == 0) *flags = 0u;
   }
   if (it + (int)gridDim.x < total) pf = load_raw(it + gridDim.x);
-  if (kCh) cp_async_wait_all();  // P1 scans the channel log decay
+  if (kCh) cp_async_wait_group<1>();  // P1 scans the channel log decay
   __syncthreads();
 
   // ---- P1: per-channel scans; thread = (channel pair, quarter of the chunk) ----
@@ -559,6 +583,10 @@ __global__ void __launch_bounds__(kK1Threads, kDecay == PDN_DECAY_CHANNEL ? 1 : 
       TAB[6 * kD + tid] = ex2_approx((Gc - B1) * kLog2e);
       TAB[7 * kD + tid] = ex2_approx((Gc - B2) * kLog2e);
       TAB[8 * kD + tid] = ex2_approx((Gc - B3) * kLog2e);
+      TAB[9 * kD + tid] = ex2_approx(-B1 * kLog2e);
+      TAB[10 * kD + tid] = ex2_approx((B1 - B2) * kLog2e);
+      TAB[11 * kD + tid] = ex2_approx((B2 - B3) * kLog2e);
+      TAB[12 * kD + tid] = ex2_approx((B3 - Gc) * kLog2e);
       uint32_t m = 0;
       if (-B1 > kSubRange) m |= 1u;
       if (B1 - B2 > kSubRange) m |= 2u;
@@ -607,7 +635,10 @@ __global__ void __launch_bounds__(kK1Threads, kDecay == PDN_DECAY_CHANNEL ? 1 : 
         float gb[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) gb[e] = 0.f;
-        if (ok)
+        if (L::kGates)
+          unpack8(*reinterpret_cast<const uint4 *>(smem + L::kGateStage + t * 256 + ((c8 ^ (t & 7)) << 4)),
+                  gb);
+        else if (ok)
           unpack8(__ldg(reinterpret_cast<const uint4 *>(
                       reinterpret_cast<const __nv_bfloat16 *>(P.beta) + etok + i0)), gb);
 #pragma unroll
@@ -621,7 +652,11 @@ __global__ void __launch_bounds__(kK1Threads, kDecay == PDN_DECAY_CHANNEL ? 1 : 
         float ge[8], gw[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) { ge[e] = 0.f; gw[e] = 0.f; }
-        if (ok) {
+        if (L::kGates) {
+          const uint8_t *gsrc = smem + L::kGateStage + t * 256 + ((c8 ^ (t & 7)) << 4);
+          unpack8(*reinterpret_cast<const uint4 *>(gsrc), ge);
+          unpack8(*reinterpret_cast<const uint4 *>(gsrc + 16384), gw);
+        } else if (ok) {
           unpack8(__ldg(reinterpret_cast<const uint4 *>(
                       reinterpret_cast<const __nv_bfloat16 *>(P.erase) + etok + i0)), ge);
           unpack8(__ldg(reinterpret_cast<const uint4 *>(
@@ -642,7 +677,7 @@ __global__ void __launch_bounds__(kK1Threads, kDecay == PDN_DECAY_CHANNEL ? 1 : 
       }
       float rr[8], qq[8], wh[8], qh[8], wb[8];
       if (kCh) {
-        float G[8], Bl[8], Bh[8], eBl[8], wbf[8];
+        float G[8], Bl[8], Bh[8], eBl[8], wbf[8], rsub[8];
         ld8f(GBUF + t * LB_LD + i0, G);
         ld8f(GBUF + (16 * a + 15) * LB_LD + i0, Bh);  // B_{a+1} (G_C for a = 3)
         if (a > 0) {
@@ -659,6 +694,7 @@ __global__ void __launch_bounds__(kK1Threads, kDecay == PDN_DECAY_CHANNEL ? 1 : 
           for (int e = 0; e < 8; ++e) wbf[e] = 1.f;
         }
         const bool bad_a = (badm >> a) & 1u;
+        ld8f(TAB + (9 + a) * kD + i0, rsub);  // e^{B_a - B_{a+1}}
         float wy[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
@@ -668,7 +704,7 @@ __global__ void __launch_bounds__(kK1Threads, kDecay == PDN_DECAY_CHANNEL ? 1 : 
           qq[e] = qf[e] * rho;
           qh[e] = qf[e] * (rho * eBl[e]);
           wb[e] = w[e] * (y * wbf[e]);
-          wh[e] = bad_a ? 0.f : w[e] * rcp_approx(rho);  // diagonal group: e^{B_a - G_t}
+          wh[e] = bad_a ? 0.f : w[e] * (y * rsub[e]);  // diagonal group: e^{B_a - G_t}
           wy[e] = w[e] * y;
         }
         *reinterpret_cast<uint4 *>(smem + L::kWH + tl128(grp_off(a) + t, c8)) = pack8(wh);
@@ -732,7 +768,10 @@ __global__ void __launch_bounds__(kK1Threads, kDecay == PDN_DECAY_CHANNEL ? 1 : 
   }
 
   if (ok_all) {
-    if (it + (int)gridDim.x < total) stage_v(it + gridDim.x);
+    if (it + (int)gridDim.x < total) {
+      stage_v(it + gridDim.x);
+      if (kCh) stage_k(it + gridDim.x);
+    }
     // ---- epilogue of MMA1: M = strict lower (rows 0-63), P = lower (rows
     // 64-127) with their in-chunk decay, first into registers ----
     const int row = 32 * (warp & 3) + lane;
@@ -811,8 +850,9 @@ __global__ void __launch_bounds__(kK1Threads, kDecay == PDN_DECAY_CHANNEL ? 1 : 
         float lo8[8], hi8[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) { lo8[e] = mv[cc][e]; hi8[e] = mv[cc][8 + e]; }
-        *reinterpret_cast<uint4 *>(smem + L::kPM + tl64(tr, s0 / 8)) = pack8(lo8);
-        *reinterpret_cast<uint4 *>(smem + L::kPM + tl64(tr, s0 / 8 + 1)) = pack8(hi8);
+        // P goes straight to the workspace (only the state kernel reads it)
+        *reinterpret_cast<uint4 *>(blk + WS_P + tl64(tr, s0 / 8)) = pack8(lo8);
+        *reinterpret_cast<uint4 *>(blk + WS_P + tl64(tr, s0 / 8 + 1)) = pack8(hi8);
       }
     }
     tc_fence_before();
@@ -923,8 +963,8 @@ __global__ void __launch_bounds__(kK1Threads, kDecay == PDN_DECAY_CHANNEL ? 1 : 
       *reinterpret_cast<float2 *>(TS + (32 + r0 + 1) * TS_LD + c0b) = make_float2(-a10, -a11);
     }
     __syncthreads();
-    // T to its bf16 tile. Scalar decay: MMA2 multiplies the undecayed R, so
-    // its tile holds T Diag(e^{G_s}) and T itself goes to the workspace here.
+    // T to the workspace and to MMA2's operand tile; for scalar decay MMA2
+    // multiplies the undecayed R, so its tile holds T Diag(e^{G_s}).
 #pragma unroll
     for (int m = 0; m < 2; ++m) {
       const int t = 8 * warp + (lane & 7), s8 = 4 * m + (lane >> 3);
@@ -932,8 +972,8 @@ __global__ void __launch_bounds__(kK1Threads, kDecay == PDN_DECAY_CHANNEL ? 1 : 
       ld8f(TS + t * TS_LD + 8 * s8, v);
 #pragma unroll
       for (int e = 0; e < 8; ++e) v[e] = (8 * s8 + e <= t) ? v[e] : 0.f;
+      *reinterpret_cast<uint4 *>(blk + WS_T + tl64(t, s8)) = pack8(v);
       if (kSc) {
-        *reinterpret_cast<uint4 *>(blk + WS_T + tl64(t, s8)) = pack8(v);
 #pragma unroll
         for (int e = 0; e < 8; ++e) v[e] *= EGS[8 * s8 + e];
       }
@@ -958,8 +998,8 @@ __global__ void __launch_bounds__(kK1Threads, kDecay == PDN_DECAY_CHANNEL ? 1 : 
     }
     if (ok_all) {
       // R is dead: the next block's k goes into its space
-      if (it + (int)gridDim.x < total) stage_k(it + gridDim.x);
-      // Y^T -> bf16 tile (rows d_k, columns tokens)
+      if (!kCh && it + (int)gridDim.x < total) stage_k(it + gridDim.x);
+      // Y^T -> bf16, straight to the workspace (rows d_k, columns tokens)
       const int i = 32 * (warp & 3) + lane;
 #pragma unroll
       for (int cc = 0; cc < 2; ++cc) {
@@ -970,18 +1010,8 @@ __global__ void __launch_bounds__(kK1Threads, kDecay == PDN_DECAY_CHANNEL ? 1 : 
 #pragma unroll
         for (int e = 0; e < 8; ++e) { lo[e] = v[e]; hi[e] = v[8 + e]; }
         const int t8 = 4 * half + 2 * cc;
-        *reinterpret_cast<uint4 *>(smem + L::kYT + tl64(i, t8)) = pack8(lo);
-        *reinterpret_cast<uint4 *>(smem + L::kYT + tl64(i, t8 + 1)) = pack8(hi);
-      }
-      // ---- the tiles that live in shared memory go out with bulk stores ----
-      fence_proxy_async_smem();
-      tc_fence_before();
-      __syncthreads();
-      if (tid == 0) {
-        bulk_s2g(blk + WS_Y, smem + L::kYT, 16384);
-        if (!kSc) bulk_s2g(blk + WS_T, smem + L::kTM, 8192);
-        bulk_s2g(blk + WS_P, smem + L::kPM, 8192);
-        bulk_commit();  // their reads are awaited before the next block rewrites the tiles
+        *reinterpret_cast<uint4 *>(blk + WS_Y + tl64(i, t8)) = pack8(lo);
+        *reinterpret_cast<uint4 *>(blk + WS_Y + tl64(i, t8 + 1)) = pack8(hi);
       }
     }
   }
@@ -989,12 +1019,11 @@ __global__ void __launch_bounds__(kK1Threads, kDecay == PDN_DECAY_CHANNEL ? 1 : 
     if (tid == 0) record_error(P.err, PDN_ERR_TIMEOUT);
     break;
   }
-  // the next block rewrites the shared-memory tiles the bulk stores read
+  // the next block reuses the shared memory and the TMEM columns read above
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   }  // chunk blocks
-  if (tid == 0) bulk_wait0();
   cp_async_wait_all();  // a prefetch issued before an abort
   tc_fence_before();
   __syncthreads();
@@ -1048,6 +1077,8 @@ constexpr uint32_t K2_UT = 3 * KM_SIZE;            // two U/T buffers
 constexpr uint32_t K2_BAR = K2_UT + 2 * KU_SIZE;   // the fifteen mbarriers above
 constexpr uint32_t K2_ABORT = K2_BAR + 16 * 8;
 constexpr uint32_t K2_TBASE = K2_ABORT + 8;
+// e^{G_C} of the current and the next chunk, one copy per compute warp (the
+// 32 key channels of its column group), fetched by the warp itself
 // e^{G_C} of the current and the next chunk, one copy per compute warp (the
 // 32 key channels of its column group), fetched by the warp itself
 constexpr uint32_t K2_EBUF = (K2_TBASE + 16 + 127) / 128 * 128;
