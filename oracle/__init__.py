@@ -30,9 +30,9 @@ _lock = threading.Lock()
 _lib = None
 
 VARIANTS = {"DN": 0, "GDN": 1, "KDA": 2, "PDN": 3, "PGDN": 4, "PKDA": 5,
-            "FG2_GDN": 6, "GDN2": 7}
+            "FG2_GDN": 6, "GDN2": 7, "PLA": 8, "FG2_GDN_PLUS": 9}
 DECAYS = {"none": 0, "scalar": 1, "channel": 2}
-PRECOND_VARIANTS = ("PDN", "PGDN", "PKDA")
+PRECOND_VARIANTS = ("PDN", "PGDN", "PKDA", "PLA")
 
 
 def build(force: bool = False) -> str:
@@ -90,8 +90,10 @@ def forward(variant, q, k, v, log_alpha=None, beta=None, erase=None, write=None,
     """Run the token-by-token recurrence for ``variant``.
 
     Shapes: q, k [B,T,H,dk]; v [B,T,H,dv]; log_alpha None | [B,T,H] (scalar
-    decay) | [B,T,H,dk] (channel decay); beta [B,T,H] | [B,T,H,dk] (FG2_GDN);
-    erase [B,T,H,dk], write [B,T,H,dv] (GDN2); S0 [B,H,dv,dk]; A0 [B,H,dk].
+    decay) | [B,T,H,dk] (channel decay); beta [B,T,H] | [B,T,H,dk] (FG2_GDN,
+    FG2_GDN_PLUS: the key-side gain); erase [B,T,H,dk] (GDN2); write
+    [B,T,H,dv] (GDN2's write gate, FG2_GDN_PLUS's value-side gain);
+    S0 [B,H,dv,dk]; A0 [B,H,dk].
     Returns (o [B,T,H,dv] or None, S_T [B,H,dv,dk], A_T [B,H,dk]) in fp64.
     """
     lib = _load()

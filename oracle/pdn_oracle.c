@@ -28,6 +28,8 @@
  *   PDN/PGDN/PKDA   r = k,          w = beta (B_t . k),  u = v
  *   FG2-GDN         r = sqrt(b).k,  w = sqrt(b).k,       u = sqrt(b).v
  *   GDN-2           r = e . k,      w = k,               u = g . v
+ *   PLA             r = 0,          w = beta k,          u = v,  query B_t . q
+ *   FG2-GDN+        r = sqrt(bk).k, w = sqrt(bk).k,      u = sqrt(bv).v
  * (". " is the elementwise product.)
  *
  * Parity status of each function is stated in its comment.
@@ -39,7 +41,7 @@
 #include <unistd.h>
 
 enum { OR_DN = 0, OR_GDN = 1, OR_KDA = 2, OR_PDN = 3, OR_PGDN = 4, OR_PKDA = 5,
-       OR_FG2 = 6, OR_GDN2 = 7 };
+       OR_FG2 = 6, OR_GDN2 = 7, OR_PLA = 8, OR_FG2P = 9 };
 enum { OR_DECAY_NONE = 0, OR_DECAY_SCALAR = 1, OR_DECAY_CHANNEL = 2 };
 
 /* ------------------------------------------------------------------------ */
@@ -131,7 +133,7 @@ typedef struct {
 } job_t;
 
 static int uses_precond(int variant) {
-  return variant == OR_PDN || variant == OR_PGDN || variant == OR_PKDA;
+  return variant == OR_PDN || variant == OR_PGDN || variant == OR_PKDA || variant == OR_PLA;
 }
 
 /* Forms r, w, u for one token (variant table in the file header).
@@ -140,7 +142,19 @@ static int uses_precond(int variant) {
  * [FG2] ja §2.1: per-channel beta vector applied as sqrt(beta) to both
  *   k and v (requires d_k = d_v).
  * [PDN] ja §2.2 "read key / write key": read key k_t, write key B_t . k_t
- *   (apply-to-key), scaled by the gain beta_t as in DeltaNet. */
+ *   (apply-to-key), scaled by the gain beta_t as in DeltaNet.
+ * [PDN] ja §2.1 and fr §2.A: preconditioned linear attention (PLA) applies
+ *   the preconditioner to the query instead (apply-to-query); linear
+ *   attention writes without erasing, so its read key is 0 and its write is
+ *   the gain times k_t (reading: the gain beta_t of the family's gain axis,
+ *   1 for plain linear attention); the query transform is applied in
+ *   run_unit.
+ * [FG2] ja §2.2: FG2-GDN+ gives the key (erase strength) and the value (write
+ *   strength) gain vectors of their own, beta^k in R^{d_k} and beta^v in
+ *   R^{d_v}. The page prints no formula; the reading taken keeps FG2-GDN's
+ *   symmetric square roots: sqrt(beta^k) on the key, sqrt(beta^v) on the
+ *   value, so beta^k = beta^v is FG2-GDN (parity against the paper
+ *   unpinned). beta^v arrives in the write-gate slot. */
 static void form_vectors(const job_t *J, size_t tok, size_t tokh, const double *Bt,
                          double *r, double *w, double *u) {
   const int dk = J->dk, dv = J->dv;
@@ -172,6 +186,21 @@ static void form_vectors(const job_t *J, size_t tok, size_t tokh, const double *
     for (int i = 0; i < dk; ++i) { r[i] = et[i] * kt[i]; w[i] = kt[i]; }
     for (int j = 0; j < dv; ++j) u[j] = gt[j] * vt[j];
   } break;
+  case OR_PLA: {
+    const double b = J->beta[tokh];
+    for (int i = 0; i < dk; ++i) { r[i] = 0.0; w[i] = b * kt[i]; }
+    for (int j = 0; j < dv; ++j) u[j] = vt[j];
+  } break;
+  case OR_FG2P: {
+    const double *bk = J->beta + tok * dk;
+    const double *bv = J->write_gate + tok * dv;
+    for (int i = 0; i < dk; ++i) {
+      const double sb = sqrt(bk[i]);
+      r[i] = sb * kt[i];
+      w[i] = sb * kt[i];
+    }
+    for (int j = 0; j < dv; ++j) u[j] = sqrt(bv[j]) * vt[j];
+  } break;
   }
 }
 
@@ -185,8 +214,9 @@ static int run_unit(job_t *J, int unit) {
   double *r = (double *)malloc(sizeof(double) * (size_t)dk);
   double *w = (double *)malloc(sizeof(double) * (size_t)dk);
   double *u = (double *)malloc(sizeof(double) * (size_t)dv);
-  if (!S || !A || !Bt || !alpha || !r || !w || !u) {
-    free(S); free(A); free(Bt); free(alpha); free(r); free(w); free(u);
+  double *qq = (double *)malloc(sizeof(double) * (size_t)dk);
+  if (!S || !A || !Bt || !alpha || !r || !w || !u || !qq) {
+    free(S); free(A); free(Bt); free(alpha); free(r); free(w); free(u); free(qq);
     return 2;
   }
   const size_t sidx = ((size_t)b * H + h) * (size_t)dk * dv;
@@ -208,7 +238,7 @@ static int run_unit(job_t *J, int unit) {
       for (int i = 0; i < dk; ++i) alpha[i] = exp(la[i]);
       al = alpha;
     }
-    const double *rr, *ww, *uu;
+    const double *rr, *ww, *uu, *qt = J->q + tokh * dk;
     if (J->generic) {
       rr = J->r + tokh * dk;
       ww = J->w + tokh * dk;
@@ -218,13 +248,16 @@ static int run_unit(job_t *J, int unit) {
         precond_step(dk, J->k + tokh * dk, A, J->x, J->eps, Bt);
       form_vectors(J, tokh, tokh, Bt, r, w, u);
       rr = r; ww = w; uu = u;
+      if (J->variant == OR_PLA) { /* apply-to-query: read out S_t (B_t . q_t) */
+        for (int i = 0; i < dk; ++i) qq[i] = Bt[i] * qt[i];
+        qt = qq;
+      }
     }
-    token_step(dk, dv, S, al, rr, ww, uu, J->q + tokh * dk, J->q_scale,
-               J->o ? J->o + tokh * dv : NULL);
+    token_step(dk, dv, S, al, rr, ww, uu, qt, J->q_scale, J->o ? J->o + tokh * dv : NULL);
   }
   if (J->ST) memcpy(J->ST + sidx, S, sizeof(double) * (size_t)dk * dv);
   if (J->AT) memcpy(J->AT + ((size_t)b * H + h) * dk, A, sizeof(double) * (size_t)dk);
-  free(S); free(A); free(Bt); free(alpha); free(r); free(w); free(u);
+  free(S); free(A); free(Bt); free(alpha); free(r); free(w); free(u); free(qq);
   return 0;
 }
 
@@ -270,8 +303,9 @@ static int run_job(job_t *J, int nthreads) {
 
 /* Variant forward: o [B,T,H,dv], ST [B,H,dv,dk], AT [B,H,dk] (any may be NULL).
  * Inputs use the [B,T,H,d] layout; log_alpha is [B,T,H] (scalar decay) or
- * [B,T,H,dk] (channel decay); beta is [B,T,H] or [B,T,H,dk] (FG2);
- * erase [B,T,H,dk] and write_gate [B,T,H,dv] for GDN-2 only.
+ * [B,T,H,dk] (channel decay); beta is [B,T,H] or [B,T,H,dk] (FG2, FG2+);
+ * erase [B,T,H,dk] for GDN-2, write_gate [B,T,H,dv] for GDN-2 (write gate)
+ * and FG2+ (value-side gain beta^v).
  * Returns 0 on success, 1 on bad arguments, 2 on allocation failure. */
 int oracle_forward(int variant, int decay, int B, int T, int H, int dk, int dv,
                    const double *q, const double *k, const double *v,
@@ -280,7 +314,7 @@ int oracle_forward(int variant, int decay, int B, int T, int H, int dk, int dv,
                    const double *S0, const double *A0, double q_scale, double x,
                    double eps, double *o, double *ST, double *AT, int nthreads) {
   if (B < 0 || T < 0 || H < 0 || dk <= 0 || dv <= 0) return 1;
-  if (variant < OR_DN || variant > OR_GDN2) return 1;
+  if (variant < OR_DN || variant > OR_FG2P) return 1;
   if (decay < OR_DECAY_NONE || decay > OR_DECAY_CHANNEL) return 1;
   if (!q || !k || !v) return 1;
   if (decay != OR_DECAY_NONE && !log_alpha) return 1;
@@ -289,6 +323,7 @@ int oracle_forward(int variant, int decay, int B, int T, int H, int dk, int dv,
   } else if (!beta) {
     return 1;
   }
+  if (variant == OR_FG2P && !write_gate) return 1;
   if (variant == OR_FG2 && dk != dv) return 1;
   job_t J;
   memset(&J, 0, sizeof(J));

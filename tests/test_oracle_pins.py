@@ -12,9 +12,10 @@ import pytest
 import oracle
 from oracle import chunked
 
-VARIANTS = ["DN", "GDN", "KDA", "PDN", "PGDN", "PKDA", "FG2_GDN", "GDN2"]
+VARIANTS = ["DN", "GDN", "KDA", "PDN", "PGDN", "PKDA", "FG2_GDN", "GDN2", "PLA", "FG2_GDN_PLUS"]
 DECAY = {"DN": "none", "PDN": "none", "GDN": "scalar", "PGDN": "scalar",
-         "KDA": "channel", "PKDA": "channel", "FG2_GDN": "channel", "GDN2": "channel"}
+         "KDA": "channel", "PKDA": "channel", "FG2_GDN": "channel", "GDN2": "channel",
+         "PLA": "channel", "FG2_GDN_PLUS": "channel"}
 
 
 def unit(x):
@@ -27,7 +28,7 @@ def rand_inputs(variant, B=2, T=9, H=2, dk=8, dv=8, seed=0, decay=None, S0=True)
     d = dict(q=unit(rng.standard_normal((B, T, H, dk))),
              k=unit(rng.standard_normal((B, T, H, dk))),
              v=rng.standard_normal((B, T, H, dv)))
-    if variant == "FG2_GDN":
+    if variant in ("FG2_GDN", "FG2_GDN_PLUS"):
         d["beta"] = 1 / (1 + np.exp(-rng.standard_normal((B, T, H, dk))))
     elif variant != "GDN2":
         d["beta"] = 1 / (1 + np.exp(-rng.standard_normal((B, T, H))))
@@ -37,6 +38,8 @@ def rand_inputs(variant, B=2, T=9, H=2, dk=8, dv=8, seed=0, decay=None, S0=True)
         d["log_alpha"] = -0.3 * np.abs(rng.standard_normal((B, T, H, dk)))
     if variant == "GDN2":
         d["erase"] = 1 / (1 + np.exp(-rng.standard_normal((B, T, H, dk))))
+        d["write"] = 1 / (1 + np.exp(-rng.standard_normal((B, T, H, dv))))
+    if variant == "FG2_GDN_PLUS":
         d["write"] = 1 / (1 + np.exp(-rng.standard_normal((B, T, H, dv))))
     if S0:
         d["S0"] = 0.5 * rng.standard_normal((B, H, dv, dk))
@@ -62,7 +65,8 @@ def test_p1_zero_gain_leaves_only_decay(variant):
     for n in ("beta", "erase", "write"):
         if n in d:
             d[n] = np.zeros_like(d[n])
-    o, ST, _ = oracle.forward(variant, **d, q_scale=0.7)
+    # (PLA reads out through the preconditioned query B_t . q: x = 1 makes B = 1)
+    o, ST, _ = oracle.forward(variant, **d, q_scale=0.7, x=1.0 if variant == "PLA" else 1.5)
     cum = decay_cum(d.get("log_alpha"), d["k"].shape)
     B, T, H, _ = d["k"].shape
     for b in range(B):
@@ -178,6 +182,11 @@ def variant_vectors(variant, d, b, t, h, Bc=None):
     if variant == "FG2_GDN":
         sb = np.sqrt(d["beta"][b, t, h])
         return sb * k, sb * k, sb * v
+    if variant == "PLA":
+        return np.zeros_like(k), d["beta"][b, t, h] * k, v
+    if variant == "FG2_GDN_PLUS":
+        sk = np.sqrt(d["beta"][b, t, h])
+        return sk * k, sk * k, np.sqrt(d["write"][b, t, h]) * v
     return d["erase"][b, t, h] * k, k, d["write"][b, t, h] * v
 
 
@@ -191,7 +200,7 @@ def test_p6_brute_force_product_expansion(variant, T):
     o, ST, AT = oracle.forward(variant, **d, q_scale=1.3)
     dk = 5
     Bc = None
-    if variant in ("PDN", "PGDN", "PKDA"):
+    if variant in ("PDN", "PGDN", "PKDA", "PLA"):
         Bc, _ = oracle.precond(d["k"][0, :, 0], x=1.5)
     la = d.get("log_alpha")
     mats, outer = [], []
@@ -214,9 +223,86 @@ def test_p6_brute_force_product_expansion(variant, T):
             for s in range(t + 1, tt):
                 term = term @ mats[s]
             S = S + term
-        np.testing.assert_allclose(o[0, tt - 1, 0], 1.3 * S @ d["q"][0, tt - 1, 0], rtol=1e-12, atol=1e-12)
+        qt = d["q"][0, tt - 1, 0] * (Bc[tt - 1] if variant == "PLA" else 1.0)
+        np.testing.assert_allclose(o[0, tt - 1, 0], 1.3 * S @ qt, rtol=1e-12, atol=1e-12)
         if tt == T:
             np.testing.assert_allclose(ST[0, 0], S, rtol=1e-12, atol=1e-12)
+
+
+# ---------------------------------------------------------------- PLA and FG2-GDN+
+@pytest.mark.parametrize("decay", ["none", "scalar", "channel"])
+def test_pla_identity_preconditioner_is_decayed_linear_attention(decay):
+    """PLA with x = 1 (B_t = 1) is linear attention with the gain and the
+    decay axes: no erase, so
+    o_t = q_scale (S_0 Diag(prod_{s<=t} alpha_s) + sum_{s<=t} beta_s v_s (k_s . prod_{s<tau<=t} alpha_tau)^T) q_t,
+    written out as the explicit sum ("Preconditioned DeltaNet" ja §2.1:
+    linear attention; fr §2.D: decay and gain axes)."""
+    d = rand_inputs("PLA", seed=31, decay=decay, T=10)
+    o, ST, _ = oracle.forward("PLA", **d, x=1.0, q_scale=0.8)
+    B, T, H, dk = d["k"].shape
+    la = d.get("log_alpha")
+    for b in range(B):
+        for h in range(H):
+            if la is None:
+                lac = np.zeros((T, dk))
+            elif la.ndim == 3:
+                lac = np.repeat(la[b, :, h][:, None], dk, axis=1)
+            else:
+                lac = la[b, :, h]
+            for t in range(T):
+                S = d["S0"][b, h] * np.exp(lac[: t + 1].sum(axis=0))[None, :]
+                for s in range(t + 1):
+                    g = np.exp(lac[s + 1: t + 1].sum(axis=0))
+                    S = S + d["beta"][b, s, h] * np.outer(d["v"][b, s, h], d["k"][b, s, h] * g)
+                np.testing.assert_allclose(o[b, t, h], 0.8 * S @ d["q"][b, t, h], rtol=1e-11, atol=1e-12)
+            np.testing.assert_allclose(ST[b, h], S, rtol=1e-11, atol=1e-12)
+
+
+def test_pla_preconditions_the_query_only():
+    """Apply-to-query ("Preconditioned DeltaNet" fr §2.A): the preconditioner
+    touches only the read-out, so PLA's state is the same for every x, and its
+    output is the x = 1 output read with the query B_t . q_t; the accumulator
+    A is the running sum of k . k either way."""
+    d = rand_inputs("PLA", seed=32, T=12)
+    o15, S15, A15 = oracle.forward("PLA", **d, x=1.5)
+    o1, S1, A1 = oracle.forward("PLA", **d, x=1.0)
+    np.testing.assert_array_equal(S15, S1)
+    B, T, H, dk = d["k"].shape
+    qB = d["q"].copy()
+    for b in range(B):
+        for h in range(H):
+            Bc, _ = oracle.precond(d["k"][b, :, h], x=1.5)
+            qB[b, :, h] *= Bc
+    oq, _, _ = oracle.forward("PLA", **dict(d, q=qB), x=1.0)
+    np.testing.assert_allclose(o15, oq, rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(A15, np.sum(d["k"] ** 2, axis=1), rtol=1e-13)
+
+
+@pytest.mark.parametrize("decay", ["scalar", "channel"])
+def test_fg2_plus_reductions(decay):
+    """FG2-GDN+ ("FG2-GDN" ja §2.2: separate key-side and value-side gain
+    vectors): beta^v = beta^k is FG2-GDN exactly; beta^k = 1 is the delta rule
+    with unit gain on the values sqrt(beta^v) . v (KDA, or GDN for scalar
+    decay); beta^v = 0 with S_0 = 0 writes nothing."""
+    d = rand_inputs("FG2_GDN_PLUS", seed=33, decay=decay)
+    d["write"] = d["beta"].copy()
+    o1, S1, _ = oracle.forward("FG2_GDN_PLUS", **d)
+    o2, S2, _ = oracle.forward("FG2_GDN", **{n: a for n, a in d.items() if n != "write"})
+    np.testing.assert_array_equal(o1, o2)
+    np.testing.assert_array_equal(S1, S2)
+    d = rand_inputs("FG2_GDN_PLUS", seed=34, decay=decay)
+    d["beta"] = np.ones_like(d["beta"])
+    o3, S3, _ = oracle.forward("FG2_GDN_PLUS", **d)
+    base = {n: d[n] for n in ("q", "k", "log_alpha", "S0")}
+    base["v"] = np.sqrt(d["write"]) * d["v"]
+    base["beta"] = np.ones(d["k"].shape[:3])
+    o4, S4, _ = oracle.forward("GDN" if decay == "scalar" else "KDA", **base)
+    np.testing.assert_allclose(o3, o4, rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(S3, S4, rtol=1e-12, atol=1e-13)
+    d = rand_inputs("FG2_GDN_PLUS", seed=35, decay=decay, S0=False)
+    d["write"] = np.zeros_like(d["write"])
+    o5, S5, _ = oracle.forward("FG2_GDN_PLUS", **d)
+    assert not o5.any() and not S5.any()
 
 
 # ---------------------------------------------------------------- P7
@@ -378,6 +464,10 @@ def test_oracle_rejects_bad_arguments():
     d = rand_inputs("FG2_GDN", dk=8, dv=6)
     with pytest.raises(ValueError):
         oracle.forward("FG2_GDN", **d)  # FG2 needs d_k == d_v
+    d = rand_inputs("FG2_GDN_PLUS")
+    del d["write"]
+    with pytest.raises(ValueError):
+        oracle.forward("FG2_GDN_PLUS", **d)  # the value-side gain is required
     d = rand_inputs("GDN2")
     del d["erase"]
     with pytest.raises(ValueError):
