@@ -14,7 +14,8 @@ timed steps. The JSON line also carries:
   decode      the recurrent decode workload (256 sequences x 16 heads,
               fp32 state, 1024 steps), tokens/s and HBM roofline;
   workloads   the other forward workloads (Preconditioned KDA B8 T8192;
-              FG2-GDN and Gated DeltaNet-2 B2 T32768): tokens/s, tensor and
+              FG2-GDN and Gated DeltaNet-2 B2 T32768; preconditioned linear
+              attention and FG2-GDN+ at the headline shape): tokens/s, tensor and
               HBM fractions, and per-kernel CUDA-event times (also given for
               the headline layer under roofline.kernel_ms);
   cpu_baseline the fp64 oracle on the host cores on a bounded sample.
@@ -52,6 +53,8 @@ def fwd_bytes_per_token_head(w):
     b = es * (2 * w.dk + 2 * w.dv)
     if w.variant in ("FG2_GDN",):
         b += es * w.dk
+    elif w.variant == "FG2_GDN_PLUS":
+        b += es * (w.dk + w.dv)
     elif w.variant != "GDN2":
         b += 4
     if w.variant == "GDN2":
@@ -406,7 +409,7 @@ def run_ours(args):
         print(json.dumps(result), flush=True)
 
 
-EXTRA_WORKLOADS = ("pkda_bf16_8k", "fg2_bf16_32k", "gdn2_bf16_32k")
+EXTRA_WORKLOADS = ("pkda_bf16_8k", "fg2_bf16_32k", "gdn2_bf16_32k", "pla_bf16_4k", "fg2p_bf16_4k")
 
 
 def profiled_kernel_ms(pdn, prob, tens, ws, sptr, reps=3):

@@ -20,6 +20,15 @@
  *       (decoupled key-side erase gate e and value-side write gate g --
  *        "Gated DeltaNet-2", ja §1 "Gated Delta Rule-2"; the page prints the
  *        transposed d_k x d_v state)
+ *   PLA                 r = 0,          w = beta k,          u = v,
+ *                       read-out o_t = q_scale S_t (B_t . q_t)
+ *       (preconditioned linear attention: the diagonal preconditioner B_t of
+ *        PDN applied to the query, apply-to-query; linear attention does not
+ *        erase -- "Preconditioned DeltaNet", ja §2.1, fr §2.A)
+ *   FG2_GDN_PLUS        r = sqrt(bk).k, w = sqrt(bk).k,      u = sqrt(bv).v
+ *       (separate key-side and value-side gain vectors bk, bv -- "FG2-GDN",
+ *        ja §2.2; the page prints no formula: this reading reduces to FG2_GDN
+ *        at bk = bv)
  * The chunked forward evaluates the same result through the chunkwise WY/UT
  * form the pages describe ("Gated DeltaNet-2", ja §3; "Preconditioned
  * DeltaNet", ja §2.3). The decode step advances one token with the state
@@ -71,7 +80,9 @@ typedef enum {
   PDN_VAR_PGDN = 4,    /* decay must be SCALAR  */
   PDN_VAR_PKDA = 5,    /* decay must be CHANNEL */
   PDN_VAR_FG2_GDN = 6, /* any decay; needs d_k == d_v */
-  PDN_VAR_GDN2 = 7     /* any decay */
+  PDN_VAR_GDN2 = 7,    /* any decay */
+  PDN_VAR_PLA = 8,     /* any decay; preconditioned (takes A0/AT) */
+  PDN_VAR_FG2_GDN_PLUS = 9 /* any decay */
 } pdn_variant_t;
 
 /* Decay axis: none (alpha = 1), scalar alpha per (token, head), or a
@@ -107,14 +118,15 @@ typedef struct {
   const void *q, *k, *v;  /* dtype; [B,T,H,d_k], [B,T,H,d_k], [B,T,H,d_v]        */
   const void *log_alpha;  /* log decay: NULL (NONE) | fp32 [B,T,H] (SCALAR)      */
                           /*            | dtype [B,T,H,d_k] (CHANNEL); values <= 0 */
-  const void *beta;       /* gain: fp32 [B,T,H]; FG2_GDN: dtype [B,T,H,d_k] in [0,1]; */
-                          /*       GDN2: must be NULL                              */
+  const void *beta;       /* gain: fp32 [B,T,H]; FG2_GDN / FG2_GDN_PLUS: dtype     */
+                          /*   [B,T,H,d_k] in [0,1] (the key-side gain); GDN2: NULL */
   const void *erase;      /* GDN2 only: dtype [B,T,H,d_k] erase gate, else NULL   */
-  const void *write;      /* GDN2 only: dtype [B,T,H,d_v] write gate, else NULL   */
+  const void *write;      /* dtype [B,T,H,d_v]: GDN2's write gate, FG2_GDN_PLUS's */
+                          /*   value-side gain in [0,1]; NULL for the others      */
   const float *S0;        /* initial state [B,H,d_v,d_k]; NULL = zeros            */
   float *ST;              /* final state [B,H,d_v,d_k]; NULL = not returned       */
-  const float *A0;        /* preconditioner accumulator [B,H,d_k] (PDN/PGDN/PKDA  */
-  float *AT;              /* only, else both NULL); NULL A0 = zeros               */
+  const float *A0;        /* preconditioner accumulator [B,H,d_k] (PDN/PGDN/PKDA/ */
+  float *AT;              /* PLA only, else both NULL); NULL A0 = zeros           */
   void *o;                /* output [B,T,H,d_v], dtype                            */
 } pdn_tensors_t;
 

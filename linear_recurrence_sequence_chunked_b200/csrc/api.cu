@@ -53,7 +53,7 @@ pdn_status_t check_problem(const pdn_problem_t *p) {
   if (!head_dim_ok(p->d_k) || !head_dim_ok(p->d_v)) return PDN_ERR_INVALID_ARG;
   const int chunk = p->chunk == 0 ? 64 : p->chunk;
   if (chunk != 16 && chunk != 32 && chunk != 64) return PDN_ERR_INVALID_ARG;
-  if ((int)p->variant < PDN_VAR_DN || (int)p->variant > PDN_VAR_GDN2) return PDN_ERR_INVALID_ARG;
+  if ((int)p->variant < PDN_VAR_DN || (int)p->variant > PDN_VAR_FG2_GDN_PLUS) return PDN_ERR_INVALID_ARG;
   if ((int)p->decay < PDN_DECAY_NONE || (int)p->decay > PDN_DECAY_CHANNEL) return PDN_ERR_INVALID_ARG;
   if (p->dtype != PDN_F32 && p->dtype != PDN_BF16) return PDN_ERR_INVALID_ARG;
   if ((int)p->impl < PDN_IMPL_AUTO || (int)p->impl > PDN_IMPL_TC) return PDN_ERR_INVALID_ARG;
@@ -78,7 +78,7 @@ pdn_status_t check_tensors(const pdn_problem_t *p, const pdn_tensors_t *t) {
   // vectors; the fp32 per-(token, head) gates (scalar log decay, scalar beta)
   // are read one element at a time and need only 4
   const bool scalar_la = p->decay == PDN_DECAY_SCALAR;
-  const bool scalar_beta = p->variant != PDN_VAR_FG2_GDN && p->variant != PDN_VAR_GDN2;
+  const bool scalar_beta = has_scalar_beta(p->variant);
   const void *v16[] = {t->q, t->k, t->v, t->o, t->erase, t->write, t->S0, t->ST, t->A0, t->AT,
                        scalar_la ? nullptr : t->log_alpha, scalar_beta ? nullptr : t->beta};
   for (const void *ptr : v16)
@@ -94,6 +94,8 @@ pdn_status_t check_tensors(const pdn_problem_t *p, const pdn_tensors_t *t) {
     if ((p->decay == PDN_DECAY_NONE) != (t->log_alpha == nullptr)) return PDN_ERR_INVALID_ARG;
     if (p->variant == PDN_VAR_GDN2) {
       if (t->beta || !t->erase || !t->write) return PDN_ERR_INVALID_ARG;
+    } else if (p->variant == PDN_VAR_FG2_GDN_PLUS) {
+      if (!t->beta || t->erase || !t->write) return PDN_ERR_INVALID_ARG;
     } else {
       if (!t->beta || t->erase || t->write) return PDN_ERR_INVALID_ARG;
     }

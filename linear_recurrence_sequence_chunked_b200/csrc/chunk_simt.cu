@@ -99,8 +99,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_simt_kernel(const KParams P
     for (int t = tid; t < C; t += kThreads) {
       const bool ok = t < Cn;
       const size_t e = tok_index(P, b, c0 + t, h);
-      sm.beta[t] = (ok && P.variant != PDN_VAR_FG2_GDN && P.variant != PDN_VAR_GDN2)
-                       ? ldf<float>(P.beta, e) : 0.f;
+      sm.beta[t] = (ok && has_scalar_beta(P.variant)) ? ldf<float>(P.beta, e) : 0.f;
       sm.la[t] = (ok && P.decay == PDN_DECAY_SCALAR) ? ldf<float>(P.log_alpha, e) : 0.f;
     }
     __syncthreads();
@@ -142,12 +141,17 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_simt_kernel(const KParams P
       const int t = idx / dk, i = idx % dk;
       const bool ok = t < Cn;
       const float kv = sm.R[t][i];
-      float r = kv, w;
+      float r = kv, w, qf = P.q_scale * sm.Q[t][i];
       switch (P.variant) {
         case PDN_VAR_PDN: case PDN_VAR_PGDN: case PDN_VAR_PKDA:
           w = sm.beta[t] * precond_coef(sm.W[t][i], sm.mu[t], P.lnx) * kv;
           break;
-        case PDN_VAR_FG2_GDN: {
+        case PDN_VAR_PLA:  // no erase; the preconditioner acts on the query
+          r = 0.f;
+          w = sm.beta[t] * kv;
+          qf *= precond_coef(sm.W[t][i], sm.mu[t], P.lnx);
+          break;
+        case PDN_VAR_FG2_GDN: case PDN_VAR_FG2_GDN_PLUS: {
           const float sb = ok ? sqrtf(ldf<Tin>(P.beta, tok_index(P, b, c0 + t, h) * dk + i)) : 0.f;
           r = sb * kv;
           w = r;
@@ -162,15 +166,17 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_simt_kernel(const KParams P
       }
       sm.R[t][i] = r;
       sm.W[t][i] = w;
-      sm.Q[t][i] = P.q_scale * sm.Q[t][i];
+      sm.Q[t][i] = qf;
     }
-    if (P.variant == PDN_VAR_FG2_GDN || P.variant == PDN_VAR_GDN2) {
+    if (P.variant == PDN_VAR_FG2_GDN || P.variant == PDN_VAR_GDN2 ||
+        P.variant == PDN_VAR_FG2_GDN_PLUS) {
       for (int idx = tid; idx < C * kDVB; idx += kThreads) {
         const int t = idx / kDVB, jj = idx % kDVB;
         if (t < Cn && jj < nj) {
           const size_t e = tok_index(P, b, c0 + t, h) * dv + j0 + jj;
           const float f = P.variant == PDN_VAR_FG2_GDN ? sqrtf(ldf<Tin>(P.beta, e))
-                                                       : ldf<Tin>(P.write, e);
+                          : P.variant == PDN_VAR_GDN2 ? ldf<Tin>(P.write, e)
+                                                      : sqrtf(ldf<Tin>(P.write, e));
           sm.U[t][jj] *= f;
         }
       }

@@ -179,8 +179,8 @@ __host__ __device__ constexpr int grp_off(int a) { return 8 * a * (a + 1); }
 
 template <int kVariant, int kDecay>
 struct K1Layout {
-  static constexpr bool kPre =
-      kVariant == PDN_VAR_PDN || kVariant == PDN_VAR_PGDN || kVariant == PDN_VAR_PKDA;
+  static constexpr bool kPre = kVariant == PDN_VAR_PDN || kVariant == PDN_VAR_PGDN ||
+                               kVariant == PDN_VAR_PKDA || kVariant == PDN_VAR_PLA;
   static constexpr bool kCh = kDecay == PDN_DECAY_CHANNEL;
   static constexpr int kN1 = kCh ? 160 : 64;                // columns of MMA1
   static constexpr uint32_t kRQ = 0;                        // TL 128 x 128: R rows 0-63, Q rows 64-127
@@ -194,9 +194,11 @@ struct K1Layout {
   static constexpr uint32_t kBC = kQS + 64 * KS_LD;
   static constexpr uint32_t kGBUF = kBC + 64 * KS_LD;
   static constexpr uint32_t kLasStage = kGBUF + 64 * LB_LD * 4;
-  // channel decay: FG2's gain vector, or GDN-2's erase and write gates,
-  // staged by cp.async with q (read in P3)
-  static constexpr int kGates = !kCh ? 0 : kVariant == PDN_VAR_FG2_GDN ? 1 : kVariant == PDN_VAR_GDN2 ? 2 : 0;
+  // channel decay: FG2's gain vector, GDN-2's erase and write gates, or
+  // FG2+'s key-side and value-side gains, staged by cp.async with q (read in P3)
+  static constexpr int kGates = !kCh ? 0
+                                : kVariant == PDN_VAR_FG2_GDN ? 1
+                                : (kVariant == PDN_VAR_GDN2 || kVariant == PDN_VAR_FG2_GDN_PLUS) ? 2 : 0;
   static constexpr uint32_t kGateStage = kLasStage + 64 * 256;
   static constexpr uint32_t kPrepEnd = kCh ? kGateStage + kGates * 16384 : kGBUF;
   // region A from the epilogue of MMA1 on: MMA2's T tile and the fp32 solve
@@ -227,6 +229,7 @@ struct K1Layout {
   static constexpr uint32_t kTmY = kN1;  // TMEM column of Y^T (after MMA1's columns)
 };
 static_assert(K1Layout<PDN_VAR_GDN2, PDN_DECAY_CHANNEL>::kBytes <= 232448 &&
+                  K1Layout<PDN_VAR_FG2_GDN_PLUS, PDN_DECAY_CHANNEL>::kBytes <= 232448 &&
                   K1Layout<PDN_VAR_PKDA, PDN_DECAY_CHANNEL>::kBytes <= 232448 &&
                   K1Layout<PDN_VAR_FG2_GDN, PDN_DECAY_CHANNEL>::kBytes <= 232448,
               "intra-chunk kernel shared memory budget");
@@ -281,7 +284,8 @@ __global__ void __launch_bounds__(kK1Threads, kDecay == PDN_DECAY_CHANNEL ? 1 : 
   constexpr bool kPre = L::kPre;
   constexpr bool kCh = L::kCh;
   constexpr bool kSc = kDecay == PDN_DECAY_SCALAR;
-  constexpr bool kScalarBeta = kVariant != PDN_VAR_FG2_GDN && kVariant != PDN_VAR_GDN2;
+  constexpr bool kScalarBeta = has_scalar_beta(kVariant);
+  constexpr bool kFG2 = kVariant == PDN_VAR_FG2_GDN || kVariant == PDN_VAR_FG2_GDN_PLUS;
   extern __shared__ __align__(1024) uint8_t smem[];
   const uint32_t sb = smem_u32(smem);
   float *Acar = reinterpret_cast<float *>(smem + L::kAcar);
@@ -431,7 +435,7 @@ __global__ void __launch_bounds__(kK1Threads, kDecay == PDN_DECAY_CHANNEL ? 1 : 
       const uint32_t gs = sb + L::kGateStage + t * 256 + ((c8 ^ (t & 7)) << 4);
       if (L::kGates >= 1)
         cp_async16(gs, reinterpret_cast<const __nv_bfloat16 *>(
-                           kVariant == PDN_VAR_FG2_GDN ? P.beta : P.erase) + e, ok);
+                           kFG2 ? P.beta : P.erase) + e, ok);
       if (L::kGates == 2)
         cp_async16(gs + 16384, reinterpret_cast<const __nv_bfloat16 *>(P.write) + e, ok);
     }
@@ -626,27 +630,43 @@ __global__ void __launch_bounds__(kK1Threads, kDecay == PDN_DECAY_CHANNEL ? 1 : 
       if (kPre) {
         float Bv[8];
         unpack8(*reinterpret_cast<const uint4 *>(smem + L::kBC + t * KS_LD + c8 * 16), Bv);
+        if (kVariant == PDN_VAR_PLA) {
+          // linear attention: no erase; the preconditioner acts on the query
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          r[e] = kf[e];
-          w[e] = be * Bv[e] * kf[e];
+          for (int e = 0; e < 8; ++e) {
+            r[e] = 0.f;
+            w[e] = be * kf[e];
+            qf[e] *= Bv[e];
+          }
+        } else {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            r[e] = kf[e];
+            w[e] = be * Bv[e] * kf[e];
+          }
         }
-      } else if (kVariant == PDN_VAR_FG2_GDN) {
-        float gb[8];
+      } else if (kFG2) {
+        // key-side gain gb (and, for FG2+, a value-side gain gv of its own)
+        float gb[8], gv[8];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) gb[e] = 0.f;
-        if (L::kGates)
-          unpack8(*reinterpret_cast<const uint4 *>(smem + L::kGateStage + t * 256 + ((c8 ^ (t & 7)) << 4)),
-                  gb);
-        else if (ok)
+        for (int e = 0; e < 8; ++e) { gb[e] = 0.f; gv[e] = 0.f; }
+        if (L::kGates) {
+          const uint8_t *gsrc = smem + L::kGateStage + t * 256 + ((c8 ^ (t & 7)) << 4);
+          unpack8(*reinterpret_cast<const uint4 *>(gsrc), gb);
+          if (kVariant == PDN_VAR_FG2_GDN_PLUS) unpack8(*reinterpret_cast<const uint4 *>(gsrc + 16384), gv);
+        } else if (ok) {
           unpack8(__ldg(reinterpret_cast<const uint4 *>(
                       reinterpret_cast<const __nv_bfloat16 *>(P.beta) + etok + i0)), gb);
+          if (kVariant == PDN_VAR_FG2_GDN_PLUS)
+            unpack8(__ldg(reinterpret_cast<const uint4 *>(
+                        reinterpret_cast<const __nv_bfloat16 *>(P.write) + etok + i0)), gv);
+        }
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
           const float sq = sqrtf(gb[e]);
           r[e] = sq * kf[e];
           w[e] = r[e];
-          vf[e] *= sq;
+          vf[e] *= kVariant == PDN_VAR_FG2_GDN_PLUS ? sqrtf(gv[e]) : sq;
         }
       } else if (kVariant == PDN_VAR_GDN2) {
         float ge[8], gw[8];
@@ -1526,7 +1546,9 @@ cudaError_t launch_chunk_split(const KParams &P, void *ws, cudaStream_t stream,
     case PDN_VAR_PGDN: e = launch_k1_decay<PDN_VAR_PGDN>(P, ws, N, stream); break;
     case PDN_VAR_PKDA: e = launch_k1_decay<PDN_VAR_PKDA>(P, ws, N, stream); break;
     case PDN_VAR_FG2_GDN: e = launch_k1_decay<PDN_VAR_FG2_GDN>(P, ws, N, stream); break;
-    default: e = launch_k1_decay<PDN_VAR_GDN2>(P, ws, N, stream); break;
+    case PDN_VAR_GDN2: e = launch_k1_decay<PDN_VAR_GDN2>(P, ws, N, stream); break;
+    case PDN_VAR_PLA: e = launch_k1_decay<PDN_VAR_PLA>(P, ws, N, stream); break;
+    default: e = launch_k1_decay<PDN_VAR_FG2_GDN_PLUS>(P, ws, N, stream); break;
   }
   if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(k2_state, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)K2_BYTES);

@@ -24,8 +24,14 @@ struct KParams {
   int *err;  // per-device error word (first error wins)
 };
 
-__host__ __device__ inline bool is_precond(int variant) {
-  return variant == PDN_VAR_PDN || variant == PDN_VAR_PGDN || variant == PDN_VAR_PKDA;
+// Variants with the diagonal preconditioner (accumulator A, coefficients B).
+__host__ __device__ constexpr bool is_precond(int variant) {
+  return variant == PDN_VAR_PDN || variant == PDN_VAR_PGDN || variant == PDN_VAR_PKDA ||
+         variant == PDN_VAR_PLA;
+}
+// Variants whose gain beta is one fp32 scalar per (token, head).
+__host__ __device__ constexpr bool has_scalar_beta(int variant) {
+  return variant != PDN_VAR_FG2_GDN && variant != PDN_VAR_GDN2 && variant != PDN_VAR_FG2_GDN_PLUS;
 }
 
 // Element load as fp32 from a tensor of the problem dtype.

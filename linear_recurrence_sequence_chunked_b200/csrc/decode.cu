@@ -91,7 +91,12 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const KParams P) {
         r = kv;
         w = ldf<float>(P.beta, tokh) * precond_coef(logA, mu, P.lnx) * kv;
         break;
-      case PDN_VAR_FG2_GDN:
+      case PDN_VAR_PLA:  // no erase; the preconditioner acts on the query
+        r = 0.f;
+        w = ldf<float>(P.beta, tokh) * kv;
+        qv *= precond_coef(logA, mu, P.lnx);
+        break;
+      case PDN_VAR_FG2_GDN: case PDN_VAR_FG2_GDN_PLUS:
         r = sqrtf(ldf<Tin>(P.beta, tokh * dk + tid)) * kv;
         w = r;
         break;
@@ -115,6 +120,7 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const KParams P) {
     float u = ldf<Tin>(P.v, tokh * dv + j);
     if (P.variant == PDN_VAR_FG2_GDN) u *= sqrtf(ldf<Tin>(P.beta, tokh * dv + j));
     else if (P.variant == PDN_VAR_GDN2) u *= ldf<Tin>(P.write, tokh * dv + j);
+    else if (P.variant == PDN_VAR_FG2_GDN_PLUS) u *= sqrtf(ldf<Tin>(P.write, tokh * dv + j));
     s_u[j] = u;
   }
   const float wq = block_sum(chan ? w * qv : 0.f, s_red);  // ends with __syncthreads
@@ -275,12 +281,14 @@ __global__ void __launch_bounds__(kTmaThreads, 1) decode_tma_kernel(const KParam
       t.q = ldf<Tin>(P.q, e);
       t.v = ldf<Tin>(P.v, e);
       if (precond) t.a = P.AT[(size_t)item * kD128 + tid];
-      if (P.variant == PDN_VAR_FG2_GDN) t.beta = ldf<Tin>(P.beta, e);
+      if (P.variant == PDN_VAR_FG2_GDN || P.variant == PDN_VAR_FG2_GDN_PLUS) t.beta = ldf<Tin>(P.beta, e);
       else if (P.variant != PDN_VAR_GDN2) t.beta = ldf<float>(P.beta, tokh);
       if (P.decay == PDN_DECAY_SCALAR) t.la = ldf<float>(P.log_alpha, tokh);
       else if (P.decay == PDN_DECAY_CHANNEL) t.la = ldf<Tin>(P.log_alpha, e);
       if (P.variant == PDN_VAR_GDN2) {
         t.ge = ldf<Tin>(P.erase, e);
+        t.gw = ldf<Tin>(P.write, e);
+      } else if (P.variant == PDN_VAR_FG2_GDN_PLUS) {
         t.gw = ldf<Tin>(P.write, e);
       }
     }
@@ -295,7 +303,8 @@ __global__ void __launch_bounds__(kTmaThreads, 1) decode_tma_kernel(const KParam
     const Tok nxt = (k + 1 < nloc) ? load_tok(k + 1) : cur;
 
     // per-token vectors (overlap the bulk loads in flight)
-    const float kv = cur.k, qv = cur.q;
+    const float kv = cur.k;
+    float qv = cur.q;
     float logA = 0.f;
     if (chan && precond) {
       const float a = cur.a + kv * kv;
@@ -312,11 +321,16 @@ __global__ void __launch_bounds__(kTmaThreads, 1) decode_tma_kernel(const KParam
           r = kv;
           w = cur.beta * precond_coef(logA, mu, P.lnx) * kv;
           break;
-        case PDN_VAR_FG2_GDN: {
+        case PDN_VAR_PLA:  // no erase; the preconditioner acts on the query
+          r = 0.f;
+          w = cur.beta * kv;
+          qv *= precond_coef(logA, mu, P.lnx);
+          break;
+        case PDN_VAR_FG2_GDN: case PDN_VAR_FG2_GDN_PLUS: {
           const float sb = sqrtf(cur.beta);
           r = sb * kv;
           w = r;
-          u *= sb;
+          u *= P.variant == PDN_VAR_FG2_GDN_PLUS ? sqrtf(cur.gw) : sb;
         } break;
         case PDN_VAR_GDN2:
           r = cur.ge * kv;

@@ -59,9 +59,9 @@ Sizes sizes_of(const pdn_problem_t *p) {
   z.q = z.k = th * p->d_k * es;
   z.v = z.o = th * p->d_v * es;
   z.la = p->decay == PDN_DECAY_SCALAR ? th * 4 : p->decay == PDN_DECAY_CHANNEL ? th * p->d_k * es : 0;
-  z.beta = p->variant == PDN_VAR_GDN2 ? 0 : p->variant == PDN_VAR_FG2_GDN ? th * p->d_k * es : th * 4;
+  z.beta = p->variant == PDN_VAR_GDN2 ? 0 : has_scalar_beta(p->variant) ? th * 4 : th * p->d_k * es;
   z.erase = p->variant == PDN_VAR_GDN2 ? th * p->d_k * es : 0;
-  z.write = p->variant == PDN_VAR_GDN2 ? th * p->d_v * es : 0;
+  z.write = (p->variant == PDN_VAR_GDN2 || p->variant == PDN_VAR_FG2_GDN_PLUS) ? th * p->d_v * es : 0;
   z.S = (size_t)p->H * p->d_v * p->d_k * 4;
   z.A = (size_t)p->H * p->d_k * 4;
   return z;

@@ -21,11 +21,12 @@ _LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libpdn.so"
 
 PDN_OK, PDN_ERR_INVALID_ARG, PDN_ERR_UNSUPPORTED, PDN_ERR_CUDA, PDN_ERR_TIMEOUT, \
     PDN_ERR_WORKSPACE = range(6)
-VARIANTS = {"DN": 0, "GDN": 1, "KDA": 2, "PDN": 3, "PGDN": 4, "PKDA": 5, "FG2_GDN": 6, "GDN2": 7}
+VARIANTS = {"DN": 0, "GDN": 1, "KDA": 2, "PDN": 3, "PGDN": 4, "PKDA": 5, "FG2_GDN": 6, "GDN2": 7,
+            "PLA": 8, "FG2_GDN_PLUS": 9}
 DECAYS = {"none": 0, "scalar": 1, "channel": 2}
 DTYPES = {torch.float32: 0, torch.bfloat16: 1}
 IMPLS = {"auto": 0, "simt": 1, "tc": 2}
-PRECOND_VARIANTS = ("PDN", "PGDN", "PKDA")
+PRECOND_VARIANTS = ("PDN", "PGDN", "PKDA", "PLA")
 
 
 class PdnProblem(ctypes.Structure):

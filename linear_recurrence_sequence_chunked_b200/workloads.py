@@ -19,13 +19,13 @@ import torch
 
 DECAY_OF_VARIANT = {"DN": "none", "PDN": "none", "GDN": "scalar", "PGDN": "scalar",
                     "KDA": "channel", "PKDA": "channel"}
-PRECOND_VARIANTS = ("PDN", "PGDN", "PKDA")
+PRECOND_VARIANTS = ("PDN", "PGDN", "PKDA", "PLA")
 
 
 @dataclasses.dataclass(frozen=True)
 class Workload:
     name: str
-    variant: str            # DN GDN KDA PDN PGDN PKDA FG2_GDN GDN2
+    variant: str            # DN GDN KDA PDN PGDN PKDA FG2_GDN GDN2 PLA FG2_GDN_PLUS
     B: int
     T: int
     H: int
@@ -52,7 +52,7 @@ class Workload:
         return torch.float32 if self.dtype == "f32" else torch.bfloat16
 
 
-# The five workloads the build is measured and checked on.
+# The workloads the build is measured and checked on.
 WORKLOADS = {
     # Preconditioned DeltaNet, fp32, tiny: parity at 1e-4.
     "pdn_f32_small": Workload("pdn_f32_small", "PDN", 1, 512, 2, 64, 64, "f32", "none"),
@@ -64,6 +64,11 @@ WORKLOADS = {
     # FG2-GDN and Gated DeltaNet-2 at 32k tokens, channel decay.
     "fg2_bf16_32k": Workload("fg2_bf16_32k", "FG2_GDN", 2, 32768, 16, 128, 128, "bf16", "channel"),
     "gdn2_bf16_32k": Workload("gdn2_bf16_32k", "GDN2", 2, 32768, 16, 128, 128, "bf16", "channel"),
+    # Preconditioned linear attention (scalar decay) and FG2-GDN+ (channel
+    # decay) at the headline layer shape.
+    "pla_bf16_4k": Workload("pla_bf16_4k", "PLA", 4, 4096, 16, 128, 128, "bf16", "scalar"),
+    "fg2p_bf16_4k": Workload("fg2p_bf16_4k", "FG2_GDN_PLUS", 4, 4096, 16, 128, 128, "bf16",
+                             "channel"),
     # Recurrent decode of Preconditioned GDN: 256 sequences x 16 heads, 1024 steps.
     "pgdn_decode_256": Workload("pgdn_decode_256", "PGDN", 256, 1024, 16, 128, 128, "bf16",
                                 "scalar", decode_steps=1024),
@@ -98,7 +103,7 @@ def make_inputs(w: Workload, device="cpu", B: Optional[int] = None, T: Optional[
     k = _l2n(randn(B, T, H, dk)).to(dt)
     v = randn(B, T, H, dv).to(dt)
     beta = None
-    if w.variant == "FG2_GDN":
+    if w.variant in ("FG2_GDN", "FG2_GDN_PLUS"):
         beta = torch.sigmoid(randn(B, T, H, dk)).to(dt)
     elif w.variant != "GDN2":
         beta = torch.sigmoid(randn(B, T, H))
@@ -121,6 +126,8 @@ def make_inputs(w: Workload, device="cpu", B: Optional[int] = None, T: Optional[
     erase = write = None
     if w.variant == "GDN2":
         erase = torch.sigmoid(randn(B, T, H, dk)).to(dt)
+        write = torch.sigmoid(randn(B, T, H, dv)).to(dt)
+    elif w.variant == "FG2_GDN_PLUS":  # the value-side gain vector
         write = torch.sigmoid(randn(B, T, H, dv)).to(dt)
     out = dict(q=q, k=k, v=v, log_alpha=log_alpha, beta=beta, erase=erase, write=write)
     return {n: (t.to(device) if t is not None else None) for n, t in out.items()}

@@ -104,7 +104,7 @@ def _problem(**over):
 
 INVALID_PROBLEMS = [
     dict(B=0), dict(H=0), dict(T=-1), dict(d_k=0), dict(d_k=24), dict(d_v=256), dict(chunk=48),
-    dict(variant=9), dict(decay=3), dict(dtype=5), dict(impl=7),
+    dict(variant=10), dict(variant=-1), dict(decay=3), dict(dtype=5), dict(impl=7),
     dict(decay=pdn.DECAYS["channel"]),              # PGDN needs scalar decay
     dict(precond_x=2.5), dict(precond_x=0.5), dict(precond_eps=0.0),
     dict(q_scale=float("nan")),
@@ -142,6 +142,15 @@ def test_variant_specific_rules(lib):
     # a non-preconditioned variant must not get an accumulator
     p = _problem(variant=pdn.VARIANTS["GDN"])
     assert pdn.pdn_chunk_fwd(p, _tensors(A0=FAKE + 0x8000), None, 0, None) == pdn.PDN_ERR_INVALID_ARG
+    # FG2-GDN+ takes the key-side gain (beta) and the value-side gain (write), no erase gate
+    p = _problem(variant=pdn.VARIANTS["FG2_GDN_PLUS"], decay=pdn.DECAYS["channel"])
+    assert pdn.pdn_chunk_fwd(p, _tensors(), None, 0, None) == pdn.PDN_ERR_INVALID_ARG
+    assert pdn.pdn_chunk_fwd(p, _tensors(write=FAKE + 0x6000, erase=FAKE + 0x7000), None, 0,
+                             None) == pdn.PDN_ERR_INVALID_ARG
+    # PLA takes the scalar gain and no gates; it is preconditioned (accumulator allowed)
+    p = _problem(variant=pdn.VARIANTS["PLA"], decay=pdn.DECAYS["channel"])
+    assert pdn.pdn_chunk_fwd(p, _tensors(write=FAKE + 0x6000), None, 0, None) == pdn.PDN_ERR_INVALID_ARG
+    assert pdn.pdn_chunk_fwd(p, _tensors(beta=None), None, 0, None) == pdn.PDN_ERR_INVALID_ARG
 
 
 def test_decode_rules(lib):

@@ -12,9 +12,10 @@ from parity_util import TOL, nmax_err, run_gpu, run_oracle
 
 pytestmark = pytest.mark.gpu
 
-VARIANTS = ["DN", "GDN", "KDA", "PDN", "PGDN", "PKDA", "FG2_GDN", "GDN2"]
+VARIANTS = ["DN", "GDN", "KDA", "PDN", "PGDN", "PKDA", "FG2_GDN", "GDN2", "PLA", "FG2_GDN_PLUS"]
 DECAY = {"DN": "none", "PDN": "none", "GDN": "scalar", "PGDN": "scalar",
-         "KDA": "channel", "PKDA": "channel", "FG2_GDN": "channel", "GDN2": "channel"}
+         "KDA": "channel", "PKDA": "channel", "FG2_GDN": "channel", "GDN2": "channel",
+         "PLA": "scalar", "FG2_GDN_PLUS": "channel"}
 
 
 def decode_all(w, x, S, A, steps):
@@ -40,7 +41,7 @@ def test_decode_matches_oracle(variant, dtype):
     x = make_inputs(w)
     g = torch.Generator().manual_seed(3)
     S0 = 0.3 * torch.randn(w.B, w.H, w.dv, w.dk, generator=g)
-    A0 = torch.rand(w.B, w.H, w.dk, generator=g) if variant in ("PDN", "PGDN", "PKDA") else None
+    A0 = torch.rand(w.B, w.H, w.dk, generator=g) if variant in ("PDN", "PGDN", "PKDA", "PLA") else None
     S = S0.cuda()
     A = A0.cuda() if A0 is not None else None
     o = decode_all(w, x, S, A, w.T)
@@ -102,7 +103,7 @@ def test_decode_d128_many_heads(variant, dtype):
     x = make_inputs(w)
     g = torch.Generator().manual_seed(4)
     S0 = 0.2 * torch.randn(w.B, w.H, 128, 128, generator=g)
-    A0 = torch.rand(w.B, w.H, 128, generator=g) if variant in ("PDN", "PGDN", "PKDA") else None
+    A0 = torch.rand(w.B, w.H, 128, generator=g) if variant in ("PDN", "PGDN", "PKDA", "PLA") else None
     S = S0.cuda()
     A = A0.cuda() if A0 is not None else None
     o = decode_all(w, x, S, A, w.T)

@@ -14,7 +14,7 @@ from parity_util import assert_parity, run_gpu, run_oracle
 pytestmark = pytest.mark.gpu
 
 DECAY = {"PGDN": "scalar", "PKDA": "channel", "FG2_GDN": "channel", "GDN2": "channel",
-         "DN": "none"}
+         "DN": "none", "PLA": "scalar", "FG2_GDN_PLUS": "channel"}
 GATES = ("log_alpha", "beta", "erase", "write")
 
 
@@ -48,7 +48,7 @@ def host_run(w, x, S0, A0, slices):
     return ho, hST, hAT
 
 
-@pytest.mark.parametrize("variant", ["PGDN", "PKDA", "FG2_GDN", "GDN2", "DN"])
+@pytest.mark.parametrize("variant", ["PGDN", "PKDA", "FG2_GDN", "GDN2", "DN", "PLA", "FG2_GDN_PLUS"])
 def test_host_path_matches_device_path(variant):
     w = Workload("host-" + variant, variant, 3, 130, 2, 128, 128, "bf16", DECAY[variant])
     x = make_inputs(w)

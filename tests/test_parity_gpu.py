@@ -11,9 +11,10 @@ from parity_util import TOL, assert_parity, run_gpu, run_oracle, nmax_err
 
 pytestmark = pytest.mark.gpu
 
-VARIANTS = ["DN", "GDN", "KDA", "PDN", "PGDN", "PKDA", "FG2_GDN", "GDN2"]
+VARIANTS = ["DN", "GDN", "KDA", "PDN", "PGDN", "PKDA", "FG2_GDN", "GDN2", "PLA", "FG2_GDN_PLUS"]
 DECAY = {"DN": "none", "PDN": "none", "GDN": "scalar", "PGDN": "scalar",
-         "KDA": "channel", "PKDA": "channel", "FG2_GDN": "channel", "GDN2": "channel"}
+         "KDA": "channel", "PKDA": "channel", "FG2_GDN": "channel", "GDN2": "channel",
+         "PLA": "scalar", "FG2_GDN_PLUS": "channel"}
 IMPLS = ["simt", "auto"]
 
 
@@ -25,7 +26,7 @@ def small(variant, dtype, B=2, T=150, H=3, d=64, dv=None, decay=None, seed=0, **
 def rand_state(w, seed=1, scale=0.3):
     g = torch.Generator().manual_seed(seed)
     S0 = scale * torch.randn(w.B, w.H, w.dv, w.dk, generator=g)
-    A0 = torch.rand(w.B, w.H, w.dk, generator=g) * 2.0 if w.variant in ("PDN", "PGDN", "PKDA") else None
+    A0 = torch.rand(w.B, w.H, w.dk, generator=g) * 2.0 if w.variant in ("PDN", "PGDN", "PKDA", "PLA") else None
     return S0, A0
 
 
@@ -43,7 +44,7 @@ def test_variants_small(variant, dtype, impl):
 
 
 @pytest.mark.parametrize("decay", ["none", "scalar", "channel"])
-@pytest.mark.parametrize("variant", ["FG2_GDN", "GDN2"])
+@pytest.mark.parametrize("variant", ["FG2_GDN", "GDN2", "PLA", "FG2_GDN_PLUS"])
 def test_free_decay_variants(variant, decay):
     w = small(variant, "bf16", decay=decay, T=97)
     x = make_inputs(w)

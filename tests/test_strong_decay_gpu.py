@@ -16,7 +16,7 @@ from parity_util import TOL, assert_parity, nmax_err, run_gpu, run_oracle
 pytestmark = pytest.mark.gpu
 
 DECAY = {"GDN": "scalar", "PGDN": "scalar", "KDA": "channel", "PKDA": "channel",
-         "FG2_GDN": "channel", "GDN2": "channel"}
+         "FG2_GDN": "channel", "GDN2": "channel", "PLA": "channel", "FG2_GDN_PLUS": "channel"}
 STRENGTHS = [-1.5, -3.0, -10.0, "hard"]
 
 
@@ -32,7 +32,7 @@ def strong(variant, mean, dtype="bf16", B=2, T=150, H=2, d=128, decay=None):
 def rand_state(w, seed=5):
     g = torch.Generator().manual_seed(seed)
     S0 = 0.3 * torch.randn(w.B, w.H, w.dv, w.dk, generator=g)
-    A0 = torch.rand(w.B, w.H, w.dk, generator=g) if w.variant in ("PDN", "PGDN", "PKDA") else None
+    A0 = torch.rand(w.B, w.H, w.dk, generator=g) if w.variant in ("PDN", "PGDN", "PKDA", "PLA") else None
     return S0, A0
 
 
@@ -62,7 +62,7 @@ def test_strong_decay_cuda_core_path(variant, mean, dtype):
 
 
 @pytest.mark.parametrize("decay", ["scalar", "channel"])
-@pytest.mark.parametrize("variant", ["FG2_GDN", "GDN2"])
+@pytest.mark.parametrize("variant", ["FG2_GDN", "GDN2", "PLA", "FG2_GDN_PLUS"])
 def test_strong_decay_free_decay_variants(variant, decay):
     w = strong(variant, -3.0, decay=decay, T=200)
     x = make_inputs(w)

@@ -12,9 +12,10 @@ from parity_util import assert_parity, nmax_err, run_gpu, run_oracle
 
 pytestmark = pytest.mark.gpu
 
-VARIANTS = ["DN", "GDN", "KDA", "PDN", "PGDN", "PKDA", "FG2_GDN", "GDN2"]
+VARIANTS = ["DN", "GDN", "KDA", "PDN", "PGDN", "PKDA", "FG2_GDN", "GDN2", "PLA", "FG2_GDN_PLUS"]
 DECAY = {"DN": "none", "PDN": "none", "GDN": "scalar", "PGDN": "scalar",
-         "KDA": "channel", "PKDA": "channel", "FG2_GDN": "channel", "GDN2": "channel"}
+         "KDA": "channel", "PKDA": "channel", "FG2_GDN": "channel", "GDN2": "channel",
+         "PLA": "scalar", "FG2_GDN_PLUS": "channel"}
 
 
 def tc_work(variant, decay=None, B=2, T=200, H=2, seed=0, **kw):
@@ -40,14 +41,14 @@ def test_tc_variants(variant, impl):
     x = make_inputs(w)
     g = torch.Generator().manual_seed(2)
     S0 = 0.3 * torch.randn(w.B, w.H, 128, 128, generator=g)
-    A0 = torch.rand(w.B, w.H, 128, generator=g) * 3 if variant in ("PDN", "PGDN", "PKDA") else None
+    A0 = torch.rand(w.B, w.H, 128, generator=g) * 3 if variant in ("PDN", "PGDN", "PKDA", "PLA") else None
     o, ST, AT = run_gpu(w, x, S0, A0, impl=impl)
     assert_parity(w, o, ST, AT, *run_oracle(w, x, S0, A0))
 
 
 @pytest.mark.parametrize("impl", TC_IMPLS)
 @pytest.mark.parametrize("decay", ["none", "scalar", "channel"])
-@pytest.mark.parametrize("variant", ["FG2_GDN", "GDN2"])
+@pytest.mark.parametrize("variant", ["FG2_GDN", "GDN2", "PLA", "FG2_GDN_PLUS"])
 def test_tc_free_decay(variant, decay, impl):
     w = tc_work(variant, decay=decay, T=130)
     x = make_inputs(w)
