@@ -385,8 +385,9 @@ def run_ours(args):
         torch.cuda.empty_cache()
         result["workloads"] = {}
         for name in EXTRA_WORKLOADS:
-            r = bench_workload(args, WORKLOADS[name], dev, stream, peaks, peaks_kind, rank, mor,
-                               barrier)
+            fused = name.endswith("+prologue")
+            r = bench_workload(args, WORKLOADS[name.split("+")[0]], dev, stream, peaks, peaks_kind,
+                               rank, mor, barrier, fused_prologue=fused)
             result["workloads"][name] = r
             result["gpu_launches"] += r["gpu_launches"]
             torch.cuda.empty_cache()
@@ -409,7 +410,10 @@ def run_ours(args):
         print(json.dumps(result), flush=True)
 
 
-EXTRA_WORKLOADS = ("pkda_bf16_8k", "fg2_bf16_32k", "gdn2_bf16_32k", "pla_bf16_4k", "fg2p_bf16_4k")
+# "+prologue": the same layer from raw projections, with L2 normalisation,
+# sigmoid gains and the softplus decay fused into the kernels
+EXTRA_WORKLOADS = ("pkda_bf16_8k", "fg2_bf16_32k", "gdn2_bf16_32k", "pla_bf16_4k", "fg2p_bf16_4k",
+                   "pgdn_bf16_4k+prologue")
 
 
 def profiled_kernel_ms(pdn, prob, tens, ws, sptr, reps=3):
@@ -426,20 +430,23 @@ def profiled_kernel_ms(pdn, prob, tens, ws, sptr, reps=3):
     return {n: v / reps for n, v in zip(names, acc)}
 
 
-def bench_workload(args, w, dev, stream, peaks, peaks_kind, rank, mor, barrier):
+def bench_workload(args, w, dev, stream, peaks, peaks_kind, rank, mor, barrier,
+                   fused_prologue=False):
     """Times `args.steps` forward calls of workload w (inputs resident in HBM
     and larger than L2, so no flush), after warm-up."""
     import torch
 
     from linear_recurrence_sequence_chunked_b200 import pdn
-    from linear_recurrence_sequence_chunked_b200.workloads import make_inputs
+    from linear_recurrence_sequence_chunked_b200.workloads import (make_inputs, make_raw_inputs,
+                                                                   raw_prologue)
 
     wr = w.replace(seed=rank_seed(w.seed, rank))
-    x = make_inputs(wr, device=dev, generator_device=dev)
+    bits, dscale = raw_prologue(w) if fused_prologue else (0, 1.0)
+    x = (make_raw_inputs if fused_prologue else make_inputs)(wr, device=dev, generator_device=dev)
     g = {n: x[n] for n in ("log_alpha", "beta", "erase", "write")}
     o = torch.empty(w.B, w.T, w.H, w.dv, dtype=x["v"].dtype, device=dev)
     prob = pdn.make_problem(w.variant, w.B, w.T, w.H, w.dk, w.dv, x["k"].dtype, w.decay, w.chunk,
-                            "auto", w.q_scale, w.precond_x, w.precond_eps)
+                            "auto", w.q_scale, w.precond_x, w.precond_eps, bits, dscale)
     ws_bytes = pdn.pdn_chunk_fwd_workspace(prob)
     ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
     ST = torch.empty(w.B, w.H, w.dv, w.dk, dtype=torch.float32, device=dev)
@@ -471,6 +478,7 @@ def bench_workload(args, w, dev, stream, peaks, peaks_kind, rank, mor, barrier):
     nbytes = fwd_bytes_per_token_head(w) * w.B * w.T * w.H + 4 * w.B * w.H * w.dv * w.dk
     launches = 4 if w.variant in pdn.PRECOND_VARIANTS else 2
     res = {"variant": w.variant, "B": w.B, "T": w.T, "H": w.H, "d": w.dk, "inputs": w.dtype,
+           "prologue": "fused (raw projections)" if fused_prologue else "none",
            "value": w.B * w.T * args.steps / (ms / 1e3), "unit": "tokens/s",
            "ms_per_step": ms / args.steps,
            "tensor": {"achieved": flops / (per / 1e3) / 1e12, "peak": peaks["bf16_tflops"],

@@ -100,6 +100,28 @@ typedef enum { PDN_F32 = 0, PDN_BF16 = 1 } pdn_dtype_t;
  * arithmetic). AUTO picks TC where it applies, else SIMT. */
 typedef enum { PDN_IMPL_AUTO = 0, PDN_IMPL_SIMT = 1, PDN_IMPL_TC = 2 } pdn_impl_t;
 
+/* Fused prologue (pdn_problem_t.prologue, a bit mask): the kernels take raw
+ * projections and apply, per token and head, the activations that otherwise
+ * run as separate passes before the recurrence (the workloads the pages
+ * train use L2-normalised q and k, sigmoid gains and gates, and a softplus
+ * or log-sigmoid decay). 0 = inputs are used as given.
+ *   PDN_PRO_L2NORM_QK       q and k are divided by their L2 norm over the head
+ *                           dimension (norm floored at 1e-12); the
+ *                           preconditioner accumulates the normalised k
+ *   PDN_PRO_SIGMOID_GATES   beta (scalar or vector), GDN2's erase and write
+ *                           gates and FG2_GDN_PLUS's value gain arrive as
+ *                           logits x and are used as sigmoid(x)
+ *   PDN_PRO_DECAY_SOFTPLUS  log_alpha arrives as x; log alpha = -decay_scale *
+ *                           softplus(x) (decay_scale > 0)
+ *   PDN_PRO_DECAY_LOGSIGMOID log_alpha arrives as x; log alpha = log sigmoid(x)
+ * The two decay bits exclude each other and need a decay (decay != NONE). */
+enum {
+  PDN_PRO_L2NORM_QK = 1,
+  PDN_PRO_SIGMOID_GATES = 2,
+  PDN_PRO_DECAY_SOFTPLUS = 4,
+  PDN_PRO_DECAY_LOGSIGMOID = 8
+};
+
 typedef struct {
   int B, T, H;          /* batch, tokens per sequence, heads; B,H >= 1, T >= 0
                            (T == 0: per-token tensors may be NULL; ST = S0) */
@@ -112,6 +134,8 @@ typedef struct {
   float q_scale;        /* read-out scale (the pages use 1)                   */
   float precond_x;      /* preconditioner bound x, B_t in [1/x, x]; 1 <= x <= 2 */
   float precond_eps;    /* > 0, added inside the log                          */
+  int prologue;         /* PDN_PRO_* bits (0 = none)                          */
+  float decay_scale;    /* PDN_PRO_DECAY_SOFTPLUS only: > 0                   */
 } pdn_problem_t;
 
 typedef struct {

@@ -62,6 +62,14 @@ pdn_status_t check_problem(const pdn_problem_t *p) {
   if (fixed && p->decay != need) return PDN_ERR_INVALID_ARG;
   if (p->variant == PDN_VAR_FG2_GDN && p->d_k != p->d_v) return PDN_ERR_INVALID_ARG;
   if (!isfinite(p->q_scale)) return PDN_ERR_INVALID_ARG;
+  const int pro_all = PDN_PRO_L2NORM_QK | PDN_PRO_SIGMOID_GATES | PDN_PRO_DECAY_SOFTPLUS |
+                      PDN_PRO_DECAY_LOGSIGMOID;
+  if (p->prologue & ~pro_all) return PDN_ERR_INVALID_ARG;
+  const int pro_decay = p->prologue & (PDN_PRO_DECAY_SOFTPLUS | PDN_PRO_DECAY_LOGSIGMOID);
+  if (pro_decay == (PDN_PRO_DECAY_SOFTPLUS | PDN_PRO_DECAY_LOGSIGMOID)) return PDN_ERR_INVALID_ARG;
+  if (pro_decay && p->decay == PDN_DECAY_NONE) return PDN_ERR_INVALID_ARG;
+  if ((p->prologue & PDN_PRO_DECAY_SOFTPLUS) && !(p->decay_scale > 0.f && isfinite(p->decay_scale)))
+    return PDN_ERR_INVALID_ARG;
   if (is_precond(p->variant)) {
     if (!(p->precond_x >= 1.0f && p->precond_x <= 2.0f)) return PDN_ERR_INVALID_ARG;
     if (!(p->precond_eps > 0.0f) || !isfinite(p->precond_eps)) return PDN_ERR_INVALID_ARG;
@@ -111,6 +119,8 @@ KParams make_params(const pdn_problem_t *p, const pdn_tensors_t *t, int *err) {
   P.chunk = p->chunk == 0 ? 64 : p->chunk;
   P.variant = p->variant; P.decay = p->decay; P.dtype = p->dtype;
   P.q_scale = p->q_scale;
+  P.prologue = p->prologue;
+  P.decay_scale = p->decay_scale;
   P.x = is_precond(p->variant) ? p->precond_x : 1.0f;
   P.lnx = logf(P.x);
   P.eps = is_precond(p->variant) ? p->precond_eps : 1.0f;

@@ -89,7 +89,8 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_simt_kernel(const KParams P
       const size_t e = tok_index(P, b, c0 + t, h) * dk + i;
       sm.R[t][i] = ok ? ldf<Tin>(P.k, e) : 0.f;
       sm.Q[t][i] = ok ? ldf<Tin>(P.q, e) : 0.f;
-      if (P.decay == PDN_DECAY_CHANNEL) sm.G[t][i] = ok ? ldf<Tin>(P.log_alpha, e) : 0.f;
+      if (P.decay == PDN_DECAY_CHANNEL)
+        sm.G[t][i] = ok ? decay_act(P.prologue, P.decay_scale, ldf<Tin>(P.log_alpha, e)) : 0.f;
     }
     for (int idx = tid; idx < C * kDVB; idx += kThreads) {
       const int t = idx / kDVB, jj = idx % kDVB;
@@ -99,10 +100,27 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_simt_kernel(const KParams P
     for (int t = tid; t < C; t += kThreads) {
       const bool ok = t < Cn;
       const size_t e = tok_index(P, b, c0 + t, h);
-      sm.beta[t] = (ok && has_scalar_beta(P.variant)) ? ldf<float>(P.beta, e) : 0.f;
-      sm.la[t] = (ok && P.decay == PDN_DECAY_SCALAR) ? ldf<float>(P.log_alpha, e) : 0.f;
+      sm.beta[t] = (ok && has_scalar_beta(P.variant)) ? gate_act(P.prologue, ldf<float>(P.beta, e)) : 0.f;
+      sm.la[t] = (ok && P.decay == PDN_DECAY_SCALAR)
+                     ? decay_act(P.prologue, P.decay_scale, ldf<float>(P.log_alpha, e)) : 0.f;
     }
     __syncthreads();
+    if (P.prologue & PDN_PRO_L2NORM_QK) {
+      // L2 normalisation of each token's k and q (8 lanes per token and tensor)
+      const int warp = tid >> 5, lane = tid & 31;
+      for (int t = warp * 2 + (lane >> 4); t < C; t += (kThreads / 32) * 2) {
+        const int part = lane & 15;  // lanes part and part ^ 8 .. cover the token
+        float (*X)[kLD] = part < 8 ? sm.R : sm.Q;
+        float ss = 0.f;
+        for (int i = part & 7; i < dk; i += 8) ss = fmaf(X[t][i], X[t][i], ss);
+        ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+        ss += __shfl_xor_sync(0xffffffffu, ss, 2);
+        ss += __shfl_xor_sync(0xffffffffu, ss, 4);
+        const float inv = inv_norm(ss);
+        for (int i = part & 7; i < dk; i += 8) X[t][i] *= inv;
+      }
+      __syncthreads();
+    }
 
     // (b) per-channel scans: cumulative log decay and the key-energy prefix sum
     for (int i = tid; i < dk; i += kThreads) {
@@ -152,12 +170,13 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_simt_kernel(const KParams P
           qf *= precond_coef(sm.W[t][i], sm.mu[t], P.lnx);
           break;
         case PDN_VAR_FG2_GDN: case PDN_VAR_FG2_GDN_PLUS: {
-          const float sb = ok ? sqrtf(ldf<Tin>(P.beta, tok_index(P, b, c0 + t, h) * dk + i)) : 0.f;
+          const float sb =
+              ok ? sqrtf(gate_act(P.prologue, ldf<Tin>(P.beta, tok_index(P, b, c0 + t, h) * dk + i))) : 0.f;
           r = sb * kv;
           w = r;
         } break;
         case PDN_VAR_GDN2: {
-          const float e = ok ? ldf<Tin>(P.erase, tok_index(P, b, c0 + t, h) * dk + i) : 0.f;
+          const float e = ok ? gate_act(P.prologue, ldf<Tin>(P.erase, tok_index(P, b, c0 + t, h) * dk + i)) : 0.f;
           r = e * kv;
           w = kv;
         } break;
@@ -174,9 +193,9 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_simt_kernel(const KParams P
         const int t = idx / kDVB, jj = idx % kDVB;
         if (t < Cn && jj < nj) {
           const size_t e = tok_index(P, b, c0 + t, h) * dv + j0 + jj;
-          const float f = P.variant == PDN_VAR_FG2_GDN ? sqrtf(ldf<Tin>(P.beta, e))
-                          : P.variant == PDN_VAR_GDN2 ? ldf<Tin>(P.write, e)
-                                                      : sqrtf(ldf<Tin>(P.write, e));
+          const float f = P.variant == PDN_VAR_FG2_GDN ? sqrtf(gate_act(P.prologue, ldf<Tin>(P.beta, e)))
+                          : P.variant == PDN_VAR_GDN2 ? gate_act(P.prologue, ldf<Tin>(P.write, e))
+                                                      : sqrtf(gate_act(P.prologue, ldf<Tin>(P.write, e)));
           sm.U[t][jj] *= f;
         }
       }

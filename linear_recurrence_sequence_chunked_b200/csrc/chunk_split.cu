@@ -89,6 +89,17 @@ __global__ void __launch_bounds__(256) k0_chunk_energy(const KParams P, void *ws
     for (int m = 0; m < 4; ++m) {
       float kf[8];
       unpack8(cur[m], kf);
+      if (P.prologue & PDN_PRO_L2NORM_QK) {
+        // the token's 128 channels sit in the 16 lanes of this half-warp
+        float ss = 0.f;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) ss = fmaf(kf[e], kf[e], ss);
+#pragma unroll
+        for (int o = 1; o < 16; o <<= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+        const float inv = inv_norm(ss);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) kf[e] *= inv;
+      }
 #pragma unroll
       for (int e = 0; e < 8; ++e) acc[e] = fmaf(kf[e], kf[e], acc[e]);
     }
@@ -344,8 +355,11 @@ __global__ void __launch_bounds__(kK1Threads, kDecay == PDN_DECAY_CHANNEL ? 1 : 
     r.las = 0.f;
     if (tid < kC && tid < Cn_) {
       const size_t e = tok_index(P, b_, c0_ + tid, h_);
-      if (kScalarBeta) r.beta = __ldg(reinterpret_cast<const float *>(P.beta) + e);
-      if (kSc) r.las = fmaxf(__ldg(reinterpret_cast<const float *>(P.log_alpha) + e), kMinLogAlpha);
+      if (kScalarBeta) r.beta = gate_act(P.prologue, __ldg(reinterpret_cast<const float *>(P.beta) + e));
+      if (kSc)
+        r.las = fmaxf(decay_act(P.prologue, P.decay_scale,
+                                __ldg(reinterpret_cast<const float *>(P.log_alpha) + e)),
+                      kMinLogAlpha);
     }
     r.acar = (kPre && tid < kD) ? reinterpret_cast<const float *>(ws_block(ws, bh_, P.B * P.H, c_) + WS_A)[tid] : 0.f;
     return r;
@@ -415,8 +429,21 @@ __global__ void __launch_bounds__(kK1Threads, kDecay == PDN_DECAY_CHANNEL ? 1 : 
 #pragma unroll
     for (int m = 0; m < 4; ++m) {
       const int t = (tid >> 4) + 16 * m, c8 = tid & 15;
-      *reinterpret_cast<uint4 *>(smem + L::kKS + t * KS_LD + c8 * 16) =
-          *reinterpret_cast<const uint4 *>(smem + kKStage + t * 256 + ((c8 ^ (t & 7)) << 4));
+      uint4 kr = *reinterpret_cast<const uint4 *>(smem + kKStage + t * 256 + ((c8 ^ (t & 7)) << 4));
+      if (P.prologue & PDN_PRO_L2NORM_QK) {
+        // the token's 128 channels sit in the 16 lanes of this half-warp
+        float kf[8], ss = 0.f;
+        unpack8(kr, kf);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) ss = fmaf(kf[e], kf[e], ss);
+#pragma unroll
+        for (int o = 1; o < 16; o <<= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+        const float inv = inv_norm(ss);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) kf[e] *= inv;
+        kr = pack8(kf);
+      }
+      *reinterpret_cast<uint4 *>(smem + L::kKS + t * KS_LD + c8 * 16) = kr;
       if (kCh) {
         const bool ok = t < Cn;
         const size_t e = ok ? tok0 + (size_t)t * tstride + c8 * 8 : 0;
@@ -475,8 +502,10 @@ __global__ void __launch_bounds__(kK1Threads, kDecay == PDN_DECAY_CHANNEL ? 1 : 
       if (kCh) {
         const float2 lv = __bfloat1622float2(
             *reinterpret_cast<const __nv_bfloat162 *>(smem + L::kLasStage + t * 256 + i0 * 2));
-        l0[e] = fmaxf(lv.x, kMinLogAlpha);
-        l1[e] = fmaxf(lv.y, kMinLogAlpha);
+        // (past the sequence end the staged zeros stay zero: no decay)
+        const bool in_seq = t < Cn;
+        l0[e] = in_seq ? fmaxf(decay_act(P.prologue, P.decay_scale, lv.x), kMinLogAlpha) : 0.f;
+        l1[e] = in_seq ? fmaxf(decay_act(P.prologue, P.decay_scale, lv.y), kMinLogAlpha) : 0.f;
       } else if (kSc) {
         l0[e] = LAS[t];
         l1[e] = l0[e];
@@ -616,7 +645,21 @@ __global__ void __launch_bounds__(kK1Threads, kDecay == PDN_DECAY_CHANNEL ? 1 : 
       if ((lane >> 3) == 0) EGS[t] = eg_s;
     }
     const float be = kScalarBeta ? BETA[t] : 0.f;
-    const float qs = P.q_scale;
+    float qs = P.q_scale;
+    if (P.prologue & PDN_PRO_L2NORM_QK) {
+      // this token's 128 query channels: 32 here, the rest in lanes ^8, ^16, ^24
+      float ss = 0.f;
+#pragma unroll
+      for (int m = 0; m < 4; ++m) {
+        float qf[8];
+        unpack8(*reinterpret_cast<const uint4 *>(smem + L::kQS + t * KS_LD + (4 * m + (lane >> 3)) * 16), qf);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) ss = fmaf(qf[e], qf[e], ss);
+      }
+      ss += __shfl_xor_sync(0xffffffffu, ss, 8);
+      ss += __shfl_xor_sync(0xffffffffu, ss, 16);
+      qs *= inv_norm(ss);
+    }
 #pragma unroll
     for (int m = 0; m < 4; ++m) {
       const int c8 = 4 * m + (lane >> 3);
@@ -663,10 +706,10 @@ __global__ void __launch_bounds__(kK1Threads, kDecay == PDN_DECAY_CHANNEL ? 1 : 
         }
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
-          const float sq = sqrtf(gb[e]);
+          const float sq = sqrtf(gate_act(P.prologue, gb[e]));
           r[e] = sq * kf[e];
           w[e] = r[e];
-          vf[e] *= kVariant == PDN_VAR_FG2_GDN_PLUS ? sqrtf(gv[e]) : sq;
+          vf[e] *= kVariant == PDN_VAR_FG2_GDN_PLUS ? sqrtf(gate_act(P.prologue, gv[e])) : sq;
         }
       } else if (kVariant == PDN_VAR_GDN2) {
         float ge[8], gw[8];
@@ -684,9 +727,9 @@ __global__ void __launch_bounds__(kK1Threads, kDecay == PDN_DECAY_CHANNEL ? 1 : 
         }
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
-          r[e] = ge[e] * kf[e];
+          r[e] = gate_act(P.prologue, ge[e]) * kf[e];
           w[e] = kf[e];
-          vf[e] *= gw[e];
+          vf[e] *= gate_act(P.prologue, gw[e]);
         }
       } else {
 #pragma unroll

@@ -15,6 +15,8 @@ struct KParams {
   int B, T, H, dk, dv, chunk;
   int variant, decay, dtype;
   float q_scale, x, lnx, eps;
+  int prologue;       // PDN_PRO_* bits
+  float decay_scale;  // PDN_PRO_DECAY_SOFTPLUS
   const void *q, *k, *v, *log_alpha, *beta, *erase, *write;
   const float *S0;
   float *ST;
@@ -70,6 +72,28 @@ __device__ __forceinline__ float precond_coef(float logA, float mu, float lnx) {
   const float c = logA - mu;
   const float s = c / (1.0f + fabsf(c));
   return expf(-s * lnx);
+}
+
+// ---- fused prologue (PDN_PRO_* bits) -----------------------------------
+// softplus(x) = log(1 + e^x), written as max(x, 0) + log(1 + e^{-|x|}) so
+// that neither exponential overflows.
+__device__ __forceinline__ float softplus_f(float x) {
+  return fmaxf(x, 0.f) + log1pf(expf(-fabsf(x)));
+}
+// A gate or gain as the kernels use it: sigmoid of the input when the
+// problem's gates arrive as logits, else the input.
+__device__ __forceinline__ float gate_act(int prologue, float x) {
+  return (prologue & PDN_PRO_SIGMOID_GATES) ? 1.f / (1.f + expf(-x)) : x;
+}
+// The log decay as the kernels use it.
+__device__ __forceinline__ float decay_act(int prologue, float decay_scale, float x) {
+  if (prologue & PDN_PRO_DECAY_SOFTPLUS) return -decay_scale * softplus_f(x);
+  if (prologue & PDN_PRO_DECAY_LOGSIGMOID) return -softplus_f(-x);
+  return x;
+}
+// 1 / max(||x||, 1e-12) from a sum of squares (L2 normalisation of q, k).
+__device__ __forceinline__ float inv_norm(float sumsq) {
+  return 1.f / fmaxf(sqrtf(sumsq), 1e-12f);
 }
 
 __device__ __forceinline__ void record_error(int *err, int code) {

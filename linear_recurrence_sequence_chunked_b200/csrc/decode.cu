@@ -76,6 +76,14 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const KParams P) {
   if (chan) {
     kv = ldf<Tin>(P.k, tokh * dk + tid);
     qv = ldf<Tin>(P.q, tokh * dk + tid);
+  }
+  if (P.prologue & PDN_PRO_L2NORM_QK) {  // fused prologue: unit-norm k and q
+    const float ssk = block_sum(chan ? kv * kv : 0.f, s_red);
+    const float ssq = block_sum(chan ? qv * qv : 0.f, s_red);
+    kv *= inv_norm(ssk);
+    qv *= inv_norm(ssq);
+  }
+  if (chan) {
     if (precond) {
       float a = P.AT[(size_t)bh * dk + tid] + kv * kv;
       P.AT[(size_t)bh * dk + tid] = a;
@@ -89,38 +97,41 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const KParams P) {
     switch (P.variant) {
       case PDN_VAR_PDN: case PDN_VAR_PGDN: case PDN_VAR_PKDA:
         r = kv;
-        w = ldf<float>(P.beta, tokh) * precond_coef(logA, mu, P.lnx) * kv;
+        w = gate_act(P.prologue, ldf<float>(P.beta, tokh)) * precond_coef(logA, mu, P.lnx) * kv;
         break;
       case PDN_VAR_PLA:  // no erase; the preconditioner acts on the query
         r = 0.f;
-        w = ldf<float>(P.beta, tokh) * kv;
+        w = gate_act(P.prologue, ldf<float>(P.beta, tokh)) * kv;
         qv *= precond_coef(logA, mu, P.lnx);
         break;
       case PDN_VAR_FG2_GDN: case PDN_VAR_FG2_GDN_PLUS:
-        r = sqrtf(ldf<Tin>(P.beta, tokh * dk + tid)) * kv;
+        r = sqrtf(gate_act(P.prologue, ldf<Tin>(P.beta, tokh * dk + tid))) * kv;
         w = r;
         break;
       case PDN_VAR_GDN2:
-        r = ldf<Tin>(P.erase, tokh * dk + tid) * kv;
+        r = gate_act(P.prologue, ldf<Tin>(P.erase, tokh * dk + tid)) * kv;
         w = kv;
         break;
       default:
         r = kv;
-        w = ldf<float>(P.beta, tokh) * kv;
+        w = gate_act(P.prologue, ldf<float>(P.beta, tokh)) * kv;
     }
     s_r[tid] = r;
     s_w[tid] = w;
     s_q[tid] = qv;
     float al = 1.f;
-    if (P.decay == PDN_DECAY_SCALAR) al = expf(ldf<float>(P.log_alpha, tokh));
-    else if (P.decay == PDN_DECAY_CHANNEL) al = expf(ldf<Tin>(P.log_alpha, tokh * dk + tid));
+    if (P.decay == PDN_DECAY_SCALAR)
+      al = expf(decay_act(P.prologue, P.decay_scale, ldf<float>(P.log_alpha, tokh)));
+    else if (P.decay == PDN_DECAY_CHANNEL)
+      al = expf(decay_act(P.prologue, P.decay_scale, ldf<Tin>(P.log_alpha, tokh * dk + tid)));
     s_al[tid] = al;
   }
   for (int j = tid; j < dv; j += kThreads) {
     float u = ldf<Tin>(P.v, tokh * dv + j);
-    if (P.variant == PDN_VAR_FG2_GDN) u *= sqrtf(ldf<Tin>(P.beta, tokh * dv + j));
-    else if (P.variant == PDN_VAR_GDN2) u *= ldf<Tin>(P.write, tokh * dv + j);
-    else if (P.variant == PDN_VAR_FG2_GDN_PLUS) u *= sqrtf(ldf<Tin>(P.write, tokh * dv + j));
+    if (P.variant == PDN_VAR_FG2_GDN) u *= sqrtf(gate_act(P.prologue, ldf<Tin>(P.beta, tokh * dv + j)));
+    else if (P.variant == PDN_VAR_GDN2) u *= gate_act(P.prologue, ldf<Tin>(P.write, tokh * dv + j));
+    else if (P.variant == PDN_VAR_FG2_GDN_PLUS)
+      u *= sqrtf(gate_act(P.prologue, ldf<Tin>(P.write, tokh * dv + j)));
     s_u[j] = u;
   }
   const float wq = block_sum(chan ? w * qv : 0.f, s_red);  // ends with __syncthreads
@@ -281,15 +292,18 @@ __global__ void __launch_bounds__(kTmaThreads, 1) decode_tma_kernel(const KParam
       t.q = ldf<Tin>(P.q, e);
       t.v = ldf<Tin>(P.v, e);
       if (precond) t.a = P.AT[(size_t)item * kD128 + tid];
-      if (P.variant == PDN_VAR_FG2_GDN || P.variant == PDN_VAR_FG2_GDN_PLUS) t.beta = ldf<Tin>(P.beta, e);
-      else if (P.variant != PDN_VAR_GDN2) t.beta = ldf<float>(P.beta, tokh);
-      if (P.decay == PDN_DECAY_SCALAR) t.la = ldf<float>(P.log_alpha, tokh);
-      else if (P.decay == PDN_DECAY_CHANNEL) t.la = ldf<Tin>(P.log_alpha, e);
+      const int pro = P.prologue;
+      if (P.variant == PDN_VAR_FG2_GDN || P.variant == PDN_VAR_FG2_GDN_PLUS)
+        t.beta = gate_act(pro, ldf<Tin>(P.beta, e));
+      else if (P.variant != PDN_VAR_GDN2)
+        t.beta = gate_act(pro, ldf<float>(P.beta, tokh));
+      if (P.decay == PDN_DECAY_SCALAR) t.la = decay_act(pro, P.decay_scale, ldf<float>(P.log_alpha, tokh));
+      else if (P.decay == PDN_DECAY_CHANNEL) t.la = decay_act(pro, P.decay_scale, ldf<Tin>(P.log_alpha, e));
       if (P.variant == PDN_VAR_GDN2) {
-        t.ge = ldf<Tin>(P.erase, e);
-        t.gw = ldf<Tin>(P.write, e);
+        t.ge = gate_act(pro, ldf<Tin>(P.erase, e));
+        t.gw = gate_act(pro, ldf<Tin>(P.write, e));
       } else if (P.variant == PDN_VAR_FG2_GDN_PLUS) {
-        t.gw = ldf<Tin>(P.write, e);
+        t.gw = gate_act(pro, ldf<Tin>(P.write, e));
       }
     }
     return t;
@@ -303,8 +317,13 @@ __global__ void __launch_bounds__(kTmaThreads, 1) decode_tma_kernel(const KParam
     const Tok nxt = (k + 1 < nloc) ? load_tok(k + 1) : cur;
 
     // per-token vectors (overlap the bulk loads in flight)
-    const float kv = cur.k;
-    float qv = cur.q;
+    float kv = cur.k, qv = cur.q;
+    if (P.prologue & PDN_PRO_L2NORM_QK) {  // fused prologue: unit-norm k and q
+      const float ssk = consumer_sum(chan ? kv * kv : 0.f, sm.red);
+      const float ssq = consumer_sum(chan ? qv * qv : 0.f, sm.red);
+      kv *= inv_norm(ssk);
+      qv *= inv_norm(ssq);
+    }
     float logA = 0.f;
     if (chan && precond) {
       const float a = cur.a + kv * kv;

@@ -27,6 +27,8 @@ DECAYS = {"none": 0, "scalar": 1, "channel": 2}
 DTYPES = {torch.float32: 0, torch.bfloat16: 1}
 IMPLS = {"auto": 0, "simt": 1, "tc": 2}
 PRECOND_VARIANTS = ("PDN", "PGDN", "PKDA", "PLA")
+# fused prologue bits (pdn_problem_t.prologue)
+PRO_L2NORM_QK, PRO_SIGMOID_GATES, PRO_DECAY_SOFTPLUS, PRO_DECAY_LOGSIGMOID = 1, 2, 4, 8
 
 
 class PdnProblem(ctypes.Structure):
@@ -34,7 +36,8 @@ class PdnProblem(ctypes.Structure):
                 ("d_k", ctypes.c_int), ("d_v", ctypes.c_int), ("chunk", ctypes.c_int),
                 ("variant", ctypes.c_int), ("decay", ctypes.c_int), ("dtype", ctypes.c_int),
                 ("impl", ctypes.c_int), ("q_scale", ctypes.c_float),
-                ("precond_x", ctypes.c_float), ("precond_eps", ctypes.c_float)]
+                ("precond_x", ctypes.c_float), ("precond_eps", ctypes.c_float),
+                ("prologue", ctypes.c_int), ("decay_scale", ctypes.c_float)]
 
 
 class PdnTensors(ctypes.Structure):
@@ -160,11 +163,12 @@ def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
 def make_problem(variant: str, B: int, T: int, H: int, d_k: int, d_v: int, dtype,
                  decay: Optional[str] = None, chunk: int = 64, impl: str = "auto",
                  q_scale: float = 1.0, precond_x: float = 1.5,
-                 precond_eps: float = 1e-6) -> PdnProblem:
+                 precond_eps: float = 1e-6, prologue: int = 0,
+                 decay_scale: float = 1.0) -> PdnProblem:
     if decay is None:
         decay = {"DN": "none", "PDN": "none", "GDN": "scalar", "PGDN": "scalar"}.get(variant, "channel")
     return PdnProblem(B, T, H, d_k, d_v, chunk, VARIANTS[variant], DECAYS[decay], DTYPES[dtype],
-                      IMPLS[impl], q_scale, precond_x, precond_eps)
+                      IMPLS[impl], q_scale, precond_x, precond_eps, prologue, decay_scale)
 
 
 def _host_ptr(t: Optional[torch.Tensor]) -> Optional[int]:
@@ -206,7 +210,7 @@ def _check(code, where):
 def chunk_fwd(variant: str, q, k, v, log_alpha=None, beta=None, erase=None, write=None,
               S0=None, A0=None, chunk: int = 64, impl: str = "auto", q_scale: float = 1.0,
               precond_x: float = 1.5, precond_eps: float = 1e-6, want_state: bool = True,
-              out=None, workspace=None):
+              out=None, workspace=None, prologue: int = 0, decay_scale: float = 1.0):
     """Chunked forward on torch tensors (all on one CUDA device, contiguous).
 
     Returns (o, S_T, A_T); S_T/A_T are None when not requested / not used.
@@ -215,7 +219,7 @@ def chunk_fwd(variant: str, q, k, v, log_alpha=None, beta=None, erase=None, writ
     d_v = v.shape[3]
     dev = k.device
     p = make_problem(variant, B, T, H, d_k, d_v, k.dtype, _decay_of(log_alpha), chunk, impl,
-                     q_scale, precond_x, precond_eps)
+                     q_scale, precond_x, precond_eps, prologue, decay_scale)
     o = out if out is not None else torch.empty(B, T, H, d_v, dtype=k.dtype, device=dev)
     ST = torch.empty(B, H, d_v, d_k, dtype=torch.float32, device=dev) if want_state else None
     AT = (torch.empty(B, H, d_k, dtype=torch.float32, device=dev)
@@ -236,14 +240,15 @@ def chunk_fwd(variant: str, q, k, v, log_alpha=None, beta=None, erase=None, writ
 
 def decode_step(variant: str, q, k, v, S, A=None, log_alpha=None, beta=None, erase=None,
                 write=None, q_scale: float = 1.0, precond_x: float = 1.5,
-                precond_eps: float = 1e-6, out=None):
+                precond_eps: float = 1e-6, out=None, prologue: int = 0,
+                decay_scale: float = 1.0):
     """One decode token per sequence: q, k [B,1,H,d_k], v [B,1,H,d_v]; updates
     the fp32 state S [B,H,d_v,d_k] (and accumulator A [B,H,d_k]) in place and
     returns o [B,1,H,d_v]."""
     B, T, H, d_k = k.shape
     d_v = v.shape[3]
     p = make_problem(variant, B, T, H, d_k, d_v, k.dtype, _decay_of(log_alpha), 64, "auto",
-                     q_scale, precond_x, precond_eps)
+                     q_scale, precond_x, precond_eps, prologue, decay_scale)
     o = out if out is not None else torch.empty(B, T, H, d_v, dtype=k.dtype, device=k.device)
     t = make_tensors(q, k, v, o, log_alpha, beta, erase, write, S, S, A, A)
     stream = torch.cuda.current_stream(k.device).cuda_stream

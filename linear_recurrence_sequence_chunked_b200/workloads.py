@@ -133,6 +133,66 @@ def make_inputs(w: Workload, device="cpu", B: Optional[int] = None, T: Optional[
     return {n: (t.to(device) if t is not None else None) for n, t in out.items()}
 
 
+# fused-prologue bits (pdn.h PDN_PRO_*)
+PRO_L2NORM_QK, PRO_SIGMOID_GATES, PRO_DECAY_SOFTPLUS, PRO_DECAY_LOGSIGMOID = 1, 2, 4, 8
+
+
+def raw_prologue(w: Workload):
+    """(prologue bits, decay scale) that turn the raw projections of
+    ``make_raw_inputs(w)`` into the inputs ``make_inputs(w)`` draws."""
+    bits = PRO_L2NORM_QK | PRO_SIGMOID_GATES
+    if w.decay == "none":
+        return bits, 1.0
+    if w.decay_recipe == "sigmoid":
+        return bits | PRO_DECAY_LOGSIGMOID, 1.0
+    if w.decay_recipe == "softplus":
+        return bits | PRO_DECAY_SOFTPLUS, 0.1
+    raise ValueError("no raw form for the %r decay recipe" % w.decay_recipe)
+
+
+def make_raw_inputs(w: Workload, device="cpu", B: Optional[int] = None, T: Optional[int] = None,
+                    generator_device: Optional[str] = None) -> dict:
+    """The raw projections behind ``make_inputs(w)``: the same seed and draw
+    order, with the activations left to a fused prologue (q and k not
+    normalised, gains and gates as logits, the decay as its pre-activation
+    z, or z + 2 for the log-sigmoid recipe)."""
+    B = w.B if B is None else B
+    T = w.T if T is None else T
+    gdev = torch.device(generator_device or device)
+    g = torch.Generator(device=gdev)
+    g.manual_seed(w.seed)
+    dt = w.torch_dtype
+    H, dk, dv = w.H, w.dk, w.dv
+
+    def randn(*shape):
+        return torch.randn(*shape, generator=g, device=gdev, dtype=torch.float32)
+
+    q = randn(B, T, H, dk).to(dt)
+    k = randn(B, T, H, dk).to(dt)
+    v = randn(B, T, H, dv).to(dt)
+    beta = None
+    if w.variant in ("FG2_GDN", "FG2_GDN_PLUS"):
+        beta = randn(B, T, H, dk).to(dt)
+    elif w.variant != "GDN2":
+        beta = randn(B, T, H)
+    log_alpha = None
+    if w.decay != "none":
+        raw_prologue(w)  # rejects recipes without a raw form
+        shape = (B, T, H) if w.decay == "scalar" else (B, T, H, dk)
+        z = randn(*shape)
+        if w.decay_recipe == "sigmoid":
+            z = z + 2.0
+        log_alpha = z if w.decay == "scalar" else z.to(dt)
+    erase = write = None
+    if w.variant == "GDN2":
+        erase = randn(B, T, H, dk).to(dt)
+        write = randn(B, T, H, dv).to(dt)
+    elif w.variant == "FG2_GDN_PLUS":
+        write = randn(B, T, H, dv).to(dt)
+    out = dict(q=q, k=k, v=v, log_alpha=log_alpha, beta=beta, erase=erase, write=write)
+    return {n: (t.to(device) if t is not None else None) for n, t in out.items()}
+
+
 def slice_chain(inputs: dict, b: int, h: int, t0: int = 0, t1: Optional[int] = None) -> dict:
     """The inputs of one (batch, head) chain over tokens [t0, t1), as a B=1,
     H=1 problem on the CPU (used to check sampled chains of large workloads)."""

@@ -97,7 +97,7 @@ def _tensors(**over):
 def _problem(**over):
     p = dict(B=2, T=100, H=4, d_k=64, d_v=64, chunk=64, variant=pdn.VARIANTS["PGDN"],
              decay=pdn.DECAYS["scalar"], dtype=1, impl=0, q_scale=1.0, precond_x=1.5,
-             precond_eps=1e-6)
+             precond_eps=1e-6, prologue=0, decay_scale=1.0)
     p.update(over)
     return pdn.PdnProblem(**p)
 
@@ -108,6 +108,9 @@ INVALID_PROBLEMS = [
     dict(decay=pdn.DECAYS["channel"]),              # PGDN needs scalar decay
     dict(precond_x=2.5), dict(precond_x=0.5), dict(precond_eps=0.0),
     dict(q_scale=float("nan")),
+    dict(prologue=16), dict(prologue=-1), dict(prologue=4 | 8),  # unknown bits / both decays
+    dict(prologue=4, decay_scale=0.0), dict(prologue=4, decay_scale=float("inf")),
+    dict(prologue=8, variant=pdn.VARIANTS["PDN"], decay=pdn.DECAYS["none"]),  # decay bit, no decay
 ]
 
 

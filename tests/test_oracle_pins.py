@@ -11,6 +11,7 @@ import pytest
 
 import oracle
 from oracle import chunked
+from oracle import prologue
 
 VARIANTS = ["DN", "GDN", "KDA", "PDN", "PGDN", "PKDA", "FG2_GDN", "GDN2", "PLA", "FG2_GDN_PLUS"]
 DECAY = {"DN": "none", "PDN": "none", "GDN": "scalar", "PGDN": "scalar",
@@ -303,6 +304,48 @@ def test_fg2_plus_reductions(decay):
     d["write"] = np.zeros_like(d["write"])
     o5, S5, _ = oracle.forward("FG2_GDN_PLUS", **d)
     assert not o5.any() and not S5.any()
+
+
+# ---------------------------------------------------------------- fused prologue
+def test_prologue_maps_closed_forms_and_references():
+    """The prologue's maps against closed forms and scipy's reference
+    implementations: sigmoid(0) = 1/2, softplus(0) = log 2, log sigmoid(x) =
+    -softplus(-x), sigmoid(x) + sigmoid(-x) = 1; unit norms after L2
+    normalisation, direction kept, zero vectors stay zero."""
+    from scipy.special import expit, log_expit
+    x = np.linspace(-60, 60, 241)
+    np.testing.assert_allclose(prologue.sigmoid(x), expit(x), rtol=1e-15, atol=0)
+    np.testing.assert_allclose(-prologue.softplus(-x), log_expit(x), rtol=1e-14, atol=1e-300)
+    np.testing.assert_allclose(prologue.sigmoid(x) + prologue.sigmoid(-x), 1.0, rtol=0, atol=1e-15)
+    assert prologue.sigmoid(np.array([0.0]))[0] == 0.5
+    assert prologue.softplus(np.array([0.0]))[0] == np.log(2.0)
+    np.testing.assert_allclose(prologue.softplus(np.array([30.0, -30.0])),
+                               [30.0 + np.exp(-30.0), np.exp(-30.0)], rtol=1e-12)
+    rng = np.random.default_rng(40)
+    v = rng.standard_normal((5, 7, 16)) * 3.0
+    n = prologue.l2_normalise(v)
+    np.testing.assert_allclose(np.linalg.norm(n, axis=-1), 1.0, rtol=1e-15)
+    np.testing.assert_allclose(n * np.linalg.norm(v, axis=-1, keepdims=True), v, rtol=1e-14)
+    assert not prologue.l2_normalise(np.zeros((2, 4))).any()
+
+
+def test_prologue_apply_selects_by_bits():
+    """Each bit touches only its tensors; the decay bits map log_alpha."""
+    rng = np.random.default_rng(41)
+    raw = dict(q=rng.standard_normal((1, 3, 2, 4)), k=rng.standard_normal((1, 3, 2, 4)),
+               v=rng.standard_normal((1, 3, 2, 4)), log_alpha=rng.standard_normal((1, 3, 2)),
+               beta=rng.standard_normal((1, 3, 2)), erase=None, write=None)
+    a = prologue.apply(raw, 0)
+    for n in ("q", "k", "v", "log_alpha", "beta"):
+        np.testing.assert_array_equal(a[n], raw[n])
+    a = prologue.apply(raw, prologue.L2NORM_QK | prologue.SIGMOID_GATES | prologue.DECAY_SOFTPLUS, 0.1)
+    np.testing.assert_array_equal(a["v"], raw["v"])
+    np.testing.assert_allclose(np.linalg.norm(a["k"], axis=-1), 1.0, rtol=1e-15)
+    np.testing.assert_allclose(a["beta"], 1 / (1 + np.exp(-raw["beta"])), rtol=1e-15)
+    np.testing.assert_allclose(a["log_alpha"], -0.1 * np.log1p(np.exp(raw["log_alpha"])), rtol=1e-14)
+    a = prologue.apply(raw, prologue.DECAY_LOGSIGMOID)
+    np.testing.assert_allclose(a["log_alpha"], np.log(1 / (1 + np.exp(-raw["log_alpha"]))), rtol=1e-14)
+    np.testing.assert_array_equal(a["beta"], raw["beta"])
 
 
 # ---------------------------------------------------------------- P7
