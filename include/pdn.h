@@ -235,6 +235,46 @@ pdn_status_t pdn_chunk_fwd_host(const pdn_problem_t *p, const pdn_tensors_t *hos
                                 const pdn_tensors_t *dev, void *workspace, size_t ws_bytes,
                                 int slices, void *stream);
 
+/* ---- Sequence-parallel prefill ("FG2-GDN", ja §4: 32k-token contexts) ----
+ * A long sequence can be cut into segments processed on different GPUs. Every
+ * update acts on the state by right-multiplication, so a segment maps its
+ * start state affinely, S_end = S_start A_seg + B_seg; the three calls below
+ * give A_seg, the accumulator's key energy and the composition, and the
+ * exchange between GPUs is the caller's (e.g. an all-gather over NCCL):
+ *   1. pdn_key_energy on each segment (A0 = NULL), exchange, prefix-sum: the
+ *      accumulator at every segment start (preconditioned variants);
+ *   2. B_seg = ST of pdn_chunk_fwd(segment, S0 = NULL, A0 = its start);
+ *      A_seg = ST of pdn_chunk_transition(segment, A0 = its start);
+ *   3. exchange (A_seg, B_seg); S_start of segment g = pdn_state_compose
+ *      folded over the segments before it, from the sequence's S0;
+ *   4. pdn_chunk_fwd(segment, S0 = S_start, A0 = its start) gives the outputs.
+ */
+
+/* Segment transition A_seg = prod_t Diag(alpha_t) (I - r_t w_t^T) over the
+ * problem's T tokens, per (batch, head), written to t->ST as [B,H,d_k,d_k]
+ * fp32: the chunked forward with zero targets from the identity state. Needs
+ * d_v == d_k; t->S0 must be NULL; t->v and t->o are not used (may be NULL);
+ * everything else (gates, A0/AT, workspace, impl) as for pdn_chunk_fwd. */
+pdn_status_t pdn_chunk_transition(const pdn_problem_t *p, const pdn_tensors_t *t,
+                                  void *workspace, size_t ws_bytes, void *stream);
+
+/* Key energy: t->AT = t->A0 + sum_t k_t . k_t over the problem's T tokens,
+ * [B,H,d_k] fp32 (A0 NULL = zeros; k L2-normalised first under
+ * PDN_PRO_L2NORM_QK). Uses p's shape, dtype and prologue and t->k, A0, AT. */
+pdn_status_t pdn_key_energy(const pdn_problem_t *p, const pdn_tensors_t *t, void *stream);
+
+/* State composition: S_out = S_in A + B_add for each of BH (batch, head)
+ * pairs, fp32: S_in, B_add, S_out [BH, d_v, d_k], A [BH, d_k, d_k]. S_in and
+ * B_add may be NULL (zero); S_out may alias B_add but not S_in or A. */
+pdn_status_t pdn_state_compose(int BH, int d_v, int d_k, const float *S_in, const float *A,
+                               const float *B_add, float *S_out, void *stream);
+
+/* out[i] = base[i] + sum_{g < n} parts[g * len + i], fp32 (base may be NULL =
+ * zero; out may alias base, not parts): the accumulator at the start of
+ * segment n from the gathered key energies of the segments before it. */
+pdn_status_t pdn_accumulate(int n, long long len, const float *parts, const float *base,
+                            float *out, void *stream);
+
 /* One decode step: p->T must be 1. The state and, for preconditioned
  * variants, the accumulator are updated IN PLACE: pass S0 == ST (non-NULL)
  * and A0 == AT (non-NULL for PDN/PGDN/PKDA, NULL otherwise). */

@@ -234,6 +234,63 @@ extern "C" pdn_status_t pdn_chunk_fwd_profiled(const pdn_problem_t *p, const pdn
   return PDN_OK;
 }
 
+extern "C" pdn_status_t pdn_chunk_transition(const pdn_problem_t *p, const pdn_tensors_t *t,
+                                             void *workspace, size_t ws_bytes, void *stream) {
+  pdn_status_t st = check_problem(p);
+  if (st != PDN_OK) return st;
+  if (!t || p->d_v != p->d_k || t->S0 || !t->ST) return PDN_ERR_INVALID_ARG;
+  // v and o are not used: check the rest with stand-ins of the right alignment
+  pdn_tensors_t c = *t;
+  if (!c.v) c.v = c.k;
+  if (!c.o) c.o = const_cast<void *>(c.k);
+  int impl = -1;
+  if ((st = check_chunk_fwd(p, &c, workspace, ws_bytes, &impl)) != PDN_OK) return st;
+  KParams P = make_params(p, t, device_error_word());
+  if (!P.err) return PDN_ERR_CUDA;
+  P.transition = 1;
+  P.v = nullptr;
+  P.o = nullptr;
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const cudaError_t e = impl == PDN_IMPL_TC ? launch_chunk_split(P, workspace, s) : launch_chunk_simt(P, s);
+  return e == cudaSuccess ? PDN_OK : PDN_ERR_CUDA;
+}
+
+extern "C" pdn_status_t pdn_key_energy(const pdn_problem_t *p, const pdn_tensors_t *t,
+                                       void *stream) {
+  pdn_status_t st = check_problem(p);
+  if (st != PDN_OK) return st;
+  if (!t || !t->AT || (p->T > 0 && !t->k)) return PDN_ERR_INVALID_ARG;
+  if ((t->k && !aligned(t->k, 16)) || !aligned(t->AT, 16) || (t->A0 && !aligned(t->A0, 16)))
+    return PDN_ERR_INVALID_ARG;
+  KParams P = make_params(p, t, nullptr);
+  return launch_key_energy(P, static_cast<cudaStream_t>(stream)) == cudaSuccess ? PDN_OK
+                                                                                 : PDN_ERR_CUDA;
+}
+
+extern "C" pdn_status_t pdn_accumulate(int n, long long len, const float *parts,
+                                       const float *base, float *out, void *stream) {
+  if (n < 0 || len < 0 || !out || (n > 0 && !parts)) return PDN_ERR_INVALID_ARG;
+  if (out == parts) return PDN_ERR_INVALID_ARG;
+  return launch_accumulate(n, len, parts, base, out, static_cast<cudaStream_t>(stream)) ==
+                 cudaSuccess
+             ? PDN_OK
+             : PDN_ERR_CUDA;
+}
+
+extern "C" pdn_status_t pdn_state_compose(int BH, int d_v, int d_k, const float *S_in,
+                                          const float *A, const float *B_add, float *S_out,
+                                          void *stream) {
+  if (BH < 1 || !head_dim_ok(d_v) || !head_dim_ok(d_k) || !A || !S_out) return PDN_ERR_INVALID_ARG;
+  if (S_out == S_in || S_out == A) return PDN_ERR_INVALID_ARG;
+  const void *all[] = {S_in, A, B_add, S_out};
+  for (const void *ptr : all)
+    if (ptr && !aligned(ptr, 16)) return PDN_ERR_INVALID_ARG;
+  return launch_compose(BH, d_v, d_k, S_in, A, B_add, S_out, static_cast<cudaStream_t>(stream)) ==
+                 cudaSuccess
+             ? PDN_OK
+             : PDN_ERR_CUDA;
+}
+
 extern "C" pdn_status_t pdn_decode_step(const pdn_problem_t *p, const pdn_tensors_t *t,
                                         void *stream) {
   pdn_status_t st = check_problem(p);

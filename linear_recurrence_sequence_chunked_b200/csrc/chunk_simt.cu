@@ -71,7 +71,9 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_simt_kernel(const KParams P
   const size_t sbase = (size_t)bh * dv * dk;
   for (int idx = tid; idx < kDVB * dk; idx += kThreads) {
     const int jj = idx / dk, i = idx % dk;
-    sm.S[jj][i] = (P.S0 && jj < nj) ? P.S0[sbase + (size_t)(j0 + jj) * dk + i] : 0.f;
+    sm.S[jj][i] = jj >= nj       ? 0.f
+                  : P.transition ? (j0 + jj == i ? 1.f : 0.f)  // the identity (d_v = d_k)
+                  : P.S0         ? P.S0[sbase + (size_t)(j0 + jj) * dk + i] : 0.f;
   }
   for (int i = tid; i < dk; i += kThreads)
     sm.A[i] = (precond && P.A0) ? P.A0[(size_t)bh * dk + i] : 0.f;
@@ -94,7 +96,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_simt_kernel(const KParams P
     }
     for (int idx = tid; idx < C * kDVB; idx += kThreads) {
       const int t = idx / kDVB, jj = idx % kDVB;
-      const bool ok = t < Cn && jj < nj;
+      const bool ok = t < Cn && jj < nj && !P.transition;  // transition mode: no targets
       sm.U[t][jj] = ok ? ldf<Tin>(P.v, tok_index(P, b, c0 + t, h) * dv + j0 + jj) : 0.f;
     }
     for (int t = tid; t < C; t += kThreads) {
@@ -297,7 +299,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_simt_kernel(const KParams P
     // (g) O = Qh S^T + P Delta for the valid tokens
     for (int idx = tid; idx < C * kDVB; idx += kThreads) {
       const int t = idx / kDVB, jj = idx % kDVB;
-      if (t < Cn && jj < nj) {
+      if (t < Cn && jj < nj && P.o) {
         float acc = 0.f;
         for (int i = 0; i < dk; ++i) acc = fmaf(sm.Q[t][i], sm.S[jj][i], acc);
         for (int s = 0; s <= t; ++s) acc = fmaf(sm.Pm[t][s], sm.U[s][jj], acc);

@@ -378,8 +378,10 @@ __global__ void __launch_bounds__(kK1Threads, kDecay == PDN_DECAY_CHANNEL ? 1 : 
       const int t = (tid >> 4) + 16 * m, c8 = tid & 15;
       const bool ok = t < Cn_;
       const size_t e = ok ? tok0_ + (size_t)t * tstride + c8 * 8 : 0;
+      // (transition mode: no targets; the zero fill reads nothing from k)
+      const bool use_v = !P.transition && P.v;
       cp_async16(sb + L::kWH + t * 256 + ((c8 ^ (t & 7)) << 4),
-                 reinterpret_cast<const __nv_bfloat16 *>(P.v) + e, ok);
+                 reinterpret_cast<const __nv_bfloat16 *>(use_v ? P.v : P.k) + e, ok && use_v);
     }
     cp_async_commit();
   };
@@ -1209,6 +1211,7 @@ __device__ __forceinline__ bool k2_wait(uint64_t *bar, uint32_t parity, volatile
 __device__ __forceinline__ void k2_store_o(const KParams &P, uint32_t taddr, int b, int h,
                                            int pc0, int Cn, int lane, int quarter, int cg,
                                            int part) {
+  if (!P.o) return;  // transition mode writes no output
   const size_t tstride = (size_t)P.H * kD;
   const int j = 32 * quarter + lane;
   __nv_bfloat16 *orow =
@@ -1405,7 +1408,10 @@ __global__ void __launch_bounds__(kK2Threads, 1) k2_state(const KParams P, void 
         if (n == 0) {
 #pragma unroll
           for (int u = 0; u < 2; ++u) {
-            if (P.S0) {
+            if (P.transition) {  // the identity: S[j][i] = (i == j)
+#pragma unroll
+              for (int e = 0; e < 16; ++e) sv[u][e] = (col0 + 16 * u + e == j) ? 1.f : 0.f;
+            } else if (P.S0) {
               const float4 *src = reinterpret_cast<const float4 *>(
                   P.S0 + ((size_t)bh * kD + j) * kD + col0 + 16 * u);
 #pragma unroll

@@ -17,6 +17,10 @@ struct KParams {
   float q_scale, x, lnx, eps;
   int prologue;       // PDN_PRO_* bits
   float decay_scale;  // PDN_PRO_DECAY_SOFTPLUS
+  // Segment transition mode (pdn_chunk_transition): the targets u are zero,
+  // the state starts from the identity (d_v = d_k) and no output is written,
+  // so the final state is prod_t Diag(alpha_t) (I - r_t w_t^T).
+  int transition;
   const void *q, *k, *v, *log_alpha, *beta, *erase, *write;
   const float *S0;
   float *ST;

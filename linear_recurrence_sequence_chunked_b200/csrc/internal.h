@@ -20,6 +20,14 @@ size_t split_workspace_bytes(const KParams &P);
 cudaError_t launch_chunk_split(const KParams &P, void *workspace, cudaStream_t stream,
                                cudaEvent_t *ev = nullptr);
 
+// Sequence-parallel pieces: AT = A0 + sum_t k.k per (batch, head); and
+// S_out = S_in A + B_add per (batch, head) (S_in, B_add may be NULL = zero).
+cudaError_t launch_key_energy(const KParams &P, cudaStream_t stream);
+cudaError_t launch_compose(int BH, int dv, int dk, const float *S_in, const float *A,
+                           const float *Badd, float *S_out, cudaStream_t stream);
+cudaError_t launch_accumulate(int n, long long len, const float *parts, const float *base,
+                              float *out, cudaStream_t stream);
+
 // One decode step (state streamed through once).
 cudaError_t launch_decode(const KParams &P, cudaStream_t stream);
 

@@ -77,6 +77,14 @@ def load() -> ctypes.CDLL:
         lib.pdn_chunk_fwd_noalloc.argtypes = [P, T, vp]
         lib.pdn_chunk_fwd_host.restype = ctypes.c_int
         lib.pdn_chunk_fwd_host.argtypes = [P, T, T, vp, ctypes.c_size_t, ctypes.c_int, vp]
+        lib.pdn_chunk_transition.restype = ctypes.c_int
+        lib.pdn_chunk_transition.argtypes = [P, T, vp, ctypes.c_size_t, vp]
+        lib.pdn_key_energy.restype = ctypes.c_int
+        lib.pdn_key_energy.argtypes = [P, T, vp]
+        lib.pdn_accumulate.restype = ctypes.c_int
+        lib.pdn_accumulate.argtypes = [ctypes.c_int, ctypes.c_longlong, vp, vp, vp, vp]
+        lib.pdn_state_compose.restype = ctypes.c_int
+        lib.pdn_state_compose.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, vp, vp, vp, vp, vp]
         lib.pdn_decode_step.restype = ctypes.c_int
         lib.pdn_decode_step.argtypes = [P, T, vp]
         lib.pdn_get_device_error.restype = ctypes.c_int
@@ -113,6 +121,26 @@ def pdn_chunk_fwd_profiled(problem: PdnProblem, tensors: PdnTensors, workspace: 
     rc = load().pdn_chunk_fwd_profiled(ctypes.byref(problem), ctypes.byref(tensors), workspace,
                                        ws_bytes, stream, ms, ctypes.byref(n))
     return rc, [float(ms[i]) for i in range(n.value)]
+
+
+def pdn_chunk_transition(problem: PdnProblem, tensors: PdnTensors, workspace: int,
+                         ws_bytes: int, stream: int) -> int:
+    return load().pdn_chunk_transition(ctypes.byref(problem), ctypes.byref(tensors), workspace,
+                                       ws_bytes, stream)
+
+
+def pdn_key_energy(problem: PdnProblem, tensors: PdnTensors, stream: int) -> int:
+    return load().pdn_key_energy(ctypes.byref(problem), ctypes.byref(tensors), stream)
+
+
+def pdn_accumulate(n: int, length: int, parts: int, base: Optional[int], out: int,
+                   stream: int) -> int:
+    return load().pdn_accumulate(n, length, parts, base, out, stream)
+
+
+def pdn_state_compose(BH: int, d_v: int, d_k: int, S_in: Optional[int], A: int,
+                      B_add: Optional[int], S_out: int, stream: int) -> int:
+    return load().pdn_state_compose(BH, d_v, d_k, S_in, A, B_add, S_out, stream)
 
 
 def pdn_chunk_fwd_noalloc(problem: PdnProblem, tensors: PdnTensors, stream: int) -> int:
