@@ -10,6 +10,8 @@ Parity status
 -------------
 * token loop (every variant): pinned by closed forms, brute force and the
   least-squares identity (tests/test_oracle_pins.py);
+* backward (every variant): the analytic reverse-time adjoint, pinned by
+  central finite differences of the token loop on every input;
 * diagonal preconditioner: pinned by its invariants; the page-level constants
   (centring, eps, base of the exponential) are readings of the pages, so the
   match with the original paper is **parity unpinned** for those constants.
@@ -62,6 +64,10 @@ def _load():
         lib.oracle_generic.restype = I
         lib.oracle_generic.argtypes = [I, I, I, I, I, D, D, D, D, D, D, ctypes.c_double,
                                        D, D, I]
+        lib.oracle_backward.restype = I
+        lib.oracle_backward.argtypes = [I, I, I, I, I, I, I, D, D, D, D, D, D, D, D, D,
+                                        ctypes.c_double, ctypes.c_double, ctypes.c_double,
+                                        D, D, D, D, D, D, D, D, D, D, D]
         lib.oracle_precond.restype = I
         lib.oracle_precond.argtypes = [I, I, D, D, ctypes.c_double, ctypes.c_double, D, D]
         _lib = lib
@@ -113,6 +119,38 @@ def forward(variant, q, k, v, log_alpha=None, beta=None, erase=None, write=None,
     if rc != 0:
         raise ValueError("oracle_forward failed with code %d" % rc)
     return o, ST, AT
+
+
+def backward(variant, q, k, v, log_alpha=None, beta=None, erase=None, write=None,
+             S0=None, A0=None, q_scale=1.0, x=1.5, eps=1e-6, dO=None, dST=None):
+    """Gradients of a scalar loss L with dL/do = dO [B,T,H,dv] and
+    dL/dS_T = dST [B,H,dv,dk] (either may be None = 0), through the token loop
+    of ``forward``: a dict with q, k, v, log_alpha, beta, erase, write, S0, A0
+    (None for inputs the variant does not take). Pinned by finite differences."""
+    lib = _load()
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, T, H, dk = k.shape
+    dv = v.shape[3]
+    la, be, er, wr = _f64(log_alpha), _f64(beta), _f64(erase), _f64(write)
+    s0, a0, do, dst = _f64(S0), _f64(A0), _f64(dO), _f64(dST)
+    decay = 0 if la is None else (1 if la.ndim == 3 else 2)
+    g = {"q": np.zeros_like(q), "k": np.zeros_like(k), "v": np.zeros_like(v),
+         "log_alpha": None if la is None else np.zeros_like(la),
+         "beta": None if be is None else np.zeros_like(be),
+         "erase": None if er is None else np.zeros_like(er),
+         "write": None if wr is None else np.zeros_like(wr),
+         "S0": np.zeros((B, H, dv, dk)), "A0": np.zeros((B, H, dk))}
+    rc = lib.oracle_backward(VARIANTS[variant], decay, B, T, H, dk, dv, _ptr(q), _ptr(k), _ptr(v),
+                             _ptr(la), _ptr(be), _ptr(er), _ptr(wr), _ptr(s0), _ptr(a0),
+                             float(q_scale), float(x), float(eps), _ptr(do), _ptr(dst),
+                             _ptr(g["q"]), _ptr(g["k"]), _ptr(g["v"]), _ptr(g["log_alpha"]),
+                             _ptr(g["beta"]), _ptr(g["erase"]), _ptr(g["write"]), _ptr(g["S0"]),
+                             _ptr(g["A0"]))
+    if rc != 0:
+        raise ValueError("oracle_backward failed with code %d" % rc)
+    if variant not in PRECOND_VARIANTS:
+        g["A0"] = None
+    return g
 
 
 def generic(q, r, w, u, log_alpha=None, S0=None, q_scale=1.0, nthreads=0):

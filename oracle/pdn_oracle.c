@@ -357,3 +357,283 @@ int oracle_generic(int B, int T, int H, int dk, int dv, const double *q,
   J.generic = 1;
   return run_job(&J, nthreads);
 }
+
+/* ------------------------------------------------------------------------ */
+/* Backward of the token loop (gradients of a scalar loss L given dL/do_t and
+ * dL/dS_T), fp64. "Gated DeltaNet-2", ja §3, single out the gate-aware
+ * backward: the erase and write gates enter the gradient through the read
+ * and write keys and the target. Written as the reverse-time adjoint of
+ *   P = S_{t-1} D_t,  delta = u - P r,  S_t = P + delta w^T,  o_t = c S_t q'
+ * (q' = q, or B_t . q for PLA):
+ *   dS_t += c do_t q'^T;  dq' = c S_t^T do_t;  ddelta = dS_t w;
+ *   dw = dS_t^T delta;  dr = -P^T ddelta;  du = ddelta;
+ *   dP = dS_t - ddelta r^T;  dalpha_i = sum_j S_{t-1}[j,i] dP[j,i];
+ *   dS_{t-1} = dP D_t,
+ * then each variant's map from (k, v, beta, gates, B_t) to (r, w, u, q') and,
+ * for the preconditioned variants, B_t's dependence on the accumulator
+ * A_t = A_{t-1} + k_t . k_t (through log, centring, squash and x^{-s}).
+ * Pinned by central finite differences of oracle_forward on every input
+ * (tests/test_oracle_pins.py). Outputs may be NULL when not wanted. */
+static void precond_coef_grad(int dk, const double *A, double x, double eps,
+                              const double *dB, double *dA) {
+  /* B_i = x^{-s_i}, s = c/(1+|c|), c_i = L_i - mean(L), L_i = log(A_i + eps) */
+  double mu = 0.0;
+  for (int i = 0; i < dk; ++i) mu += log(A[i] + eps);
+  mu /= (double)dk;
+  const double lnx = log(x);
+  double mean_dc = 0.0;
+  for (int i = 0; i < dk; ++i) {
+    const double c = log(A[i] + eps) - mu;
+    const double s = c / (1.0 + fabs(c));
+    const double B = exp(-s * lnx);
+    const double ds = dB[i] * (-lnx) * B;
+    const double den = 1.0 + fabs(c);
+    dA[i] = ds / (den * den); /* dc, temporarily */
+    mean_dc += dA[i];
+  }
+  mean_dc /= (double)dk;
+  for (int i = 0; i < dk; ++i) dA[i] = (dA[i] - mean_dc) / (A[i] + eps);
+}
+
+typedef struct {
+  job_t *J;
+  const double *dO, *dST;
+  double *dq, *dk, *dv, *dla, *dbeta, *derase, *dwrite, *dS0, *dA0;
+} bjob_t;
+
+static int run_unit_bwd(bjob_t *BJ, int unit) {
+  job_t *J = BJ->J;
+  const int b = unit / J->H, h = unit % J->H;
+  const int dk = J->dk, dv = J->dv, T = J->T, H = J->H;
+  const size_t SS = (size_t)dk * dv;
+  const int pre = uses_precond(J->variant);
+  double *S = (double *)malloc(sizeof(double) * SS * (size_t)(T + 1)); /* S_0 .. S_T */
+  double *Ahist = (double *)malloc(sizeof(double) * (size_t)dk * (size_t)(T + 1));
+  double *Bc = (double *)malloc(sizeof(double) * (size_t)dk * (size_t)(T > 0 ? T : 1));
+  double *dS = (double *)malloc(sizeof(double) * SS);
+  double *dP = (double *)malloc(sizeof(double) * SS);
+  double *dAcc = (double *)calloc((size_t)dk, sizeof(double)); /* sum_{s>=t} dA_s */
+  double *dAt = (double *)malloc(sizeof(double) * (size_t)dk);
+  double *dBt = (double *)malloc(sizeof(double) * (size_t)dk);
+  double *alpha = (double *)malloc(sizeof(double) * (size_t)dk);
+  double *r = (double *)malloc(sizeof(double) * (size_t)dk);
+  double *w = (double *)malloc(sizeof(double) * (size_t)dk);
+  double *u = (double *)malloc(sizeof(double) * (size_t)dv);
+  double *qq = (double *)malloc(sizeof(double) * (size_t)dk);
+  double *delta = (double *)malloc(sizeof(double) * (size_t)dv);
+  double *dd = (double *)malloc(sizeof(double) * (size_t)dv);
+  double *dqq = (double *)malloc(sizeof(double) * (size_t)dk);
+  double *dr = (double *)malloc(sizeof(double) * (size_t)dk);
+  double *dw = (double *)malloc(sizeof(double) * (size_t)dk);
+  if (!S || !Ahist || !Bc || !dS || !dP || !dAcc || !dAt || !dBt || !alpha || !r || !w || !u ||
+      !qq || !delta || !dd || !dqq || !dr || !dw) {
+    free(S); free(Ahist); free(Bc); free(dS); free(dP); free(dAcc); free(dAt); free(dBt);
+    free(alpha); free(r); free(w); free(u); free(qq); free(delta); free(dd); free(dqq);
+    free(dr); free(dw);
+    return 2;
+  }
+  const size_t sidx = ((size_t)b * H + h) * SS;
+  if (J->S0) memcpy(S, J->S0 + sidx, sizeof(double) * SS);
+  else memset(S, 0, sizeof(double) * SS);
+  if (J->A0) memcpy(Ahist, J->A0 + ((size_t)b * H + h) * dk, sizeof(double) * (size_t)dk);
+  else memset(Ahist, 0, sizeof(double) * (size_t)dk);
+
+  /* alpha of token t (per key channel) */
+#define ALPHA_OF(t_)                                                         \
+  do {                                                                       \
+    const size_t th_ = ((size_t)b * T + (t_)) * H + h;                       \
+    for (int i = 0; i < dk; ++i)                                             \
+      alpha[i] = J->decay == OR_DECAY_SCALAR ? exp(J->log_alpha[th_])        \
+                 : J->decay == OR_DECAY_CHANNEL ? exp(J->log_alpha[th_ * dk + i]) \
+                                                : 1.0;                       \
+  } while (0)
+
+  /* forward, keeping every state, accumulator and coefficient */
+  for (int t = 0; t < T; ++t) {
+    const size_t tokh = ((size_t)b * T + t) * H + h;
+    double *A = Ahist + (size_t)(t + 1) * dk;
+    memcpy(A, Ahist + (size_t)t * dk, sizeof(double) * (size_t)dk);
+    if (pre) precond_step(dk, J->k + tokh * dk, A, J->x, J->eps, Bc + (size_t)t * dk);
+    form_vectors(J, tokh, tokh, Bc + (size_t)t * dk, r, w, u);
+    ALPHA_OF(t);
+    memcpy(S + (size_t)(t + 1) * SS, S + (size_t)t * SS, sizeof(double) * SS);
+    token_step(dk, dv, S + (size_t)(t + 1) * SS, alpha, r, w, u, J->q + tokh * dk, 1.0, NULL);
+  }
+
+  /* reverse sweep */
+  if (BJ->dST) memcpy(dS, BJ->dST + sidx, sizeof(double) * SS);
+  else memset(dS, 0, sizeof(double) * SS);
+  const double c = J->q_scale;
+  for (int t = T - 1; t >= 0; --t) {
+    const size_t tokh = ((size_t)b * T + t) * H + h;
+    const double *St = S + (size_t)(t + 1) * SS, *Sp = S + (size_t)t * SS;
+    const double *Bt = Bc + (size_t)t * dk;
+    form_vectors(J, tokh, tokh, Bt, r, w, u);
+    ALPHA_OF(t);
+    const double *qt = J->q + tokh * dk;
+    for (int i = 0; i < dk; ++i) qq[i] = J->variant == OR_PLA ? Bt[i] * qt[i] : qt[i];
+    const double *dot = BJ->dO ? BJ->dO + tokh * dv : NULL;
+    /* output */
+    for (int i = 0; i < dk; ++i) dqq[i] = 0.0;
+    if (dot)
+      for (int j = 0; j < dv; ++j)
+        for (int i = 0; i < dk; ++i) {
+          dS[(size_t)j * dk + i] += c * dot[j] * qq[i];
+          dqq[i] += c * St[(size_t)j * dk + i] * dot[j];
+        }
+    /* delta = u - P r, P = S_{t-1} D */
+    for (int j = 0; j < dv; ++j) {
+      double y = 0.0;
+      for (int i = 0; i < dk; ++i) y += Sp[(size_t)j * dk + i] * alpha[i] * r[i];
+      delta[j] = u[j] - y;
+      double s = 0.0;
+      for (int i = 0; i < dk; ++i) s += dS[(size_t)j * dk + i] * w[i];
+      dd[j] = s;
+    }
+    for (int i = 0; i < dk; ++i) {
+      double sw = 0.0, sr = 0.0, sa = 0.0;
+      for (int j = 0; j < dv; ++j) {
+        const double P = Sp[(size_t)j * dk + i] * alpha[i];
+        const double g = dS[(size_t)j * dk + i] - dd[j] * r[i];
+        dP[(size_t)j * dk + i] = g;
+        sw += dS[(size_t)j * dk + i] * delta[j];
+        sr += P * dd[j];
+        sa += Sp[(size_t)j * dk + i] * g;
+      }
+      dw[i] = sw;
+      dr[i] = -sr;
+      /* dL/dalpha_i = sa; dlog_alpha = alpha * sa */
+      if (BJ->dla) {
+        if (J->decay == OR_DECAY_CHANNEL) BJ->dla[tokh * dk + i] = alpha[i] * sa;
+        else if (J->decay == OR_DECAY_SCALAR) {
+          if (i == 0) BJ->dla[tokh] = 0.0;
+          BJ->dla[tokh] += alpha[i] * sa;
+        }
+      }
+    }
+    for (int j = 0; j < dv; ++j)
+      for (int i = 0; i < dk; ++i) dS[(size_t)j * dk + i] = dP[(size_t)j * dk + i] * alpha[i];
+
+    /* variant maps: (r, w, u, q') -> inputs */
+    const double *kt = J->k + tokh * dk, *vt = J->v + tokh * dv;
+    double *gq = BJ->dq ? BJ->dq + tokh * dk : NULL;
+    double *gk = BJ->dk ? BJ->dk + tokh * dk : NULL;
+    double *gv = BJ->dv ? BJ->dv + tokh * dv : NULL;
+    for (int i = 0; i < dk; ++i) dBt[i] = 0.0;
+    switch (J->variant) {
+    case OR_DN: case OR_GDN: case OR_KDA: {
+      const double be = J->beta[tokh];
+      double db = 0.0;
+      for (int i = 0; i < dk; ++i) {
+        if (gk) gk[i] = dr[i] + be * dw[i];
+        db += kt[i] * dw[i];
+      }
+      if (BJ->dbeta) BJ->dbeta[tokh] = db;
+      if (gv) for (int j = 0; j < dv; ++j) gv[j] = dd[j];
+      if (gq) for (int i = 0; i < dk; ++i) gq[i] = dqq[i];
+    } break;
+    case OR_PDN: case OR_PGDN: case OR_PKDA: {
+      const double be = J->beta[tokh];
+      double db = 0.0;
+      for (int i = 0; i < dk; ++i) {
+        if (gk) gk[i] = dr[i] + be * Bt[i] * dw[i];
+        db += Bt[i] * kt[i] * dw[i];
+        dBt[i] = be * kt[i] * dw[i];
+      }
+      if (BJ->dbeta) BJ->dbeta[tokh] = db;
+      if (gv) for (int j = 0; j < dv; ++j) gv[j] = dd[j];
+      if (gq) for (int i = 0; i < dk; ++i) gq[i] = dqq[i];
+    } break;
+    case OR_PLA: {
+      const double be = J->beta[tokh];
+      double db = 0.0;
+      for (int i = 0; i < dk; ++i) {
+        if (gk) gk[i] = be * dw[i];
+        db += kt[i] * dw[i];
+        dBt[i] = qt[i] * dqq[i];
+        if (gq) gq[i] = Bt[i] * dqq[i];
+      }
+      if (BJ->dbeta) BJ->dbeta[tokh] = db;
+      if (gv) for (int j = 0; j < dv; ++j) gv[j] = dd[j];
+    } break;
+    case OR_FG2: case OR_FG2P: {
+      const double *bk = J->beta + tokh * dk;
+      const double *bv = J->variant == OR_FG2 ? J->beta + tokh * dv : J->write_gate + tokh * dv;
+      for (int i = 0; i < dk; ++i) {
+        const double sb = sqrt(bk[i]);
+        if (gk) gk[i] = sb * (dr[i] + dw[i]);
+        if (BJ->dbeta) BJ->dbeta[tokh * dk + i] = kt[i] * (dr[i] + dw[i]) / (2.0 * sb);
+        if (gq) gq[i] = dqq[i];
+      }
+      for (int j = 0; j < dv; ++j) {
+        const double sv = sqrt(bv[j]);
+        if (gv) gv[j] = sv * dd[j];
+        const double g = vt[j] * dd[j] / (2.0 * sv);
+        if (J->variant == OR_FG2) {
+          if (BJ->dbeta) BJ->dbeta[tokh * dk + j] += g;
+        } else if (BJ->dwrite) {
+          BJ->dwrite[tokh * dv + j] = g;
+        }
+      }
+    } break;
+    case OR_GDN2: {
+      const double *et = J->erase + tokh * dk, *gt = J->write_gate + tokh * dv;
+      for (int i = 0; i < dk; ++i) {
+        if (gk) gk[i] = et[i] * dr[i] + dw[i];
+        if (BJ->derase) BJ->derase[tokh * dk + i] = kt[i] * dr[i];
+        if (gq) gq[i] = dqq[i];
+      }
+      for (int j = 0; j < dv; ++j) {
+        if (gv) gv[j] = gt[j] * dd[j];
+        if (BJ->dwrite) BJ->dwrite[tokh * dv + j] = vt[j] * dd[j];
+      }
+    } break;
+    }
+    /* preconditioner: B_t depends on A_t = A_{t-1} + k_t . k_t, and A_t feeds
+     * every later token: dA_t (total) = dA_t (own coefficient) + dA_{t+1} */
+    if (pre) {
+      precond_coef_grad(dk, Ahist + (size_t)(t + 1) * dk, J->x, J->eps, dBt, dAt);
+      for (int i = 0; i < dk; ++i) {
+        dAcc[i] += dAt[i];
+        if (gk) gk[i] += 2.0 * kt[i] * dAcc[i];
+      }
+    }
+  }
+#undef ALPHA_OF
+  if (BJ->dS0) memcpy(BJ->dS0 + sidx, dS, sizeof(double) * SS);
+  if (BJ->dA0 && pre) memcpy(BJ->dA0 + ((size_t)b * H + h) * dk, dAcc, sizeof(double) * (size_t)dk);
+  free(S); free(Ahist); free(Bc); free(dS); free(dP); free(dAcc); free(dAt); free(dBt);
+  free(alpha); free(r); free(w); free(u); free(qq); free(delta); free(dd); free(dqq);
+  free(dr); free(dw);
+  return 0;
+}
+
+int oracle_backward(int variant, int decay, int B, int T, int H, int dk, int dv,
+                    const double *q, const double *k, const double *v,
+                    const double *log_alpha, const double *beta, const double *erase,
+                    const double *write_gate, const double *S0, const double *A0,
+                    double q_scale, double x, double eps, const double *dO, const double *dST,
+                    double *dq, double *dkk, double *dvv, double *dla, double *dbeta,
+                    double *derase, double *dwrite, double *dS0, double *dA0) {
+  if (B < 0 || T < 0 || H < 0 || dk <= 0 || dv <= 0) return 1;
+  if (variant < OR_DN || variant > OR_FG2P) return 1;
+  if (!q || !k || !v) return 1;
+  if (decay != OR_DECAY_NONE && !log_alpha) return 1;
+  if (variant == OR_GDN2 ? (!erase || !write_gate) : !beta) return 1;
+  if (variant == OR_FG2P && !write_gate) return 1;
+  if (variant == OR_FG2 && dk != dv) return 1;
+  job_t J;
+  memset(&J, 0, sizeof(J));
+  J.variant = variant; J.decay = decay;
+  J.B = B; J.T = T; J.H = H; J.dk = dk; J.dv = dv;
+  J.q = q; J.k = k; J.v = v; J.log_alpha = log_alpha; J.beta = beta;
+  J.erase = erase; J.write_gate = write_gate; J.S0 = S0; J.A0 = A0;
+  J.q_scale = q_scale; J.x = x; J.eps = eps;
+  bjob_t BJ = {&J, dO, dST, dq, dkk, dvv, dla, dbeta, derase, dwrite, dS0, dA0};
+  int err = 0;
+  for (int unit = 0; unit < B * H; ++unit) {
+    const int rc = run_unit_bwd(&BJ, unit);
+    if (rc) err = rc;
+  }
+  return err;
+}

@@ -348,6 +348,50 @@ def test_prologue_apply_selects_by_bits():
     np.testing.assert_array_equal(a["beta"], raw["beta"])
 
 
+# ---------------------------------------------------------------- backward
+def _loss(variant, d, dO, dST, **kw):
+    o, ST, _ = oracle.forward(variant, **d, **kw)
+    return float(np.sum(o * dO) + np.sum(ST * dST))
+
+
+@pytest.mark.parametrize("decay", ["none", "scalar", "channel"])
+@pytest.mark.parametrize("variant", VARIANTS)
+def test_backward_matches_central_differences(variant, decay):
+    """The analytic backward of the token loop equals central finite
+    differences of the forward, on every element of every input (q, k, v, the
+    decay, the gains and gates, S0 and A0), for L = <o, dO> + <S_T, dST>. The
+    gate-aware backward of "Gated DeltaNet-2" (ja §3) is this gradient."""
+    fixed = {"DN": "none", "PDN": "none", "GDN": "scalar", "PGDN": "scalar", "KDA": "channel",
+             "PKDA": "channel"}
+    if variant in fixed and fixed[variant] != decay:
+        pytest.skip("decay fixed by the variant")
+    dk = dv = 4
+    d = rand_inputs(variant, B=1, T=5, H=2, dk=dk, dv=dv, seed=50, decay=decay)
+    if decay != "none":
+        d["log_alpha"] = d["log_alpha"] * 3.0  # stronger decay
+    if variant in ("PDN", "PGDN", "PKDA", "PLA"):
+        d["A0"] = np.random.default_rng(51).uniform(0.2, 1.0, (1, 2, dk))
+    rng = np.random.default_rng(52)
+    dO = rng.standard_normal(d["v"].shape)
+    dST = rng.standard_normal(d["S0"].shape)
+    kw = dict(q_scale=0.8, x=1.5)
+    g = oracle.backward(variant, **d, dO=dO, dST=dST, **kw)
+    h = 1e-6
+    for name, arr in d.items():
+        ga = g[name]
+        assert ga is not None and ga.shape == arr.shape, name
+        num = np.zeros_like(arr)
+        for idx in np.ndindex(arr.shape):
+            x0 = arr[idx]
+            arr[idx] = x0 + h
+            lp = _loss(variant, d, dO, dST, **kw)
+            arr[idx] = x0 - h
+            lm = _loss(variant, d, dO, dST, **kw)
+            arr[idx] = x0
+            num[idx] = (lp - lm) / (2 * h)
+        np.testing.assert_allclose(ga, num, rtol=2e-6, atol=2e-7, err_msg=name)
+
+
 # ---------------------------------------------------------------- P7
 @pytest.mark.parametrize("lam", [0.5, 2.0])
 def test_p7_exact_preconditioning_is_least_squares(lam):
