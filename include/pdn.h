@@ -280,6 +280,45 @@ pdn_status_t pdn_accumulate(int n, long long len, const float *parts, const floa
  * and A0 == AT (non-NULL for PDN/PGDN/PKDA, NULL otherwise). */
 pdn_status_t pdn_decode_step(const pdn_problem_t *p, const pdn_tensors_t *t, void *stream);
 
+/* ---- Backward ("Gated DeltaNet-2", ja §3, the gate-aware backward) ------
+ * Gradient of pdn_chunk_fwd's outputs (o, ST) with respect to its inputs,
+ * for every variant and decay. Reverse mode of the token recurrence: two
+ * sweeps over the state rows (delta_t forward, d delta_t backward), two over
+ * the key columns (dq', dr forward, dw backward), a suffix sum over tokens
+ * for the decay and the preconditioner, and per-token chain rules (the erase
+ * and write gates receive k . dr and v . du). fp32 arithmetic on CUDA cores;
+ * no per-token state is stored. Gradients are fp32, laid out like the inputs
+ * they belong to; every pointer may be NULL (that gradient is not written)
+ * except that a gradient must be NULL when its input is (dlog_alpha for
+ * decay NONE, dbeta for GDN2, derase except for GDN2, dwrite except for GDN2
+ * and FG2_GDN_PLUS, dA0 except for the preconditioned variants). Each
+ * tensor is 16-byte aligned (4 bytes for the fp32 [B,T,H] ones). */
+typedef struct {
+  const void *dO;     /* cotangent of o: dtype [B,T,H,d_v]; NULL = zeros       */
+  const float *dST;   /* cotangent of ST: [B,H,d_v,d_k]; NULL = zeros          */
+  float *dq, *dk;     /* [B,T,H,d_k]                                          */
+  float *dv;          /* [B,T,H,d_v]                                          */
+  float *dlog_alpha;  /* [B,T,H] (SCALAR) or [B,T,H,d_k] (CHANNEL)            */
+  float *dbeta;       /* [B,T,H], or [B,T,H,d_k] for FG2_GDN / FG2_GDN_PLUS     */
+  float *derase;      /* GDN2: [B,T,H,d_k]                                    */
+  float *dwrite;      /* GDN2 / FG2_GDN_PLUS: [B,T,H,d_v]                      */
+  float *dS0;         /* [B,H,d_v,d_k]                                        */
+  float *dA0;         /* preconditioned variants: [B,H,d_k]                   */
+} pdn_grads_t;
+
+/* Bytes of workspace pdn_chunk_bwd needs ((size_t)-1 if p is invalid). */
+size_t pdn_chunk_bwd_workspace(const pdn_problem_t *p);
+
+/* Backward of pdn_chunk_fwd for problem p and forward inputs t (q, k, v,
+ * log_alpha, beta, erase, write, S0, A0 as given to the forward; o, ST and
+ * AT are not used and may be NULL). p->chunk and p->impl are validated as
+ * for the forward but do not change the result; p->prologue must be 0 (PDN_ERR_UNSUPPORTED otherwise: the activations'
+ * derivatives are the caller's). The gradients overwrite the buffers in g.
+ * `workspace`: 256-byte aligned, at least pdn_chunk_bwd_workspace(p) bytes.
+ * Returns PDN_OK once the work is enqueued on `stream`. */
+pdn_status_t pdn_chunk_bwd(const pdn_problem_t *p, const pdn_tensors_t *t, const pdn_grads_t *g,
+                           void *workspace, size_t ws_bytes, void *stream);
+
 /* Synchronises `stream`, returns the first device-side error recorded on the
  * current device since the last call (PDN_OK if none) and clears it. */
 pdn_status_t pdn_get_device_error(void *stream);

@@ -80,7 +80,7 @@ pdn_status_t check_problem(const pdn_problem_t *p) {
   return PDN_OK;
 }
 
-pdn_status_t check_tensors(const pdn_problem_t *p, const pdn_tensors_t *t) {
+pdn_status_t check_tensors(const pdn_problem_t *p, const pdn_tensors_t *t, bool need_o = true) {
   if (!t) return PDN_ERR_INVALID_ARG;
   // 16-byte alignment for every tensor the kernels read or write in 16-byte
   // vectors; the fp32 per-(token, head) gates (scalar log decay, scalar beta)
@@ -98,7 +98,7 @@ pdn_status_t check_tensors(const pdn_problem_t *p, const pdn_tensors_t *t) {
   if (p->T == 0) {
     if (p->variant == PDN_VAR_GDN2 && t->beta) return PDN_ERR_INVALID_ARG;
   } else {
-    if (!t->q || !t->k || !t->v || !t->o) return PDN_ERR_INVALID_ARG;
+    if (!t->q || !t->k || !t->v || (need_o && !t->o)) return PDN_ERR_INVALID_ARG;
     if ((p->decay == PDN_DECAY_NONE) != (t->log_alpha == nullptr)) return PDN_ERR_INVALID_ARG;
     if (p->variant == PDN_VAR_GDN2) {
       if (t->beta || !t->erase || !t->write) return PDN_ERR_INVALID_ARG;
@@ -165,6 +165,35 @@ pdn_status_t check_chunk_fwd(const pdn_problem_t *p, const pdn_tensors_t *t,
   return PDN_OK;
 }
 
+// Everything pdn_chunk_bwd checks before it enqueues work (host-only).
+pdn_status_t check_chunk_bwd(const pdn_problem_t *p, const pdn_tensors_t *t, const pdn_grads_t *g,
+                             const void *workspace, size_t ws_bytes) {
+  pdn_status_t st = check_problem(p);
+  if (st != PDN_OK) return st;
+  if ((st = check_tensors(p, t, false)) != PDN_OK) return st;
+  if (!g) return PDN_ERR_INVALID_ARG;
+  if (p->prologue != 0) return PDN_ERR_UNSUPPORTED;
+  const bool scalar_la = p->decay == PDN_DECAY_SCALAR;
+  const bool scalar_beta = has_scalar_beta(p->variant);
+  const void *v16[] = {g->dO, g->dST, g->dq, g->dk, g->dv, g->derase, g->dwrite, g->dS0, g->dA0,
+                       scalar_la ? nullptr : g->dlog_alpha, scalar_beta ? nullptr : g->dbeta};
+  for (const void *ptr : v16)
+    if (ptr && !aligned(ptr, 16)) return PDN_ERR_INVALID_ARG;
+  if (scalar_la && g->dlog_alpha && !aligned(g->dlog_alpha, 4)) return PDN_ERR_INVALID_ARG;
+  if (scalar_beta && g->dbeta && !aligned(g->dbeta, 4)) return PDN_ERR_INVALID_ARG;
+  // a gradient only where the forward has the input
+  if (p->decay == PDN_DECAY_NONE && g->dlog_alpha) return PDN_ERR_INVALID_ARG;
+  if (p->variant == PDN_VAR_GDN2 && g->dbeta) return PDN_ERR_INVALID_ARG;
+  if (p->variant != PDN_VAR_GDN2 && g->derase) return PDN_ERR_INVALID_ARG;
+  if (p->variant != PDN_VAR_GDN2 && p->variant != PDN_VAR_FG2_GDN_PLUS && g->dwrite)
+    return PDN_ERR_INVALID_ARG;
+  if (!is_precond(p->variant) && g->dA0) return PDN_ERR_INVALID_ARG;
+  const KParams P = make_params(p, t, nullptr);
+  if (p->T > 0 && (!workspace || ws_bytes < bwd_workspace_bytes(P) || ((uintptr_t)workspace & 255u)))
+    return PDN_ERR_WORKSPACE;
+  return PDN_OK;
+}
+
 }  // namespace pdn
 
 using namespace pdn;
@@ -199,6 +228,26 @@ extern "C" pdn_status_t pdn_chunk_fwd(const pdn_problem_t *p, const pdn_tensors_
   if (impl == PDN_IMPL_TC) e = launch_chunk_split(P, workspace, s);
   else e = launch_chunk_simt(P, s);
   return e == cudaSuccess ? PDN_OK : PDN_ERR_CUDA;
+}
+
+extern "C" size_t pdn_chunk_bwd_workspace(const pdn_problem_t *p) {
+  if (check_problem(p) != PDN_OK) return (size_t)-1;
+  pdn_tensors_t dummy;
+  memset(&dummy, 0, sizeof(dummy));
+  return p->T == 0 ? 0 : bwd_workspace_bytes(make_params(p, &dummy, nullptr));
+}
+
+extern "C" pdn_status_t pdn_chunk_bwd(const pdn_problem_t *p, const pdn_tensors_t *t,
+                                      const pdn_grads_t *g, void *workspace, size_t ws_bytes,
+                                      void *stream) {
+  const pdn_status_t st = check_chunk_bwd(p, t, g, workspace, ws_bytes);
+  if (st != PDN_OK) return st;
+  KParams P = make_params(p, t, nullptr);
+  P.err = device_error_word();
+  if (!P.err) return PDN_ERR_CUDA;
+  return launch_chunk_bwd(P, g, workspace, static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? PDN_OK
+             : PDN_ERR_CUDA;
 }
 
 extern "C" pdn_status_t pdn_chunk_fwd_profiled(const pdn_problem_t *p, const pdn_tensors_t *t,

@@ -1,0 +1,994 @@
+// backward.cu -- gradient of the chunked forward ("Gated DeltaNet-2", ja §3:
+// the gate-aware backward; the erase and write gates enter the gradient
+// through the read key, the write key and the target).
+//
+// Generic token step (every variant; r read key, w write key, u target,
+// alpha the decay, q' the read-out query, c = q_scale):
+//   P_t = S_{t-1} Diag(alpha_t),  delta_t = u_t - P_t r_t,
+//   S_t = P_t + delta_t w_t^T,    o_t = c S_t q'_t.
+// Reverse mode, with dS~_t the total cotangent of S_t:
+//   dS~_t = dS_t + c dO_t q'_t^T,  dd_t = dS~_t w_t        (= d delta = du)
+//   dw_t = dS~_t^T delta_t,        dr_t = -P_t^T dd_t,      dq'_t = c S_t^T dO_t
+//   dS_{t-1} = (dS~_t - dd_t r_t^T) Diag(alpha_t).
+// Every row of S and of dS evolves on its own; only the read-outs mix rows.
+// The work is split so that no per-token state is ever stored:
+//   F1  forward, warp per state row:  delta_t (a row reduction per token)
+//   R1  reverse, warp per state row:  dd_t, dS0
+//   F2  forward, thread per key column, delta given: dq'_t and dr_t
+//   R2  reverse, thread per key column, dd given:    dw_t
+// F2 and R2 have no reduction on their sequential path (a gated linear
+// attention pass each); their column sums over a CTA's rows are written per
+// row group and added in the epilogue.
+//
+// The decay gradient needs no state either. With psi_t,i = sum_j P_t[j,i]
+// dP_t[j,i] (the cotangent of log alpha_t,i), expanding S_t = P_t + delta_t
+// w_t^T and dS~_t gives psi_t = psi_{t+1} + q'_t.dq'_t - w_t.dw_t + r_t.dr_t
+// (elementwise), started from psi_T,i = sum_j S_T[j,i] dS_T[j,i]: a suffix
+// sum over tokens. A scalar decay takes sum_i psi_t,i.
+//
+// The preconditioner's coefficients B_t depend on A_t = A_{t-1} + k_t.k_t
+// ("Preconditioned DeltaNet", ja §2.2); each token's dB_t gives a dA_t, and
+// A_t feeds every later token, so k_t receives 2 k_t (sum_{s>=t} dA_s).
+//
+// All arithmetic is fp32; inputs of either dtype are widened on load and
+// every gradient is written in fp32.
+#include <string.h>
+
+#include "common.cuh"
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace pdn {
+
+// Workspace plan (floats), shared by the size query and the launcher.
+struct BwdPlan {
+  int GS;          // floats per (token, head) of the generic vectors: q'|r|w|a|u
+  int R, G;        // rows per CTA of F2/R2, row groups (d_v / R)
+  int nb;          // scan blocks per sequence
+  size_t gen, acc, delta, dd, st, part, cpsi, sigma, dacc, bsum, phi, total;
+};
+
+namespace {
+
+constexpr int kScanBlk = 64;     // tokens per scan block
+constexpr int kRowsF = 16;       // state rows per CTA of F1 / R1 (4 warps x 4)
+constexpr int kLC = 16;          // tokens staged per chunk in F1 / R1 / F2 / R2
+
+size_t up64(size_t n) { return (n + 63) & ~(size_t)63; }
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+}  // namespace
+
+static BwdPlan bwd_plan(const KParams &P) {
+  BwdPlan L;
+  memset(&L, 0, sizeof(L));
+  const size_t BH = (size_t)P.B * P.H, T = (size_t)P.T;
+  const int dk = P.dk, dv = P.dv;
+  L.GS = 4 * dk + dv;
+  const long long rows32 = (long long)BH * (dv / 32);
+  L.R = (dv % 32 == 0 && rows32 >= 2 * 148) ? 32 : 16;
+  L.G = dv / L.R;
+  L.nb = (int)((T + kScanBlk - 1) / kScanBlk);
+  size_t off = 0;
+  auto take = [&](size_t n) { const size_t o = off; off += up64(n); return o; };
+  L.gen = take(BH * T * L.GS);
+  L.acc = take(is_precond(P.variant) ? BH * T * dk : 0);
+  L.delta = take(BH * T * dv);
+  L.dd = take(BH * T * dv);
+  L.st = take(BH * dv * dk);
+  L.part = take((size_t)L.G * BH * T * 3 * dk);
+  L.cpsi = take(P.decay == PDN_DECAY_CHANNEL ? BH * T * dk : 0);
+  L.sigma = take(P.decay == PDN_DECAY_SCALAR ? BH * T : 0);
+  L.dacc = take(is_precond(P.variant) ? BH * T * dk : 0);
+  L.bsum = take(BH * (size_t)L.nb * dk);
+  L.phi = take(BH * dk + BH);
+  L.total = off;
+  return L;
+}
+
+namespace {
+
+// Everything the backward kernels read and write, by value.
+struct BParams {
+  KParams P;
+  const void *dO;     // dtype [B,T,H,dv] or NULL
+  const float *dST;   // [B,H,dv,dk] or NULL
+  float *dq, *dk, *dv, *dla, *dbeta, *derase, *dwrite, *dS0, *dA0;
+  float *gen, *acc, *delta, *dd, *st, *part, *cpsi, *sigma, *dacc, *bsum, *phi;
+  int GS, R, G, nb;
+};
+
+// Generic vectors of one token, in the workspace order q'|r|w|a|u.
+__device__ __forceinline__ float *gen_at(const BParams &Q, int bh, int t) {
+  return Q.gen + ((size_t)bh * Q.P.T + t) * Q.GS;
+}
+
+// ---------------------------------------------------------------------------
+// Suffix / prefix sums over tokens, per (batch, head, channel), in three
+// passes: block totals, the carry into each block, the sums inside blocks.
+// A tensor is addressed either as workspace [BH][T][nch] (tok = false) or as
+// a [B,T,H,nch] tensor (tok = true).
+struct ScanArr {
+  float *p;
+  bool tok;
+};
+__device__ __forceinline__ size_t scan_off(const KParams &P, const ScanArr &a, int nch, int bh,
+                                           int t, int c) {
+  if (a.tok) return tok_index(P, bh / P.H, t, bh % P.H) * nch + c;
+  return ((size_t)bh * P.T + t) * nch + c;
+}
+
+__global__ void scan_part_kernel(const KParams P, ScanArr X, int nch, int nb, float *bsum) {
+  const long long n = (long long)P.B * P.H * nb * nch;
+  for (long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x; e < n;
+       e += (long long)gridDim.x * blockDim.x) {
+    const int c = (int)(e % nch);
+    const long long r = e / nch;
+    const int blk = (int)(r % nb), bh = (int)(r / nb);
+    const int t0 = blk * kScanBlk, t1 = min(P.T, t0 + kScanBlk);
+    float s = 0.f;
+#pragma unroll 8
+    for (int t = t0; t < t1; ++t) s += X.p[scan_off(P, X, nch, bh, t, c)];
+    bsum[e] = s;
+  }
+}
+
+// Replaces each block total by the sum carried into that block (from the
+// sequence start when !rev, from its end when rev), seeded with init
+// ([BH][nch], may be NULL). total (may be NULL) gets the full sum + init.
+__global__ void scan_carry_kernel(const KParams P, int nch, int nb, bool rev, float *bsum,
+                                  const float *init, float *total) {
+  const long long n = (long long)P.B * P.H * nch;
+  for (long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x; e < n;
+       e += (long long)gridDim.x * blockDim.x) {
+    const int c = (int)(e % nch), bh = (int)(e / nch);
+    float carry = init ? init[e] : 0.f;
+    for (int k = 0; k < nb; ++k) {
+      const int blk = rev ? nb - 1 - k : k;
+      float *p = bsum + ((size_t)bh * nb + blk) * nch + c;
+      const float s = *p;
+      *p = carry;
+      carry += s;
+    }
+    if (total) total[e] = carry;
+  }
+}
+
+// Y_t = carry + inclusive sum of X inside the block (Y may alias X).
+__global__ void scan_fill_kernel(const KParams P, ScanArr X, ScanArr Y, int nch, int nb, bool rev,
+                                 const float *bsum) {
+  const long long n = (long long)P.B * P.H * nb * nch;
+  for (long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x; e < n;
+       e += (long long)gridDim.x * blockDim.x) {
+    const int c = (int)(e % nch);
+    const long long r = e / nch;
+    const int blk = (int)(r % nb), bh = (int)(r / nb);
+    const int t0 = blk * kScanBlk, t1 = min(P.T, t0 + kScanBlk);
+    float y = bsum[e];
+    if (!rev) {
+      for (int t = t0; t < t1; ++t) {
+        y += X.p[scan_off(P, X, nch, bh, t, c)];
+        Y.p[scan_off(P, Y, nch, bh, t, c)] = y;
+      }
+    } else {
+      for (int t = t1 - 1; t >= t0; --t) {
+        y += X.p[scan_off(P, X, nch, bh, t, c)];
+        Y.p[scan_off(P, Y, nch, bh, t, c)] = y;
+      }
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Prep. acc[bh][t][i] = k_{t,i}^2 (preconditioned variants; the prefix sum
+// over tokens then makes it A_t).
+template <typename Tin>
+__global__ void prep_sq_kernel(const BParams Q) {
+  const KParams &P = Q.P;
+  const int dk = P.dk;
+  const long long n = (long long)P.B * P.H * P.T * dk;
+  for (long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x; e < n;
+       e += (long long)gridDim.x * blockDim.x) {
+    const int i = (int)(e % dk);
+    const long long r = e / dk;
+    const int t = (int)(r % P.T), bh = (int)(r / P.T);
+    const float k = ldf<Tin>(P.k, tok_index(P, bh / P.H, t, bh % P.H) * dk + i);
+    Q.acc[e] = k * k;
+  }
+}
+
+// The variant's (q', r, w, alpha, u) of every token, one warp per (token,
+// head); lane l holds channels 4l..4l+3 of the key side and of the value side.
+// Variant table: DN/GDN/KDA r = k, w = beta k, u = v; PDN/PGDN/PKDA w = beta
+// (B_t . k); FG2-GDN r = w = sqrt(beta) . k, u = sqrt(beta) . v; GDN-2 r = e . k,
+// w = k, u = g . v; PLA r = 0, w = beta k, q' = B_t . q; FG2-GDN+ r = w =
+// sqrt(beta_k) . k, u = sqrt(beta_v) . v.
+template <typename Tin>
+__global__ void prep_gen_kernel(const BParams Q) {
+  const KParams &P = Q.P;
+  const int lane = threadIdx.x & 31, dk = P.dk, dv = P.dv;
+  const long long n = (long long)P.B * P.H * P.T;
+  const long long nw = ((long long)gridDim.x * blockDim.x) >> 5;
+  for (long long wid = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5; wid < n; wid += nw) {
+    const int bh = (int)(wid / P.T), t = (int)(wid % P.T);
+    const size_t tk = tok_index(P, bh / P.H, t, bh % P.H);
+    const int c = 4 * lane;
+    const bool ak = c < dk, av = c < dv;
+    float k[4], q[4], v[4], Bc[4], a[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      k[e] = ak ? ldf<Tin>(P.k, tk * dk + c + e) : 0.f;
+      q[e] = ak ? ldf<Tin>(P.q, tk * dk + c + e) : 0.f;
+      v[e] = av ? ldf<Tin>(P.v, tk * dv + c + e) : 0.f;
+      Bc[e] = 1.f;
+      a[e] = 1.f;
+    }
+    if (is_precond(P.variant)) {
+      const float *A = Q.acc + ((size_t)bh * P.T + t) * dk;
+      float L[4], s = 0.f;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        L[e] = ak ? logf(A[c + e] + P.eps) : 0.f;
+        s += L[e];
+      }
+      const float mu = warp_sum(s) / (float)dk;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) Bc[e] = precond_coef(L[e], mu, P.lnx);
+    }
+    if (P.decay == PDN_DECAY_SCALAR) {
+      const float ea = expf(reinterpret_cast<const float *>(P.log_alpha)[tk]);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) a[e] = ea;
+    } else if (P.decay == PDN_DECAY_CHANNEL) {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) a[e] = ak ? expf(ldf<Tin>(P.log_alpha, tk * dk + c + e)) : 1.f;
+    }
+    float r[4], w[4], u[4], qq[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      r[e] = k[e];
+      w[e] = k[e];
+      u[e] = v[e];
+      qq[e] = q[e];
+    }
+    switch (P.variant) {
+      case PDN_VAR_DN: case PDN_VAR_GDN: case PDN_VAR_KDA: {
+        const float be = reinterpret_cast<const float *>(P.beta)[tk];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) w[e] = be * k[e];
+      } break;
+      case PDN_VAR_PDN: case PDN_VAR_PGDN: case PDN_VAR_PKDA: {
+        const float be = reinterpret_cast<const float *>(P.beta)[tk];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) w[e] = be * Bc[e] * k[e];
+      } break;
+      case PDN_VAR_PLA: {
+        const float be = reinterpret_cast<const float *>(P.beta)[tk];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          r[e] = 0.f;
+          w[e] = be * k[e];
+          qq[e] = Bc[e] * q[e];
+        }
+      } break;
+      case PDN_VAR_FG2_GDN: case PDN_VAR_FG2_GDN_PLUS: {
+        const bool plus = P.variant == PDN_VAR_FG2_GDN_PLUS;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float sb = ak ? sqrtf(ldf<Tin>(P.beta, tk * dk + c + e)) : 0.f;
+          r[e] = sb * k[e];
+          w[e] = sb * k[e];
+          const float bv = av ? (plus ? ldf<Tin>(P.write, tk * dv + c + e)
+                                      : ldf<Tin>(P.beta, tk * dk + c + e))
+                              : 0.f;
+          u[e] = sqrtf(bv) * v[e];
+        }
+      } break;
+      case PDN_VAR_GDN2: {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          r[e] = ak ? ldf<Tin>(P.erase, tk * dk + c + e) * k[e] : 0.f;
+          u[e] = av ? ldf<Tin>(P.write, tk * dv + c + e) * v[e] : 0.f;
+        }
+      } break;
+      default: break;
+    }
+    float *g = gen_at(Q, bh, t);
+    if (ak) {
+      *reinterpret_cast<float4 *>(g + c) = make_float4(qq[0], qq[1], qq[2], qq[3]);
+      *reinterpret_cast<float4 *>(g + dk + c) = make_float4(r[0], r[1], r[2], r[3]);
+      *reinterpret_cast<float4 *>(g + 2 * dk + c) = make_float4(w[0], w[1], w[2], w[3]);
+      *reinterpret_cast<float4 *>(g + 3 * dk + c) = make_float4(a[0], a[1], a[2], a[3]);
+    }
+    if (av) *reinterpret_cast<float4 *>(g + 4 * dk + c) = make_float4(u[0], u[1], u[2], u[3]);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Row sweeps F1 / R1. CTA = 4 warps = 16 consecutive state rows of one (batch,
+// head); warp w owns rows j0 + 4w .. j0 + 4w + 3 and lane l key channels
+// 4l..4l+3, so a row's reduction over key channels stays inside its warp.
+// The per-token vectors are staged through shared memory kLC tokens at a
+// time with cp.async, double-buffered.
+
+// Sums each of the four rows' partials over the warp; every lane gets all
+// four sums. Rows are transposed across lane halves and quarters first, so
+// the four sums take 10 shuffles instead of 20 (fixed order: deterministic).
+__device__ __forceinline__ void rowsum4(const float (&p)[4], float (&y)[4], int lane) {
+  const bool h16 = lane & 16, h8 = lane & 8;
+  float a0 = h16 ? p[2] : p[0], a1 = h16 ? p[3] : p[1];
+  const float b0 = h16 ? p[0] : p[2], b1 = h16 ? p[1] : p[3];
+  a0 += __shfl_xor_sync(0xffffffffu, b0, 16);
+  a1 += __shfl_xor_sync(0xffffffffu, b1, 16);
+  float k = h8 ? a1 : a0;
+  const float s = h8 ? a0 : a1;
+  k += __shfl_xor_sync(0xffffffffu, s, 8);
+  k += __shfl_xor_sync(0xffffffffu, k, 4);
+  k += __shfl_xor_sync(0xffffffffu, k, 2);
+  k += __shfl_xor_sync(0xffffffffu, k, 1);
+  // lane holds row 2 * h16 + h8, i.e. row m sits in lane 8m
+#pragma unroll
+  for (int m = 0; m < 4; ++m) y[m] = __shfl_sync(0xffffffffu, k, 8 * m);
+}
+
+__device__ __forceinline__ float pick4(const float (&v)[4], int i) {
+  return i == 0 ? v[0] : i == 1 ? v[1] : i == 2 ? v[2] : v[3];
+}
+__device__ __forceinline__ void ld4(const float *p, bool ok, float (&v)[4]) {
+  const float4 x = ok ? *reinterpret_cast<const float4 *>(p) : make_float4(0.f, 0.f, 0.f, 0.f);
+  v[0] = x.x; v[1] = x.y; v[2] = x.z; v[3] = x.w;
+}
+
+// F1: the forward recurrence, writing delta_t of every row, and S_T.
+__global__ void __launch_bounds__(128) f1_kernel(const BParams Q) {
+  extern __shared__ float4 smem4[];
+  float *sm = reinterpret_cast<float *>(smem4);
+  const KParams &P = Q.P;
+  const int dk = P.dk, dv = P.dv, T = P.T;
+  const int nrg = dv / kRowsF;
+  const int bh = blockIdx.x / nrg, j0 = (blockIdx.x % nrg) * kRowsF;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, c = 4 * lane;
+  const bool act = c < dk;
+  const int TS = 3 * dk + 16;  // staged floats per token: r | w | alpha | u of the 16 rows
+  const int nv = 3 * dk / 4;   // 16-byte copies of the vectors per token
+  const int nc = (T + kLC - 1) / kLC;
+  auto issue = [&](int ch) {
+    float *buf = sm + (ch & 1) * kLC * TS;
+    const int t0 = ch * kLC, n = min(kLC, T - t0), per = nv + 4;
+    for (int e = threadIdx.x; e < n * per; e += blockDim.x) {
+      const int tt = e / per, k = e % per;
+      const float *g = gen_at(Q, bh, t0 + tt);
+      const float *src = k < nv ? g + dk + 4 * k : g + 4 * dk + j0 + 4 * (k - nv);
+      cp_async16(smem_u32(buf + tt * TS + 4 * k), src, true);
+    }
+  };
+  float S[4][4];
+#pragma unroll
+  for (int m = 0; m < 4; ++m)
+    ld4(P.S0 ? P.S0 + ((size_t)bh * dv + j0 + 4 * warp + m) * dk + c : nullptr, act && P.S0, S[m]);
+  issue(0);
+  cp_async_commit();
+  for (int ch = 0; ch < nc; ++ch) {
+    if (ch + 1 < nc) issue(ch + 1);
+    cp_async_commit();
+    cp_async_wait_group<1>();
+    __syncthreads();
+    const float *buf = sm + (ch & 1) * kLC * TS;
+    const int t0 = ch * kLC, n = min(kLC, T - t0);
+    for (int tt = 0; tt < n; ++tt) {
+      const float *sv = buf + tt * TS;
+      float r[4], w[4], a[4], u[4], p[4], y[4], d[4];
+      ld4(sv + c, act, r);
+      ld4(sv + dk + c, act, w);
+      ld4(sv + 2 * dk + c, act, a);
+      ld4(sv + 3 * dk + 4 * warp, true, u);
+#pragma unroll
+      for (int m = 0; m < 4; ++m) {
+        p[m] = 0.f;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          S[m][e] *= a[e];
+          p[m] = fmaf(S[m][e], r[e], p[m]);
+        }
+      }
+      rowsum4(p, y, lane);
+#pragma unroll
+      for (int m = 0; m < 4; ++m) {
+        d[m] = u[m] - y[m];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) S[m][e] = fmaf(d[m], w[e], S[m][e]);
+      }
+      if (lane < 4)
+        Q.delta[((size_t)bh * T + t0 + tt) * dv + j0 + 4 * warp + lane] = pick4(d, lane);
+    }
+    __syncthreads();  // the buffer is refilled two chunks on
+  }
+  if (act) {
+#pragma unroll
+    for (int m = 0; m < 4; ++m)
+      *reinterpret_cast<float4 *>(Q.st + ((size_t)bh * dv + j0 + 4 * warp + m) * dk + c) =
+          make_float4(S[m][0], S[m][1], S[m][2], S[m][3]);
+  }
+}
+
+// The four dO entries of rows j..j+3 of a staged token, widened to fp32.
+template <typename Tin>
+__device__ __forceinline__ void ld_rows4(const float *sv, int j, float (&v)[4]);
+template <>
+__device__ __forceinline__ void ld_rows4<float>(const float *sv, int j, float (&v)[4]) {
+  const float4 x = *reinterpret_cast<const float4 *>(sv + j);
+  v[0] = x.x; v[1] = x.y; v[2] = x.z; v[3] = x.w;
+}
+template <>
+__device__ __forceinline__ void ld_rows4<__nv_bfloat16>(const float *sv, int j, float (&v)[4]) {
+  const uint2 x = *reinterpret_cast<const uint2 *>(reinterpret_cast<const __nv_bfloat16 *>(sv) + j);
+  v[0] = __uint_as_float(x.x << 16); v[1] = __uint_as_float(x.x & 0xffff0000u);
+  v[2] = __uint_as_float(x.y << 16); v[3] = __uint_as_float(x.y & 0xffff0000u);
+}
+
+// Stages the dO entries of rows j0 .. j0 + nrow - 1 of token t (raw dtype) at
+// dst; `part` selects one 16-byte piece.
+template <typename Tin>
+__device__ __forceinline__ void stage_dO(const BParams &Q, int bh, int t, int j0, int part,
+                                         float *dst) {
+  const KParams &P = Q.P;
+  const char *src = reinterpret_cast<const char *>(Q.dO) +
+                    (tok_index(P, bh / P.H, t, bh % P.H) * P.dv + j0) * sizeof(Tin) + 16 * part;
+  cp_async16(smem_u32(reinterpret_cast<char *>(dst) + 16 * part), src, true);
+}
+
+// R1: the reverse recurrence of the cotangent, writing dd_t of every row, and
+// dS0.
+template <typename Tin>
+__global__ void __launch_bounds__(128) r1_kernel(const BParams Q) {
+  extern __shared__ float4 smem4[];
+  float *sm = reinterpret_cast<float *>(smem4);
+  const KParams &P = Q.P;
+  const int dk = P.dk, dv = P.dv, T = P.T;
+  const int nrg = dv / kRowsF;
+  const int bh = blockIdx.x / nrg, j0 = (blockIdx.x % nrg) * kRowsF;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, c = 4 * lane;
+  const bool act = c < dk;
+  const float cq = P.q_scale;
+  const int TS = 4 * dk + 16;  // staged floats per token: q' | r | w | alpha | dO of the 16 rows
+  const int nv = dk;           // 16-byte copies of the vectors per token
+  const int nd = Q.dO ? kRowsF * (int)sizeof(Tin) / 16 : 0;
+  const int nc = (T + kLC - 1) / kLC;
+  auto issue = [&](int ch) {
+    float *buf = sm + (ch & 1) * kLC * TS;
+    const int t0 = ch * kLC, n = min(kLC, T - t0), per = nv + nd;
+    for (int e = threadIdx.x; e < n * per; e += blockDim.x) {
+      const int tt = e / per, k = e % per;
+      if (k < nv)
+        cp_async16(smem_u32(buf + tt * TS + 4 * k), gen_at(Q, bh, t0 + tt) + 4 * k, true);
+      else
+        stage_dO<Tin>(Q, bh, t0 + tt, j0, k - nv, buf + tt * TS + 4 * dk);
+    }
+  };
+  float D[4][4];
+#pragma unroll
+  for (int m = 0; m < 4; ++m)
+    ld4(Q.dST ? Q.dST + ((size_t)bh * dv + j0 + 4 * warp + m) * dk + c : nullptr, act && Q.dST,
+        D[m]);
+  if (nc > 0) issue(nc - 1);
+  cp_async_commit();
+  for (int ch = nc - 1; ch >= 0; --ch) {
+    if (ch > 0) issue(ch - 1);
+    cp_async_commit();
+    cp_async_wait_group<1>();
+    __syncthreads();
+    const float *buf = sm + (ch & 1) * kLC * TS;
+    const int t0 = ch * kLC, n = min(kLC, T - t0);
+    for (int tt = n - 1; tt >= 0; --tt) {
+      const float *sv = buf + tt * TS;
+      float q[4], r[4], w[4], a[4], g[4], p[4], dd[4];
+      ld4(sv + c, act, q);
+      ld4(sv + dk + c, act, r);
+      ld4(sv + 2 * dk + c, act, w);
+      ld4(sv + 3 * dk + c, act, a);
+      if (Q.dO) {
+        ld_rows4<Tin>(sv + 4 * dk, 4 * warp, g);
+      } else {
+        g[0] = g[1] = g[2] = g[3] = 0.f;
+      }
+#pragma unroll
+      for (int m = 0; m < 4; ++m) {
+        const float cg = cq * g[m];
+        p[m] = 0.f;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          D[m][e] = fmaf(cg, q[e], D[m][e]);
+          p[m] = fmaf(D[m][e], w[e], p[m]);
+        }
+      }
+      rowsum4(p, dd, lane);
+#pragma unroll
+      for (int m = 0; m < 4; ++m) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) D[m][e] = fmaf(-dd[m], r[e], D[m][e]) * a[e];
+      }
+      if (lane < 4) Q.dd[((size_t)bh * T + t0 + tt) * dv + j0 + 4 * warp + lane] = pick4(dd, lane);
+    }
+    __syncthreads();
+  }
+  if (act && Q.dS0) {
+#pragma unroll
+    for (int m = 0; m < 4; ++m)
+      *reinterpret_cast<float4 *>(Q.dS0 + ((size_t)bh * dv + j0 + 4 * warp + m) * dk + c) =
+          make_float4(D[m][0], D[m][1], D[m][2], D[m][3]);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Column sweeps F2 / R2. CTA = d_k threads, thread i = key channel i, holding
+// rows j0 .. j0 + R - 1 of that column; with delta (F2) or dd (R2) known the
+// rows need no reduction, and the column sums over the CTA's rows are
+// per-thread. Per token the CTA writes its row group's partial sums to
+// part[g][bh][t][3][d_k] (slots: c S^T dO, -P^T dd, dS~^T delta).
+
+// Stages R floats of a per-row workspace vector (delta or dd) of token t.
+__device__ __forceinline__ void stage_rows(const float *src, int part, float *dst) {
+  cp_async16(smem_u32(dst + 4 * part), src + 4 * part, true);
+}
+
+// F2: forward, S_t = S_{t-1} Diag(alpha_t) + delta_t w_t^T;
+// dq'_t = c S_t^T dO_t and dr_t = -P_t^T dd_t.
+template <typename Tin, int R>
+__global__ void __launch_bounds__(128) f2_kernel(const BParams Q) {
+  extern __shared__ float4 smem4[];
+  float *sm = reinterpret_cast<float *>(smem4);
+  const KParams &P = Q.P;
+  const int dk = P.dk, dv = P.dv, T = P.T, BH = P.B * P.H;
+  const int bh = blockIdx.x / Q.G, g = blockIdx.x % Q.G, j0 = g * R;
+  const int i = threadIdx.x;
+  const float cq = P.q_scale;
+  const int TS = 2 * dk + 3 * R;  // w | alpha | delta | dd | dO (raw)
+  const int nv = dk / 2, nr = R / 4, nd = Q.dO ? R * (int)sizeof(Tin) / 16 : 0;
+  const int nc = (T + kLC - 1) / kLC;
+  auto issue = [&](int ch) {
+    float *buf = sm + (ch & 1) * kLC * TS;
+    const int t0 = ch * kLC, n = min(kLC, T - t0), per = nv + 2 * nr + nd;
+    for (int e = threadIdx.x; e < n * per; e += blockDim.x) {
+      const int tt = e / per, k = e % per, t = t0 + tt;
+      float *d = buf + tt * TS;
+      if (k < nv)
+        cp_async16(smem_u32(d + 4 * k), gen_at(Q, bh, t) + 2 * dk + 4 * k, true);
+      else if (k < nv + nr)
+        stage_rows(Q.delta + ((size_t)bh * T + t) * dv + j0, k - nv, d + 2 * dk);
+      else if (k < nv + 2 * nr)
+        stage_rows(Q.dd + ((size_t)bh * T + t) * dv + j0, k - nv - nr, d + 2 * dk + R);
+      else
+        stage_dO<Tin>(Q, bh, t, j0, k - nv - 2 * nr, d + 2 * dk + 2 * R);
+    }
+  };
+  float S[R];
+#pragma unroll
+  for (int j = 0; j < R; ++j) S[j] = P.S0 ? P.S0[((size_t)bh * dv + j0 + j) * dk + i] : 0.f;
+  issue(0);
+  cp_async_commit();
+  for (int ch = 0; ch < nc; ++ch) {
+    if (ch + 1 < nc) issue(ch + 1);
+    cp_async_commit();
+    cp_async_wait_group<1>();
+    __syncthreads();
+    const float *buf = sm + (ch & 1) * kLC * TS;
+    const int t0 = ch * kLC, n = min(kLC, T - t0);
+    for (int tt = 0; tt < n; ++tt) {
+      const float *sv = buf + tt * TS;
+      const float w = sv[i], a = sv[dk + i];
+      float accq = 0.f, accr = 0.f;
+#pragma unroll
+      for (int j = 0; j < R; j += 4) {
+        float de[4], dd[4], go[4];
+        ld4(sv + 2 * dk + j, true, de);
+        ld4(sv + 2 * dk + R + j, true, dd);
+        if (Q.dO) {
+          ld_rows4<Tin>(sv + 2 * dk + 2 * R, j, go);
+        } else {
+          go[0] = go[1] = go[2] = go[3] = 0.f;
+        }
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float p = S[j + e] * a;
+          accr = fmaf(p, dd[e], accr);
+          S[j + e] = fmaf(de[e], w, p);
+          accq = fmaf(S[j + e], go[e], accq);
+        }
+      }
+      float *o = Q.part + (((size_t)g * BH + bh) * T + t0 + tt) * 3 * dk;
+      o[i] = cq * accq;
+      o[dk + i] = -accr;
+    }
+    __syncthreads();
+  }
+}
+
+// R2: reverse, dS~_t = dS_t + c dO_t q'_t^T, dS_{t-1} = (dS~_t - dd_t r_t^T)
+// Diag(alpha_t); dw_t = dS~_t^T delta_t.
+template <typename Tin, int R>
+__global__ void __launch_bounds__(128) r2_kernel(const BParams Q) {
+  extern __shared__ float4 smem4[];
+  float *sm = reinterpret_cast<float *>(smem4);
+  const KParams &P = Q.P;
+  const int dk = P.dk, dv = P.dv, T = P.T, BH = P.B * P.H;
+  const int bh = blockIdx.x / Q.G, g = blockIdx.x % Q.G, j0 = g * R;
+  const int i = threadIdx.x;
+  const float cq = P.q_scale;
+  const int TS = 4 * dk + 3 * R;  // q' | r | w | alpha | delta | dd | dO (raw)
+  const int nv = dk, nr = R / 4, nd = Q.dO ? R * (int)sizeof(Tin) / 16 : 0;
+  const int nc = (T + kLC - 1) / kLC;
+  auto issue = [&](int ch) {
+    float *buf = sm + (ch & 1) * kLC * TS;
+    const int t0 = ch * kLC, n = min(kLC, T - t0), per = nv + 2 * nr + nd;
+    for (int e = threadIdx.x; e < n * per; e += blockDim.x) {
+      const int tt = e / per, k = e % per, t = t0 + tt;
+      float *d = buf + tt * TS;
+      if (k < nv)
+        cp_async16(smem_u32(d + 4 * k), gen_at(Q, bh, t) + 4 * k, true);
+      else if (k < nv + nr)
+        stage_rows(Q.delta + ((size_t)bh * T + t) * dv + j0, k - nv, d + 4 * dk);
+      else if (k < nv + 2 * nr)
+        stage_rows(Q.dd + ((size_t)bh * T + t) * dv + j0, k - nv - nr, d + 4 * dk + R);
+      else
+        stage_dO<Tin>(Q, bh, t, j0, k - nv - 2 * nr, d + 4 * dk + 2 * R);
+    }
+  };
+  float D[R];
+#pragma unroll
+  for (int j = 0; j < R; ++j) D[j] = Q.dST ? Q.dST[((size_t)bh * dv + j0 + j) * dk + i] : 0.f;
+  if (nc > 0) issue(nc - 1);
+  cp_async_commit();
+  for (int ch = nc - 1; ch >= 0; --ch) {
+    if (ch > 0) issue(ch - 1);
+    cp_async_commit();
+    cp_async_wait_group<1>();
+    __syncthreads();
+    const float *buf = sm + (ch & 1) * kLC * TS;
+    const int t0 = ch * kLC, n = min(kLC, T - t0);
+    for (int tt = n - 1; tt >= 0; --tt) {
+      const float *sv = buf + tt * TS;
+      const float q = sv[i], r = sv[dk + i], a = sv[3 * dk + i];
+      const float cqq = cq * q;
+      float accw = 0.f;
+#pragma unroll
+      for (int j = 0; j < R; j += 4) {
+        float de[4], dd[4], go[4];
+        ld4(sv + 4 * dk + j, true, de);
+        ld4(sv + 4 * dk + R + j, true, dd);
+        if (Q.dO) {
+          ld_rows4<Tin>(sv + 4 * dk + 2 * R, j, go);
+        } else {
+          go[0] = go[1] = go[2] = go[3] = 0.f;
+        }
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float dt = fmaf(cqq, go[e], D[j + e]);
+          accw = fmaf(dt, de[e], accw);
+          D[j + e] = fmaf(-dd[e], r, dt) * a;
+        }
+      }
+      Q.part[(((size_t)g * BH + bh) * T + t0 + tt) * 3 * dk + 2 * dk + i] = accw;
+    }
+    __syncthreads();
+  }
+}
+
+// ---------------------------------------------------------------------------
+// E1: per (token, head), one warp: the row groups' partial sums are added,
+// then each variant's map from (q', r, w, u) to its inputs is differentiated
+// ("Gated DeltaNet-2" ja §3: the gates' own gradients, derase = k . dr and
+// dwrite = v . du). Also the token's term of the decay suffix sum and, for
+// the preconditioner, the dA_t of its own coefficients:
+//   B = x^-s, s = c / (1 + |c|), c = L - mean(L), L = log(A + eps)
+//   => dA = (dc - mean(dc)) / (A + eps), dc = -ln x B dB / (1 + |c|)^2.
+template <typename Tin>
+__global__ void e1_kernel(const BParams Q) {
+  const KParams &P = Q.P;
+  const int lane = threadIdx.x & 31, dk = P.dk, dv = P.dv, T = P.T, BH = P.B * P.H;
+  const long long n = (long long)BH * T;
+  const long long nw = ((long long)gridDim.x * blockDim.x) >> 5;
+  for (long long wid = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5; wid < n; wid += nw) {
+    const int bh = (int)(wid / T), t = (int)(wid % T);
+    const size_t tk = tok_index(P, bh / P.H, t, bh % P.H);
+    const int c = 4 * lane;
+    const bool ak = c < dk, av = c < dv;
+    float dq[4], dr[4], dw[4], du[4], qq[4], r[4], w[4], k[4], v[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) dq[e] = dr[e] = dw[e] = 0.f;
+    for (int g = 0; g < Q.G; ++g) {
+      const float *pp = Q.part + (((size_t)g * BH + bh) * T + t) * 3 * dk + c;
+      float x[4], y[4], z[4];
+      ld4(pp, ak, x);
+      ld4(pp + dk, ak, y);
+      ld4(pp + 2 * dk, ak, z);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        dq[e] += x[e];
+        dr[e] += y[e];
+        dw[e] += z[e];
+      }
+    }
+    const float *gv = gen_at(Q, bh, t);
+    ld4(gv + c, ak, qq);
+    ld4(gv + dk + c, ak, r);
+    ld4(gv + 2 * dk + c, ak, w);
+    ld4(Q.dd + ((size_t)bh * T + t) * dv + c, av, du);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      k[e] = ak ? ldf<Tin>(P.k, tk * dk + c + e) : 0.f;
+      v[e] = av ? ldf<Tin>(P.v, tk * dv + c + e) : 0.f;
+    }
+    // decay: this token's term q'.dq' - w.dw + r.dr
+    if (P.decay != PDN_DECAY_NONE) {
+      float cp[4], s = 0.f;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        cp[e] = qq[e] * dq[e] - w[e] * dw[e] + r[e] * dr[e];
+        s += cp[e];
+      }
+      if (P.decay == PDN_DECAY_CHANNEL) {
+        if (ak)
+          *reinterpret_cast<float4 *>(Q.cpsi + ((size_t)bh * T + t) * dk + c) =
+              make_float4(cp[0], cp[1], cp[2], cp[3]);
+      } else {
+        s = warp_sum(s);
+        if (lane == 0) Q.sigma[(size_t)bh * T + t] = s;
+      }
+    }
+    float gq[4], gk[4], gvv[4], dB[4], Bc[4], A[4], L[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      gq[e] = dq[e];
+      gk[e] = dr[e] + dw[e];
+      gvv[e] = du[e];
+      dB[e] = 0.f;
+      Bc[e] = 1.f;
+    }
+    const bool pre = is_precond(P.variant);
+    float mu = 0.f;
+    if (pre) {
+      float s = 0.f;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        A[e] = ak ? Q.acc[((size_t)bh * T + t) * dk + c + e] : 0.f;
+        L[e] = ak ? logf(A[e] + P.eps) : 0.f;
+        s += L[e];
+      }
+      mu = warp_sum(s) / (float)dk;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) Bc[e] = precond_coef(L[e], mu, P.lnx);
+    }
+    switch (P.variant) {
+      case PDN_VAR_DN: case PDN_VAR_GDN: case PDN_VAR_KDA:
+      case PDN_VAR_PDN: case PDN_VAR_PGDN: case PDN_VAR_PKDA: {
+        const float be = reinterpret_cast<const float *>(P.beta)[tk];
+        float db = 0.f;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          gk[e] = dr[e] + be * Bc[e] * dw[e];
+          db = fmaf(Bc[e] * k[e], dw[e], db);
+          dB[e] = be * k[e] * dw[e];
+        }
+        db = warp_sum(db);
+        if (lane == 0 && Q.dbeta) Q.dbeta[tk] = db;
+      } break;
+      case PDN_VAR_PLA: {
+        const float be = reinterpret_cast<const float *>(P.beta)[tk];
+        float db = 0.f;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float q = ak ? ldf<Tin>(P.q, tk * dk + c + e) : 0.f;
+          gk[e] = be * dw[e];
+          db = fmaf(k[e], dw[e], db);
+          dB[e] = q * dq[e];
+          gq[e] = Bc[e] * dq[e];
+        }
+        db = warp_sum(db);
+        if (lane == 0 && Q.dbeta) Q.dbeta[tk] = db;
+      } break;
+      case PDN_VAR_FG2_GDN: case PDN_VAR_FG2_GDN_PLUS: {
+        const bool plus = P.variant == PDN_VAR_FG2_GDN_PLUS;
+        float dbk[4], dwr[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float bk = ak ? ldf<Tin>(P.beta, tk * dk + c + e) : 1.f;
+          const float sb = sqrtf(bk);
+          gk[e] = sb * (dr[e] + dw[e]);
+          dbk[e] = k[e] * (dr[e] + dw[e]) / (2.f * sb);
+          const float bv = av ? (plus ? ldf<Tin>(P.write, tk * dv + c + e) : bk) : 1.f;
+          const float sv = sqrtf(bv);
+          gvv[e] = sv * du[e];
+          dwr[e] = v[e] * du[e] / (2.f * sv);
+          if (!plus) dbk[e] += dwr[e];
+        }
+        if (Q.dbeta && ak)
+          *reinterpret_cast<float4 *>(Q.dbeta + tk * dk + c) = make_float4(dbk[0], dbk[1], dbk[2], dbk[3]);
+        if (plus && Q.dwrite && av)
+          *reinterpret_cast<float4 *>(Q.dwrite + tk * dv + c) = make_float4(dwr[0], dwr[1], dwr[2], dwr[3]);
+      } break;
+      case PDN_VAR_GDN2: {
+        float de[4], dg[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float er = ak ? ldf<Tin>(P.erase, tk * dk + c + e) : 0.f;
+          const float gw = av ? ldf<Tin>(P.write, tk * dv + c + e) : 0.f;
+          gk[e] = er * dr[e] + dw[e];
+          de[e] = k[e] * dr[e];
+          gvv[e] = gw * du[e];
+          dg[e] = v[e] * du[e];
+        }
+        if (Q.derase && ak)
+          *reinterpret_cast<float4 *>(Q.derase + tk * dk + c) = make_float4(de[0], de[1], de[2], de[3]);
+        if (Q.dwrite && av)
+          *reinterpret_cast<float4 *>(Q.dwrite + tk * dv + c) = make_float4(dg[0], dg[1], dg[2], dg[3]);
+      } break;
+      default: break;
+    }
+    if (pre) {
+      // dA of this token's own coefficients
+      float dc[4], s = 0.f;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float cc = L[e] - mu;
+        const float den = 1.f + fabsf(cc);
+        dc[e] = ak ? -P.lnx * Bc[e] * dB[e] / (den * den) : 0.f;
+        s += dc[e];
+      }
+      const float mdc = warp_sum(s) / (float)dk;
+      if (ak) {
+        float da[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) da[e] = (dc[e] - mdc) / (A[e] + P.eps);
+        *reinterpret_cast<float4 *>(Q.dacc + ((size_t)bh * T + t) * dk + c) =
+            make_float4(da[0], da[1], da[2], da[3]);
+      }
+    }
+    if (Q.dq && ak) *reinterpret_cast<float4 *>(Q.dq + tk * dk + c) = make_float4(gq[0], gq[1], gq[2], gq[3]);
+    if (Q.dk && ak) *reinterpret_cast<float4 *>(Q.dk + tk * dk + c) = make_float4(gk[0], gk[1], gk[2], gk[3]);
+    if (Q.dv && av)
+      *reinterpret_cast<float4 *>(Q.dv + tk * dv + c) = make_float4(gvv[0], gvv[1], gvv[2], gvv[3]);
+  }
+}
+
+// E3 (preconditioned variants): k_t feeds A_s for every s >= t, so
+// dk_t += 2 k_t . (sum_{s>=t} dA_s) (the suffix sums sit in dacc).
+template <typename Tin>
+__global__ void e3_kernel(const BParams Q) {
+  const KParams &P = Q.P;
+  const int dk = P.dk;
+  const long long n = (long long)P.B * P.H * P.T * dk;
+  for (long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x; e < n;
+       e += (long long)gridDim.x * blockDim.x) {
+    const int i = (int)(e % dk);
+    const long long r = e / dk;
+    const int t = (int)(r % P.T), bh = (int)(r / P.T);
+    const size_t o = tok_index(P, bh / P.H, t, bh % P.H) * dk + i;
+    Q.dk[o] += 2.f * ldf<Tin>(P.k, o) * Q.dacc[e];
+  }
+}
+
+// psi_T,i = sum_j S_T[j,i] dS_T[j,i] per (batch, head), and its sum over i
+// (the start of the scalar decay's suffix sum) at phi[BH * d_k + bh].
+__global__ void __launch_bounds__(128) phi_kernel(const BParams Q) {
+  __shared__ float red[4];
+  const KParams &P = Q.P;
+  const int bh = blockIdx.x, i = threadIdx.x, dk = P.dk, dv = P.dv;
+  float s = 0.f;
+  if (i < dk) {
+    const size_t base = (size_t)bh * dv * dk + i;
+    for (int j = 0; j < dv; ++j) s = fmaf(Q.st[base + (size_t)j * dk], Q.dST[base + (size_t)j * dk], s);
+    Q.phi[(size_t)bh * dk + i] = s;
+  }
+  s = warp_sum(s);
+  if ((i & 31) == 0) red[i >> 5] = s;
+  __syncthreads();
+  if (i == 0) Q.phi[(size_t)P.B * P.H * dk + bh] = red[0] + red[1] + red[2] + red[3];
+}
+
+unsigned grid_for(long long n, int threads) {
+  const long long b = (n + threads - 1) / threads;
+  return (unsigned)(b < 1 ? 1 : (b > 148 * 16 ? 148 * 16 : b));
+}
+
+void run_scan(const KParams &P, ScanArr X, ScanArr Y, int nch, int nb, bool rev, const float *init,
+              float *total, float *bsum, cudaStream_t st) {
+  const long long BH = (long long)P.B * P.H;
+  scan_part_kernel<<<grid_for(BH * nb * nch, 256), 256, 0, st>>>(P, X, nch, nb, bsum);
+  scan_carry_kernel<<<grid_for(BH * nch, 128), 128, 0, st>>>(P, nch, nb, rev, bsum, init, total);
+  scan_fill_kernel<<<grid_for(BH * nb * nch, 256), 256, 0, st>>>(P, X, Y, nch, nb, rev, bsum);
+}
+
+template <typename K>
+cudaError_t set_smem(K kernel, size_t bytes) {
+  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+}
+
+template <typename Tin, int R>
+cudaError_t launch_bwd_t(const BParams &Q, cudaStream_t st) {
+  const KParams &P = Q.P;
+  const int dk = P.dk, dv = P.dv;
+  const long long BH = (long long)P.B * P.H, BHT = BH * P.T;
+  cudaError_t err;
+  if (is_precond(P.variant)) {
+    prep_sq_kernel<Tin><<<grid_for(BHT * dk, 256), 256, 0, st>>>(Q);
+    run_scan(P, ScanArr{Q.acc, false}, ScanArr{Q.acc, false}, dk, Q.nb, false, P.A0, nullptr,
+             Q.bsum, st);
+  }
+  prep_gen_kernel<Tin><<<grid_for(BHT * 32, 256), 256, 0, st>>>(Q);
+
+  const size_t sm_f1 = 2 * kLC * (3 * dk + 16) * sizeof(float);
+  const size_t sm_r1 = 2 * kLC * (4 * dk + 16) * sizeof(float);
+  const size_t sm_f2 = 2 * kLC * (2 * dk + 3 * R) * sizeof(float);
+  const size_t sm_r2 = 2 * kLC * (4 * dk + 3 * R) * sizeof(float);
+  if ((err = set_smem(f1_kernel, sm_f1)) != cudaSuccess) return err;
+  if ((err = set_smem(r1_kernel<Tin>, sm_r1)) != cudaSuccess) return err;
+  if ((err = set_smem(f2_kernel<Tin, R>, sm_f2)) != cudaSuccess) return err;
+  if ((err = set_smem(r2_kernel<Tin, R>, sm_r2)) != cudaSuccess) return err;
+  const unsigned grid_rows = (unsigned)(BH * (dv / kRowsF));
+  const unsigned grid_cols = (unsigned)(BH * Q.G);
+  f1_kernel<<<grid_rows, 128, sm_f1, st>>>(Q);
+  r1_kernel<Tin><<<grid_rows, 128, sm_r1, st>>>(Q);
+  f2_kernel<Tin, R><<<grid_cols, dk, sm_f2, st>>>(Q);
+  r2_kernel<Tin, R><<<grid_cols, dk, sm_r2, st>>>(Q);
+  e1_kernel<Tin><<<grid_for(BHT * 32, 256), 256, 0, st>>>(Q);
+
+  if (P.decay != PDN_DECAY_NONE && Q.dla) {
+    if (Q.dST) phi_kernel<<<(unsigned)BH, 128, 0, st>>>(Q);
+    if (P.decay == PDN_DECAY_CHANNEL)
+      run_scan(P, ScanArr{Q.cpsi, false}, ScanArr{Q.dla, true}, dk, Q.nb, true,
+               Q.dST ? Q.phi : nullptr, nullptr, Q.bsum, st);
+    else
+      run_scan(P, ScanArr{Q.sigma, false}, ScanArr{Q.dla, true}, 1, Q.nb, true,
+               Q.dST ? Q.phi + BH * dk : nullptr, nullptr, Q.bsum, st);
+  }
+  if (is_precond(P.variant) && (Q.dk || Q.dA0)) {
+    run_scan(P, ScanArr{Q.dacc, false}, ScanArr{Q.dacc, false}, dk, Q.nb, true, nullptr, Q.dA0,
+             Q.bsum, st);
+    if (Q.dk) e3_kernel<Tin><<<grid_for(BHT * dk, 256), 256, 0, st>>>(Q);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+size_t bwd_workspace_bytes(const KParams &P) { return bwd_plan(P).total * sizeof(float); }
+
+cudaError_t launch_chunk_bwd(const KParams &P, const pdn_grads_t *g, void *workspace,
+                             cudaStream_t stream) {
+  const long long BH = (long long)P.B * P.H;
+  if (P.T == 0) {
+    // no token: the initial state is the final state, A0 reaches nothing
+    cudaError_t err = cudaSuccess;
+    if (g->dS0) {
+      const size_t bytes = (size_t)BH * P.dv * P.dk * sizeof(float);
+      err = g->dST ? cudaMemcpyAsync(g->dS0, g->dST, bytes, cudaMemcpyDeviceToDevice, stream)
+                   : cudaMemsetAsync(g->dS0, 0, bytes, stream);
+      if (err != cudaSuccess) return err;
+    }
+    if (g->dA0 && is_precond(P.variant))
+      err = cudaMemsetAsync(g->dA0, 0, (size_t)BH * P.dk * sizeof(float), stream);
+    return err;
+  }
+  const BwdPlan L = bwd_plan(P);
+  float *ws = static_cast<float *>(workspace);
+  BParams Q;
+  memset(&Q, 0, sizeof(Q));
+  Q.P = P;
+  Q.dO = g->dO; Q.dST = g->dST;
+  Q.dq = g->dq; Q.dk = g->dk; Q.dv = g->dv; Q.dla = g->dlog_alpha; Q.dbeta = g->dbeta;
+  Q.derase = g->derase; Q.dwrite = g->dwrite; Q.dS0 = g->dS0; Q.dA0 = g->dA0;
+  Q.gen = ws + L.gen; Q.acc = ws + L.acc; Q.delta = ws + L.delta; Q.dd = ws + L.dd;
+  Q.st = ws + L.st; Q.part = ws + L.part; Q.cpsi = ws + L.cpsi; Q.sigma = ws + L.sigma;
+  Q.dacc = ws + L.dacc; Q.bsum = ws + L.bsum; Q.phi = ws + L.phi;
+  Q.GS = L.GS; Q.R = L.R; Q.G = L.G; Q.nb = L.nb;
+  const bool bf = P.dtype == PDN_BF16;
+  if (L.R == 32) return bf ? launch_bwd_t<__nv_bfloat16, 32>(Q, stream) : launch_bwd_t<float, 32>(Q, stream);
+  return bf ? launch_bwd_t<__nv_bfloat16, 16>(Q, stream) : launch_bwd_t<float, 16>(Q, stream);
+}
+
+}  // namespace pdn

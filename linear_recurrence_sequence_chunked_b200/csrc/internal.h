@@ -36,6 +36,12 @@ cudaError_t launch_decode(const KParams &P, cudaStream_t stream);
 pdn_status_t check_chunk_fwd(const pdn_problem_t *p, const pdn_tensors_t *t,
                              const void *workspace, size_t ws_bytes, int *impl_out);
 
+// Backward (gradient of the chunked forward): workspace bytes, and the
+// enqueue of every kernel of it (CUDA cores, fp32).
+size_t bwd_workspace_bytes(const KParams &P);
+cudaError_t launch_chunk_bwd(const KParams &P, const pdn_grads_t *g, void *workspace,
+                             cudaStream_t stream);
+
 // Bounded-wait self test.
 cudaError_t launch_selftest_wait(long long limit_ns, int *err, cudaStream_t stream);
 

@@ -45,6 +45,12 @@ class PdnTensors(ctypes.Structure):
                 ("q", "k", "v", "log_alpha", "beta", "erase", "write", "S0", "ST", "A0", "AT", "o")]
 
 
+class PdnGrads(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in
+                ("dO", "dST", "dq", "dk", "dv", "dlog_alpha", "dbeta", "derase", "dwrite", "dS0",
+                 "dA0")]
+
+
 class PdnError(RuntimeError):
     def __init__(self, code, where):
         self.code = code
@@ -77,6 +83,11 @@ def load() -> ctypes.CDLL:
         lib.pdn_chunk_fwd_noalloc.argtypes = [P, T, vp]
         lib.pdn_chunk_fwd_host.restype = ctypes.c_int
         lib.pdn_chunk_fwd_host.argtypes = [P, T, T, vp, ctypes.c_size_t, ctypes.c_int, vp]
+        G = ctypes.POINTER(PdnGrads)
+        lib.pdn_chunk_bwd_workspace.restype = ctypes.c_size_t
+        lib.pdn_chunk_bwd_workspace.argtypes = [P]
+        lib.pdn_chunk_bwd.restype = ctypes.c_int
+        lib.pdn_chunk_bwd.argtypes = [P, T, G, vp, ctypes.c_size_t, vp]
         lib.pdn_chunk_transition.restype = ctypes.c_int
         lib.pdn_chunk_transition.argtypes = [P, T, vp, ctypes.c_size_t, vp]
         lib.pdn_key_energy.restype = ctypes.c_int
@@ -121,6 +132,16 @@ def pdn_chunk_fwd_profiled(problem: PdnProblem, tensors: PdnTensors, workspace: 
     rc = load().pdn_chunk_fwd_profiled(ctypes.byref(problem), ctypes.byref(tensors), workspace,
                                        ws_bytes, stream, ms, ctypes.byref(n))
     return rc, [float(ms[i]) for i in range(n.value)]
+
+
+def pdn_chunk_bwd_workspace(problem: PdnProblem) -> int:
+    return load().pdn_chunk_bwd_workspace(ctypes.byref(problem))
+
+
+def pdn_chunk_bwd(problem: PdnProblem, tensors: PdnTensors, grads: PdnGrads, workspace: int,
+                  ws_bytes: int, stream: int) -> int:
+    return load().pdn_chunk_bwd(ctypes.byref(problem), ctypes.byref(tensors), ctypes.byref(grads),
+                                workspace, ws_bytes, stream)
 
 
 def pdn_chunk_transition(problem: PdnProblem, tensors: PdnTensors, workspace: int,
@@ -264,6 +285,51 @@ def chunk_fwd(variant: str, q, k, v, log_alpha=None, beta=None, erase=None, writ
     stream = torch.cuda.current_stream(dev).cuda_stream
     _check(pdn_chunk_fwd(p, t, ws_ptr, ws_bytes, stream), "pdn_chunk_fwd")
     return o, ST, AT
+
+
+def make_grads(dO=None, dST=None, dq=None, dk=None, dv=None, dlog_alpha=None, dbeta=None,
+               derase=None, dwrite=None, dS0=None, dA0=None) -> PdnGrads:
+    return PdnGrads(_ptr(dO), _ptr(dST), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dlog_alpha),
+                    _ptr(dbeta), _ptr(derase), _ptr(dwrite), _ptr(dS0), _ptr(dA0))
+
+
+def chunk_bwd(variant: str, q, k, v, dO=None, dST=None, log_alpha=None, beta=None, erase=None,
+              write=None, S0=None, A0=None, q_scale: float = 1.0, precond_x: float = 1.5,
+              precond_eps: float = 1e-6, workspace=None):
+    """Gradients of chunk_fwd's (o, S_T) with respect to its inputs, given the
+    cotangents dO [B,T,H,d_v] (input dtype) and dST [B,H,d_v,d_k] (fp32);
+    either may be None (zero). Returns a dict of fp32 tensors with keys q, k,
+    v, log_alpha, beta, erase, write, S0, A0 (None where the variant has no
+    such input)."""
+    B, T, H, d_k = k.shape
+    d_v = v.shape[3]
+    dev = k.device
+    p = make_problem(variant, B, T, H, d_k, d_v, k.dtype, _decay_of(log_alpha), 64, "auto",
+                     q_scale, precond_x, precond_eps)
+    f32 = dict(dtype=torch.float32, device=dev)
+    g = {"q": torch.empty(B, T, H, d_k, **f32), "k": torch.empty(B, T, H, d_k, **f32),
+         "v": torch.empty(B, T, H, d_v, **f32),
+         "log_alpha": None if log_alpha is None else torch.empty(log_alpha.shape, **f32),
+         "beta": None if beta is None else torch.empty(beta.shape, **f32),
+         "erase": None if variant != "GDN2" else torch.empty(B, T, H, d_k, **f32),
+         "write": (torch.empty(B, T, H, d_v, **f32) if variant in ("GDN2", "FG2_GDN_PLUS")
+                   else None),
+         "S0": torch.empty(B, H, d_v, d_k, **f32),
+         "A0": torch.empty(B, H, d_k, **f32) if variant in PRECOND_VARIANTS else None}
+    t = make_tensors(q, k, v, None, log_alpha, beta, erase, write, S0, None, A0, None)
+    gr = make_grads(dO, dST, g["q"], g["k"], g["v"], g["log_alpha"], g["beta"], g["erase"],
+                    g["write"], g["S0"], g["A0"])
+    need = pdn_chunk_bwd_workspace(p)
+    if need == ctypes.c_size_t(-1).value:
+        raise PdnError(PDN_ERR_INVALID_ARG, "pdn_chunk_bwd_workspace")
+    ws_ptr, ws_bytes = None, 0
+    if need > 0:
+        if workspace is None or workspace.numel() * workspace.element_size() < need:
+            workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+        ws_ptr, ws_bytes = workspace.data_ptr(), workspace.numel() * workspace.element_size()
+    stream = torch.cuda.current_stream(dev).cuda_stream
+    _check(pdn_chunk_bwd(p, t, gr, ws_ptr, ws_bytes, stream), "pdn_chunk_bwd")
+    return g
 
 
 def decode_step(variant: str, q, k, v, S, A=None, log_alpha=None, beta=None, erase=None,

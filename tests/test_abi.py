@@ -55,25 +55,30 @@ def test_struct_layout_matches_header(tmp_path):
     src = tmp_path / "layout.c"
     fields_p = [f[0] for f in pdn.PdnProblem._fields_]
     fields_t = [f[0] for f in pdn.PdnTensors._fields_]
+    fields_g = [f[0] for f in pdn.PdnGrads._fields_]
     lines = ['#include <stdio.h>', '#include <stddef.h>', '#include "pdn.h"', 'int main(void){',
-             'printf("%zu %zu\\n", sizeof(pdn_problem_t), sizeof(pdn_tensors_t));']
+             'printf("%zu %zu %zu\\n", sizeof(pdn_problem_t), sizeof(pdn_tensors_t), '
+             'sizeof(pdn_grads_t));']
     for f in fields_p:
         lines.append('printf("p %s %%zu\\n", offsetof(pdn_problem_t, %s));' % (f, f))
     for f in fields_t:
         lines.append('printf("t %s %%zu\\n", offsetof(pdn_tensors_t, %s));' % (f, f))
+    for f in fields_g:
+        lines.append('printf("g %s %%zu\\n", offsetof(pdn_grads_t, %s));' % (f, f))
     lines.append("return 0;}")
     src.write_text("\n".join(lines))
     exe = tmp_path / "layout"
     subprocess.check_call(["gcc", "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe)])
     out = subprocess.check_output([str(exe)], text=True).split("\n")
-    sp, stt = map(int, out[0].split())
+    sp, stt, sg = map(int, out[0].split())
     assert sp == ctypes.sizeof(pdn.PdnProblem)
     assert stt == ctypes.sizeof(pdn.PdnTensors)
+    assert sg == ctypes.sizeof(pdn.PdnGrads)
     for line in out[1:]:
         if not line:
             continue
         kind, name, off = line.split()
-        cls = pdn.PdnProblem if kind == "p" else pdn.PdnTensors
+        cls = {"p": pdn.PdnProblem, "t": pdn.PdnTensors, "g": pdn.PdnGrads}[kind]
         assert getattr(cls, name).offset == int(off), name
 
 
@@ -264,3 +269,62 @@ def test_host_pipeline_validates_before_enqueueing(lib):
                                   None) == pdn.PDN_ERR_INVALID_ARG
     # T * H odd: slice 1's scalar gates are 4-byte aligned, which is accepted
     assert pdn.pdn_chunk_fwd_host(p, t, t, ws, need, 2, None) == pdn.PDN_ERR_CUDA
+
+
+# ------------------------------------------------------------------ backward
+def _grads(**over):
+    d = dict(dO=FAKE + 0x10000, dST=None, dq=FAKE + 0x11000, dk=FAKE + 0x12000,
+             dv=FAKE + 0x13000, dlog_alpha=FAKE + 0x14000, dbeta=FAKE + 0x15000, derase=None,
+             dwrite=None, dS0=None, dA0=None)
+    d.update(over)
+    return pdn.PdnGrads(**d)
+
+
+@pytest.mark.parametrize("over", INVALID_PROBLEMS)
+def test_backward_invalid_problem_rejected(lib, over):
+    p = _problem(**over)
+    assert pdn.pdn_chunk_bwd(p, _tensors(), _grads(), None, 0, None) == pdn.PDN_ERR_INVALID_ARG
+    assert pdn.pdn_chunk_bwd_workspace(p) == ctypes.c_size_t(-1).value
+
+
+BWD_INVALID = [
+    (dict(), dict(dq=FAKE + 0x11008)),                       # misaligned gradient
+    (dict(), dict(dO=FAKE + 0x10004)),                       # misaligned cotangent
+    (dict(), dict(dlog_alpha=FAKE + 0x14002)),               # scalar decay: 4-byte rule
+    (dict(variant=pdn.VARIANTS["PDN"], decay=pdn.DECAYS["none"]), dict()),  # dlog_alpha, no decay
+    (dict(), dict(derase=FAKE + 0x16000)),                   # GDN2-only gradient
+    (dict(), dict(dwrite=FAKE + 0x16000)),                   # GDN2 / FG2+ only
+    (dict(variant=pdn.VARIANTS["GDN"]), dict(dA0=FAKE + 0x17000)),  # no accumulator
+]
+
+
+@pytest.mark.parametrize("pover,gover", BWD_INVALID)
+def test_backward_invalid_gradients_rejected(lib, pover, gover):
+    p = _problem(**pover)
+    t = _tensors(log_alpha=None) if p.decay == 0 else _tensors()
+    assert pdn.pdn_chunk_bwd(p, t, _grads(**gover), FAKE, 1 << 40, None) == pdn.PDN_ERR_INVALID_ARG
+
+
+def test_backward_rules(lib):
+    # the forward output is not needed
+    p = _problem()
+    ws_need = pdn.pdn_chunk_bwd_workspace(p)
+    assert 0 < ws_need < (1 << 40)
+    # workspace missing, too small or misaligned
+    assert pdn.pdn_chunk_bwd(p, _tensors(o=None), _grads(), None, 0, None) == pdn.PDN_ERR_WORKSPACE
+    assert pdn.pdn_chunk_bwd(p, _tensors(o=None), _grads(), FAKE, ws_need - 1,
+                             None) == pdn.PDN_ERR_WORKSPACE
+    assert pdn.pdn_chunk_bwd(p, _tensors(o=None), _grads(), FAKE + 128, ws_need,
+                             None) == pdn.PDN_ERR_WORKSPACE
+    # a fused prologue is the forward's alone
+    assert pdn.pdn_chunk_bwd(_problem(prologue=1), _tensors(), _grads(), FAKE, ws_need,
+                             None) == pdn.PDN_ERR_UNSUPPORTED
+    # T == 0 needs no workspace
+    assert pdn.pdn_chunk_bwd_workspace(_problem(T=0)) == 0
+    # the gradient struct itself is required
+    assert load_bwd_null(lib) == pdn.PDN_ERR_INVALID_ARG
+
+
+def load_bwd_null(lib):
+    return lib.pdn_chunk_bwd(ctypes.byref(_problem()), ctypes.byref(_tensors()), None, None, 0,
+                             None)

@@ -1,0 +1,193 @@
+"""GPU parity of the backward: pdn_chunk_bwd through the C ABI against the
+fp64 oracle's reverse-mode gradient of the token loop (itself pinned by
+central finite differences), on the same seeded inputs and cotangents.
+
+The CUDA backward runs in fp32 for both input dtypes (bf16 inputs are widened
+exactly), so one bar holds for both: normalised max-abs error <= 2e-4 per
+gradient tensor (the forward's fp32 bar 1e-4, doubled for the extra passes:
+the decay gradient is a suffix sum over every later token)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from linear_recurrence_sequence_chunked_b200 import pdn
+from linear_recurrence_sequence_chunked_b200.workloads import (WORKLOADS, Workload, make_inputs,
+                                                               slice_chain)
+
+from parity_util import REPORT, elem_rel_err, nmax_err
+
+pytestmark = pytest.mark.gpu
+
+TOL_BWD = 2e-4
+VARIANTS = ["DN", "GDN", "KDA", "PDN", "PGDN", "PKDA", "FG2_GDN", "GDN2", "PLA", "FG2_GDN_PLUS"]
+DECAY = {"DN": "none", "PDN": "none", "GDN": "scalar", "PGDN": "scalar",
+         "KDA": "channel", "PKDA": "channel", "FG2_GDN": "channel", "GDN2": "channel",
+         "PLA": "scalar", "FG2_GDN_PLUS": "channel"}
+PRECOND = ("PDN", "PGDN", "PKDA", "PLA")
+
+
+def small(variant, dtype, B=2, T=150, H=3, dk=64, dv=None, decay=None, seed=0, **kw):
+    return Workload("bwd-%s-%s" % (variant, dtype), variant, B, T, H, dk, dk if dv is None else dv,
+                    dtype, decay or DECAY[variant], seed=seed, **kw)
+
+
+def states(w, seed=1, scale=0.3):
+    g = torch.Generator().manual_seed(seed)
+    S0 = scale * torch.randn(w.B, w.H, w.dv, w.dk, generator=g)
+    A0 = torch.rand(w.B, w.H, w.dk, generator=g) * 2.0 if w.variant in PRECOND else None
+    return S0, A0
+
+
+def cotangents(w, seed=5):
+    g = torch.Generator().manual_seed(seed)
+    dt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    dO = torch.randn(w.B, w.T, w.H, w.dv, generator=g).to(dt)
+    dST = 0.5 * torch.randn(w.B, w.H, w.dv, w.dk, generator=g)
+    return dO, dST
+
+
+def run_gpu(w, x, S0, A0, dO, dST):
+    dev = torch.device("cuda")
+    d = {n: (t.to(dev) if t is not None else None) for n, t in x.items()}
+    on = lambda t: None if t is None else t.to(dev)
+    g = pdn.chunk_bwd(w.variant, d["q"], d["k"], d["v"], dO=on(dO), dST=on(dST),
+                      log_alpha=d["log_alpha"], beta=d["beta"], erase=d["erase"], write=d["write"],
+                      S0=on(S0), A0=on(A0), q_scale=w.q_scale, precond_x=w.precond_x,
+                      precond_eps=w.precond_eps)
+    torch.cuda.synchronize()
+    assert pdn.device_error() == pdn.PDN_OK
+    return {n: (None if t is None else t.cpu().numpy()) for n, t in g.items()}
+
+
+def run_oracle(w, x, S0, A0, dO, dST):
+    return oracle.backward(w.variant, x["q"], x["k"], x["v"], log_alpha=x["log_alpha"],
+                           beta=x["beta"], erase=x["erase"], write=x["write"], S0=S0, A0=A0,
+                           q_scale=w.q_scale, x=w.precond_x, eps=w.precond_eps, dO=dO, dST=dST)
+
+
+def assert_grads(w, gg, gr, tol=TOL_BWD, label=""):
+    bad = []
+    for name, ref in gr.items():
+        if ref is None:
+            assert gg[name] is None, name
+            continue
+        e = nmax_err(gg[name], ref)
+        REPORT.append(("%s%s:d%s" % (w.name, label, name), w.dtype, e, 0.0,
+                       elem_rel_err(gg[name], ref), 0.0))
+        if not e <= tol:
+            bad.append((name, e))
+    assert not bad, bad
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("variant", VARIANTS)
+def test_backward_variants(variant, dtype):
+    """Every variant: ragged T (two 64-token scan blocks and a tail), random
+    S0 / A0 / dO / dS_T, q_scale != 1."""
+    w = small(variant, dtype, q_scale=0.8)
+    x = make_inputs(w)
+    S0, A0 = states(w)
+    dO, dST = cotangents(w)
+    assert_grads(w, run_gpu(w, x, S0, A0, dO, dST), run_oracle(w, x, S0, A0, dO, dST))
+
+
+@pytest.mark.parametrize("decay", ["none", "scalar", "channel"])
+@pytest.mark.parametrize("variant", ["FG2_GDN", "GDN2", "PLA", "FG2_GDN_PLUS"])
+def test_backward_free_decay(variant, decay):
+    w = small(variant, "bf16", decay=decay, T=97)
+    x = make_inputs(w)
+    S0, A0 = states(w)
+    dO, dST = cotangents(w)
+    assert_grads(w, run_gpu(w, x, S0, A0, dO, dST), run_oracle(w, x, S0, A0, dO, dST))
+
+
+@pytest.mark.parametrize("T", [1, 15, 16, 17, 63, 64, 65, 129])
+def test_backward_lengths(T):
+    """Token counts around the 16-token staging chunks and the 64-token scan
+    blocks; d = 32 leaves three quarters of each warp's lanes without a key
+    channel."""
+    w = small("PKDA", "f32", B=1, H=2, T=T, dk=32)
+    x = make_inputs(w)
+    S0, A0 = states(w)
+    dO, dST = cotangents(w)
+    assert_grads(w, run_gpu(w, x, S0, A0, dO, dST), run_oracle(w, x, S0, A0, dO, dST))
+
+
+@pytest.mark.parametrize("dk,dv", [(128, 64), (48, 80), (128, 128), (16, 16)])
+@pytest.mark.parametrize("variant", ["GDN2", "PGDN", "FG2_GDN_PLUS"])
+def test_backward_head_dims(variant, dk, dv):
+    w = small(variant, "bf16", B=1, H=2, T=70, dk=dk, dv=dv)
+    x = make_inputs(w)
+    S0, A0 = states(w)
+    dO, dST = cotangents(w)
+    assert_grads(w, run_gpu(w, x, S0, A0, dO, dST), run_oracle(w, x, S0, A0, dO, dST))
+
+
+@pytest.mark.parametrize("which", ["dO", "dST", "both"])
+def test_backward_absent_cotangents(which):
+    """A NULL cotangent is zero: the loss reads only o, only S_T, or neither."""
+    w = small("PKDA", "f32", T=40)
+    x = make_inputs(w)
+    S0, A0 = states(w)
+    dO, dST = cotangents(w)
+    if which in ("dO", "both"):
+        dO = None
+    if which in ("dST", "both"):
+        dST = None
+    gg = run_gpu(w, x, S0, A0, dO, dST)
+    gr = run_oracle(w, x, S0, A0, dO, dST)
+    if which == "both":
+        for n, t in gg.items():
+            if t is not None:
+                assert np.abs(t).max() == 0.0, n
+    else:
+        assert_grads(w, gg, gr)
+
+
+@pytest.mark.parametrize("variant", ["GDN", "KDA", "PKDA", "GDN2"])
+def test_backward_strong_decay(variant):
+    """Decays down to the per-token floor: the token-level backward never
+    divides by a cumulative decay, so it stays exact at any strength."""
+    w = small(variant, "f32", T=130, decay_recipe="strong", decay_mean=-20.0)
+    x = make_inputs(w)
+    S0, A0 = states(w)
+    dO, dST = cotangents(w)
+    assert_grads(w, run_gpu(w, x, S0, A0, dO, dST), run_oracle(w, x, S0, A0, dO, dST))
+
+
+@pytest.mark.parametrize("name,chains", [("pgdn_bf16_4k", [(0, 0), (3, 15)]),
+                                         ("pkda_bf16_8k", [(7, 15)]),
+                                         ("gdn2_bf16_32k", [(1, 9)])])
+def test_backward_full_size_sampled(name, chains):
+    """Full-size workloads: the whole backward on the GPU, the oracle on
+    sampled (batch, head) chains over all T tokens."""
+    w = WORKLOADS[name]
+    x = make_inputs(w, device="cuda")
+    g = torch.Generator().manual_seed(11)
+    dt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    dO = torch.randn(w.B, w.T, w.H, w.dv, generator=g).to(dt)
+    dST = 0.5 * torch.randn(w.B, w.H, w.dv, w.dk, generator=g)
+    gd = pdn.chunk_bwd(w.variant, x["q"], x["k"], x["v"], dO=dO.cuda(), dST=dST.cuda(),
+                       log_alpha=x["log_alpha"], beta=x["beta"], erase=x["erase"],
+                       write=x["write"], q_scale=w.q_scale, precond_x=w.precond_x,
+                       precond_eps=w.precond_eps)
+    torch.cuda.synchronize()
+    assert pdn.device_error() == pdn.PDN_OK
+    for b, h in chains:
+        xs = slice_chain(x, b, h)
+        gr = oracle.backward(w.variant, xs["q"], xs["k"], xs["v"], log_alpha=xs["log_alpha"],
+                             beta=xs["beta"], erase=xs["erase"], write=xs["write"],
+                             q_scale=w.q_scale, x=w.precond_x, eps=w.precond_eps,
+                             dO=dO[b:b + 1, :, h:h + 1], dST=dST[b:b + 1, h:h + 1])
+        gs = {}
+        for n, t in gd.items():
+            if t is None:
+                gs[n] = None
+            elif n == "S0":
+                gs[n] = t[b:b + 1, h:h + 1].cpu().numpy()
+            elif n == "A0":
+                gs[n] = t[b:b + 1, h:h + 1].cpu().numpy()
+            else:
+                gs[n] = t[b:b + 1, :, h:h + 1].cpu().numpy()
+        assert_grads(w, gs, gr, label="[b%d,h%d]" % (b, h))
