@@ -51,7 +51,6 @@ struct BwdPlan {
 namespace {
 
 constexpr int kScanBlk = 64;     // tokens per scan block
-constexpr int kRowsF = 16;       // state rows per CTA of F1 / R1 (4 warps x 4)
 constexpr int kLC = 16;          // tokens staged per chunk in F1 / R1 / F2 / R2
 
 size_t up64(size_t n) { return (n + 63) & ~(size_t)63; }
@@ -71,7 +70,7 @@ static BwdPlan bwd_plan(const KParams &P) {
   const int dk = P.dk, dv = P.dv;
   L.GS = 4 * dk + dv;
   const long long rows32 = (long long)BH * (dv / 32);
-  L.R = (dv % 32 == 0 && rows32 >= 2 * 148) ? 32 : 16;
+  L.R = (dv % 32 == 0 && rows32 >= 148) ? 32 : 16;
   L.G = dv / L.R;
   L.nb = (int)((T + kScanBlk - 1) / kScanBlk);
   size_t off = 0;
@@ -310,67 +309,99 @@ __global__ void prep_gen_kernel(const BParams Q) {
 }
 
 // ---------------------------------------------------------------------------
-// Row sweeps F1 / R1. CTA = 4 warps = 16 consecutive state rows of one (batch,
-// head); warp w owns rows j0 + 4w .. j0 + 4w + 3 and lane l key channels
-// 4l..4l+3, so a row's reduction over key channels stays inside its warp.
-// The per-token vectors are staged through shared memory kLC tokens at a
-// time with cp.async, double-buffered.
+// Row sweeps F1 / R1. CTA = 4 warps = 32 consecutive state rows of one (batch,
+// head); in warp w, lanes 4p .. 4p + 3 share row j0 + 8w + p and lane 4p + s
+// holds key channels s CPL .. s CPL + CPL - 1 (CPL = 8, 16 or 32 by d_k), so a
+// row's reduction over key channels is two shuffles. The per-token vectors are
+// staged through shared memory kLC tokens at a time with cp.async (double
+// buffered), each vector as four CPL-float segments kSegPad floats apart so
+// that the four segments a warp reads at once fall in different banks; key
+// channels >= d_k and rows >= d_v are staged as zeros.
+constexpr int kRowsF = 32;   // state rows per CTA
+constexpr int kSegPad = 4;   // floats of padding after each staged segment
 
-// Sums each of the four rows' partials over the warp; every lane gets all
-// four sums. Rows are transposed across lane halves and quarters first, so
-// the four sums take 10 shuffles instead of 20 (fixed order: deterministic).
-__device__ __forceinline__ void rowsum4(const float (&p)[4], float (&y)[4], int lane) {
-  const bool h16 = lane & 16, h8 = lane & 8;
-  float a0 = h16 ? p[2] : p[0], a1 = h16 ? p[3] : p[1];
-  const float b0 = h16 ? p[0] : p[2], b1 = h16 ? p[1] : p[3];
-  a0 += __shfl_xor_sync(0xffffffffu, b0, 16);
-  a1 += __shfl_xor_sync(0xffffffffu, b1, 16);
-  float k = h8 ? a1 : a0;
-  const float s = h8 ? a0 : a1;
-  k += __shfl_xor_sync(0xffffffffu, s, 8);
-  k += __shfl_xor_sync(0xffffffffu, k, 4);
-  k += __shfl_xor_sync(0xffffffffu, k, 2);
-  k += __shfl_xor_sync(0xffffffffu, k, 1);
-  // lane holds row 2 * h16 + h8, i.e. row m sits in lane 8m
-#pragma unroll
-  for (int m = 0; m < 4; ++m) y[m] = __shfl_sync(0xffffffffu, k, 8 * m);
-}
-
-__device__ __forceinline__ float pick4(const float (&v)[4], int i) {
-  return i == 0 ? v[0] : i == 1 ? v[1] : i == 2 ? v[2] : v[3];
-}
 __device__ __forceinline__ void ld4(const float *p, bool ok, float (&v)[4]) {
   const float4 x = ok ? *reinterpret_cast<const float4 *>(p) : make_float4(0.f, 0.f, 0.f, 0.f);
   v[0] = x.x; v[1] = x.y; v[2] = x.z; v[3] = x.w;
 }
 
+// Stages `nvec` consecutive d_k-vectors starting at `src` into the padded
+// segment layout at dst (one 16-byte piece per call; piece k < nvec CPL).
+template <int CPL>
+__device__ __forceinline__ void stage_vec_piece(const float *src, int dk, int k, float *dst) {
+  const int v = k / CPL, c = 4 * (k % CPL);  // vector, first key channel of the piece
+  const int col = c;                          // channels c .. c + 3 of vector v
+  const int seg = col / CPL, off = col % CPL;
+  cp_async16(smem_u32(dst + v * 4 * (CPL + kSegPad) + seg * (CPL + kSegPad) + off),
+             src + (size_t)v * dk + (col < dk ? col : 0), col < dk);
+}
+
+// The dO entries of rows j0 .. j0 + nrow - 1 of token t (raw dtype), one
+// 16-byte piece; rows >= d_v are zero-filled.
+template <typename Tin>
+__device__ __forceinline__ void stage_dO(const BParams &Q, int bh, int t, int j0, int part,
+                                         float *dst) {
+  const KParams &P = Q.P;
+  constexpr int per = 16 / (int)sizeof(Tin);  // rows per piece
+  const bool ok = j0 + per * part < P.dv;
+  const char *src = reinterpret_cast<const char *>(Q.dO) +
+                    (tok_index(P, bh / P.H, t, bh % P.H) * P.dv + (ok ? j0 + per * part : 0)) *
+                        sizeof(Tin);
+  cp_async16(smem_u32(reinterpret_cast<char *>(dst) + 16 * part), src, ok);
+}
+
+template <typename Tin>
+__device__ __forceinline__ float ld_row(const float *base, int j);
+template <>
+__device__ __forceinline__ float ld_row<float>(const float *base, int j) {
+  return base[j];
+}
+template <>
+__device__ __forceinline__ float ld_row<__nv_bfloat16>(const float *base, int j) {
+  return __bfloat162float(reinterpret_cast<const __nv_bfloat16 *>(base)[j]);
+}
+
 // F1: the forward recurrence, writing delta_t of every row, and S_T.
+template <int CPL>
 __global__ void __launch_bounds__(128) f1_kernel(const BParams Q) {
   extern __shared__ float4 smem4[];
   float *sm = reinterpret_cast<float *>(smem4);
+  constexpr int SS = CPL + kSegPad, VS = 4 * SS;  // segment, vector strides
+  constexpr int TS = 3 * VS + kRowsF;              // r | w | alpha | u of the 32 rows
   const KParams &P = Q.P;
   const int dk = P.dk, dv = P.dv, T = P.T;
-  const int nrg = dv / kRowsF;
+  const int nrg = (dv + kRowsF - 1) / kRowsF;
   const int bh = blockIdx.x / nrg, j0 = (blockIdx.x % nrg) * kRowsF;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, c = 4 * lane;
-  const bool act = c < dk;
-  const int TS = 3 * dk + 16;  // staged floats per token: r | w | alpha | u of the 16 rows
-  const int nv = 3 * dk / 4;   // 16-byte copies of the vectors per token
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int s = lane & 3, rl = 8 * warp + (lane >> 2), j = j0 + rl;  // segment, local row, row
+  const bool rok = j < dv;
   const int nc = (T + kLC - 1) / kLC;
   auto issue = [&](int ch) {
     float *buf = sm + (ch & 1) * kLC * TS;
-    const int t0 = ch * kLC, n = min(kLC, T - t0), per = nv + 4;
-    for (int e = threadIdx.x; e < n * per; e += blockDim.x) {
-      const int tt = e / per, k = e % per;
+    const int t0 = ch * kLC, n = min(kLC, T - t0);
+    for (int tt = 0; tt < n; ++tt) {
       const float *g = gen_at(Q, bh, t0 + tt);
-      const float *src = k < nv ? g + dk + 4 * k : g + 4 * dk + j0 + 4 * (k - nv);
-      cp_async16(smem_u32(buf + tt * TS + 4 * k), src, true);
+      float *d = buf + tt * TS;
+      for (int k = threadIdx.x; k < 3 * CPL + kRowsF / 4; k += blockDim.x) {
+        if (k < 3 * CPL) {
+          stage_vec_piece<CPL>(g + dk, dk, k, d);
+        } else {
+          const int r4 = 4 * (k - 3 * CPL);
+          const bool ok = j0 + r4 < dv;
+          cp_async16(smem_u32(d + 3 * VS + r4), g + 4 * dk + (ok ? j0 + r4 : 0), ok);
+        }
+      }
     }
   };
-  float S[4][4];
+  float S[CPL];
 #pragma unroll
-  for (int m = 0; m < 4; ++m)
-    ld4(P.S0 ? P.S0 + ((size_t)bh * dv + j0 + 4 * warp + m) * dk + c : nullptr, act && P.S0, S[m]);
+  for (int e = 0; e < CPL; e += 4) {
+    const int col = s * CPL + e;
+    float v[4];
+    ld4(rok && P.S0 && col < dk ? P.S0 + ((size_t)bh * dv + j) * dk + col : nullptr,
+        rok && P.S0 && col < dk, v);
+    S[e] = v[0]; S[e + 1] = v[1]; S[e + 2] = v[2]; S[e + 3] = v[3];
+  }
   issue(0);
   cp_async_commit();
   for (int ch = 0; ch < nc; ++ch) {
@@ -381,42 +412,141 @@ __global__ void __launch_bounds__(128) f1_kernel(const BParams Q) {
     const float *buf = sm + (ch & 1) * kLC * TS;
     const int t0 = ch * kLC, n = min(kLC, T - t0);
     for (int tt = 0; tt < n; ++tt) {
-      const float *sv = buf + tt * TS;
-      float r[4], w[4], a[4], u[4], p[4], y[4], d[4];
-      ld4(sv + c, act, r);
-      ld4(sv + dk + c, act, w);
-      ld4(sv + 2 * dk + c, act, a);
-      ld4(sv + 3 * dk + 4 * warp, true, u);
+      const float *sv = buf + tt * TS + s * SS;
+      float y[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int m = 0; m < 4; ++m) {
-        p[m] = 0.f;
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          S[m][e] *= a[e];
-          p[m] = fmaf(S[m][e], r[e], p[m]);
-        }
+      for (int e = 0; e < CPL; e += 4) {
+        const float4 r = *reinterpret_cast<const float4 *>(sv + e);
+        const float4 a = *reinterpret_cast<const float4 *>(sv + 2 * VS + e);
+        S[e] *= a.x; S[e + 1] *= a.y; S[e + 2] *= a.z; S[e + 3] *= a.w;
+        y[0] = fmaf(S[e], r.x, y[0]);
+        y[1] = fmaf(S[e + 1], r.y, y[1]);
+        y[2] = fmaf(S[e + 2], r.z, y[2]);
+        y[3] = fmaf(S[e + 3], r.w, y[3]);
       }
-      rowsum4(p, y, lane);
+      float yy = (y[0] + y[1]) + (y[2] + y[3]);
+      yy += __shfl_xor_sync(0xffffffffu, yy, 1);
+      yy += __shfl_xor_sync(0xffffffffu, yy, 2);
+      const float d = buf[tt * TS + 3 * VS + rl] - yy;
 #pragma unroll
-      for (int m = 0; m < 4; ++m) {
-        d[m] = u[m] - y[m];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) S[m][e] = fmaf(d[m], w[e], S[m][e]);
+      for (int e = 0; e < CPL; e += 4) {
+        const float4 w = *reinterpret_cast<const float4 *>(sv + VS + e);
+        S[e] = fmaf(d, w.x, S[e]);
+        S[e + 1] = fmaf(d, w.y, S[e + 1]);
+        S[e + 2] = fmaf(d, w.z, S[e + 2]);
+        S[e + 3] = fmaf(d, w.w, S[e + 3]);
       }
-      if (lane < 4)
-        Q.delta[((size_t)bh * T + t0 + tt) * dv + j0 + 4 * warp + lane] = pick4(d, lane);
+      if (s == 0 && rok) Q.delta[((size_t)bh * T + t0 + tt) * dv + j] = d;
     }
     __syncthreads();  // the buffer is refilled two chunks on
   }
-  if (act) {
+  if (rok) {
 #pragma unroll
-    for (int m = 0; m < 4; ++m)
-      *reinterpret_cast<float4 *>(Q.st + ((size_t)bh * dv + j0 + 4 * warp + m) * dk + c) =
-          make_float4(S[m][0], S[m][1], S[m][2], S[m][3]);
+    for (int e = 0; e < CPL; e += 4) {
+      const int col = s * CPL + e;
+      if (col < dk)
+        *reinterpret_cast<float4 *>(Q.st + ((size_t)bh * dv + j) * dk + col) =
+            make_float4(S[e], S[e + 1], S[e + 2], S[e + 3]);
+    }
   }
 }
 
-// The four dO entries of rows j..j+3 of a staged token, widened to fp32.
+// R1: the reverse recurrence of the cotangent, writing dd_t of every row, and
+// dS0.
+template <typename Tin, int CPL>
+__global__ void __launch_bounds__(128) r1_kernel(const BParams Q) {
+  extern __shared__ float4 smem4[];
+  float *sm = reinterpret_cast<float *>(smem4);
+  constexpr int SS = CPL + kSegPad, VS = 4 * SS;
+  constexpr int TS = 4 * VS + kRowsF;  // q' | r | w | alpha | dO of the 32 rows (raw)
+  constexpr int ND = kRowsF * (int)sizeof(Tin) / 16;
+  const KParams &P = Q.P;
+  const int dk = P.dk, dv = P.dv, T = P.T;
+  const int nrg = (dv + kRowsF - 1) / kRowsF;
+  const int bh = blockIdx.x / nrg, j0 = (blockIdx.x % nrg) * kRowsF;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int s = lane & 3, rl = 8 * warp + (lane >> 2), j = j0 + rl;
+  const bool rok = j < dv;
+  const float cq = P.q_scale;
+  const int nd = Q.dO ? ND : 0;
+  const int nc = (T + kLC - 1) / kLC;
+  auto issue = [&](int ch) {
+    float *buf = sm + (ch & 1) * kLC * TS;
+    const int t0 = ch * kLC, n = min(kLC, T - t0);
+    for (int tt = 0; tt < n; ++tt) {
+      const float *g = gen_at(Q, bh, t0 + tt);
+      float *d = buf + tt * TS;
+      for (int k = threadIdx.x; k < 4 * CPL + nd; k += blockDim.x) {
+        if (k < 4 * CPL)
+          stage_vec_piece<CPL>(g, dk, k, d);
+        else
+          stage_dO<Tin>(Q, bh, t0 + tt, j0, k - 4 * CPL, d + 4 * VS);
+      }
+    }
+  };
+  float D[CPL];
+#pragma unroll
+  for (int e = 0; e < CPL; e += 4) {
+    const int col = s * CPL + e;
+    float v[4];
+    ld4(rok && Q.dST && col < dk ? Q.dST + ((size_t)bh * dv + j) * dk + col : nullptr,
+        rok && Q.dST && col < dk, v);
+    D[e] = v[0]; D[e + 1] = v[1]; D[e + 2] = v[2]; D[e + 3] = v[3];
+  }
+  if (nc > 0) issue(nc - 1);
+  cp_async_commit();
+  for (int ch = nc - 1; ch >= 0; --ch) {
+    if (ch > 0) issue(ch - 1);
+    cp_async_commit();
+    cp_async_wait_group<1>();
+    __syncthreads();
+    const float *buf = sm + (ch & 1) * kLC * TS;
+    const int t0 = ch * kLC, n = min(kLC, T - t0);
+    for (int tt = n - 1; tt >= 0; --tt) {
+      const float *sv = buf + tt * TS + s * SS;
+      const float cg = Q.dO ? cq * ld_row<Tin>(buf + tt * TS + 4 * VS, rl) : 0.f;
+      float p[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int e = 0; e < CPL; e += 4) {
+        const float4 q = *reinterpret_cast<const float4 *>(sv + e);
+        const float4 w = *reinterpret_cast<const float4 *>(sv + 2 * VS + e);
+        D[e] = fmaf(cg, q.x, D[e]);
+        D[e + 1] = fmaf(cg, q.y, D[e + 1]);
+        D[e + 2] = fmaf(cg, q.z, D[e + 2]);
+        D[e + 3] = fmaf(cg, q.w, D[e + 3]);
+        p[0] = fmaf(D[e], w.x, p[0]);
+        p[1] = fmaf(D[e + 1], w.y, p[1]);
+        p[2] = fmaf(D[e + 2], w.z, p[2]);
+        p[3] = fmaf(D[e + 3], w.w, p[3]);
+      }
+      float dd = (p[0] + p[1]) + (p[2] + p[3]);
+      dd += __shfl_xor_sync(0xffffffffu, dd, 1);
+      dd += __shfl_xor_sync(0xffffffffu, dd, 2);
+#pragma unroll
+      for (int e = 0; e < CPL; e += 4) {
+        const float4 r = *reinterpret_cast<const float4 *>(sv + VS + e);
+        const float4 a = *reinterpret_cast<const float4 *>(sv + 3 * VS + e);
+        D[e] = fmaf(-dd, r.x, D[e]) * a.x;
+        D[e + 1] = fmaf(-dd, r.y, D[e + 1]) * a.y;
+        D[e + 2] = fmaf(-dd, r.z, D[e + 2]) * a.z;
+        D[e + 3] = fmaf(-dd, r.w, D[e + 3]) * a.w;
+      }
+      if (s == 0 && rok) Q.dd[((size_t)bh * T + t0 + tt) * dv + j] = dd;
+    }
+    __syncthreads();
+  }
+  if (rok && Q.dS0) {
+#pragma unroll
+    for (int e = 0; e < CPL; e += 4) {
+      const int col = s * CPL + e;
+      if (col < dk)
+        *reinterpret_cast<float4 *>(Q.dS0 + ((size_t)bh * dv + j) * dk + col) =
+            make_float4(D[e], D[e + 1], D[e + 2], D[e + 3]);
+    }
+  }
+}
+
+// Four consecutive staged dO rows from j, widened to fp32.
 template <typename Tin>
 __device__ __forceinline__ void ld_rows4(const float *sv, int j, float (&v)[4]);
 template <>
@@ -429,99 +559,6 @@ __device__ __forceinline__ void ld_rows4<__nv_bfloat16>(const float *sv, int j, 
   const uint2 x = *reinterpret_cast<const uint2 *>(reinterpret_cast<const __nv_bfloat16 *>(sv) + j);
   v[0] = __uint_as_float(x.x << 16); v[1] = __uint_as_float(x.x & 0xffff0000u);
   v[2] = __uint_as_float(x.y << 16); v[3] = __uint_as_float(x.y & 0xffff0000u);
-}
-
-// Stages the dO entries of rows j0 .. j0 + nrow - 1 of token t (raw dtype) at
-// dst; `part` selects one 16-byte piece.
-template <typename Tin>
-__device__ __forceinline__ void stage_dO(const BParams &Q, int bh, int t, int j0, int part,
-                                         float *dst) {
-  const KParams &P = Q.P;
-  const char *src = reinterpret_cast<const char *>(Q.dO) +
-                    (tok_index(P, bh / P.H, t, bh % P.H) * P.dv + j0) * sizeof(Tin) + 16 * part;
-  cp_async16(smem_u32(reinterpret_cast<char *>(dst) + 16 * part), src, true);
-}
-
-// R1: the reverse recurrence of the cotangent, writing dd_t of every row, and
-// dS0.
-template <typename Tin>
-__global__ void __launch_bounds__(128) r1_kernel(const BParams Q) {
-  extern __shared__ float4 smem4[];
-  float *sm = reinterpret_cast<float *>(smem4);
-  const KParams &P = Q.P;
-  const int dk = P.dk, dv = P.dv, T = P.T;
-  const int nrg = dv / kRowsF;
-  const int bh = blockIdx.x / nrg, j0 = (blockIdx.x % nrg) * kRowsF;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, c = 4 * lane;
-  const bool act = c < dk;
-  const float cq = P.q_scale;
-  const int TS = 4 * dk + 16;  // staged floats per token: q' | r | w | alpha | dO of the 16 rows
-  const int nv = dk;           // 16-byte copies of the vectors per token
-  const int nd = Q.dO ? kRowsF * (int)sizeof(Tin) / 16 : 0;
-  const int nc = (T + kLC - 1) / kLC;
-  auto issue = [&](int ch) {
-    float *buf = sm + (ch & 1) * kLC * TS;
-    const int t0 = ch * kLC, n = min(kLC, T - t0), per = nv + nd;
-    for (int e = threadIdx.x; e < n * per; e += blockDim.x) {
-      const int tt = e / per, k = e % per;
-      if (k < nv)
-        cp_async16(smem_u32(buf + tt * TS + 4 * k), gen_at(Q, bh, t0 + tt) + 4 * k, true);
-      else
-        stage_dO<Tin>(Q, bh, t0 + tt, j0, k - nv, buf + tt * TS + 4 * dk);
-    }
-  };
-  float D[4][4];
-#pragma unroll
-  for (int m = 0; m < 4; ++m)
-    ld4(Q.dST ? Q.dST + ((size_t)bh * dv + j0 + 4 * warp + m) * dk + c : nullptr, act && Q.dST,
-        D[m]);
-  if (nc > 0) issue(nc - 1);
-  cp_async_commit();
-  for (int ch = nc - 1; ch >= 0; --ch) {
-    if (ch > 0) issue(ch - 1);
-    cp_async_commit();
-    cp_async_wait_group<1>();
-    __syncthreads();
-    const float *buf = sm + (ch & 1) * kLC * TS;
-    const int t0 = ch * kLC, n = min(kLC, T - t0);
-    for (int tt = n - 1; tt >= 0; --tt) {
-      const float *sv = buf + tt * TS;
-      float q[4], r[4], w[4], a[4], g[4], p[4], dd[4];
-      ld4(sv + c, act, q);
-      ld4(sv + dk + c, act, r);
-      ld4(sv + 2 * dk + c, act, w);
-      ld4(sv + 3 * dk + c, act, a);
-      if (Q.dO) {
-        ld_rows4<Tin>(sv + 4 * dk, 4 * warp, g);
-      } else {
-        g[0] = g[1] = g[2] = g[3] = 0.f;
-      }
-#pragma unroll
-      for (int m = 0; m < 4; ++m) {
-        const float cg = cq * g[m];
-        p[m] = 0.f;
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          D[m][e] = fmaf(cg, q[e], D[m][e]);
-          p[m] = fmaf(D[m][e], w[e], p[m]);
-        }
-      }
-      rowsum4(p, dd, lane);
-#pragma unroll
-      for (int m = 0; m < 4; ++m) {
-#pragma unroll
-        for (int e = 0; e < 4; ++e) D[m][e] = fmaf(-dd[m], r[e], D[m][e]) * a[e];
-      }
-      if (lane < 4) Q.dd[((size_t)bh * T + t0 + tt) * dv + j0 + 4 * warp + lane] = pick4(dd, lane);
-    }
-    __syncthreads();
-  }
-  if (act && Q.dS0) {
-#pragma unroll
-    for (int m = 0; m < 4; ++m)
-      *reinterpret_cast<float4 *>(Q.dS0 + ((size_t)bh * dv + j0 + 4 * warp + m) * dk + c) =
-          make_float4(D[m][0], D[m][1], D[m][2], D[m][3]);
-  }
 }
 
 // ---------------------------------------------------------------------------
@@ -553,8 +590,9 @@ __global__ void __launch_bounds__(128) f2_kernel(const BParams Q) {
   auto issue = [&](int ch) {
     float *buf = sm + (ch & 1) * kLC * TS;
     const int t0 = ch * kLC, n = min(kLC, T - t0), per = nv + 2 * nr + nd;
-    for (int e = threadIdx.x; e < n * per; e += blockDim.x) {
-      const int tt = e / per, k = e % per, t = t0 + tt;
+    for (int tt = 0; tt < n; ++tt)
+    for (int k = threadIdx.x; k < per; k += blockDim.x) {
+      const int t = t0 + tt;
       float *d = buf + tt * TS;
       if (k < nv)
         cp_async16(smem_u32(d + 4 * k), gen_at(Q, bh, t) + 2 * dk + 4 * k, true);
@@ -625,8 +663,9 @@ __global__ void __launch_bounds__(128) r2_kernel(const BParams Q) {
   auto issue = [&](int ch) {
     float *buf = sm + (ch & 1) * kLC * TS;
     const int t0 = ch * kLC, n = min(kLC, T - t0), per = nv + 2 * nr + nd;
-    for (int e = threadIdx.x; e < n * per; e += blockDim.x) {
-      const int tt = e / per, k = e % per, t = t0 + tt;
+    for (int tt = 0; tt < n; ++tt)
+    for (int k = threadIdx.x; k < per; k += blockDim.x) {
+      const int t = t0 + tt;
       float *d = buf + tt * TS;
       if (k < nv)
         cp_async16(smem_u32(d + 4 * k), gen_at(Q, bh, t) + 4 * k, true);
@@ -908,7 +947,7 @@ cudaError_t set_smem(K kernel, size_t bytes) {
   return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
 }
 
-template <typename Tin, int R>
+template <typename Tin, int R, int CPL>
 cudaError_t launch_bwd_t(const BParams &Q, cudaStream_t st) {
   const KParams &P = Q.P;
   const int dk = P.dk, dv = P.dv;
@@ -921,18 +960,19 @@ cudaError_t launch_bwd_t(const BParams &Q, cudaStream_t st) {
   }
   prep_gen_kernel<Tin><<<grid_for(BHT * 32, 256), 256, 0, st>>>(Q);
 
-  const size_t sm_f1 = 2 * kLC * (3 * dk + 16) * sizeof(float);
-  const size_t sm_r1 = 2 * kLC * (4 * dk + 16) * sizeof(float);
+  constexpr int SS = CPL + kSegPad;
+  const size_t sm_f1 = 2 * kLC * (3 * 4 * SS + kRowsF) * sizeof(float);
+  const size_t sm_r1 = 2 * kLC * (4 * 4 * SS + kRowsF) * sizeof(float);
   const size_t sm_f2 = 2 * kLC * (2 * dk + 3 * R) * sizeof(float);
   const size_t sm_r2 = 2 * kLC * (4 * dk + 3 * R) * sizeof(float);
-  if ((err = set_smem(f1_kernel, sm_f1)) != cudaSuccess) return err;
-  if ((err = set_smem(r1_kernel<Tin>, sm_r1)) != cudaSuccess) return err;
+  if ((err = set_smem(f1_kernel<CPL>, sm_f1)) != cudaSuccess) return err;
+  if ((err = set_smem(r1_kernel<Tin, CPL>, sm_r1)) != cudaSuccess) return err;
   if ((err = set_smem(f2_kernel<Tin, R>, sm_f2)) != cudaSuccess) return err;
   if ((err = set_smem(r2_kernel<Tin, R>, sm_r2)) != cudaSuccess) return err;
-  const unsigned grid_rows = (unsigned)(BH * (dv / kRowsF));
+  const unsigned grid_rows = (unsigned)(BH * ((dv + kRowsF - 1) / kRowsF));
   const unsigned grid_cols = (unsigned)(BH * Q.G);
-  f1_kernel<<<grid_rows, 128, sm_f1, st>>>(Q);
-  r1_kernel<Tin><<<grid_rows, 128, sm_r1, st>>>(Q);
+  f1_kernel<CPL><<<grid_rows, 128, sm_f1, st>>>(Q);
+  r1_kernel<Tin, CPL><<<grid_rows, 128, sm_r1, st>>>(Q);
   f2_kernel<Tin, R><<<grid_cols, dk, sm_f2, st>>>(Q);
   r2_kernel<Tin, R><<<grid_cols, dk, sm_r2, st>>>(Q);
   e1_kernel<Tin><<<grid_for(BHT * 32, 256), 256, 0, st>>>(Q);
@@ -952,6 +992,18 @@ cudaError_t launch_bwd_t(const BParams &Q, cudaStream_t st) {
     if (Q.dk) e3_kernel<Tin><<<grid_for(BHT * dk, 256), 256, 0, st>>>(Q);
   }
   return cudaGetLastError();
+}
+
+template <typename Tin>
+cudaError_t launch_bwd_d(const BParams &Q, int R, int cpl, cudaStream_t st) {
+  if (R == 32) {
+    if (cpl == 32) return launch_bwd_t<Tin, 32, 32>(Q, st);
+    if (cpl == 16) return launch_bwd_t<Tin, 32, 16>(Q, st);
+    return launch_bwd_t<Tin, 32, 8>(Q, st);
+  }
+  if (cpl == 32) return launch_bwd_t<Tin, 16, 32>(Q, st);
+  if (cpl == 16) return launch_bwd_t<Tin, 16, 16>(Q, st);
+  return launch_bwd_t<Tin, 16, 8>(Q, st);
 }
 
 }  // namespace
@@ -986,9 +1038,10 @@ cudaError_t launch_chunk_bwd(const KParams &P, const pdn_grads_t *g, void *works
   Q.st = ws + L.st; Q.part = ws + L.part; Q.cpsi = ws + L.cpsi; Q.sigma = ws + L.sigma;
   Q.dacc = ws + L.dacc; Q.bsum = ws + L.bsum; Q.phi = ws + L.phi;
   Q.GS = L.GS; Q.R = L.R; Q.G = L.G; Q.nb = L.nb;
-  const bool bf = P.dtype == PDN_BF16;
-  if (L.R == 32) return bf ? launch_bwd_t<__nv_bfloat16, 32>(Q, stream) : launch_bwd_t<float, 32>(Q, stream);
-  return bf ? launch_bwd_t<__nv_bfloat16, 16>(Q, stream) : launch_bwd_t<float, 16>(Q, stream);
+  // key channels per lane in the row sweeps: 4 lanes cover d_k
+  const int cpl = P.dk <= 32 ? 8 : P.dk <= 64 ? 16 : 32;
+  if (P.dtype == PDN_BF16) return launch_bwd_d<__nv_bfloat16>(Q, L.R, cpl, stream);
+  return launch_bwd_d<float>(Q, L.R, cpl, stream);
 }
 
 }  // namespace pdn
