@@ -309,30 +309,36 @@ __global__ void prep_gen_kernel(const BParams Q) {
 }
 
 // ---------------------------------------------------------------------------
-// Row sweeps F1 / R1. CTA = 4 warps = 32 consecutive state rows of one (batch,
-// head); in warp w, lanes 4p .. 4p + 3 share row j0 + 8w + p and lane 4p + s
-// holds key channels s CPL .. s CPL + CPL - 1 (CPL = 8, 16 or 32 by d_k), so a
-// row's reduction over key channels is two shuffles. The per-token vectors are
-// staged through shared memory kLC tokens at a time with cp.async (double
-// buffered), each vector as four CPL-float segments kSegPad floats apart so
-// that the four segments a warp reads at once fall in different banks; key
-// channels >= d_k and rows >= d_v are staged as zeros.
-constexpr int kRowsF = 32;   // state rows per CTA
-constexpr int kSegPad = 4;   // floats of padding after each staged segment
+// Row sweeps F1 / R1. CTA = 4 warps = 16 consecutive state rows of one (batch,
+// head); in warp w, lanes 8p .. 8p + 7 share row j0 + 4w + p and lane 8p + s
+// holds key channels s CPL .. s CPL + CPL - 1 (CPL = 4, 8 or 16 by d_k), so a
+// row's reduction over key channels is three shuffles. The sequential chain
+// per token is short and there are many warps to interleave (the sweeps are
+// latency bound: one token after the other). The per-token vectors are
+// staged through shared memory kLCR tokens at a time with cp.async (double
+// buffered), each vector as eight CPL-float segments seg_stride(CPL) floats
+// apart, an odd multiple of four, so that the eight segments a quarter-warp
+// reads at once fall in different banks; key channels >= d_k are staged as
+// zeros.
+constexpr int kRowsF = 16;   // state rows per CTA
+constexpr int kLPR = 8;      // lanes per state row
+constexpr int kLCR = 8;      // tokens staged per chunk in F1 / R1
+__host__ __device__ constexpr int seg_stride(int cpl) { return cpl % 8 == 0 ? cpl + 4 : cpl; }
 
 __device__ __forceinline__ void ld4(const float *p, bool ok, float (&v)[4]) {
   const float4 x = ok ? *reinterpret_cast<const float4 *>(p) : make_float4(0.f, 0.f, 0.f, 0.f);
   v[0] = x.x; v[1] = x.y; v[2] = x.z; v[3] = x.w;
 }
 
-// Stages `nvec` consecutive d_k-vectors starting at `src` into the padded
-// segment layout at dst (one 16-byte piece per call; piece k < nvec CPL).
+// Stages consecutive d_k-vectors starting at `src` into the padded segment
+// layout at dst, one 16-byte piece per call (piece k: vector k / (2 CPL),
+// key channels 4 (k % (2 CPL)) .. + 3).
 template <int CPL>
 __device__ __forceinline__ void stage_vec_piece(const float *src, int dk, int k, float *dst) {
-  const int v = k / CPL, c = 4 * (k % CPL);  // vector, first key channel of the piece
-  const int col = c;                          // channels c .. c + 3 of vector v
+  constexpr int SS = seg_stride(CPL), PV = kLPR * CPL / 4;  // pieces per vector
+  const int v = k / PV, col = 4 * (k % PV);
   const int seg = col / CPL, off = col % CPL;
-  cp_async16(smem_u32(dst + v * 4 * (CPL + kSegPad) + seg * (CPL + kSegPad) + off),
+  cp_async16(smem_u32(dst + v * kLPR * SS + seg * SS + off),
              src + (size_t)v * dk + (col < dk ? col : 0), col < dk);
 }
 
@@ -366,27 +372,27 @@ template <int CPL>
 __global__ void __launch_bounds__(128) f1_kernel(const BParams Q) {
   extern __shared__ float4 smem4[];
   float *sm = reinterpret_cast<float *>(smem4);
-  constexpr int SS = CPL + kSegPad, VS = 4 * SS;  // segment, vector strides
-  constexpr int TS = 3 * VS + kRowsF;              // r | w | alpha | u of the 32 rows
+  constexpr int SS = seg_stride(CPL), VS = kLPR * SS;  // segment, vector strides
+  constexpr int TS = 3 * VS + kRowsF;                   // r | w | alpha | u of the 16 rows
   const KParams &P = Q.P;
   const int dk = P.dk, dv = P.dv, T = P.T;
   const int nrg = (dv + kRowsF - 1) / kRowsF;
   const int bh = blockIdx.x / nrg, j0 = (blockIdx.x % nrg) * kRowsF;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int s = lane & 3, rl = 8 * warp + (lane >> 2), j = j0 + rl;  // segment, local row, row
+  const int s = lane & 7, rl = 4 * warp + (lane >> 3), j = j0 + rl;  // segment, local row, row
   const bool rok = j < dv;
-  const int nc = (T + kLC - 1) / kLC;
+  const int nc = (T + kLCR - 1) / kLCR;
   auto issue = [&](int ch) {
-    float *buf = sm + (ch & 1) * kLC * TS;
-    const int t0 = ch * kLC, n = min(kLC, T - t0);
+    float *buf = sm + (ch & 1) * kLCR * TS;
+    const int t0 = ch * kLCR, n = min(kLCR, T - t0);
     for (int tt = 0; tt < n; ++tt) {
       const float *g = gen_at(Q, bh, t0 + tt);
       float *d = buf + tt * TS;
-      for (int k = threadIdx.x; k < 3 * CPL + kRowsF / 4; k += blockDim.x) {
-        if (k < 3 * CPL) {
+      for (int k = threadIdx.x; k < 6 * CPL + kRowsF / 4; k += blockDim.x) {
+        if (k < 6 * CPL) {
           stage_vec_piece<CPL>(g + dk, dk, k, d);
         } else {
-          const int r4 = 4 * (k - 3 * CPL);
+          const int r4 = 4 * (k - 6 * CPL);
           const bool ok = j0 + r4 < dv;
           cp_async16(smem_u32(d + 3 * VS + r4), g + 4 * dk + (ok ? j0 + r4 : 0), ok);
         }
@@ -409,8 +415,8 @@ __global__ void __launch_bounds__(128) f1_kernel(const BParams Q) {
     cp_async_commit();
     cp_async_wait_group<1>();
     __syncthreads();
-    const float *buf = sm + (ch & 1) * kLC * TS;
-    const int t0 = ch * kLC, n = min(kLC, T - t0);
+    const float *buf = sm + (ch & 1) * kLCR * TS;
+    const int t0 = ch * kLCR, n = min(kLCR, T - t0);
     for (int tt = 0; tt < n; ++tt) {
       const float *sv = buf + tt * TS + s * SS;
       float y[4] = {0.f, 0.f, 0.f, 0.f};
@@ -427,6 +433,7 @@ __global__ void __launch_bounds__(128) f1_kernel(const BParams Q) {
       float yy = (y[0] + y[1]) + (y[2] + y[3]);
       yy += __shfl_xor_sync(0xffffffffu, yy, 1);
       yy += __shfl_xor_sync(0xffffffffu, yy, 2);
+      yy += __shfl_xor_sync(0xffffffffu, yy, 4);
       const float d = buf[tt * TS + 3 * VS + rl] - yy;
 #pragma unroll
       for (int e = 0; e < CPL; e += 4) {
@@ -457,30 +464,30 @@ template <typename Tin, int CPL>
 __global__ void __launch_bounds__(128) r1_kernel(const BParams Q) {
   extern __shared__ float4 smem4[];
   float *sm = reinterpret_cast<float *>(smem4);
-  constexpr int SS = CPL + kSegPad, VS = 4 * SS;
-  constexpr int TS = 4 * VS + kRowsF;  // q' | r | w | alpha | dO of the 32 rows (raw)
+  constexpr int SS = seg_stride(CPL), VS = kLPR * SS;
+  constexpr int TS = 4 * VS + kRowsF;  // q' | r | w | alpha | dO of the 16 rows (raw)
   constexpr int ND = kRowsF * (int)sizeof(Tin) / 16;
   const KParams &P = Q.P;
   const int dk = P.dk, dv = P.dv, T = P.T;
   const int nrg = (dv + kRowsF - 1) / kRowsF;
   const int bh = blockIdx.x / nrg, j0 = (blockIdx.x % nrg) * kRowsF;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int s = lane & 3, rl = 8 * warp + (lane >> 2), j = j0 + rl;
+  const int s = lane & 7, rl = 4 * warp + (lane >> 3), j = j0 + rl;
   const bool rok = j < dv;
   const float cq = P.q_scale;
   const int nd = Q.dO ? ND : 0;
-  const int nc = (T + kLC - 1) / kLC;
+  const int nc = (T + kLCR - 1) / kLCR;
   auto issue = [&](int ch) {
-    float *buf = sm + (ch & 1) * kLC * TS;
-    const int t0 = ch * kLC, n = min(kLC, T - t0);
+    float *buf = sm + (ch & 1) * kLCR * TS;
+    const int t0 = ch * kLCR, n = min(kLCR, T - t0);
     for (int tt = 0; tt < n; ++tt) {
       const float *g = gen_at(Q, bh, t0 + tt);
       float *d = buf + tt * TS;
-      for (int k = threadIdx.x; k < 4 * CPL + nd; k += blockDim.x) {
-        if (k < 4 * CPL)
+      for (int k = threadIdx.x; k < 8 * CPL + nd; k += blockDim.x) {
+        if (k < 8 * CPL)
           stage_vec_piece<CPL>(g, dk, k, d);
         else
-          stage_dO<Tin>(Q, bh, t0 + tt, j0, k - 4 * CPL, d + 4 * VS);
+          stage_dO<Tin>(Q, bh, t0 + tt, j0, k - 8 * CPL, d + 4 * VS);
       }
     }
   };
@@ -500,8 +507,8 @@ __global__ void __launch_bounds__(128) r1_kernel(const BParams Q) {
     cp_async_commit();
     cp_async_wait_group<1>();
     __syncthreads();
-    const float *buf = sm + (ch & 1) * kLC * TS;
-    const int t0 = ch * kLC, n = min(kLC, T - t0);
+    const float *buf = sm + (ch & 1) * kLCR * TS;
+    const int t0 = ch * kLCR, n = min(kLCR, T - t0);
     for (int tt = n - 1; tt >= 0; --tt) {
       const float *sv = buf + tt * TS + s * SS;
       const float cg = Q.dO ? cq * ld_row<Tin>(buf + tt * TS + 4 * VS, rl) : 0.f;
@@ -522,6 +529,7 @@ __global__ void __launch_bounds__(128) r1_kernel(const BParams Q) {
       float dd = (p[0] + p[1]) + (p[2] + p[3]);
       dd += __shfl_xor_sync(0xffffffffu, dd, 1);
       dd += __shfl_xor_sync(0xffffffffu, dd, 2);
+      dd += __shfl_xor_sync(0xffffffffu, dd, 4);
 #pragma unroll
       for (int e = 0; e < CPL; e += 4) {
         const float4 r = *reinterpret_cast<const float4 *>(sv + VS + e);
@@ -960,9 +968,9 @@ cudaError_t launch_bwd_t(const BParams &Q, cudaStream_t st) {
   }
   prep_gen_kernel<Tin><<<grid_for(BHT * 32, 256), 256, 0, st>>>(Q);
 
-  constexpr int SS = CPL + kSegPad;
-  const size_t sm_f1 = 2 * kLC * (3 * 4 * SS + kRowsF) * sizeof(float);
-  const size_t sm_r1 = 2 * kLC * (4 * 4 * SS + kRowsF) * sizeof(float);
+  constexpr int VS = kLPR * seg_stride(CPL);
+  const size_t sm_f1 = 2 * kLCR * (3 * VS + kRowsF) * sizeof(float);
+  const size_t sm_r1 = 2 * kLCR * (4 * VS + kRowsF) * sizeof(float);
   const size_t sm_f2 = 2 * kLC * (2 * dk + 3 * R) * sizeof(float);
   const size_t sm_r2 = 2 * kLC * (4 * dk + 3 * R) * sizeof(float);
   if ((err = set_smem(f1_kernel<CPL>, sm_f1)) != cudaSuccess) return err;
@@ -997,13 +1005,13 @@ cudaError_t launch_bwd_t(const BParams &Q, cudaStream_t st) {
 template <typename Tin>
 cudaError_t launch_bwd_d(const BParams &Q, int R, int cpl, cudaStream_t st) {
   if (R == 32) {
-    if (cpl == 32) return launch_bwd_t<Tin, 32, 32>(Q, st);
     if (cpl == 16) return launch_bwd_t<Tin, 32, 16>(Q, st);
-    return launch_bwd_t<Tin, 32, 8>(Q, st);
+    if (cpl == 8) return launch_bwd_t<Tin, 32, 8>(Q, st);
+    return launch_bwd_t<Tin, 32, 4>(Q, st);
   }
-  if (cpl == 32) return launch_bwd_t<Tin, 16, 32>(Q, st);
   if (cpl == 16) return launch_bwd_t<Tin, 16, 16>(Q, st);
-  return launch_bwd_t<Tin, 16, 8>(Q, st);
+  if (cpl == 8) return launch_bwd_t<Tin, 16, 8>(Q, st);
+  return launch_bwd_t<Tin, 16, 4>(Q, st);
 }
 
 }  // namespace
@@ -1038,8 +1046,8 @@ cudaError_t launch_chunk_bwd(const KParams &P, const pdn_grads_t *g, void *works
   Q.st = ws + L.st; Q.part = ws + L.part; Q.cpsi = ws + L.cpsi; Q.sigma = ws + L.sigma;
   Q.dacc = ws + L.dacc; Q.bsum = ws + L.bsum; Q.phi = ws + L.phi;
   Q.GS = L.GS; Q.R = L.R; Q.G = L.G; Q.nb = L.nb;
-  // key channels per lane in the row sweeps: 4 lanes cover d_k
-  const int cpl = P.dk <= 32 ? 8 : P.dk <= 64 ? 16 : 32;
+  // key channels per lane in the row sweeps: 8 lanes cover d_k
+  const int cpl = P.dk <= 32 ? 4 : P.dk <= 64 ? 8 : 16;
   if (P.dtype == PDN_BF16) return launch_bwd_d<__nv_bfloat16>(Q, L.R, cpl, stream);
   return launch_bwd_d<float>(Q, L.R, cpl, stream);
 }
