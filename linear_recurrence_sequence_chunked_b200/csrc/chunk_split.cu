@@ -662,14 +662,16 @@ __global__ void __launch_bounds__(kK1Threads, kDecay == PDN_DECAY_CHANNEL ? 1 : 
       ss += __shfl_xor_sync(0xffffffffu, ss, 16);
       qs *= inv_norm(ss);
     }
-#pragma unroll
+    // channel decay: one copy of the (long) body, not four, so that the
+    // kernel's straight-line code stays within the instruction cache
+#pragma unroll(kCh ? 1 : 4)
     for (int m = 0; m < 4; ++m) {
       const int c8 = 4 * m + (lane >> 3);
       const int i0 = 8 * c8;
       float kf[8], qf[8], vf[8], r[8], w[8];
       unpack8(*reinterpret_cast<const uint4 *>(smem + L::kKS + t * KS_LD + c8 * 16), kf);
       unpack8(*reinterpret_cast<const uint4 *>(smem + L::kQS + t * KS_LD + c8 * 16), qf);
-      unpack8(vcur[m], vf);
+      unpack8(m == 0 ? vcur[0] : m == 1 ? vcur[1] : m == 2 ? vcur[2] : vcur[3], vf);
 #pragma unroll
       for (int e = 0; e < 8; ++e) qf[e] *= qs;
       if (kPre) {
