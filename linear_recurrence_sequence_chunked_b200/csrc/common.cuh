@@ -84,15 +84,24 @@ __device__ __forceinline__ float precond_coef(float logA, float mu, float lnx) {
 __device__ __forceinline__ float softplus_f(float x) {
   return fmaxf(x, 0.f) + log1pf(expf(-fabsf(x)));
 }
+// The activations themselves live out of line: the kernels call them per
+// element inside fully unrolled loops, and inlined copies of expf / log1pf
+// there would multiply the code every block has to fetch even when the
+// prologue is off (a uniform branch skips the call).
+static __device__ __noinline__ float sigmoid_call(float x) { return 1.f / (1.f + expf(-x)); }
+static __device__ __noinline__ float decay_act_call(int prologue, float decay_scale, float x) {
+  if (prologue & PDN_PRO_DECAY_SOFTPLUS) return -decay_scale * softplus_f(x);
+  return -softplus_f(-x);
+}
 // A gate or gain as the kernels use it: sigmoid of the input when the
 // problem's gates arrive as logits, else the input.
 __device__ __forceinline__ float gate_act(int prologue, float x) {
-  return (prologue & PDN_PRO_SIGMOID_GATES) ? 1.f / (1.f + expf(-x)) : x;
+  return (prologue & PDN_PRO_SIGMOID_GATES) ? sigmoid_call(x) : x;
 }
 // The log decay as the kernels use it.
 __device__ __forceinline__ float decay_act(int prologue, float decay_scale, float x) {
-  if (prologue & PDN_PRO_DECAY_SOFTPLUS) return -decay_scale * softplus_f(x);
-  if (prologue & PDN_PRO_DECAY_LOGSIGMOID) return -softplus_f(-x);
+  if (prologue & (PDN_PRO_DECAY_SOFTPLUS | PDN_PRO_DECAY_LOGSIGMOID))
+    return decay_act_call(prologue, decay_scale, x);
   return x;
 }
 // 1 / max(||x||, 1e-12) from a sum of squares (L2 normalisation of q, k).
