@@ -247,6 +247,10 @@ static_assert(K1Layout<PDN_VAR_GDN2, PDN_DECAY_CHANNEL>::kBytes <= 232448 &&
 static_assert(2 * (K1Layout<PDN_VAR_PGDN, PDN_DECAY_SCALAR>::kBytes + 1024) <= 233472,
               "two intra-chunk CTAs per SM for scalar decay");
 
+// sqrt of a gain in [0, 1] as x * x^(-1/2) (rsqrtf, a couple of ulp): short
+// straight-line code for the per-element gains of FG2-GDN(+); 0 stays 0.
+__device__ __forceinline__ float sqrt_gain(float x) { return x > 0.f ? x * rsqrtf(x) : 0.f; }
+
 __device__ __forceinline__ void sync_for_mma() {
   fence_proxy_async_smem();
   tc_fence_before();
@@ -710,10 +714,10 @@ __global__ void __launch_bounds__(kK1Threads, kDecay == PDN_DECAY_CHANNEL ? 1 : 
         }
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
-          const float sq = sqrtf(gate_act(P.prologue, gb[e]));
+          const float sq = sqrt_gain(gate_act(P.prologue, gb[e]));
           r[e] = sq * kf[e];
           w[e] = r[e];
-          vf[e] *= kVariant == PDN_VAR_FG2_GDN_PLUS ? sqrtf(gate_act(P.prologue, gv[e])) : sq;
+          vf[e] *= kVariant == PDN_VAR_FG2_GDN_PLUS ? sqrt_gain(gate_act(P.prologue, gv[e])) : sq;
         }
       } else if (kVariant == PDN_VAR_GDN2) {
         float ge[8], gw[8];
