@@ -18,6 +18,8 @@
 // auxiliaries Y and U). Splitting it trades extra HBM traffic (about 80 KiB of
 // operand tiles per chunk and head, written once and read once) for running
 // the intra-chunk work with thousands of CTAs instead of one per chain.
+#include <mutex>
+
 #include "common.cuh"
 #include "internal.h"
 #include "ptx.cuh"
@@ -294,7 +296,8 @@ __device__ __forceinline__ void diag_exact(const uint8_t *xrow, const uint8_t *w
 }
 
 template <int kVariant, int kDecay>
-__global__ void __launch_bounds__(kK1Threads, kDecay == PDN_DECAY_CHANNEL ? 1 : 2) k1_intra(const KParams P, void *ws, int N) {
+__global__ void __launch_bounds__(kK1Threads, kDecay == PDN_DECAY_CHANNEL ? 1 : 2) k1_intra(const KParams P, void *ws, int N,
+                                                                         int it_begin, int it_end) {
   using L = K1Layout<kVariant, kDecay>;
   constexpr bool kPre = L::kPre;
   constexpr bool kCh = L::kCh;
@@ -328,7 +331,10 @@ __global__ void __launch_bounds__(kK1Threads, kDecay == PDN_DECAY_CHANNEL ? 1 : 
   const uint32_t lane_q = (uint32_t)(32 * (warp & 3)) << 16;
   const int half = warp >> 2;
   const int BH = P.B * P.H;
-  const int total = N * BH;  // chunk blocks, chunk-major: block index = c * BH + bh
+  // chunk blocks, chunk-major: block index = c * BH + bh; this launch takes
+  // blocks it_begin .. it_end - 1 (a range of whole chunks)
+  const int total = it_end;
+  const int first = it_begin + (int)blockIdx.x;
 
   if (warp == 0) {
     tmem_alloc(tbase_p, L::kTmemCols);
@@ -410,14 +416,14 @@ __global__ void __launch_bounds__(kK1Threads, kDecay == PDN_DECAY_CHANNEL ? 1 : 
     }
     cp_async_commit();
   };
-  Raw pf = load_raw(blockIdx.x < total ? blockIdx.x : 0);
-  if (blockIdx.x < total) {
-    stage_v(blockIdx.x);
-    stage_k(blockIdx.x);
+  Raw pf = load_raw(first < total ? first : 0);
+  if (first < total) {
+    stage_v(first);
+    stage_k(first);
   }
 
   int iter = 0;
-  for (int it = blockIdx.x; it < total; it += gridDim.x, ++iter) {
+  for (int it = first; it < total; it += gridDim.x, ++iter) {
   const int c = it / BH, bh = it % BH;
   const int b = bh / P.H, h = bh % P.H;
   const int c0 = c * kC, Cn = min(kC, P.T - c0);
@@ -1317,7 +1323,10 @@ __device__ __forceinline__ bool k2_issue_o(uint32_t tm, uint32_t sb, const K2Bar
   return true;
 }
 
-__global__ void __launch_bounds__(kK2Threads, 1) k2_state(const KParams P, void *ws, int N) {
+// Walks chunks cb .. cb + N - 1, from P.S0 (or zeros; the identity in
+// transition mode when P.S0 is NULL) to P.ST.
+__global__ void __launch_bounds__(kK2Threads, 1) k2_state(const KParams P, void *ws, int N,
+                                                          int cb) {
   extern __shared__ __align__(1024) uint8_t smem[];
   const uint32_t sb = smem_u32(smem);
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + K2_BAR);
@@ -1360,9 +1369,9 @@ __global__ void __launch_bounds__(kK2Threads, 1) k2_state(const KParams P, void 
     if (lane == 0) {
       const int BH = P.B * P.H;
       for (int m = 0; m < 3 && m < N; ++m)
-        load_main(smem + main_buf(m), ws_block(ws, bh, BH, m), B.fmain + m);
+        load_main(smem + main_buf(m), ws_block(ws, bh, BH, cb + m), B.fmain + m);
       for (int m = 0; m < 2 && m < N; ++m)
-        load_ut(smem + ut_buf(m), ws_block(ws, bh, BH, m), B.fut + m);
+        load_ut(smem + ut_buf(m), ws_block(ws, bh, BH, cb + m), B.fut + m);
       // after MMA3 of chunk n, its U/T buffer takes chunk n + 2; after every
       // MMA of chunk n, its main buffer takes chunk n + 3
       for (int n = 0; n + 2 < N; ++n) {
@@ -1370,13 +1379,13 @@ __global__ void __launch_bounds__(kK2Threads, 1) k2_state(const KParams P, void 
           *abort_flag = 1;
           break;
         }
-        load_ut(smem + ut_buf(n), ws_block(ws, bh, BH, n + 2), B.fut + (n & 1));
+        load_ut(smem + ut_buf(n), ws_block(ws, bh, BH, cb + n + 2), B.fut + (n & 1));
         if (n + 3 < N) {
           if (!k2_wait(B.mfree + (n % 3), (uint32_t)((n / 3) & 1), abort_flag)) {
             *abort_flag = 1;
             break;
           }
-          load_main(smem + main_buf(n), ws_block(ws, bh, BH, n + 3), B.fmain + (n % 3));
+          load_main(smem + main_buf(n), ws_block(ws, bh, BH, cb + n + 3), B.fmain + (n % 3));
         }
       }
     }
@@ -1390,7 +1399,7 @@ __global__ void __launch_bounds__(kK2Threads, 1) k2_state(const KParams P, void 
     auto fetch_e = [&](int c) {
       if (lane < 8)
         cp_async16(sb + K2_EBUF + (warp * 2 + (c & 1)) * 128 + lane * 16,
-                   reinterpret_cast<const float *>(ws_block(ws, bh, P.B * P.H, c) + WS_E) + 32 * cg +
+                   reinterpret_cast<const float *>(ws_block(ws, bh, P.B * P.H, cb + c) + WS_E) + 32 * cg +
                        4 * lane,
                    true);
       cp_async_commit();
@@ -1414,7 +1423,7 @@ __global__ void __launch_bounds__(kK2Threads, 1) k2_state(const KParams P, void 
         if (n == 0) {
 #pragma unroll
           for (int u = 0; u < 2; ++u) {
-            if (P.transition) {  // the identity: S[j][i] = (i == j)
+            if (P.transition && !P.S0) {  // the identity: S[j][i] = (i == j)
 #pragma unroll
               for (int e = 0; e < 16; ++e) sv[u][e] = (col0 + 16 * u + e == j) ? 1.f : 0.f;
             } else if (P.S0) {
@@ -1463,7 +1472,7 @@ __global__ void __launch_bounds__(kK2Threads, 1) k2_state(const KParams P, void 
       // O^T buffer they free takes chunk n + 1, whose MMA6 comes after this
       // chunk's epilogues)
       const uint32_t ot_prev = tm + lane_q + (s ? TM_OT0 : TM_OT1);
-      const int pc_prev = (n - 1) * kC;
+      const int pc_prev = (cb + n - 1) * kC;
       if (n > 0) {
         if (!(ok = k2_warp_wait(B.baro, (uint32_t)((n - 1) & 1), abort_flag, lane))) break;
         k2_store_o(P, ot_prev, b, h, pc_prev, min(kC, P.T - pc_prev), lane, quarter, cg, 0);
@@ -1488,7 +1497,7 @@ __global__ void __launch_bounds__(kK2Threads, 1) k2_state(const KParams P, void 
     }
     // the last chunk's output
     if (ok && N > 0 && k2_warp_wait(B.baro, (uint32_t)((N - 1) & 1), abort_flag, lane)) {
-      const int pc0 = (N - 1) * kC;
+      const int pc0 = (cb + N - 1) * kC;
       for (int part = 0; part < 2; ++part)
         k2_store_o(P, tm + lane_q + (((N - 1) & 1) ? TM_OT1 : TM_OT0), b, h, pc0,
                    min(kC, P.T - pc0), lane, quarter, cg, part);
@@ -1526,7 +1535,8 @@ __global__ void __launch_bounds__(kK2Threads, 1) k2_state(const KParams P, void 
 }
 
 template <int V, int Dc>
-cudaError_t launch_k1(const KParams &P, void *ws, int N, cudaStream_t stream) {
+cudaError_t launch_k1(const KParams &P, void *ws, int N, int it0, int it1, int sm_budget,
+                      cudaStream_t stream) {
   using L = K1Layout<V, Dc>;
   auto kern = k1_intra<V, Dc>;
   cudaError_t e =
@@ -1541,22 +1551,64 @@ cudaError_t launch_k1(const KParams &P, void *ws, int N, cudaStream_t stream) {
   if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kK1Threads, L::kBytes) != cudaSuccess ||
       per_sm < 1)
     per_sm = 1;
-  const long long total = (long long)N * P.B * P.H;
-  // At least two CTAs per SM: the blocks are independent, so a CTA that does
-  // not fit yet simply starts when one finishes, at no loss.
-  if (per_sm < 2) per_sm = 2;
+  if (sm_budget > 0 && sm_budget < sms) sms = sm_budget;
+  const long long total = (long long)it1 - it0;
+  if (total <= 0) return cudaSuccess;
+  // At least two CTAs per SM (unless the SMs are budgeted): the blocks are
+  // independent, so a CTA that does not fit yet simply starts when one
+  // finishes, at no loss.
+  if (per_sm < 2 && sm_budget <= 0) per_sm = 2;
   const long long grid = total < (long long)sms * per_sm ? total : (long long)sms * per_sm;
-  kern<<<(unsigned)grid, kK1Threads, L::kBytes, stream>>>(P, ws, N);
+  kern<<<(unsigned)grid, kK1Threads, L::kBytes, stream>>>(P, ws, N, it0, it1);
   return cudaGetLastError();
 }
 
 template <int V>
-cudaError_t launch_k1_decay(const KParams &P, void *ws, int N, cudaStream_t stream) {
+cudaError_t launch_k1_decay(const KParams &P, void *ws, int N, int it0, int it1, int sm_budget,
+                            cudaStream_t stream) {
   switch (P.decay) {
-    case PDN_DECAY_NONE: return launch_k1<V, PDN_DECAY_NONE>(P, ws, N, stream);
-    case PDN_DECAY_SCALAR: return launch_k1<V, PDN_DECAY_SCALAR>(P, ws, N, stream);
-    default: return launch_k1<V, PDN_DECAY_CHANNEL>(P, ws, N, stream);
+    case PDN_DECAY_NONE: return launch_k1<V, PDN_DECAY_NONE>(P, ws, N, it0, it1, sm_budget, stream);
+    case PDN_DECAY_SCALAR:
+      return launch_k1<V, PDN_DECAY_SCALAR>(P, ws, N, it0, it1, sm_budget, stream);
+    default: return launch_k1<V, PDN_DECAY_CHANNEL>(P, ws, N, it0, it1, sm_budget, stream);
   }
+}
+
+cudaError_t launch_k1_range(const KParams &P, void *ws, int N, int it0, int it1, int sm_budget,
+                            cudaStream_t stream) {
+  switch (P.variant) {
+    case PDN_VAR_DN: return launch_k1_decay<PDN_VAR_DN>(P, ws, N, it0, it1, sm_budget, stream);
+    case PDN_VAR_GDN: return launch_k1_decay<PDN_VAR_GDN>(P, ws, N, it0, it1, sm_budget, stream);
+    case PDN_VAR_KDA: return launch_k1_decay<PDN_VAR_KDA>(P, ws, N, it0, it1, sm_budget, stream);
+    case PDN_VAR_PDN: return launch_k1_decay<PDN_VAR_PDN>(P, ws, N, it0, it1, sm_budget, stream);
+    case PDN_VAR_PGDN: return launch_k1_decay<PDN_VAR_PGDN>(P, ws, N, it0, it1, sm_budget, stream);
+    case PDN_VAR_PKDA: return launch_k1_decay<PDN_VAR_PKDA>(P, ws, N, it0, it1, sm_budget, stream);
+    case PDN_VAR_FG2_GDN:
+      return launch_k1_decay<PDN_VAR_FG2_GDN>(P, ws, N, it0, it1, sm_budget, stream);
+    case PDN_VAR_GDN2: return launch_k1_decay<PDN_VAR_GDN2>(P, ws, N, it0, it1, sm_budget, stream);
+    case PDN_VAR_PLA: return launch_k1_decay<PDN_VAR_PLA>(P, ws, N, it0, it1, sm_budget, stream);
+    default:
+      return launch_k1_decay<PDN_VAR_FG2_GDN_PLUS>(P, ws, N, it0, it1, sm_budget, stream);
+  }
+}
+
+// Long sequences over few chains: the state pass runs one CTA per chain, so
+// with B*H well below the SM count most SMs idle through it. The chunks are
+// then cut into kSegs time segments; K1 of segment i + 1 runs on the SMs the
+// state pass leaves free while K2 walks segment i on a second stream, joined
+// by events (no kernel waits on another). K2 carries the state from segment
+// to segment through P.ST (each CTA reads its rows before it rewrites them).
+constexpr int kSegs = 8;
+constexpr int kMaxDev = 64;
+struct SegRes {
+  cudaStream_t s2 = nullptr;
+  cudaEvent_t ev[kSegs + 1] = {};
+};
+SegRes g_seg[kMaxDev];
+std::mutex g_seg_mu;
+
+bool use_segments(const KParams &P, int N, int sms) {
+  return P.ST != nullptr && N >= 8 * kSegs && (long long)P.B * P.H * 3 <= sms;
 }
 
 }  // namespace
@@ -1593,25 +1645,46 @@ cudaError_t launch_chunk_split(const KParams &P, void *ws, cudaStream_t stream,
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   if (ev && (e = cudaEventRecord(ev[1], stream)) != cudaSuccess) return e;
-  switch (P.variant) {
-    case PDN_VAR_DN: e = launch_k1_decay<PDN_VAR_DN>(P, ws, N, stream); break;
-    case PDN_VAR_GDN: e = launch_k1_decay<PDN_VAR_GDN>(P, ws, N, stream); break;
-    case PDN_VAR_KDA: e = launch_k1_decay<PDN_VAR_KDA>(P, ws, N, stream); break;
-    case PDN_VAR_PDN: e = launch_k1_decay<PDN_VAR_PDN>(P, ws, N, stream); break;
-    case PDN_VAR_PGDN: e = launch_k1_decay<PDN_VAR_PGDN>(P, ws, N, stream); break;
-    case PDN_VAR_PKDA: e = launch_k1_decay<PDN_VAR_PKDA>(P, ws, N, stream); break;
-    case PDN_VAR_FG2_GDN: e = launch_k1_decay<PDN_VAR_FG2_GDN>(P, ws, N, stream); break;
-    case PDN_VAR_GDN2: e = launch_k1_decay<PDN_VAR_GDN2>(P, ws, N, stream); break;
-    case PDN_VAR_PLA: e = launch_k1_decay<PDN_VAR_PLA>(P, ws, N, stream); break;
-    default: e = launch_k1_decay<PDN_VAR_FG2_GDN_PLUS>(P, ws, N, stream); break;
-  }
-  if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(k2_state, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)K2_BYTES);
   if (e != cudaSuccess) return e;
-  if (ev && (e = cudaEventRecord(ev[2], stream)) != cudaSuccess) return e;
-  k2_state<<<BH, kK2Threads, K2_BYTES, stream>>>(P, ws, N);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  return ev ? cudaEventRecord(ev[3], stream) : cudaSuccess;
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess)
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (ev || dev < 0 || dev >= kMaxDev || !use_segments(P, N, sms)) {
+    if ((e = launch_k1_range(P, ws, N, 0, N * BH, 0, stream)) != cudaSuccess) return e;
+    if (ev && (e = cudaEventRecord(ev[2], stream)) != cudaSuccess) return e;
+    k2_state<<<BH, kK2Threads, K2_BYTES, stream>>>(P, ws, N, 0);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    return ev ? cudaEventRecord(ev[3], stream) : cudaSuccess;
+  }
+  // segmented: the calls share the device's second stream and events, so
+  // their enqueueing is serialised
+  std::lock_guard<std::mutex> lock(g_seg_mu);
+  SegRes &R = g_seg[dev];
+  if (!R.s2) {
+    if ((e = cudaStreamCreateWithFlags(&R.s2, cudaStreamNonBlocking)) != cudaSuccess) {
+      R.s2 = nullptr;
+      return e;
+    }
+    for (int i = 0; i <= kSegs; ++i)
+      if ((e = cudaEventCreateWithFlags(&R.ev[i], cudaEventDisableTiming)) != cudaSuccess) return e;
+  }
+  for (int g = 0; g < kSegs; ++g) {
+    const int c0 = (int)((long long)N * g / kSegs), c1 = (int)((long long)N * (g + 1) / kSegs);
+    // the first segment has the whole GPU; later ones leave the state pass its SMs
+    e = launch_k1_range(P, ws, N, c0 * BH, c1 * BH, g == 0 ? 0 : sms - BH, stream);
+    if (e == cudaSuccess) e = cudaEventRecord(R.ev[g], stream);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(R.s2, R.ev[g], 0);
+    if (e != cudaSuccess) break;
+    KParams Pg = P;
+    if (g > 0) Pg.S0 = P.ST;  // the state where the previous segment left it
+    k2_state<<<BH, kK2Threads, K2_BYTES, R.s2>>>(Pg, ws, c1 - c0, c0);
+    if ((e = cudaGetLastError()) != cudaSuccess) break;
+  }
+  // join the second stream back into the caller's on every path
+  cudaError_t j = cudaEventRecord(R.ev[kSegs], R.s2);
+  if (j == cudaSuccess) j = cudaStreamWaitEvent(stream, R.ev[kSegs], 0);
+  return e != cudaSuccess ? e : j;
 }
 
 }  // namespace pdn
