@@ -263,8 +263,9 @@ __device__ __forceinline__ void sync_for_mma() {
 // Exact diagonal-block entries of row t against columns s0 .. s0 + 15 of a
 // flagged sub-chunk: sum_c x_tc w_sc e^{G_tc - G_sc} for s <= t (s < t when
 // `strict`), from the undecayed bf16 rows x (row t) and w (rows s) and the
-// fp32 cumulative log decay.
-__device__ __forceinline__ void diag_exact(const uint8_t *xrow, const uint8_t *wbase,
+// fp32 cumulative log decay. Out of line: only flagged sub-chunks (very
+// strong decay) take it, and inlined copies would sit in the hot epilogue.
+__device__ __noinline__ void diag_exact(const uint8_t *xrow, const uint8_t *wbase,
                                            const float *gbuf, int t, int s0, bool strict,
                                            float (&out)[16]) {
   float acc[16];
@@ -877,9 +878,13 @@ __global__ void __launch_bounds__(kK1Threads, kDecay == PDN_DECAY_CHANNEL ? 1 : 
           if (s0 > sd || (s0 == sd && (isP ? s > tr : s >= tr))) x = 0.f;
           mv[cc][e] = x;
         }
-        if (s0 == sd && ((badm >> a) & 1u))
+        if (s0 == sd && ((badm >> a) & 1u)) {
+          float ex[16];  // (its own array: mv stays in registers)
           diag_exact(smem + (isP ? L::kQS : L::kKS) + tr * KS_LD, smem + L::kBC, GBUF, tr, s0,
-                     !isP, mv[cc]);
+                     !isP, ex);
+#pragma unroll
+          for (int e = 0; e < 16; ++e) mv[cc][e] = ex[e];
+        }
       }
       // R with the chunk-start reference for MMA2: e^{G_t} r = e^{B_a} (rho_t r)
 #pragma unroll
