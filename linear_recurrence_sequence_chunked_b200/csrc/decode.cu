@@ -392,21 +392,49 @@ __global__ void __launch_bounds__(kTmaThreads, 1) decode_tma_kernel(const KParam
     const float4 qq = make_float4(sm.q[c], sm.q[c + 1], sm.q[c + 2], sm.q[c + 3]);
     const float4 aa = make_float4(sm.al[c], sm.al[c + 1], sm.al[c + 2], sm.al[c + 3]);
     float *S = sm.buf[s];
-#pragma unroll 4
-    for (int m = 0; m < kD128 / kWarps; ++m) {
+    // The warp's 16 rows j = warp + 8 m at once: decayed rows in registers,
+    // their 32 partial sums (y_m = S'_j r, then z_m = S'_j q) reduced together
+    // by a transposed butterfly (31 shuffles; lane l ends with sum l), the
+    // deltas broadcast back, the rows updated and stored.
+    constexpr int kR = kD128 / kWarps;  // 16 rows per warp
+    static_assert(2 * kR == 32, "two partial sums per row, one lane per sum");
+    float4 X[kR];
+    float v[2 * kR];
+#pragma unroll
+    for (int m = 0; m < kR; ++m) {
       const int j = warp + m * kWarps;
       float4 x = *reinterpret_cast<const float4 *>(S + j * kD128 + c);
       x.x *= aa.x; x.y *= aa.y; x.z *= aa.z; x.w *= aa.w;
-      const float y = warp_sum(x.x * rr.x + x.y * rr.y + x.z * rr.z + x.w * rr.w);
-      const float z = warp_sum(x.x * qq.x + x.y * qq.y + x.z * qq.z + x.w * qq.w);
-      const float delta = sm.u[j] - y;
+      X[m] = x;
+      v[m] = x.x * rr.x + x.y * rr.y + x.z * rr.z + x.w * rr.w;
+      v[kR + m] = x.x * qq.x + x.y * qq.y + x.z * qq.z + x.w * qq.w;
+    }
+#pragma unroll
+    for (int off = 16, len = kR; off >= 1; off >>= 1, len >>= 1) {
+      const bool upper = (lane & off) != 0;
+#pragma unroll
+      for (int e = 0; e < len; ++e) {
+        const float send = upper ? v[e] : v[e + len];
+        const float keep = upper ? v[e + len] : v[e];
+        v[e] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+      }
+    }
+    // lane m < 16: y of row m -> its delta; lane 16 + m: z of row m
+    const float dl = lane < kR ? sm.u[warp + lane * kWarps] - v[0] : 0.f;
+    const float dz = __shfl_up_sync(0xffffffffu, dl, kR);  // delta of row lane - 16
+#pragma unroll
+    for (int m = 0; m < kR; ++m) {
+      const int j = warp + m * kWarps;
+      const float delta = __shfl_sync(0xffffffffu, dl, m);
+      float4 x = X[m];
       x.x = fmaf(delta, ww.x, x.x);
       x.y = fmaf(delta, ww.y, x.y);
       x.z = fmaf(delta, ww.z, x.z);
       x.w = fmaf(delta, ww.w, x.w);
       *reinterpret_cast<float4 *>(S + j * kD128 + c) = x;
-      if (lane == 0) stf<Tin>(P.o, tokh * kD128 + j, P.q_scale * fmaf(delta, wq, z));
     }
+    if (lane >= kR)
+      stf<Tin>(P.o, tokh * kD128 + warp + (lane - kR) * kWarps, P.q_scale * fmaf(dz, wq, v[0]));
     // hand the buffer back: generic writes -> async proxy, then one arrive per warp
     fence_proxy_async_smem();
     __syncwarp();
