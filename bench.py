@@ -18,6 +18,9 @@ timed steps. The JSON line also carries:
               attention and FG2-GDN+ at the headline shape): tokens/s, tensor and
               HBM fractions, and per-kernel CUDA-event times (also given for
               the headline layer under roofline.kernel_ms);
+  backward    the gradient of the headline layer (pdn_chunk_bwd, every
+              input's gradient from dO and dS_T): tokens/s and its fraction
+              of the fp32 CUDA-core peak (an ALU-bound pass);
   cpu_baseline the fp64 oracle on the host cores on a bounded sample.
 Multi-GPU (torchrun): every rank runs its own independent batch (weak
 scaling, no collective on the data path); the time is the max over ranks.
@@ -392,6 +395,13 @@ def run_ours(args):
             result["gpu_launches"] += r["gpu_launches"]
             torch.cuda.empty_cache()
 
+    # ---------------- backward of the headline layer
+    if not args.no_backward:
+        torch.cuda.empty_cache()
+        result["backward"] = bench_backward(args, w, dev, stream, rank, mor, barrier)
+        result["gpu_launches"] += result["backward"]["gpu_launches"]
+        torch.cuda.empty_cache()
+
     # ---------------- decode workload
     if not args.no_decode:
         result["decode"] = bench_decode(args, dev, stream, peaks, peaks_kind, world, rank,
@@ -492,6 +502,83 @@ def bench_workload(args, w, dev, stream, peaks, peaks_kind, rank, mor, barrier,
            "l2": "inputs larger than L2 (no flush)",
            "gpu_launches": args.steps * launches}
     del x, g, o, ws, ST, AT, tens
+    return res
+
+
+# fp32 CUDA-core peak from the unit counts and the maximum SM clock: 148 SMs x
+# 128 fp32 lanes x 2 flops (FMA) x 1965 MHz
+FP32_ALU_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+
+
+def bwd_flops_per_token_head(dk, dv):
+    """Elementwise state work of the four backward sweeps per (token, head),
+    an FMA counted as 2: forward delta sweep 5, reverse cotangent sweep 7,
+    forward dq'/dr sweep 7, reverse dw sweep 7 flops per state element."""
+    return 26 * dk * dv
+
+
+def bench_backward(args, w, dev, stream, rank, mor, barrier):
+    """Times `args.steps` pdn_chunk_bwd calls of the headline layer (inputs and
+    cotangents resident in HBM, larger than L2), after warm-up."""
+    import torch
+
+    from linear_recurrence_sequence_chunked_b200 import pdn
+    from linear_recurrence_sequence_chunked_b200.workloads import make_inputs
+
+    wr = w.replace(seed=rank_seed(w.seed, rank))
+    x = make_inputs(wr, device=dev, generator_device=dev)
+    gen = torch.Generator(device=dev).manual_seed(rank_seed(7, rank))
+    dO = torch.randn(w.B, w.T, w.H, w.dv, generator=gen, device=dev).to(x["v"].dtype)
+    dST = torch.randn(w.B, w.H, w.dv, w.dk, generator=gen, device=dev)
+    prob = pdn.make_problem(w.variant, w.B, w.T, w.H, w.dk, w.dv, x["k"].dtype, w.decay, w.chunk,
+                            "auto", w.q_scale, w.precond_x, w.precond_eps)
+    f32 = dict(dtype=torch.float32, device=dev)
+    g = {n: torch.empty_like(x[n], **f32) for n in ("q", "k", "v")}
+    g["log_alpha"] = torch.empty_like(x["log_alpha"], **f32)
+    g["beta"] = torch.empty_like(x["beta"], **f32)
+    g["S0"] = torch.empty(w.B, w.H, w.dv, w.dk, **f32)
+    g["A0"] = torch.empty(w.B, w.H, w.dk, **f32)
+    tens = pdn.make_tensors(x["q"], x["k"], x["v"], None, x["log_alpha"], x["beta"])
+    grads = pdn.make_grads(dO, dST, g["q"], g["k"], g["v"], g["log_alpha"], g["beta"], None, None,
+                           g["S0"], g["A0"])
+    ws = torch.empty(pdn.pdn_chunk_bwd_workspace(prob), dtype=torch.uint8, device=dev)
+    sptr = stream.cuda_stream
+
+    def step():
+        rc = pdn.pdn_chunk_bwd(prob, tens, grads, ws.data_ptr(), ws.numel(), sptr)
+        if rc != pdn.PDN_OK:
+            raise pdn.PdnError(rc, "pdn_chunk_bwd")
+
+    for _ in range(args.warmup):
+        step()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    barrier()
+    ms_local = e0.elapsed_time(e1)
+    ms = mor(ms_local)
+    if pdn.device_error() != pdn.PDN_OK:
+        raise SystemExit("device error during the backward timed region")
+    per = ms_local / args.steps
+    flops = bwd_flops_per_token_head(w.dk, w.dv) * w.B * w.T * w.H
+    # generic vectors, four sweeps, epilogue; then the preconditioner's prefix
+    # (squares + 3 scan passes) and suffix (3 scan passes + dk update) and the
+    # decay's final-state term + suffix sum
+    launches = 1 + 4 + 1 + (1 + 3 + 3 + 1) + (1 + 3)
+    res = {"workload": w.name, "variant": w.variant, "value": w.B * w.T * args.steps / (ms / 1e3),
+           "unit": "tokens/s", "ms_per_step": ms / args.steps,
+           "roofline": {"bound": "alu", "achieved": flops / (per / 1e3) / 1e12,
+                        "peak": FP32_ALU_TFLOPS, "unit": "TFLOP/s",
+                        "frac": flops / (per / 1e3) / 1e12 / FP32_ALU_TFLOPS,
+                        "flops_per_launch": flops,
+                        "peak_kind": "fp32 CUDA-core peak from unit counts x 1965 MHz"},
+           "gradients": "q, k, v, log_alpha, beta, S0, A0 (fp32) from dO and dS_T",
+           "l2": "inputs larger than L2 (no flush)",
+           "gpu_launches": args.steps * launches}
+    del x, dO, dST, g, ws, grads, tens
     return res
 
 
@@ -601,6 +688,7 @@ def main():
     ap.add_argument("--decode-steps", type=int, default=1024)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-backward", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     args = ap.parse_args()
