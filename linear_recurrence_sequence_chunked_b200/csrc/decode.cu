@@ -171,19 +171,23 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const KParams P) {
 // per-token prologue and the row updates in shared memory. Full/empty
 // mbarriers hand buffers between the two; every wait is bounded.
 constexpr int kTmaBufs = 3;
+constexpr float kLog2eD = 1.4426950408889634f, kLn2D = 0.6931471805599453f;
 constexpr int kD128 = 128;
 constexpr int kConsumers = kThreads;      // 8 consumer warps
 constexpr int kTmaThreads = kThreads + 32;  // + 1 producer warp
 constexpr uint32_t kStateBytes = kD128 * kD128 * 4;
 constexpr uint32_t kPart = 16384;  // bytes per bulk copy
 
+// The token vectors and the reduction slots are double-buffered by item
+// parity: item k + 1's prologue writes the other half, and item k - 1's
+// readers are all past item k's first barrier, so no barrier closes an item.
 struct DecSmem {
   float buf[kTmaBufs][kD128 * kD128];
-  float r[kD128], w[kD128], q[kD128], al[kD128], u[kD128];
-  float red[kWarps];
+  float r[2][kD128], w[2][kD128], q[2][kD128], al[2][kD128], u[2][kD128];
+  float red[2][4][kWarps];  // per parity: |k|^2, |q|^2, mean log A, w.q
   uint64_t full[kTmaBufs];
   uint64_t empty[kTmaBufs];
-  int vote[kWarps];
+  int vote[2][kWarps];
   int abort_flag;
 };
 
@@ -192,10 +196,11 @@ __device__ __forceinline__ void consumer_sync() {
   asm volatile("bar.sync 1, %0;" ::"r"(kConsumers) : "memory");
 }
 
+// Sum over the consumer warps through `red` (kWarps slots no other reduction
+// of the same item uses): one barrier.
 __device__ __forceinline__ float consumer_sum(float v, float *red) {
   v = warp_sum(v);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  consumer_sync();
   if (lane == 0) red[warp] = v;
   consumer_sync();
   float s = 0.f;
@@ -317,10 +322,11 @@ __global__ void __launch_bounds__(kTmaThreads, 1) decode_tma_kernel(const KParam
     const Tok nxt = (k + 1 < nloc) ? load_tok(k + 1) : cur;
 
     // per-token vectors (overlap the bulk loads in flight)
+    const int par = k & 1;
     float kv = cur.k, qv = cur.q;
     if (P.prologue & PDN_PRO_L2NORM_QK) {  // fused prologue: unit-norm k and q
-      const float ssk = consumer_sum(chan ? kv * kv : 0.f, sm.red);
-      const float ssq = consumer_sum(chan ? qv * qv : 0.f, sm.red);
+      const float ssk = consumer_sum(chan ? kv * kv : 0.f, sm.red[par][0]);
+      const float ssq = consumer_sum(chan ? qv * qv : 0.f, sm.red[par][1]);
       kv *= inv_norm(ssk);
       qv *= inv_norm(ssq);
     }
@@ -328,22 +334,27 @@ __global__ void __launch_bounds__(kTmaThreads, 1) decode_tma_kernel(const KParam
     if (chan && precond) {
       const float a = cur.a + kv * kv;
       P.AT[(size_t)item * kD128 + tid] = a;
-      logA = logf(a + P.eps);
+      logA = lg2_approx(a + P.eps);  // base 2, as the intra-chunk kernel
     }
     float mu = 0.f;
-    if (precond) mu = consumer_sum(chan ? logA : 0.f, sm.red) / (float)kD128;
+    if (precond) mu = consumer_sum(chan ? logA : 0.f, sm.red[par][2]) * (1.f / (float)kD128);
+    // B = x^{-s}, s = c / (1 + |c|), c = ln(A + eps) - mean (hardware exp2 / rcp)
+    auto coef = [&]() {
+      const float cc = (logA - mu) * kLn2D;
+      return ex2_approx(-(cc * rcp_approx(1.f + fabsf(cc))) * (P.lnx * kLog2eD));
+    };
     float w = 0.f;
     if (chan) {
       float r, u = cur.v;
       switch (P.variant) {
         case PDN_VAR_PDN: case PDN_VAR_PGDN: case PDN_VAR_PKDA:
           r = kv;
-          w = cur.beta * precond_coef(logA, mu, P.lnx) * kv;
+          w = cur.beta * coef() * kv;
           break;
         case PDN_VAR_PLA:  // no erase; the preconditioner acts on the query
           r = 0.f;
           w = cur.beta * kv;
-          qv *= precond_coef(logA, mu, P.lnx);
+          qv *= coef();
           break;
         case PDN_VAR_FG2_GDN: case PDN_VAR_FG2_GDN_PLUS: {
           const float sb = sqrtf(cur.beta);
@@ -360,13 +371,13 @@ __global__ void __launch_bounds__(kTmaThreads, 1) decode_tma_kernel(const KParam
           r = kv;
           w = cur.beta * kv;
       }
-      sm.r[tid] = r;
-      sm.w[tid] = w;
-      sm.q[tid] = qv;
-      sm.al[tid] = P.decay == PDN_DECAY_NONE ? 1.f : expf(cur.la);
-      sm.u[tid] = u;
+      sm.r[par][tid] = r;
+      sm.w[par][tid] = w;
+      sm.q[par][tid] = qv;
+      sm.al[par][tid] = P.decay == PDN_DECAY_NONE ? 1.f : ex2_approx(cur.la * kLog2eD);
+      sm.u[par][tid] = u;
     }
-    const float wq = consumer_sum(chan ? w * qv : 0.f, sm.red);  // ends with consumer_sync
+    const float wq = consumer_sum(chan ? w * qv : 0.f, sm.red[par][3]);  // ends with a barrier
 
     // Wait for the state. The decision to stop must be the same in every
     // consumer warp (they meet at named barriers): each warp votes once,
@@ -375,22 +386,22 @@ __global__ void __launch_bounds__(kTmaThreads, 1) decode_tma_kernel(const KParam
     int vote = __all_sync(0xffffffffu, ok) ? 1 : 0;
     if (lane == 0) {
       if (*reinterpret_cast<volatile int *>(&sm.abort_flag)) vote = 0;
-      sm.vote[warp] = vote;
+      sm.vote[par][warp] = vote;
     }
     consumer_sync();
     bool all_ok = true;
 #pragma unroll
-    for (int i = 0; i < kWarps; ++i) all_ok = all_ok && sm.vote[i];
+    for (int i = 0; i < kWarps; ++i) all_ok = all_ok && sm.vote[par][i];
     if (!all_ok) {
       if (tid == 0) atomicExch(&sm.abort_flag, 1);
       break;
     }
 
     const int c = lane * 4;
-    const float4 rr = make_float4(sm.r[c], sm.r[c + 1], sm.r[c + 2], sm.r[c + 3]);
-    const float4 ww = make_float4(sm.w[c], sm.w[c + 1], sm.w[c + 2], sm.w[c + 3]);
-    const float4 qq = make_float4(sm.q[c], sm.q[c + 1], sm.q[c + 2], sm.q[c + 3]);
-    const float4 aa = make_float4(sm.al[c], sm.al[c + 1], sm.al[c + 2], sm.al[c + 3]);
+    const float4 rr = *reinterpret_cast<const float4 *>(&sm.r[par][c]);
+    const float4 ww = *reinterpret_cast<const float4 *>(&sm.w[par][c]);
+    const float4 qq = *reinterpret_cast<const float4 *>(&sm.q[par][c]);
+    const float4 aa = *reinterpret_cast<const float4 *>(&sm.al[par][c]);
     float *S = sm.buf[s];
     // The warp's 16 rows j = warp + 8 m at once: decayed rows in registers,
     // their 32 partial sums (y_m = S'_j r, then z_m = S'_j q) reduced together
@@ -420,7 +431,7 @@ __global__ void __launch_bounds__(kTmaThreads, 1) decode_tma_kernel(const KParam
       }
     }
     // lane m < 16: y of row m -> its delta; lane 16 + m: z of row m
-    const float dl = lane < kR ? sm.u[warp + lane * kWarps] - v[0] : 0.f;
+    const float dl = lane < kR ? sm.u[par][warp + lane * kWarps] - v[0] : 0.f;
     const float dz = __shfl_up_sync(0xffffffffu, dl, kR);  // delta of row lane - 16
 #pragma unroll
     for (int m = 0; m < kR; ++m) {
@@ -439,8 +450,6 @@ __global__ void __launch_bounds__(kTmaThreads, 1) decode_tma_kernel(const KParam
     fence_proxy_async_smem();
     __syncwarp();
     if (lane == 0) mbar_arrive(&sm.empty[s]);
-    // r/w/q/al/u are rewritten by the next prologue: all warps must be past the rows
-    consumer_sync();
     cur = nxt;
   }
 }
