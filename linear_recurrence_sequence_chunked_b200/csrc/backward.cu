@@ -16,9 +16,10 @@
 //   R1  reverse, warp per state row:  dd_t, dS0
 //   F2  forward, thread per key column, delta given: dq'_t and dr_t
 //   R2  reverse, thread per key column, dd given:    dw_t
-// F2 and R2 have no reduction on their sequential path (a gated linear
-// attention pass each); their column sums over a CTA's rows are written per
-// row group and added in the epilogue.
+// F2 and R2 have no reduction and no feedback (a gated linear attention pass
+// each), so they run every 64-token chunk in parallel from the states F1 and
+// R1 leave at the chunk boundaries; their column sums over a CTA's rows are
+// written per row group and added in the epilogue.
 //
 // The decay gradient needs no state either. With psi_t,i = sum_j P_t[j,i]
 // dP_t[j,i] (the cotangent of log alpha_t,i), expanding S_t = P_t + delta_t
@@ -45,13 +46,15 @@ struct BwdPlan {
   int GS;          // floats per (token, head) of the generic vectors: q'|r|w|a|u
   int R, G;        // rows per CTA of F2/R2, row groups (d_v / R)
   int nb;          // scan blocks per sequence
-  size_t gen, acc, delta, dd, st, part, cpsi, sigma, dacc, bsum, phi, total;
+  int nck;         // state checkpoints per sequence (one per kCk tokens)
+  size_t gen, acc, delta, dd, st, part, cpsi, sigma, dacc, bsum, phi, ckS, ckD, total;
 };
 
 namespace {
 
 constexpr int kScanBlk = 64;     // tokens per scan block
-constexpr int kLC = 16;          // tokens staged per chunk in F1 / R1 / F2 / R2
+constexpr int kCk = 64;          // tokens per state checkpoint (F2 / R2 run chunk-parallel)
+constexpr int kLCC = 8;          // tokens staged per chunk in F2 / R2
 
 size_t up64(size_t n) { return (n + 63) & ~(size_t)63; }
 
@@ -69,8 +72,7 @@ static BwdPlan bwd_plan(const KParams &P) {
   const size_t BH = (size_t)P.B * P.H, T = (size_t)P.T;
   const int dk = P.dk, dv = P.dv;
   L.GS = 4 * dk + dv;
-  const long long rows32 = (long long)BH * (dv / 32);
-  L.R = (dv % 32 == 0 && rows32 >= 148) ? 32 : 16;
+  L.R = dv % 32 == 0 ? 32 : 16;  // F2 / R2 are chunk-parallel: wide row groups
   L.G = dv / L.R;
   L.nb = (int)((T + kScanBlk - 1) / kScanBlk);
   size_t off = 0;
@@ -86,6 +88,9 @@ static BwdPlan bwd_plan(const KParams &P) {
   L.dacc = take(is_precond(P.variant) ? BH * T * dk : 0);
   L.bsum = take(BH * (size_t)L.nb * dk);
   L.phi = take(BH * dk + BH);
+  L.nck = (int)((T + kCk - 1) / kCk);
+  L.ckS = take(BH * (size_t)L.nck * dv * dk);
+  L.ckD = take(BH * (size_t)L.nck * dv * dk);
   L.total = off;
   return L;
 }
@@ -99,7 +104,10 @@ struct BParams {
   const float *dST;   // [B,H,dv,dk] or NULL
   float *dq, *dk, *dv, *dla, *dbeta, *derase, *dwrite, *dS0, *dA0;
   float *gen, *acc, *delta, *dd, *st, *part, *cpsi, *sigma, *dacc, *bsum, *phi;
-  int GS, R, G, nb;
+  // S before the first token of each kCk-token chunk (F1) and the cotangent
+  // entering each chunk's last token (R1): [BH][nck][d_v][d_k]
+  float *ckS, *ckD;
+  int GS, R, G, nb, nck;
 };
 
 // Generic vectors of one token, in the workspace order q'|r|w|a|u.
@@ -417,6 +425,13 @@ __global__ void __launch_bounds__(128) f1_kernel(const BParams Q) {
     __syncthreads();
     const float *buf = sm + (ch & 1) * kLCR * TS;
     const int t0 = ch * kLCR, n = min(kLCR, T - t0);
+    if (t0 % kCk == 0 && rok) {  // the state before chunk t0 / kCk
+      float *ck = Q.ckS + (((size_t)bh * Q.nck + t0 / kCk) * dv + j) * dk;
+#pragma unroll
+      for (int e = 0; e < CPL; e += 4)
+        if (s * CPL + e < dk)
+          *reinterpret_cast<float4 *>(ck + s * CPL + e) = make_float4(S[e], S[e + 1], S[e + 2], S[e + 3]);
+    }
     for (int tt = 0; tt < n; ++tt) {
       const float *sv = buf + tt * TS + s * SS;
       float y[4] = {0.f, 0.f, 0.f, 0.f};
@@ -509,6 +524,13 @@ __global__ void __launch_bounds__(128) r1_kernel(const BParams Q) {
     __syncthreads();
     const float *buf = sm + (ch & 1) * kLCR * TS;
     const int t0 = ch * kLCR, n = min(kLCR, T - t0);
+    if (((t0 + n) % kCk == 0 || t0 + n == T) && rok) {  // entering chunk (t0 + n - 1) / kCk
+      float *ck = Q.ckD + (((size_t)bh * Q.nck + (t0 + n - 1) / kCk) * dv + j) * dk;
+#pragma unroll
+      for (int e = 0; e < CPL; e += 4)
+        if (s * CPL + e < dk)
+          *reinterpret_cast<float4 *>(ck + s * CPL + e) = make_float4(D[e], D[e + 1], D[e + 2], D[e + 3]);
+    }
     for (int tt = n - 1; tt >= 0; --tt) {
       const float *sv = buf + tt * TS + s * SS;
       const float cg = Q.dO ? cq * ld_row<Tin>(buf + tt * TS + 4 * VS, rl) : 0.f;
@@ -573,7 +595,8 @@ __device__ __forceinline__ void ld_rows4<__nv_bfloat16>(const float *sv, int j, 
 // Column sweeps F2 / R2. CTA = d_k threads, thread i = key channel i, holding
 // rows j0 .. j0 + R - 1 of that column; with delta (F2) or dd (R2) known the
 // rows need no reduction, and the column sums over the CTA's rows are
-// per-thread. Per token the CTA writes its row group's partial sums to
+// per-thread. With no feedback left, every kCk-token chunk runs on its own
+// CTA from the checkpoint F1 (state) or R1 (cotangent) left at its boundary. Per token the CTA writes its row group's partial sums to
 // part[g][bh][t][3][d_k] (slots: c S^T dO, -P^T dd, dS~^T delta).
 
 // Stages R floats of a per-row workspace vector (delta or dd) of token t.
@@ -589,15 +612,18 @@ __global__ void __launch_bounds__(128) f2_kernel(const BParams Q) {
   float *sm = reinterpret_cast<float *>(smem4);
   const KParams &P = Q.P;
   const int dk = P.dk, dv = P.dv, T = P.T, BH = P.B * P.H;
-  const int bh = blockIdx.x / Q.G, g = blockIdx.x % Q.G, j0 = g * R;
+  // one CTA per (batch-head, kCk-token chunk, row group)
+  const int bh = blockIdx.x / (Q.nck * Q.G), ck = (blockIdx.x / Q.G) % Q.nck;
+  const int g = blockIdx.x % Q.G, j0 = g * R;
+  const int tb = ck * kCk, te = min(T, tb + kCk);  // this CTA's tokens
   const int i = threadIdx.x;
   const float cq = P.q_scale;
   const int TS = 2 * dk + 3 * R;  // w | alpha | delta | dd | dO (raw)
   const int nv = dk / 2, nr = R / 4, nd = Q.dO ? R * (int)sizeof(Tin) / 16 : 0;
-  const int nc = (T + kLC - 1) / kLC;
+  const int nc = (te - tb + kLCC - 1) / kLCC;
   auto issue = [&](int ch) {
-    float *buf = sm + (ch & 1) * kLC * TS;
-    const int t0 = ch * kLC, n = min(kLC, T - t0), per = nv + 2 * nr + nd;
+    float *buf = sm + (ch & 1) * kLCC * TS;
+    const int t0 = tb + ch * kLCC, n = min(kLCC, te - t0), per = nv + 2 * nr + nd;
     for (int tt = 0; tt < n; ++tt)
     for (int k = threadIdx.x; k < per; k += blockDim.x) {
       const int t = t0 + tt;
@@ -614,7 +640,7 @@ __global__ void __launch_bounds__(128) f2_kernel(const BParams Q) {
   };
   float S[R];
 #pragma unroll
-  for (int j = 0; j < R; ++j) S[j] = P.S0 ? P.S0[((size_t)bh * dv + j0 + j) * dk + i] : 0.f;
+  for (int j = 0; j < R; ++j) S[j] = Q.ckS[(((size_t)bh * Q.nck + ck) * dv + j0 + j) * dk + i];
   issue(0);
   cp_async_commit();
   for (int ch = 0; ch < nc; ++ch) {
@@ -622,8 +648,8 @@ __global__ void __launch_bounds__(128) f2_kernel(const BParams Q) {
     cp_async_commit();
     cp_async_wait_group<1>();
     __syncthreads();
-    const float *buf = sm + (ch & 1) * kLC * TS;
-    const int t0 = ch * kLC, n = min(kLC, T - t0);
+    const float *buf = sm + (ch & 1) * kLCC * TS;
+    const int t0 = tb + ch * kLCC, n = min(kLCC, te - t0);
     for (int tt = 0; tt < n; ++tt) {
       const float *sv = buf + tt * TS;
       const float w = sv[i], a = sv[dk + i];
@@ -662,15 +688,18 @@ __global__ void __launch_bounds__(128) r2_kernel(const BParams Q) {
   float *sm = reinterpret_cast<float *>(smem4);
   const KParams &P = Q.P;
   const int dk = P.dk, dv = P.dv, T = P.T, BH = P.B * P.H;
-  const int bh = blockIdx.x / Q.G, g = blockIdx.x % Q.G, j0 = g * R;
+  // one CTA per (batch-head, kCk-token chunk, row group)
+  const int bh = blockIdx.x / (Q.nck * Q.G), ck = (blockIdx.x / Q.G) % Q.nck;
+  const int g = blockIdx.x % Q.G, j0 = g * R;
+  const int tb = ck * kCk, te = min(T, tb + kCk);  // this CTA's tokens
   const int i = threadIdx.x;
   const float cq = P.q_scale;
   const int TS = 4 * dk + 3 * R;  // q' | r | w | alpha | delta | dd | dO (raw)
   const int nv = dk, nr = R / 4, nd = Q.dO ? R * (int)sizeof(Tin) / 16 : 0;
-  const int nc = (T + kLC - 1) / kLC;
+  const int nc = (te - tb + kLCC - 1) / kLCC;
   auto issue = [&](int ch) {
-    float *buf = sm + (ch & 1) * kLC * TS;
-    const int t0 = ch * kLC, n = min(kLC, T - t0), per = nv + 2 * nr + nd;
+    float *buf = sm + (ch & 1) * kLCC * TS;
+    const int t0 = tb + ch * kLCC, n = min(kLCC, te - t0), per = nv + 2 * nr + nd;
     for (int tt = 0; tt < n; ++tt)
     for (int k = threadIdx.x; k < per; k += blockDim.x) {
       const int t = t0 + tt;
@@ -687,7 +716,7 @@ __global__ void __launch_bounds__(128) r2_kernel(const BParams Q) {
   };
   float D[R];
 #pragma unroll
-  for (int j = 0; j < R; ++j) D[j] = Q.dST ? Q.dST[((size_t)bh * dv + j0 + j) * dk + i] : 0.f;
+  for (int j = 0; j < R; ++j) D[j] = Q.ckD[(((size_t)bh * Q.nck + ck) * dv + j0 + j) * dk + i];
   if (nc > 0) issue(nc - 1);
   cp_async_commit();
   for (int ch = nc - 1; ch >= 0; --ch) {
@@ -695,8 +724,8 @@ __global__ void __launch_bounds__(128) r2_kernel(const BParams Q) {
     cp_async_commit();
     cp_async_wait_group<1>();
     __syncthreads();
-    const float *buf = sm + (ch & 1) * kLC * TS;
-    const int t0 = ch * kLC, n = min(kLC, T - t0);
+    const float *buf = sm + (ch & 1) * kLCC * TS;
+    const int t0 = tb + ch * kLCC, n = min(kLCC, te - t0);
     for (int tt = n - 1; tt >= 0; --tt) {
       const float *sv = buf + tt * TS;
       const float q = sv[i], r = sv[dk + i], a = sv[3 * dk + i];
@@ -971,14 +1000,14 @@ cudaError_t launch_bwd_t(const BParams &Q, cudaStream_t st) {
   constexpr int VS = kLPR * seg_stride(CPL);
   const size_t sm_f1 = 2 * kLCR * (3 * VS + kRowsF) * sizeof(float);
   const size_t sm_r1 = 2 * kLCR * (4 * VS + kRowsF) * sizeof(float);
-  const size_t sm_f2 = 2 * kLC * (2 * dk + 3 * R) * sizeof(float);
-  const size_t sm_r2 = 2 * kLC * (4 * dk + 3 * R) * sizeof(float);
+  const size_t sm_f2 = 2 * kLCC * (2 * dk + 3 * R) * sizeof(float);
+  const size_t sm_r2 = 2 * kLCC * (4 * dk + 3 * R) * sizeof(float);
   if ((err = set_smem(f1_kernel<CPL>, sm_f1)) != cudaSuccess) return err;
   if ((err = set_smem(r1_kernel<Tin, CPL>, sm_r1)) != cudaSuccess) return err;
   if ((err = set_smem(f2_kernel<Tin, R>, sm_f2)) != cudaSuccess) return err;
   if ((err = set_smem(r2_kernel<Tin, R>, sm_r2)) != cudaSuccess) return err;
   const unsigned grid_rows = (unsigned)(BH * ((dv + kRowsF - 1) / kRowsF));
-  const unsigned grid_cols = (unsigned)(BH * Q.G);
+  const unsigned grid_cols = (unsigned)(BH * Q.nck * Q.G);
   f1_kernel<CPL><<<grid_rows, 128, sm_f1, st>>>(Q);
   r1_kernel<Tin, CPL><<<grid_rows, 128, sm_r1, st>>>(Q);
   f2_kernel<Tin, R><<<grid_cols, dk, sm_f2, st>>>(Q);
@@ -1045,7 +1074,8 @@ cudaError_t launch_chunk_bwd(const KParams &P, const pdn_grads_t *g, void *works
   Q.gen = ws + L.gen; Q.acc = ws + L.acc; Q.delta = ws + L.delta; Q.dd = ws + L.dd;
   Q.st = ws + L.st; Q.part = ws + L.part; Q.cpsi = ws + L.cpsi; Q.sigma = ws + L.sigma;
   Q.dacc = ws + L.dacc; Q.bsum = ws + L.bsum; Q.phi = ws + L.phi;
-  Q.GS = L.GS; Q.R = L.R; Q.G = L.G; Q.nb = L.nb;
+  Q.ckS = ws + L.ckS; Q.ckD = ws + L.ckD;
+  Q.GS = L.GS; Q.R = L.R; Q.G = L.G; Q.nb = L.nb; Q.nck = L.nck;
   // key channels per lane in the row sweeps: 8 lanes cover d_k
   const int cpl = P.dk <= 32 ? 4 : P.dk <= 64 ? 8 : 16;
   if (P.dtype == PDN_BF16) return launch_bwd_d<__nv_bfloat16>(Q, L.R, cpl, stream);
