@@ -72,7 +72,8 @@ static BwdPlan bwd_plan(const KParams &P) {
   const size_t BH = (size_t)P.B * P.H, T = (size_t)P.T;
   const int dk = P.dk, dv = P.dv;
   L.GS = 4 * dk + dv;
-  L.R = dv % 32 == 0 ? 32 : 16;  // F2 / R2 are chunk-parallel: wide row groups
+  // F2 / R2 are chunk-parallel: wide row groups (fewer partial sums)
+  L.R = dv % 64 == 0 ? 64 : dv % 32 == 0 ? 32 : 16;
   L.G = dv / L.R;
   L.nb = (int)((T + kScanBlk - 1) / kScanBlk);
   size_t off = 0;
@@ -1033,6 +1034,11 @@ cudaError_t launch_bwd_t(const BParams &Q, cudaStream_t st) {
 
 template <typename Tin>
 cudaError_t launch_bwd_d(const BParams &Q, int R, int cpl, cudaStream_t st) {
+  if (R == 64) {
+    if (cpl == 16) return launch_bwd_t<Tin, 64, 16>(Q, st);
+    if (cpl == 8) return launch_bwd_t<Tin, 64, 8>(Q, st);
+    return launch_bwd_t<Tin, 64, 4>(Q, st);
+  }
   if (R == 32) {
     if (cpl == 16) return launch_bwd_t<Tin, 32, 16>(Q, st);
     if (cpl == 8) return launch_bwd_t<Tin, 32, 8>(Q, st);
