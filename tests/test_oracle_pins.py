@@ -392,6 +392,36 @@ def test_backward_matches_central_differences(variant, decay):
         np.testing.assert_allclose(ga, num, rtol=2e-6, atol=2e-7, err_msg=name)
 
 
+@pytest.mark.parametrize("decay", ["scalar", "channel"])
+def test_decay_gradient_suffix_sum(decay):
+    """The decay gradient as a suffix sum over tokens (the form the CUDA
+    backward uses; no per-token state): with psi_t,i the cotangent of
+    log alpha_t,i and S_t = P_t + delta_t w_t^T,
+        psi_t = psi_{t+1} + q'_t . dq'_t - w_t . dw_t + r_t . dr_t,
+        psi_T,i = sum_j S_T[j,i] dS_T[j,i].
+    Checked in fp64 against the oracle's directly computed gradient
+    (sum_j S_{t-1}[j,i] dP_t[j,i] alpha_t,i) on GDN-2, whose (r, w, q')
+    cotangents follow from its input gradients: dr = derase / k,
+    dw = dk - e . dr, dq' = dq."""
+    rng = np.random.default_rng(61)
+    d = rand_inputs("GDN2", B=1, T=12, H=2, dk=6, dv=5, seed=60, decay=decay)
+    d["log_alpha"] = d["log_alpha"] * 2.0
+    dO = rng.standard_normal(d["v"].shape)
+    dST = rng.standard_normal(d["S0"].shape)
+    g = oracle.backward("GDN2", **d, dO=dO, dST=dST, q_scale=0.7)
+    _, ST, _ = oracle.forward("GDN2", d["q"], d["k"], d["v"], log_alpha=d["log_alpha"],
+                           erase=d["erase"], write=d["write"], S0=d["S0"], q_scale=0.7)
+    k, e, q = d["k"], d["erase"], d["q"]
+    dr = g["erase"] / k
+    dw = g["k"] - e * dr
+    r, w = e * k, k
+    term = q * g["q"] - w * dw + r * dr                      # [B,T,H,dk]
+    psi = np.einsum("bhji,bhji->bhi", ST, dST)[:, None]        # psi_T, [B,1,H,dk]
+    suffix = np.flip(np.cumsum(np.flip(term, axis=1), axis=1), axis=1) + psi
+    want = suffix.sum(axis=3) if decay == "scalar" else suffix
+    np.testing.assert_allclose(g["log_alpha"], want, rtol=1e-9, atol=1e-12)
+
+
 # ---------------------------------------------------------------- P7
 @pytest.mark.parametrize("lam", [0.5, 2.0])
 def test_p7_exact_preconditioning_is_least_squares(lam):
