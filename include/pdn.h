@@ -67,7 +67,10 @@ typedef enum {
   PDN_ERR_UNSUPPORTED = 2, /* valid problem that this build has no kernel for */
   PDN_ERR_CUDA = 3,        /* a CUDA runtime call or kernel launch failed */
   PDN_ERR_TIMEOUT = 4,     /* a bounded device wait ran out (device error word) */
-  PDN_ERR_WORKSPACE = 5    /* workspace pointer NULL or smaller than required */
+  PDN_ERR_WORKSPACE = 5,   /* workspace pointer NULL or smaller than required */
+  PDN_ERR_BOUNDS = 6       /* debug build only (libpdn_debug.so): an index check in
+                              a kernel failed; the access was skipped (device
+                              error word) */
 } pdn_status_t;
 
 /* Variant: the gain / preconditioner axes of the pages' decay-gain-

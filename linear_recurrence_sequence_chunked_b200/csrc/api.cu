@@ -381,6 +381,7 @@ extern "C" const char *pdn_status_string(pdn_status_t s) {
     case PDN_ERR_CUDA: return "PDN_ERR_CUDA";
     case PDN_ERR_TIMEOUT: return "PDN_ERR_TIMEOUT";
     case PDN_ERR_WORKSPACE: return "PDN_ERR_WORKSPACE";
+    case PDN_ERR_BOUNDS: return "PDN_ERR_BOUNDS";
   }
   return "PDN_ERR_UNKNOWN";
 }

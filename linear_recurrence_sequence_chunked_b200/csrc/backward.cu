@@ -109,6 +109,8 @@ struct BParams {
   // entering each chunk's last token (R1): [BH][nck][d_v][d_k]
   float *ckS, *ckD;
   int GS, R, G, nb, nck;
+  // element counts of the workspace arrays (index checks of the debug build)
+  size_t n_rows, n_part, n_ck;
 };
 
 // Generic vectors of one token, in the workspace order q'|r|w|a|u.
@@ -426,8 +428,9 @@ __global__ void __launch_bounds__(128) f1_kernel(const BParams Q) {
     __syncthreads();
     const float *buf = sm + (ch & 1) * kLCR * TS;
     const int t0 = ch * kLCR, n = min(kLCR, T - t0);
-    if (t0 % kCk == 0 && rok) {  // the state before chunk t0 / kCk
-      float *ck = Q.ckS + (((size_t)bh * Q.nck + t0 / kCk) * dv + j) * dk;
+    const size_t cks = (((size_t)bh * Q.nck + t0 / kCk) * dv + j) * dk;
+    if (t0 % kCk == 0 && rok && in_bounds(P.err, cks + dk <= Q.n_ck)) {  // the state before chunk t0 / kCk
+      float *ck = Q.ckS + cks;
 #pragma unroll
       for (int e = 0; e < CPL; e += 4)
         if (s * CPL + e < dk)
@@ -459,7 +462,8 @@ __global__ void __launch_bounds__(128) f1_kernel(const BParams Q) {
         S[e + 2] = fmaf(d, w.z, S[e + 2]);
         S[e + 3] = fmaf(d, w.w, S[e + 3]);
       }
-      if (s == 0 && rok) Q.delta[((size_t)bh * T + t0 + tt) * dv + j] = d;
+      const size_t di = ((size_t)bh * T + t0 + tt) * dv + j;
+      if (s == 0 && rok && in_bounds(P.err, di < Q.n_rows)) Q.delta[di] = d;
     }
     __syncthreads();  // the buffer is refilled two chunks on
   }
@@ -525,8 +529,10 @@ __global__ void __launch_bounds__(128) r1_kernel(const BParams Q) {
     __syncthreads();
     const float *buf = sm + (ch & 1) * kLCR * TS;
     const int t0 = ch * kLCR, n = min(kLCR, T - t0);
-    if (((t0 + n) % kCk == 0 || t0 + n == T) && rok) {  // entering chunk (t0 + n - 1) / kCk
-      float *ck = Q.ckD + (((size_t)bh * Q.nck + (t0 + n - 1) / kCk) * dv + j) * dk;
+    const size_t ckd = (((size_t)bh * Q.nck + (t0 + n - 1) / kCk) * dv + j) * dk;
+    if (((t0 + n) % kCk == 0 || t0 + n == T) && rok &&
+        in_bounds(P.err, ckd + dk <= Q.n_ck)) {  // entering chunk (t0 + n - 1) / kCk
+      float *ck = Q.ckD + ckd;
 #pragma unroll
       for (int e = 0; e < CPL; e += 4)
         if (s * CPL + e < dk)
@@ -562,7 +568,8 @@ __global__ void __launch_bounds__(128) r1_kernel(const BParams Q) {
         D[e + 2] = fmaf(-dd, r.z, D[e + 2]) * a.z;
         D[e + 3] = fmaf(-dd, r.w, D[e + 3]) * a.w;
       }
-      if (s == 0 && rok) Q.dd[((size_t)bh * T + t0 + tt) * dv + j] = dd;
+      const size_t di = ((size_t)bh * T + t0 + tt) * dv + j;
+      if (s == 0 && rok && in_bounds(P.err, di < Q.n_rows)) Q.dd[di] = dd;
     }
     __syncthreads();
   }
@@ -600,6 +607,14 @@ __device__ __forceinline__ void ld_rows4<__nv_bfloat16>(const float *sv, int j, 
 // CTA from the checkpoint F1 (state) or R1 (cotangent) left at its boundary. Per token the CTA writes its row group's partial sums to
 // part[g][bh][t][3][d_k] (slots: c S^T dO, -P^T dd, dS~^T delta).
 
+// Offset of rows j0 .. j0 + R - 1 of token t in a [BH][T][d_v] workspace
+// vector (0, after recording the error, when the debug build finds it out of
+// range).
+__device__ __forceinline__ size_t row_base(const BParams &Q, int bh, int t, int j0, int R) {
+  const size_t e = ((size_t)bh * Q.P.T + t) * Q.P.dv + j0;
+  return in_bounds(Q.P.err, e + R <= Q.n_rows) ? e : 0;
+}
+
 // Stages R floats of a per-row workspace vector (delta or dd) of token t.
 __device__ __forceinline__ void stage_rows(const float *src, int part, float *dst) {
   cp_async16(smem_u32(dst + 4 * part), src + 4 * part, true);
@@ -632,16 +647,19 @@ __global__ void __launch_bounds__(128) f2_kernel(const BParams Q) {
       if (k < nv)
         cp_async16(smem_u32(d + 4 * k), gen_at(Q, bh, t) + 2 * dk + 4 * k, true);
       else if (k < nv + nr)
-        stage_rows(Q.delta + ((size_t)bh * T + t) * dv + j0, k - nv, d + 2 * dk);
+        stage_rows(Q.delta + row_base(Q, bh, t, j0, R), k - nv, d + 2 * dk);
       else if (k < nv + 2 * nr)
-        stage_rows(Q.dd + ((size_t)bh * T + t) * dv + j0, k - nv - nr, d + 2 * dk + R);
+        stage_rows(Q.dd + row_base(Q, bh, t, j0, R), k - nv - nr, d + 2 * dk + R);
       else
         stage_dO<Tin>(Q, bh, t, j0, k - nv - 2 * nr, d + 2 * dk + 2 * R);
     }
   };
   float S[R];
 #pragma unroll
-  for (int j = 0; j < R; ++j) S[j] = Q.ckS[(((size_t)bh * Q.nck + ck) * dv + j0 + j) * dk + i];
+  for (int j = 0; j < R; ++j) {
+    const size_t e = (((size_t)bh * Q.nck + ck) * dv + j0 + j) * dk + i;
+    S[j] = in_bounds(P.err, e < Q.n_ck) ? Q.ckS[e] : 0.f;
+  }
   issue(0);
   cp_async_commit();
   for (int ch = 0; ch < nc; ++ch) {
@@ -673,9 +691,11 @@ __global__ void __launch_bounds__(128) f2_kernel(const BParams Q) {
           accq = fmaf(S[j + e], go[e], accq);
         }
       }
-      float *o = Q.part + (((size_t)g * BH + bh) * T + t0 + tt) * 3 * dk;
-      o[i] = cq * accq;
-      o[dk + i] = -accr;
+      const size_t po = (((size_t)g * BH + bh) * T + t0 + tt) * 3 * dk;
+      if (in_bounds(P.err, po + 3 * dk <= Q.n_part)) {
+        Q.part[po + i] = cq * accq;
+        Q.part[po + dk + i] = -accr;
+      }
     }
     __syncthreads();
   }
@@ -708,16 +728,19 @@ __global__ void __launch_bounds__(128) r2_kernel(const BParams Q) {
       if (k < nv)
         cp_async16(smem_u32(d + 4 * k), gen_at(Q, bh, t) + 4 * k, true);
       else if (k < nv + nr)
-        stage_rows(Q.delta + ((size_t)bh * T + t) * dv + j0, k - nv, d + 4 * dk);
+        stage_rows(Q.delta + row_base(Q, bh, t, j0, R), k - nv, d + 4 * dk);
       else if (k < nv + 2 * nr)
-        stage_rows(Q.dd + ((size_t)bh * T + t) * dv + j0, k - nv - nr, d + 4 * dk + R);
+        stage_rows(Q.dd + row_base(Q, bh, t, j0, R), k - nv - nr, d + 4 * dk + R);
       else
         stage_dO<Tin>(Q, bh, t, j0, k - nv - 2 * nr, d + 4 * dk + 2 * R);
     }
   };
   float D[R];
 #pragma unroll
-  for (int j = 0; j < R; ++j) D[j] = Q.ckD[(((size_t)bh * Q.nck + ck) * dv + j0 + j) * dk + i];
+  for (int j = 0; j < R; ++j) {
+    const size_t e = (((size_t)bh * Q.nck + ck) * dv + j0 + j) * dk + i;
+    D[j] = in_bounds(P.err, e < Q.n_ck) ? Q.ckD[e] : 0.f;
+  }
   if (nc > 0) issue(nc - 1);
   cp_async_commit();
   for (int ch = nc - 1; ch >= 0; --ch) {
@@ -749,7 +772,8 @@ __global__ void __launch_bounds__(128) r2_kernel(const BParams Q) {
           D[j + e] = fmaf(-dd[e], r, dt) * a;
         }
       }
-      Q.part[(((size_t)g * BH + bh) * T + t0 + tt) * 3 * dk + 2 * dk + i] = accw;
+      const size_t po = (((size_t)g * BH + bh) * T + t0 + tt) * 3 * dk;
+      if (in_bounds(P.err, po + 3 * dk <= Q.n_part)) Q.part[po + 2 * dk + i] = accw;
     }
     __syncthreads();
   }
@@ -778,7 +802,9 @@ __global__ void e1_kernel(const BParams Q) {
 #pragma unroll
     for (int e = 0; e < 4; ++e) dq[e] = dr[e] = dw[e] = 0.f;
     for (int g = 0; g < Q.G; ++g) {
-      const float *pp = Q.part + (((size_t)g * BH + bh) * T + t) * 3 * dk + c;
+      size_t po = (((size_t)g * BH + bh) * T + t) * 3 * dk;
+      if (!in_bounds(P.err, po + 3 * dk <= Q.n_part)) po = 0;
+      const float *pp = Q.part + po + c;
       float x[4], y[4], z[4];
       ld4(pp, ak, x);
       ld4(pp + dk, ak, y);
@@ -1082,6 +1108,9 @@ cudaError_t launch_chunk_bwd(const KParams &P, const pdn_grads_t *g, void *works
   Q.dacc = ws + L.dacc; Q.bsum = ws + L.bsum; Q.phi = ws + L.phi;
   Q.ckS = ws + L.ckS; Q.ckD = ws + L.ckD;
   Q.GS = L.GS; Q.R = L.R; Q.G = L.G; Q.nb = L.nb; Q.nck = L.nck;
+  Q.n_rows = (size_t)BH * P.T * P.dv;
+  Q.n_part = (size_t)L.G * BH * P.T * 3 * P.dk;
+  Q.n_ck = (size_t)BH * L.nck * P.dv * P.dk;
   // key channels per lane in the row sweeps: 8 lanes cover d_k
   const int cpl = P.dk <= 32 ? 4 : P.dk <= 64 ? 8 : 16;
   if (P.dtype == PDN_BF16) return launch_bwd_d<__nv_bfloat16>(Q, L.R, cpl, stream);

@@ -45,6 +45,13 @@ constexpr size_t WS_CH = 82944;     // bytes per block (256-aligned)
 
 // Chunk-major: the blocks of one chunk index, over all (batch, head), are
 // adjacent, so the state pass's concurrent loads stream one contiguous range.
+// A chunk index as the kernels use it; the debug build checks it against the
+// problem's chunk count (recording PDN_ERR_BOUNDS and taking chunk 0, so
+// that no copy another warp waits for is skipped).
+__device__ __forceinline__ int chunk_ok(const KParams &P, int c) {
+  return in_bounds(P.err, c >= 0 && c < (P.T + kC - 1) / kC) ? c : 0;
+}
+
 __device__ __forceinline__ uint8_t *ws_block(void *ws, int bh, int BH, int c) {
   return reinterpret_cast<uint8_t *>(ws) + ((size_t)c * BH + bh) * WS_CH;
 }
@@ -429,7 +436,7 @@ __global__ void __launch_bounds__(kK1Threads, kDecay == PDN_DECAY_CHANNEL ? 1 : 
   const int b = bh / P.H, h = bh % P.H;
   const int c0 = c * kC, Cn = min(kC, P.T - c0);
   const size_t tok0 = tok_index(P, b, c0, h) * kD;  // element offset of token c0
-  uint8_t *blk = ws_block(ws, bh, P.B * P.H, c);
+  uint8_t *blk = ws_block(ws, bh, P.B * P.H, chunk_ok(P, c));
   const uint32_t par = (uint32_t)(iter & 1);  // mbarrier parity of this block's MMAs
 
   // ---- P0: k (staged a block ahead) into its padded rows; q (and the
@@ -1374,9 +1381,9 @@ __global__ void __launch_bounds__(kK2Threads, 1) k2_state(const KParams P, void 
     if (lane == 0) {
       const int BH = P.B * P.H;
       for (int m = 0; m < 3 && m < N; ++m)
-        load_main(smem + main_buf(m), ws_block(ws, bh, BH, cb + m), B.fmain + m);
+        load_main(smem + main_buf(m), ws_block(ws, bh, BH, chunk_ok(P, cb + m)), B.fmain + m);
       for (int m = 0; m < 2 && m < N; ++m)
-        load_ut(smem + ut_buf(m), ws_block(ws, bh, BH, cb + m), B.fut + m);
+        load_ut(smem + ut_buf(m), ws_block(ws, bh, BH, chunk_ok(P, cb + m)), B.fut + m);
       // after MMA3 of chunk n, its U/T buffer takes chunk n + 2; after every
       // MMA of chunk n, its main buffer takes chunk n + 3
       for (int n = 0; n + 2 < N; ++n) {
@@ -1384,13 +1391,14 @@ __global__ void __launch_bounds__(kK2Threads, 1) k2_state(const KParams P, void 
           *abort_flag = 1;
           break;
         }
-        load_ut(smem + ut_buf(n), ws_block(ws, bh, BH, cb + n + 2), B.fut + (n & 1));
+        load_ut(smem + ut_buf(n), ws_block(ws, bh, BH, chunk_ok(P, cb + n + 2)), B.fut + (n & 1));
         if (n + 3 < N) {
           if (!k2_wait(B.mfree + (n % 3), (uint32_t)((n / 3) & 1), abort_flag)) {
             *abort_flag = 1;
             break;
           }
-          load_main(smem + main_buf(n), ws_block(ws, bh, BH, cb + n + 3), B.fmain + (n % 3));
+          load_main(smem + main_buf(n), ws_block(ws, bh, BH, chunk_ok(P, cb + n + 3)),
+                    B.fmain + (n % 3));
         }
       }
     }
@@ -1404,7 +1412,7 @@ __global__ void __launch_bounds__(kK2Threads, 1) k2_state(const KParams P, void 
     auto fetch_e = [&](int c) {
       if (lane < 8)
         cp_async16(sb + K2_EBUF + (warp * 2 + (c & 1)) * 128 + lane * 16,
-                   reinterpret_cast<const float *>(ws_block(ws, bh, P.B * P.H, cb + c) + WS_E) + 32 * cg +
+                   reinterpret_cast<const float *>(ws_block(ws, bh, P.B * P.H, chunk_ok(P, cb + c)) + WS_E) + 32 * cg +
                        4 * lane,
                    true);
       cp_async_commit();

@@ -113,4 +113,17 @@ __device__ __forceinline__ void record_error(int *err, int code) {
   if (err) atomicCAS(err, 0, code);
 }
 
+// Index checks of the debug build (compiled with PDN_DEBUG_BOUNDS, shipped as
+// libpdn_debug.so): `in_bounds(err, idx < n)` records PDN_ERR_BOUNDS in the
+// device error word when the condition fails, and the caller skips the
+// access. In the release build it is the constant true and vanishes.
+#ifdef PDN_DEBUG_BOUNDS
+__device__ __forceinline__ bool in_bounds(int *err, bool ok) {
+  if (!ok) record_error(err, PDN_ERR_BOUNDS);
+  return ok;
+}
+#else
+__device__ __forceinline__ constexpr bool in_bounds(int *, bool) { return true; }
+#endif
+
 }  // namespace pdn

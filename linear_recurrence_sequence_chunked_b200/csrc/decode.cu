@@ -233,7 +233,12 @@ __global__ void __launch_bounds__(kTmaThreads, 1) decode_tma_kernel(const KParam
   const int G = gridDim.x;
   const int nloc = blockIdx.x < items ? (items - blockIdx.x + G - 1) / G : 0;
   const bool precond = is_precond(P.variant);
-  auto state_of = [&](int k) { return P.ST + (size_t)(blockIdx.x + k * G) * (kD128 * kD128); };
+  // (the debug build checks the item index; a bad one records PDN_ERR_BOUNDS
+  // and streams item 0 instead, so that no copy a consumer waits for is lost)
+  auto state_of = [&](int k) {
+    const int it = blockIdx.x + k * G;
+    return P.ST + (size_t)(in_bounds(P.err, it < items) ? it : 0) * (kD128 * kD128);
+  };
 
   if (tid == 0) {
     for (int s = 0; s < kTmaBufs; ++s) {

@@ -17,10 +17,14 @@ from typing import Optional
 
 import torch
 
-_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libpdn.so")
+# The release library; PDN_LIBRARY may name another build of the same ABI
+# (libpdn_debug.so: the kernels' index checks compiled in).
+_LIB_PATH = os.environ.get("PDN_LIBRARY") or os.path.join(
+    os.path.dirname(os.path.abspath(__file__)), "libpdn.so")
+DEBUG_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libpdn_debug.so")
 
 PDN_OK, PDN_ERR_INVALID_ARG, PDN_ERR_UNSUPPORTED, PDN_ERR_CUDA, PDN_ERR_TIMEOUT, \
-    PDN_ERR_WORKSPACE = range(6)
+    PDN_ERR_WORKSPACE, PDN_ERR_BOUNDS = range(7)
 VARIANTS = {"DN": 0, "GDN": 1, "KDA": 2, "PDN": 3, "PGDN": 4, "PKDA": 5, "FG2_GDN": 6, "GDN2": 7,
             "PLA": 8, "FG2_GDN_PLUS": 9}
 DECAYS = {"none": 0, "scalar": 1, "channel": 2}

@@ -328,3 +328,16 @@ def test_backward_rules(lib):
 def load_bwd_null(lib):
     return lib.pdn_chunk_bwd(ctypes.byref(_problem()), ctypes.byref(_tensors()), None, None, 0,
                              None)
+
+
+def test_debug_library_exports_every_declared_symbol():
+    """libpdn_debug.so (index checks compiled in) offers the same C ABI."""
+    lib = pdn_build.build(debug_bounds=True)
+    out = subprocess.run(["nm", "-D", "--defined-only", lib], capture_output=True,
+                         text=True).stdout
+    for n in declared_functions():
+        assert re.search(r"\bT %s$" % n, out, flags=re.M), n
+
+
+def test_bounds_status_string(lib):
+    assert pdn.pdn_status_string(pdn.PDN_ERR_BOUNDS) == "PDN_ERR_BOUNDS"

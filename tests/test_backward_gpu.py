@@ -191,3 +191,16 @@ def test_backward_full_size_sampled(name, chains):
             else:
                 gs[n] = t[b:b + 1, :, h:h + 1].cpu().numpy()
         assert_grads(w, gs, gr, label="[b%d,h%d]" % (b, h))
+
+
+def test_backward_is_deterministic():
+    """Fixed-order reductions throughout (no atomics): two runs agree bitwise."""
+    w = small("PKDA", "bf16", T=150)
+    x = make_inputs(w)
+    S0, A0 = states(w)
+    dO, dST = cotangents(w)
+    a = run_gpu(w, x, S0, A0, dO, dST)
+    b = run_gpu(w, x, S0, A0, dO, dST)
+    for n in a:
+        if a[n] is not None:
+            assert np.array_equal(a[n], b[n]), n
