@@ -393,22 +393,36 @@ __global__ void __launch_bounds__(128) f1_kernel(const BParams Q) {
   const int s = lane & 7, rl = 4 * warp + (lane >> 3), j = j0 + rl;  // segment, local row, row
   const bool rok = j < dv;
   const int nc = (T + kLCR - 1) / kLCR;
+  // This thread's 16-byte piece of every staged token (at most one: 6 CPL +
+  // 4 <= 100 pieces for 128 threads), fixed for the whole sweep: vector
+  // pieces of r | w | alpha, then the u of the CTA's rows.
+  int src_off = 0, dst_off = 0;
+  bool piece = false, valid = false;
+  {
+    const int k = threadIdx.x;
+    constexpr int PV = kLPR * CPL / 4;  // pieces per vector
+    if (k < 6 * CPL) {
+      const int v = k / PV, col = 4 * (k % PV);
+      piece = true;
+      valid = col < dk;
+      src_off = dk + v * dk + (valid ? col : 0);
+      dst_off = v * VS + (col / CPL) * SS + col % CPL;
+    } else if (k < 6 * CPL + kRowsF / 4) {
+      const int r4 = 4 * (k - 6 * CPL);
+      piece = true;
+      valid = j0 + r4 < dv;
+      src_off = 4 * dk + (valid ? j0 + r4 : 0);
+      dst_off = 3 * VS + r4;
+    }
+  }
   auto issue = [&](int ch) {
     float *buf = sm + (ch & 1) * kLCR * TS;
     const int t0 = ch * kLCR, n = min(kLCR, T - t0);
-    for (int tt = 0; tt < n; ++tt) {
-      const float *g = gen_at(Q, bh, t0 + tt);
-      float *d = buf + tt * TS;
-      for (int k = threadIdx.x; k < 6 * CPL + kRowsF / 4; k += blockDim.x) {
-        if (k < 6 * CPL) {
-          stage_vec_piece<CPL>(g + dk, dk, k, d);
-        } else {
-          const int r4 = 4 * (k - 6 * CPL);
-          const bool ok = j0 + r4 < dv;
-          cp_async16(smem_u32(d + 3 * VS + r4), g + 4 * dk + (ok ? j0 + r4 : 0), ok);
-        }
-      }
-    }
+    if (!piece || !in_bounds(P.err, t0 + n <= T)) return;
+    const float *g = gen_at(Q, bh, t0) + src_off;
+    const uint32_t d = smem_u32(buf + dst_off);
+    for (int tt = 0; tt < n; ++tt)
+      cp_async16(d + tt * TS * 4, g + (size_t)tt * Q.GS, valid);
   };
   float S[CPL];
 #pragma unroll
@@ -497,17 +511,51 @@ __global__ void __launch_bounds__(128) r1_kernel(const BParams Q) {
   const float cq = P.q_scale;
   const int nd = Q.dO ? ND : 0;
   const int nc = (T + kLCR - 1) / kLCR;
+  // This thread's 16-byte pieces of every staged token (up to two: 8 CPL +
+  // ND <= 136 pieces for 128 threads), fixed for the whole sweep: vector
+  // pieces of q' | r | w | alpha (source: the token's generic vectors) and the
+  // dO of the CTA's rows (source: the token's dO row).
+  int src_off[2] = {0, 0}, dst_off[2] = {0, 0};
+  bool piece[2] = {false, false}, valid[2] = {false, false}, is_do[2] = {false, false};
+#pragma unroll
+  for (int p2 = 0; p2 < 2; ++p2) {
+    const int k = threadIdx.x + p2 * (int)blockDim.x;
+    constexpr int PV = kLPR * CPL / 4;
+    if (k < 8 * CPL) {
+      const int v = k / PV, col = 4 * (k % PV);
+      piece[p2] = true;
+      valid[p2] = col < dk;
+      src_off[p2] = v * dk + (valid[p2] ? col : 0);
+      dst_off[p2] = v * VS + (col / CPL) * SS + col % CPL;
+    } else if (k < 8 * CPL + nd) {
+      constexpr int per = 16 / (int)sizeof(Tin);  // dO rows per piece
+      const int part = k - 8 * CPL;
+      piece[p2] = true;
+      is_do[p2] = true;
+      valid[p2] = j0 + per * part < dv;
+      src_off[p2] = valid[p2] ? j0 + per * part : 0;  // elements into the token's dO row
+      dst_off[p2] = 4 * VS + 4 * part;
+    }
+  }
+  const size_t do_stride = (size_t)P.H * dv;  // dO elements from one token to the next
   auto issue = [&](int ch) {
     float *buf = sm + (ch & 1) * kLCR * TS;
     const int t0 = ch * kLCR, n = min(kLCR, T - t0);
-    for (int tt = 0; tt < n; ++tt) {
-      const float *g = gen_at(Q, bh, t0 + tt);
-      float *d = buf + tt * TS;
-      for (int k = threadIdx.x; k < 8 * CPL + nd; k += blockDim.x) {
-        if (k < 8 * CPL)
-          stage_vec_piece<CPL>(g, dk, k, d);
-        else
-          stage_dO<Tin>(Q, bh, t0 + tt, j0, k - 8 * CPL, d + 4 * VS);
+    if (!in_bounds(P.err, t0 + n <= T)) return;
+    const float *g = gen_at(Q, bh, t0);
+    const Tin *o0 = Q.dO ? reinterpret_cast<const Tin *>(Q.dO) +
+                               tok_index(P, bh / P.H, t0, bh % P.H) * dv
+                         : nullptr;
+#pragma unroll
+    for (int p2 = 0; p2 < 2; ++p2) {
+      if (!piece[p2]) continue;
+      const uint32_t d = smem_u32(buf + dst_off[p2]);
+      if (is_do[p2]) {
+        const Tin *src = o0 + src_off[p2];
+        for (int tt = 0; tt < n; ++tt) cp_async16(d + tt * TS * 4, src + tt * do_stride, valid[p2]);
+      } else {
+        const float *src = g + src_off[p2];
+        for (int tt = 0; tt < n; ++tt) cp_async16(d + tt * TS * 4, src + (size_t)tt * Q.GS, valid[p2]);
       }
     }
   };
