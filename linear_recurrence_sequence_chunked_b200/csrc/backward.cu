@@ -668,6 +668,61 @@ __device__ __forceinline__ void stage_rows(const float *src, int part, float *ds
   cp_async16(smem_u32(dst + 4 * part), src + 4 * part, true);
 }
 
+// One 16-byte piece of a staged token in F2 / R2: from the token's generic
+// vectors (kind 0), its delta or dd rows (1, 2) or its dO row (3); src counts
+// elements from that row's start (or, kind 0, from the token's vectors), dst
+// floats from the staged token's start. kind -1: no piece.
+struct ColPiece {
+  int kind, src, dst;
+  bool valid;
+};
+template <typename Tin>
+__device__ __forceinline__ ColPiece col_piece(int k, int gen_off, int nv, int rows_dst, int R,
+                                              int nd, int j0, int dv) {
+  const int nr = R / 4;
+  if (k < nv) return ColPiece{0, gen_off + 4 * k, 4 * k, true};
+  if (k < nv + nr) return ColPiece{1, j0 + 4 * (k - nv), rows_dst + 4 * (k - nv), true};
+  if (k < nv + 2 * nr)
+    return ColPiece{2, j0 + 4 * (k - nv - nr), rows_dst + R + 4 * (k - nv - nr), true};
+  if (k < nv + 2 * nr + nd) {
+    constexpr int per = 16 / (int)sizeof(Tin);  // dO rows per piece
+    const int part = k - nv - 2 * nr;
+    const bool ok = j0 + per * part < dv;
+    return ColPiece{3, ok ? j0 + per * part : 0, rows_dst + 2 * R + 4 * part, ok};
+  }
+  return ColPiece{-1, 0, 0, false};
+}
+
+// Issues the pieces pc of tokens t0 .. t0 + n - 1 into buf (TS floats per
+// token); per token each source advances by one row.
+template <typename Tin>
+__device__ __forceinline__ void col_issue(const BParams &Q, const ColPiece (&pc)[4], int bh, int t0,
+                                          int n, float *buf, int TS) {
+  const KParams &P = Q.P;
+  const int dv = P.dv;
+  if (!in_bounds(P.err, ((size_t)bh * P.T + t0 + n) * dv <= Q.n_rows)) return;
+  const float *g0 = gen_at(Q, bh, t0);
+  const float *de0 = Q.delta + ((size_t)bh * P.T + t0) * dv;
+  const float *dd0 = Q.dd + ((size_t)bh * P.T + t0) * dv;
+  const Tin *o0 = Q.dO ? reinterpret_cast<const Tin *>(Q.dO) + tok_index(P, bh / P.H, t0, bh % P.H) * dv
+                       : nullptr;
+  const size_t ostride = (size_t)P.H * dv;
+#pragma unroll
+  for (int p2 = 0; p2 < 4; ++p2) {
+    const ColPiece c = pc[p2];
+    if (c.kind < 0) continue;
+    const uint32_t d = smem_u32(buf + c.dst);
+    if (c.kind == 0) {
+      for (int tt = 0; tt < n; ++tt) cp_async16(d + tt * TS * 4, g0 + (size_t)tt * Q.GS + c.src, true);
+    } else if (c.kind == 3) {
+      for (int tt = 0; tt < n; ++tt) cp_async16(d + tt * TS * 4, o0 + tt * ostride + c.src, c.valid);
+    } else {
+      const float *r0 = (c.kind == 1 ? de0 : dd0) + c.src;
+      for (int tt = 0; tt < n; ++tt) cp_async16(d + tt * TS * 4, r0 + (size_t)tt * dv, true);
+    }
+  }
+}
+
 // F2: forward, S_t = S_{t-1} Diag(alpha_t) + delta_t w_t^T;
 // dq'_t = c S_t^T dO_t and dr_t = -P_t^T dd_t.
 template <typename Tin, int R>
@@ -685,11 +740,18 @@ __global__ void __launch_bounds__(128) f2_kernel(const BParams Q) {
   const int TS = 2 * dk + 3 * R;  // w | alpha | delta | dd | dO (raw)
   const int nv = dk / 2, nr = R / 4, nd = Q.dO ? R * (int)sizeof(Tin) / 16 : 0;
   const int nc = (te - tb + kLCC - 1) / kLCC;
+  // this thread's pieces of every staged token (w | alpha, delta, dd, dO)
+  ColPiece pc[4];
+#pragma unroll
+  for (int p2 = 0; p2 < 4; ++p2)
+    pc[p2] = col_piece<Tin>(threadIdx.x + p2 * (int)blockDim.x, 2 * dk, nv, 2 * dk, R, nd, j0, dv);
   auto issue = [&](int ch) {
     float *buf = sm + (ch & 1) * kLCC * TS;
     const int t0 = tb + ch * kLCC, n = min(kLCC, te - t0), per = nv + 2 * nr + nd;
+    col_issue<Tin>(Q, pc, bh, t0, n, buf, TS);
+    // (pieces past four per thread: no shape with d_k >= 16 and R <= 64 has any)
     for (int tt = 0; tt < n; ++tt)
-    for (int k = threadIdx.x; k < per; k += blockDim.x) {
+    for (int k = threadIdx.x + 4 * (int)blockDim.x; k < per; k += blockDim.x) {
       const int t = t0 + tt;
       float *d = buf + tt * TS;
       if (k < nv)
@@ -766,11 +828,18 @@ __global__ void __launch_bounds__(128) r2_kernel(const BParams Q) {
   const int TS = 4 * dk + 3 * R;  // q' | r | w | alpha | delta | dd | dO (raw)
   const int nv = dk, nr = R / 4, nd = Q.dO ? R * (int)sizeof(Tin) / 16 : 0;
   const int nc = (te - tb + kLCC - 1) / kLCC;
+  // this thread's pieces of every staged token (q' | r | w | alpha, delta, dd, dO)
+  ColPiece pc[4];
+#pragma unroll
+  for (int p2 = 0; p2 < 4; ++p2)
+    pc[p2] = col_piece<Tin>(threadIdx.x + p2 * (int)blockDim.x, 0, nv, 4 * dk, R, nd, j0, dv);
   auto issue = [&](int ch) {
     float *buf = sm + (ch & 1) * kLCC * TS;
     const int t0 = tb + ch * kLCC, n = min(kLCC, te - t0), per = nv + 2 * nr + nd;
+    col_issue<Tin>(Q, pc, bh, t0, n, buf, TS);
+    // (pieces past four per thread: no shape with d_k >= 16 and R <= 64 has any)
     for (int tt = 0; tt < n; ++tt)
-    for (int k = threadIdx.x; k < per; k += blockDim.x) {
+    for (int k = threadIdx.x + 4 * (int)blockDim.x; k < per; k += blockDim.x) {
       const int t = t0 + tt;
       float *d = buf + tt * TS;
       if (k < nv)
