@@ -320,99 +320,117 @@ __global__ void prep_gen_kernel(const BParams Q) {
 }
 
 // ---------------------------------------------------------------------------
-// Row sweeps F1 / R1. CTA = 4 warps = 16 consecutive state rows of one (batch,
-// head); in warp w, lanes 8p .. 8p + 7 share row j0 + 4w + p and lane 8p + s
-// holds key channels s CPL .. s CPL + CPL - 1 (CPL = 4, 8 or 16 by d_k), so a
-// row's reduction over key channels is three shuffles. The sequential chain
-// per token is short and there are many warps to interleave (the sweeps are
-// latency bound: one token after the other). The per-token vectors are
-// staged through shared memory kLCR tokens at a time with cp.async (double
-// buffered), each vector as eight CPL-float segments seg_stride(CPL) floats
-// apart, an odd multiple of four, so that the eight segments a quarter-warp
-// reads at once fall in different banks; key channels >= d_k are staged as
-// zeros.
-constexpr int kRowsF = 16;   // state rows per CTA
-constexpr int kLPR = 8;      // lanes per state row
-constexpr int kLCR = 8;      // tokens staged per chunk in F1 / R1
-__host__ __device__ constexpr int seg_stride(int cpl) { return cpl % 8 == 0 ? cpl + 4 : cpl; }
+// Row sweeps F1 / R1, blocked over rows in registers. A warp owns RW = 8
+// consecutive state rows of one (batch, head) -- a CTA, 4 warps, owns 32
+// rows -- and lane l holds key channels C l .. C l + C - 1 (C = 1, 2 or 4 by
+// d_k) of all of them, so every per-token vector a lane reads from shared
+// memory serves RW rows and the 32 lanes of one load read 32 distinct
+// pieces. (With lanes of different rows reading the same vector, a 16-byte
+// load is served a quarter-warp at a time and every row-token costs the whole
+// vector in shared-memory wavefronts: at the headline sizes that pipe, not the
+// arithmetic, bounds the sweeps.) The RW row reductions over key channels
+// share one transposed butterfly (rows_sum), and the finished row values
+// return to every lane by one shuffle each. The per-token vectors are staged
+// through shared memory kLCR tokens at a time with cp.async (double
+// buffered), each padded to 32 C floats with zeros.
+//
+// F1 and R1 share no data (F1 reads S0 and the generic vectors, R1 dS_T, dO
+// and the generic vectors), so they run as one launch, R1's CTAs first (the
+// longer sweep), both resident at once.
+constexpr int kLCR = 8;  // tokens staged per chunk in F1 / R1
 
 __device__ __forceinline__ void ld4(const float *p, bool ok, float (&v)[4]) {
   const float4 x = ok ? *reinterpret_cast<const float4 *>(p) : make_float4(0.f, 0.f, 0.f, 0.f);
   v[0] = x.x; v[1] = x.y; v[2] = x.z; v[3] = x.w;
 }
 
-// Stages consecutive d_k-vectors starting at `src` into the padded segment
-// layout at dst, one 16-byte piece per call (piece k: vector k / (2 CPL),
-// key channels 4 (k % (2 CPL)) .. + 3).
-template <int CPL>
-__device__ __forceinline__ void stage_vec_piece(const float *src, int dk, int k, float *dst) {
-  constexpr int SS = seg_stride(CPL), PV = kLPR * CPL / 4;  // pieces per vector
-  const int v = k / PV, col = 4 * (k % PV);
-  const int seg = col / CPL, off = col % CPL;
-  cp_async16(smem_u32(dst + v * kLPR * SS + seg * SS + off),
-             src + (size_t)v * dk + (col < dk ? col : 0), col < dk);
+// C consecutive floats (16-, 8- or 4-byte aligned) to registers and back;
+// a NULL source reads zeros.
+template <int C>
+__device__ __forceinline__ void ld_c(const float *p, float (&v)[C]) {
+  if constexpr (C == 4) {
+    const float4 x = p ? *reinterpret_cast<const float4 *>(p) : make_float4(0.f, 0.f, 0.f, 0.f);
+    v[0] = x.x; v[1] = x.y; v[2] = x.z; v[3] = x.w;
+  } else if constexpr (C == 2) {
+    const float2 x = p ? *reinterpret_cast<const float2 *>(p) : make_float2(0.f, 0.f);
+    v[0] = x.x; v[1] = x.y;
+  } else {
+    v[0] = p ? *p : 0.f;
+  }
+}
+template <int C>
+__device__ __forceinline__ void st_c(float *p, const float (&v)[C]) {
+  if constexpr (C == 4)
+    *reinterpret_cast<float4 *>(p) = make_float4(v[0], v[1], v[2], v[3]);
+  else if constexpr (C == 2)
+    *reinterpret_cast<float2 *>(p) = make_float2(v[0], v[1]);
+  else
+    *p = v[0];
 }
 
-// The dO entries of rows j0 .. j0 + nrow - 1 of token t (raw dtype), one
-// 16-byte piece; rows >= d_v are zero-filled.
-template <typename Tin>
-__device__ __forceinline__ void stage_dO(const BParams &Q, int bh, int t, int j0, int part,
-                                         float *dst) {
-  const KParams &P = Q.P;
-  constexpr int per = 16 / (int)sizeof(Tin);  // rows per piece
-  const bool ok = j0 + per * part < P.dv;
-  const char *src = reinterpret_cast<const char *>(Q.dO) +
-                    (tok_index(P, bh / P.H, t, bh % P.H) * P.dv + (ok ? j0 + per * part : 0)) *
-                        sizeof(Tin);
-  cp_async16(smem_u32(reinterpret_cast<char *>(dst) + 16 * part), src, ok);
+// Row sums of a warp's RW rows: p[r] is this lane's partial sum of row r. The
+// first log2(RW) exchanges (across lane bits 4, 3, ...) each hand half of the
+// partial sums a lane still carries to the partner lane and add the other
+// half to the partner's, so that afterwards lane l carries one value, row
+// l / (32 / RW) summed over RW lanes; the remaining xor levels finish it.
+// Returns the full sum of row l / (32 / RW) on every lane l.
+template <int RW>
+__device__ __forceinline__ float rows_sum(const float (&p)[RW], int lane) {
+  float c[RW];
+#pragma unroll
+  for (int r = 0; r < RW; ++r) c[r] = p[r];
+#pragma unroll
+  for (int n = RW, m = 16; n > 1; n >>= 1, m >>= 1) {
+    const bool hi = lane & m;  // this lane keeps the upper half of the rows it carries
+#pragma unroll
+    for (int k = 0; k < n / 2; ++k) {
+      const float send = hi ? c[k] : c[k + n / 2];
+      const float keep = hi ? c[k + n / 2] : c[k];
+      c[k] = keep + __shfl_xor_sync(0xffffffffu, send, m);
+    }
+  }
+  float v = c[0];
+#pragma unroll
+  for (int m = 16 / RW; m >= 1; m >>= 1) v += __shfl_xor_sync(0xffffffffu, v, m);
+  return v;
 }
 
-template <typename Tin>
-__device__ __forceinline__ float ld_row(const float *base, int j);
-template <>
-__device__ __forceinline__ float ld_row<float>(const float *base, int j) {
-  return base[j];
-}
-template <>
-__device__ __forceinline__ float ld_row<__nv_bfloat16>(const float *base, int j) {
-  return __bfloat162float(reinterpret_cast<const __nv_bfloat16 *>(base)[j]);
-}
-
-// F1: the forward recurrence, writing delta_t of every row, and S_T.
-template <int CPL>
-__global__ void __launch_bounds__(128) f1_kernel(const BParams Q) {
-  extern __shared__ float4 smem4[];
-  float *sm = reinterpret_cast<float *>(smem4);
-  constexpr int SS = seg_stride(CPL), VS = kLPR * SS;  // segment, vector strides
-  constexpr int TS = 3 * VS + kRowsF;                   // r | w | alpha | u of the 16 rows
+// F1: the forward recurrence, writing delta_t of every row, the state
+// checkpoints and S_T; `blk` numbers the CTA among F1's.
+template <int C, int RW>
+__device__ __forceinline__ void f1_body(const BParams &Q, int blk, float *sm) {
+  constexpr int VW = 32 * C;            // staged floats per vector
+  constexpr int NR = 4 * RW;            // rows per CTA
+  constexpr int TS = 3 * VW + NR;       // r | w | alpha | u of the CTA's rows
   const KParams &P = Q.P;
   const int dk = P.dk, dv = P.dv, T = P.T;
-  const int nrg = (dv + kRowsF - 1) / kRowsF;
-  const int bh = blockIdx.x / nrg, j0 = (blockIdx.x % nrg) * kRowsF;
+  const int nrg = (dv + NR - 1) / NR;
+  const int bh = blk / nrg, j0 = (blk % nrg) * NR;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int s = lane & 7, rl = 4 * warp + (lane >> 3), j = j0 + rl;  // segment, local row, row
-  const bool rok = j < dv;
+  const int jw = j0 + RW * warp;        // the warp's first row
+  const int jl = lane / (32 / RW);      // the row (of the warp's) rows_sum leaves on this lane
+  const int c0 = C * lane;              // this lane's first key channel
+  const bool cok = c0 < dk;
   const int nc = (T + kLCR - 1) / kLCR;
-  // This thread's 16-byte piece of every staged token (at most one: 6 CPL +
-  // 4 <= 100 pieces for 128 threads), fixed for the whole sweep: vector
-  // pieces of r | w | alpha, then the u of the CTA's rows.
+  // This thread's 16-byte piece of every staged token (at most one: 24 C +
+  // RW <= 104 pieces for 128 threads), fixed for the whole sweep: r | w |
+  // alpha, then the u of the CTA's rows.
   int src_off = 0, dst_off = 0;
   bool piece = false, valid = false;
   {
     const int k = threadIdx.x;
-    constexpr int PV = kLPR * CPL / 4;  // pieces per vector
-    if (k < 6 * CPL) {
-      const int v = k / PV, col = 4 * (k % PV);
+    if (k < 24 * C) {
+      const int v = k / (8 * C), col = 4 * (k % (8 * C));
       piece = true;
       valid = col < dk;
-      src_off = dk + v * dk + (valid ? col : 0);
-      dst_off = v * VS + (col / CPL) * SS + col % CPL;
-    } else if (k < 6 * CPL + kRowsF / 4) {
-      const int r4 = 4 * (k - 6 * CPL);
+      src_off = (v + 1) * dk + (valid ? col : 0);
+      dst_off = v * VW + col;
+    } else if (k < 24 * C + NR / 4) {
+      const int r4 = 4 * (k - 24 * C);
       piece = true;
       valid = j0 + r4 < dv;
       src_off = 4 * dk + (valid ? j0 + r4 : 0);
-      dst_off = 3 * VS + r4;
+      dst_off = 3 * VW + r4;
     }
   }
   auto issue = [&](int ch) {
@@ -424,15 +442,10 @@ __global__ void __launch_bounds__(128) f1_kernel(const BParams Q) {
     for (int tt = 0; tt < n; ++tt)
       cp_async16(d + tt * TS * 4, g + (size_t)tt * Q.GS, valid);
   };
-  float S[CPL];
+  float S[RW][C];
 #pragma unroll
-  for (int e = 0; e < CPL; e += 4) {
-    const int col = s * CPL + e;
-    float v[4];
-    ld4(rok && P.S0 && col < dk ? P.S0 + ((size_t)bh * dv + j) * dk + col : nullptr,
-        rok && P.S0 && col < dk, v);
-    S[e] = v[0]; S[e + 1] = v[1]; S[e + 2] = v[2]; S[e + 3] = v[3];
-  }
+  for (int r = 0; r < RW; ++r)
+    ld_c<C>(P.S0 && cok && jw + r < dv ? P.S0 + ((size_t)bh * dv + jw + r) * dk + c0 : nullptr, S[r]);
   issue(0);
   cp_async_commit();
   for (int ch = 0; ch < nc; ++ch) {
@@ -442,99 +455,113 @@ __global__ void __launch_bounds__(128) f1_kernel(const BParams Q) {
     __syncthreads();
     const float *buf = sm + (ch & 1) * kLCR * TS;
     const int t0 = ch * kLCR, n = min(kLCR, T - t0);
-    const size_t cks = (((size_t)bh * Q.nck + t0 / kCk) * dv + j) * dk;
-    if (t0 % kCk == 0 && rok && in_bounds(P.err, cks + dk <= Q.n_ck)) {  // the state before chunk t0 / kCk
-      float *ck = Q.ckS + cks;
+    if (t0 % kCk == 0 && cok) {  // the state before chunk t0 / kCk
+      const size_t cks = (((size_t)bh * Q.nck + t0 / kCk) * dv + jw) * dk + c0;
 #pragma unroll
-      for (int e = 0; e < CPL; e += 4)
-        if (s * CPL + e < dk)
-          *reinterpret_cast<float4 *>(ck + s * CPL + e) = make_float4(S[e], S[e + 1], S[e + 2], S[e + 3]);
+      for (int r = 0; r < RW; ++r)
+        if (jw + r < dv && in_bounds(P.err, cks + (size_t)r * dk + C <= Q.n_ck))
+          st_c<C>(Q.ckS + cks + (size_t)r * dk, S[r]);
     }
     for (int tt = 0; tt < n; ++tt) {
-      const float *sv = buf + tt * TS + s * SS;
-      float y[4] = {0.f, 0.f, 0.f, 0.f};
+      const float *sv = buf + tt * TS + c0;
+      float rr[C], ww[C], al[C];
+      ld_c<C>(sv, rr);
+      ld_c<C>(sv + VW, ww);
+      ld_c<C>(sv + 2 * VW, al);
+      float y[RW];
 #pragma unroll
-      for (int e = 0; e < CPL; e += 4) {
-        const float4 r = *reinterpret_cast<const float4 *>(sv + e);
-        const float4 a = *reinterpret_cast<const float4 *>(sv + 2 * VS + e);
-        S[e] *= a.x; S[e + 1] *= a.y; S[e + 2] *= a.z; S[e + 3] *= a.w;
-        y[0] = fmaf(S[e], r.x, y[0]);
-        y[1] = fmaf(S[e + 1], r.y, y[1]);
-        y[2] = fmaf(S[e + 2], r.z, y[2]);
-        y[3] = fmaf(S[e + 3], r.w, y[3]);
-      }
-      float yy = (y[0] + y[1]) + (y[2] + y[3]);
-      yy += __shfl_xor_sync(0xffffffffu, yy, 1);
-      yy += __shfl_xor_sync(0xffffffffu, yy, 2);
-      yy += __shfl_xor_sync(0xffffffffu, yy, 4);
-      const float d = buf[tt * TS + 3 * VS + rl] - yy;
+      for (int r = 0; r < RW; ++r) {
+        float acc = 0.f;
 #pragma unroll
-      for (int e = 0; e < CPL; e += 4) {
-        const float4 w = *reinterpret_cast<const float4 *>(sv + VS + e);
-        S[e] = fmaf(d, w.x, S[e]);
-        S[e + 1] = fmaf(d, w.y, S[e + 1]);
-        S[e + 2] = fmaf(d, w.z, S[e + 2]);
-        S[e + 3] = fmaf(d, w.w, S[e + 3]);
+        for (int e = 0; e < C; ++e) {
+          S[r][e] *= al[e];
+          acc = fmaf(S[r][e], rr[e], acc);
+        }
+        y[r] = acc;
       }
-      const size_t di = ((size_t)bh * T + t0 + tt) * dv + j;
-      if (s == 0 && rok && in_bounds(P.err, di < Q.n_rows)) Q.delta[di] = d;
+      // delta of row jw + jl, then every row's delta to every lane
+      const float d = buf[tt * TS + 3 * VW + RW * warp + jl] - rows_sum<RW>(y, lane);
+      const size_t di = ((size_t)bh * T + t0 + tt) * dv + jw + jl;
+      if (lane % (32 / RW) == 0 && jw + jl < dv && in_bounds(P.err, di < Q.n_rows)) Q.delta[di] = d;
+#pragma unroll
+      for (int r = 0; r < RW; ++r) {
+        const float dr = __shfl_sync(0xffffffffu, d, r * (32 / RW));
+#pragma unroll
+        for (int e = 0; e < C; ++e) S[r][e] = fmaf(dr, ww[e], S[r][e]);
+      }
     }
     __syncthreads();  // the buffer is refilled two chunks on
   }
-  if (rok) {
+  if (cok) {
 #pragma unroll
-    for (int e = 0; e < CPL; e += 4) {
-      const int col = s * CPL + e;
-      if (col < dk)
-        *reinterpret_cast<float4 *>(Q.st + ((size_t)bh * dv + j) * dk + col) =
-            make_float4(S[e], S[e + 1], S[e + 2], S[e + 3]);
+    for (int r = 0; r < RW; ++r)
+      if (jw + r < dv) st_c<C>(Q.st + ((size_t)bh * dv + jw + r) * dk + c0, S[r]);
+  }
+}
+
+// The dO entries of rows j .. j + RW - 1 as staged (raw dtype), widened to
+// fp32 and scaled by c.
+template <typename Tin, int RW>
+__device__ __forceinline__ void ld_dO_rows(const float *slot, int j, float c, float (&g)[RW]) {
+  if constexpr (sizeof(Tin) == 4) {
+#pragma unroll
+    for (int r = 0; r < RW; r += 4) {
+      const float4 x = *reinterpret_cast<const float4 *>(slot + j + r);
+      g[r] = c * x.x; g[r + 1] = c * x.y; g[r + 2] = c * x.z; g[r + 3] = c * x.w;
+    }
+  } else {
+    const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(
+        reinterpret_cast<const __nv_bfloat16 *>(slot) + j);
+#pragma unroll
+    for (int r = 0; r < RW; r += 2) {
+      const float2 x = __bfloat1622float2(h[r / 2]);
+      g[r] = c * x.x; g[r + 1] = c * x.y;
     }
   }
 }
 
-// R1: the reverse recurrence of the cotangent, writing dd_t of every row, and
-// dS0.
-template <typename Tin, int CPL>
-__global__ void __launch_bounds__(128) r1_kernel(const BParams Q) {
-  extern __shared__ float4 smem4[];
-  float *sm = reinterpret_cast<float *>(smem4);
-  constexpr int SS = seg_stride(CPL), VS = kLPR * SS;
-  constexpr int TS = 4 * VS + kRowsF;  // q' | r | w | alpha | dO of the 16 rows (raw)
-  constexpr int ND = kRowsF * (int)sizeof(Tin) / 16;
+// R1: the reverse recurrence of the cotangent, writing dd_t of every row, the
+// cotangent checkpoints and dS0; `blk` numbers the CTA among R1's.
+template <typename Tin, int C, int RW>
+__device__ __forceinline__ void r1_body(const BParams &Q, int blk, float *sm) {
+  constexpr int VW = 32 * C;
+  constexpr int NR = 4 * RW;
+  constexpr int TS = 4 * VW + NR;  // q' | r | w | alpha | dO of the CTA's rows (raw)
+  constexpr int ND = NR * (int)sizeof(Tin) / 16;  // dO pieces per token
   const KParams &P = Q.P;
   const int dk = P.dk, dv = P.dv, T = P.T;
-  const int nrg = (dv + kRowsF - 1) / kRowsF;
-  const int bh = blockIdx.x / nrg, j0 = (blockIdx.x % nrg) * kRowsF;
+  const int nrg = (dv + NR - 1) / NR;
+  const int bh = blk / nrg, j0 = (blk % nrg) * NR;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int s = lane & 7, rl = 4 * warp + (lane >> 3), j = j0 + rl;
-  const bool rok = j < dv;
+  const int jw = j0 + RW * warp, jl = lane / (32 / RW);
+  const int c0 = C * lane;
+  const bool cok = c0 < dk;
   const float cq = P.q_scale;
   const int nd = Q.dO ? ND : 0;
   const int nc = (T + kLCR - 1) / kLCR;
-  // This thread's 16-byte pieces of every staged token (up to two: 8 CPL +
-  // ND <= 136 pieces for 128 threads), fixed for the whole sweep: vector
-  // pieces of q' | r | w | alpha (source: the token's generic vectors) and the
-  // dO of the CTA's rows (source: the token's dO row).
+  // This thread's 16-byte pieces of every staged token (up to two: 32 C + ND
+  // <= 136 pieces for 128 threads), fixed for the whole sweep: q' | r | w |
+  // alpha (source: the token's generic vectors), then the dO of the CTA's
+  // rows (source: the token's dO row).
   int src_off[2] = {0, 0}, dst_off[2] = {0, 0};
   bool piece[2] = {false, false}, valid[2] = {false, false}, is_do[2] = {false, false};
 #pragma unroll
   for (int p2 = 0; p2 < 2; ++p2) {
     const int k = threadIdx.x + p2 * (int)blockDim.x;
-    constexpr int PV = kLPR * CPL / 4;
-    if (k < 8 * CPL) {
-      const int v = k / PV, col = 4 * (k % PV);
+    if (k < 32 * C) {
+      const int v = k / (8 * C), col = 4 * (k % (8 * C));
       piece[p2] = true;
       valid[p2] = col < dk;
       src_off[p2] = v * dk + (valid[p2] ? col : 0);
-      dst_off[p2] = v * VS + (col / CPL) * SS + col % CPL;
-    } else if (k < 8 * CPL + nd) {
+      dst_off[p2] = v * VW + col;
+    } else if (k < 32 * C + nd) {
       constexpr int per = 16 / (int)sizeof(Tin);  // dO rows per piece
-      const int part = k - 8 * CPL;
+      const int part = k - 32 * C;
       piece[p2] = true;
       is_do[p2] = true;
       valid[p2] = j0 + per * part < dv;
       src_off[p2] = valid[p2] ? j0 + per * part : 0;  // elements into the token's dO row
-      dst_off[p2] = 4 * VS + 4 * part;
+      dst_off[p2] = 4 * VW + 4 * part;
     }
   }
   const size_t do_stride = (size_t)P.H * dv;  // dO elements from one token to the next
@@ -559,15 +586,10 @@ __global__ void __launch_bounds__(128) r1_kernel(const BParams Q) {
       }
     }
   };
-  float D[CPL];
+  float D[RW][C];
 #pragma unroll
-  for (int e = 0; e < CPL; e += 4) {
-    const int col = s * CPL + e;
-    float v[4];
-    ld4(rok && Q.dST && col < dk ? Q.dST + ((size_t)bh * dv + j) * dk + col : nullptr,
-        rok && Q.dST && col < dk, v);
-    D[e] = v[0]; D[e + 1] = v[1]; D[e + 2] = v[2]; D[e + 3] = v[3];
-  }
+  for (int r = 0; r < RW; ++r)
+    ld_c<C>(Q.dST && cok && jw + r < dv ? Q.dST + ((size_t)bh * dv + jw + r) * dk + c0 : nullptr, D[r]);
   if (nc > 0) issue(nc - 1);
   cp_async_commit();
   for (int ch = nc - 1; ch >= 0; --ch) {
@@ -577,59 +599,80 @@ __global__ void __launch_bounds__(128) r1_kernel(const BParams Q) {
     __syncthreads();
     const float *buf = sm + (ch & 1) * kLCR * TS;
     const int t0 = ch * kLCR, n = min(kLCR, T - t0);
-    const size_t ckd = (((size_t)bh * Q.nck + (t0 + n - 1) / kCk) * dv + j) * dk;
-    if (((t0 + n) % kCk == 0 || t0 + n == T) && rok &&
-        in_bounds(P.err, ckd + dk <= Q.n_ck)) {  // entering chunk (t0 + n - 1) / kCk
-      float *ck = Q.ckD + ckd;
+    if (((t0 + n) % kCk == 0 || t0 + n == T) && cok) {  // entering chunk (t0 + n - 1) / kCk
+      const size_t ckd = (((size_t)bh * Q.nck + (t0 + n - 1) / kCk) * dv + jw) * dk + c0;
 #pragma unroll
-      for (int e = 0; e < CPL; e += 4)
-        if (s * CPL + e < dk)
-          *reinterpret_cast<float4 *>(ck + s * CPL + e) = make_float4(D[e], D[e + 1], D[e + 2], D[e + 3]);
+      for (int r = 0; r < RW; ++r)
+        if (jw + r < dv && in_bounds(P.err, ckd + (size_t)r * dk + C <= Q.n_ck))
+          st_c<C>(Q.ckD + ckd + (size_t)r * dk, D[r]);
     }
     for (int tt = n - 1; tt >= 0; --tt) {
-      const float *sv = buf + tt * TS + s * SS;
-      const float cg = Q.dO ? cq * ld_row<Tin>(buf + tt * TS + 4 * VS, rl) : 0.f;
-      float p[4] = {0.f, 0.f, 0.f, 0.f};
+      const float *sv = buf + tt * TS + c0;
+      float qq[C], rr[C], ww[C], al[C];
+      ld_c<C>(sv, qq);
+      ld_c<C>(sv + VW, rr);
+      ld_c<C>(sv + 2 * VW, ww);
+      ld_c<C>(sv + 3 * VW, al);
+      float cg[RW];
+      if (Q.dO) {
+        ld_dO_rows<Tin, RW>(buf + tt * TS + 4 * VW, RW * warp, cq, cg);
+      } else {
 #pragma unroll
-      for (int e = 0; e < CPL; e += 4) {
-        const float4 q = *reinterpret_cast<const float4 *>(sv + e);
-        const float4 w = *reinterpret_cast<const float4 *>(sv + 2 * VS + e);
-        D[e] = fmaf(cg, q.x, D[e]);
-        D[e + 1] = fmaf(cg, q.y, D[e + 1]);
-        D[e + 2] = fmaf(cg, q.z, D[e + 2]);
-        D[e + 3] = fmaf(cg, q.w, D[e + 3]);
-        p[0] = fmaf(D[e], w.x, p[0]);
-        p[1] = fmaf(D[e + 1], w.y, p[1]);
-        p[2] = fmaf(D[e + 2], w.z, p[2]);
-        p[3] = fmaf(D[e + 3], w.w, p[3]);
+        for (int r = 0; r < RW; ++r) cg[r] = 0.f;
       }
-      float dd = (p[0] + p[1]) + (p[2] + p[3]);
-      dd += __shfl_xor_sync(0xffffffffu, dd, 1);
-      dd += __shfl_xor_sync(0xffffffffu, dd, 2);
-      dd += __shfl_xor_sync(0xffffffffu, dd, 4);
+      float pr[RW];
 #pragma unroll
-      for (int e = 0; e < CPL; e += 4) {
-        const float4 r = *reinterpret_cast<const float4 *>(sv + VS + e);
-        const float4 a = *reinterpret_cast<const float4 *>(sv + 3 * VS + e);
-        D[e] = fmaf(-dd, r.x, D[e]) * a.x;
-        D[e + 1] = fmaf(-dd, r.y, D[e + 1]) * a.y;
-        D[e + 2] = fmaf(-dd, r.z, D[e + 2]) * a.z;
-        D[e + 3] = fmaf(-dd, r.w, D[e + 3]) * a.w;
+      for (int r = 0; r < RW; ++r) {
+        float acc = 0.f;
+#pragma unroll
+        for (int e = 0; e < C; ++e) {
+          D[r][e] = fmaf(cg[r], qq[e], D[r][e]);
+          acc = fmaf(D[r][e], ww[e], acc);
+        }
+        pr[r] = acc;
       }
-      const size_t di = ((size_t)bh * T + t0 + tt) * dv + j;
-      if (s == 0 && rok && in_bounds(P.err, di < Q.n_rows)) Q.dd[di] = dd;
+      const float dd = rows_sum<RW>(pr, lane);  // dd of row jw + jl
+      const size_t di = ((size_t)bh * T + t0 + tt) * dv + jw + jl;
+      if (lane % (32 / RW) == 0 && jw + jl < dv && in_bounds(P.err, di < Q.n_rows)) Q.dd[di] = dd;
+#pragma unroll
+      for (int r = 0; r < RW; ++r) {
+        const float dr = __shfl_sync(0xffffffffu, dd, r * (32 / RW));
+#pragma unroll
+        for (int e = 0; e < C; ++e) D[r][e] = fmaf(-dr, rr[e], D[r][e]) * al[e];
+      }
     }
     __syncthreads();
   }
-  if (rok && Q.dS0) {
+  if (cok && Q.dS0) {
 #pragma unroll
-    for (int e = 0; e < CPL; e += 4) {
-      const int col = s * CPL + e;
-      if (col < dk)
-        *reinterpret_cast<float4 *>(Q.dS0 + ((size_t)bh * dv + j) * dk + col) =
-            make_float4(D[e], D[e + 1], D[e + 2], D[e + 3]);
-    }
+    for (int r = 0; r < RW; ++r)
+      if (jw + r < dv) st_c<C>(Q.dS0 + ((size_t)bh * dv + jw + r) * dk + c0, D[r]);
   }
+}
+
+// The two row sweeps in one launch: CTAs [0, n_r1) run R1, the rest F1.
+template <typename Tin, int C, int RW>
+__global__ void __launch_bounds__(128) fr1_kernel(const BParams Q, int n_r1) {
+  extern __shared__ float4 smem4[];
+  float *sm = reinterpret_cast<float *>(smem4);
+  if ((int)blockIdx.x < n_r1)
+    r1_body<Tin, C, RW>(Q, blockIdx.x, sm);
+  else
+    f1_body<C, RW>(Q, blockIdx.x - n_r1, sm);
+}
+
+// The dO entries of rows j0 .. j0 + nrow - 1 of token t (raw dtype), one
+// 16-byte piece; rows >= d_v are zero-filled.
+template <typename Tin>
+__device__ __forceinline__ void stage_dO(const BParams &Q, int bh, int t, int j0, int part,
+                                         float *dst) {
+  const KParams &P = Q.P;
+  constexpr int per = 16 / (int)sizeof(Tin);  // rows per piece
+  const bool ok = j0 + per * part < P.dv;
+  const char *src = reinterpret_cast<const char *>(Q.dO) +
+                    (tok_index(P, bh / P.H, t, bh % P.H) * P.dv + (ok ? j0 + per * part : 0)) *
+                        sizeof(Tin);
+  cp_async16(smem_u32(reinterpret_cast<char *>(dst) + 16 * part), src, ok);
 }
 
 // Four consecutive staged dO rows from j, widened to fp32.
@@ -1128,10 +1171,33 @@ cudaError_t set_smem(K kernel, size_t bytes) {
   return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
 }
 
-template <typename Tin, int R, int CPL>
+// The merged row sweeps for C key channels per lane and RW rows per warp.
+template <typename Tin, int C, int RW>
+cudaError_t launch_fr1_t(const BParams &Q, cudaStream_t st) {
+  const KParams &P = Q.P;
+  const size_t smem = 2 * kLCR * (4 * 32 * C + 4 * RW) * sizeof(float);  // R1's (> F1's)
+  const cudaError_t err = set_smem(fr1_kernel<Tin, C, RW>, smem);
+  if (err != cudaSuccess) return err;
+  const unsigned n = (unsigned)((long long)P.B * P.H * ((P.dv + 4 * RW - 1) / (4 * RW)));
+  fr1_kernel<Tin, C, RW><<<2 * n, 128, smem, st>>>(Q, (int)n);
+  return cudaSuccess;
+}
+
+// Key channels per lane: 32 lanes cover d_k. Rows per warp: 8 (measured
+// against 4 on B200: as fast or faster on every workload, including 32
+// (batch, head) pairs of 32k tokens, where 4 gives twice the CTAs).
+template <typename Tin>
+cudaError_t launch_fr1(const BParams &Q, cudaStream_t st) {
+  const int C = Q.P.dk <= 32 ? 1 : Q.P.dk <= 64 ? 2 : 4;
+  if (C == 4) return launch_fr1_t<Tin, 4, 8>(Q, st);
+  if (C == 2) return launch_fr1_t<Tin, 2, 8>(Q, st);
+  return launch_fr1_t<Tin, 1, 8>(Q, st);
+}
+
+template <typename Tin, int R>
 cudaError_t launch_bwd_t(const BParams &Q, cudaStream_t st) {
   const KParams &P = Q.P;
-  const int dk = P.dk, dv = P.dv;
+  const int dk = P.dk;
   const long long BH = (long long)P.B * P.H, BHT = BH * P.T;
   cudaError_t err;
   if (is_precond(P.variant)) {
@@ -1141,19 +1207,12 @@ cudaError_t launch_bwd_t(const BParams &Q, cudaStream_t st) {
   }
   prep_gen_kernel<Tin><<<grid_for(BHT * 32, 256), 256, 0, st>>>(Q);
 
-  constexpr int VS = kLPR * seg_stride(CPL);
-  const size_t sm_f1 = 2 * kLCR * (3 * VS + kRowsF) * sizeof(float);
-  const size_t sm_r1 = 2 * kLCR * (4 * VS + kRowsF) * sizeof(float);
   const size_t sm_f2 = 2 * kLCC * (2 * dk + 3 * R) * sizeof(float);
   const size_t sm_r2 = 2 * kLCC * (4 * dk + 3 * R) * sizeof(float);
-  if ((err = set_smem(f1_kernel<CPL>, sm_f1)) != cudaSuccess) return err;
-  if ((err = set_smem(r1_kernel<Tin, CPL>, sm_r1)) != cudaSuccess) return err;
   if ((err = set_smem(f2_kernel<Tin, R>, sm_f2)) != cudaSuccess) return err;
   if ((err = set_smem(r2_kernel<Tin, R>, sm_r2)) != cudaSuccess) return err;
-  const unsigned grid_rows = (unsigned)(BH * ((dv + kRowsF - 1) / kRowsF));
   const unsigned grid_cols = (unsigned)(BH * Q.nck * Q.G);
-  f1_kernel<CPL><<<grid_rows, 128, sm_f1, st>>>(Q);
-  r1_kernel<Tin, CPL><<<grid_rows, 128, sm_r1, st>>>(Q);
+  if ((err = launch_fr1<Tin>(Q, st)) != cudaSuccess) return err;
   f2_kernel<Tin, R><<<grid_cols, dk, sm_f2, st>>>(Q);
   r2_kernel<Tin, R><<<grid_cols, dk, sm_r2, st>>>(Q);
   e1_kernel<Tin><<<grid_for(BHT * 32, 256), 256, 0, st>>>(Q);
@@ -1176,20 +1235,10 @@ cudaError_t launch_bwd_t(const BParams &Q, cudaStream_t st) {
 }
 
 template <typename Tin>
-cudaError_t launch_bwd_d(const BParams &Q, int R, int cpl, cudaStream_t st) {
-  if (R == 64) {
-    if (cpl == 16) return launch_bwd_t<Tin, 64, 16>(Q, st);
-    if (cpl == 8) return launch_bwd_t<Tin, 64, 8>(Q, st);
-    return launch_bwd_t<Tin, 64, 4>(Q, st);
-  }
-  if (R == 32) {
-    if (cpl == 16) return launch_bwd_t<Tin, 32, 16>(Q, st);
-    if (cpl == 8) return launch_bwd_t<Tin, 32, 8>(Q, st);
-    return launch_bwd_t<Tin, 32, 4>(Q, st);
-  }
-  if (cpl == 16) return launch_bwd_t<Tin, 16, 16>(Q, st);
-  if (cpl == 8) return launch_bwd_t<Tin, 16, 8>(Q, st);
-  return launch_bwd_t<Tin, 16, 4>(Q, st);
+cudaError_t launch_bwd_d(const BParams &Q, int R, cudaStream_t st) {
+  if (R == 64) return launch_bwd_t<Tin, 64>(Q, st);
+  if (R == 32) return launch_bwd_t<Tin, 32>(Q, st);
+  return launch_bwd_t<Tin, 16>(Q, st);
 }
 
 }  // namespace
@@ -1228,10 +1277,8 @@ cudaError_t launch_chunk_bwd(const KParams &P, const pdn_grads_t *g, void *works
   Q.n_rows = (size_t)BH * P.T * P.dv;
   Q.n_part = (size_t)L.G * BH * P.T * 3 * P.dk;
   Q.n_ck = (size_t)BH * L.nck * P.dv * P.dk;
-  // key channels per lane in the row sweeps: 8 lanes cover d_k
-  const int cpl = P.dk <= 32 ? 4 : P.dk <= 64 ? 8 : 16;
-  if (P.dtype == PDN_BF16) return launch_bwd_d<__nv_bfloat16>(Q, L.R, cpl, stream);
-  return launch_bwd_d<float>(Q, L.R, cpl, stream);
+  if (P.dtype == PDN_BF16) return launch_bwd_d<__nv_bfloat16>(Q, L.R, stream);
+  return launch_bwd_d<float>(Q, L.R, stream);
 }
 
 }  // namespace pdn

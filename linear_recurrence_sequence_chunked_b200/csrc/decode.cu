@@ -459,20 +459,6 @@ __global__ void __launch_bounds__(kTmaThreads, 1) decode_tma_kernel(const KParam
   }
 }
 
-int g_num_sms[64];
-
-int num_sms() {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
-  if (!g_num_sms[dev]) {
-    int n = 0;
-    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
-      n = 148;
-    g_num_sms[dev] = n;
-  }
-  return g_num_sms[dev];
-}
-
 __global__ void selftest_wait_kernel(long long limit_ns, int *err) {
   __shared__ __align__(8) uint64_t bar;
   if (threadIdx.x == 0) {
@@ -485,6 +471,20 @@ __global__ void selftest_wait_kernel(long long limit_ns, int *err) {
 }
 
 }  // namespace
+
+static int g_num_sms[64];
+
+int num_sms() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (!g_num_sms[dev]) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+      n = 148;
+    g_num_sms[dev] = n;
+  }
+  return g_num_sms[dev];
+}
 
 cudaError_t launch_decode(const KParams &P, cudaStream_t stream) {
   const long long grid = (long long)P.B * P.H;

@@ -31,6 +31,9 @@ cudaError_t launch_accumulate(int n, long long len, const float *parts, const fl
 // One decode step (state streamed through once).
 cudaError_t launch_decode(const KParams &P, cudaStream_t stream);
 
+// Multiprocessors of the current device (cached per device).
+int num_sms();
+
 // Every check pdn_chunk_fwd makes before it enqueues work (host-only);
 // on PDN_OK, *impl_out (if non-NULL) is the path it would run.
 pdn_status_t check_chunk_fwd(const pdn_problem_t *p, const pdn_tensors_t *t,
