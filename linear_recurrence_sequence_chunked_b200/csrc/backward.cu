@@ -329,10 +329,15 @@ __global__ void prep_gen_kernel(const BParams Q) {
 // load is served a quarter-warp at a time and every row-token costs the whole
 // vector in shared-memory wavefronts: at the headline sizes that pipe, not the
 // arithmetic, bounds the sweeps.) The RW row reductions over key channels
-// share one transposed butterfly (rows_sum), and the finished row values
-// return to every lane by one shuffle each. The per-token vectors are staged
+// share one transposed butterfly (rows_sum) and the finished row values
+// return to every lane by its reverse (rows_spread); a lane-dependent order
+// of the rows in registers spares both every select. The arithmetic stays
+// scalar fp32: packed pair instructions would need a register pair for every
+// broadcast operand, and the moves that builds cost as much as the pairs
+// save (measured). The per-token vectors are staged
 // through shared memory kLCR tokens at a time with cp.async (double
-// buffered), each padded to 32 C floats with zeros.
+// buffered), each padded to 32 C floats with zeros, and every full chunk of
+// kLCR tokens runs unrolled (constant shared-memory offsets).
 //
 // F1 and R1 share no data (F1 reads S0 and the generic vectors, R1 dS_T, dO
 // and the generic vectors), so they run as one launch, R1's CTAs first (the
@@ -368,36 +373,70 @@ __device__ __forceinline__ void st_c(float *p, const float (&v)[C]) {
     *p = v[0];
 }
 
-// Row sums of a warp's RW rows: p[r] is this lane's partial sum of row r. The
-// first log2(RW) exchanges (across lane bits 4, 3, ...) each hand half of the
-// partial sums a lane still carries to the partner lane and add the other
-// half to the partner's, so that afterwards lane l carries one value, row
-// l / (32 / RW) summed over RW lanes; the remaining xor levels finish it.
-// Returns the full sum of row l / (32 / RW) on every lane l.
+// Packed fp32 pairs (one instruction for two lanes' worth of FMA or MUL; each
+// element rounds exactly as fmaf / a single multiply).
+__device__ __forceinline__ float2 dup2(float a) { return make_float2(a, a); }
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
+
+// Row sums of a warp's RW rows. Lane l keeps its rows in a lane-dependent
+// order: register slot s holds row s ^ jl, jl = l / (32 / RW). p[s] is this
+// lane's partial sum of the row in slot s. Each of the first log2(RW)
+// exchanges (across lane bits 4, 3, ...) adds the upper half of the slots a
+// lane still carries to the lower half of its partner's -- with the xor
+// order the two hold the same rows there, so no lane selects -- and the
+// remaining xor levels finish the sum. Returns the full sum of row jl.
 template <int RW>
-__device__ __forceinline__ float rows_sum(const float (&p)[RW], int lane) {
+__device__ __forceinline__ float rows_sum(const float (&p)[RW]) {
   float c[RW];
 #pragma unroll
-  for (int r = 0; r < RW; ++r) c[r] = p[r];
+  for (int s = 0; s < RW; ++s) c[s] = p[s];
 #pragma unroll
-  for (int n = RW, m = 16; n > 1; n >>= 1, m >>= 1) {
-    const bool hi = lane & m;  // this lane keeps the upper half of the rows it carries
+  for (int n = RW, m = 16; n > 1; n >>= 1, m >>= 1)
 #pragma unroll
-    for (int k = 0; k < n / 2; ++k) {
-      const float send = hi ? c[k] : c[k + n / 2];
-      const float keep = hi ? c[k + n / 2] : c[k];
-      c[k] = keep + __shfl_xor_sync(0xffffffffu, send, m);
-    }
-  }
+    for (int k = 0; k < n / 2; ++k) c[k] += __shfl_xor_sync(0xffffffffu, c[k + n / 2], m);
   float v = c[0];
 #pragma unroll
   for (int m = 16 / RW; m >= 1; m >>= 1) v += __shfl_xor_sync(0xffffffffu, v, m);
   return v;
 }
 
+// The reverse: v is a value of row jl (the same on the lanes of a row);
+// o[s] receives the value of row s ^ jl, slot order as above.
+template <int RW>
+__device__ __forceinline__ void rows_spread(float v, float (&o)[RW]) {
+  o[0] = v;
+#pragma unroll
+  for (int n = 1, m = 32 / RW; n < RW; n <<= 1, m <<= 1)
+#pragma unroll
+    for (int k = 0; k < n; ++k) o[k + n] = __shfl_xor_sync(0xffffffffu, o[k], m);
+}
+
+// State rows held in slot order: X[s][e] is row jw + (s ^ jl) at key channel
+// c0 + e (base: row 0, channel c0 of the (batch, head) block).
+template <int C, int RW>
+__device__ __forceinline__ void ld_state(const float *base, int dv, int dk, int jw, int jl,
+                                         bool cok, float (&X)[RW][C]) {
+#pragma unroll
+  for (int s = 0; s < RW; ++s) {
+    const int j = jw + (s ^ jl);
+    ld_c<C>(base && cok && j < dv ? base + (size_t)j * dk : nullptr, X[s]);
+  }
+}
+template <int C, int RW>
+__device__ __forceinline__ void st_state(float *base, int dv, int dk, int jw, int jl,
+                                         const float (&X)[RW][C], int *err, size_t limit,
+                                         size_t base_off) {
+#pragma unroll
+  for (int s = 0; s < RW; ++s) {
+    const int j = jw + (s ^ jl);
+    if (j < dv && in_bounds(err, base_off + (size_t)j * dk + C <= limit)) st_c<C>(base + (size_t)j * dk, X[s]);
+  }
+}
+
 // F1: the forward recurrence, writing delta_t of every row, the state
 // checkpoints and S_T; `blk` numbers the CTA among F1's.
-template <int C, int RW>
+template <int C, int RW, bool UNR>
 __device__ __forceinline__ void f1_body(const BParams &Q, int blk, float *sm) {
   constexpr int VW = 32 * C;            // staged floats per vector
   constexpr int NR = 4 * RW;            // rows per CTA
@@ -408,7 +447,7 @@ __device__ __forceinline__ void f1_body(const BParams &Q, int blk, float *sm) {
   const int bh = blk / nrg, j0 = (blk % nrg) * NR;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int jw = j0 + RW * warp;        // the warp's first row
-  const int jl = lane / (32 / RW);      // the row (of the warp's) rows_sum leaves on this lane
+  const int jl = lane / (32 / RW);      // slot s of this lane holds row jw + (s ^ jl)
   const int c0 = C * lane;              // this lane's first key channel
   const bool cok = c0 < dk;
   const int nc = (T + kLCR - 1) / kLCR;
@@ -443,9 +482,7 @@ __device__ __forceinline__ void f1_body(const BParams &Q, int blk, float *sm) {
       cp_async16(d + tt * TS * 4, g + (size_t)tt * Q.GS, valid);
   };
   float S[RW][C];
-#pragma unroll
-  for (int r = 0; r < RW; ++r)
-    ld_c<C>(P.S0 && cok && jw + r < dv ? P.S0 + ((size_t)bh * dv + jw + r) * dk + c0 : nullptr, S[r]);
+  ld_state<C, RW>(P.S0 ? P.S0 + (size_t)bh * dv * dk + c0 : nullptr, dv, dk, jw, jl, cok, S);
   issue(0);
   cp_async_commit();
   for (int ch = 0; ch < nc; ++ch) {
@@ -456,13 +493,12 @@ __device__ __forceinline__ void f1_body(const BParams &Q, int blk, float *sm) {
     const float *buf = sm + (ch & 1) * kLCR * TS;
     const int t0 = ch * kLCR, n = min(kLCR, T - t0);
     if (t0 % kCk == 0 && cok) {  // the state before chunk t0 / kCk
-      const size_t cks = (((size_t)bh * Q.nck + t0 / kCk) * dv + jw) * dk + c0;
-#pragma unroll
-      for (int r = 0; r < RW; ++r)
-        if (jw + r < dv && in_bounds(P.err, cks + (size_t)r * dk + C <= Q.n_ck))
-          st_c<C>(Q.ckS + cks + (size_t)r * dk, S[r]);
+      const size_t off = ((size_t)bh * Q.nck + t0 / kCk) * dv * dk + c0;
+      st_state<C, RW>(Q.ckS + off, dv, dk, jw, jl, S, P.err, Q.n_ck, off);
     }
-    for (int tt = 0; tt < n; ++tt) {
+    // one token (with UNR, unrolled over a full chunk: constant shared-memory
+    // offsets)
+    auto step = [&](int tt) {
       const float *sv = buf + tt * TS + c0;
       float rr[C], ww[C], al[C];
       ld_c<C>(sv, rr);
@@ -480,49 +516,39 @@ __device__ __forceinline__ void f1_body(const BParams &Q, int blk, float *sm) {
         y[r] = acc;
       }
       // delta of row jw + jl, then every row's delta to every lane
-      const float d = buf[tt * TS + 3 * VW + RW * warp + jl] - rows_sum<RW>(y, lane);
+      const float d = buf[tt * TS + 3 * VW + RW * warp + jl] - rows_sum<RW>(y);
       const size_t di = ((size_t)bh * T + t0 + tt) * dv + jw + jl;
       if (lane % (32 / RW) == 0 && jw + jl < dv && in_bounds(P.err, di < Q.n_rows)) Q.delta[di] = d;
+      float ds[RW];
+      rows_spread<RW>(d, ds);
 #pragma unroll
-      for (int r = 0; r < RW; ++r) {
-        const float dr = __shfl_sync(0xffffffffu, d, r * (32 / RW));
+      for (int r = 0; r < RW; ++r)
 #pragma unroll
-        for (int e = 0; e < C; ++e) S[r][e] = fmaf(dr, ww[e], S[r][e]);
-      }
+        for (int e = 0; e < C; ++e) S[r][e] = fmaf(ds[r], ww[e], S[r][e]);
+    };
+    if (UNR && n == kLCR) {
+#pragma unroll
+      for (int tt = 0; tt < kLCR; ++tt) step(tt);
+    } else {
+      for (int tt = 0; tt < n; ++tt) step(tt);
     }
     __syncthreads();  // the buffer is refilled two chunks on
   }
-  if (cok) {
-#pragma unroll
-    for (int r = 0; r < RW; ++r)
-      if (jw + r < dv) st_c<C>(Q.st + ((size_t)bh * dv + jw + r) * dk + c0, S[r]);
-  }
+  if (cok) st_state<C, RW>(Q.st + (size_t)bh * dv * dk + c0, dv, dk, jw, jl, S, P.err, ~(size_t)0, 0);
 }
 
-// The dO entries of rows j .. j + RW - 1 as staged (raw dtype), widened to
-// fp32 and scaled by c.
-template <typename Tin, int RW>
-__device__ __forceinline__ void ld_dO_rows(const float *slot, int j, float c, float (&g)[RW]) {
-  if constexpr (sizeof(Tin) == 4) {
-#pragma unroll
-    for (int r = 0; r < RW; r += 4) {
-      const float4 x = *reinterpret_cast<const float4 *>(slot + j + r);
-      g[r] = c * x.x; g[r + 1] = c * x.y; g[r + 2] = c * x.z; g[r + 3] = c * x.w;
-    }
-  } else {
-    const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(
-        reinterpret_cast<const __nv_bfloat16 *>(slot) + j);
-#pragma unroll
-    for (int r = 0; r < RW; r += 2) {
-      const float2 x = __bfloat1622float2(h[r / 2]);
-      g[r] = c * x.x; g[r + 1] = c * x.y;
-    }
-  }
+// The staged dO entry (raw dtype) of row j of the CTA's rows, widened.
+template <typename Tin>
+__device__ __forceinline__ float ld_dO_row(const float *slot, int j) {
+  if constexpr (sizeof(Tin) == 4)
+    return slot[j];
+  else
+    return __bfloat162float(reinterpret_cast<const __nv_bfloat16 *>(slot)[j]);
 }
 
 // R1: the reverse recurrence of the cotangent, writing dd_t of every row, the
 // cotangent checkpoints and dS0; `blk` numbers the CTA among R1's.
-template <typename Tin, int C, int RW>
+template <typename Tin, int C, int RW, bool UNR>
 __device__ __forceinline__ void r1_body(const BParams &Q, int blk, float *sm) {
   constexpr int VW = 32 * C;
   constexpr int NR = 4 * RW;
@@ -587,9 +613,7 @@ __device__ __forceinline__ void r1_body(const BParams &Q, int blk, float *sm) {
     }
   };
   float D[RW][C];
-#pragma unroll
-  for (int r = 0; r < RW; ++r)
-    ld_c<C>(Q.dST && cok && jw + r < dv ? Q.dST + ((size_t)bh * dv + jw + r) * dk + c0 : nullptr, D[r]);
+  ld_state<C, RW>(Q.dST ? Q.dST + (size_t)bh * dv * dk + c0 : nullptr, dv, dk, jw, jl, cok, D);
   if (nc > 0) issue(nc - 1);
   cp_async_commit();
   for (int ch = nc - 1; ch >= 0; --ch) {
@@ -600,65 +624,60 @@ __device__ __forceinline__ void r1_body(const BParams &Q, int blk, float *sm) {
     const float *buf = sm + (ch & 1) * kLCR * TS;
     const int t0 = ch * kLCR, n = min(kLCR, T - t0);
     if (((t0 + n) % kCk == 0 || t0 + n == T) && cok) {  // entering chunk (t0 + n - 1) / kCk
-      const size_t ckd = (((size_t)bh * Q.nck + (t0 + n - 1) / kCk) * dv + jw) * dk + c0;
-#pragma unroll
-      for (int r = 0; r < RW; ++r)
-        if (jw + r < dv && in_bounds(P.err, ckd + (size_t)r * dk + C <= Q.n_ck))
-          st_c<C>(Q.ckD + ckd + (size_t)r * dk, D[r]);
+      const size_t off = ((size_t)bh * Q.nck + (t0 + n - 1) / kCk) * dv * dk + c0;
+      st_state<C, RW>(Q.ckD + off, dv, dk, jw, jl, D, P.err, Q.n_ck, off);
     }
-    for (int tt = n - 1; tt >= 0; --tt) {
+    auto step = [&](int tt) {
       const float *sv = buf + tt * TS + c0;
       float qq[C], rr[C], ww[C], al[C];
       ld_c<C>(sv, qq);
       ld_c<C>(sv + VW, rr);
       ld_c<C>(sv + 2 * VW, ww);
       ld_c<C>(sv + 3 * VW, al);
-      float cg[RW];
-      if (Q.dO) {
-        ld_dO_rows<Tin, RW>(buf + tt * TS + 4 * VW, RW * warp, cq, cg);
-      } else {
-#pragma unroll
-        for (int r = 0; r < RW; ++r) cg[r] = 0.f;
-      }
+      const float *slot = buf + tt * TS + 4 * VW;
       float pr[RW];
 #pragma unroll
       for (int r = 0; r < RW; ++r) {
+        // c dO of the row in slot r
+        const float cg = Q.dO ? cq * ld_dO_row<Tin>(slot, RW * warp + (r ^ jl)) : 0.f;
         float acc = 0.f;
 #pragma unroll
         for (int e = 0; e < C; ++e) {
-          D[r][e] = fmaf(cg[r], qq[e], D[r][e]);
+          D[r][e] = fmaf(cg, qq[e], D[r][e]);
           acc = fmaf(D[r][e], ww[e], acc);
         }
         pr[r] = acc;
       }
-      const float dd = rows_sum<RW>(pr, lane);  // dd of row jw + jl
+      const float dd = rows_sum<RW>(pr);  // dd of row jw + jl
       const size_t di = ((size_t)bh * T + t0 + tt) * dv + jw + jl;
       if (lane % (32 / RW) == 0 && jw + jl < dv && in_bounds(P.err, di < Q.n_rows)) Q.dd[di] = dd;
+      float dds[RW];
+      rows_spread<RW>(dd, dds);
 #pragma unroll
-      for (int r = 0; r < RW; ++r) {
-        const float dr = __shfl_sync(0xffffffffu, dd, r * (32 / RW));
+      for (int r = 0; r < RW; ++r)
 #pragma unroll
-        for (int e = 0; e < C; ++e) D[r][e] = fmaf(-dr, rr[e], D[r][e]) * al[e];
-      }
+        for (int e = 0; e < C; ++e) D[r][e] = fmaf(-dds[r], rr[e], D[r][e]) * al[e];
+    };
+    if (UNR && n == kLCR) {
+#pragma unroll
+      for (int tt = kLCR - 1; tt >= 0; --tt) step(tt);
+    } else {
+      for (int tt = n - 1; tt >= 0; --tt) step(tt);
     }
     __syncthreads();
   }
-  if (cok && Q.dS0) {
-#pragma unroll
-    for (int r = 0; r < RW; ++r)
-      if (jw + r < dv) st_c<C>(Q.dS0 + ((size_t)bh * dv + jw + r) * dk + c0, D[r]);
-  }
+  if (cok && Q.dS0) st_state<C, RW>(Q.dS0 + (size_t)bh * dv * dk + c0, dv, dk, jw, jl, D, P.err, ~(size_t)0, 0);
 }
 
 // The two row sweeps in one launch: CTAs [0, n_r1) run R1, the rest F1.
-template <typename Tin, int C, int RW>
+template <typename Tin, int C, int RW, bool UNR>
 __global__ void __launch_bounds__(128) fr1_kernel(const BParams Q, int n_r1) {
   extern __shared__ float4 smem4[];
   float *sm = reinterpret_cast<float *>(smem4);
   if ((int)blockIdx.x < n_r1)
-    r1_body<Tin, C, RW>(Q, blockIdx.x, sm);
+    r1_body<Tin, C, RW, UNR>(Q, blockIdx.x, sm);
   else
-    f1_body<C, RW>(Q, blockIdx.x - n_r1, sm);
+    f1_body<C, RW, UNR>(Q, blockIdx.x - n_r1, sm);
 }
 
 // The dO entries of rows j0 .. j0 + nrow - 1 of token t (raw dtype), one
@@ -807,11 +826,13 @@ __global__ void __launch_bounds__(128) f2_kernel(const BParams Q) {
         stage_dO<Tin>(Q, bh, t, j0, k - nv - 2 * nr, d + 2 * dk + 2 * R);
     }
   };
-  float S[R];
+  float2 S[R / 2];  // rows (2h, 2h + 1) of this column
 #pragma unroll
   for (int j = 0; j < R; ++j) {
     const size_t e = (((size_t)bh * Q.nck + ck) * dv + j0 + j) * dk + i;
-    S[j] = in_bounds(P.err, e < Q.n_ck) ? Q.ckS[e] : 0.f;
+    const float x = in_bounds(P.err, e < Q.n_ck) ? Q.ckS[e] : 0.f;
+    if (j & 1) S[j / 2].y = x;
+    else S[j / 2].x = x;
   }
   issue(0);
   cp_async_commit();
@@ -824,8 +845,8 @@ __global__ void __launch_bounds__(128) f2_kernel(const BParams Q) {
     const int t0 = tb + ch * kLCC, n = min(kLCC, te - t0);
     for (int tt = 0; tt < n; ++tt) {
       const float *sv = buf + tt * TS;
-      const float w = sv[i], a = sv[dk + i];
-      float accq = 0.f, accr = 0.f;
+      const float2 w = dup2(sv[i]), a = dup2(sv[dk + i]);
+      float2 accq = make_float2(0.f, 0.f), accr = make_float2(0.f, 0.f);  // even | odd rows
 #pragma unroll
       for (int j = 0; j < R; j += 4) {
         float de[4], dd[4], go[4];
@@ -837,17 +858,18 @@ __global__ void __launch_bounds__(128) f2_kernel(const BParams Q) {
           go[0] = go[1] = go[2] = go[3] = 0.f;
         }
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float p = S[j + e] * a;
-          accr = fmaf(p, dd[e], accr);
-          S[j + e] = fmaf(de[e], w, p);
-          accq = fmaf(S[j + e], go[e], accq);
+        for (int h = 0; h < 2; ++h) {
+          float2 &s2 = S[j / 2 + h];
+          const float2 p = mul2(s2, a);
+          accr = fma2(p, make_float2(dd[2 * h], dd[2 * h + 1]), accr);
+          s2 = fma2(make_float2(de[2 * h], de[2 * h + 1]), w, p);
+          accq = fma2(s2, make_float2(go[2 * h], go[2 * h + 1]), accq);
         }
       }
       const size_t po = (((size_t)g * BH + bh) * T + t0 + tt) * 3 * dk;
       if (in_bounds(P.err, po + 3 * dk <= Q.n_part)) {
-        Q.part[po + i] = cq * accq;
-        Q.part[po + dk + i] = -accr;
+        Q.part[po + i] = cq * (accq.x + accq.y);
+        Q.part[po + dk + i] = -(accr.x + accr.y);
       }
     }
     __syncthreads();
@@ -895,11 +917,13 @@ __global__ void __launch_bounds__(128) r2_kernel(const BParams Q) {
         stage_dO<Tin>(Q, bh, t, j0, k - nv - 2 * nr, d + 4 * dk + 2 * R);
     }
   };
-  float D[R];
+  float2 D[R / 2];  // rows (2h, 2h + 1) of this column
 #pragma unroll
   for (int j = 0; j < R; ++j) {
     const size_t e = (((size_t)bh * Q.nck + ck) * dv + j0 + j) * dk + i;
-    D[j] = in_bounds(P.err, e < Q.n_ck) ? Q.ckD[e] : 0.f;
+    const float x = in_bounds(P.err, e < Q.n_ck) ? Q.ckD[e] : 0.f;
+    if (j & 1) D[j / 2].y = x;
+    else D[j / 2].x = x;
   }
   if (nc > 0) issue(nc - 1);
   cp_async_commit();
@@ -912,9 +936,8 @@ __global__ void __launch_bounds__(128) r2_kernel(const BParams Q) {
     const int t0 = tb + ch * kLCC, n = min(kLCC, te - t0);
     for (int tt = n - 1; tt >= 0; --tt) {
       const float *sv = buf + tt * TS;
-      const float q = sv[i], r = sv[dk + i], a = sv[3 * dk + i];
-      const float cqq = cq * q;
-      float accw = 0.f;
+      const float2 cqq = dup2(cq * sv[i]), nr = dup2(-sv[dk + i]), a = dup2(sv[3 * dk + i]);
+      float2 accw = make_float2(0.f, 0.f);  // even | odd rows
 #pragma unroll
       for (int j = 0; j < R; j += 4) {
         float de[4], dd[4], go[4];
@@ -926,14 +949,15 @@ __global__ void __launch_bounds__(128) r2_kernel(const BParams Q) {
           go[0] = go[1] = go[2] = go[3] = 0.f;
         }
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float dt = fmaf(cqq, go[e], D[j + e]);
-          accw = fmaf(dt, de[e], accw);
-          D[j + e] = fmaf(-dd[e], r, dt) * a;
+        for (int h = 0; h < 2; ++h) {
+          float2 &d2 = D[j / 2 + h];
+          const float2 dt = fma2(cqq, make_float2(go[2 * h], go[2 * h + 1]), d2);
+          accw = fma2(dt, make_float2(de[2 * h], de[2 * h + 1]), accw);
+          d2 = mul2(fma2(make_float2(dd[2 * h], dd[2 * h + 1]), nr, dt), a);
         }
       }
       const size_t po = (((size_t)g * BH + bh) * T + t0 + tt) * 3 * dk;
-      if (in_bounds(P.err, po + 3 * dk <= Q.n_part)) Q.part[po + 2 * dk + i] = accw;
+      if (in_bounds(P.err, po + 3 * dk <= Q.n_part)) Q.part[po + 2 * dk + i] = accw.x + accw.y;
     }
     __syncthreads();
   }
@@ -1172,26 +1196,35 @@ cudaError_t set_smem(K kernel, size_t bytes) {
 }
 
 // The merged row sweeps for C key channels per lane and RW rows per warp.
-template <typename Tin, int C, int RW>
-cudaError_t launch_fr1_t(const BParams &Q, cudaStream_t st) {
-  const KParams &P = Q.P;
+template <typename Tin, int C, int RW, bool UNR>
+cudaError_t launch_fr1_t(const BParams &Q, unsigned n, cudaStream_t st) {
   const size_t smem = 2 * kLCR * (4 * 32 * C + 4 * RW) * sizeof(float);  // R1's (> F1's)
-  const cudaError_t err = set_smem(fr1_kernel<Tin, C, RW>, smem);
+  const cudaError_t err = set_smem(fr1_kernel<Tin, C, RW, UNR>, smem);
   if (err != cudaSuccess) return err;
-  const unsigned n = (unsigned)((long long)P.B * P.H * ((P.dv + 4 * RW - 1) / (4 * RW)));
-  fr1_kernel<Tin, C, RW><<<2 * n, 128, smem, st>>>(Q, (int)n);
+  fr1_kernel<Tin, C, RW, UNR><<<2 * n, 128, smem, st>>>(Q, (int)n);
   return cudaSuccess;
 }
 
 // Key channels per lane: 32 lanes cover d_k. Rows per warp: 8 (measured
 // against 4 on B200: as fast or faster on every workload, including 32
-// (batch, head) pairs of 32k tokens, where 4 gives twice the CTAs).
+// (batch, head) pairs of 32k tokens, where 4 gives twice the CTAs). The
+// unrolled chunk loop issues fewer instructions but schedules worse when
+// there are too few warps to hide latency (under two CTAs per SM, measured:
+// 26.1 against 28.7 ms on 32 pairs of 32k tokens; 6.07 against 6.28 ms on
+// the headline layer's 512 CTAs).
 template <typename Tin>
 cudaError_t launch_fr1(const BParams &Q, cudaStream_t st) {
-  const int C = Q.P.dk <= 32 ? 1 : Q.P.dk <= 64 ? 2 : 4;
-  if (C == 4) return launch_fr1_t<Tin, 4, 8>(Q, st);
-  if (C == 2) return launch_fr1_t<Tin, 2, 8>(Q, st);
-  return launch_fr1_t<Tin, 1, 8>(Q, st);
+  const KParams &P = Q.P;
+  const int C = P.dk <= 32 ? 1 : P.dk <= 64 ? 2 : 4;
+  const unsigned n = (unsigned)((long long)P.B * P.H * ((P.dv + 31) / 32));  // CTAs per sweep
+  if (2LL * n >= 2LL * num_sms()) {
+    if (C == 4) return launch_fr1_t<Tin, 4, 8, true>(Q, n, st);
+    if (C == 2) return launch_fr1_t<Tin, 2, 8, true>(Q, n, st);
+    return launch_fr1_t<Tin, 1, 8, true>(Q, n, st);
+  }
+  if (C == 4) return launch_fr1_t<Tin, 4, 8, false>(Q, n, st);
+  if (C == 2) return launch_fr1_t<Tin, 2, 8, false>(Q, n, st);
+  return launch_fr1_t<Tin, 1, 8, false>(Q, n, st);
 }
 
 template <typename Tin, int R>

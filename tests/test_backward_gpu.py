@@ -162,7 +162,19 @@ def test_backward_strong_decay(variant):
 def test_backward_full_size_sampled(name, chains):
     """Full-size workloads: the whole backward on the GPU, the oracle on
     sampled (batch, head) chains over all T tokens."""
-    w = WORKLOADS[name]
+    check_sampled_chains(WORKLOADS[name], chains)
+
+
+@pytest.mark.parametrize("variant,dk", [("PKDA", 128), ("GDN2", 64), ("FG2_GDN_PLUS", 128)])
+def test_backward_many_chains_ragged(variant, dk):
+    """Enough (batch, head) pairs for the row sweeps' unrolled chunk loop (at
+    least one CTA per SM), with a token count that leaves a ragged last chunk
+    of 3 tokens; sampled chains, the last one included."""
+    w = small(variant, "bf16", B=10 if dk == 64 else 5, T=203, H=16, dk=dk)
+    check_sampled_chains(w, [(0, 0), (w.B // 2, 7), (w.B - 1, w.H - 1)])
+
+
+def check_sampled_chains(w, chains):
     x = make_inputs(w, device="cuda")
     g = torch.Generator().manual_seed(11)
     dt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
