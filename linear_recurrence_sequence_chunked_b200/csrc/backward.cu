@@ -47,7 +47,7 @@ struct BwdPlan {
   int R, G;        // rows per CTA of F2/R2, row groups (d_v / R)
   int nb;          // scan blocks per sequence
   int nck;         // state checkpoints per sequence (one per kCk tokens)
-  size_t gen, acc, delta, dd, st, part, cpsi, sigma, dacc, bsum, phi, ckS, ckD, total;
+  size_t gen, acc, delta, dd, cdo, st, part, cpsi, sigma, dacc, bsum, phi, ckS, ckD, total;
 };
 
 namespace {
@@ -82,6 +82,7 @@ static BwdPlan bwd_plan(const KParams &P) {
   L.acc = take(is_precond(P.variant) ? BH * T * dk : 0);
   L.delta = take(BH * T * dv);
   L.dd = take(BH * T * dv);
+  L.cdo = take(BH * T * dv);
   L.st = take(BH * dv * dk);
   L.part = take((size_t)L.G * BH * T * 3 * dk);
   L.cpsi = take(P.decay == PDN_DECAY_CHANNEL ? BH * T * dk : 0);
@@ -105,6 +106,8 @@ struct BParams {
   const float *dST;   // [B,H,dv,dk] or NULL
   float *dq, *dk, *dv, *dla, *dbeta, *derase, *dwrite, *dS0, *dA0;
   float *gen, *acc, *delta, *dd, *st, *part, *cpsi, *sigma, *dacc, *bsum, *phi;
+  // c dO in fp32, [BH][T][d_v] like delta and dd (written when dO is given)
+  float *cdo;
   // S before the first token of each kCk-token chunk (F1) and the cotangent
   // entering each chunk's last token (R1): [BH][nck][d_v][d_k]
   float *ckS, *ckD;
@@ -316,6 +319,12 @@ __global__ void prep_gen_kernel(const BParams Q) {
       *reinterpret_cast<float4 *>(g + 3 * dk + c) = make_float4(a[0], a[1], a[2], a[3]);
     }
     if (av) *reinterpret_cast<float4 *>(g + 4 * dk + c) = make_float4(u[0], u[1], u[2], u[3]);
+    if (Q.dO && av) {  // c dO of the token, once, for the three sweeps that read it
+      float o[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) o[e] = P.q_scale * ldf<Tin>(Q.dO, tk * dv + c + e);
+      *reinterpret_cast<float4 *>(Q.cdo + ((size_t)bh * P.T + t) * dv + c) = make_float4(o[0], o[1], o[2], o[3]);
+    }
   }
 }
 
@@ -339,7 +348,7 @@ __global__ void prep_gen_kernel(const BParams Q) {
 // buffered), each padded to 32 C floats with zeros, and every full chunk of
 // kLCR tokens runs unrolled (constant shared-memory offsets).
 //
-// F1 and R1 share no data (F1 reads S0 and the generic vectors, R1 dS_T, dO
+// F1 and R1 share no data (F1 reads S0 and the generic vectors, R1 dS_T, c dO
 // and the generic vectors), so they run as one launch, R1's CTAs first (the
 // longer sweep), both resident at once.
 constexpr int kLCR = 8;  // tokens staged per chunk in F1 / R1
@@ -537,23 +546,14 @@ __device__ __forceinline__ void f1_body(const BParams &Q, int blk, float *sm) {
   if (cok) st_state<C, RW>(Q.st + (size_t)bh * dv * dk + c0, dv, dk, jw, jl, S, P.err, ~(size_t)0, 0);
 }
 
-// The staged dO entry (raw dtype) of row j of the CTA's rows, widened.
-template <typename Tin>
-__device__ __forceinline__ float ld_dO_row(const float *slot, int j) {
-  if constexpr (sizeof(Tin) == 4)
-    return slot[j];
-  else
-    return __bfloat162float(reinterpret_cast<const __nv_bfloat16 *>(slot)[j]);
-}
-
 // R1: the reverse recurrence of the cotangent, writing dd_t of every row, the
 // cotangent checkpoints and dS0; `blk` numbers the CTA among R1's.
-template <typename Tin, int C, int RW, bool UNR>
+template <int C, int RW, bool UNR>
 __device__ __forceinline__ void r1_body(const BParams &Q, int blk, float *sm) {
   constexpr int VW = 32 * C;
   constexpr int NR = 4 * RW;
-  constexpr int TS = 4 * VW + NR;  // q' | r | w | alpha | dO of the CTA's rows (raw)
-  constexpr int ND = NR * (int)sizeof(Tin) / 16;  // dO pieces per token
+  constexpr int TS = 4 * VW + NR;  // q' | r | w | alpha | c dO of the CTA's rows
+  constexpr int ND = NR / 4;       // c dO pieces per token
   const KParams &P = Q.P;
   const int dk = P.dk, dv = P.dv, T = P.T;
   const int nrg = (dv + NR - 1) / NR;
@@ -562,13 +562,12 @@ __device__ __forceinline__ void r1_body(const BParams &Q, int blk, float *sm) {
   const int jw = j0 + RW * warp, jl = lane / (32 / RW);
   const int c0 = C * lane;
   const bool cok = c0 < dk;
-  const float cq = P.q_scale;
   const int nd = Q.dO ? ND : 0;
   const int nc = (T + kLCR - 1) / kLCR;
   // This thread's 16-byte pieces of every staged token (up to two: 32 C + ND
   // <= 136 pieces for 128 threads), fixed for the whole sweep: q' | r | w |
-  // alpha (source: the token's generic vectors), then the dO of the CTA's
-  // rows (source: the token's dO row).
+  // alpha (source: the token's generic vectors), then c dO of the CTA's rows
+  // (source: the token's row of cdo).
   int src_off[2] = {0, 0}, dst_off[2] = {0, 0};
   bool piece[2] = {false, false}, valid[2] = {false, false}, is_do[2] = {false, false};
 #pragma unroll
@@ -581,31 +580,27 @@ __device__ __forceinline__ void r1_body(const BParams &Q, int blk, float *sm) {
       src_off[p2] = v * dk + (valid[p2] ? col : 0);
       dst_off[p2] = v * VW + col;
     } else if (k < 32 * C + nd) {
-      constexpr int per = 16 / (int)sizeof(Tin);  // dO rows per piece
       const int part = k - 32 * C;
       piece[p2] = true;
       is_do[p2] = true;
-      valid[p2] = j0 + per * part < dv;
-      src_off[p2] = valid[p2] ? j0 + per * part : 0;  // elements into the token's dO row
+      valid[p2] = j0 + 4 * part < dv;
+      src_off[p2] = valid[p2] ? j0 + 4 * part : 0;  // floats into the token's cdo row
       dst_off[p2] = 4 * VW + 4 * part;
     }
   }
-  const size_t do_stride = (size_t)P.H * dv;  // dO elements from one token to the next
   auto issue = [&](int ch) {
     float *buf = sm + (ch & 1) * kLCR * TS;
     const int t0 = ch * kLCR, n = min(kLCR, T - t0);
-    if (!in_bounds(P.err, t0 + n <= T)) return;
+    if (!in_bounds(P.err, ((size_t)bh * T + t0 + n) * dv <= Q.n_rows)) return;
     const float *g = gen_at(Q, bh, t0);
-    const Tin *o0 = Q.dO ? reinterpret_cast<const Tin *>(Q.dO) +
-                               tok_index(P, bh / P.H, t0, bh % P.H) * dv
-                         : nullptr;
+    const float *o0 = Q.cdo + ((size_t)bh * T + t0) * dv;
 #pragma unroll
     for (int p2 = 0; p2 < 2; ++p2) {
       if (!piece[p2]) continue;
       const uint32_t d = smem_u32(buf + dst_off[p2]);
       if (is_do[p2]) {
-        const Tin *src = o0 + src_off[p2];
-        for (int tt = 0; tt < n; ++tt) cp_async16(d + tt * TS * 4, src + tt * do_stride, valid[p2]);
+        const float *src = o0 + src_off[p2];
+        for (int tt = 0; tt < n; ++tt) cp_async16(d + tt * TS * 4, src + (size_t)tt * dv, valid[p2]);
       } else {
         const float *src = g + src_off[p2];
         for (int tt = 0; tt < n; ++tt) cp_async16(d + tt * TS * 4, src + (size_t)tt * Q.GS, valid[p2]);
@@ -639,7 +634,7 @@ __device__ __forceinline__ void r1_body(const BParams &Q, int blk, float *sm) {
 #pragma unroll
       for (int r = 0; r < RW; ++r) {
         // c dO of the row in slot r
-        const float cg = Q.dO ? cq * ld_dO_row<Tin>(slot, RW * warp + (r ^ jl)) : 0.f;
+        const float cg = Q.dO ? slot[RW * warp + (r ^ jl)] : 0.f;
         float acc = 0.f;
 #pragma unroll
         for (int e = 0; e < C; ++e) {
@@ -670,43 +665,14 @@ __device__ __forceinline__ void r1_body(const BParams &Q, int blk, float *sm) {
 }
 
 // The two row sweeps in one launch: CTAs [0, n_r1) run R1, the rest F1.
-template <typename Tin, int C, int RW, bool UNR>
+template <int C, int RW, bool UNR>
 __global__ void __launch_bounds__(128) fr1_kernel(const BParams Q, int n_r1) {
   extern __shared__ float4 smem4[];
   float *sm = reinterpret_cast<float *>(smem4);
   if ((int)blockIdx.x < n_r1)
-    r1_body<Tin, C, RW, UNR>(Q, blockIdx.x, sm);
+    r1_body<C, RW, UNR>(Q, blockIdx.x, sm);
   else
     f1_body<C, RW, UNR>(Q, blockIdx.x - n_r1, sm);
-}
-
-// The dO entries of rows j0 .. j0 + nrow - 1 of token t (raw dtype), one
-// 16-byte piece; rows >= d_v are zero-filled.
-template <typename Tin>
-__device__ __forceinline__ void stage_dO(const BParams &Q, int bh, int t, int j0, int part,
-                                         float *dst) {
-  const KParams &P = Q.P;
-  constexpr int per = 16 / (int)sizeof(Tin);  // rows per piece
-  const bool ok = j0 + per * part < P.dv;
-  const char *src = reinterpret_cast<const char *>(Q.dO) +
-                    (tok_index(P, bh / P.H, t, bh % P.H) * P.dv + (ok ? j0 + per * part : 0)) *
-                        sizeof(Tin);
-  cp_async16(smem_u32(reinterpret_cast<char *>(dst) + 16 * part), src, ok);
-}
-
-// Four consecutive staged dO rows from j, widened to fp32.
-template <typename Tin>
-__device__ __forceinline__ void ld_rows4(const float *sv, int j, float (&v)[4]);
-template <>
-__device__ __forceinline__ void ld_rows4<float>(const float *sv, int j, float (&v)[4]) {
-  const float4 x = *reinterpret_cast<const float4 *>(sv + j);
-  v[0] = x.x; v[1] = x.y; v[2] = x.z; v[3] = x.w;
-}
-template <>
-__device__ __forceinline__ void ld_rows4<__nv_bfloat16>(const float *sv, int j, float (&v)[4]) {
-  const uint2 x = *reinterpret_cast<const uint2 *>(reinterpret_cast<const __nv_bfloat16 *>(sv) + j);
-  v[0] = __uint_as_float(x.x << 16); v[1] = __uint_as_float(x.x & 0xffff0000u);
-  v[2] = __uint_as_float(x.y << 16); v[3] = __uint_as_float(x.y & 0xffff0000u);
 }
 
 // ---------------------------------------------------------------------------
@@ -725,50 +691,39 @@ __device__ __forceinline__ size_t row_base(const BParams &Q, int bh, int t, int 
   return in_bounds(Q.P.err, e + R <= Q.n_rows) ? e : 0;
 }
 
-// Stages R floats of a per-row workspace vector (delta or dd) of token t.
+// Stages R floats of a per-row workspace vector (delta, dd or c dO) of token t.
 __device__ __forceinline__ void stage_rows(const float *src, int part, float *dst) {
   cp_async16(smem_u32(dst + 4 * part), src + 4 * part, true);
 }
 
 // One 16-byte piece of a staged token in F2 / R2: from the token's generic
-// vectors (kind 0), its delta or dd rows (1, 2) or its dO row (3); src counts
-// elements from that row's start (or, kind 0, from the token's vectors), dst
-// floats from the staged token's start. kind -1: no piece.
+// vectors (kind 0) or its delta, dd or c dO rows (1, 2, 3); src counts floats
+// from that row's start (or, kind 0, from the token's vectors), dst floats
+// from the staged token's start. kind -1: no piece. (R divides d_v: every
+// row piece is in range.)
 struct ColPiece {
   int kind, src, dst;
-  bool valid;
 };
-template <typename Tin>
 __device__ __forceinline__ ColPiece col_piece(int k, int gen_off, int nv, int rows_dst, int R,
-                                              int nd, int j0, int dv) {
+                                              int nd, int j0) {
   const int nr = R / 4;
-  if (k < nv) return ColPiece{0, gen_off + 4 * k, 4 * k, true};
-  if (k < nv + nr) return ColPiece{1, j0 + 4 * (k - nv), rows_dst + 4 * (k - nv), true};
-  if (k < nv + 2 * nr)
-    return ColPiece{2, j0 + 4 * (k - nv - nr), rows_dst + R + 4 * (k - nv - nr), true};
+  if (k < nv) return ColPiece{0, gen_off + 4 * k, 4 * k};
   if (k < nv + 2 * nr + nd) {
-    constexpr int per = 16 / (int)sizeof(Tin);  // dO rows per piece
-    const int part = k - nv - 2 * nr;
-    const bool ok = j0 + per * part < dv;
-    return ColPiece{3, ok ? j0 + per * part : 0, rows_dst + 2 * R + 4 * part, ok};
+    const int q = (k - nv) / nr, part = (k - nv) % nr;  // row vector, piece within it
+    return ColPiece{1 + q, j0 + 4 * part, rows_dst + q * R + 4 * part};
   }
-  return ColPiece{-1, 0, 0, false};
+  return ColPiece{-1, 0, 0};
 }
 
 // Issues the pieces pc of tokens t0 .. t0 + n - 1 into buf (TS floats per
 // token); per token each source advances by one row.
-template <typename Tin>
 __device__ __forceinline__ void col_issue(const BParams &Q, const ColPiece (&pc)[4], int bh, int t0,
                                           int n, float *buf, int TS) {
   const KParams &P = Q.P;
   const int dv = P.dv;
   if (!in_bounds(P.err, ((size_t)bh * P.T + t0 + n) * dv <= Q.n_rows)) return;
   const float *g0 = gen_at(Q, bh, t0);
-  const float *de0 = Q.delta + ((size_t)bh * P.T + t0) * dv;
-  const float *dd0 = Q.dd + ((size_t)bh * P.T + t0) * dv;
-  const Tin *o0 = Q.dO ? reinterpret_cast<const Tin *>(Q.dO) + tok_index(P, bh / P.H, t0, bh % P.H) * dv
-                       : nullptr;
-  const size_t ostride = (size_t)P.H * dv;
+  const size_t r0 = ((size_t)bh * P.T + t0) * dv;
 #pragma unroll
   for (int p2 = 0; p2 < 4; ++p2) {
     const ColPiece c = pc[p2];
@@ -776,18 +731,16 @@ __device__ __forceinline__ void col_issue(const BParams &Q, const ColPiece (&pc)
     const uint32_t d = smem_u32(buf + c.dst);
     if (c.kind == 0) {
       for (int tt = 0; tt < n; ++tt) cp_async16(d + tt * TS * 4, g0 + (size_t)tt * Q.GS + c.src, true);
-    } else if (c.kind == 3) {
-      for (int tt = 0; tt < n; ++tt) cp_async16(d + tt * TS * 4, o0 + tt * ostride + c.src, c.valid);
     } else {
-      const float *r0 = (c.kind == 1 ? de0 : dd0) + c.src;
-      for (int tt = 0; tt < n; ++tt) cp_async16(d + tt * TS * 4, r0 + (size_t)tt * dv, true);
+      const float *src = (c.kind == 1 ? Q.delta : c.kind == 2 ? Q.dd : Q.cdo) + r0 + c.src;
+      for (int tt = 0; tt < n; ++tt) cp_async16(d + tt * TS * 4, src + (size_t)tt * dv, true);
     }
   }
 }
 
 // F2: forward, S_t = S_{t-1} Diag(alpha_t) + delta_t w_t^T;
 // dq'_t = c S_t^T dO_t and dr_t = -P_t^T dd_t.
-template <typename Tin, int R>
+template <int R>
 __global__ void __launch_bounds__(128) f2_kernel(const BParams Q) {
   extern __shared__ float4 smem4[];
   float *sm = reinterpret_cast<float *>(smem4);
@@ -798,19 +751,18 @@ __global__ void __launch_bounds__(128) f2_kernel(const BParams Q) {
   const int g = blockIdx.x % Q.G, j0 = g * R;
   const int tb = ck * kCk, te = min(T, tb + kCk);  // this CTA's tokens
   const int i = threadIdx.x;
-  const float cq = P.q_scale;
-  const int TS = 2 * dk + 3 * R;  // w | alpha | delta | dd | dO (raw)
-  const int nv = dk / 2, nr = R / 4, nd = Q.dO ? R * (int)sizeof(Tin) / 16 : 0;
+  const int TS = 2 * dk + 3 * R;  // w | alpha | delta | dd | c dO
+  const int nv = dk / 2, nr = R / 4, nd = Q.dO ? nr : 0;
   const int nc = (te - tb + kLCC - 1) / kLCC;
-  // this thread's pieces of every staged token (w | alpha, delta, dd, dO)
+  // this thread's pieces of every staged token (w | alpha, delta, dd, c dO)
   ColPiece pc[4];
 #pragma unroll
   for (int p2 = 0; p2 < 4; ++p2)
-    pc[p2] = col_piece<Tin>(threadIdx.x + p2 * (int)blockDim.x, 2 * dk, nv, 2 * dk, R, nd, j0, dv);
+    pc[p2] = col_piece(threadIdx.x + p2 * (int)blockDim.x, 2 * dk, nv, 2 * dk, R, nd, j0);
   auto issue = [&](int ch) {
     float *buf = sm + (ch & 1) * kLCC * TS;
     const int t0 = tb + ch * kLCC, n = min(kLCC, te - t0), per = nv + 2 * nr + nd;
-    col_issue<Tin>(Q, pc, bh, t0, n, buf, TS);
+    col_issue(Q, pc, bh, t0, n, buf, TS);
     // (pieces past four per thread: no shape with d_k >= 16 and R <= 64 has any)
     for (int tt = 0; tt < n; ++tt)
     for (int k = threadIdx.x + 4 * (int)blockDim.x; k < per; k += blockDim.x) {
@@ -823,7 +775,7 @@ __global__ void __launch_bounds__(128) f2_kernel(const BParams Q) {
       else if (k < nv + 2 * nr)
         stage_rows(Q.dd + row_base(Q, bh, t, j0, R), k - nv - nr, d + 2 * dk + R);
       else
-        stage_dO<Tin>(Q, bh, t, j0, k - nv - 2 * nr, d + 2 * dk + 2 * R);
+        stage_rows(Q.cdo + row_base(Q, bh, t, j0, R), k - nv - 2 * nr, d + 2 * dk + 2 * R);
     }
   };
   float2 S[R / 2];  // rows (2h, 2h + 1) of this column
@@ -853,7 +805,7 @@ __global__ void __launch_bounds__(128) f2_kernel(const BParams Q) {
         ld4(sv + 2 * dk + j, true, de);
         ld4(sv + 2 * dk + R + j, true, dd);
         if (Q.dO) {
-          ld_rows4<Tin>(sv + 2 * dk + 2 * R, j, go);
+          ld4(sv + 2 * dk + 2 * R + j, true, go);
         } else {
           go[0] = go[1] = go[2] = go[3] = 0.f;
         }
@@ -868,7 +820,7 @@ __global__ void __launch_bounds__(128) f2_kernel(const BParams Q) {
       }
       const size_t po = (((size_t)g * BH + bh) * T + t0 + tt) * 3 * dk;
       if (in_bounds(P.err, po + 3 * dk <= Q.n_part)) {
-        Q.part[po + i] = cq * (accq.x + accq.y);
+        Q.part[po + i] = accq.x + accq.y;
         Q.part[po + dk + i] = -(accr.x + accr.y);
       }
     }
@@ -878,7 +830,7 @@ __global__ void __launch_bounds__(128) f2_kernel(const BParams Q) {
 
 // R2: reverse, dS~_t = dS_t + c dO_t q'_t^T, dS_{t-1} = (dS~_t - dd_t r_t^T)
 // Diag(alpha_t); dw_t = dS~_t^T delta_t.
-template <typename Tin, int R>
+template <int R>
 __global__ void __launch_bounds__(128) r2_kernel(const BParams Q) {
   extern __shared__ float4 smem4[];
   float *sm = reinterpret_cast<float *>(smem4);
@@ -889,19 +841,18 @@ __global__ void __launch_bounds__(128) r2_kernel(const BParams Q) {
   const int g = blockIdx.x % Q.G, j0 = g * R;
   const int tb = ck * kCk, te = min(T, tb + kCk);  // this CTA's tokens
   const int i = threadIdx.x;
-  const float cq = P.q_scale;
-  const int TS = 4 * dk + 3 * R;  // q' | r | w | alpha | delta | dd | dO (raw)
-  const int nv = dk, nr = R / 4, nd = Q.dO ? R * (int)sizeof(Tin) / 16 : 0;
+  const int TS = 4 * dk + 3 * R;  // q' | r | w | alpha | delta | dd | c dO
+  const int nv = dk, nr = R / 4, nd = Q.dO ? nr : 0;
   const int nc = (te - tb + kLCC - 1) / kLCC;
-  // this thread's pieces of every staged token (q' | r | w | alpha, delta, dd, dO)
+  // this thread's pieces of every staged token (q' | r | w | alpha, delta, dd, c dO)
   ColPiece pc[4];
 #pragma unroll
   for (int p2 = 0; p2 < 4; ++p2)
-    pc[p2] = col_piece<Tin>(threadIdx.x + p2 * (int)blockDim.x, 0, nv, 4 * dk, R, nd, j0, dv);
+    pc[p2] = col_piece(threadIdx.x + p2 * (int)blockDim.x, 0, nv, 4 * dk, R, nd, j0);
   auto issue = [&](int ch) {
     float *buf = sm + (ch & 1) * kLCC * TS;
     const int t0 = tb + ch * kLCC, n = min(kLCC, te - t0), per = nv + 2 * nr + nd;
-    col_issue<Tin>(Q, pc, bh, t0, n, buf, TS);
+    col_issue(Q, pc, bh, t0, n, buf, TS);
     // (pieces past four per thread: no shape with d_k >= 16 and R <= 64 has any)
     for (int tt = 0; tt < n; ++tt)
     for (int k = threadIdx.x + 4 * (int)blockDim.x; k < per; k += blockDim.x) {
@@ -914,7 +865,7 @@ __global__ void __launch_bounds__(128) r2_kernel(const BParams Q) {
       else if (k < nv + 2 * nr)
         stage_rows(Q.dd + row_base(Q, bh, t, j0, R), k - nv - nr, d + 4 * dk + R);
       else
-        stage_dO<Tin>(Q, bh, t, j0, k - nv - 2 * nr, d + 4 * dk + 2 * R);
+        stage_rows(Q.cdo + row_base(Q, bh, t, j0, R), k - nv - 2 * nr, d + 4 * dk + 2 * R);
     }
   };
   float2 D[R / 2];  // rows (2h, 2h + 1) of this column
@@ -936,7 +887,7 @@ __global__ void __launch_bounds__(128) r2_kernel(const BParams Q) {
     const int t0 = tb + ch * kLCC, n = min(kLCC, te - t0);
     for (int tt = n - 1; tt >= 0; --tt) {
       const float *sv = buf + tt * TS;
-      const float2 cqq = dup2(cq * sv[i]), nr = dup2(-sv[dk + i]), a = dup2(sv[3 * dk + i]);
+      const float2 q2 = dup2(sv[i]), nr2 = dup2(-sv[dk + i]), a = dup2(sv[3 * dk + i]);
       float2 accw = make_float2(0.f, 0.f);  // even | odd rows
 #pragma unroll
       for (int j = 0; j < R; j += 4) {
@@ -944,16 +895,16 @@ __global__ void __launch_bounds__(128) r2_kernel(const BParams Q) {
         ld4(sv + 4 * dk + j, true, de);
         ld4(sv + 4 * dk + R + j, true, dd);
         if (Q.dO) {
-          ld_rows4<Tin>(sv + 4 * dk + 2 * R, j, go);
+          ld4(sv + 4 * dk + 2 * R + j, true, go);
         } else {
           go[0] = go[1] = go[2] = go[3] = 0.f;
         }
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
           float2 &d2 = D[j / 2 + h];
-          const float2 dt = fma2(cqq, make_float2(go[2 * h], go[2 * h + 1]), d2);
+          const float2 dt = fma2(q2, make_float2(go[2 * h], go[2 * h + 1]), d2);
           accw = fma2(dt, make_float2(de[2 * h], de[2 * h + 1]), accw);
-          d2 = mul2(fma2(make_float2(dd[2 * h], dd[2 * h + 1]), nr, dt), a);
+          d2 = mul2(fma2(make_float2(dd[2 * h], dd[2 * h + 1]), nr2, dt), a);
         }
       }
       const size_t po = (((size_t)g * BH + bh) * T + t0 + tt) * 3 * dk;
@@ -1196,12 +1147,12 @@ cudaError_t set_smem(K kernel, size_t bytes) {
 }
 
 // The merged row sweeps for C key channels per lane and RW rows per warp.
-template <typename Tin, int C, int RW, bool UNR>
+template <int C, int RW, bool UNR>
 cudaError_t launch_fr1_t(const BParams &Q, unsigned n, cudaStream_t st) {
   const size_t smem = 2 * kLCR * (4 * 32 * C + 4 * RW) * sizeof(float);  // R1's (> F1's)
-  const cudaError_t err = set_smem(fr1_kernel<Tin, C, RW, UNR>, smem);
+  const cudaError_t err = set_smem(fr1_kernel<C, RW, UNR>, smem);
   if (err != cudaSuccess) return err;
-  fr1_kernel<Tin, C, RW, UNR><<<2 * n, 128, smem, st>>>(Q, (int)n);
+  fr1_kernel<C, RW, UNR><<<2 * n, 128, smem, st>>>(Q, (int)n);
   return cudaSuccess;
 }
 
@@ -1212,19 +1163,18 @@ cudaError_t launch_fr1_t(const BParams &Q, unsigned n, cudaStream_t st) {
 // there are too few warps to hide latency (under two CTAs per SM, measured:
 // 26.1 against 28.7 ms on 32 pairs of 32k tokens; 6.07 against 6.28 ms on
 // the headline layer's 512 CTAs).
-template <typename Tin>
 cudaError_t launch_fr1(const BParams &Q, cudaStream_t st) {
   const KParams &P = Q.P;
   const int C = P.dk <= 32 ? 1 : P.dk <= 64 ? 2 : 4;
   const unsigned n = (unsigned)((long long)P.B * P.H * ((P.dv + 31) / 32));  // CTAs per sweep
   if (2LL * n >= 2LL * num_sms()) {
-    if (C == 4) return launch_fr1_t<Tin, 4, 8, true>(Q, n, st);
-    if (C == 2) return launch_fr1_t<Tin, 2, 8, true>(Q, n, st);
-    return launch_fr1_t<Tin, 1, 8, true>(Q, n, st);
+    if (C == 4) return launch_fr1_t<4, 8, true>(Q, n, st);
+    if (C == 2) return launch_fr1_t<2, 8, true>(Q, n, st);
+    return launch_fr1_t<1, 8, true>(Q, n, st);
   }
-  if (C == 4) return launch_fr1_t<Tin, 4, 8, false>(Q, n, st);
-  if (C == 2) return launch_fr1_t<Tin, 2, 8, false>(Q, n, st);
-  return launch_fr1_t<Tin, 1, 8, false>(Q, n, st);
+  if (C == 4) return launch_fr1_t<4, 8, false>(Q, n, st);
+  if (C == 2) return launch_fr1_t<2, 8, false>(Q, n, st);
+  return launch_fr1_t<1, 8, false>(Q, n, st);
 }
 
 template <typename Tin, int R>
@@ -1242,12 +1192,12 @@ cudaError_t launch_bwd_t(const BParams &Q, cudaStream_t st) {
 
   const size_t sm_f2 = 2 * kLCC * (2 * dk + 3 * R) * sizeof(float);
   const size_t sm_r2 = 2 * kLCC * (4 * dk + 3 * R) * sizeof(float);
-  if ((err = set_smem(f2_kernel<Tin, R>, sm_f2)) != cudaSuccess) return err;
-  if ((err = set_smem(r2_kernel<Tin, R>, sm_r2)) != cudaSuccess) return err;
+  if ((err = set_smem(f2_kernel<R>, sm_f2)) != cudaSuccess) return err;
+  if ((err = set_smem(r2_kernel<R>, sm_r2)) != cudaSuccess) return err;
   const unsigned grid_cols = (unsigned)(BH * Q.nck * Q.G);
-  if ((err = launch_fr1<Tin>(Q, st)) != cudaSuccess) return err;
-  f2_kernel<Tin, R><<<grid_cols, dk, sm_f2, st>>>(Q);
-  r2_kernel<Tin, R><<<grid_cols, dk, sm_r2, st>>>(Q);
+  if ((err = launch_fr1(Q, st)) != cudaSuccess) return err;
+  f2_kernel<R><<<grid_cols, dk, sm_f2, st>>>(Q);
+  r2_kernel<R><<<grid_cols, dk, sm_r2, st>>>(Q);
   e1_kernel<Tin><<<grid_for(BHT * 32, 256), 256, 0, st>>>(Q);
 
   if (P.decay != PDN_DECAY_NONE && Q.dla) {
@@ -1303,6 +1253,7 @@ cudaError_t launch_chunk_bwd(const KParams &P, const pdn_grads_t *g, void *works
   Q.dq = g->dq; Q.dk = g->dk; Q.dv = g->dv; Q.dla = g->dlog_alpha; Q.dbeta = g->dbeta;
   Q.derase = g->derase; Q.dwrite = g->dwrite; Q.dS0 = g->dS0; Q.dA0 = g->dA0;
   Q.gen = ws + L.gen; Q.acc = ws + L.acc; Q.delta = ws + L.delta; Q.dd = ws + L.dd;
+  Q.cdo = ws + L.cdo;
   Q.st = ws + L.st; Q.part = ws + L.part; Q.cpsi = ws + L.cpsi; Q.sigma = ws + L.sigma;
   Q.dacc = ws + L.dacc; Q.bsum = ws + L.bsum; Q.phi = ws + L.phi;
   Q.ckS = ws + L.ckS; Q.ckD = ws + L.ckD;
