@@ -154,19 +154,30 @@ __global__ void scan_part_kernel(const KParams P, ScanArr X, int nch, int nb, fl
 // Replaces each block total by the sum carried into that block (from the
 // sequence start when !rev, from its end when rev), seeded with init
 // ([BH][nch], may be NULL). total (may be NULL) gets the full sum + init.
+// Eight block totals are loaded at a time, so the walk over the blocks waits
+// on memory once per eight.
 __global__ void scan_carry_kernel(const KParams P, int nch, int nb, bool rev, float *bsum,
                                   const float *init, float *total) {
+  constexpr int kB = 8;
   const long long n = (long long)P.B * P.H * nch;
   for (long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x; e < n;
        e += (long long)gridDim.x * blockDim.x) {
     const int c = (int)(e % nch), bh = (int)(e / nch);
     float carry = init ? init[e] : 0.f;
-    for (int k = 0; k < nb; ++k) {
-      const int blk = rev ? nb - 1 - k : k;
-      float *p = bsum + ((size_t)bh * nb + blk) * nch + c;
-      const float s = *p;
-      *p = carry;
-      carry += s;
+    float *base = bsum + (size_t)bh * nb * nch + c;
+    for (int k0 = 0; k0 < nb; k0 += kB) {
+      float v[kB];
+#pragma unroll
+      for (int u = 0; u < kB; ++u) {
+        const int blk = rev ? nb - 1 - (k0 + u) : k0 + u;
+        v[u] = k0 + u < nb ? base[(size_t)blk * nch] : 0.f;
+      }
+#pragma unroll
+      for (int u = 0; u < kB; ++u) {
+        const int blk = rev ? nb - 1 - (k0 + u) : k0 + u;
+        if (k0 + u < nb) base[(size_t)blk * nch] = carry;
+        carry += v[u];
+      }
     }
     if (total) total[e] = carry;
   }
@@ -198,20 +209,47 @@ __global__ void scan_fill_kernel(const KParams P, ScanArr X, ScanArr Y, int nch,
 }
 
 // ---------------------------------------------------------------------------
+// Four consecutive input elements from element i (8- or 16-byte aligned),
+// widened to fp32.
+template <typename Tin>
+__device__ __forceinline__ void ld4_in(const void *p, size_t i, float (&v)[4]) {
+  if constexpr (sizeof(Tin) == 4) {
+    const float4 x = *reinterpret_cast<const float4 *>(static_cast<const float *>(p) + i);
+    v[0] = x.x; v[1] = x.y; v[2] = x.z; v[3] = x.w;
+  } else {
+    const uint2 x = *reinterpret_cast<const uint2 *>(static_cast<const __nv_bfloat16 *>(p) + i);
+    v[0] = __uint_as_float(x.x << 16); v[1] = __uint_as_float(x.x & 0xffff0000u);
+    v[2] = __uint_as_float(x.y << 16); v[3] = __uint_as_float(x.y & 0xffff0000u);
+  }
+}
+
+// The same where `ok`, else four copies of `fill`.
+template <typename Tin>
+__device__ __forceinline__ void ld4_opt(const void *p, size_t i, bool ok, float (&v)[4],
+                                        float fill = 0.f) {
+  if (ok) {
+    ld4_in<Tin>(p, i, v);
+  } else {
+    v[0] = v[1] = v[2] = v[3] = fill;
+  }
+}
+
 // Prep. acc[bh][t][i] = k_{t,i}^2 (preconditioned variants; the prefix sum
-// over tokens then makes it A_t).
+// over tokens then makes it A_t). One warp per (token, head), lane l on key
+// channels 4l .. 4l + 3.
 template <typename Tin>
 __global__ void prep_sq_kernel(const BParams Q) {
   const KParams &P = Q.P;
-  const int dk = P.dk;
-  const long long n = (long long)P.B * P.H * P.T * dk;
-  for (long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x; e < n;
-       e += (long long)gridDim.x * blockDim.x) {
-    const int i = (int)(e % dk);
-    const long long r = e / dk;
-    const int t = (int)(r % P.T), bh = (int)(r / P.T);
-    const float k = ldf<Tin>(P.k, tok_index(P, bh / P.H, t, bh % P.H) * dk + i);
-    Q.acc[e] = k * k;
+  const int lane = threadIdx.x & 31, dk = P.dk, c = 4 * lane;
+  const long long n = (long long)P.B * P.H * P.T;
+  const long long nw = ((long long)gridDim.x * blockDim.x) >> 5;
+  if (c >= dk) return;
+  for (long long wid = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5; wid < n; wid += nw) {
+    const int bh = (int)(wid / P.T), t = (int)(wid % P.T);
+    float k[4];
+    ld4_in<Tin>(P.k, tok_index(P, bh / P.H, t, bh % P.H) * dk + c, k);
+    *reinterpret_cast<float4 *>(Q.acc + (size_t)wid * dk + c) =
+        make_float4(k[0] * k[0], k[1] * k[1], k[2] * k[2], k[3] * k[3]);
   }
 }
 
@@ -233,11 +271,11 @@ __global__ void prep_gen_kernel(const BParams Q) {
     const int c = 4 * lane;
     const bool ak = c < dk, av = c < dv;
     float k[4], q[4], v[4], Bc[4], a[4];
+    ld4_opt<Tin>(P.k, tk * dk + c, ak, k);
+    ld4_opt<Tin>(P.q, tk * dk + c, ak, q);
+    ld4_opt<Tin>(P.v, tk * dv + c, av, v);
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
-      k[e] = ak ? ldf<Tin>(P.k, tk * dk + c + e) : 0.f;
-      q[e] = ak ? ldf<Tin>(P.q, tk * dk + c + e) : 0.f;
-      v[e] = av ? ldf<Tin>(P.v, tk * dv + c + e) : 0.f;
       Bc[e] = 1.f;
       a[e] = 1.f;
     }
@@ -258,8 +296,10 @@ __global__ void prep_gen_kernel(const BParams Q) {
 #pragma unroll
       for (int e = 0; e < 4; ++e) a[e] = ea;
     } else if (P.decay == PDN_DECAY_CHANNEL) {
+      float la[4];
+      ld4_opt<Tin>(P.log_alpha, tk * dk + c, ak, la);
 #pragma unroll
-      for (int e = 0; e < 4; ++e) a[e] = ak ? expf(ldf<Tin>(P.log_alpha, tk * dk + c + e)) : 1.f;
+      for (int e = 0; e < 4; ++e) a[e] = ak ? expf(la[e]) : 1.f;
     }
     float r[4], w[4], u[4], qq[4];
 #pragma unroll
@@ -291,22 +331,27 @@ __global__ void prep_gen_kernel(const BParams Q) {
       } break;
       case PDN_VAR_FG2_GDN: case PDN_VAR_FG2_GDN_PLUS: {
         const bool plus = P.variant == PDN_VAR_FG2_GDN_PLUS;
+        float bk[4], bv[4];
+        ld4_opt<Tin>(P.beta, tk * dk + c, ak, bk);
+        if (plus) ld4_opt<Tin>(P.write, tk * dv + c, av, bv);
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const float sb = ak ? sqrtf(ldf<Tin>(P.beta, tk * dk + c + e)) : 0.f;
+          const float sb = ak ? sqrtf(bk[e]) : 0.f;
           r[e] = sb * k[e];
           w[e] = sb * k[e];
-          const float bv = av ? (plus ? ldf<Tin>(P.write, tk * dv + c + e)
-                                      : ldf<Tin>(P.beta, tk * dk + c + e))
-                              : 0.f;
-          u[e] = sqrtf(bv) * v[e];
+          // (FG2-GDN: one gain for both sides, d_k = d_v)
+          const float g = av ? (plus ? bv[e] : bk[e]) : 0.f;
+          u[e] = sqrtf(g) * v[e];
         }
       } break;
       case PDN_VAR_GDN2: {
+        float er[4], gw[4];
+        ld4_opt<Tin>(P.erase, tk * dk + c, ak, er);
+        ld4_opt<Tin>(P.write, tk * dv + c, av, gw);
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          r[e] = ak ? ldf<Tin>(P.erase, tk * dk + c + e) * k[e] : 0.f;
-          u[e] = av ? ldf<Tin>(P.write, tk * dv + c + e) * v[e] : 0.f;
+          r[e] = er[e] * k[e];
+          u[e] = gw[e] * v[e];
         }
       } break;
       default: break;
@@ -321,8 +366,9 @@ __global__ void prep_gen_kernel(const BParams Q) {
     if (av) *reinterpret_cast<float4 *>(g + 4 * dk + c) = make_float4(u[0], u[1], u[2], u[3]);
     if (Q.dO && av) {  // c dO of the token, once, for the three sweeps that read it
       float o[4];
+      ld4_in<Tin>(Q.dO, tk * dv + c, o);
 #pragma unroll
-      for (int e = 0; e < 4; ++e) o[e] = P.q_scale * ldf<Tin>(Q.dO, tk * dv + c + e);
+      for (int e = 0; e < 4; ++e) o[e] *= P.q_scale;
       *reinterpret_cast<float4 *>(Q.cdo + ((size_t)bh * P.T + t) * dv + c) = make_float4(o[0], o[1], o[2], o[3]);
     }
   }
@@ -956,11 +1002,8 @@ __global__ void e1_kernel(const BParams Q) {
     ld4(gv + dk + c, ak, r);
     ld4(gv + 2 * dk + c, ak, w);
     ld4(Q.dd + ((size_t)bh * T + t) * dv + c, av, du);
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      k[e] = ak ? ldf<Tin>(P.k, tk * dk + c + e) : 0.f;
-      v[e] = av ? ldf<Tin>(P.v, tk * dv + c + e) : 0.f;
-    }
+    ld4_opt<Tin>(P.k, tk * dk + c, ak, k);
+    ld4_opt<Tin>(P.v, tk * dv + c, av, v);
     // decay: this token's term q'.dq' - w.dw + r.dr
     if (P.decay != PDN_DECAY_NONE) {
       float cp[4], s = 0.f;
@@ -991,9 +1034,9 @@ __global__ void e1_kernel(const BParams Q) {
     float mu = 0.f;
     if (pre) {
       float s = 0.f;
+      ld4(Q.acc + ((size_t)bh * T + t) * dk + c, ak, A);
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        A[e] = ak ? Q.acc[((size_t)bh * T + t) * dk + c + e] : 0.f;
         L[e] = ak ? logf(A[e] + P.eps) : 0.f;
         s += L[e];
       }
@@ -1017,10 +1060,11 @@ __global__ void e1_kernel(const BParams Q) {
       } break;
       case PDN_VAR_PLA: {
         const float be = reinterpret_cast<const float *>(P.beta)[tk];
-        float db = 0.f;
+        float db = 0.f, qv[4];
+        ld4_opt<Tin>(P.q, tk * dk + c, ak, qv);
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const float q = ak ? ldf<Tin>(P.q, tk * dk + c + e) : 0.f;
+          const float q = qv[e];
           gk[e] = be * dw[e];
           db = fmaf(k[e], dw[e], db);
           dB[e] = q * dq[e];
@@ -1031,14 +1075,16 @@ __global__ void e1_kernel(const BParams Q) {
       } break;
       case PDN_VAR_FG2_GDN: case PDN_VAR_FG2_GDN_PLUS: {
         const bool plus = P.variant == PDN_VAR_FG2_GDN_PLUS;
-        float dbk[4], dwr[4];
+        float dbk[4], dwr[4], bkv[4], bvv[4];
+        ld4_opt<Tin>(P.beta, tk * dk + c, ak, bkv, 1.f);
+        if (plus) ld4_opt<Tin>(P.write, tk * dv + c, av, bvv, 1.f);
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const float bk = ak ? ldf<Tin>(P.beta, tk * dk + c + e) : 1.f;
+          const float bk = bkv[e];
           const float sb = sqrtf(bk);
           gk[e] = sb * (dr[e] + dw[e]);
           dbk[e] = k[e] * (dr[e] + dw[e]) / (2.f * sb);
-          const float bv = av ? (plus ? ldf<Tin>(P.write, tk * dv + c + e) : bk) : 1.f;
+          const float bv = av ? (plus ? bvv[e] : bk) : 1.f;
           const float sv = sqrtf(bv);
           gvv[e] = sv * du[e];
           dwr[e] = v[e] * du[e] / (2.f * sv);
@@ -1050,11 +1096,13 @@ __global__ void e1_kernel(const BParams Q) {
           *reinterpret_cast<float4 *>(Q.dwrite + tk * dv + c) = make_float4(dwr[0], dwr[1], dwr[2], dwr[3]);
       } break;
       case PDN_VAR_GDN2: {
-        float de[4], dg[4];
+        float de[4], dg[4], erv[4], gwv[4];
+        ld4_opt<Tin>(P.erase, tk * dk + c, ak, erv);
+        ld4_opt<Tin>(P.write, tk * dv + c, av, gwv);
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const float er = ak ? ldf<Tin>(P.erase, tk * dk + c + e) : 0.f;
-          const float gw = av ? ldf<Tin>(P.write, tk * dv + c + e) : 0.f;
+          const float er = erv[e];
+          const float gw = gwv[e];
           gk[e] = er * dr[e] + dw[e];
           de[e] = k[e] * dr[e];
           gvv[e] = gw * du[e];
@@ -1098,15 +1146,22 @@ __global__ void e1_kernel(const BParams Q) {
 template <typename Tin>
 __global__ void e3_kernel(const BParams Q) {
   const KParams &P = Q.P;
-  const int dk = P.dk;
-  const long long n = (long long)P.B * P.H * P.T * dk;
-  for (long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x; e < n;
-       e += (long long)gridDim.x * blockDim.x) {
-    const int i = (int)(e % dk);
-    const long long r = e / dk;
-    const int t = (int)(r % P.T), bh = (int)(r / P.T);
-    const size_t o = tok_index(P, bh / P.H, t, bh % P.H) * dk + i;
-    Q.dk[o] += 2.f * ldf<Tin>(P.k, o) * Q.dacc[e];
+  const int lane = threadIdx.x & 31, dk = P.dk, c = 4 * lane;
+  const long long n = (long long)P.B * P.H * P.T;
+  const long long nw = ((long long)gridDim.x * blockDim.x) >> 5;
+  if (c >= dk) return;
+  for (long long wid = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5; wid < n; wid += nw) {
+    const int bh = (int)(wid / P.T), t = (int)(wid % P.T);
+    const size_t o = tok_index(P, bh / P.H, t, bh % P.H) * dk + c;
+    float k[4];
+    ld4_in<Tin>(P.k, o, k);
+    const float4 da = *reinterpret_cast<const float4 *>(Q.dacc + (size_t)wid * dk + c);
+    float4 g = *reinterpret_cast<const float4 *>(Q.dk + o);
+    g.x += 2.f * k[0] * da.x;
+    g.y += 2.f * k[1] * da.y;
+    g.z += 2.f * k[2] * da.z;
+    g.w += 2.f * k[3] * da.w;
+    *reinterpret_cast<float4 *>(Q.dk + o) = g;
   }
 }
 
@@ -1184,7 +1239,7 @@ cudaError_t launch_bwd_t(const BParams &Q, cudaStream_t st) {
   const long long BH = (long long)P.B * P.H, BHT = BH * P.T;
   cudaError_t err;
   if (is_precond(P.variant)) {
-    prep_sq_kernel<Tin><<<grid_for(BHT * dk, 256), 256, 0, st>>>(Q);
+    prep_sq_kernel<Tin><<<grid_for(BHT * 32, 256), 256, 0, st>>>(Q);
     run_scan(P, ScanArr{Q.acc, false}, ScanArr{Q.acc, false}, dk, Q.nb, false, P.A0, nullptr,
              Q.bsum, st);
   }
@@ -1212,7 +1267,7 @@ cudaError_t launch_bwd_t(const BParams &Q, cudaStream_t st) {
   if (is_precond(P.variant) && (Q.dk || Q.dA0)) {
     run_scan(P, ScanArr{Q.dacc, false}, ScanArr{Q.dacc, false}, dk, Q.nb, true, nullptr, Q.dA0,
              Q.bsum, st);
-    if (Q.dk) e3_kernel<Tin><<<grid_for(BHT * dk, 256), 256, 0, st>>>(Q);
+    if (Q.dk) e3_kernel<Tin><<<grid_for(BHT * 32, 256), 256, 0, st>>>(Q);
   }
   return cudaGetLastError();
 }
