@@ -968,8 +968,10 @@ __global__ void __launch_bounds__(128) r2_kernel(const BParams Q) {
 // the preconditioner, the dA_t of its own coefficients:
 //   B = x^-s, s = c / (1 + |c|), c = L - mean(L), L = log(A + eps)
 //   => dA = (dc - mean(dc)) / (A + eps), dc = -ln x B dB / (1 + |c|)^2.
+// (At most 64 registers: four 256-thread blocks per SM keep enough loads in
+// flight; with the compiler's 85, two blocks left it waiting on memory.)
 template <typename Tin>
-__global__ void e1_kernel(const BParams Q) {
+__global__ void __launch_bounds__(256, 4) e1_kernel(const BParams Q) {
   const KParams &P = Q.P;
   const int lane = threadIdx.x & 31, dk = P.dk, dv = P.dv, T = P.T, BH = P.B * P.H;
   const long long n = (long long)BH * T;

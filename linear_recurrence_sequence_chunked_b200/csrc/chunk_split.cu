@@ -65,7 +65,7 @@ constexpr float kLn2 = 0.6931471805599453f;
 // One CTA per (batch, head, chunk): thread (8-channel group, token lane)
 // loads 16-byte rows and squares them; the 16 token lanes are summed in
 // shared memory.
-__global__ void __launch_bounds__(256) k0_chunk_energy(const KParams P, void *ws, int N) {
+__global__ void __launch_bounds__(256, 4) k0_chunk_energy(const KParams P, void *ws, int N) {
   __shared__ float part[16][kD + 4];
   const int tid = threadIdx.x, c8 = tid & 15, tl = tid >> 4;
   const int BH = P.B * P.H, total = N * BH;
