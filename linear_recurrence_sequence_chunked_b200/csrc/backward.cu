@@ -1215,25 +1215,30 @@ cudaError_t launch_fr1_t(const BParams &Q, unsigned n, cudaStream_t st) {
   return cudaSuccess;
 }
 
-// Key channels per lane: 32 lanes cover d_k. Rows per warp: 8 (measured
-// against 4 on B200: as fast or faster on every workload, including 32
-// (batch, head) pairs of 32k tokens, where 4 gives twice the CTAs). The
-// unrolled chunk loop issues fewer instructions but schedules worse when
-// there are too few warps to hide latency (under two CTAs per SM, measured:
-// 26.1 against 28.7 ms on 32 pairs of 32k tokens; 6.07 against 6.28 ms on
-// the headline layer's 512 CTAs).
+// Key channels per lane: 32 lanes cover d_k. Rows per warp: 8 (each staged
+// vector serves more rows) when that still gives at least two CTAs per SM,
+// else 4 (twice the CTAs). The unrolled chunk loop issues fewer instructions
+// but schedules worse when too few warps hide its latency, so it runs only
+// from one CTA per SM per sweep on. Measured on B200 (ms per backward):
+// headline layer (512 CTAs at 8 rows) 5.31 with 8 rows against 5.62 with 4;
+// 32 (batch, head) pairs of 32k tokens 24.3 with 8 rows (rolled) against 22.6
+// with 4 (unrolled); unrolled against rolled at 8 rows there: 28.7 against
+// 26.1.
+template <int C>
+cudaError_t launch_fr1_c(const BParams &Q, unsigned n, bool rw8, bool unr, cudaStream_t st) {
+  if (rw8) return unr ? launch_fr1_t<C, 8, true>(Q, n, st) : launch_fr1_t<C, 8, false>(Q, n, st);
+  return unr ? launch_fr1_t<C, 4, true>(Q, n, st) : launch_fr1_t<C, 4, false>(Q, n, st);
+}
 cudaError_t launch_fr1(const BParams &Q, cudaStream_t st) {
   const KParams &P = Q.P;
-  const int C = P.dk <= 32 ? 1 : P.dk <= 64 ? 2 : 4;
-  const unsigned n = (unsigned)((long long)P.B * P.H * ((P.dv + 31) / 32));  // CTAs per sweep
-  if (2LL * n >= 2LL * num_sms()) {
-    if (C == 4) return launch_fr1_t<4, 8, true>(Q, n, st);
-    if (C == 2) return launch_fr1_t<2, 8, true>(Q, n, st);
-    return launch_fr1_t<1, 8, true>(Q, n, st);
-  }
-  if (C == 4) return launch_fr1_t<4, 8, false>(Q, n, st);
-  if (C == 2) return launch_fr1_t<2, 8, false>(Q, n, st);
-  return launch_fr1_t<1, 8, false>(Q, n, st);
+  const long long BH = (long long)P.B * P.H, sms = num_sms();
+  const long long n8 = BH * ((P.dv + 31) / 32);  // CTAs per sweep at 8 rows per warp
+  const bool rw8 = 2 * n8 >= 2 * sms;
+  const unsigned n = (unsigned)(rw8 ? n8 : BH * ((P.dv + 15) / 16));
+  const bool unr = (long long)n >= sms;
+  if (P.dk > 64) return launch_fr1_c<4>(Q, n, rw8, unr, st);
+  if (P.dk > 32) return launch_fr1_c<2>(Q, n, rw8, unr, st);
+  return launch_fr1_c<1>(Q, n, rw8, unr, st);
 }
 
 template <typename Tin, int R>

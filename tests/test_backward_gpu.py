@@ -165,12 +165,14 @@ def test_backward_full_size_sampled(name, chains):
     check_sampled_chains(WORKLOADS[name], chains)
 
 
-@pytest.mark.parametrize("variant,dk", [("PKDA", 128), ("GDN2", 64), ("FG2_GDN_PLUS", 128)])
-def test_backward_many_chains_ragged(variant, dk):
-    """Enough (batch, head) pairs for the row sweeps' unrolled chunk loop (at
-    least one CTA per SM), with a token count that leaves a ragged last chunk
-    of 3 tokens; sampled chains, the last one included."""
-    w = small(variant, "bf16", B=10 if dk == 64 else 5, T=203, H=16, dk=dk)
+@pytest.mark.parametrize("variant,dk,dv,B", [("PKDA", 128, 128, 5), ("GDN2", 64, 64, 10),
+                                            ("FG2_GDN_PLUS", 128, 128, 5), ("GDN2", 48, 80, 8)])
+def test_backward_many_chains_ragged(variant, dk, dv, B):
+    """Enough (batch, head) pairs for the row sweeps' widest layout (8 rows per
+    warp) and their unrolled chunk loop, with a token count that leaves a
+    ragged last chunk of 3 tokens (and, for d_v = 80, a partial group of
+    rows); sampled chains, the last one included."""
+    w = small(variant, "bf16", B=B, T=203, H=16, dk=dk, dv=dv)
     check_sampled_chains(w, [(0, 0), (w.B // 2, 7), (w.B - 1, w.H - 1)])
 
 
