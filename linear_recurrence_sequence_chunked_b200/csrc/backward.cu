@@ -209,6 +209,12 @@ __global__ void scan_fill_kernel(const KParams P, ScanArr X, ScanArr Y, int nch,
 }
 
 // ---------------------------------------------------------------------------
+// Four consecutive floats from p (16-byte aligned) where `ok`, else zeros.
+__device__ __forceinline__ void ld4(const float *p, bool ok, float (&v)[4]) {
+  const float4 x = ok ? *reinterpret_cast<const float4 *>(p) : make_float4(0.f, 0.f, 0.f, 0.f);
+  v[0] = x.x; v[1] = x.y; v[2] = x.z; v[3] = x.w;
+}
+
 // Four consecutive input elements from element i (8- or 16-byte aligned),
 // widened to fp32.
 template <typename Tin>
@@ -234,27 +240,36 @@ __device__ __forceinline__ void ld4_opt(const void *p, size_t i, bool ok, float 
   }
 }
 
-// Prep. acc[bh][t][i] = k_{t,i}^2 (preconditioned variants; the prefix sum
-// over tokens then makes it A_t). One warp per (token, head), lane l on key
-// channels 4l .. 4l + 3.
+// Prep (preconditioned variants): the block totals of k_{t,i}^2 over each
+// kScanBlk-token block, into bsum[bh][block][i], for the carry pass; the
+// generic-vector pass then accumulates A_t = A_0 + sum_{s<=t} k_s^2 inside
+// each block in the same order as the sums here.
 template <typename Tin>
-__global__ void prep_sq_kernel(const BParams Q) {
+__global__ void ksq_part_kernel(const BParams Q) {
   const KParams &P = Q.P;
-  const int lane = threadIdx.x & 31, dk = P.dk, c = 4 * lane;
-  const long long n = (long long)P.B * P.H * P.T;
-  const long long nw = ((long long)gridDim.x * blockDim.x) >> 5;
-  if (c >= dk) return;
-  for (long long wid = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5; wid < n; wid += nw) {
-    const int bh = (int)(wid / P.T), t = (int)(wid % P.T);
-    float k[4];
-    ld4_in<Tin>(P.k, tok_index(P, bh / P.H, t, bh % P.H) * dk + c, k);
-    *reinterpret_cast<float4 *>(Q.acc + (size_t)wid * dk + c) =
-        make_float4(k[0] * k[0], k[1] * k[1], k[2] * k[2], k[3] * k[3]);
+  const int dk = P.dk, nb = Q.nb;
+  const long long n = (long long)P.B * P.H * nb * dk;
+  for (long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x; e < n;
+       e += (long long)gridDim.x * blockDim.x) {
+    const int c = (int)(e % dk);
+    const long long r = e / dk;
+    const int blk = (int)(r % nb), bh = (int)(r / nb);
+    const int t0 = blk * kScanBlk, t1 = min(P.T, t0 + kScanBlk);
+    float s = 0.f;
+#pragma unroll 8
+    for (int t = t0; t < t1; ++t) {
+      const float k = ldf<Tin>(P.k, tok_index(P, bh / P.H, t, bh % P.H) * dk + c);
+      s += k * k;
+    }
+    Q.bsum[e] = s;
   }
 }
 
-// The variant's (q', r, w, alpha, u) of every token, one warp per (token,
-// head); lane l holds channels 4l..4l+3 of the key side and of the value side.
+// The variant's (q', r, w, alpha, u) of every token, one warp per (head,
+// kScanBlk-token block) walking its tokens in order; lane l holds channels
+// 4l..4l+3 of the key side and of the value side. For the preconditioned
+// variants the warp carries A_t from the block's carry-in (bsum) and writes
+// it to acc for the chain rules.
 // Variant table: DN/GDN/KDA r = k, w = beta k, u = v; PDN/PGDN/PKDA w = beta
 // (B_t . k); FG2-GDN r = w = sqrt(beta) . k, u = sqrt(beta) . v; GDN-2 r = e . k,
 // w = k, u = g . v; PLA r = 0, w = beta k, q' = B_t . q; FG2-GDN+ r = w =
@@ -263,113 +278,123 @@ template <typename Tin>
 __global__ void prep_gen_kernel(const BParams Q) {
   const KParams &P = Q.P;
   const int lane = threadIdx.x & 31, dk = P.dk, dv = P.dv;
-  const long long n = (long long)P.B * P.H * P.T;
+  const long long nblk = (long long)P.B * P.H * Q.nb;
   const long long nw = ((long long)gridDim.x * blockDim.x) >> 5;
-  for (long long wid = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5; wid < n; wid += nw) {
-    const int bh = (int)(wid / P.T), t = (int)(wid % P.T);
-    const size_t tk = tok_index(P, bh / P.H, t, bh % P.H);
-    const int c = 4 * lane;
-    const bool ak = c < dk, av = c < dv;
-    float k[4], q[4], v[4], Bc[4], a[4];
-    ld4_opt<Tin>(P.k, tk * dk + c, ak, k);
-    ld4_opt<Tin>(P.q, tk * dk + c, ak, q);
-    ld4_opt<Tin>(P.v, tk * dv + c, av, v);
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      Bc[e] = 1.f;
-      a[e] = 1.f;
-    }
-    if (is_precond(P.variant)) {
-      const float *A = Q.acc + ((size_t)bh * P.T + t) * dk;
-      float L[4], s = 0.f;
+  const bool pre = is_precond(P.variant);
+  const int c = 4 * lane;
+  const bool ak = c < dk, av = c < dv;
+  for (long long wid = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5; wid < nblk; wid += nw) {
+    const int bh = (int)(wid / Q.nb), blk = (int)(wid % Q.nb);
+    const int t_begin = blk * kScanBlk, t_end = min(P.T, t_begin + kScanBlk);
+    float Arun[4];  // A before the current token (the block's carry-in first)
+    ld4(pre ? Q.bsum + ((size_t)bh * Q.nb + blk) * dk + c : nullptr, pre && ak, Arun);
+    for (int t = t_begin; t < t_end; ++t) {
+      const size_t tk = tok_index(P, bh / P.H, t, bh % P.H);
+      float k[4], q[4], v[4], Bc[4], a[4];
+      ld4_opt<Tin>(P.k, tk * dk + c, ak, k);
+      ld4_opt<Tin>(P.q, tk * dk + c, ak, q);
+      ld4_opt<Tin>(P.v, tk * dv + c, av, v);
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        L[e] = ak ? logf(A[c + e] + P.eps) : 0.f;
-        s += L[e];
+        Bc[e] = 1.f;
+        a[e] = 1.f;
       }
-      const float mu = warp_sum(s) / (float)dk;
+      if (pre) {
+        float L[4], s = 0.f;
 #pragma unroll
-      for (int e = 0; e < 4; ++e) Bc[e] = precond_coef(L[e], mu, P.lnx);
-    }
-    if (P.decay == PDN_DECAY_SCALAR) {
-      const float ea = expf(reinterpret_cast<const float *>(P.log_alpha)[tk]);
-#pragma unroll
-      for (int e = 0; e < 4; ++e) a[e] = ea;
-    } else if (P.decay == PDN_DECAY_CHANNEL) {
-      float la[4];
-      ld4_opt<Tin>(P.log_alpha, tk * dk + c, ak, la);
-#pragma unroll
-      for (int e = 0; e < 4; ++e) a[e] = ak ? expf(la[e]) : 1.f;
-    }
-    float r[4], w[4], u[4], qq[4];
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      r[e] = k[e];
-      w[e] = k[e];
-      u[e] = v[e];
-      qq[e] = q[e];
-    }
-    switch (P.variant) {
-      case PDN_VAR_DN: case PDN_VAR_GDN: case PDN_VAR_KDA: {
-        const float be = reinterpret_cast<const float *>(P.beta)[tk];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) w[e] = be * k[e];
-      } break;
-      case PDN_VAR_PDN: case PDN_VAR_PGDN: case PDN_VAR_PKDA: {
-        const float be = reinterpret_cast<const float *>(P.beta)[tk];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) w[e] = be * Bc[e] * k[e];
-      } break;
-      case PDN_VAR_PLA: {
-        const float be = reinterpret_cast<const float *>(P.beta)[tk];
+        for (int e = 0; e < 4; ++e) Arun[e] += k[e] * k[e];
+        if (ak)
+          *reinterpret_cast<float4 *>(Q.acc + ((size_t)bh * P.T + t) * dk + c) =
+              make_float4(Arun[0], Arun[1], Arun[2], Arun[3]);
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          r[e] = 0.f;
-          w[e] = be * k[e];
-          qq[e] = Bc[e] * q[e];
+          L[e] = ak ? logf(Arun[e] + P.eps) : 0.f;
+          s += L[e];
         }
-      } break;
-      case PDN_VAR_FG2_GDN: case PDN_VAR_FG2_GDN_PLUS: {
-        const bool plus = P.variant == PDN_VAR_FG2_GDN_PLUS;
-        float bk[4], bv[4];
-        ld4_opt<Tin>(P.beta, tk * dk + c, ak, bk);
-        if (plus) ld4_opt<Tin>(P.write, tk * dv + c, av, bv);
+        const float mu = warp_sum(s) / (float)dk;
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float sb = ak ? sqrtf(bk[e]) : 0.f;
-          r[e] = sb * k[e];
-          w[e] = sb * k[e];
-          // (FG2-GDN: one gain for both sides, d_k = d_v)
-          const float g = av ? (plus ? bv[e] : bk[e]) : 0.f;
-          u[e] = sqrtf(g) * v[e];
-        }
-      } break;
-      case PDN_VAR_GDN2: {
-        float er[4], gw[4];
-        ld4_opt<Tin>(P.erase, tk * dk + c, ak, er);
-        ld4_opt<Tin>(P.write, tk * dv + c, av, gw);
+        for (int e = 0; e < 4; ++e) Bc[e] = precond_coef(L[e], mu, P.lnx);
+      }
+      if (P.decay == PDN_DECAY_SCALAR) {
+        const float ea = expf(reinterpret_cast<const float *>(P.log_alpha)[tk]);
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          r[e] = er[e] * k[e];
-          u[e] = gw[e] * v[e];
-        }
-      } break;
-      default: break;
-    }
-    float *g = gen_at(Q, bh, t);
-    if (ak) {
-      *reinterpret_cast<float4 *>(g + c) = make_float4(qq[0], qq[1], qq[2], qq[3]);
-      *reinterpret_cast<float4 *>(g + dk + c) = make_float4(r[0], r[1], r[2], r[3]);
-      *reinterpret_cast<float4 *>(g + 2 * dk + c) = make_float4(w[0], w[1], w[2], w[3]);
-      *reinterpret_cast<float4 *>(g + 3 * dk + c) = make_float4(a[0], a[1], a[2], a[3]);
-    }
-    if (av) *reinterpret_cast<float4 *>(g + 4 * dk + c) = make_float4(u[0], u[1], u[2], u[3]);
-    if (Q.dO && av) {  // c dO of the token, once, for the three sweeps that read it
-      float o[4];
-      ld4_in<Tin>(Q.dO, tk * dv + c, o);
+        for (int e = 0; e < 4; ++e) a[e] = ea;
+      } else if (P.decay == PDN_DECAY_CHANNEL) {
+        float la[4];
+        ld4_opt<Tin>(P.log_alpha, tk * dk + c, ak, la);
 #pragma unroll
-      for (int e = 0; e < 4; ++e) o[e] *= P.q_scale;
-      *reinterpret_cast<float4 *>(Q.cdo + ((size_t)bh * P.T + t) * dv + c) = make_float4(o[0], o[1], o[2], o[3]);
+        for (int e = 0; e < 4; ++e) a[e] = ak ? expf(la[e]) : 1.f;
+      }
+      float r[4], w[4], u[4], qq[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        r[e] = k[e];
+        w[e] = k[e];
+        u[e] = v[e];
+        qq[e] = q[e];
+      }
+      switch (P.variant) {
+        case PDN_VAR_DN: case PDN_VAR_GDN: case PDN_VAR_KDA: {
+          const float be = reinterpret_cast<const float *>(P.beta)[tk];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) w[e] = be * k[e];
+        } break;
+        case PDN_VAR_PDN: case PDN_VAR_PGDN: case PDN_VAR_PKDA: {
+          const float be = reinterpret_cast<const float *>(P.beta)[tk];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) w[e] = be * Bc[e] * k[e];
+        } break;
+        case PDN_VAR_PLA: {
+          const float be = reinterpret_cast<const float *>(P.beta)[tk];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            r[e] = 0.f;
+            w[e] = be * k[e];
+            qq[e] = Bc[e] * q[e];
+          }
+        } break;
+        case PDN_VAR_FG2_GDN: case PDN_VAR_FG2_GDN_PLUS: {
+          const bool plus = P.variant == PDN_VAR_FG2_GDN_PLUS;
+          float bk[4], bv[4];
+          ld4_opt<Tin>(P.beta, tk * dk + c, ak, bk);
+          if (plus) ld4_opt<Tin>(P.write, tk * dv + c, av, bv);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float sb = ak ? sqrtf(bk[e]) : 0.f;
+            r[e] = sb * k[e];
+            w[e] = sb * k[e];
+            // (FG2-GDN: one gain for both sides, d_k = d_v)
+            const float g = av ? (plus ? bv[e] : bk[e]) : 0.f;
+            u[e] = sqrtf(g) * v[e];
+          }
+        } break;
+        case PDN_VAR_GDN2: {
+          float er[4], gw[4];
+          ld4_opt<Tin>(P.erase, tk * dk + c, ak, er);
+          ld4_opt<Tin>(P.write, tk * dv + c, av, gw);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            r[e] = er[e] * k[e];
+            u[e] = gw[e] * v[e];
+          }
+        } break;
+        default: break;
+      }
+      float *g = gen_at(Q, bh, t);
+      if (ak) {
+        *reinterpret_cast<float4 *>(g + c) = make_float4(qq[0], qq[1], qq[2], qq[3]);
+        *reinterpret_cast<float4 *>(g + dk + c) = make_float4(r[0], r[1], r[2], r[3]);
+        *reinterpret_cast<float4 *>(g + 2 * dk + c) = make_float4(w[0], w[1], w[2], w[3]);
+        *reinterpret_cast<float4 *>(g + 3 * dk + c) = make_float4(a[0], a[1], a[2], a[3]);
+      }
+      if (av) *reinterpret_cast<float4 *>(g + 4 * dk + c) = make_float4(u[0], u[1], u[2], u[3]);
+      if (Q.dO && av) {  // c dO of the token, once, for the three sweeps that read it
+        float o[4];
+        ld4_in<Tin>(Q.dO, tk * dv + c, o);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) o[e] *= P.q_scale;
+        *reinterpret_cast<float4 *>(Q.cdo + ((size_t)bh * P.T + t) * dv + c) = make_float4(o[0], o[1], o[2], o[3]);
+      }
     }
   }
 }
@@ -398,11 +423,6 @@ __global__ void prep_gen_kernel(const BParams Q) {
 // and the generic vectors), so they run as one launch, R1's CTAs first (the
 // longer sweep), both resident at once.
 constexpr int kLCR = 8;  // tokens staged per chunk in F1 / R1
-
-__device__ __forceinline__ void ld4(const float *p, bool ok, float (&v)[4]) {
-  const float4 x = ok ? *reinterpret_cast<const float4 *>(p) : make_float4(0.f, 0.f, 0.f, 0.f);
-  v[0] = x.x; v[1] = x.y; v[2] = x.z; v[3] = x.w;
-}
 
 // C consecutive floats (16-, 8- or 4-byte aligned) to registers and back;
 // a NULL source reads zeros.
@@ -1248,11 +1268,11 @@ cudaError_t launch_bwd_t(const BParams &Q, cudaStream_t st) {
   const long long BH = (long long)P.B * P.H, BHT = BH * P.T;
   cudaError_t err;
   if (is_precond(P.variant)) {
-    prep_sq_kernel<Tin><<<grid_for(BHT * 32, 256), 256, 0, st>>>(Q);
-    run_scan(P, ScanArr{Q.acc, false}, ScanArr{Q.acc, false}, dk, Q.nb, false, P.A0, nullptr,
-             Q.bsum, st);
+    ksq_part_kernel<Tin><<<grid_for(BH * Q.nb * dk, 256), 256, 0, st>>>(Q);
+    scan_carry_kernel<<<grid_for(BH * dk, 128), 128, 0, st>>>(P, dk, Q.nb, false, Q.bsum, P.A0,
+                                                             nullptr);
   }
-  prep_gen_kernel<Tin><<<grid_for(BHT * 32, 256), 256, 0, st>>>(Q);
+  prep_gen_kernel<Tin><<<grid_for(BH * Q.nb * 32, 256), 256, 0, st>>>(Q);
 
   const size_t sm_f2 = 2 * kLCC * (2 * dk + 3 * R) * sizeof(float);
   const size_t sm_r2 = 2 * kLCC * (4 * dk + 3 * R) * sizeof(float);
