@@ -1166,26 +1166,33 @@ __global__ void __launch_bounds__(256, 4) e1_kernel(const BParams Q) {
 }
 
 // E3 (preconditioned variants): k_t feeds A_s for every s >= t, so
-// dk_t += 2 k_t . (sum_{s>=t} dA_s) (the suffix sums sit in dacc).
+// dk_t += 2 k_t . (sum_{s>=t} dA_s). One warp per (head, kScanBlk-token
+// block) walks its tokens from the last, the suffix sum starting from the
+// block's carry (the sum over all later blocks, in bsum).
 template <typename Tin>
 __global__ void e3_kernel(const BParams Q) {
   const KParams &P = Q.P;
   const int lane = threadIdx.x & 31, dk = P.dk, c = 4 * lane;
-  const long long n = (long long)P.B * P.H * P.T;
+  const long long nblk = (long long)P.B * P.H * Q.nb;
   const long long nw = ((long long)gridDim.x * blockDim.x) >> 5;
   if (c >= dk) return;
-  for (long long wid = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5; wid < n; wid += nw) {
-    const int bh = (int)(wid / P.T), t = (int)(wid % P.T);
-    const size_t o = tok_index(P, bh / P.H, t, bh % P.H) * dk + c;
-    float k[4];
-    ld4_in<Tin>(P.k, o, k);
-    const float4 da = *reinterpret_cast<const float4 *>(Q.dacc + (size_t)wid * dk + c);
-    float4 g = *reinterpret_cast<const float4 *>(Q.dk + o);
-    g.x += 2.f * k[0] * da.x;
-    g.y += 2.f * k[1] * da.y;
-    g.z += 2.f * k[2] * da.z;
-    g.w += 2.f * k[3] * da.w;
-    *reinterpret_cast<float4 *>(Q.dk + o) = g;
+  for (long long wid = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5; wid < nblk; wid += nw) {
+    const int bh = (int)(wid / Q.nb), blk = (int)(wid % Q.nb);
+    const int t_begin = blk * kScanBlk, t_end = min(P.T, t_begin + kScanBlk);
+    float4 y = *reinterpret_cast<const float4 *>(Q.bsum + ((size_t)bh * Q.nb + blk) * dk + c);
+    for (int t = t_end - 1; t >= t_begin; --t) {
+      const size_t o = tok_index(P, bh / P.H, t, bh % P.H) * dk + c;
+      float k[4];
+      ld4_in<Tin>(P.k, o, k);
+      const float4 da = *reinterpret_cast<const float4 *>(Q.dacc + ((size_t)bh * P.T + t) * dk + c);
+      y.x += da.x; y.y += da.y; y.z += da.z; y.w += da.w;
+      float4 g = *reinterpret_cast<const float4 *>(Q.dk + o);
+      g.x += 2.f * k[0] * y.x;
+      g.y += 2.f * k[1] * y.y;
+      g.z += 2.f * k[2] * y.z;
+      g.w += 2.f * k[3] * y.w;
+      *reinterpret_cast<float4 *>(Q.dk + o) = g;
+    }
   }
 }
 
@@ -1294,9 +1301,13 @@ cudaError_t launch_bwd_t(const BParams &Q, cudaStream_t st) {
                Q.dST ? Q.phi + BH * dk : nullptr, nullptr, Q.bsum, st);
   }
   if (is_precond(P.variant) && (Q.dk || Q.dA0)) {
-    run_scan(P, ScanArr{Q.dacc, false}, ScanArr{Q.dacc, false}, dk, Q.nb, true, nullptr, Q.dA0,
-             Q.bsum, st);
-    if (Q.dk) e3_kernel<Tin><<<grid_for(BHT * 32, 256), 256, 0, st>>>(Q);
+    // block totals of dA and the carries from the sequence end (dA0 gets
+    // the full sum); E3 finishes the suffix sums inside the blocks
+    scan_part_kernel<<<grid_for(BH * Q.nb * dk, 256), 256, 0, st>>>(P, ScanArr{Q.dacc, false}, dk,
+                                                                    Q.nb, Q.bsum);
+    scan_carry_kernel<<<grid_for(BH * dk, 128), 128, 0, st>>>(P, dk, Q.nb, true, Q.bsum, nullptr,
+                                                             Q.dA0);
+    if (Q.dk) e3_kernel<Tin><<<grid_for(BH * Q.nb * 32, 256), 256, 0, st>>>(Q);
   }
   return cudaGetLastError();
 }
