@@ -106,7 +106,7 @@ struct BParams {
   const float *dST;   // [B,H,dv,dk] or NULL
   float *dq, *dk, *dv, *dla, *dbeta, *derase, *dwrite, *dS0, *dA0;
   float *gen, *acc, *delta, *dd, *st, *part, *cpsi, *sigma, *dacc, *bsum, *phi;
-  // c dO in fp32, [BH][T][d_v] like delta and dd (written when dO is given)
+  // c dO in fp32, [BH][T][d_v] like delta and dd (zeros when dO is not given)
   float *cdo;
   // S before the first token of each kCk-token chunk (F1) and the cotangent
   // entering each chunk's last token (R1): [BH][nck][d_v][d_k]
@@ -388,9 +388,9 @@ __global__ void prep_gen_kernel(const BParams Q) {
         *reinterpret_cast<float4 *>(g + 3 * dk + c) = make_float4(a[0], a[1], a[2], a[3]);
       }
       if (av) *reinterpret_cast<float4 *>(g + 4 * dk + c) = make_float4(u[0], u[1], u[2], u[3]);
-      if (Q.dO && av) {  // c dO of the token, once, for the three sweeps that read it
+      if (av) {  // c dO of the token (zeros without dO), once, for the three sweeps that read it
         float o[4];
-        ld4_in<Tin>(Q.dO, tk * dv + c, o);
+        ld4_opt<Tin>(Q.dO, tk * dv + c, Q.dO != nullptr, o);
 #pragma unroll
         for (int e = 0; e < 4; ++e) o[e] *= P.q_scale;
         *reinterpret_cast<float4 *>(Q.cdo + ((size_t)bh * P.T + t) * dv + c) = make_float4(o[0], o[1], o[2], o[3]);
@@ -628,7 +628,7 @@ __device__ __forceinline__ void r1_body(const BParams &Q, int blk, float *sm) {
   const int jw = j0 + RW * warp, jl = lane / (32 / RW);
   const int c0 = C * lane;
   const bool cok = c0 < dk;
-  const int nd = Q.dO ? ND : 0;
+  constexpr int nd = ND;
   const int nc = (T + kLCR - 1) / kLCR;
   // This thread's 16-byte pieces of every staged token (up to two: 32 C + ND
   // <= 136 pieces for 128 threads), fixed for the whole sweep: q' | r | w |
@@ -700,7 +700,7 @@ __device__ __forceinline__ void r1_body(const BParams &Q, int blk, float *sm) {
 #pragma unroll
       for (int r = 0; r < RW; ++r) {
         // c dO of the row in slot r
-        const float cg = Q.dO ? slot[RW * warp + (r ^ jl)] : 0.f;
+        const float cg = slot[RW * warp + (r ^ jl)];
         float acc = 0.f;
 #pragma unroll
         for (int e = 0; e < C; ++e) {
@@ -820,7 +820,7 @@ __global__ void __launch_bounds__(128, 4) f2_kernel(const BParams Q) {
   const int tb = ck * kCk, te = min(T, tb + kCk);  // this CTA's tokens
   const int i = threadIdx.x;
   const int TS = 2 * dk + 3 * R;  // w | alpha | delta | dd | c dO
-  const int nv = dk / 2, nr = R / 4, nd = Q.dO ? nr : 0;
+  const int nv = dk / 2, nr = R / 4, nd = nr;
   const int nc = (te - tb + kLCC - 1) / kLCC;
   // this thread's pieces of every staged token (w | alpha, delta, dd, c dO)
   ColPiece pc[4];
@@ -872,11 +872,7 @@ __global__ void __launch_bounds__(128, 4) f2_kernel(const BParams Q) {
         float de[4], dd[4], go[4];
         ld4(sv + 2 * dk + j, true, de);
         ld4(sv + 2 * dk + R + j, true, dd);
-        if (Q.dO) {
-          ld4(sv + 2 * dk + 2 * R + j, true, go);
-        } else {
-          go[0] = go[1] = go[2] = go[3] = 0.f;
-        }
+        ld4(sv + 2 * dk + 2 * R + j, true, go);
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
           float2 &s2 = S[j / 2 + h];
@@ -910,7 +906,7 @@ __global__ void __launch_bounds__(128, 4) r2_kernel(const BParams Q) {
   const int tb = ck * kCk, te = min(T, tb + kCk);  // this CTA's tokens
   const int i = threadIdx.x;
   const int TS = 4 * dk + 3 * R;  // q' | r | w | alpha | delta | dd | c dO
-  const int nv = dk, nr = R / 4, nd = Q.dO ? nr : 0;
+  const int nv = dk, nr = R / 4, nd = nr;
   const int nc = (te - tb + kLCC - 1) / kLCC;
   // this thread's pieces of every staged token (q' | r | w | alpha, delta, dd, c dO)
   ColPiece pc[4];
@@ -962,11 +958,7 @@ __global__ void __launch_bounds__(128, 4) r2_kernel(const BParams Q) {
         float de[4], dd[4], go[4];
         ld4(sv + 4 * dk + j, true, de);
         ld4(sv + 4 * dk + R + j, true, dd);
-        if (Q.dO) {
-          ld4(sv + 4 * dk + 2 * R + j, true, go);
-        } else {
-          go[0] = go[1] = go[2] = go[3] = 0.f;
-        }
+        ld4(sv + 4 * dk + 2 * R + j, true, go);
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
           float2 &d2 = D[j / 2 + h];
