@@ -166,12 +166,16 @@ def test_backward_full_size_sampled(name, chains):
 
 
 @pytest.mark.parametrize("variant,dk,dv,B", [("PKDA", 128, 128, 5), ("GDN2", 64, 64, 10),
-                                            ("FG2_GDN_PLUS", 128, 128, 5), ("GDN2", 48, 80, 8)])
+                                            ("FG2_GDN_PLUS", 128, 128, 5), ("GDN2", 48, 80, 8),
+                                            ("PGDN", 32, 32, 10), ("PGDN", 32, 32, 6),
+                                            ("GDN2", 64, 32, 6)])
 def test_backward_many_chains_ragged(variant, dk, dv, B):
-    """Enough (batch, head) pairs for the row sweeps' widest layout (8 rows per
-    warp) and their unrolled chunk loop, with a token count that leaves a
-    ragged last chunk of 3 tokens (and, for d_v = 80, a partial group of
-    rows); sampled chains, the last one included."""
+    """Enough (batch, head) pairs for the row sweeps' unrolled chunk loop, in
+    each layout the dispatch picks: 8 rows per warp with 4, 2 and 1 key
+    channels per lane (B = 5, 10, 10 at d_k = 128, 64, 32) and 4 rows per
+    warp with 1 and 2 (B = 6 at d_v = 32). The token count leaves a ragged
+    last chunk of 3 tokens (and d_v = 80 a partial group of rows); sampled
+    chains, the last one included."""
     w = small(variant, "bf16", B=B, T=203, H=16, dk=dk, dv=dv)
     check_sampled_chains(w, [(0, 0), (w.B // 2, 7), (w.B - 1, w.H - 1)])
 
