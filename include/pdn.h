@@ -315,8 +315,11 @@ size_t pdn_chunk_bwd_workspace(const pdn_problem_t *p);
 /* Backward of pdn_chunk_fwd for problem p and forward inputs t (q, k, v,
  * log_alpha, beta, erase, write, S0, A0 as given to the forward; o, ST and
  * AT are not used and may be NULL). p->chunk and p->impl are validated as
- * for the forward but do not change the result; p->prologue must be 0 (PDN_ERR_UNSUPPORTED otherwise: the activations'
- * derivatives are the caller's). The gradients overwrite the buffers in g.
+ * for the forward but do not change the result. With a fused prologue
+ * (p->prologue, as for the forward) the inputs are the raw projections and
+ * the gradients are with respect to them: through the L2 normalisation of
+ * q and k, the sigmoid of the gains and gates, and the softplus or
+ * log-sigmoid of the decay. The gradients overwrite the buffers in g.
  * `workspace`: 256-byte aligned, at least pdn_chunk_bwd_workspace(p) bytes.
  * Returns PDN_OK once the work is enqueued on `stream`. */
 pdn_status_t pdn_chunk_bwd(const pdn_problem_t *p, const pdn_tensors_t *t, const pdn_grads_t *g,

@@ -172,7 +172,6 @@ pdn_status_t check_chunk_bwd(const pdn_problem_t *p, const pdn_tensors_t *t, con
   if (st != PDN_OK) return st;
   if ((st = check_tensors(p, t, false)) != PDN_OK) return st;
   if (!g) return PDN_ERR_INVALID_ARG;
-  if (p->prologue != 0) return PDN_ERR_UNSUPPORTED;
   const bool scalar_la = p->decay == PDN_DECAY_SCALAR;
   const bool scalar_beta = has_scalar_beta(p->variant);
   const void *v16[] = {g->dO, g->dST, g->dq, g->dk, g->dv, g->derase, g->dwrite, g->dS0, g->dA0,

@@ -240,28 +240,72 @@ __device__ __forceinline__ void ld4_opt(const void *p, size_t i, bool ok, float 
   }
 }
 
+// q and k as the recurrence uses them: under PDN_PRO_L2NORM_QK they arrive
+// raw and are divided by their norm over the head dimension (lane l holds
+// channels 4l..4l+3; every lane of the warp takes part). Returns the
+// inverse norm (1 without the prologue bit).
+__device__ __forceinline__ float l2norm_fwd(int prologue, float (&x)[4]) {
+  if (!(prologue & PDN_PRO_L2NORM_QK)) return 1.f;
+  float s = 0.f;
+#pragma unroll
+  for (int e = 0; e < 4; ++e) s = fmaf(x[e], x[e], s);
+  const float inv = inv_norm(warp_sum(s));
+#pragma unroll
+  for (int e = 0; e < 4; ++e) x[e] *= inv;
+  return inv;
+}
+
+// The gradient through y = x / max(||x||, 1e-12): dy (this lane's 4
+// channels) becomes dx = (dy - y (y . dy)) / ||x||, or dy / 1e-12 where the
+// floor applies. inv = 1 / max(||x||, 1e-12), y the normalised vector.
+__device__ __forceinline__ void l2norm_bwd(const float (&y)[4], float (&dy)[4], float inv) {
+  float s = 0.f;
+#pragma unroll
+  for (int e = 0; e < 4; ++e) s = fmaf(y[e], dy[e], s);
+  s = warp_sum(s);
+  const bool floored = !(inv < 1e12f);
+#pragma unroll
+  for (int e = 0; e < 4; ++e) dy[e] = (floored ? dy[e] : dy[e] - y[e] * s) * inv;
+}
+
+// d gate / d logit of a sigmoid gate g = sigmoid(x), from g.
+__device__ __forceinline__ float sigmoid_grad(float g) { return g * (1.f - g); }
+// Four gate or gain values as the recurrence uses them (sigmoid of logits
+// under PDN_PRO_SIGMOID_GATES).
+__device__ __forceinline__ void gate4(int prologue, float (&x)[4]) {
+  if (prologue & PDN_PRO_SIGMOID_GATES) {
+#pragma unroll
+    for (int e = 0; e < 4; ++e) x[e] = sigmoid_call(x[e]);
+  }
+}
+
 // Prep (preconditioned variants): the block totals of k_{t,i}^2 over each
 // kScanBlk-token block, into bsum[bh][block][i], for the carry pass; the
 // generic-vector pass then accumulates A_t = A_0 + sum_{s<=t} k_s^2 inside
-// each block in the same order as the sums here.
+// each block in the same order as the sums here. One warp per (head,
+// block), lane l on key channels 4l .. 4l + 3 (k normalised first under the
+// prologue, as in the generic-vector pass).
 template <typename Tin>
 __global__ void ksq_part_kernel(const BParams Q) {
   const KParams &P = Q.P;
-  const int dk = P.dk, nb = Q.nb;
-  const long long n = (long long)P.B * P.H * nb * dk;
-  for (long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x; e < n;
-       e += (long long)gridDim.x * blockDim.x) {
-    const int c = (int)(e % dk);
-    const long long r = e / dk;
-    const int blk = (int)(r % nb), bh = (int)(r / nb);
-    const int t0 = blk * kScanBlk, t1 = min(P.T, t0 + kScanBlk);
-    float s = 0.f;
-#pragma unroll 8
-    for (int t = t0; t < t1; ++t) {
-      const float k = ldf<Tin>(P.k, tok_index(P, bh / P.H, t, bh % P.H) * dk + c);
-      s += k * k;
+  const int lane = threadIdx.x & 31, dk = P.dk, c = 4 * lane;
+  const bool ak = c < dk;
+  const long long nblk = (long long)P.B * P.H * Q.nb;
+  const long long nw = ((long long)gridDim.x * blockDim.x) >> 5;
+  for (long long wid = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5; wid < nblk; wid += nw) {
+    const int bh = (int)(wid / Q.nb), blk = (int)(wid % Q.nb);
+    const int t_begin = blk * kScanBlk, t_end = min(P.T, t_begin + kScanBlk);
+    float s[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int t = t_begin; t < t_end; ++t) {
+      float k[4];
+      ld4_opt<Tin>(P.k, tok_index(P, bh / P.H, t, bh % P.H) * dk + c, ak, k);
+      l2norm_fwd(P.prologue, k);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) s[e] += k[e] * k[e];
     }
-    Q.bsum[e] = s;
+    if (ak)
+      *reinterpret_cast<float4 *>(Q.bsum + ((size_t)bh * Q.nb + blk) * dk + c) =
+          make_float4(s[0], s[1], s[2], s[3]);
   }
 }
 
@@ -294,6 +338,8 @@ __global__ void prep_gen_kernel(const BParams Q) {
       ld4_opt<Tin>(P.k, tk * dk + c, ak, k);
       ld4_opt<Tin>(P.q, tk * dk + c, ak, q);
       ld4_opt<Tin>(P.v, tk * dv + c, av, v);
+      l2norm_fwd(P.prologue, k);
+      l2norm_fwd(P.prologue, q);
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         Bc[e] = 1.f;
@@ -316,14 +362,15 @@ __global__ void prep_gen_kernel(const BParams Q) {
         for (int e = 0; e < 4; ++e) Bc[e] = precond_coef(L[e], mu, P.lnx);
       }
       if (P.decay == PDN_DECAY_SCALAR) {
-        const float ea = expf(reinterpret_cast<const float *>(P.log_alpha)[tk]);
+        const float ea = expf(decay_act(P.prologue, P.decay_scale,
+                                        reinterpret_cast<const float *>(P.log_alpha)[tk]));
 #pragma unroll
         for (int e = 0; e < 4; ++e) a[e] = ea;
       } else if (P.decay == PDN_DECAY_CHANNEL) {
         float la[4];
         ld4_opt<Tin>(P.log_alpha, tk * dk + c, ak, la);
 #pragma unroll
-        for (int e = 0; e < 4; ++e) a[e] = ak ? expf(la[e]) : 1.f;
+        for (int e = 0; e < 4; ++e) a[e] = ak ? expf(decay_act(P.prologue, P.decay_scale, la[e])) : 1.f;
       }
       float r[4], w[4], u[4], qq[4];
 #pragma unroll
@@ -335,17 +382,17 @@ __global__ void prep_gen_kernel(const BParams Q) {
       }
       switch (P.variant) {
         case PDN_VAR_DN: case PDN_VAR_GDN: case PDN_VAR_KDA: {
-          const float be = reinterpret_cast<const float *>(P.beta)[tk];
+          const float be = gate_act(P.prologue, reinterpret_cast<const float *>(P.beta)[tk]);
 #pragma unroll
           for (int e = 0; e < 4; ++e) w[e] = be * k[e];
         } break;
         case PDN_VAR_PDN: case PDN_VAR_PGDN: case PDN_VAR_PKDA: {
-          const float be = reinterpret_cast<const float *>(P.beta)[tk];
+          const float be = gate_act(P.prologue, reinterpret_cast<const float *>(P.beta)[tk]);
 #pragma unroll
           for (int e = 0; e < 4; ++e) w[e] = be * Bc[e] * k[e];
         } break;
         case PDN_VAR_PLA: {
-          const float be = reinterpret_cast<const float *>(P.beta)[tk];
+          const float be = gate_act(P.prologue, reinterpret_cast<const float *>(P.beta)[tk]);
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             r[e] = 0.f;
@@ -357,7 +404,11 @@ __global__ void prep_gen_kernel(const BParams Q) {
           const bool plus = P.variant == PDN_VAR_FG2_GDN_PLUS;
           float bk[4], bv[4];
           ld4_opt<Tin>(P.beta, tk * dk + c, ak, bk);
-          if (plus) ld4_opt<Tin>(P.write, tk * dv + c, av, bv);
+          gate4(P.prologue, bk);
+          if (plus) {
+            ld4_opt<Tin>(P.write, tk * dv + c, av, bv);
+            gate4(P.prologue, bv);
+          }
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const float sb = ak ? sqrtf(bk[e]) : 0.f;
@@ -372,6 +423,8 @@ __global__ void prep_gen_kernel(const BParams Q) {
           float er[4], gw[4];
           ld4_opt<Tin>(P.erase, tk * dk + c, ak, er);
           ld4_opt<Tin>(P.write, tk * dv + c, av, gw);
+          gate4(P.prologue, er);
+          gate4(P.prologue, gw);
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             r[e] = er[e] * k[e];
@@ -1020,6 +1073,14 @@ __global__ void __launch_bounds__(256, 4) e1_kernel(const BParams Q) {
     ld4(Q.dd + ((size_t)bh * T + t) * dv + c, av, du);
     ld4_opt<Tin>(P.k, tk * dk + c, ak, k);
     ld4_opt<Tin>(P.v, tk * dv + c, av, v);
+    // q and k as the recurrence used them (normalised under the prologue)
+    const bool l2 = P.prologue & PDN_PRO_L2NORM_QK;
+    float qn[4] = {0.f, 0.f, 0.f, 0.f}, iq = 1.f;
+    const float ik = l2norm_fwd(P.prologue, k);
+    if (l2 || P.variant == PDN_VAR_PLA) {
+      ld4_opt<Tin>(P.q, tk * dk + c, ak, qn);
+      iq = l2norm_fwd(P.prologue, qn);
+    }
     // decay: this token's term q'.dq' - w.dw + r.dr
     if (P.decay != PDN_DECAY_NONE) {
       float cp[4], s = 0.f;
@@ -1063,7 +1124,7 @@ __global__ void __launch_bounds__(256, 4) e1_kernel(const BParams Q) {
     switch (P.variant) {
       case PDN_VAR_DN: case PDN_VAR_GDN: case PDN_VAR_KDA:
       case PDN_VAR_PDN: case PDN_VAR_PGDN: case PDN_VAR_PKDA: {
-        const float be = reinterpret_cast<const float *>(P.beta)[tk];
+        const float be = gate_act(P.prologue, reinterpret_cast<const float *>(P.beta)[tk]);
         float db = 0.f;
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
@@ -1072,21 +1133,21 @@ __global__ void __launch_bounds__(256, 4) e1_kernel(const BParams Q) {
           dB[e] = be * k[e] * dw[e];
         }
         db = warp_sum(db);
+        if (P.prologue & PDN_PRO_SIGMOID_GATES) db *= sigmoid_grad(be);
         if (lane == 0 && Q.dbeta) Q.dbeta[tk] = db;
       } break;
       case PDN_VAR_PLA: {
-        const float be = reinterpret_cast<const float *>(P.beta)[tk];
-        float db = 0.f, qv[4];
-        ld4_opt<Tin>(P.q, tk * dk + c, ak, qv);
+        const float be = gate_act(P.prologue, reinterpret_cast<const float *>(P.beta)[tk]);
+        float db = 0.f;
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const float q = qv[e];
           gk[e] = be * dw[e];
           db = fmaf(k[e], dw[e], db);
-          dB[e] = q * dq[e];
+          dB[e] = qn[e] * dq[e];
           gq[e] = Bc[e] * dq[e];
         }
         db = warp_sum(db);
+        if (P.prologue & PDN_PRO_SIGMOID_GATES) db *= sigmoid_grad(be);
         if (lane == 0 && Q.dbeta) Q.dbeta[tk] = db;
       } break;
       case PDN_VAR_FG2_GDN: case PDN_VAR_FG2_GDN_PLUS: {
@@ -1094,6 +1155,13 @@ __global__ void __launch_bounds__(256, 4) e1_kernel(const BParams Q) {
         float dbk[4], dwr[4], bkv[4], bvv[4];
         ld4_opt<Tin>(P.beta, tk * dk + c, ak, bkv, 1.f);
         if (plus) ld4_opt<Tin>(P.write, tk * dv + c, av, bvv, 1.f);
+        if (P.prologue & PDN_PRO_SIGMOID_GATES) {  // gains as used, sigmoid of the logits (lanes in range)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            if (ak) bkv[e] = sigmoid_call(bkv[e]);
+            if (plus && av) bvv[e] = sigmoid_call(bvv[e]);
+          }
+        }
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const float bk = bkv[e];
@@ -1105,6 +1173,10 @@ __global__ void __launch_bounds__(256, 4) e1_kernel(const BParams Q) {
           gvv[e] = sv * du[e];
           dwr[e] = v[e] * du[e] / (2.f * sv);
           if (!plus) dbk[e] += dwr[e];
+          if (P.prologue & PDN_PRO_SIGMOID_GATES) {  // back to the logits
+            dbk[e] *= sigmoid_grad(bk);
+            if (plus) dwr[e] *= sigmoid_grad(bv);
+          }
         }
         if (Q.dbeta && ak)
           *reinterpret_cast<float4 *>(Q.dbeta + tk * dk + c) = make_float4(dbk[0], dbk[1], dbk[2], dbk[3]);
@@ -1115,6 +1187,8 @@ __global__ void __launch_bounds__(256, 4) e1_kernel(const BParams Q) {
         float de[4], dg[4], erv[4], gwv[4];
         ld4_opt<Tin>(P.erase, tk * dk + c, ak, erv);
         ld4_opt<Tin>(P.write, tk * dv + c, av, gwv);
+        gate4(P.prologue, erv);
+        gate4(P.prologue, gwv);
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const float er = erv[e];
@@ -1123,6 +1197,10 @@ __global__ void __launch_bounds__(256, 4) e1_kernel(const BParams Q) {
           de[e] = k[e] * dr[e];
           gvv[e] = gw * du[e];
           dg[e] = v[e] * du[e];
+          if (P.prologue & PDN_PRO_SIGMOID_GATES) {  // back to the logits
+            de[e] *= sigmoid_grad(er);
+            dg[e] *= sigmoid_grad(gw);
+          }
         }
         if (Q.derase && ak)
           *reinterpret_cast<float4 *>(Q.derase + tk * dk + c) = make_float4(de[0], de[1], de[2], de[3]);
@@ -1150,6 +1228,12 @@ __global__ void __launch_bounds__(256, 4) e1_kernel(const BParams Q) {
             make_float4(da[0], da[1], da[2], da[3]);
       }
     }
+    // back through the normalisation of q, and of k unless the
+    // preconditioner's term is still to come (then E3 does it)
+    if (l2) {
+      l2norm_bwd(qn, gq, iq);
+      if (!pre) l2norm_bwd(k, gk, ik);
+    }
     if (Q.dq && ak) *reinterpret_cast<float4 *>(Q.dq + tk * dk + c) = make_float4(gq[0], gq[1], gq[2], gq[3]);
     if (Q.dk && ak) *reinterpret_cast<float4 *>(Q.dk + tk * dk + c) = make_float4(gk[0], gk[1], gk[2], gk[3]);
     if (Q.dv && av)
@@ -1160,31 +1244,52 @@ __global__ void __launch_bounds__(256, 4) e1_kernel(const BParams Q) {
 // E3 (preconditioned variants): k_t feeds A_s for every s >= t, so
 // dk_t += 2 k_t . (sum_{s>=t} dA_s). One warp per (head, kScanBlk-token
 // block) walks its tokens from the last, the suffix sum starting from the
-// block's carry (the sum over all later blocks, in bsum).
+// block's carry (the sum over all later blocks, in bsum). Under the L2
+// prologue the whole gradient of the normalised k is then taken back
+// through the normalisation here.
 template <typename Tin>
 __global__ void e3_kernel(const BParams Q) {
   const KParams &P = Q.P;
   const int lane = threadIdx.x & 31, dk = P.dk, c = 4 * lane;
+  const bool ak = c < dk;
   const long long nblk = (long long)P.B * P.H * Q.nb;
   const long long nw = ((long long)gridDim.x * blockDim.x) >> 5;
-  if (c >= dk) return;
   for (long long wid = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5; wid < nblk; wid += nw) {
     const int bh = (int)(wid / Q.nb), blk = (int)(wid % Q.nb);
     const int t_begin = blk * kScanBlk, t_end = min(P.T, t_begin + kScanBlk);
-    float4 y = *reinterpret_cast<const float4 *>(Q.bsum + ((size_t)bh * Q.nb + blk) * dk + c);
+    float y[4];
+    ld4(Q.bsum + ((size_t)bh * Q.nb + blk) * dk + c, ak, y);
     for (int t = t_end - 1; t >= t_begin; --t) {
       const size_t o = tok_index(P, bh / P.H, t, bh % P.H) * dk + c;
-      float k[4];
-      ld4_in<Tin>(P.k, o, k);
-      const float4 da = *reinterpret_cast<const float4 *>(Q.dacc + ((size_t)bh * P.T + t) * dk + c);
-      y.x += da.x; y.y += da.y; y.z += da.z; y.w += da.w;
-      float4 g = *reinterpret_cast<const float4 *>(Q.dk + o);
-      g.x += 2.f * k[0] * y.x;
-      g.y += 2.f * k[1] * y.y;
-      g.z += 2.f * k[2] * y.z;
-      g.w += 2.f * k[3] * y.w;
-      *reinterpret_cast<float4 *>(Q.dk + o) = g;
+      float k[4], da[4], g[4];
+      ld4_opt<Tin>(P.k, o, ak, k);
+      const float ik = l2norm_fwd(P.prologue, k);
+      ld4(Q.dacc + ((size_t)bh * P.T + t) * dk + c, ak, da);
+      ld4(Q.dk + o, ak, g);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        y[e] += da[e];
+        g[e] += 2.f * k[e] * y[e];
+      }
+      if (P.prologue & PDN_PRO_L2NORM_QK) l2norm_bwd(k, g, ik);
+      if (ak) *reinterpret_cast<float4 *>(Q.dk + o) = make_float4(g[0], g[1], g[2], g[3]);
     }
+  }
+}
+
+// dlog_alpha with respect to the raw decay input x under the decay prologue:
+// log alpha = -s softplus(x) gives -s sigmoid(x); log alpha = log sigmoid(x)
+// gives sigmoid(-x). Same layout as the input ([B,T,H] or [B,T,H,d_k]).
+template <typename Tin>
+__global__ void decay_pro_kernel(const BParams Q, long long n) {
+  const KParams &P = Q.P;
+  const bool ch = P.decay == PDN_DECAY_CHANNEL;
+  for (long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x; e < n;
+       e += (long long)gridDim.x * blockDim.x) {
+    const float x = ch ? ldf<Tin>(P.log_alpha, (size_t)e) : reinterpret_cast<const float *>(P.log_alpha)[e];
+    const float d = (P.prologue & PDN_PRO_DECAY_SOFTPLUS) ? -P.decay_scale / (1.f + expf(-x))
+                                                          : 1.f / (1.f + expf(x));
+    Q.dla[e] *= d;
   }
 }
 
@@ -1267,7 +1372,7 @@ cudaError_t launch_bwd_t(const BParams &Q, cudaStream_t st) {
   const long long BH = (long long)P.B * P.H, BHT = BH * P.T;
   cudaError_t err;
   if (is_precond(P.variant)) {
-    ksq_part_kernel<Tin><<<grid_for(BH * Q.nb * dk, 256), 256, 0, st>>>(Q);
+    ksq_part_kernel<Tin><<<grid_for(BH * Q.nb * 32, 256), 256, 0, st>>>(Q);
     scan_carry_kernel<<<grid_for(BH * dk, 128), 128, 0, st>>>(P, dk, Q.nb, false, Q.bsum, P.A0,
                                                              nullptr);
   }
@@ -1290,7 +1395,10 @@ cudaError_t launch_bwd_t(const BParams &Q, cudaStream_t st) {
                Q.dST ? Q.phi : nullptr, nullptr, Q.bsum, st);
     else
       run_scan(P, ScanArr{Q.sigma, false}, ScanArr{Q.dla, true}, 1, Q.nb, true,
-               Q.dST ? Q.phi + BH * dk : nullptr, nullptr, Q.bsum, st);
+               Q.dST ? Q.phi + BH * dk : nullptr, nullptr, Q.bsum, st);    if (P.prologue & (PDN_PRO_DECAY_SOFTPLUS | PDN_PRO_DECAY_LOGSIGMOID)) {
+      const long long n = BHT * (P.decay == PDN_DECAY_CHANNEL ? dk : 1);
+      decay_pro_kernel<Tin><<<grid_for(n, 256), 256, 0, st>>>(Q, n);
+    }
   }
   if (is_precond(P.variant) && (Q.dk || Q.dA0)) {
     // block totals of dA and the carries from the sequence end (dA0 gets

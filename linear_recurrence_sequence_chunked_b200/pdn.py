@@ -299,17 +299,19 @@ def make_grads(dO=None, dST=None, dq=None, dk=None, dv=None, dlog_alpha=None, db
 
 def chunk_bwd(variant: str, q, k, v, dO=None, dST=None, log_alpha=None, beta=None, erase=None,
               write=None, S0=None, A0=None, q_scale: float = 1.0, precond_x: float = 1.5,
-              precond_eps: float = 1e-6, workspace=None):
+              precond_eps: float = 1e-6, workspace=None, prologue: int = 0,
+              decay_scale: float = 1.0):
     """Gradients of chunk_fwd's (o, S_T) with respect to its inputs, given the
     cotangents dO [B,T,H,d_v] (input dtype) and dST [B,H,d_v,d_k] (fp32);
     either may be None (zero). Returns a dict of fp32 tensors with keys q, k,
     v, log_alpha, beta, erase, write, S0, A0 (None where the variant has no
-    such input)."""
+    such input). With ``prologue`` bits the inputs are raw projections and the
+    gradients are with respect to them."""
     B, T, H, d_k = k.shape
     d_v = v.shape[3]
     dev = k.device
     p = make_problem(variant, B, T, H, d_k, d_v, k.dtype, _decay_of(log_alpha), 64, "auto",
-                     q_scale, precond_x, precond_eps)
+                     q_scale, precond_x, precond_eps, prologue, decay_scale)
     f32 = dict(dtype=torch.float32, device=dev)
     g = {"q": torch.empty(B, T, H, d_k, **f32), "k": torch.empty(B, T, H, d_k, **f32),
          "v": torch.empty(B, T, H, d_v, **f32),

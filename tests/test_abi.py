@@ -316,9 +316,11 @@ def test_backward_rules(lib):
                              None) == pdn.PDN_ERR_WORKSPACE
     assert pdn.pdn_chunk_bwd(p, _tensors(o=None), _grads(), FAKE + 128, ws_need,
                              None) == pdn.PDN_ERR_WORKSPACE
-    # a fused prologue is the forward's alone
-    assert pdn.pdn_chunk_bwd(_problem(prologue=1), _tensors(), _grads(), FAKE, ws_need,
-                             None) == pdn.PDN_ERR_UNSUPPORTED
+    # prologue bits are checked as for the forward: unknown bits, both decay
+    # maps, a softplus decay without a positive scale
+    for bad in (dict(prologue=16), dict(prologue=4 | 8), dict(prologue=4, decay_scale=0.0)):
+        assert pdn.pdn_chunk_bwd(_problem(**bad), _tensors(), _grads(), FAKE, ws_need,
+                                 None) == pdn.PDN_ERR_INVALID_ARG, bad
     # T == 0 needs no workspace
     assert pdn.pdn_chunk_bwd_workspace(_problem(T=0)) == 0
     # the gradient struct itself is required

@@ -11,8 +11,10 @@ import pytest
 import torch
 
 import oracle
+from oracle import prologue as oracle_prologue
 from linear_recurrence_sequence_chunked_b200 import pdn
 from linear_recurrence_sequence_chunked_b200.workloads import (WORKLOADS, Workload, make_inputs,
+                                                               make_raw_inputs, raw_prologue,
                                                                slice_chain)
 
 from parity_util import REPORT, elem_rel_err, nmax_err
@@ -222,3 +224,60 @@ def test_backward_is_deterministic():
     for n in a:
         if a[n] is not None:
             assert np.array_equal(a[n], b[n]), n
+
+
+@pytest.mark.parametrize("variant,recipe,dtype,dk", [("PGDN", "softplus", "bf16", 64),
+                                                    ("GDN2", "sigmoid", "bf16", 64),
+                                                    ("FG2_GDN_PLUS", "softplus", "f32", 32),
+                                                    ("PKDA", "sigmoid", "f32", 32),
+                                                    ("PLA", "softplus", "bf16", 32),
+                                                    ("FG2_GDN", "sigmoid", "bf16", 32)])
+def test_backward_prologue_finite_differences(variant, recipe, dtype, dk):
+    """With the fused prologue (raw projections in: L2 normalisation of q and
+    k, sigmoid gains and gates, softplus or log-sigmoid decay) the gradients
+    are with respect to the raw inputs. Checked element by element against
+    central differences of L = sum(dO . o) + sum(dST . S_T), with o and S_T
+    from the fp64 oracle on the activated inputs, at sampled elements of every
+    input tensor."""
+    w = Workload("bwdpro-%s" % variant, variant, 1, 37, 2, dk, dk, dtype, DECAY[variant],
+                 decay_recipe=recipe, seed=3)
+    raw = make_raw_inputs(w)
+    bits, dscale = raw_prologue(w)
+    dO, dST = cotangents(w)
+    dev = torch.device("cuda")
+    d = {n: (t.to(dev) if t is not None else None) for n, t in raw.items()}
+    g = pdn.chunk_bwd(w.variant, d["q"], d["k"], d["v"], dO=dO.to(dev), dST=dST.to(dev),
+                      log_alpha=d["log_alpha"], beta=d["beta"], erase=d["erase"],
+                      write=d["write"], q_scale=w.q_scale, precond_x=w.precond_x,
+                      precond_eps=w.precond_eps, prologue=bits, decay_scale=dscale)
+    torch.cuda.synchronize()
+    assert pdn.device_error() == pdn.PDN_OK
+    base = {n: (t.double().numpy() if t is not None else None) for n, t in raw.items()}
+    dO64, dST64 = dO.double().numpy(), dST.double().numpy()
+
+    def loss(x):
+        a = oracle_prologue.apply(x, bits, dscale)
+        o, ST, _ = oracle.forward(w.variant, a["q"], a["k"], a["v"], log_alpha=a["log_alpha"],
+                                  beta=a["beta"], erase=a["erase"], write=a["write"],
+                                  q_scale=w.q_scale, x=w.precond_x, eps=w.precond_eps)
+        return float((o * dO64).sum() + (ST * dST64).sum())
+
+    rng = np.random.default_rng(1)
+    bad = []
+    for name in ("q", "k", "v", "log_alpha", "beta", "erase", "write"):
+        if base[name] is None:
+            assert g[name] is None, name
+            continue
+        G = g[name].cpu().numpy()
+        gmax = float(np.abs(G).max())
+        for _ in range(4):
+            idx = tuple(int(rng.integers(0, n)) for n in base[name].shape)
+            h = 1e-5 * max(1.0, abs(base[name][idx]))
+            xp, xm = dict(base), dict(base)
+            xp[name], xm[name] = base[name].copy(), base[name].copy()
+            xp[name][idx] += h
+            xm[name][idx] -= h
+            fd = (loss(xp) - loss(xm)) / (2 * h)
+            if not abs(G[idx] - fd) <= 2e-3 * gmax + 1e-6:
+                bad.append((name, idx, float(G[idx]), fd, gmax))
+    assert not bad, bad
