@@ -21,6 +21,8 @@ timed steps. The JSON line also carries:
   backward    the gradient of the headline layer (pdn_chunk_bwd, every
               input's gradient from dO and dS_T): tokens/s and its fraction
               of the fp32 CUDA-core peak (an ALU-bound pass);
+  backward_prologue  the same from the layer's raw projections (gradients
+              through the fused prologue's activations);
   cpu_baseline the fp64 oracle on the host cores on a bounded sample.
 Multi-GPU (torchrun): every rank runs its own independent batch (weak
 scaling, no collective on the data path); the time is the max over ranks.
@@ -399,7 +401,10 @@ def run_ours(args):
     if not args.no_backward:
         torch.cuda.empty_cache()
         result["backward"] = bench_backward(args, w, dev, stream, rank, mor, barrier)
-        result["gpu_launches"] += result["backward"]["gpu_launches"]
+        result["backward_prologue"] = bench_backward(args, w, dev, stream, rank, mor, barrier,
+                                                     raw=True)
+        result["gpu_launches"] += (result["backward"]["gpu_launches"]
+                                   + result["backward_prologue"]["gpu_launches"])
         torch.cuda.empty_cache()
 
     # ---------------- decode workload
@@ -517,21 +522,28 @@ def bwd_flops_per_token_head(dk, dv):
     return 26 * dk * dv
 
 
-def bench_backward(args, w, dev, stream, rank, mor, barrier):
+def bench_backward(args, w, dev, stream, rank, mor, barrier, raw=False):
     """Times `args.steps` pdn_chunk_bwd calls of the headline layer (inputs and
-    cotangents resident in HBM, larger than L2), after warm-up."""
+    cotangents resident in HBM, larger than L2), after warm-up; with `raw`,
+    from the raw projections through the fused prologue."""
     import torch
 
     from linear_recurrence_sequence_chunked_b200 import pdn
-    from linear_recurrence_sequence_chunked_b200.workloads import make_inputs
+    from linear_recurrence_sequence_chunked_b200.workloads import (make_inputs, make_raw_inputs,
+                                                                   raw_prologue)
 
     wr = w.replace(seed=rank_seed(w.seed, rank))
-    x = make_inputs(wr, device=dev, generator_device=dev)
+    if raw:
+        x = make_raw_inputs(wr, device=dev, generator_device=dev)
+        bits, dscale = raw_prologue(w)
+    else:
+        x = make_inputs(wr, device=dev, generator_device=dev)
+        bits, dscale = 0, 1.0
     gen = torch.Generator(device=dev).manual_seed(rank_seed(7, rank))
     dO = torch.randn(w.B, w.T, w.H, w.dv, generator=gen, device=dev).to(x["v"].dtype)
     dST = torch.randn(w.B, w.H, w.dv, w.dk, generator=gen, device=dev)
     prob = pdn.make_problem(w.variant, w.B, w.T, w.H, w.dk, w.dv, x["k"].dtype, w.decay, w.chunk,
-                            "auto", w.q_scale, w.precond_x, w.precond_eps)
+                            "auto", w.q_scale, w.precond_x, w.precond_eps, bits, dscale)
     f32 = dict(dtype=torch.float32, device=dev)
     g = {n: torch.empty_like(x[n], **f32) for n in ("q", "k", "v")}
     g["log_alpha"] = torch.empty_like(x["log_alpha"], **f32)
@@ -564,10 +576,12 @@ def bench_backward(args, w, dev, stream, rank, mor, barrier):
         raise SystemExit("device error during the backward timed region")
     per = ms_local / args.steps
     flops = bwd_flops_per_token_head(w.dk, w.dv) * w.B * w.T * w.H
-    # generic vectors, four sweeps, epilogue; then the preconditioner's prefix
-    # (squares + 3 scan passes) and suffix (3 scan passes + dk update) and the
-    # decay's final-state term + suffix sum
-    launches = 1 + 4 + 1 + (1 + 3 + 3 + 1) + (1 + 3)
+    # preconditioner prefix (block totals of k.k, carries), generic vectors,
+    # the row sweeps (one launch), F2, R2, the chain rules; the decay's
+    # final-state term and suffix sum (3 scan passes; the decay map's
+    # derivative under the prologue); the preconditioner's suffix (block
+    # totals, carries, dk update)
+    launches = 2 + 1 + 1 + 2 + 1 + (1 + 3 + (1 if bits else 0)) + 3
     res = {"workload": w.name, "variant": w.variant, "value": w.B * w.T * args.steps / (ms / 1e3),
            "unit": "tokens/s", "ms_per_step": ms / args.steps,
            "roofline": {"bound": "alu", "achieved": flops / (per / 1e3) / 1e12,
@@ -575,7 +589,8 @@ def bench_backward(args, w, dev, stream, rank, mor, barrier):
                         "frac": flops / (per / 1e3) / 1e12 / FP32_ALU_TFLOPS,
                         "flops_per_launch": flops,
                         "peak_kind": "fp32 CUDA-core peak from unit counts x 1965 MHz"},
-           "gradients": "q, k, v, log_alpha, beta, S0, A0 (fp32) from dO and dS_T",
+           "gradients": ("q, k, v, log_alpha, beta, S0, A0 (fp32) from dO and dS_T"
+                         + (", with respect to the raw projections (fused prologue)" if raw else "")),
            "l2": "inputs larger than L2 (no flush)",
            "gpu_launches": args.steps * launches}
     del x, dO, dST, g, ws, grads, tens
