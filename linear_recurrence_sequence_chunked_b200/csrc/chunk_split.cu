@@ -65,65 +65,58 @@ constexpr float kLn2 = 0.6931471805599453f;
 // One CTA per (batch, head, chunk): thread (8-channel group, token lane)
 // loads 16-byte rows and squares them; the 16 token lanes are summed in
 // shared memory.
-__global__ void __launch_bounds__(256, 4) k0_chunk_energy(const KParams P, void *ws, int N) {
+__global__ void __launch_bounds__(256) k0_chunk_energy(const KParams P, void *ws, int N) {
   __shared__ float part[16][kD + 4];
   const int tid = threadIdx.x, c8 = tid & 15, tl = tid >> 4;
-  const int BH = P.B * P.H, total = N * BH;
+  const int BH = P.B * P.H;
+  const long long total = (long long)N * BH;
+  // chunk blocks in the workspace's chunk-major order; one per CTA up to the
+  // grid cap, so each CTA keeps only one block's rows in flight and more
+  // CTAs fit per SM
+  for (long long it = blockIdx.x; it < total; it += gridDim.x) {
+  const int c = (int)(it / BH), bh = (int)(it % BH);
+  const int c0 = c * kC, Cn = min(kC, P.T - c0);
   const size_t tstride = (size_t)P.H * kD;
-  // The k rows of chunk block `it` (chunk-major, like the workspace): thread
-  // (c8, tl) takes 8 channels of tokens tl, tl + 16, tl + 32, tl + 48.
-  auto load = [&](int it, uint4 (&r)[4]) {
-    const int c = it / BH, bh = it % BH;
-    const int c0 = c * kC, Cn = min(kC, P.T - c0);
-    const __nv_bfloat16 *kp = reinterpret_cast<const __nv_bfloat16 *>(P.k) +
-                              tok_index(P, bh / P.H, c0, bh % P.H) * kD + c8 * 8;
+  const __nv_bfloat16 *kp = reinterpret_cast<const __nv_bfloat16 *>(P.k) +
+                            tok_index(P, bh / P.H, c0, bh % P.H) * kD + c8 * 8;
+  // thread (c8, tl): 8 channels of tokens tl, tl + 16, tl + 32, tl + 48
+  uint4 r[4];
 #pragma unroll
-    for (int m = 0; m < 4; ++m) {
-      const int t = tl + 16 * m;
-      r[m] = t < Cn ? __ldg(reinterpret_cast<const uint4 *>(kp + t * tstride))
-                    : make_uint4(0u, 0u, 0u, 0u);
-    }
-  };
-  // grid-stride over the blocks, the next block's rows in flight while the
-  // current one is reduced
-  uint4 cur[4];
-  if ((int)blockIdx.x < total) load(blockIdx.x, cur);
-  for (int it = blockIdx.x; it < total; it += gridDim.x) {
-    uint4 nxt[4];
-    if (it + (int)gridDim.x < total) load(it + gridDim.x, nxt);
-    float acc[8];
+  for (int m = 0; m < 4; ++m) {
+    const int t = tl + 16 * m;
+    r[m] = t < Cn ? __ldg(reinterpret_cast<const uint4 *>(kp + t * tstride)) : make_uint4(0u, 0u, 0u, 0u);
+  }
+  float acc[8];
 #pragma unroll
-    for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+  for (int e = 0; e < 8; ++e) acc[e] = 0.f;
 #pragma unroll
-    for (int m = 0; m < 4; ++m) {
-      float kf[8];
-      unpack8(cur[m], kf);
-      if (P.prologue & PDN_PRO_L2NORM_QK) {
-        // the token's 128 channels sit in the 16 lanes of this half-warp
-        float ss = 0.f;
+  for (int m = 0; m < 4; ++m) {
+    float kf[8];
+    unpack8(r[m], kf);
+    if (P.prologue & PDN_PRO_L2NORM_QK) {
+      // the token's 128 channels sit in the 16 lanes of this half-warp
+      float ss = 0.f;
 #pragma unroll
-        for (int e = 0; e < 8; ++e) ss = fmaf(kf[e], kf[e], ss);
+      for (int e = 0; e < 8; ++e) ss = fmaf(kf[e], kf[e], ss);
 #pragma unroll
-        for (int o = 1; o < 16; o <<= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-        const float inv = inv_norm(ss);
+      for (int o = 1; o < 16; o <<= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+      const float inv = inv_norm(ss);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) kf[e] *= inv;
-      }
-#pragma unroll
-      for (int e = 0; e < 8; ++e) acc[e] = fmaf(kf[e], kf[e], acc[e]);
+      for (int e = 0; e < 8; ++e) kf[e] *= inv;
     }
 #pragma unroll
-    for (int e = 0; e < 8; ++e) part[tl][c8 * 8 + e] = acc[e];
-    __syncthreads();
-    if (tid < kD) {
-      float sum = 0.f;
+    for (int e = 0; e < 8; ++e) acc[e] = fmaf(kf[e], kf[e], acc[e]);
+  }
 #pragma unroll
-      for (int r = 0; r < 16; ++r) sum += part[r][tid];
-      reinterpret_cast<float *>(ws_block(ws, it % BH, BH, it / BH) + WS_A)[tid] = sum;
-    }
-    __syncthreads();  // part is rewritten by the next block
+  for (int e = 0; e < 8; ++e) part[tl][c8 * 8 + e] = acc[e];
+  __syncthreads();
+  if (tid < kD) {
+    float sum = 0.f;
 #pragma unroll
-    for (int m = 0; m < 4; ++m) cur[m] = nxt[m];
+    for (int q = 0; q < 16; ++q) sum += part[q][tid];
+    reinterpret_cast<float *>(ws_block(ws, bh, BH, c) + WS_A)[tid] = sum;
+  }
+  __syncthreads();  // part is rewritten by the next block
   }
 }
 
@@ -1644,15 +1637,8 @@ cudaError_t launch_chunk_split(const KParams &P, void *ws, cudaStream_t stream,
   cudaError_t e;
   if (ev && (e = cudaEventRecord(ev[0], stream)) != cudaSuccess) return e;
   if (is_precond(P.variant)) {
-    int dev = 0, sms = 148, per_sm = 1;
-    if (cudaGetDevice(&dev) == cudaSuccess)
-      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k0_chunk_energy, 256, 0) !=
-            cudaSuccess || per_sm < 1)
-      per_sm = 1;
     const long long blocks = (long long)N * BH;
-    const long long grid0 = blocks < (long long)sms * per_sm ? blocks : (long long)sms * per_sm;
-    k0_chunk_energy<<<(unsigned)grid0, 256, 0, stream>>>(P, ws, N);
+    k0_chunk_energy<<<(unsigned)(blocks < (1LL << 30) ? blocks : (1LL << 30)), 256, 0, stream>>>(P, ws, N);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     k0_prefix<<<BH, kD * kK0Groups, 0, stream>>>(P, ws, N);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
