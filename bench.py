@@ -8,7 +8,8 @@ resident in HBM before the timed region; L2 is flushed (256 MiB write) between
 timed steps. The JSON line also carries:
   e2e         the same metric end to end through pdn_chunk_fwd_host from
               pinned HOST buffers (host->device inputs and device->host
-              output per step, overlapped with the compute over batch slices);
+              output, final state and accumulator per step, overlapped with
+              the compute over batch slices);
   roofline    one pdn_chunk_fwd call (its kernels timed as one launch by the
               CUDA events around it) against the measured bf16 tensor peak;
   decode      the recurrent decode workload (256 sequences x 16 heads,
@@ -351,14 +352,18 @@ def run_ours(args):
     if not args.no_e2e:
         hx = {n: (t.cpu().pin_memory() if t is not None else None) for n, t in x.items()}
         ho = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+        # the final state (and accumulator) come back too: what a caller
+        # continuing the sequence needs
+        hST = torch.empty(ST.shape, dtype=ST.dtype).pin_memory()
+        hAT = torch.empty(AT.shape, dtype=AT.dtype).pin_memory() if AT is not None else None
         dx = {n: (torch.empty_like(t, device=dev) if t is not None else None) for n, t in hx.items()}
         dtens = pdn.make_tensors(dx["q"], dx["k"], dx["v"], o, dx["log_alpha"], dx["beta"],
                                  dx["erase"], dx["write"], ST=ST, AT=AT)
         h2d = sum(t.numel() * t.element_size() for t in hx.values() if t is not None)
-        d2h = ho.numel() * ho.element_size()
+        d2h = sum(t.numel() * t.element_size() for t in (ho, hST, hAT) if t is not None)
 
         htens = pdn.make_host_tensors(hx["q"], hx["k"], hx["v"], ho, hx["log_alpha"],
-                                      hx["beta"], hx["erase"], hx["write"])
+                                      hx["beta"], hx["erase"], hx["write"], ST=hST, AT=hAT)
         slices = w.B  # one batch element per part: copy in / compute / copy out overlap
 
         def e2e_step():
@@ -382,7 +387,7 @@ def run_ours(args):
                          "ms_per_step": ems / args.steps,
                          "path": "pdn_chunk_fwd_host, %d batch slices" % slices}
         result["gpu_launches"] += args.steps * launches_per_step * slices
-        del hx, ho, dx
+        del hx, ho, hST, hAT, dx
 
     # ---------------- the other forward workloads
     if not args.no_extra:
