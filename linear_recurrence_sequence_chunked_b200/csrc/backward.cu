@@ -12,8 +12,10 @@
 //   dS_{t-1} = (dS~_t - dd_t r_t^T) Diag(alpha_t).
 // Every row of S and of dS evolves on its own; only the read-outs mix rows.
 // The work is split so that no per-token state is ever stored:
-//   F1  forward, warp per state row:  delta_t (a row reduction per token)
-//   R1  reverse, warp per state row:  dd_t, dS0
+//   F1  forward, 8 (or 4) state rows per warp: delta_t (a row reduction
+//       per token)
+//   R1  reverse, likewise: dd_t, dS0 (F1 and R1 share no data and run as
+//       one launch)
 //   F2  forward, thread per key column, delta given: dq'_t and dr_t
 //   R2  reverse, thread per key column, dd given:    dw_t
 // F2 and R2 have no reduction and no feedback (a gated linear attention pass
@@ -30,6 +32,11 @@
 // The preconditioner's coefficients B_t depend on A_t = A_{t-1} + k_t.k_t
 // ("Preconditioned DeltaNet", ja §2.2); each token's dB_t gives a dA_t, and
 // A_t feeds every later token, so k_t receives 2 k_t (sum_{s>=t} dA_s).
+//
+// Under a fused prologue the inputs are raw projections: the activations
+// are applied where the inputs are read and the gradients are taken back
+// through them (to the logits of the gates, through the L2 normalisation of
+// q and k, through the decay map).
 //
 // All arithmetic is fp32; inputs of either dtype are widened on load and
 // every gradient is written in fp32.
