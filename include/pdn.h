@@ -212,11 +212,15 @@ pdn_status_t pdn_chunk_fwd_profiled(const pdn_problem_t *p, const pdn_tensors_t 
 pdn_status_t pdn_chunk_fwd_noalloc(const pdn_problem_t *p, const pdn_tensors_t *t, void *stream);
 
 /* Chunked forward from host memory, end to end: copies the inputs in, runs
- * pdn_chunk_fwd and copies the outputs out, with the batch cut into `slices`
- * contiguous parts so that on the GPU the host-to-device copy of part i + 1,
- * the forward of part i and the device-to-host copy of part i - 1 overlap
- * (the batch elements are independent chains, so the result is that of one
- * pdn_chunk_fwd over the whole batch).
+ * pdn_chunk_fwd and copies the outputs out, in `slices` parts so that on the
+ * GPU the host-to-device copy of part i + 1, the forward of part i and the
+ * device-to-host copy of part i - 1 overlap. Up to B parts cut the batch
+ * into contiguous groups (the batch elements are independent chains, so the
+ * result is that of one pdn_chunk_fwd over the whole batch); with more parts
+ * each sequence is also cut into ceil(slices / B) runs of whole chunks, run
+ * in order, each starting from the state (and accumulator) the previous run
+ * left in the device ST (AT) -- the forward's own continuation, the same
+ * result up to the rounding of the accumulator's sums.
  *   - `dev`: the device tensors of the whole problem, as pdn_chunk_fwd takes
  *     them (they are also the staging buffers). `workspace` as for
  *     pdn_chunk_fwd on the whole problem.
@@ -226,7 +230,9 @@ pdn_status_t pdn_chunk_fwd_noalloc(const pdn_problem_t *p, const pdn_tensors_t *
  *     non-NULL host output (o, ST, AT) receives the result; a NULL one leaves
  *     that tensor on the device (an input already there, an output kept).
  *     Every non-NULL host pointer needs its device buffer.
- *   - 1 <= slices <= B. Work is ordered after the work already on `stream`,
+ *   - 1 <= slices <= 128, and B x (runs per sequence) <= 128. More parts
+ *     than batch elements need the device ST (and AT for the preconditioned
+ *     variants). Work is ordered after the work already on `stream`,
  *     and `stream` waits for all of it; the compute runs on `stream`, the
  *     copies on two streams of the library's own, created on first use on
  *     each device together with their events (nothing is created later).

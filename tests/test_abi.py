@@ -186,9 +186,14 @@ def test_host_pipeline_argument_errors(lib):
     t = _tensors()
     need = pdn.pdn_chunk_fwd_workspace(p)
     ws = FAKE + 0x100000
-    # slices outside [1, B]
+    # slices outside [1, 128]
     assert pdn.pdn_chunk_fwd_host(p, t, t, ws, need, 0, None) == pdn.PDN_ERR_INVALID_ARG
+    assert pdn.pdn_chunk_fwd_host(p, t, t, ws, need, 129, None) == pdn.PDN_ERR_INVALID_ARG
+    # more parts than batch elements cut the sequences into runs that hand
+    # the state on through the device ST (and AT, preconditioned variants)
     assert pdn.pdn_chunk_fwd_host(p, t, t, ws, need, p.B + 1, None) == pdn.PDN_ERR_INVALID_ARG
+    assert pdn.pdn_chunk_fwd_host(p, t, _tensors(ST=FAKE + 0x6000), ws, need, p.B + 1,
+                                  None) == pdn.PDN_ERR_INVALID_ARG
     # a host tensor without its device buffer
     assert pdn.pdn_chunk_fwd_host(p, _tensors(S0=FAKE + 0x9000), t, ws, need, 1,
                                   None) == pdn.PDN_ERR_INVALID_ARG

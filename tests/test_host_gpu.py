@@ -83,3 +83,57 @@ def test_host_path_odd_token_head_count(variant):
         o, ST, AT = host_run(w, x, None, None, slices)
         assert torch.equal(o, ref[0].cpu()), (variant, slices)
         assert torch.equal(ST, ref[1].cpu()), (variant, slices)
+
+
+def device_runs(w, x, S0, A0, slices):
+    """The device path cut the way pdn_chunk_fwd_host cuts sequences when
+    slices > B: per batch element, runs of whole chunks in order, each
+    pdn_chunk_fwd continuing from the previous run's S_T and A_T."""
+    dev = torch.device("cuda")
+    N = (w.T + 63) // 64
+    runs = min(-(-slices // w.B), N)
+    L = -(-N // runs)
+    runs = -(-N // L)
+    os, Ss, As = [], [], []
+    for b in range(w.B):
+        S = S0[b:b + 1].to(dev) if S0 is not None else None
+        A = A0[b:b + 1].to(dev) if A0 is not None else None
+        ob = []
+        for j in range(runs):
+            t0, t1 = j * L * 64, (w.T if j + 1 == runs else (j + 1) * L * 64)
+            sl = {n: (t[b:b + 1, t0:t1].contiguous().to(dev) if t is not None else None)
+                  for n, t in x.items()}
+            o, S, A = pdn.chunk_fwd(w.variant, sl["q"], sl["k"], sl["v"],
+                                    **{n: sl[n] for n in GATES}, S0=S, A0=A)
+            ob.append(o)
+        os.append(torch.cat(ob, 1))
+        Ss.append(S)
+        As.append(A)
+    torch.cuda.synchronize()
+    o = torch.cat(os, 0).cpu()
+    ST = torch.cat(Ss, 0).cpu()
+    AT = torch.cat(As, 0).cpu() if As[0] is not None else None
+    return o, ST, AT
+
+
+@pytest.mark.parametrize("variant,dk,dtype", [("PGDN", 128, "bf16"), ("GDN2", 128, "bf16"),
+                                              ("PKDA", 128, "bf16"), ("PGDN", 64, "f32")])
+def test_host_path_cuts_sequences_into_runs(variant, dk, dtype):
+    """slices > B: every sequence is also cut into runs of whole chunks that
+    hand the state and accumulator on through the device S_T and A_T. The
+    outputs equal the device path cut at the same chunk boundaries bitwise,
+    and the oracle within the parity bar; runs of 2, 3 and 5 per sequence
+    (the last with a ragged 44-token tail)."""
+    w = Workload("host-runs-" + variant, variant, 2, 300, 2, dk, dk, dtype, DECAY[variant])
+    x = make_inputs(w)
+    g = torch.Generator().manual_seed(9)
+    S0 = 0.2 * torch.randn(w.B, w.H, dk, dk, generator=g)
+    A0 = torch.rand(w.B, w.H, dk, generator=g) if variant in pdn.PRECOND_VARIANTS else None
+    for slices in (3, 5, 10):
+        o, ST, AT = host_run(w, x, S0, A0, slices)
+        ro, rS, rA = device_runs(w, x, S0, A0, slices)
+        assert torch.equal(o, ro), (variant, slices)
+        assert torch.equal(ST, rS), (variant, slices)
+        if AT is not None:
+            assert torch.equal(AT, rA), (variant, slices)
+    assert_parity(w, o, ST, AT, *run_oracle(w, x, S0, A0))
