@@ -24,6 +24,9 @@ timed steps. The JSON line also carries:
               of the fp32 CUDA-core peak (an ALU-bound pass);
   backward_prologue  the same from the layer's raw projections (gradients
               through the fused prologue's activations);
+  train_step  one forward + backward of the headline layer in training mode
+              (the forward saves delta and the chunk-start states, the
+              backward skips its forward sweep), against the plain pair;
   cpu_baseline the fp64 oracle on the host cores on a bounded sample.
 Multi-GPU (torchrun): every rank runs its own independent batch (weak
 scaling, no collective on the data path); the time is the max over ranks.
@@ -411,6 +414,12 @@ def run_ours(args):
         result["gpu_launches"] += (result["backward"]["gpu_launches"]
                                    + result["backward_prologue"]["gpu_launches"])
         torch.cuda.empty_cache()
+        if tc:
+            result["train_step"] = bench_train(args, w, dev, stream, rank, mor, barrier,
+                                               result["ms_per_step"]
+                                               + result["backward"]["ms_per_step"])
+            result["gpu_launches"] += result["train_step"]["gpu_launches"]
+            torch.cuda.empty_cache()
 
     # ---------------- decode workload
     if not args.no_decode:
@@ -599,6 +608,86 @@ def bench_backward(args, w, dev, stream, rank, mor, barrier, raw=False):
            "l2": "inputs larger than L2 (no flush)",
            "gpu_launches": args.steps * launches}
     del x, dO, dST, g, ws, grads, tens
+    return res
+
+
+def bench_train(args, w, dev, stream, rank, mor, barrier, plain_ms):
+    """Times `args.steps` training steps of the headline layer in training
+    mode: pdn_chunk_fwd_save (the forward, also leaving every token's delta and
+    the chunk-start states) then pdn_chunk_bwd_saved (the backward without its
+    forward sweep). Each half is also timed alone; `plain_ms` is the forward
+    plus backward measured above, for comparison."""
+    import torch
+
+    from linear_recurrence_sequence_chunked_b200 import pdn
+    from linear_recurrence_sequence_chunked_b200.workloads import make_inputs
+
+    wr = w.replace(seed=rank_seed(w.seed, rank))
+    x = make_inputs(wr, device=dev, generator_device=dev)
+    gen = torch.Generator(device=dev).manual_seed(rank_seed(7, rank))
+    dO = torch.randn(w.B, w.T, w.H, w.dv, generator=gen, device=dev).to(x["v"].dtype)
+    dST = torch.randn(w.B, w.H, w.dv, w.dk, generator=gen, device=dev)
+    prob = pdn.make_problem(w.variant, w.B, w.T, w.H, w.dk, w.dv, x["k"].dtype, w.decay, w.chunk,
+                            "auto", w.q_scale, w.precond_x, w.precond_eps)
+    f32 = dict(dtype=torch.float32, device=dev)
+    o = torch.empty(w.B, w.T, w.H, w.dv, dtype=x["v"].dtype, device=dev)
+    ST = torch.empty(w.B, w.H, w.dv, w.dk, **f32)
+    AT = torch.empty(w.B, w.H, w.dk, **f32) if w.variant in pdn.PRECOND_VARIANTS else None
+    delta = torch.empty(w.B, w.H, w.T, w.dv, **f32)
+    ckpt = torch.empty(w.B, w.H, (w.T + 63) // 64, w.dk, w.dv, **f32)
+    g = {n: torch.empty_like(x[n], **f32) for n in ("q", "k", "v")}
+    g["log_alpha"] = torch.empty_like(x["log_alpha"], **f32)
+    g["beta"] = torch.empty_like(x["beta"], **f32)
+    g["S0"] = torch.empty(w.B, w.H, w.dv, w.dk, **f32)
+    g["A0"] = torch.empty(w.B, w.H, w.dk, **f32)
+    tens = pdn.make_tensors(x["q"], x["k"], x["v"], o, x["log_alpha"], x["beta"], ST=ST, AT=AT)
+    grads = pdn.make_grads(dO, dST, g["q"], g["k"], g["v"], g["log_alpha"], g["beta"], None, None,
+                           g["S0"], g["A0"])
+    fws = torch.empty(max(1, pdn.pdn_chunk_fwd_workspace(prob)), dtype=torch.uint8, device=dev)
+    bws = torch.empty(pdn.pdn_chunk_bwd_workspace(prob), dtype=torch.uint8, device=dev)
+    sptr = stream.cuda_stream
+
+    def fwd():
+        rc = pdn.pdn_chunk_fwd_save(prob, tens, delta.data_ptr(), ckpt.data_ptr(), fws.data_ptr(),
+                                    fws.numel(), sptr)
+        if rc != pdn.PDN_OK:
+            raise pdn.PdnError(rc, "pdn_chunk_fwd_save")
+
+    def bwd():
+        rc = pdn.pdn_chunk_bwd_saved(prob, tens, grads, delta.data_ptr(), ckpt.data_ptr(),
+                                     bws.data_ptr(), bws.numel(), sptr)
+        if rc != pdn.PDN_OK:
+            raise pdn.PdnError(rc, "pdn_chunk_bwd_saved")
+
+    def timed(body):
+        for _ in range(args.warmup):
+            body()
+        barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            body()
+        e1.record(stream)
+        barrier()
+        return mor(e0.elapsed_time(e1)) / args.steps
+
+    ms = timed(lambda: (fwd(), bwd()))
+    ms_fwd = timed(fwd)
+    ms_bwd = timed(bwd)
+    if pdn.device_error() != pdn.PDN_OK:
+        raise SystemExit("device error during the training-step timed region")
+    fwd_launches = 4 if w.variant in pdn.PRECOND_VARIANTS else 2
+    launches = fwd_launches + 2 + 1 + 1 + 2 + 1 + 4 + 3
+    res = {"workload": w.name, "variant": w.variant,
+           "value": w.B * w.T / (ms / 1e3), "unit": "tokens/s", "ms_per_step": ms,
+           "forward_save_ms": ms_fwd, "backward_saved_ms": ms_bwd,
+           "plain_step_ms": plain_ms, "speedup_vs_plain": plain_ms / ms if plain_ms else None,
+           "what": ("pdn_chunk_fwd_save + pdn_chunk_bwd_saved: the forward leaves delta and the "
+                    "chunk-start states (fp32), the backward skips its forward row sweep; "
+                    "gradients at bf16 accuracy"),
+           "l2": "inputs larger than L2 (no flush)",
+           "gpu_launches": 3 * args.steps * launches}
+    del x, dO, dST, g, fws, bws, grads, tens, delta, ckpt
     return res
 
 

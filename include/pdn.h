@@ -331,6 +331,31 @@ size_t pdn_chunk_bwd_workspace(const pdn_problem_t *p);
 pdn_status_t pdn_chunk_bwd(const pdn_problem_t *p, const pdn_tensors_t *t, const pdn_grads_t *g,
                            void *workspace, size_t ws_bytes, void *stream);
 
+/* Training mode ("Gated DeltaNet-2", ja §3: the chunkwise form's Delta = U~ -
+ * Y~ S^T holds every token's delta_t = u_t - S_{t-1} D_t r_t). The
+ * tensor-core forward can leave, besides o, ST and AT, what the backward's
+ * forward sweep would otherwise recompute: every token's delta_t and the
+ * state at the start of every 64-token chunk. pdn_chunk_bwd_saved then
+ * skips that sweep. The saved values carry the forward's bf16-operand
+ * rounding, so these gradients meet the bf16 bar (normalised error 2e-2),
+ * not the fp32 backward's.
+ *   - `delta`: fp32 [B,H,T,d_v]; `ckpt`: fp32 [B,H,ceil(T/64),d_k,d_v],
+ *     the state S (d_v x d_k) before each chunk's first token stored
+ *     transposed (ckpt[..][c][i][j] = S[j][i]); device pointers, 16-byte
+ *     aligned, written by pdn_chunk_fwd_save.
+ *   - Only problems the tensor-core path takes (pdn_chunk_fwd_impl ==
+ *     PDN_IMPL_TC, p->impl not SIMT; T >= 1); others: PDN_ERR_UNSUPPORTED.
+ * pdn_chunk_fwd_save: as pdn_chunk_fwd (same arguments and checks), also
+ * writing delta and ckpt.
+ * pdn_chunk_bwd_saved: as pdn_chunk_bwd for the same problem and inputs,
+ * from the saved delta and ckpt and the forward's final state t->ST
+ * (required). */
+pdn_status_t pdn_chunk_fwd_save(const pdn_problem_t *p, const pdn_tensors_t *t, float *delta,
+                                float *ckpt, void *workspace, size_t ws_bytes, void *stream);
+pdn_status_t pdn_chunk_bwd_saved(const pdn_problem_t *p, const pdn_tensors_t *t,
+                                 const pdn_grads_t *g, const float *delta, const float *ckpt,
+                                 void *workspace, size_t ws_bytes, void *stream);
+
 /* Synchronises `stream`, returns the first device-side error recorded on the
  * current device since the last call (PDN_OK if none) and clears it. */
 pdn_status_t pdn_get_device_error(void *stream);

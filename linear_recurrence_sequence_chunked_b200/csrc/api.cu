@@ -249,6 +249,45 @@ extern "C" pdn_status_t pdn_chunk_bwd(const pdn_problem_t *p, const pdn_tensors_
              : PDN_ERR_CUDA;
 }
 
+// Training mode: the forward that also leaves every token's delta and the
+// chunk-start states, and the backward that reuses them.
+extern "C" pdn_status_t pdn_chunk_fwd_save(const pdn_problem_t *p, const pdn_tensors_t *t,
+                                           float *delta, float *ckpt, void *workspace,
+                                           size_t ws_bytes, void *stream) {
+  int impl = -1;
+  const pdn_status_t st = check_chunk_fwd(p, t, workspace, ws_bytes, &impl);
+  if (st != PDN_OK) return st;
+  if (!delta || !ckpt || !aligned(delta, 16) || !aligned(ckpt, 16)) return PDN_ERR_INVALID_ARG;
+  if (impl != PDN_IMPL_TC || p->T == 0) return PDN_ERR_UNSUPPORTED;
+  KParams P = make_params(p, t, nullptr);
+  P.sv_delta = delta;
+  P.sv_ckpt = ckpt;
+  P.err = device_error_word();
+  if (!P.err) return PDN_ERR_CUDA;
+  return launch_chunk_split(P, workspace, static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? PDN_OK
+             : PDN_ERR_CUDA;
+}
+
+extern "C" pdn_status_t pdn_chunk_bwd_saved(const pdn_problem_t *p, const pdn_tensors_t *t,
+                                            const pdn_grads_t *g, const float *delta,
+                                            const float *ckpt, void *workspace, size_t ws_bytes,
+                                            void *stream) {
+  const pdn_status_t st = check_chunk_bwd(p, t, g, workspace, ws_bytes);
+  if (st != PDN_OK) return st;
+  if (!delta || !ckpt || !aligned(delta, 16) || !aligned(ckpt, 16) || !t->ST)
+    return PDN_ERR_INVALID_ARG;
+  KParams P = make_params(p, t, nullptr);
+  if (select_impl(p, P) != PDN_IMPL_TC || p->T == 0) return PDN_ERR_UNSUPPORTED;
+  P.sv_delta = const_cast<float *>(delta);
+  P.sv_ckpt = const_cast<float *>(ckpt);
+  P.err = device_error_word();
+  if (!P.err) return PDN_ERR_CUDA;
+  return launch_chunk_bwd(P, g, workspace, static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? PDN_OK
+             : PDN_ERR_CUDA;
+}
+
 extern "C" pdn_status_t pdn_chunk_fwd_profiled(const pdn_problem_t *p, const pdn_tensors_t *t,
                                                void *workspace, size_t ws_bytes, void *stream,
                                                float *kernel_ms, int *n_kernels) {

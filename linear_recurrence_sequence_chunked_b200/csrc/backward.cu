@@ -116,8 +116,11 @@ struct BParams {
   // c dO in fp32, [BH][T][d_v] like delta and dd (zeros when dO is not given)
   float *cdo;
   // S before the first token of each kCk-token chunk (F1) and the cotangent
-  // entering each chunk's last token (R1): [BH][nck][d_v][d_k]
+  // entering each chunk's last token (R1): [BH][nck][d_v][d_k]; the states
+  // saved by the forward in training mode are transposed, [BH][nck][d_k][d_v]
+  // (ck_t)
   float *ckS, *ckD;
+  bool ck_t;
   int GS, R, G, nb, nck;
   // element counts of the workspace arrays (index checks of the debug build)
   size_t n_rows, n_part, n_ck;
@@ -868,7 +871,9 @@ __device__ __forceinline__ void col_issue(const BParams &Q, const ColPiece (&pc)
 // dq'_t = c S_t^T dO_t and dr_t = -P_t^T dd_t. (F2 and R2: at most 128
 // registers, four CTAs per SM -- a few spilled bytes, but more warps to wait
 // on shared-memory loads with; measured 1.5 % faster than three CTAs.)
-template <int R>
+// CKT: the chunk-start states are the forward's transposed checkpoint
+// (training mode).
+template <int R, bool CKT>
 __global__ void __launch_bounds__(128, 4) f2_kernel(const BParams Q) {
   extern __shared__ float4 smem4[];
   float *sm = reinterpret_cast<float *>(smem4);
@@ -907,12 +912,38 @@ __global__ void __launch_bounds__(128, 4) f2_kernel(const BParams Q) {
     }
   };
   float2 S[R / 2];  // rows (2h, 2h + 1) of this column
+  if (CKT && R % 32 == 0 && j0 + R <= dv) {
+    // the forward's transposed checkpoint, 32 rows at a time through shared
+    // memory (the staging buffer is not in use yet): read straight, each
+    // thread's rows are one 128-byte run and a warp load spans 32 lines
 #pragma unroll
-  for (int j = 0; j < R; ++j) {
-    const size_t e = (((size_t)bh * Q.nck + ck) * dv + j0 + j) * dk + i;
-    const float x = in_bounds(P.err, e < Q.n_ck) ? Q.ckS[e] : 0.f;
-    if (j & 1) S[j / 2].y = x;
-    else S[j / 2].x = x;
+    for (int h = 0; h < R / 32; ++h) {
+      for (int k = threadIdx.x; k < dk * 8; k += blockDim.x) {
+        const int c = k >> 3, q4 = k & 7;  // column, float4 of its 32 rows
+        const size_t e = (((size_t)bh * Q.nck + ck) * dk + c) * dv + j0 + 32 * h + 4 * q4;
+        float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (in_bounds(P.err, e + 4 <= Q.n_ck)) x = *reinterpret_cast<const float4 *>(Q.ckS + e);
+        float *d = sm + c * 33 + 4 * q4;  // padded rows: no bank conflicts either way
+        d[0] = x.x; d[1] = x.y; d[2] = x.z; d[3] = x.w;
+      }
+      __syncthreads();
+#pragma unroll
+      for (int jj = 0; jj < 32; ++jj) {
+        const int j = 32 * h + jj;
+        if (j & 1) S[j / 2].y = sm[i * 33 + jj];
+        else S[j / 2].x = sm[i * 33 + jj];
+      }
+      __syncthreads();
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < R; ++j) {
+      const size_t e = CKT ? (((size_t)bh * Q.nck + ck) * dk + i) * dv + j0 + j
+                           : (((size_t)bh * Q.nck + ck) * dv + j0 + j) * dk + i;
+      const float x = in_bounds(P.err, e < Q.n_ck) ? Q.ckS[e] : 0.f;
+      if (j & 1) S[j / 2].y = x;
+      else S[j / 2].x = x;
+    }
   }
   issue(0);
   cp_async_commit();
@@ -1338,11 +1369,11 @@ cudaError_t set_smem(K kernel, size_t bytes) {
 
 // The merged row sweeps for C key channels per lane and RW rows per warp.
 template <int C, int RW, bool UNR>
-cudaError_t launch_fr1_t(const BParams &Q, unsigned n, cudaStream_t st) {
+cudaError_t launch_fr1_t(const BParams &Q, unsigned n, bool r1_only, cudaStream_t st) {
   const size_t smem = 2 * kLCR * (4 * 32 * C + 4 * RW) * sizeof(float);  // R1's (> F1's)
   const cudaError_t err = set_smem(fr1_kernel<C, RW, UNR>, smem);
   if (err != cudaSuccess) return err;
-  fr1_kernel<C, RW, UNR><<<2 * n, 128, smem, st>>>(Q, (int)n);
+  fr1_kernel<C, RW, UNR><<<r1_only ? n : 2 * n, 128, smem, st>>>(Q, (int)n);
   return cudaSuccess;
 }
 
@@ -1356,20 +1387,23 @@ cudaError_t launch_fr1_t(const BParams &Q, unsigned n, cudaStream_t st) {
 // with 4 (unrolled); unrolled against rolled at 8 rows there: 28.7 against
 // 26.1.
 template <int C>
-cudaError_t launch_fr1_c(const BParams &Q, unsigned n, bool rw8, bool unr, cudaStream_t st) {
-  if (rw8) return unr ? launch_fr1_t<C, 8, true>(Q, n, st) : launch_fr1_t<C, 8, false>(Q, n, st);
-  return unr ? launch_fr1_t<C, 4, true>(Q, n, st) : launch_fr1_t<C, 4, false>(Q, n, st);
+cudaError_t launch_fr1_c(const BParams &Q, unsigned n, bool rw8, bool unr, bool r1_only,
+                         cudaStream_t st) {
+  if (rw8)
+    return unr ? launch_fr1_t<C, 8, true>(Q, n, r1_only, st) : launch_fr1_t<C, 8, false>(Q, n, r1_only, st);
+  return unr ? launch_fr1_t<C, 4, true>(Q, n, r1_only, st) : launch_fr1_t<C, 4, false>(Q, n, r1_only, st);
 }
 cudaError_t launch_fr1(const BParams &Q, cudaStream_t st) {
   const KParams &P = Q.P;
+  const bool r1_only = P.sv_delta && P.sv_ckpt;  // training mode: F1's outputs are saved
   const long long BH = (long long)P.B * P.H, sms = num_sms();
   const long long n8 = BH * ((P.dv + 31) / 32);  // CTAs per sweep at 8 rows per warp
-  const bool rw8 = 2 * n8 >= 2 * sms;
+  const bool rw8 = (r1_only ? 1 : 2) * n8 >= 2 * sms;  // >= 2 CTAs per SM in the launch
   const unsigned n = (unsigned)(rw8 ? n8 : BH * ((P.dv + 15) / 16));
   const bool unr = (long long)n >= sms;
-  if (P.dk > 64) return launch_fr1_c<4>(Q, n, rw8, unr, st);
-  if (P.dk > 32) return launch_fr1_c<2>(Q, n, rw8, unr, st);
-  return launch_fr1_c<1>(Q, n, rw8, unr, st);
+  if (P.dk > 64) return launch_fr1_c<4>(Q, n, rw8, unr, r1_only, st);
+  if (P.dk > 32) return launch_fr1_c<2>(Q, n, rw8, unr, r1_only, st);
+  return launch_fr1_c<1>(Q, n, rw8, unr, r1_only, st);
 }
 
 template <typename Tin, int R>
@@ -1387,11 +1421,13 @@ cudaError_t launch_bwd_t(const BParams &Q, cudaStream_t st) {
 
   const size_t sm_f2 = 2 * kLCC * (2 * dk + 3 * R) * sizeof(float);
   const size_t sm_r2 = 2 * kLCC * (4 * dk + 3 * R) * sizeof(float);
-  if ((err = set_smem(f2_kernel<R>, sm_f2)) != cudaSuccess) return err;
+  if ((err = set_smem(Q.ck_t ? f2_kernel<R, true> : f2_kernel<R, false>, sm_f2)) != cudaSuccess)
+    return err;
   if ((err = set_smem(r2_kernel<R>, sm_r2)) != cudaSuccess) return err;
   const unsigned grid_cols = (unsigned)(BH * Q.nck * Q.G);
   if ((err = launch_fr1(Q, st)) != cudaSuccess) return err;
-  f2_kernel<R><<<grid_cols, dk, sm_f2, st>>>(Q);
+  if (Q.ck_t) f2_kernel<R, true><<<grid_cols, dk, sm_f2, st>>>(Q);
+  else f2_kernel<R, false><<<grid_cols, dk, sm_f2, st>>>(Q);
   r2_kernel<R><<<grid_cols, dk, sm_r2, st>>>(Q);
   e1_kernel<Tin><<<grid_for(BHT * 32, 256), 256, 0, st>>>(Q);
 
@@ -1402,7 +1438,8 @@ cudaError_t launch_bwd_t(const BParams &Q, cudaStream_t st) {
                Q.dST ? Q.phi : nullptr, nullptr, Q.bsum, st);
     else
       run_scan(P, ScanArr{Q.sigma, false}, ScanArr{Q.dla, true}, 1, Q.nb, true,
-               Q.dST ? Q.phi + BH * dk : nullptr, nullptr, Q.bsum, st);    if (P.prologue & (PDN_PRO_DECAY_SOFTPLUS | PDN_PRO_DECAY_LOGSIGMOID)) {
+               Q.dST ? Q.phi + BH * dk : nullptr, nullptr, Q.bsum, st);
+    if (P.prologue & (PDN_PRO_DECAY_SOFTPLUS | PDN_PRO_DECAY_LOGSIGMOID)) {
       const long long n = BHT * (P.decay == PDN_DECAY_CHANNEL ? dk : 1);
       decay_pro_kernel<Tin><<<grid_for(n, 256), 256, 0, st>>>(Q, n);
     }
@@ -1459,6 +1496,14 @@ cudaError_t launch_chunk_bwd(const KParams &P, const pdn_grads_t *g, void *works
   Q.st = ws + L.st; Q.part = ws + L.part; Q.cpsi = ws + L.cpsi; Q.sigma = ws + L.sigma;
   Q.dacc = ws + L.dacc; Q.bsum = ws + L.bsum; Q.phi = ws + L.phi;
   Q.ckS = ws + L.ckS; Q.ckD = ws + L.ckD;
+  if (P.sv_delta && P.sv_ckpt) {
+    // training mode: delta, the chunk-start states and S_T come from the
+    // forward (pdn_chunk_fwd_save); the forward row sweep F1 is skipped
+    Q.delta = P.sv_delta;
+    Q.ckS = P.sv_ckpt;
+    Q.ck_t = true;
+    Q.st = P.ST;
+  }
   Q.GS = L.GS; Q.R = L.R; Q.G = L.G; Q.nb = L.nb; Q.nck = L.nck;
   Q.n_rows = (size_t)BH * P.T * P.dv;
   Q.n_part = (size_t)L.G * BH * P.T * 3 * P.dk;

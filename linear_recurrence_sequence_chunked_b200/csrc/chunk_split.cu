@@ -1451,6 +1451,19 @@ __global__ void __launch_bounds__(kK2Threads, 1) k2_state(const KParams P, void 
           tmem_ld16(tm + lane_q + TM_S + col0 + 16, sv[1]);
           tmem_wait_ld();
         }
+        if (P.sv_ckpt) {
+          // training mode: the state at the start of chunk cb + n, stored
+          // transposed ([d_k][d_v] per chunk) so that a warp's 32 rows j of
+          // one column are one 128-byte line (row-major, each lane's float4s
+          // scattered over 32 lines and held up the epilogue on the
+          // load/store unit)
+          const size_t nch = (size_t)(P.T + kC - 1) / kC;
+          float *dst = P.sv_ckpt + (((size_t)bh * nch + chunk_ok(P, cb + n)) * kD + col0) * kD + j;
+#pragma unroll
+          for (int u = 0; u < 2; ++u)
+#pragma unroll
+            for (int e = 0; e < 16; ++e) dst[(size_t)(16 * u + e) * kD] = sv[u][e];
+        }
         {
           uint32_t pk[16];
 #pragma unroll
@@ -1495,8 +1508,15 @@ __global__ void __launch_bounds__(kK2Threads, 1) k2_state(const KParams P, void 
         for (int e = 0; e < 8; ++e) pk[e] = pack_bf16(v[2 * e], v[2 * e + 1]);
         tmem_st8u(tm + lane_q + tm_db(n) + 8 * cg, pk);
         tmem_wait_st();
+        k2_warp_arrive(B.depi, lane);
+        if (P.sv_delta) {  // training mode: delta of tokens 16 cg .. 16 cg + 15, row j (after the hand-back)
+          const int t0 = chunk_ok(P, cb + n) * kC + 16 * cg;
+          float *dst = P.sv_delta + ((size_t)bh * P.T + t0) * kD + j;
+#pragma unroll
+          for (int e = 0; e < 16; ++e)
+            if (t0 + e < P.T) dst[(size_t)e * kD] = v[e];
+        }
       }
-      k2_warp_arrive(B.depi, lane);
       if (n + 1 < N) fetch_e(n + 1);
       if (n > 0) k2_store_o(P, ot_prev, b, h, pc_prev, min(kC, P.T - pc_prev), lane, quarter, cg, 1);
       if (!(ok = k2_warp_wait(B.bar7, (uint32_t)(n & 1), abort_flag, lane))) break;

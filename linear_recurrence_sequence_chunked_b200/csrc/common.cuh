@@ -27,6 +27,10 @@ struct KParams {
   const float *A0;
   float *AT;
   void *o;
+  // Training mode (tensor-core state pass; NULL = off): every token's delta
+  // [B*H][T][d_v] and the state at the start of every chunk, transposed
+  // [B*H][ceil(T/64)][d_k][d_v], both fp32, for the backward to reuse.
+  float *sv_delta, *sv_ckpt;
   int *err;  // per-device error word (first error wins)
 };
 

@@ -92,6 +92,10 @@ def load() -> ctypes.CDLL:
         lib.pdn_chunk_bwd_workspace.argtypes = [P]
         lib.pdn_chunk_bwd.restype = ctypes.c_int
         lib.pdn_chunk_bwd.argtypes = [P, T, G, vp, ctypes.c_size_t, vp]
+        lib.pdn_chunk_fwd_save.restype = ctypes.c_int
+        lib.pdn_chunk_fwd_save.argtypes = [P, T, vp, vp, vp, ctypes.c_size_t, vp]
+        lib.pdn_chunk_bwd_saved.restype = ctypes.c_int
+        lib.pdn_chunk_bwd_saved.argtypes = [P, T, G, vp, vp, vp, ctypes.c_size_t, vp]
         lib.pdn_chunk_transition.restype = ctypes.c_int
         lib.pdn_chunk_transition.argtypes = [P, T, vp, ctypes.c_size_t, vp]
         lib.pdn_key_energy.restype = ctypes.c_int
@@ -146,6 +150,19 @@ def pdn_chunk_bwd(problem: PdnProblem, tensors: PdnTensors, grads: PdnGrads, wor
                   ws_bytes: int, stream: int) -> int:
     return load().pdn_chunk_bwd(ctypes.byref(problem), ctypes.byref(tensors), ctypes.byref(grads),
                                 workspace, ws_bytes, stream)
+
+
+def pdn_chunk_fwd_save(problem: PdnProblem, tensors: PdnTensors, delta: int, ckpt: int,
+                       workspace: int, ws_bytes: int, stream: int) -> int:
+    return load().pdn_chunk_fwd_save(ctypes.byref(problem), ctypes.byref(tensors), delta, ckpt,
+                                     workspace, ws_bytes, stream)
+
+
+def pdn_chunk_bwd_saved(problem: PdnProblem, tensors: PdnTensors, grads: PdnGrads, delta: int,
+                        ckpt: int, workspace: int, ws_bytes: int, stream: int) -> int:
+    return load().pdn_chunk_bwd_saved(ctypes.byref(problem), ctypes.byref(tensors),
+                                      ctypes.byref(grads), delta, ckpt, workspace, ws_bytes,
+                                      stream)
 
 
 def pdn_chunk_transition(problem: PdnProblem, tensors: PdnTensors, workspace: int,
@@ -263,10 +280,14 @@ def _check(code, where):
 def chunk_fwd(variant: str, q, k, v, log_alpha=None, beta=None, erase=None, write=None,
               S0=None, A0=None, chunk: int = 64, impl: str = "auto", q_scale: float = 1.0,
               precond_x: float = 1.5, precond_eps: float = 1e-6, want_state: bool = True,
-              out=None, workspace=None, prologue: int = 0, decay_scale: float = 1.0):
+              out=None, workspace=None, prologue: int = 0, decay_scale: float = 1.0,
+              saved: Optional[dict] = None):
     """Chunked forward on torch tensors (all on one CUDA device, contiguous).
 
     Returns (o, S_T, A_T); S_T/A_T are None when not requested / not used.
+    With ``saved`` (a dict) the tensor-core forward also leaves every token's
+    delta and the chunk-start states in saved["delta"] / saved["ckpt"] for
+    ``chunk_bwd(..., saved=saved, ST=S_T)`` (training mode, pdn_chunk_fwd_save).
     """
     B, T, H, d_k = k.shape
     d_v = v.shape[3]
@@ -287,7 +308,14 @@ def chunk_fwd(variant: str, q, k, v, log_alpha=None, beta=None, erase=None, writ
             workspace = torch.empty(need, dtype=torch.uint8, device=dev)
         ws_ptr, ws_bytes = workspace.data_ptr(), workspace.numel() * workspace.element_size()
     stream = torch.cuda.current_stream(dev).cuda_stream
-    _check(pdn_chunk_fwd(p, t, ws_ptr, ws_bytes, stream), "pdn_chunk_fwd")
+    if saved is not None:
+        f32 = dict(dtype=torch.float32, device=dev)
+        saved["delta"] = torch.empty(B, H, T, d_v, **f32)
+        saved["ckpt"] = torch.empty(B, H, (T + 63) // 64, d_k, d_v, **f32)  # S^T per chunk
+        _check(pdn_chunk_fwd_save(p, t, saved["delta"].data_ptr(), saved["ckpt"].data_ptr(),
+                                  ws_ptr, ws_bytes, stream), "pdn_chunk_fwd_save")
+    else:
+        _check(pdn_chunk_fwd(p, t, ws_ptr, ws_bytes, stream), "pdn_chunk_fwd")
     return o, ST, AT
 
 
@@ -300,13 +328,15 @@ def make_grads(dO=None, dST=None, dq=None, dk=None, dv=None, dlog_alpha=None, db
 def chunk_bwd(variant: str, q, k, v, dO=None, dST=None, log_alpha=None, beta=None, erase=None,
               write=None, S0=None, A0=None, q_scale: float = 1.0, precond_x: float = 1.5,
               precond_eps: float = 1e-6, workspace=None, prologue: int = 0,
-              decay_scale: float = 1.0):
+              decay_scale: float = 1.0, saved: Optional[dict] = None, ST=None):
     """Gradients of chunk_fwd's (o, S_T) with respect to its inputs, given the
     cotangents dO [B,T,H,d_v] (input dtype) and dST [B,H,d_v,d_k] (fp32);
     either may be None (zero). Returns a dict of fp32 tensors with keys q, k,
     v, log_alpha, beta, erase, write, S0, A0 (None where the variant has no
     such input). With ``prologue`` bits the inputs are raw projections and the
-    gradients are with respect to them."""
+    gradients are with respect to them. With ``saved`` (from chunk_fwd(...,
+    saved=...)) and the forward's final state ``ST`` the backward reuses the
+    forward's deltas and chunk-start states (pdn_chunk_bwd_saved)."""
     B, T, H, d_k = k.shape
     d_v = v.shape[3]
     dev = k.device
@@ -322,7 +352,7 @@ def chunk_bwd(variant: str, q, k, v, dO=None, dST=None, log_alpha=None, beta=Non
                    else None),
          "S0": torch.empty(B, H, d_v, d_k, **f32),
          "A0": torch.empty(B, H, d_k, **f32) if variant in PRECOND_VARIANTS else None}
-    t = make_tensors(q, k, v, None, log_alpha, beta, erase, write, S0, None, A0, None)
+    t = make_tensors(q, k, v, None, log_alpha, beta, erase, write, S0, ST, A0, None)
     gr = make_grads(dO, dST, g["q"], g["k"], g["v"], g["log_alpha"], g["beta"], g["erase"],
                     g["write"], g["S0"], g["A0"])
     need = pdn_chunk_bwd_workspace(p)
@@ -334,7 +364,11 @@ def chunk_bwd(variant: str, q, k, v, dO=None, dST=None, log_alpha=None, beta=Non
             workspace = torch.empty(need, dtype=torch.uint8, device=dev)
         ws_ptr, ws_bytes = workspace.data_ptr(), workspace.numel() * workspace.element_size()
     stream = torch.cuda.current_stream(dev).cuda_stream
-    _check(pdn_chunk_bwd(p, t, gr, ws_ptr, ws_bytes, stream), "pdn_chunk_bwd")
+    if saved is not None:
+        _check(pdn_chunk_bwd_saved(p, t, gr, saved["delta"].data_ptr(), saved["ckpt"].data_ptr(),
+                                   ws_ptr, ws_bytes, stream), "pdn_chunk_bwd_saved")
+    else:
+        _check(pdn_chunk_bwd(p, t, gr, ws_ptr, ws_bytes, stream), "pdn_chunk_bwd")
     return g
 
 

@@ -281,3 +281,56 @@ def test_backward_prologue_finite_differences(variant, recipe, dtype, dk):
             if not abs(G[idx] - fd) <= 2e-3 * gmax + 1e-6:
                 bad.append((name, idx, float(G[idx]), fd, gmax))
     assert not bad, bad
+
+
+@pytest.mark.parametrize("variant,T", [("PGDN", 200), ("GDN2", 130), ("PKDA", 257),
+                                       ("FG2_GDN_PLUS", 64), ("PLA", 100)])
+def test_backward_training_mode(variant, T):
+    """Training mode: the tensor-core forward also leaves every token's delta
+    and the chunk-start states (pdn_chunk_fwd_save) and the backward reuses
+    them instead of its forward sweep (pdn_chunk_bwd_saved). Saving leaves
+    the forward's outputs bitwise unchanged; the gradients, which carry the
+    forward's bf16-operand rounding, meet the bf16 bar against the oracle."""
+    w = small(variant, "bf16", B=2, T=T, H=2, dk=128)
+    x = make_inputs(w)
+    S0, A0 = states(w)
+    dO, dST = cotangents(w)
+    dev = torch.device("cuda")
+    d = {n: (t.to(dev) if t is not None else None) for n, t in x.items()}
+    kw = dict(log_alpha=d["log_alpha"], beta=d["beta"], erase=d["erase"], write=d["write"],
+              S0=S0.to(dev), A0=None if A0 is None else A0.to(dev), q_scale=w.q_scale,
+              precond_x=w.precond_x, precond_eps=w.precond_eps)
+    o1, ST1, AT1 = pdn.chunk_fwd(w.variant, d["q"], d["k"], d["v"], **kw)
+    saved = {}
+    o2, ST2, AT2 = pdn.chunk_fwd(w.variant, d["q"], d["k"], d["v"], saved=saved, **kw)
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2) and torch.equal(ST1, ST2)
+    g = pdn.chunk_bwd(w.variant, d["q"], d["k"], d["v"], dO=dO.to(dev), dST=dST.to(dev),
+                      saved=saved, ST=ST2, **kw)
+    torch.cuda.synchronize()
+    assert pdn.device_error() == pdn.PDN_OK
+    gg = {n: (None if t is None else t.cpu().numpy()) for n, t in g.items()}
+    assert_grads(w, gg, run_oracle(w, x, S0, A0, dO, dST), tol=2e-2, label="[saved]")
+
+
+def test_backward_training_mode_time_segments():
+    """Training mode through the time-segmented forward (few chains, a long
+    sequence): the reused deltas and states index the whole sequence; the
+    gradients match the exact backward within the bf16 bar."""
+    w = small("PGDN", "bf16", B=1, T=4096, H=16, dk=128)
+    x = make_inputs(w, device="cuda")
+    gen = torch.Generator(device="cuda").manual_seed(5)
+    dO = torch.randn(w.B, w.T, w.H, w.dv, generator=gen, device="cuda").to(torch.bfloat16)
+    dST = torch.randn(w.B, w.H, w.dv, w.dk, generator=gen, device="cuda")
+    kw = dict(log_alpha=x["log_alpha"], beta=x["beta"], precond_x=w.precond_x,
+              precond_eps=w.precond_eps)
+    saved = {}
+    _, ST, _ = pdn.chunk_fwd(w.variant, x["q"], x["k"], x["v"], saved=saved, **kw)
+    gs = pdn.chunk_bwd(w.variant, x["q"], x["k"], x["v"], dO=dO, dST=dST, saved=saved, ST=ST, **kw)
+    ge = pdn.chunk_bwd(w.variant, x["q"], x["k"], x["v"], dO=dO, dST=dST, **kw)
+    torch.cuda.synchronize()
+    assert pdn.device_error() == pdn.PDN_OK
+    for n, t in ge.items():
+        if t is not None:
+            e = nmax_err(gs[n].cpu().numpy(), t.cpu().numpy())
+            assert e <= 2e-2, (n, e)
