@@ -1378,8 +1378,11 @@ cudaError_t launch_fr1_t(const BParams &Q, unsigned n, bool r1_only, cudaStream_
 }
 
 // Key channels per lane: 32 lanes cover d_k. Rows per warp: 8 (each staged
-// vector serves more rows) when that still gives at least two CTAs per SM,
-// else 4 (twice the CTAs). The unrolled chunk loop issues fewer instructions
+// vector serves more rows) when that still gives each sweep at least one CTA
+// per SM, else 4 (twice the CTAs); the same rule holds for R1 launched alone
+// (training mode): 4.23 ms against 4.37 with 8 rows on the headline layer
+// (256 CTAs), 19.25 against 20.79 with 4 on 32 pairs of 32k tokens (128 CTAs
+// at 8 rows). The unrolled chunk loop issues fewer instructions
 // but schedules worse when too few warps hide its latency, so it runs only
 // from one CTA per SM per sweep on. Measured on B200 (ms per backward):
 // headline layer (512 CTAs at 8 rows) 5.31 with 8 rows against 5.62 with 4;
@@ -1398,7 +1401,7 @@ cudaError_t launch_fr1(const BParams &Q, cudaStream_t st) {
   const bool r1_only = P.sv_delta && P.sv_ckpt;  // training mode: F1's outputs are saved
   const long long BH = (long long)P.B * P.H, sms = num_sms();
   const long long n8 = BH * ((P.dv + 31) / 32);  // CTAs per sweep at 8 rows per warp
-  const bool rw8 = (r1_only ? 1 : 2) * n8 >= 2 * sms;  // >= 2 CTAs per SM in the launch
+  const bool rw8 = n8 >= sms;  // >= 1 CTA per SM per sweep
   const unsigned n = (unsigned)(rw8 ? n8 : BH * ((P.dv + 15) / 16));
   const bool unr = (long long)n >= sms;
   if (P.dk > 64) return launch_fr1_c<4>(Q, n, rw8, unr, r1_only, st);

@@ -3,7 +3,8 @@ point a profiler at (``ncu ... python -m linear_recurrence_sequence_chunked_b200
 --op fwd --workload gdn2_bf16_32k --batch 1 --tokens 8192``).
 
 ``--op fwd`` calls pdn_chunk_fwd, ``bwd`` pdn_chunk_bwd (from random dO and
-dS_T), ``decode`` pdn_decode_step once per token. Inputs are the seeded
+dS_T), ``train`` pdn_chunk_fwd_save then pdn_chunk_bwd_saved (training mode),
+``decode`` pdn_decode_step once per token. Inputs are the seeded
 synthetic ones of ``workloads.py``; ``--batch`` and ``--tokens`` override the
 workload's B and T. Exits non-zero if a call fails or the device error word is
 set.
@@ -22,7 +23,7 @@ from .workloads import WORKLOADS, make_inputs
 def main(argv=None) -> int:
     ap = argparse.ArgumentParser()
     ap.add_argument("--workload", default="pgdn_bf16_4k", choices=sorted(WORKLOADS))
-    ap.add_argument("--op", default="fwd", choices=("fwd", "bwd", "decode"))
+    ap.add_argument("--op", default="fwd", choices=("fwd", "bwd", "train", "decode"))
     ap.add_argument("--batch", type=int, default=0)
     ap.add_argument("--tokens", type=int, default=0)
     ap.add_argument("--calls", type=int, default=2)
@@ -57,7 +58,14 @@ def main(argv=None) -> int:
             dO = torch.randn(w.B, w.T, w.H, w.dv, generator=gen, device=dev).to(x["v"].dtype)
             dST = torch.randn(w.B, w.H, w.dv, w.dk, generator=gen, device=dev)
             for _ in range(args.calls):
-                pdn.chunk_bwd(w.variant, x["q"], x["k"], x["v"], dO=dO, dST=dST, **g, **kw)
+                if args.op == "train":
+                    saved = {}
+                    _, ST, _ = pdn.chunk_fwd(w.variant, x["q"], x["k"], x["v"], **g, chunk=w.chunk,
+                                             saved=saved, **kw)
+                    pdn.chunk_bwd(w.variant, x["q"], x["k"], x["v"], dO=dO, dST=dST, **g,
+                                  saved=saved, ST=ST, **kw)
+                else:
+                    pdn.chunk_bwd(w.variant, x["q"], x["k"], x["v"], dO=dO, dST=dST, **g, **kw)
     torch.cuda.synchronize()
     if pdn.device_error() != pdn.PDN_OK:
         print("device error word set", file=sys.stderr)
