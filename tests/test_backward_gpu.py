@@ -313,6 +313,37 @@ def test_backward_training_mode(variant, T):
     assert_grads(w, gg, run_oracle(w, x, S0, A0, dO, dST), tol=2e-2, label="[saved]")
 
 
+@pytest.mark.parametrize("variant,recipe", [("PGDN", "softplus"), ("GDN2", "sigmoid"),
+                                            ("PKDA", "sigmoid")])
+def test_backward_training_mode_prologue(variant, recipe):
+    """Training mode from raw projections (fused prologue in both directions):
+    the saved deltas and states are those of the activated inputs, and the
+    gradients with respect to the raw projections match the exact backward's
+    (itself pinned by finite differences) within the bf16 bar."""
+    w = Workload("trainpro-%s" % variant, variant, 2, 150, 2, 128, 128, "bf16", DECAY[variant],
+                 decay_recipe=recipe, seed=11)
+    raw = make_raw_inputs(w, device="cuda")
+    bits, dscale = raw_prologue(w)
+    dO, dST = cotangents(w)
+    dO, dST = dO.cuda(), dST.cuda()
+    kw = dict(log_alpha=raw["log_alpha"], beta=raw["beta"], erase=raw["erase"],
+              write=raw["write"], q_scale=w.q_scale, precond_x=w.precond_x,
+              precond_eps=w.precond_eps, prologue=bits, decay_scale=dscale)
+    o1, ST1, _ = pdn.chunk_fwd(w.variant, raw["q"], raw["k"], raw["v"], **kw)
+    saved = {}
+    o2, ST2, _ = pdn.chunk_fwd(w.variant, raw["q"], raw["k"], raw["v"], saved=saved, **kw)
+    gs = pdn.chunk_bwd(w.variant, raw["q"], raw["k"], raw["v"], dO=dO, dST=dST, saved=saved,
+                       ST=ST2, **kw)
+    ge = pdn.chunk_bwd(w.variant, raw["q"], raw["k"], raw["v"], dO=dO, dST=dST, **kw)
+    torch.cuda.synchronize()
+    assert pdn.device_error() == pdn.PDN_OK
+    assert torch.equal(o1, o2) and torch.equal(ST1, ST2)
+    for n, t in ge.items():
+        if t is not None:
+            e = nmax_err(gs[n].cpu().numpy(), t.cpu().numpy())
+            assert e <= 2e-2, (n, e)
+
+
 def test_backward_training_mode_time_segments():
     """Training mode through the time-segmented forward (few chains, a long
     sequence): the reused deltas and states index the whole sequence; the

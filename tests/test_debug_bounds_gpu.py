@@ -23,7 +23,7 @@ def test_parity_suites_under_the_debug_build():
     assert os.path.basename(lib) == os.path.basename(pdn.DEBUG_LIB_PATH)
     env = dict(os.environ, PDN_LIBRARY=lib)
     sel = ("test_backward_lengths or test_backward_head_dims or test_backward_variants or "
-           "test_backward_many_chains or test_backward_prologue or "
+           "test_backward_many_chains or test_backward_prologue or test_backward_training_mode or "
            "test_tc_variants or time_segments or test_decode or test_variants_small")
     cmd = [sys.executable, "-m", "pytest", "-q", "-x", "-m", "gpu", "-p", "no:cacheprovider",
            "-k", sel, "tests/test_backward_gpu.py", "tests/test_tc_gpu.py",
