@@ -348,3 +348,33 @@ def test_debug_library_exports_every_declared_symbol():
 
 def test_bounds_status_string(lib):
     assert pdn.pdn_status_string(pdn.PDN_ERR_BOUNDS) == "PDN_ERR_BOUNDS"
+
+
+def test_training_mode_argument_errors(lib):
+    """pdn_chunk_fwd_save / pdn_chunk_bwd_saved: the forward's and the
+    backward's own checks first, then the saved buffers (present, 16-byte
+    aligned; the backward also needs the forward's S_T), then the path: only
+    problems the tensor-core forward takes. All decided before any launch."""
+    D, C = FAKE + 0x20000, FAKE + 0x40000
+    # the forward's checks come first
+    p = _problem(B=0)
+    assert pdn.pdn_chunk_fwd_save(p, _tensors(), D, C, None, 0, None) == pdn.PDN_ERR_INVALID_ARG
+    # the saved buffers
+    p = _problem()
+    for d, c in ((None, C), (D, None), (D + 4, C), (D, C + 8)):
+        assert pdn.pdn_chunk_fwd_save(p, _tensors(), d, c, None, 0,
+                                      None) == pdn.PDN_ERR_INVALID_ARG, (d, c)
+    # d = 64 runs on the CUDA-core path, which saves nothing
+    assert pdn.pdn_chunk_fwd_save(p, _tensors(), D, C, None, 0, None) == pdn.PDN_ERR_UNSUPPORTED
+    # the backward: its own checks, then the saved buffers and S_T, then the path
+    ws = pdn.pdn_chunk_bwd_workspace(p)
+    assert pdn.pdn_chunk_bwd_saved(_problem(B=0), _tensors(ST=FAKE + 0x9000), _grads(), D, C,
+                                   FAKE, ws, None) == pdn.PDN_ERR_INVALID_ARG
+    assert pdn.pdn_chunk_bwd_saved(p, _tensors(ST=FAKE + 0x9000), _grads(), D, C, None, 0,
+                                   None) == pdn.PDN_ERR_WORKSPACE
+    for d, c, st in ((None, C, FAKE + 0x9000), (D, None, FAKE + 0x9000), (D + 4, C, FAKE + 0x9000),
+                     (D, C, None)):
+        assert pdn.pdn_chunk_bwd_saved(p, _tensors(ST=st), _grads(), d, c, FAKE, ws,
+                                       None) == pdn.PDN_ERR_INVALID_ARG, (d, c, st)
+    assert pdn.pdn_chunk_bwd_saved(p, _tensors(ST=FAKE + 0x9000), _grads(), D, C, FAKE, ws,
+                                   None) == pdn.PDN_ERR_UNSUPPORTED
