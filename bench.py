@@ -686,7 +686,8 @@ def bench_train(args, w, dev, stream, rank, mor, barrier, plain_ms):
                     "chunk-start states (fp32), the backward skips its forward row sweep; "
                     "gradients at bf16 accuracy"),
            "l2": "inputs larger than L2 (no flush)",
-           "gpu_launches": 3 * args.steps * launches}
+           # the step loop, then the forward and the backward loops alone
+           "gpu_launches": 2 * args.steps * launches}
     del x, dO, dST, g, fws, bws, grads, tens, delta, ckpt
     return res
 
