@@ -1379,16 +1379,17 @@ cudaError_t launch_fr1_t(const BParams &Q, unsigned n, bool r1_only, cudaStream_
 
 // Key channels per lane: 32 lanes cover d_k. Rows per warp: 8 (each staged
 // vector serves more rows) when that still gives each sweep at least one CTA
-// per SM, else 4 (twice the CTAs); the same rule holds for R1 launched alone
-// (training mode): 4.23 ms against 4.37 with 8 rows on the headline layer
-// (256 CTAs), 19.25 against 20.79 with 4 on 32 pairs of 32k tokens (128 CTAs
-// at 8 rows). The unrolled chunk loop issues fewer instructions
-// but schedules worse when too few warps hide its latency, so it runs only
-// from one CTA per SM per sweep on. Measured on B200 (ms per backward):
-// headline layer (512 CTAs at 8 rows) 5.31 with 8 rows against 5.62 with 4;
-// 32 (batch, head) pairs of 32k tokens 24.3 with 8 rows (rolled) against 22.6
-// with 4 (unrolled); unrolled against rolled at 8 rows there: 28.7 against
-// 26.1.
+// per SM, else 4 (twice the CTAs). The unrolled chunk loop issues fewer
+// instructions but schedules worse when too few warps hide its latency, so
+// it runs only from one CTA per SM per sweep on. Measured on B200 (ms per
+// backward): headline layer (512 CTAs at 8 rows) 5.31 with 8 rows against
+// 5.62 with 4; 32 (batch, head) pairs of 32k tokens 24.3 with 8 rows (rolled)
+// against 22.6 with 4 (unrolled); unrolled against rolled at 8 rows there:
+// 28.7 against 26.1. The same rules hold for R1 launched alone (training
+// mode, ms per training-mode backward): headline layer (256 CTAs at 8 rows)
+// 4.23 with 8 rows against 4.37 with 4, and 4.25 unrolled against 4.53
+// rolled; 32 pairs of 32k tokens (128 CTAs at 8 rows) 19.25 with 4 rows
+// against 20.79 with 8, and 19.3 unrolled against 20.3 rolled.
 template <int C>
 cudaError_t launch_fr1_c(const BParams &Q, unsigned n, bool rw8, bool unr, bool r1_only,
                          cudaStream_t st) {
