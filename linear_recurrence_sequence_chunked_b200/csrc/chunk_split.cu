@@ -1451,6 +1451,20 @@ __global__ void __launch_bounds__(kK2Threads, 1) k2_state(const KParams P, void 
           tmem_ld16(tm + lane_q + TM_S + col0 + 16, sv[1]);
           tmem_wait_ld();
         }
+        {
+          uint32_t pk[16];
+#pragma unroll
+          for (int u = 0; u < 2; ++u)
+#pragma unroll
+            for (int e = 0; e < 8; ++e) pk[8 * u + e] = pack_bf16(sv[u][2 * e], sv[u][2 * e + 1]);
+          tmem_st16u(tm + lane_q + tm_sb(n) + 16 * cg, pk);
+        }
+        tmem_wait_st();
+        // MMA5 and MMA6 read only the bf16 copy: hand it over now. The decayed
+        // fp32 state below is MMA8's accumulator, and MMA8 waits for this
+        // warp's D-epilogue arrive, which follows a tcgen05.wait::st covering
+        // these stores too; nothing issued before it touches TM_S.
+        k2_warp_arrive(B.sepi, lane);
         if (P.sv_ckpt) {
           // training mode: the state at the start of chunk cb + n, stored
           // transposed ([d_k][d_v] per chunk) so that a warp's 32 rows j of
@@ -1463,14 +1477,6 @@ __global__ void __launch_bounds__(kK2Threads, 1) k2_state(const KParams P, void 
           for (int u = 0; u < 2; ++u)
 #pragma unroll
             for (int e = 0; e < 16; ++e) dst[(size_t)(16 * u + e) * kD] = sv[u][e];
-        }
-        {
-          uint32_t pk[16];
-#pragma unroll
-          for (int u = 0; u < 2; ++u)
-#pragma unroll
-            for (int e = 0; e < 8; ++e) pk[8 * u + e] = pack_bf16(sv[u][2 * e], sv[u][2 * e + 1]);
-          tmem_st16u(tm + lane_q + tm_sb(n) + 16 * cg, pk);
         }
 #pragma unroll
         for (int u = 0; u < 2; ++u) {
@@ -1486,7 +1492,6 @@ __global__ void __launch_bounds__(kK2Threads, 1) k2_state(const KParams P, void 
         }
         tmem_wait_st();
       }
-      k2_warp_arrive(B.sepi, lane);
       // chunk n - 1's output in two halves, under MMA5 and under MMA8 (the
       // O^T buffer they free takes chunk n + 1, whose MMA6 comes after this
       // chunk's epilogues)
