@@ -64,7 +64,7 @@ extern "C" {
 typedef enum {
   PDN_OK = 0,
   PDN_ERR_INVALID_ARG = 1, /* bad shape, pointer, alignment or variant/gate mix */
-  PDN_ERR_UNSUPPORTED = 2, /* valid problem that this build has no kernel for */
+  PDN_ERR_UNSUPPORTED = 2, /* valid problem that the library has no kernel for */
   PDN_ERR_CUDA = 3,        /* a CUDA runtime call or kernel launch failed */
   PDN_ERR_TIMEOUT = 4,     /* a bounded device wait ran out (device error word) */
   PDN_ERR_WORKSPACE = 5,   /* workspace pointer NULL or smaller than required */
@@ -162,7 +162,7 @@ typedef struct {
 size_t pdn_chunk_fwd_workspace(const pdn_problem_t *p);
 
 /* Which path pdn_chunk_fwd runs for problem p: PDN_IMPL_SIMT or PDN_IMPL_TC;
- * -1 if p is invalid or no kernel of this build supports it. Host-only,
+ * -1 if p is invalid or no kernel of the library supports it. Host-only,
  * touches no device. */
 int pdn_chunk_fwd_impl(const pdn_problem_t *p);
 

@@ -7,7 +7,7 @@
 // implicit synchronisation is not acceptable, or plugins that are handed
 // input/output buffers but no allocator. This entry point serves them: the
 // scratch the tensor-core path needs lives in one file-scope device array,
-// reserved by the driver when the library's device code is loaded on a GPU
+// reserved by the CUDA driver when the library's device code is loaded on a GPU
 // and held until the process exits.
 #include <mutex>
 
